@@ -1,0 +1,156 @@
+/*
+ * tlp.h — C ABI of the B200 (sm_100a) fused Transformer encoder layer,
+ * forward and backward, pre-LN and post-LN.
+ *
+ * The layer computed is the BERT-style encoder layer of the "DeepSpeed
+ * Transformer Kernel usage guide" (Step 1: one layer object per encoder
+ * layer; Step 2: the configuration parameters batch_size, max_seq_length,
+ * hidden_size, heads, attn_dropout_ratio, hidden_dropout_ratio,
+ * pre_layer_norm, seed, fp16, intermediate_size, layer_norm_eps, training;
+ * Step 3: the memory switches attn_dropout_checkpoint, normalize_invertible,
+ * gelu_checkpoint), with the module order of "Forward-pass compute-graph
+ * optimisation in the Transformer", section 2 (QKV projection, scaled
+ * dot-product attention softmax(Q K^T / sqrt(d_k)) V, output projection,
+ * residual + LayerNorm, FFN, residual + LayerNorm).
+ *
+ * Pre-LN:  h1 = LN1(x);  [Q|K|V] = h1 Wqkv^T + bqkv;
+ *          ctx = dropout_a(softmax(Q K^T / sqrt(d) + mask)) V   (per head)
+ *          x2 = x + dropout_h(ctx Wo^T + bo);  h2 = LN2(x2);
+ *          y  = x2 + dropout_h(GELU(h2 W1^T + b1) W2^T + b2)
+ * Post-LN: x2 = LN1(x + dropout_h(attn(x) Wo^T + bo));
+ *          y  = LN2(x2 + dropout_h(FFN(x2)))
+ * GELU is the erf form; LayerNorm is per token over the hidden axis with the
+ * biased variance and eps inside the square root.
+ *
+ * Conventions shared by every entry point
+ *  - All tensor pointers are DEVICE pointers on the device that was current
+ *    when the layer's buffers were allocated; the caller owns them.
+ *  - Tensors are dense row-major.  Activations are (batch, seq, hidden) =
+ *    (T, H) with T = batch*seq.  Weights use the Linear convention
+ *    [out_features, in_features]: wqkv (3H, H) with row blocks [Q; K; V] and
+ *    head h owning rows h*d .. h*d+d-1 of each block; wo (H, H);
+ *    w1 (F, H); w2 (H, F); biases and LayerNorm gamma/beta are vectors.
+ *  - Activations and weights are in the layer's storage dtype (tl_dtype);
+ *    the padding mask and every gradient of a weight are float32.
+ *  - `stream` is a cudaStream_t (NULL = legacy default stream).  All work is
+ *    enqueued on it; calls return before the GPU finishes.  Argument errors
+ *    are reported synchronously and enqueue nothing.
+ *  - Dropout draws its bits from Philox4x32-10 (Salmon et al., SC'11): the
+ *    element with flat index e of dropout site s uses counter
+ *    (e/8 mod 2^32, e/8 div 2^32, s, philox_offset) under key
+ *    (seed mod 2^32, seed div 2^32); lane e mod 8 = k reads the 16-bit half
+ *    (k mod 2) of output word (k div 2) and the element is kept when that
+ *    lane is >= floor(p * 65536).  Kept values are scaled by 1/(1-p).
+ *    Sites: 0 = attention probabilities, e = ((b*heads+h)*seq+i)*seq+j;
+ *    1 = attention-block output, e = t*H+c; 2 = FFN output, e = t*H+c.
+ */
+#ifndef TLP_H
+#define TLP_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct tl_layer tl_layer; /* opaque; owns saved activations + workspace */
+
+typedef enum {
+  TL_OK = 0,
+  TL_EINVAL = 1,        /* bad argument; nothing was enqueued */
+  TL_ENOMEM = 2,        /* device allocation failed */
+  TL_ESTATE = 3,        /* call out of order (e.g. backward before a training forward) */
+  TL_ECUDA = 4,         /* a CUDA call failed; see layer_last_error() */
+  TL_ETIMEOUT = 5,      /* a bounded device-side wait gave up */
+  TL_EUNSUPPORTED = 6   /* valid but not implemented for this configuration */
+} tl_status;
+
+typedef enum { TL_F32 = 0, TL_F16 = 1, TL_BF16 = 2 } tl_dtype;
+
+/* Options ("DeepSpeed Transformer Kernel usage guide", Step 2 extra
+ * parameters and Step 3 memory switches). */
+typedef struct {
+  int dtype;                     /* tl_dtype; default TL_F32 (fp16 = False) */
+  float ln_eps;                  /* default 1e-12 */
+  uint64_t philox_offset;        /* 4th Philox counter word; the layer id in a stack (default 0) */
+  int gelu_checkpoint;           /* 1: keep only the FFN1 pre-activation U; GELU(U) is
+                                    recomputed in backward.  Results are bitwise identical. */
+  int attn_dropout_checkpoint;   /* accepted; the attention kernels never store the
+                                    dropped probabilities, so this is always in effect */
+  int normalize_invertible;      /* 1: LayerNorm backward from its output, the LayerNorm
+                                    input is not needed (layer_backward may get x = NULL
+                                    in pre-LN form); requires every gamma != 0 */
+  int training;                  /* 1 (default): forward keeps what backward needs and applies
+                                    dropout; 0: inference, dropout off, no backward */
+} tl_options;
+
+/* The twelve parameter tensors, all passed on every call (Step 2: the layer
+ * hands all weights to the fused function at once).  Storage dtype. */
+typedef struct {
+  const void *wqkv, *bqkv, *wo, *bo, *ln1_g, *ln1_b;
+  const void *w1, *b1, *w2, *b2, *ln2_g, *ln2_b;
+} tl_weights;
+
+/* Gradients of the twelve parameters, float32, same shapes as tl_weights.
+ * Overwritten (not accumulated) by layer_backward. */
+typedef struct {
+  float *wqkv, *bqkv, *wo, *bo, *ln1_g, *ln1_b;
+  float *w1, *b1, *w2, *b2, *ln2_g, *ln2_b;
+} tl_grads;
+
+/* Creates a layer.  ffn <= 0 means 4*hidden.  Rejected with TL_EINVAL:
+ * non-positive sizes, hidden % heads != 0, head dim not in {16,32,64,128},
+ * seq % 8 != 0, hidden % 8 != 0, ffn % 8 != 0, dropout ratios outside [0, 1).
+ * No device memory is touched until layer_set_options or the first forward. */
+tl_status layer_create(int batch, int seq, int hidden, int heads, int ffn,
+                       float attn_dropout, float hidden_dropout, int pre_layer_norm,
+                       uint64_t seed, tl_layer** out);
+
+/* Fills *opt with the defaults listed in tl_options. */
+void layer_default_options(tl_options* opt);
+
+/* Sets the options and (re)allocates the layer's device buffers on the
+ * current device (TL_ENOMEM on failure).  Must precede the first forward if
+ * non-default options are wanted; afterwards it discards saved activations. */
+tl_status layer_set_options(tl_layer* layer, const tl_options* opt);
+tl_status layer_get_options(const tl_layer* layer, tl_options* opt);
+
+/* Forward.  x, y: (batch, seq, hidden) storage dtype; y must not alias x.
+ * mask: NULL or (batch, seq) float32 additive key mask (0 for a valid key,
+ * -inf for padding), broadcast over heads and queries.  A query row whose
+ * keys are all masked gets zero attention output.  In training mode the
+ * layer keeps what backward needs (it does not keep x: pass it again). */
+tl_status layer_forward(tl_layer* layer, const void* x, const float* mask,
+                        const tl_weights* w, void* y, void* stream);
+
+/* Backward of the most recent training-mode forward (TL_ESTATE otherwise).
+ * x: that forward's input (may be NULL only with normalize_invertible in
+ * pre-LN form); dy: (batch, seq, hidden) upstream gradient; dx receives the
+ * input gradient; g receives every parameter gradient (float32, overwritten).
+ * The mask of that forward is reused and must still be valid. */
+tl_status layer_backward(tl_layer* layer, const void* x, const void* dy,
+                         const tl_weights* w, tl_grads* g, void* dx, void* stream);
+
+/* Device bytes the layer holds (saved activations + scratch). */
+size_t layer_workspace_bytes(const tl_layer* layer);
+
+/* Text of the last error on this layer ("" if none).  Valid until the next call. */
+const char* layer_last_error(const tl_layer* layer);
+
+/* Releases every device buffer of the layer.  Synchronises the device first. */
+void layer_destroy(tl_layer* layer);
+
+/* Test hook: writes keep[i] = 1 if flat element e0+i of `site` is kept under
+ * the Philox contract above, else 0, for i < n (device buffer of n bytes).
+ * e0 and n must be multiples of 8.  Uses the same device code as the layer. */
+tl_status tl_dropout_keep_mask(uint64_t seed, uint64_t philox_offset, int site, float p,
+                               uint64_t e0, uint64_t n, uint8_t* keep, void* stream);
+
+const char* tl_status_string(tl_status s);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* TLP_H */
