@@ -147,6 +147,12 @@ void layer_destroy(tl_layer* layer);
 tl_status tl_dropout_keep_mask(uint64_t seed, uint64_t philox_offset, int site, float p,
                                uint64_t e0, uint64_t n, uint8_t* keep, void* stream);
 
+/* Waits for all work on the current device, then reports TL_ECUDA if a CUDA
+ * error is pending, TL_ETIMEOUT if a bounded device-side wait of a
+ * tensor-core kernel gave up since the last call (the flag is cleared), else
+ * TL_OK.  Blocks the host. */
+tl_status tl_device_check(void);
+
 const char* tl_status_string(tl_status s);
 
 #ifdef __cplusplus

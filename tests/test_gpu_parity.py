@@ -1,0 +1,79 @@
+"""Parity of the CUDA layer (through the C ABI) with the float64 oracle on
+the same seeded inputs, element by element.
+
+Cases: the tiny float32 layer; ragged shapes (token counts, widths and FFN
+sizes that are not multiples of any tile) in both layer orders; the
+BERT-base bf16 workload at full size; the BERT-Large fp16 workload at a
+reduced batch; the long-sequence post-LN bf16 workload at batch 1."""
+import dataclasses
+
+import numpy as np
+import pytest
+import torch
+
+from parity import check_layer, run_gpu, run_oracle
+from transformer_layer_pre_b200.synthetic import WORKLOADS, Workload, make_inputs
+
+pytestmark = pytest.mark.gpu
+
+RAGGED_F16 = Workload("ragged-f16", 3, 72, 192, 3, 520, "f16", 0.1, 0.1, lengths=(40, 72))
+RAGGED_POST_BF16 = Workload("ragged-post-bf16", 2, 40, 128, 2, 264, "bf16", 0.1, 0.1, pre_layer_norm=False,
+                            lengths=(17, 40))
+RAGGED_F32 = Workload("ragged-f32", 2, 24, 96, 6, 200, "f32", 0.1, 0.2, lengths=(9, 24))
+
+
+def _parity(w: Workload, batch=None, **kw):
+    inp = make_inputs(w, batch=batch)
+    gpu = run_gpu(inp, **kw)
+    pure = run_oracle(inp)
+    rounded = None if w.dtype == "f32" else run_oracle(inp, storage_rounded=True)
+    return check_layer(gpu, pure, rounded, w.dtype)
+
+
+def test_tiny_f32():
+    _parity(WORKLOADS["tiny-f32"])
+
+
+def test_ragged_f32_with_dropout_and_mask():
+    _parity(RAGGED_F32)
+
+
+def test_ragged_f16_pre_ln():
+    _parity(RAGGED_F16)
+
+
+def test_ragged_bf16_post_ln():
+    _parity(RAGGED_POST_BF16)
+
+
+def test_bert_base_bf16_full_size():
+    _parity(WORKLOADS["bert-base-bf16"])
+
+
+def test_bert_large_f16_batch4():
+    _parity(WORKLOADS["bert-large-f16"], batch=4)
+
+
+def test_long_post_ln_bf16_batch1():
+    _parity(WORKLOADS["long-postln-bf16"], batch=1)
+
+
+def test_gelu_checkpoint_is_bitwise_identical():
+    w = dataclasses.replace(WORKLOADS["bert-large-stack-f16"], batch=2, seq=128, layers=1)
+    inp = make_inputs(w)
+    a = run_gpu(inp, gelu_checkpoint=False)
+    b = run_gpu(inp, gelu_checkpoint=True)
+    assert np.array_equal(a["y"], b["y"]) and np.array_equal(a["dx"], b["dx"])
+    for n in a["grads"]:
+        assert np.array_equal(a["grads"][n], b["grads"][n]), n
+
+
+def test_philox_offset_changes_masks_and_matches_oracle():
+    w = dataclasses.replace(RAGGED_F16, batch=2)
+    inp = make_inputs(w)
+    gpu = run_gpu(inp, philox_offset=7)
+    pure = run_oracle(inp, philox_offset=7)
+    rounded = run_oracle(inp, storage_rounded=True, philox_offset=7)
+    check_layer(gpu, pure, rounded, w.dtype)
+    other = run_gpu(inp, philox_offset=0)
+    assert not np.array_equal(gpu["y"], other["y"])

@@ -1,0 +1,206 @@
+"""B200 (sm_100a) fused Transformer encoder layer: Python binding of libtlp.so.
+
+The binding only marshals arguments: every step of the layer runs in the
+CUDA kernels behind the C ABI declared in include/tlp.h.  PyTorch supplies
+device memory and streams.  There is no fallback: if the library is missing,
+LibraryMissing is raised.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+__all__ = ["Layer", "Options", "TlError", "LibraryMissing", "load_library", "dropout_keep_mask",
+           "WEIGHT_NAMES", "DTYPE_CODES", "EXPORTED_SYMBOLS", "device_check"]
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libtlp.so")
+
+WEIGHT_NAMES = (
+    "wqkv", "bqkv", "wo", "bo", "ln1_g", "ln1_b",
+    "w1", "b1", "w2", "b2", "ln2_g", "ln2_b",
+)
+DTYPE_CODES = {torch.float32: 0, torch.float16: 1, torch.bfloat16: 2}
+EXPORTED_SYMBOLS = (
+    "layer_create", "layer_default_options", "layer_set_options", "layer_get_options",
+    "layer_forward", "layer_backward", "layer_workspace_bytes", "layer_last_error",
+    "layer_destroy", "tl_dropout_keep_mask", "tl_device_check", "tl_status_string",
+)
+
+
+class LibraryMissing(RuntimeError):
+    pass
+
+
+class TlError(RuntimeError):
+    def __init__(self, status: int, msg: str):
+        super().__init__(f"tlp status {status}: {msg}")
+        self.status = status
+
+
+class Options(ctypes.Structure):
+    _fields_ = [
+        ("dtype", ctypes.c_int),
+        ("ln_eps", ctypes.c_float),
+        ("philox_offset", ctypes.c_uint64),
+        ("gelu_checkpoint", ctypes.c_int),
+        ("attn_dropout_checkpoint", ctypes.c_int),
+        ("normalize_invertible", ctypes.c_int),
+        ("training", ctypes.c_int),
+    ]
+
+
+class _Weights(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_void_p) for n in WEIGHT_NAMES]
+
+
+_lib = None
+
+
+def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
+    """Loads libtlp.so once.  Raises LibraryMissing when it has not been built."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(path):
+        raise LibraryMissing(f"{path} not found: build it with `python -m transformer_layer_pre_b200.build_ext`")
+    lib = ctypes.CDLL(path)
+    vp, i, f, u64 = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_uint64
+    lib.layer_create.argtypes = [i, i, i, i, i, f, f, i, u64, ctypes.POINTER(vp)]
+    lib.layer_create.restype = i
+    lib.layer_default_options.argtypes = [ctypes.POINTER(Options)]
+    lib.layer_default_options.restype = None
+    lib.layer_set_options.argtypes = [vp, ctypes.POINTER(Options)]
+    lib.layer_set_options.restype = i
+    lib.layer_get_options.argtypes = [vp, ctypes.POINTER(Options)]
+    lib.layer_get_options.restype = i
+    lib.layer_forward.argtypes = [vp, vp, vp, ctypes.POINTER(_Weights), vp, vp]
+    lib.layer_forward.restype = i
+    lib.layer_backward.argtypes = [vp, vp, vp, ctypes.POINTER(_Weights), ctypes.POINTER(_Weights), vp, vp]
+    lib.layer_backward.restype = i
+    lib.layer_workspace_bytes.argtypes = [vp]
+    lib.layer_workspace_bytes.restype = ctypes.c_size_t
+    lib.layer_last_error.argtypes = [vp]
+    lib.layer_last_error.restype = ctypes.c_char_p
+    lib.layer_destroy.argtypes = [vp]
+    lib.layer_destroy.restype = None
+    lib.tl_dropout_keep_mask.argtypes = [u64, u64, i, f, u64, u64, vp, vp]
+    lib.tl_dropout_keep_mask.restype = i
+    lib.tl_device_check.argtypes = []
+    lib.tl_device_check.restype = i
+    lib.tl_status_string.argtypes = [i]
+    lib.tl_status_string.restype = ctypes.c_char_p
+    _lib = lib
+    return lib
+
+
+def _ptr(t: torch.Tensor | None) -> int | None:
+    return None if t is None else t.data_ptr()
+
+
+def _stream(stream) -> int:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return stream.cuda_stream
+
+
+class Layer:
+    """One encoder layer (a handle of the C ABI).
+
+    Layer(batch, seq, hidden, heads, ffn=0, attn_dropout=0., hidden_dropout=0.,
+    pre_layer_norm=True, seed=1234, dtype=torch.float16, ...options)
+    """
+
+    def __init__(self, batch, seq, hidden, heads, ffn=0, attn_dropout=0.0, hidden_dropout=0.0,
+                 pre_layer_norm=True, seed=1234, dtype=torch.float16, ln_eps=1e-12, philox_offset=0,
+                 gelu_checkpoint=False, attn_dropout_checkpoint=False, normalize_invertible=False,
+                 training=True):
+        self.lib = load_library()
+        self.handle = None
+        h = ctypes.c_void_p()
+        st = self.lib.layer_create(batch, seq, hidden, heads, ffn, attn_dropout, hidden_dropout,
+                                   int(pre_layer_norm), seed, ctypes.byref(h))
+        if st != 0:
+            raise TlError(st, self.lib.tl_status_string(st).decode())
+        self.handle = h
+        self.batch, self.seq, self.hidden, self.heads = batch, seq, hidden, heads
+        self.ffn = ffn if ffn > 0 else 4 * hidden
+        self.dtype = dtype
+        opt = Options()
+        self.lib.layer_default_options(ctypes.byref(opt))
+        opt.dtype = DTYPE_CODES[dtype]
+        opt.ln_eps = ln_eps
+        opt.philox_offset = philox_offset
+        opt.gelu_checkpoint = int(gelu_checkpoint)
+        opt.attn_dropout_checkpoint = int(attn_dropout_checkpoint)
+        opt.normalize_invertible = int(normalize_invertible)
+        opt.training = int(training)
+        self._check(self.lib.layer_set_options(self.handle, ctypes.byref(opt)))
+
+    def _check(self, st: int) -> None:
+        if st != 0:
+            msg = self.lib.layer_last_error(self.handle).decode() if self.handle else ""
+            raise TlError(st, msg or self.lib.tl_status_string(st).decode())
+
+    @staticmethod
+    def _weights(w: dict) -> _Weights:
+        return _Weights(*[_ptr(w[n]) for n in WEIGHT_NAMES])
+
+    def forward(self, x, mask, weights, y=None, stream=None):
+        """x (B, S, H) storage dtype on the device; mask (B, S) float32 or None."""
+        if y is None:
+            y = torch.empty_like(x)
+        wt = self._weights(weights)
+        self._check(self.lib.layer_forward(self.handle, _ptr(x), _ptr(mask), ctypes.byref(wt), _ptr(y),
+                                           _stream(stream)))
+        return y
+
+    def backward(self, x, dy, weights, grads=None, dx=None, stream=None):
+        """Returns (dx, grads) with grads a dict of float32 tensors."""
+        if dx is None:
+            dx = torch.empty_like(dy)
+        if grads is None:
+            grads = {n: torch.empty(tuple(weights[n].shape), dtype=torch.float32, device=dy.device)
+                     for n in WEIGHT_NAMES}
+        wt = self._weights(weights)
+        gt = self._weights(grads)
+        self._check(self.lib.layer_backward(self.handle, _ptr(x), _ptr(dy), ctypes.byref(wt), ctypes.byref(gt),
+                                            _ptr(dx), _stream(stream)))
+        return dx, grads
+
+    @property
+    def workspace_bytes(self) -> int:
+        return int(self.lib.layer_workspace_bytes(self.handle))
+
+    def close(self) -> None:
+        if self.handle:
+            self.lib.layer_destroy(self.handle)
+            self.handle = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+
+def device_check() -> None:
+    """Synchronises the device; raises TlError on a pending CUDA error or a
+    bounded device-side wait that gave up."""
+    lib = load_library()
+    st = lib.tl_device_check()
+    if st != 0:
+        raise TlError(st, lib.tl_status_string(st).decode())
+
+
+def dropout_keep_mask(seed: int, offset: int, site: int, p: float, e0: int, n: int, device="cuda") -> torch.Tensor:
+    """Keep bits computed on the device by the layer's own Philox code."""
+    lib = load_library()
+    out = torch.empty(n, dtype=torch.uint8, device=device)
+    st = lib.tl_dropout_keep_mask(seed, offset, site, p, e0, n, _ptr(out), _stream(None))
+    if st != 0:
+        raise TlError(st, lib.tl_status_string(st).decode())
+    return out

@@ -1,0 +1,32 @@
+// dispatch.cu — picks the kernel family that serves each dtype: the tcgen05
+// tensor-core GEMM for 16-bit storage, the exact-float32 SIMT GEMM for float32.
+#include "kernels.h"
+
+namespace tlp {
+
+void gemm_simt_run(int dtype, const GemmDesc& g, const EpiParams& e, cudaStream_t s);
+int gemm_tc_run(int dtype, const GemmDesc& g, const EpiParams& e, cudaStream_t s);
+size_t gemm_tc_splitk_ws_floats(int M, int N, int K);
+int gemm_tc_take_error();
+
+int gemm_uses_tensor_cores(int dtype) { return dtype != DT_F32; }
+
+int gemm_run(int dtype, const GemmDesc& g, const EpiParams& e, cudaStream_t s) {
+  if (dtype == DT_F32) {
+    gemm_simt_run(dtype, g, e, s);
+    return 0;
+  }
+  return gemm_tc_run(dtype, g, e, s);
+}
+
+size_t gemm_splitk_ws_floats(int dtype, int M, int N, int K) {
+  return dtype == DT_F32 ? 0 : gemm_tc_splitk_ws_floats(M, N, K);
+}
+
+int device_take_error() { return gemm_tc_take_error(); }
+
+bool attn_tc_supports(int dt, const AttnArgs& a) { (void)dt; (void)a; return false; }
+void attn_tc_fwd_run(int, const AttnArgs&, cudaStream_t) {}
+void attn_tc_bwd_run(int, const AttnArgs&, cudaStream_t) {}
+
+}  // namespace tlp

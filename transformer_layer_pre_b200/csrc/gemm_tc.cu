@@ -1,0 +1,388 @@
+// gemm_tc.cu — tcgen05 tensor-core GEMM for 16-bit storage (fp16 / bf16),
+// float32 accumulation in TMEM, with the layer's fused epilogues.
+//
+// C[m, n] = sum_k A(m, k) B(n, k).  Each operand is K-major (row-major with
+// K contiguous: activations and weights in forward, the output gradient in
+// dgrad) or MN-major (K rows with M or N contiguous: the weight in dgrad,
+// both operands of a weight gradient), so no operand is ever transposed in
+// memory ("AI-infra engineers and the Transformer", section 2.3: the second
+// FFN weight stored transposed for the backward pass is made unnecessary here
+// by reading either major directly).
+//
+// Structure (one CTA per SM, persistent over output tiles of 128 x BN):
+//   warp 0   TMA producer: per K block of 64, one 128-byte-swizzled box per
+//            64-wide slice of each operand into a STAGES-deep ring
+//            (no cluster multicast: every CTA loads its own tiles);
+//   warp 1   allocates TMEM (two BN-column fp32 accumulators) and issues
+//            tcgen05.mma (M=128, N=BN, K=16) from one thread, committing each
+//            stage back to the producer and each finished tile to the epilogue;
+//   warps 2-5  epilogue: tcgen05.ld 16 columns at a time from the lanes the
+//            warp may access, fused epilogue (epilogue.cuh), global stores.
+// Accumulators are double-buffered so a tile's epilogue overlaps the next
+// tile's main loop.  Weight gradients (K = tokens) may split K across CTAs
+// into float32 partial tiles that a second kernel sums in a fixed order.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cstring>
+#include <type_traits>
+
+#include "epilogue.cuh"
+#include "kernels.h"
+#include "sm100.cuh"
+
+namespace tlp {
+
+using namespace sm100;
+
+namespace {
+
+constexpr int BM = 128;
+constexpr int BK = 64;
+constexpr int kThreads = 192;
+
+template <int BN> struct TileCfg {
+  static constexpr int kStages = BN == 256 ? 4 : 6;
+  static constexpr int kABytes = BM * BK * 2;
+  static constexpr int kBBytes = BN * BK * 2;
+  static constexpr int kStageBytes = kABytes + kBBytes;
+  static constexpr int kSmem = kStages * kStageBytes + 1024 + 256;
+  static constexpr int kTmemCols = 2 * BN;
+};
+
+struct TcArgs {
+  int M, N, K;
+  int a_mn, b_mn;      // operand is MN-major
+  int bf16;
+  int tiles_m, tiles_n, splits, kb_per_split, kblocks;
+  size_t split_stride;  // floats between the partial outputs of consecutive splits
+  int* err;
+};
+
+__device__ __forceinline__ void decode_tile(const TcArgs& g, int t, int& mb, int& nb, int& sp) {
+  const int per = g.tiles_m * g.tiles_n;
+  sp = t / per;
+  const int r = t - sp * per;
+  mb = r / g.tiles_n;
+  nb = r - mb * g.tiles_n;
+}
+
+template <typename T, int BN, int KIND>
+__global__ void __launch_bounds__(kThreads, 1)
+    gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, TcArgs g,
+                   EpiParams e) {
+  using C = TileCfg<BN>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::kStages * C::kStageBytes);
+  uint64_t* empty = full + C::kStages;
+  uint64_t* tfull = empty + C::kStages;
+  uint64_t* tempty = tfull + 2;
+  uint32_t* tslot = reinterpret_cast<uint32_t*>(tempty + 2);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < C::kStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&tfull[a], 1);
+      mbar_init(&tempty[a], 128);
+    }
+    fence_barrier_init();
+  }
+  if (warp == 1) tmem_alloc(tslot, C::kTmemCols);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tslot;
+  const int total = g.tiles_m * g.tiles_n * g.splits;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      prefetch_tensormap(&tmA);
+      prefetch_tensormap(&tmB);
+      int s = 0;
+      uint32_t ph = 0;
+      bool ok = true;
+      uint32_t issued_phase[8];
+      bool issued[8];
+      for (int i = 0; i < C::kStages; ++i) issued[i] = false;
+      for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
+        int mb, nb, sp;
+        decode_tile(g, t, mb, nb, sp);
+        const int kb0 = sp * g.kb_per_split;
+        const int kb1 = min(g.kblocks, kb0 + g.kb_per_split);
+        for (int kb = kb0; kb < kb1; ++kb) {
+          if (!mbar_wait(&empty[s], ph ^ 1u, g.err, 1)) { ok = false; break; }
+          uint8_t* a_dst = smem + s * C::kStageBytes;
+          uint8_t* b_dst = a_dst + C::kABytes;
+          mbar_arrive_expect_tx(&full[s], C::kStageBytes);
+          const int k0 = kb * BK;
+          if (!g.a_mn) {
+            tma_load_2d(a_dst, &tmA, &full[s], k0, mb * BM);
+          } else {
+#pragma unroll
+            for (int j = 0; j < BM / 64; ++j) tma_load_2d(a_dst + j * 8192, &tmA, &full[s], mb * BM + 64 * j, k0);
+          }
+          if (!g.b_mn) {
+            tma_load_2d(b_dst, &tmB, &full[s], k0, nb * BN);
+          } else {
+#pragma unroll
+            for (int j = 0; j < BN / 64; ++j) tma_load_2d(b_dst + j * 8192, &tmB, &full[s], nb * BN + 64 * j, k0);
+          }
+          issued[s] = true;
+          issued_phase[s] = ph;
+          if (++s == C::kStages) { s = 0; ph ^= 1u; }
+        }
+      }
+      if (!ok) {
+        // wind down: let every load already issued land before the CTA exits
+        for (int i = 0; i < C::kStages; ++i)
+          if (issued[i]) mbar_wait(&full[i], issued_phase[i], nullptr, 0);
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      const uint32_t idesc = idesc_f16(BM, BN, g.bf16 != 0, g.a_mn != 0, g.b_mn != 0);
+      int s = 0;
+      uint32_t ph = 0;
+      int acc = 0;
+      uint32_t aph = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
+        int mb, nb, sp;
+        decode_tile(g, t, mb, nb, sp);
+        const int kb0 = sp * g.kb_per_split;
+        const int kb1 = min(g.kblocks, kb0 + g.kb_per_split);
+        if (!mbar_wait(&tempty[acc], aph ^ 1u, g.err, 2)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t d = tmem + acc * BN;
+        for (int kb = kb0; kb < kb1; ++kb) {
+          if (!mbar_wait(&full[s], ph, g.err, 3)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t a_base = smem_u32(smem + s * C::kStageBytes);
+          const uint32_t b_base = a_base + C::kABytes;
+#pragma unroll
+          for (int k = 0; k < BK / 16; ++k) {
+            const uint64_t ad = g.a_mn ? smem_desc_sw128(a_base + k * 2048, 8192, 1024)
+                                       : smem_desc_sw128(a_base + k * 32, 16, 1024);
+            const uint64_t bd = g.b_mn ? smem_desc_sw128(b_base + k * 2048, 8192, 1024)
+                                       : smem_desc_sw128(b_base + k * 32, 16, 1024);
+            mma_f16(d, ad, bd, idesc, (kb > kb0 || k > 0) ? 1u : 0u);
+          }
+          mma_commit(&empty[s]);
+          if (++s == C::kStages) { s = 0; ph ^= 1u; }
+        }
+        if (!ok) break;
+        mma_commit(&tfull[acc]);
+        acc ^= 1;
+        if (acc == 0) aph ^= 1u;
+      }
+    }
+  } else {
+    const int quarter = warp & 3;  // this warp may access TMEM lanes 32*quarter .. +31
+    const int row = quarter * 32 + lane;
+    int acc = 0;
+    uint32_t aph = 0;
+    for (int t = blockIdx.x; t < total; t += gridDim.x) {
+      int mb, nb, sp;
+      decode_tile(g, t, mb, nb, sp);
+      if (!mbar_wait(&tfull[acc], aph, g.err, 4)) break;
+      tc_fence_after();
+      const int m = mb * BM + row;
+      EpiParams ep = e;
+      if constexpr (KIND == EPI_F32) ep.out = static_cast<float*>(e.out) + (size_t)sp * g.split_stride;
+      const uint32_t tbase = tmem + ((uint32_t)(quarter * 32) << 16) + acc * BN;
+#pragma unroll 1
+      for (int c0 = 0; c0 < BN; c0 += 16) {
+        float v[16];
+        tmem_ld16(tbase + c0, v);
+        const int n = nb * BN + c0;
+        if (m < g.M) {
+          float* v0 = v;
+          float* v1 = v + 8;
+          if (n < g.N) epi_apply8<T, KIND>(ep, m, n, *reinterpret_cast<float(*)[8]>(v0));
+          if (n + 8 < g.N) epi_apply8<T, KIND>(ep, m, n + 8, *reinterpret_cast<float(*)[8]>(v1));
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(&tempty[acc]);
+      acc ^= 1;
+      if (acc == 0) aph ^= 1u;
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc(tmem, C::kTmemCols);
+}
+
+__global__ void splitk_reduce_kernel(const float* __restrict__ part, int splits, size_t stride, size_t n4,
+                                     float* __restrict__ out) {
+  for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n4; i += (size_t)gridDim.x * blockDim.x) {
+    float4 s = reinterpret_cast<const float4*>(part)[i];
+    for (int k = 1; k < splits; ++k) {
+      const float4 v = reinterpret_cast<const float4*>(part + k * stride)[i];
+      s.x += v.x; s.y += v.y; s.z += v.z; s.w += v.w;
+    }
+    reinterpret_cast<float4*>(out)[i] = s;
+  }
+}
+
+// ------------------------------------------------------------------ host side
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    cudaDriverEntryPointQueryResult q;
+    void* p = nullptr;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  return fn;
+}
+
+// 2-D map over a row-major (outer, inner) matrix with row stride ld elements;
+// box = 64 inner elements (128 bytes, swizzled) x box_outer rows.
+bool make_map(CUtensorMap* m, const void* ptr, bool bf16, uint64_t inner, uint64_t outer, uint64_t ld,
+              uint32_t box_outer) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {inner, outer};
+  cuuint64_t strides[1] = {ld * 2};
+  cuuint32_t box[2] = {64, box_outer};
+  cuuint32_t es[2] = {1, 1};
+  return fn(m, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<void*>(ptr),
+            dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+int num_sms() {
+  static int n = 0;
+  if (!n) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    if (n <= 0) n = 148;
+  }
+  return n;
+}
+
+int* error_word() {
+  static int* p = nullptr;
+  if (!p) cudaMalloc(&p, sizeof(int)), cudaMemset(p, 0, sizeof(int));
+  return p;
+}
+
+template <typename T, int BN, int KIND>
+int launch_tc(const GemmDesc& gd, const EpiParams& e, int splits, cudaStream_t s) {
+  using C = TileCfg<BN>;
+  const bool bf16 = sizeof(T) == 2 && std::is_same<T, bf16_t>::value;
+  CUtensorMap ma, mb;
+  bool ok;
+  if (gd.a_kmajor) ok = make_map(&ma, gd.A, bf16, gd.K, gd.M, gd.lda, BM);
+  else ok = make_map(&ma, gd.A, bf16, gd.M, gd.K, gd.lda, 64);
+  if (ok) {
+    if (gd.b_kmajor) ok = make_map(&mb, gd.B, bf16, gd.K, gd.N, gd.ldb, BN);
+    else ok = make_map(&mb, gd.B, bf16, gd.N, gd.K, gd.ldb, 64);
+  }
+  if (!ok) return 1;
+  TcArgs g;
+  g.M = gd.M; g.N = gd.N; g.K = gd.K;
+  g.a_mn = gd.a_kmajor ? 0 : 1;
+  g.b_mn = gd.b_kmajor ? 0 : 1;
+  g.bf16 = bf16 ? 1 : 0;
+  g.tiles_m = (gd.M + BM - 1) / BM;
+  g.tiles_n = (gd.N + BN - 1) / BN;
+  g.kblocks = (gd.K + BK - 1) / BK;
+  g.kb_per_split = (g.kblocks + splits - 1) / splits;
+  g.splits = (g.kblocks + g.kb_per_split - 1) / g.kb_per_split;
+  g.split_stride = (size_t)gd.M * gd.N;
+  g.err = error_word();
+  const int total = g.tiles_m * g.tiles_n * g.splits;
+  const int grid = std::min(total, num_sms());
+  static bool attr = false;
+  if (!attr) {
+    cudaFuncSetAttribute(gemm_tc_kernel<T, BN, KIND>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
+    attr = true;
+  }
+  gemm_tc_kernel<T, BN, KIND><<<grid, kThreads, C::kSmem, s>>>(ma, mb, g, e);
+  return 0;
+}
+
+// Weight gradients (K = tokens) split K when the output has too few tiles
+// to occupy the SMs; each split writes a float32 partial tile.
+int splitk_count(int M, int N, int K) {
+  const int tiles = ((M + BM - 1) / BM) * ((N + 255) / 256);
+  const int kblocks = (K + BK - 1) / BK;
+  if (tiles >= (3 * num_sms()) / 4) return 1;
+  return std::max(1, std::min(std::min(4, kblocks / 8), num_sms() / tiles));
+}
+
+bool aligned16(const void* p, int ld) {
+  return (reinterpret_cast<uintptr_t>(p) & 15) == 0 && ((size_t)ld * 2) % 16 == 0;
+}
+
+template <typename T>
+int run_t(const GemmDesc& g, const EpiParams& e, cudaStream_t s) {
+  if (!aligned16(g.A, g.lda) || !aligned16(g.B, g.ldb)) return 2;
+  // N <= 128 keeps the 128-wide tile; otherwise 256
+  const bool wide = g.N > 128;
+  if (e.kind == EPI_F32) {
+    const int kblocks = (g.K + BK - 1) / BK;
+    int splits = g.splitk_ws ? splitk_count(g.M, g.N, g.K) : 1;
+    while (splits > 1 && (size_t)splits * g.M * g.N > g.splitk_ws_floats) --splits;
+    if (splits > 1) {
+      EpiParams ep = e;
+      ep.out = g.splitk_ws;
+      int rc = launch_tc<T, 256, EPI_F32>(g, ep, splits, s);
+      if (rc) return rc;
+      const int kb_per = (kblocks + splits - 1) / splits;
+      const int real = (kblocks + kb_per - 1) / kb_per;
+      const size_t n4 = (size_t)g.M * g.N / 4;
+      splitk_reduce_kernel<<<(int)std::min<size_t>((n4 + 255) / 256, 148 * 8), 256, 0, s>>>(
+          g.splitk_ws, real, (size_t)g.M * g.N, n4, static_cast<float*>(e.out));
+      return 0;
+    }
+    return launch_tc<T, 256, EPI_F32>(g, e, 1, s);
+  }
+  switch (e.kind) {
+    case EPI_QKV: return wide ? launch_tc<T, 256, EPI_QKV>(g, e, 1, s) : launch_tc<T, 128, EPI_QKV>(g, e, 1, s);
+    case EPI_BIAS_DROP_RES:
+      return wide ? launch_tc<T, 256, EPI_BIAS_DROP_RES>(g, e, 1, s) : launch_tc<T, 128, EPI_BIAS_DROP_RES>(g, e, 1, s);
+    case EPI_BIAS_GELU:
+      return wide ? launch_tc<T, 256, EPI_BIAS_GELU>(g, e, 1, s) : launch_tc<T, 128, EPI_BIAS_GELU>(g, e, 1, s);
+    case EPI_DGELU: return wide ? launch_tc<T, 256, EPI_DGELU>(g, e, 1, s) : launch_tc<T, 128, EPI_DGELU>(g, e, 1, s);
+    case EPI_STORE: return wide ? launch_tc<T, 256, EPI_STORE>(g, e, 1, s) : launch_tc<T, 128, EPI_STORE>(g, e, 1, s);
+  }
+  return 1;
+}
+
+}  // namespace
+
+int gemm_tc_run(int dtype, const GemmDesc& g, const EpiParams& e, cudaStream_t s) {
+  return dtype == DT_F16 ? run_t<half_t>(g, e, s) : run_t<bf16_t>(g, e, s);
+}
+
+size_t gemm_tc_splitk_ws_floats(int M, int N, int K) {
+  const int sp = splitk_count(M, N, K);
+  return sp > 1 ? (size_t)sp * M * N : 0;
+}
+
+// Reads and clears the bounded-wait error word of the tensor-core kernels.
+int gemm_tc_take_error() {
+  int v = 0;
+  int* p = error_word();
+  cudaMemcpy(&v, p, sizeof(int), cudaMemcpyDeviceToHost);
+  if (v) cudaMemset(p, 0, sizeof(int));
+  return v;
+}
+
+}  // namespace tlp

@@ -1,0 +1,122 @@
+// kernels.h — host-side launchers of the layer's kernels (internal).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "common.cuh"
+
+namespace tlp {
+
+enum Dtype { DT_F32 = 0, DT_F16 = 1, DT_BF16 = 2 };
+inline size_t dtype_size(int dt) { return dt == DT_F32 ? 4 : 2; }
+
+// ------------------------------------------------------------------ GEMM
+// C[m, n] = sum_k A(m, k) * B(n, k), float32 accumulation, then an epilogue.
+// A(m, k) = A[m*lda + k] when a_kmajor, else A[k*lda + m]; B likewise.
+struct GemmDesc {
+  int M, N, K;
+  const void* A; int lda; bool a_kmajor;
+  const void* B; int ldb; bool b_kmajor;
+  float* splitk_ws;          // float32 scratch for split-K weight gradients, or null
+  size_t splitk_ws_floats;
+};
+
+enum EpiKind {
+  EPI_QKV = 0,        // + bias, scattered into Q, K, V laid out (B, heads, S, d)
+  EPI_BIAS_DROP_RES,  // out = res + dropout(acc + bias); element index m*N + n
+  EPI_BIAS_GELU,      // U = acc + bias (stored), G = GELU(stored U) (stored if out2)
+  EPI_DGELU,          // out = acc * GELU'(U)
+  EPI_STORE,          // out = acc (+ res if given)
+  EPI_F32             // float32 out = acc
+};
+
+struct EpiParams {
+  int kind;
+  const void* bias;   // N entries, storage type
+  const void* res;    // residual (M, N) storage type, or null
+  const void* aux;    // EPI_DGELU: U (M, N)
+  void* out;          // (M, N) with row stride ldo (EPI_QKV: Q|K|V base)
+  void* out2;         // EPI_BIAS_GELU: G, may be null
+  int ldo;
+  // dropout (EPI_BIAS_DROP_RES)
+  DropoutParams drop;
+  int site;
+  // head split (EPI_QKV)
+  int seq, hidden, head_dim, heads, tokens;
+};
+
+// Returns 0, or non-zero when an operand cannot be described to the TMA unit
+// (unaligned base address or row stride).
+int gemm_run(int dtype, const GemmDesc& g, const EpiParams& e, cudaStream_t s);
+// 1 when the tensor-core (tcgen05) GEMM serves this dtype, 0 for the SIMT one.
+int gemm_uses_tensor_cores(int dtype);
+// Split-K scratch (floats) the tensor-core GEMM would use for an EPI_F32 GEMM of this shape.
+size_t gemm_splitk_ws_floats(int dtype, int M, int N, int K);
+// Reads and clears the error word set by a bounded device-side wait that gave up.
+int device_take_error();
+
+// ------------------------------------------------------------------ LayerNorm
+void ln_fwd_run(int dtype, const void* x, const void* gamma, const void* beta, void* y, float* mean,
+                float* rstd, int rows, int H, float eps, cudaStream_t s);
+
+// LayerNorm backward of one row block + residual-gradient add + optional
+// dropout of the result, with column partial sums for dgamma, dbeta and the
+// sum of the dropped output.  Partials are (nparts, H) float32 each.
+struct LnBwdArgs {
+  const void* dy;       // gradient w.r.t. the LayerNorm output (rows, H)
+  const void* x;        // LayerNorm input (rows, H), or null when invertible
+  const void* y;        // LayerNorm output (invertible mode), else null
+  const float* mean;
+  const float* rstd;
+  const void* gamma;
+  const void* beta;     // invertible mode
+  const void* res;      // added to dx, or null
+  void* dx;             // (rows, H)
+  void* drop_out;       // dropout(dx) (rows, H), or null
+  DropoutParams drop;
+  int site;
+  float* part_dgamma;
+  float* part_dbeta;
+  float* part_dsum;     // column sums of drop_out, or null
+  int rows, H;
+};
+int ln_bwd_parts(int rows);
+void ln_bwd_run(int dtype, const LnBwdArgs& a, cudaStream_t s);
+
+// ------------------------------------------------------------------ elementwise / reductions
+// out = dropout(in) (site, element t*H + c) with column partial sums of out.
+int rowdrop_parts(int rows);
+void dropout_rows_run(int dtype, const void* in, void* out, const DropoutParams& dp, int site, int rows, int H,
+                      float* part_sum, cudaStream_t s);
+// Column partial sums of a (rows, cols) storage-typed matrix: (colsum_parts(rows), cols) floats.
+int colsum_parts(int rows);
+void colsum_run(int dtype, const void* X, int rows, int cols, float* part, cudaStream_t s);
+// out[c] = sum_p part[p*cols + c] (fixed order).
+void colsum_finalize_run(const float* part, int nparts, int cols, float* out, cudaStream_t s);
+// G = GELU(U), elementwise, n a multiple of 8.
+void gelu_run(int dtype, const void* U, void* G, size_t n, cudaStream_t s);
+// keep[i] = dropout keep bit of element e0 + i of `site`.
+void dropout_mask_run(const DropoutParams& dp, int site, uint64_t e0, uint64_t n, uint8_t* keep, cudaStream_t s);
+
+// ------------------------------------------------------------------ attention
+struct AttnArgs {
+  int B, S, nh, d;
+  const void* q;        // (B, nh, S, d)
+  const void* k;
+  const void* v;
+  const float* mask;    // (B, S) additive or null
+  float scale;          // 1/sqrt(d)
+  DropoutParams drop;   // site 0
+  void* ctx;            // (B*S, nh*d)
+  float* lse;           // (B, nh, S); +inf marks a row with every key masked
+  // backward
+  const void* dctx;     // (B*S, nh*d)
+  float* dvec;          // (B, nh, S) rowsum(dctx * ctx)
+  void* dqkv;           // (B*S, 3*nh*d): [dQ | dK | dV]
+};
+void attn_fwd_run(int dtype, const AttnArgs& a, cudaStream_t s);
+void attn_bwd_run(int dtype, const AttnArgs& a, cudaStream_t s);
+
+}  // namespace tlp

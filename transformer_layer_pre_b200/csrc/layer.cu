@@ -1,0 +1,499 @@
+// layer.cu — the C ABI (include/tlp.h): layer handle, buffers and the
+// forward/backward schedules of the encoder layer.
+//
+// Schedules (T tokens, storage type of the layer):
+//  pre-LN forward   LN1 -> QKV GEMM (+bias, head split) -> attention ->
+//                   out-proj GEMM (+bias, dropout, +x) -> LN2 ->
+//                   FFN1 GEMM (+bias, GELU) -> FFN2 GEMM (+bias, dropout, +x2)
+//  pre-LN backward  dropout'(dY) + db2 -> dW2, dU = (dZ2 W2) GELU'(U) -> db1,
+//                   dW1, dH2 -> LN2' (+dY, dropout' -> dA, dbo) -> dWo, dctx ->
+//                   attention' -> dbqkv, dWqkv, dH1 -> LN1' (+dx2) = dx
+//  post-LN          the same kernels wired per "Forward-pass compute-graph
+//                   optimisation in the Transformer", section 2 (residual add
+//                   then LayerNorm after each block).
+// Bias gradients are column sums of the stored output gradient of their
+// Linear; weight gradients are float32 GEMMs over the tokens.
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cmath>
+#include <cstdio>
+#include <cstring>
+#include <string>
+
+#include "../../include/tlp.h"
+#include "kernels.h"
+
+namespace tlp {
+bool rowwise_supports_hidden(int H);
+void attn_simt_fwd_run(int dt, const AttnArgs& a, cudaStream_t s);
+void attn_simt_bwd_run(int dt, const AttnArgs& a, cudaStream_t s);
+void attn_tc_fwd_run(int dt, const AttnArgs& a, cudaStream_t s);
+void attn_tc_bwd_run(int dt, const AttnArgs& a, cudaStream_t s);
+bool attn_tc_supports(int dt, const AttnArgs& a);
+}  // namespace tlp
+
+using namespace tlp;
+
+struct tl_layer {
+  int B, S, H, nh, d, F, T;
+  float pa, ph;
+  int pre_ln;
+  uint64_t seed;
+  tl_options opt;
+  int device = -1;
+  char* arena = nullptr;
+  size_t arena_bytes = 0;
+  bool have_fwd = false;
+  const float* mask = nullptr;
+  std::string err;
+
+  // saved activations
+  void *h1 = nullptr, *qkv = nullptr, *ctx = nullptr, *x2 = nullptr, *h2 = nullptr;
+  void *u = nullptr, *g = nullptr, *res1 = nullptr, *res2 = nullptr, *yout = nullptr;
+  float *mean1 = nullptr, *rstd1 = nullptr, *mean2 = nullptr, *rstd2 = nullptr, *lse = nullptr;
+  // backward scratch
+  void *big = nullptr;     // (T, F): G recompute / dU
+  void *dz2 = nullptr, *dh = nullptr, *dx2 = nullptr, *da = nullptr, *dctx = nullptr, *dres = nullptr;
+  void *dqkv = nullptr;
+  float *dvec = nullptr, *part = nullptr;
+  size_t part_floats = 0;
+  float* splitk = nullptr;
+  size_t splitk_floats = 0;
+  int gemm_err = 0;
+};
+
+namespace {
+
+tl_status fail(tl_layer* L, tl_status st, const char* msg) {
+  if (L) L->err = msg;
+  return st;
+}
+
+tl_status check_cuda(tl_layer* L, const char* where) {
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) {
+    if (L) L->err = std::string(where) + ": " + cudaGetErrorString(e);
+    return TL_ECUDA;
+  }
+  return TL_OK;
+}
+
+DropoutParams make_drop(const tl_layer* L, float p) {
+  DropoutParams d;
+  d.seed = L->seed;
+  d.offset = L->opt.philox_offset;
+  const bool on = L->opt.training && p > 0.0f;
+  d.thr = on ? (uint32_t)std::floor((double)p * 65536.0) : 0u;
+  d.scale = on ? 1.0f / (1.0f - p) : 1.0f;
+  return d;
+}
+
+void free_buffers(tl_layer* L) {
+  if (L->arena) {
+    cudaDeviceSynchronize();
+    cudaFree(L->arena);
+  }
+  L->arena = nullptr;
+  L->arena_bytes = 0;
+  L->have_fwd = false;
+}
+
+struct Carver {
+  char* base;
+  size_t off = 0;
+  explicit Carver(char* b) : base(b) {}
+  void* take(size_t bytes) {
+    void* p = base ? base + off : nullptr;
+    off += (bytes + 255) & ~(size_t)255;
+    return p;
+  }
+};
+
+// Lays out every buffer; with base == nullptr it only measures.
+size_t carve(tl_layer* L, char* base) {
+  Carver c(base);
+  const size_t es = dtype_size(L->opt.dtype);
+  const size_t TH = (size_t)L->T * L->H, TF = (size_t)L->T * L->F;
+  const bool ckpt = L->opt.gelu_checkpoint != 0;
+  L->qkv = c.take(3 * TH * es);
+  L->ctx = c.take(TH * es);
+  L->lse = (float*)c.take((size_t)L->B * L->nh * L->S * 4);
+  L->mean1 = (float*)c.take((size_t)L->T * 4);
+  L->rstd1 = (float*)c.take((size_t)L->T * 4);
+  L->mean2 = (float*)c.take((size_t)L->T * 4);
+  L->rstd2 = (float*)c.take((size_t)L->T * 4);
+  L->x2 = c.take(TH * es);
+  L->u = c.take(TF * es);
+  L->big = c.take(TF * es);
+  L->g = ckpt ? L->big : c.take(TF * es);
+  if (L->pre_ln) {
+    L->h1 = c.take(TH * es);
+    L->h2 = c.take(TH * es);
+    L->res1 = L->res2 = L->yout = nullptr;
+  } else {
+    L->h1 = L->h2 = nullptr;
+    L->res1 = L->opt.normalize_invertible ? nullptr : c.take(TH * es);
+    L->res2 = L->opt.normalize_invertible ? nullptr : c.take(TH * es);
+    L->yout = L->opt.normalize_invertible ? c.take(TH * es) : nullptr;
+  }
+  L->dz2 = c.take(TH * es);
+  L->dh = c.take(TH * es);
+  L->dx2 = c.take(TH * es);
+  L->da = c.take(TH * es);
+  L->dctx = c.take(TH * es);
+  L->dres = c.take(TH * es);
+  L->dqkv = c.take(3 * TH * es);
+  L->dvec = (float*)c.take((size_t)L->B * L->nh * L->S * 4);
+  const int np = std::max(std::max(ln_bwd_parts(L->T), rowdrop_parts(L->T)), colsum_parts(L->T));
+  const int maxc = std::max(3 * L->H, L->F);
+  L->part_floats = (size_t)np * maxc;
+  L->part = (float*)c.take(3 * L->part_floats * 4);
+  const int dt = L->opt.dtype, T = L->T, H = L->H, F = L->F;
+  L->splitk_floats = std::max(std::max(gemm_splitk_ws_floats(dt, H, F, T), gemm_splitk_ws_floats(dt, F, H, T)),
+                              std::max(gemm_splitk_ws_floats(dt, H, H, T), gemm_splitk_ws_floats(dt, 3 * H, H, T)));
+  L->splitk = L->splitk_floats ? (float*)c.take(L->splitk_floats * 4) : nullptr;
+  return c.off;
+}
+
+tl_status ensure_buffers(tl_layer* L) {
+  if (L->arena) {
+    int dev = -1;
+    cudaGetDevice(&dev);
+    if (dev != L->device) return fail(L, TL_EINVAL, "layer used on a different device than it was allocated on");
+    return TL_OK;
+  }
+  const size_t bytes = carve(L, nullptr);
+  cudaGetDevice(&L->device);
+  void* p = nullptr;
+  if (cudaMalloc(&p, bytes) != cudaSuccess) {
+    cudaGetLastError();
+    return fail(L, TL_ENOMEM, "cudaMalloc of the layer workspace failed");
+  }
+  L->arena = (char*)p;
+  L->arena_bytes = bytes;
+  carve(L, L->arena);
+  return TL_OK;
+}
+
+void gemm(tl_layer* L, int M, int N, int K, const void* A, int lda, bool ak, const void* B, int ldb, bool bk,
+          const EpiParams& e, cudaStream_t s) {
+  GemmDesc g{M, N, K, A, lda, ak, B, ldb, bk, L->splitk, L->splitk_floats};
+  if (gemm_run(L->opt.dtype, g, e, s) != 0) L->gemm_err = 1;
+}
+
+// Tensor pointers must be 16-byte aligned (vector loads and TMA).
+bool aligned(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
+
+EpiParams epi(int kind, void* out, int ldo) {
+  EpiParams e;
+  std::memset(&e, 0, sizeof(e));
+  e.kind = kind;
+  e.out = out;
+  e.ldo = ldo;
+  return e;
+}
+
+// Column sums of a (T, cols) stored matrix into a float32 vector.
+void bias_grad(tl_layer* L, const void* X, int cols, float* out, cudaStream_t s) {
+  colsum_run(L->opt.dtype, X, L->T, cols, L->part, s);
+  colsum_finalize_run(L->part, colsum_parts(L->T), cols, out, s);
+}
+
+void attn_fwd(tl_layer* L, const AttnArgs& a, cudaStream_t s) {
+  if (attn_tc_supports(L->opt.dtype, a)) attn_tc_fwd_run(L->opt.dtype, a, s);
+  else attn_simt_fwd_run(L->opt.dtype, a, s);
+}
+void attn_bwd(tl_layer* L, const AttnArgs& a, cudaStream_t s) {
+  if (attn_tc_supports(L->opt.dtype, a)) attn_tc_bwd_run(L->opt.dtype, a, s);
+  else attn_simt_bwd_run(L->opt.dtype, a, s);
+}
+
+AttnArgs attn_args(tl_layer* L, const float* mask) {
+  AttnArgs a;
+  std::memset(&a, 0, sizeof(a));
+  const size_t es = dtype_size(L->opt.dtype);
+  const size_t TH = (size_t)L->T * L->H;
+  a.B = L->B; a.S = L->S; a.nh = L->nh; a.d = L->d;
+  a.q = L->qkv;
+  a.k = (char*)L->qkv + TH * es;
+  a.v = (char*)L->qkv + 2 * TH * es;
+  a.mask = mask;
+  a.scale = (float)(1.0 / std::sqrt((double)L->d));
+  a.drop = make_drop(L, L->pa);
+  a.ctx = L->ctx;
+  a.lse = L->lse;
+  a.dctx = L->dctx;
+  a.dvec = L->dvec;
+  a.dqkv = L->dqkv;
+  return a;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* tl_status_string(tl_status s) {
+  switch (s) {
+    case TL_OK: return "ok";
+    case TL_EINVAL: return "invalid argument";
+    case TL_ENOMEM: return "out of device memory";
+    case TL_ESTATE: return "call out of order";
+    case TL_ECUDA: return "CUDA error";
+    case TL_ETIMEOUT: return "device wait timed out";
+    case TL_EUNSUPPORTED: return "unsupported configuration";
+  }
+  return "unknown status";
+}
+
+void layer_default_options(tl_options* o) {
+  if (!o) return;
+  std::memset(o, 0, sizeof(*o));
+  o->dtype = TL_F32;
+  o->ln_eps = 1e-12f;
+  o->philox_offset = 0;
+  o->training = 1;
+}
+
+tl_status layer_create(int batch, int seq, int hidden, int heads, int ffn, float attn_dropout, float hidden_dropout,
+                       int pre_layer_norm, uint64_t seed, tl_layer** out) {
+  if (!out) return TL_EINVAL;
+  *out = nullptr;
+  if (batch <= 0 || seq <= 0 || hidden <= 0 || heads <= 0) return TL_EINVAL;
+  if (hidden % heads != 0) return TL_EINVAL;
+  const int d = hidden / heads;
+  if (d != 16 && d != 32 && d != 64 && d != 128) return TL_EINVAL;
+  if (seq % 8 != 0 || hidden % 8 != 0) return TL_EINVAL;
+  const int F = ffn <= 0 ? 4 * hidden : ffn;
+  if (F % 8 != 0) return TL_EINVAL;
+  if (!(attn_dropout >= 0.0f && attn_dropout < 1.0f) || !(hidden_dropout >= 0.0f && hidden_dropout < 1.0f))
+    return TL_EINVAL;
+  if (!rowwise_supports_hidden(hidden)) return TL_EUNSUPPORTED;
+  if ((long long)batch * seq > (1LL << 30)) return TL_EUNSUPPORTED;
+  tl_layer* L = new (std::nothrow) tl_layer();
+  if (!L) return TL_ENOMEM;
+  L->B = batch; L->S = seq; L->H = hidden; L->nh = heads; L->d = d; L->F = F; L->T = batch * seq;
+  L->pa = attn_dropout; L->ph = hidden_dropout;
+  L->pre_ln = pre_layer_norm ? 1 : 0;
+  L->seed = seed;
+  layer_default_options(&L->opt);
+  *out = L;
+  return TL_OK;
+}
+
+tl_status layer_set_options(tl_layer* L, const tl_options* o) {
+  if (!L || !o) return TL_EINVAL;
+  if (o->dtype < TL_F32 || o->dtype > TL_BF16) return fail(L, TL_EINVAL, "unknown dtype");
+  if (!(o->ln_eps > 0.0f)) return fail(L, TL_EINVAL, "ln_eps must be positive");
+  free_buffers(L);
+  L->opt = *o;
+  L->opt.training = o->training ? 1 : 0;
+  return ensure_buffers(L);
+}
+
+tl_status layer_get_options(const tl_layer* L, tl_options* o) {
+  if (!L || !o) return TL_EINVAL;
+  *o = L->opt;
+  return TL_OK;
+}
+
+size_t layer_workspace_bytes(const tl_layer* L) { return L ? L->arena_bytes : 0; }
+
+const char* layer_last_error(const tl_layer* L) { return L ? L->err.c_str() : "null layer"; }
+
+void layer_destroy(tl_layer* L) {
+  if (!L) return;
+  free_buffers(L);
+  delete L;
+}
+
+static bool weights_ok(const tl_weights* w) {
+  return w && w->wqkv && w->bqkv && w->wo && w->bo && w->ln1_g && w->ln1_b && w->w1 && w->b1 && w->w2 && w->b2 &&
+         w->ln2_g && w->ln2_b;
+}
+
+tl_status layer_forward(tl_layer* L, const void* x, const float* mask, const tl_weights* w, void* y, void* stream) {
+  if (!L) return TL_EINVAL;
+  L->err.clear();
+  if (!x || !y || !weights_ok(w)) return fail(L, TL_EINVAL, "null tensor pointer");
+  if (x == y) return fail(L, TL_EINVAL, "y must not alias x");
+  if (!aligned(x) || !aligned(y) || !aligned(w->wqkv) || !aligned(w->wo) || !aligned(w->w1) || !aligned(w->w2) ||
+      !aligned(w->bqkv) || !aligned(w->bo) || !aligned(w->b1) || !aligned(w->b2) || !aligned(w->ln1_g) ||
+      !aligned(w->ln1_b) || !aligned(w->ln2_g) || !aligned(w->ln2_b))
+    return fail(L, TL_EINVAL, "tensor pointers must be 16-byte aligned");
+  tl_status st = ensure_buffers(L);
+  if (st != TL_OK) return st;
+  cudaStream_t s = (cudaStream_t)stream;
+  const int dt = L->opt.dtype, T = L->T, H = L->H, F = L->F;
+  const bool train = L->opt.training != 0;
+  L->have_fwd = false;
+
+  EpiParams eq = epi(EPI_QKV, L->qkv, 3 * H);
+  eq.bias = w->bqkv; eq.seq = L->S; eq.hidden = H; eq.head_dim = L->d; eq.heads = L->nh; eq.tokens = T;
+  AttnArgs aa = attn_args(L, mask);
+
+  EpiParams eo = epi(EPI_BIAS_DROP_RES, nullptr, H);
+  eo.bias = w->bo; eo.res = x; eo.drop = make_drop(L, L->ph); eo.site = 1;
+  EpiParams e1 = epi(EPI_BIAS_GELU, L->u, F);
+  e1.bias = w->b1; e1.out2 = L->g;
+  EpiParams e2 = epi(EPI_BIAS_DROP_RES, nullptr, H);
+  e2.bias = w->b2; e2.drop = make_drop(L, L->ph); e2.site = 2;
+
+  if (L->pre_ln) {
+    ln_fwd_run(dt, x, w->ln1_g, w->ln1_b, L->h1, L->mean1, L->rstd1, T, H, L->opt.ln_eps, s);
+    gemm(L, T, 3 * H, H, L->h1, H, true, w->wqkv, H, true, eq, s);
+    attn_fwd(L, aa, s);
+    eo.out = L->x2;
+    gemm(L, T, H, H, L->ctx, H, true, w->wo, H, true, eo, s);
+    ln_fwd_run(dt, L->x2, w->ln2_g, w->ln2_b, L->h2, L->mean2, L->rstd2, T, H, L->opt.ln_eps, s);
+    gemm(L, T, F, H, L->h2, H, true, w->w1, H, true, e1, s);
+    e2.res = L->x2; e2.out = y;
+    gemm(L, T, H, F, L->g, F, true, w->w2, F, true, e2, s);
+  } else {
+    // post-LN: the residual sums are kept unless LayerNorm backward runs from its outputs
+    void* r1 = L->res1 ? L->res1 : L->dres;
+    void* r2 = L->res2 ? L->res2 : L->dres;
+    gemm(L, T, 3 * H, H, x, H, true, w->wqkv, H, true, eq, s);
+    attn_fwd(L, aa, s);
+    eo.out = r1;
+    gemm(L, T, H, H, L->ctx, H, true, w->wo, H, true, eo, s);
+    ln_fwd_run(dt, r1, w->ln1_g, w->ln1_b, L->x2, L->mean1, L->rstd1, T, H, L->opt.ln_eps, s);
+    gemm(L, T, F, H, L->x2, H, true, w->w1, H, true, e1, s);
+    e2.res = L->x2; e2.out = r2;
+    gemm(L, T, H, F, L->g, F, true, w->w2, F, true, e2, s);
+    ln_fwd_run(dt, r2, w->ln2_g, w->ln2_b, y, L->mean2, L->rstd2, T, H, L->opt.ln_eps, s);
+    if (L->yout) cudaMemcpyAsync(L->yout, y, (size_t)T * H * dtype_size(dt), cudaMemcpyDeviceToDevice, s);
+  }
+  st = check_cuda(L, "layer_forward");
+  if (st != TL_OK) return st;
+  if (L->gemm_err) {
+    L->gemm_err = 0;
+    return fail(L, TL_ECUDA, "a GEMM operand could not be described to the TMA unit");
+  }
+  L->mask = mask;
+  L->have_fwd = train;
+  return TL_OK;
+}
+
+tl_status layer_backward(tl_layer* L, const void* x, const void* dy, const tl_weights* w, tl_grads* g, void* dx,
+                         void* stream) {
+  if (!L) return TL_EINVAL;
+  L->err.clear();
+  if (!L->have_fwd) return fail(L, TL_ESTATE, "backward needs a preceding training-mode forward");
+  if (!dy || !dx || !weights_ok(w) || !g) return fail(L, TL_EINVAL, "null tensor pointer");
+  if (!g->wqkv || !g->bqkv || !g->wo || !g->bo || !g->ln1_g || !g->ln1_b || !g->w1 || !g->b1 || !g->w2 || !g->b2 ||
+      !g->ln2_g || !g->ln2_b)
+    return fail(L, TL_EINVAL, "null gradient pointer");
+  const bool inv = L->opt.normalize_invertible != 0;
+  if (!x && !(inv && L->pre_ln)) return fail(L, TL_EINVAL, "x is required (only pre-LN with normalize_invertible may omit it)");
+  if (!aligned(dy) || !aligned(dx) || (x && !aligned(x))) return fail(L, TL_EINVAL, "tensor pointers must be 16-byte aligned");
+  tl_status st = ensure_buffers(L);
+  if (st != TL_OK) return st;
+  cudaStream_t s = (cudaStream_t)stream;
+  const int dt = L->opt.dtype, T = L->T, H = L->H, F = L->F;
+  const size_t es = dtype_size(dt);
+  const int lnp = ln_bwd_parts(T);
+  float* pa = L->part;
+  float* pb = L->part + L->part_floats;
+  float* pc = L->part + 2 * L->part_floats;
+  const DropoutParams dh = make_drop(L, L->ph);
+
+  auto ln_bwd = [&](const void* dyln, const void* xin, const void* yln, const float* mean, const float* rstd,
+                    const void* gamma, const void* beta, const void* res, void* dxo, void* drop_out, int site,
+                    float* dgamma, float* dbeta, float* dsum) {
+    LnBwdArgs a;
+    std::memset(&a, 0, sizeof(a));
+    a.dy = dyln; a.x = inv ? nullptr : xin; a.y = inv ? yln : nullptr;
+    a.mean = mean; a.rstd = rstd; a.gamma = gamma; a.beta = beta;
+    a.res = res; a.dx = dxo; a.drop_out = drop_out; a.drop = dh; a.site = site;
+    a.part_dgamma = pa; a.part_dbeta = pb; a.part_dsum = drop_out ? pc : nullptr;
+    a.rows = T; a.H = H;
+    ln_bwd_run(dt, a, s);
+    colsum_finalize_run(pa, lnp, H, dgamma, s);
+    colsum_finalize_run(pb, lnp, H, dbeta, s);
+    if (drop_out) colsum_finalize_run(pc, lnp, H, dsum, s);
+  };
+
+  // FFN block: dZ2 -> dW2, dU (into big), db1, dW1; returns with dU in L->big
+  auto ffn_bwd = [&](const void* ffn_in) {
+    EpiParams ew2 = epi(EPI_F32, g->w2, F);
+    if (L->opt.gelu_checkpoint) gelu_run(dt, L->u, L->big, (size_t)T * F, s);
+    gemm(L, H, F, T, L->dz2, H, false, L->g, F, false, ew2, s);          // dW2 = dZ2^T G
+    EpiParams edu = epi(EPI_DGELU, L->big, F);
+    edu.aux = L->u;
+    gemm(L, T, F, H, L->dz2, H, true, w->w2, F, false, edu, s);          // dU = (dZ2 W2) GELU'(U)
+    bias_grad(L, L->big, F, g->b1, s);                                     // db1
+    EpiParams ew1 = epi(EPI_F32, g->w1, H);
+    gemm(L, F, H, T, L->big, F, false, ffn_in, H, false, ew1, s);         // dW1 = dU^T in
+  };
+  // attention block from dA: dWo, dctx, attention backward, dbqkv, dWqkv
+  auto attn_bwd_block = [&](const void* attn_in) {
+    EpiParams ewo = epi(EPI_F32, g->wo, H);
+    gemm(L, H, H, T, L->da, H, false, L->ctx, H, false, ewo, s);          // dWo = dA^T ctx
+    EpiParams edc = epi(EPI_STORE, L->dctx, H);
+    gemm(L, T, H, H, L->da, H, true, w->wo, H, false, edc, s);            // dctx = dA Wo
+    AttnArgs aa = attn_args(L, L->mask);
+    attn_bwd(L, aa, s);
+    bias_grad(L, L->dqkv, 3 * H, g->bqkv, s);
+    EpiParams ewq = epi(EPI_F32, g->wqkv, H);
+    gemm(L, 3 * H, H, T, L->dqkv, 3 * H, false, attn_in, H, false, ewq, s);  // dWqkv = dQKV^T in
+  };
+
+  if (L->pre_ln) {
+    dropout_rows_run(dt, dy, L->dz2, dh, 2, T, H, pc, s);
+    colsum_finalize_run(pc, rowdrop_parts(T), H, g->b2, s);
+    ffn_bwd(L->h2);
+    EpiParams edh = epi(EPI_STORE, L->dh, H);
+    gemm(L, T, H, F, L->big, F, true, w->w1, H, false, edh, s);           // dH2 = dU W1
+    ln_bwd(L->dh, L->x2, L->h2, L->mean2, L->rstd2, w->ln2_g, w->ln2_b, dy, L->dx2, L->da, 1,
+           g->ln2_g, g->ln2_b, g->bo);
+    attn_bwd_block(L->h1);
+    EpiParams edh1 = epi(EPI_STORE, L->dh, H);
+    gemm(L, T, H, 3 * H, L->dqkv, 3 * H, true, w->wqkv, H, false, edh1, s);  // dH1 = dQKV Wqkv
+    ln_bwd(L->dh, x, L->h1, L->mean1, L->rstd1, w->ln1_g, w->ln1_b, L->dx2, dx, nullptr, 0,
+           g->ln1_g, g->ln1_b, nullptr);
+  } else {
+    const void* r2 = L->res2;
+    const void* r1 = L->res1;
+    ln_bwd(dy, r2, L->yout, L->mean2, L->rstd2, w->ln2_g, w->ln2_b, nullptr, L->dres, L->dz2, 2,
+           g->ln2_g, g->ln2_b, g->b2);
+    ffn_bwd(L->x2);
+    EpiParams edx2 = epi(EPI_STORE, L->dx2, H);
+    edx2.res = L->dres;
+    gemm(L, T, H, F, L->big, F, true, w->w1, H, false, edx2, s);          // dx2 = dU W1 + dres2
+    ln_bwd(L->dx2, r1, L->x2, L->mean1, L->rstd1, w->ln1_g, w->ln1_b, nullptr, L->dres, L->da, 1,
+           g->ln1_g, g->ln1_b, g->bo);
+    attn_bwd_block(x);
+    EpiParams edx = epi(EPI_STORE, dx, H);
+    edx.res = L->dres;
+    gemm(L, T, H, 3 * H, L->dqkv, 3 * H, true, w->wqkv, H, false, edx, s);  // dx = dQKV Wqkv + dres1
+  }
+  (void)es;
+  st = check_cuda(L, "layer_backward");
+  if (st == TL_OK && L->gemm_err) {
+    L->gemm_err = 0;
+    return fail(L, TL_ECUDA, "a GEMM operand could not be described to the TMA unit");
+  }
+  return st;
+}
+
+tl_status tl_device_check(void) {
+  cudaError_t e = cudaDeviceSynchronize();
+  if (e != cudaSuccess) return TL_ECUDA;
+  return device_take_error() ? TL_ETIMEOUT : TL_OK;
+}
+
+tl_status tl_dropout_keep_mask(uint64_t seed, uint64_t philox_offset, int site, float p, uint64_t e0, uint64_t n,
+                               uint8_t* keep, void* stream) {
+  if (!keep || (e0 % 8) || (n % 8) || !(p >= 0.0f && p < 1.0f) || site < 0) return TL_EINVAL;
+  if (n == 0) return TL_OK;
+  DropoutParams d;
+  d.seed = seed;
+  d.offset = philox_offset;
+  d.thr = (uint32_t)std::floor((double)p * 65536.0);
+  d.scale = 1.0f / (1.0f - p);
+  dropout_mask_run(d, site, e0, n, keep, (cudaStream_t)stream);
+  return cudaGetLastError() == cudaSuccess ? TL_OK : TL_ECUDA;
+}
+
+}  // extern "C"
