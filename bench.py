@@ -1,0 +1,405 @@
+#!/usr/bin/env python
+"""Benchmark of the fused encoder layer: forward + backward tokens/s.
+
+Workload: the BERT-Large layer of the "DeepSpeed Transformer Kernel usage
+guide" (Step 1: hidden 1024, 16 heads, sequence 128, batch 64), fp16 storage,
+attention and hidden dropout 0.1, pre-LN, no padding; synthetic seeded inputs
+(weights N(0, 0.02), x and dY N(0, 1)).  One step = layer_forward +
+layer_backward of one layer over one batch, inputs resident in HBM.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+For N > 1 it runs under torchrun, one rank per GPU, each rank an independent
+replica on its own batch (weak scaling); the time is the max over ranks.
+Rank 0 prints one JSON line.  `--impl reference` times the float64 oracle
+(the reference arm) on the host cores instead.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+from transformer_layer_pre_b200.synthetic import WORKLOADS, make_inputs  # noqa: E402
+
+METRIC = "fwd+bwd tokens/s per BERT-Large layer (B64,S128,fp16); % of tensor peak"
+WORKLOAD = "bert-large-f16"
+L2_FLUSH_BYTES = 256 << 20   # > 126 MB of L2
+CLOCK_FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+                "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+                "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+
+# ---------------------------------------------------------------- algorithmic work
+def linear_flops_per_token(h: int, f: int) -> float:
+    """Forward + backward FLOPs of the four Linear layers per token: forward
+    2*(4H^2 + 2HF) (QKV 3H^2, out-proj H^2, FFN 2HF), backward twice that."""
+    return 3.0 * 2.0 * (4 * h * h + 2 * h * f)
+
+
+def attn_flops_per_token(s: int, h: int) -> float:
+    """Forward + backward attention FLOPs per token: forward Q K^T and P V are
+    2*S*d each per head (4*S*H per token), backward four such products."""
+    return 3.0 * 4.0 * s * h
+
+
+def class_work(cls: str, w, tokens: int, elem: int) -> tuple[float, str]:
+    """(algorithmic work per step, unit) of a kernel class of the step."""
+    h, f, s = w.hidden, w.ffn, w.seq
+    th = tokens * h * elem
+    if cls == "gemm":
+        return linear_flops_per_token(h, f) * tokens, "flop"
+    if cls == "attn_fwd":
+        return 4.0 * s * h * tokens, "flop"
+    if cls == "attn_bwd":
+        return 8.0 * s * h * tokens, "flop"
+    if cls == "ln_fwd":      # two LayerNorms: read x, write y
+        return 2 * (2 * th), "byte"
+    if cls == "ln_bwd":      # two LayerNorm backwards: read dy, x, residual grad; write dx (+ dropout copy once)
+        return 2 * (4 * th) + th, "byte"
+    # dropout backward of dY (read, write) + bias-gradient column sums of dU and dQKV
+    return 2 * th + tokens * f * elem + 3 * th, "byte"
+
+
+def load_peaks() -> dict:
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as fh:
+            d = json.load(fh)
+        return {"hbm_gbs": d["hbm_gbs"], "tflops": d["bf16_tflops"], "tflops_sustained": d["bf16_tflops_sustained"],
+                "source": "measured"}
+    return {"hbm_gbs": 6650.0, "tflops": 1590.0, "tflops_sustained": 1400.0, "source": "fallback"}
+
+
+def alu_peak_tflops(sm_mhz: float, sms: int = 148) -> float:
+    """float32 FMA peak: 128 FP32 lanes per SM x 2 FLOP x SM clock."""
+    return sms * 128 * 2 * sm_mhz * 1e6 / 1e12
+
+
+# ---------------------------------------------------------------- distributed helpers
+def dist_env() -> tuple[int, int, int]:
+    return int(os.environ.get("RANK", 0)), int(os.environ.get("WORLD_SIZE", 1)), int(os.environ.get("LOCAL_RANK", 0))
+
+
+def reduce_max(value: float) -> float:
+    """Max of a float over all ranks (identity without a process group)."""
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return value
+    dev = torch.device("cuda", torch.cuda.current_device()) if dist.get_backend() == "nccl" else torch.device("cpu")
+    t = torch.tensor([value], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier() -> None:
+    import torch.distributed as dist
+    if dist.is_available() and dist.is_initialized():
+        dist.barrier()
+
+
+# ---------------------------------------------------------------- clocks
+class ClockSampler:
+    """nvidia-smi sampling of SM clocks and throttle reasons in the background."""
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={CLOCK_FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self) -> dict | None:
+        if self.proc is None or not self.path or not os.path.exists(self.path):
+            return None
+        rows = []
+        for ln in open(self.path):
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                rows.append(dict(sm=float(parts[1]), smax=float(parts[2]), power=float(parts[3]),
+                                 hw=parts[5], hwt=parts[6], swt=parts[7], cap=parts[8]))
+            except ValueError:
+                continue
+        os.unlink(self.path)
+        if not rows:
+            return None
+        load = [r for r in rows if r["power"] > 300.0] or rows
+        reasons = set()
+        for r in load:
+            for k, name in (("hw", "hw_slowdown"), ("hwt", "hw_thermal_slowdown"), ("swt", "sw_thermal_slowdown"),
+                            ("cap", "sw_power_cap")):
+                if r[k].lower().startswith("active"):
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(r["sm"] for r in load), "sm_max_mhz": max(r["smax"] for r in rows),
+                "reasons": sorted(reasons), "samples": len(rows), "samples_under_load": len(load)}
+
+
+# ---------------------------------------------------------------- oracle (reference arm / CPU baseline)
+def oracle_step(w, inp, nseq: int) -> float:
+    """Runs the float64 oracle forward + backward on the first nseq sequences
+    of the workload; returns seconds."""
+    import oracle
+    from transformer_layer_pre_b200.synthetic import to_f64
+    cfg = oracle.LayerConfig(batch=nseq, seq=w.seq, hidden=w.hidden, heads=w.heads, ffn=w.ffn,
+                             attn_dropout=float(np.float32(w.attn_dropout)),
+                             hidden_dropout=float(np.float32(w.hidden_dropout)),
+                             pre_layer_norm=w.pre_layer_norm, seed=w.seed, storage=w.dtype)
+    idx = np.arange(nseq)
+    wt = {n: to_f64(inp.weights[0][n]) for n in oracle.WEIGHT_NAMES}
+    x = to_f64(inp.x)[:nseq]
+    dy = to_f64(inp.dy)[:nseq]
+    t0 = time.perf_counter()
+    oracle.layer_forward_backward(cfg, x, None, wt, dy, seq_index=idx)
+    return time.perf_counter() - t0
+
+
+def blas_threads() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 0) for i in threadpool_info() if i.get("user_api") == "blas"]
+        if n:
+            return int(max(n))
+    except Exception:
+        pass
+    return os.cpu_count() or 1
+
+
+def size_sample(w, inp, target_s: float) -> tuple[int, float]:
+    t1 = oracle_step(w, inp, 1)
+    nseq = int(max(1, min(w.batch, round(target_s / max(t1, 1e-3)))))
+    return nseq, t1
+
+
+def cpu_baseline(w, inp, target_s: float = 15.0) -> dict:
+    nseq, _ = size_sample(w, inp, target_s)
+    t = oracle_step(w, inp, nseq)
+    return {"value": nseq * w.seq / t, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
+            "sample": f"float64 oracle forward+backward of {nseq} of the {w.batch} sequences "
+                      f"({nseq * w.seq} tokens), {t:.1f} s"}
+
+
+def run_reference(args) -> None:
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return
+    w = WORKLOADS[args.workload]
+    inp = make_inputs(w)
+    nseq, _ = size_sample(w, inp, 3.0)
+    for _ in range(args.warmup):
+        oracle_step(w, inp, nseq)
+    times = [oracle_step(w, inp, nseq) for _ in range(args.steps)]
+    tot = sum(times)
+    value = args.steps * nseq * w.seq / tot
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * tot / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": workload_config(w),
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
+                         "sample": f"each step: float64 oracle forward+backward of {nseq} of the {w.batch} "
+                                   f"sequences ({nseq * w.seq} tokens)"},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def workload_config(w) -> dict:
+    return {"workload": w.name, "batch": w.batch, "seq": w.seq, "hidden": w.hidden, "heads": w.heads,
+            "ffn": w.ffn, "attn_dropout": w.attn_dropout, "hidden_dropout": w.hidden_dropout,
+            "layer_norm": "pre" if w.pre_layer_norm else "post", "padding": w.lengths is not None,
+            "l2": "flushed (256 MiB write) between timed steps", "parallelism": "replicas"}
+
+
+# ---------------------------------------------------------------- GPU arm
+def run_ours(args) -> None:
+    import transformer_layer_pre_b200 as tlp
+    from transformer_layer_pre_b200 import Layer, WEIGHT_NAMES
+    rank, world, local = dist_env()
+    torch.cuda.set_device(local)
+    if world > 1:
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    dev = torch.device("cuda", local)
+    w = WORKLOADS[args.workload]
+    dt = {"f16": torch.float16, "bf16": torch.bfloat16, "f32": torch.float32}[w.dtype]
+    elem = 2 if w.dtype != "f32" else 4
+    inp = make_inputs(w)
+    T = w.tokens
+    layer = Layer(w.batch, w.seq, w.hidden, w.heads, w.ffn, w.attn_dropout, w.hidden_dropout, w.pre_layer_norm,
+                  w.seed, dtype=dt, gelu_checkpoint=w.gelu_checkpoint)
+    wt = {n: inp.weights[0][n].to(dev) for n in WEIGHT_NAMES}
+    x = inp.x.to(dev)
+    dy = inp.dy.to(dev)
+    mask = None if inp.mask is None else inp.mask.to(dev)
+    y = torch.empty_like(x)
+    dx = torch.empty_like(x)
+    grads = {n: torch.empty(tuple(wt[n].shape), dtype=torch.float32, device=dev) for n in WEIGHT_NAMES}
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        layer.forward(x, mask, wt, y=y)
+        layer.backward(x, dy, wt, grads=grads, dx=dx)
+
+    for _ in range(max(3, args.warmup)):
+        step()
+    tlp.device_check()
+
+    # ---- timed region: per-step events, L2 flushed between steps (outside the events)
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    barrier()
+    torch.cuda.synchronize()
+    launches0 = tlp.launch_count()
+    with ClockSampler(local) as clk:
+        for a, b in evs:
+            flush.zero_()
+            a.record(stream)
+            step()
+            b.record(stream)
+        torch.cuda.synchronize()
+    barrier()
+    launches = tlp.launch_count() - launches0
+    step_ms = [a.elapsed_time(b) for a, b in evs]
+    ms = reduce_max(sum(step_ms) / len(step_ms))
+    tlp.device_check()
+    value = world * T / (ms / 1e3)
+
+    # ---- kernel-class breakdown (same steps, library event profiler on)
+    tlp.profile_enable(True)
+    for _ in range(args.steps):
+        flush.zero_()
+        step()
+    prof = tlp.profile_read()
+    tlp.profile_enable(False)
+    peaks = load_peaks()
+    clocks = clk.summary()
+    classes = {}
+    for c, (cms, n) in prof.items():
+        if n == 0:
+            continue
+        work, unit = class_work(c, w, T, elem)
+        per_step_ms = cms / args.steps
+        classes[c] = {"ms_per_step": per_step_ms, "launch_groups_per_step": n / args.steps,
+                      "achieved": (work / (per_step_ms / 1e3)) / (1e12 if unit == "flop" else 1e9),
+                      "unit": "TFLOP/s" if unit == "flop" else "GB/s"}
+    dom = max(classes, key=lambda c: classes[c]["ms_per_step"])
+    d = classes[dom]
+    if d["unit"] == "TFLOP/s":
+        tensor = dom == "gemm" or tlp_uses_tensor_attention(dom, w)
+        if tensor:
+            bound, peak, src = "tensor", peaks["tflops_sustained"], f"{peaks['source']} bf16 sustained (fp16:bf16 = 1:1)"
+        else:
+            mhz = (clocks or {}).get("sm_mhz") or 1965.0
+            bound, peak, src = "alu", alu_peak_tflops(mhz), f"148 SMs x 128 FP32 lanes x 2 x {mhz:.0f} MHz"
+    else:
+        bound, peak, src = "hbm", peaks["hbm_gbs"], f"{peaks['source']} copy bandwidth"
+    groups = d["launch_groups_per_step"]
+    roofline = {"bound": bound, "kernel": dom, "achieved": d["achieved"], "peak": peak, "unit": d["unit"],
+                "frac": d["achieved"] / peak, "traffic": None, "peak_source": src,
+                "launches_per_step": groups}
+    step_flops = (linear_flops_per_token(w.hidden, w.ffn) + attn_flops_per_token(w.seq, w.hidden)) * T
+    tensor_frac = (step_flops / (ms / 1e3)) / (peaks["tflops_sustained"] * 1e12)
+
+    # ---- end to end through the public API, host buffers (pinned), copies inside the timed region
+    hx = inp.x.pin_memory()
+    hdy = inp.dy.pin_memory()
+    hy = torch.empty(x.shape, dtype=dt).pin_memory()
+    hdx = torch.empty(x.shape, dtype=dt).pin_memory()
+    e2e_ms = []
+    for i in range(args.warmup + args.steps):
+        flush.zero_()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        x.copy_(hx, non_blocking=True)
+        dy.copy_(hdy, non_blocking=True)
+        step()
+        hy.copy_(y, non_blocking=True)
+        hdx.copy_(dx, non_blocking=True)
+        b.record(stream)
+        b.synchronize()
+        if i >= args.warmup:
+            e2e_ms.append(a.elapsed_time(b))
+    e2e = reduce_max(sum(e2e_ms) / len(e2e_ms))
+    io = T * w.hidden * elem
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(w, inp)
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": w.dtype, "data": "synthetic (seeded N(0,0.02) weights, N(0,1) x and dY)",
+            "config": workload_config(w), "tensor_peak_frac": tensor_frac,
+            "roofline": roofline, "kernel_classes": classes, "cpu_baseline": cpu,
+            "e2e": {"value": world * T / (e2e / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": 2 * io,
+                    "d2h_bytes_per_step": 2 * io},
+            "gpu_launches": launches, "clocks": clocks,
+        }
+        print(json.dumps(line), flush=True)
+    layer.close()
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+def tlp_uses_tensor_attention(cls: str, w) -> bool:
+    """Attention runs on tensor cores when the library's tensor-core attention
+    serves this shape (16-bit storage); the SIMT kernels otherwise."""
+    import transformer_layer_pre_b200 as tlp
+    return bool(getattr(tlp, "attention_uses_tensor_cores", lambda *a: False)(w.dtype, w.heads, w.hidden // w.heads,
+                                                                              w.seq))
+
+
+def main() -> None:
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
+    ap.add_argument("--workload", default=WORKLOAD, choices=sorted(WORKLOADS))
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

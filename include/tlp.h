@@ -153,6 +153,19 @@ tl_status tl_dropout_keep_mask(uint64_t seed, uint64_t philox_offset, int site, 
  * TL_OK.  Blocks the host. */
 tl_status tl_device_check(void);
 
+/* Profiling (off by default).  While enabled, the library brackets each of
+ * its kernel launches with a pair of CUDA events on the launching stream.
+ * tl_profile_read synchronises the device, fills ms[c] (summed elapsed
+ * milliseconds) and launches[c] (bracketed launch groups) for each class c <
+ * n accumulated since the previous read, clears them, and returns the number
+ * of classes: 0 GEMM, 1 attention forward, 2 attention backward,
+ * 3 LayerNorm forward, 4 LayerNorm backward, 5 other bandwidth kernels. */
+void tl_profile_enable(int on);
+int tl_profile_read(double* ms, long long* launches, int n);
+
+/* Total number of kernels the library has launched since it was loaded. */
+long long tl_launch_count(void);
+
 const char* tl_status_string(tl_status s);
 
 #ifdef __cplusplus

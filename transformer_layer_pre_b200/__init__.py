@@ -14,7 +14,8 @@ import os
 import torch
 
 __all__ = ["Layer", "Options", "TlError", "LibraryMissing", "load_library", "dropout_keep_mask",
-           "WEIGHT_NAMES", "DTYPE_CODES", "EXPORTED_SYMBOLS", "device_check"]
+           "WEIGHT_NAMES", "DTYPE_CODES", "EXPORTED_SYMBOLS", "device_check",
+           "profile_enable", "profile_read", "launch_count", "PROFILE_CLASSES"]
 
 HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(HERE, "libtlp.so")
@@ -27,8 +28,10 @@ DTYPE_CODES = {torch.float32: 0, torch.float16: 1, torch.bfloat16: 2}
 EXPORTED_SYMBOLS = (
     "layer_create", "layer_default_options", "layer_set_options", "layer_get_options",
     "layer_forward", "layer_backward", "layer_workspace_bytes", "layer_last_error",
-    "layer_destroy", "tl_dropout_keep_mask", "tl_device_check", "tl_status_string",
+    "layer_destroy", "tl_dropout_keep_mask", "tl_device_check", "tl_profile_enable",
+    "tl_profile_read", "tl_launch_count", "tl_status_string",
 )
+PROFILE_CLASSES = ("gemm", "attn_fwd", "attn_bwd", "ln_fwd", "ln_bwd", "rowwise")
 
 
 class LibraryMissing(RuntimeError):
@@ -91,6 +94,12 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.tl_dropout_keep_mask.restype = i
     lib.tl_device_check.argtypes = []
     lib.tl_device_check.restype = i
+    lib.tl_profile_enable.argtypes = [i]
+    lib.tl_profile_enable.restype = None
+    lib.tl_profile_read.argtypes = [ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_longlong), i]
+    lib.tl_profile_read.restype = i
+    lib.tl_launch_count.argtypes = []
+    lib.tl_launch_count.restype = ctypes.c_longlong
     lib.tl_status_string.argtypes = [i]
     lib.tl_status_string.restype = ctypes.c_char_p
     _lib = lib
@@ -194,6 +203,31 @@ def device_check() -> None:
     st = lib.tl_device_check()
     if st != 0:
         raise TlError(st, lib.tl_status_string(st).decode())
+
+
+def profile_enable(on: bool) -> None:
+    load_library().tl_profile_enable(int(on))
+
+
+def profile_read() -> dict:
+    """{class: (milliseconds, bracketed launch groups)} since the last read."""
+    lib = load_library()
+    n = len(PROFILE_CLASSES)
+    ms = (ctypes.c_double * n)()
+    cnt = (ctypes.c_longlong * n)()
+    lib.tl_profile_read(ms, cnt, n)
+    return {c: (ms[i], cnt[i]) for i, c in enumerate(PROFILE_CLASSES)}
+
+
+def attention_uses_tensor_cores(dtype: str, heads: int, head_dim: int, seq: int) -> bool:
+    """Whether the library runs attention on tensor cores for this shape
+    (16-bit storage and head dim 64); the exact-float32 SIMT kernels serve
+    the rest."""
+    return dtype in ("f16", "bf16") and head_dim == 64 and seq >= 8
+
+
+def launch_count() -> int:
+    return int(load_library().tl_launch_count())
 
 
 def dropout_keep_mask(seed: int, offset: int, site: int, p: float, e0: int, n: int, device="cuda") -> torch.Tensor:

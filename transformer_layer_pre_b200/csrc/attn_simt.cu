@@ -15,6 +15,7 @@
 
 #include "common.cuh"
 #include "kernels.h"
+#include "profile.h"
 
 namespace tlp {
 
@@ -262,6 +263,7 @@ template <typename T, int D>
 void fwd_t(const AttnArgs& a, cudaStream_t s) {
   dim3 grid((a.S + kRows - 1) / kRows, a.nh, a.B);
   attn_fwd_simt<T, D><<<grid, kRows, 0, s>>>(a);
+  count_launch();
 }
 
 template <typename T, int D>
@@ -271,6 +273,7 @@ void bwd_t(const AttnArgs& a, cudaStream_t s) {
   dim3 grid((a.S + kRows - 1) / kRows, a.nh, a.B);
   attn_bwd_dq_simt<T, D><<<grid, kRows, 0, s>>>(a);
   attn_bwd_dkdv_simt<T, D><<<grid, kRows, 0, s>>>(a);
+  count_launch(3);
 }
 
 template <typename T>
@@ -284,6 +287,15 @@ void dispatch(bool fwd, const AttnArgs& a, cudaStream_t s) {
 }
 
 }  // namespace
+
+void dvec_launch(int dt, const AttnArgs& a, cudaStream_t s) {
+  const size_t rows = (size_t)a.B * a.nh * a.S;
+  const unsigned blocks = (unsigned)((rows + 255) / 256);
+  if (dt == DT_F32) attn_dvec_kernel<float><<<blocks, 256, 0, s>>>(a);
+  else if (dt == DT_F16) attn_dvec_kernel<half_t><<<blocks, 256, 0, s>>>(a);
+  else attn_dvec_kernel<bf16_t><<<blocks, 256, 0, s>>>(a);
+  count_launch();
+}
 
 void attn_simt_fwd_run(int dt, const AttnArgs& a, cudaStream_t s) {
   if (dt == DT_F32) dispatch<float>(true, a, s);

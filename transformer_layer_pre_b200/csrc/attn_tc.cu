@@ -1,0 +1,773 @@
+// attn_tc.cu — tensor-core (tcgen05) attention for 16-bit storage, head dim 64,
+// forward and backward.  The S x S score matrix never reaches HBM.
+//
+// Computes, per (sequence b, head h), with d = 64 and c = 1/sqrt(d):
+//   S = Q K^T * c + mask_b (additive over keys); P = softmax over keys;
+//   Pd = P * keep / (1 - p) (dropout on the probabilities, site 0);
+//   ctx = Pd V, heads merged into (B*S, H); LSE per row kept for backward.
+// ("Transformer deployment", section 1 pseudo-code: softmax(Q K^T / sqrt(d_k))
+// then the product with V; "DeepSpeed Transformer Kernel usage guide", Step 3:
+// the attention-dropout input is not stored, backward regenerates it.)
+// Backward regenerates P from LSE and the dropout bits from Philox:
+//   dV = Pd^T dO; dPd = dO V^T; dP = dPd * keep / (1 - p);
+//   dS = P * (dP - D) with D = rowsum(dO * O); dQ = dS K c; dK = dS^T Q c.
+//
+// Tiles are 128 queries x 128 keys.  One elected thread issues every MMA
+// (M = 128) into TMEM; softmax warps own one TMEM lane (one query row) each,
+// so each thread's dropout bits are its own row's Philox draws.  P and dS go
+// back to shared memory in the 128-byte-swizzled layout TMA uses for a
+// [rows][64] tile, which serves as a K-major operand (rows x keys) and as an
+// MN-major operand (keys x rows) alike; Q, K, V and dO tiles likewise serve
+// both roles without any transpose.  TMA loads are per CTA (no multicast).
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <math.h>
+
+#include <algorithm>
+#include <type_traits>
+
+#include "kernels.h"
+#include "profile.h"
+#include "sm100.cuh"
+
+namespace tlp {
+
+using namespace sm100;
+
+// D = rowsum(dO * O) per (b, h, query), attn_simt.cu.
+void dvec_launch(int dt, const AttnArgs& a, cudaStream_t s);
+
+namespace {
+
+constexpr int HD = 64;                  // head dim served here
+constexpr int TILE = 128;               // queries or keys per tile
+constexpr int TB = TILE * HD * 2;       // bytes of one [128][64] 16-bit tile (16 KB)
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kLn2 = 0.6931471805599453f;
+
+struct AttnTc {
+  int B, S, nh, H;
+  const float* mask;
+  float scale;          // 1/sqrt(d)
+  DropoutParams drop;
+  void* ctx;
+  float* lse;
+  const void* ctx_in;   // backward: forward output O (for D)
+  const void* dctx;
+  const float* dvec;    // precomputed D, or null to compute it in-kernel
+  void* dqkv;
+  int fuse_dq;
+  int bf16;
+  int* err;
+};
+
+__device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
+  return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
+}
+
+// Descriptors of a [128 rows][64] swizzled tile at `base` (K-major operand:
+// rows x 64, K step kk of 16 columns) and of a [128 rows][128] pair of such
+// tiles (regions of 16 KB holding columns 0-63 and 64-127).
+__device__ __forceinline__ uint64_t dk_tile(uint32_t base, int kk) { return smem_desc_sw128(base + kk * 32, 16, 1024); }
+__device__ __forceinline__ uint64_t dk_pair(uint32_t base, int kk) {
+  return smem_desc_sw128(base + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024);
+}
+// MN-major views (K runs along the rows, 16 rows per step): a single tile
+// (64 MN elements) or a pair (128 MN elements, second 64 at +16 KB).
+__device__ __forceinline__ uint64_t dmn_tile(uint32_t base, int kk) { return smem_desc_sw128(base + kk * 2048, 8192, 1024); }
+__device__ __forceinline__ uint64_t dmn_pair(uint32_t base, int kk) { return smem_desc_sw128(base + kk * 2048, 16384, 1024); }
+
+// Stores 8 values as the 8-element chunk k8 (0..15) of row r of a
+// [128][128] swizzled pair.
+template <typename T>
+__device__ __forceinline__ void pair_store8(uint8_t* pair, int r, int k8, const float (&v)[8]) {
+  const int region = k8 >> 3, c = k8 & 7;
+  store8<T>(reinterpret_cast<T*>(pair + region * 16384 + r * 128 + ((c ^ (r & 7)) << 4)), v);
+}
+
+__device__ __forceinline__ float mask_log2(const AttnTc& a, int b, int key) {
+  if (key >= a.S) return -INFINITY;
+  return a.mask ? a.mask[(size_t)b * a.S + key] * kLog2e : 0.0f;
+}
+
+// ============================================================================ forward
+// Warps: 0 TMA, 1 MMA (+TMEM owner), 2-5 softmax (thread = query row).
+constexpr int kFwdThreads = 192;
+constexpr int kFwdSmem = 5 * TB + 1024 + 256;   // Q, K, V, P pair
+
+template <typename T>
+__global__ void __launch_bounds__(kFwdThreads)
+    attn_fwd_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
+                const __grid_constant__ CUtensorMap tv, AttnTc a) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* sm = align1024(smem_raw);
+  uint8_t* sQ = sm;
+  uint8_t* sK = sm + TB;
+  uint8_t* sV = sm + 2 * TB;
+  uint8_t* sP = sm + 3 * TB;
+  uint64_t* bar = reinterpret_cast<uint64_t*>(sm + 5 * TB);
+  uint64_t *q_full = bar, *kv_full = bar + 1, *kv_empty = bar + 2, *s_full = bar + 3, *s_free = bar + 4,
+           *p_full = bar + 5, *o_full = bar + 6, *o_free = bar + 7;
+  uint32_t* tslot = reinterpret_cast<uint32_t*>(bar + 8);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int h = blockIdx.y, b = blockIdx.z;
+  const int S = a.S;
+  const int row0 = (b * a.nh + h) * S;
+  const int q0 = blockIdx.x * TILE;
+  const int ntiles = (S + TILE - 1) / TILE;
+
+  if (threadIdx.x == 0) {
+    mbar_init(q_full, 1);
+    mbar_init(kv_full, 1);
+    mbar_init(kv_empty, 1);
+    mbar_init(s_full, 1);
+    mbar_init(s_free, 128);
+    mbar_init(p_full, 128);
+    mbar_init(o_full, 1);
+    mbar_init(o_free, 128);
+    fence_barrier_init();
+  }
+  if (warp == 1) tmem_alloc(tslot, 256);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tslot;
+  const uint32_t tS = tmem, tO = tmem + 128;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      bool ok = true;
+      mbar_arrive_expect_tx(q_full, TB);
+      tma_load_2d(sQ, &tq, q_full, 0, row0 + q0);
+      int j = 0;
+      for (; j < ntiles; ++j) {
+        if (!mbar_wait(kv_empty, (j & 1) ^ 1, a.err, 11)) { ok = false; break; }
+        mbar_arrive_expect_tx(kv_full, 2 * TB);
+        tma_load_2d(sK, &tk, kv_full, 0, row0 + j * TILE);
+        tma_load_2d(sV, &tv, kv_full, 0, row0 + j * TILE);
+      }
+      if (!ok) {
+        mbar_wait(q_full, 0, nullptr, 0);
+        if (j > 0) mbar_wait(kv_full, (j - 1) & 1, nullptr, 0);
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      const uint32_t id_s = idesc_f16(128, 128, a.bf16 != 0, false, false);
+      const uint32_t id_o = idesc_f16(128, 64, a.bf16 != 0, false, true);
+      const uint32_t aQ = smem_u32(sQ), aK = smem_u32(sK), aV = smem_u32(sV), aP = smem_u32(sP);
+      if (mbar_wait(q_full, 0, a.err, 12)) {
+        for (int j = 0; j < ntiles; ++j) {
+          if (!mbar_wait(kv_full, j & 1, a.err, 13)) break;
+          if (!mbar_wait(s_free, (j & 1) ^ 1, a.err, 14)) break;
+          tc_fence_after();
+#pragma unroll
+          for (int kk = 0; kk < HD / 16; ++kk) mma_f16(tS, dk_tile(aQ, kk), dk_tile(aK, kk), id_s, kk > 0);
+          mma_commit(s_full);
+          if (!mbar_wait(p_full, j & 1, a.err, 15)) break;
+          if (!mbar_wait(o_free, (j & 1) ^ 1, a.err, 16)) break;
+          tc_fence_after();
+#pragma unroll
+          for (int kk = 0; kk < TILE / 16; ++kk) mma_f16(tO, dk_pair(aP, kk), dmn_tile(aV, kk), id_o, kk > 0);
+          mma_commit(o_full);
+          mma_commit(kv_empty);
+        }
+      }
+    }
+  } else {
+    const int quarter = warp & 3;
+    const int r = quarter * 32 + lane;
+    const int i = q0 + r;
+    const uint32_t lo = (uint32_t)(quarter * 32) << 16;
+    const float c2 = a.scale * kLog2e;
+    const float dsc = a.drop.thr ? a.drop.scale : 1.0f;
+    const uint64_t erow = ((uint64_t)row0 + (uint64_t)i) * (uint64_t)S;
+    float o[HD];
+#pragma unroll
+    for (int c = 0; c < HD; ++c) o[c] = 0.0f;
+    float m = -INFINITY, l = 0.0f, alpha_prev = 0.0f;
+    bool ok = true;
+    for (int j = 0; j < ntiles && ok; ++j) {
+      const int k0 = j * TILE;
+      if (!mbar_wait_warp(s_full, j & 1, a.err, 17)) { ok = false; break; }
+      tc_fence_after();
+      // pass 1: row maximum of the scaled, masked scores (log2 domain)
+      float mx = -INFINITY;
+#pragma unroll 1
+      for (int c = 0; c < 4; ++c) {
+        float sv[32];
+        tmem_ld32(tS + lo + c * 32, sv);
+#pragma unroll
+        for (int t = 0; t < 32; ++t) mx = fmaxf(mx, fmaf(sv[t], c2, mask_log2(a, b, k0 + c * 32 + t)));
+      }
+      const float m_new = fmaxf(m, mx);
+      const float alpha = (m == -INFINITY) ? 0.0f : exp2f(m - m_new);
+      // the P buffer and O_part of the previous tile must be consumed first
+      if (j > 0) {
+        if (!mbar_wait_warp(o_full, (j - 1) & 1, a.err, 18)) { ok = false; break; }
+        tc_fence_after();
+        float pv[32];
+        tmem_ld32(tO + lo, pv);
+#pragma unroll
+        for (int c = 0; c < 32; ++c) o[c] = fmaf(o[c], alpha_prev, pv[c]);
+        tmem_ld32(tO + lo + 32, pv);
+#pragma unroll
+        for (int c = 0; c < 32; ++c) o[32 + c] = fmaf(o[32 + c], alpha_prev, pv[c]);
+        tc_fence_before();
+        mbar_arrive(o_free);
+      }
+      // pass 2: probabilities, dropout, P to shared memory
+      float lsum = 0.0f;
+#pragma unroll 1
+      for (int c = 0; c < 4; ++c) {
+        float sv[32];
+        tmem_ld32(tS + lo + c * 32, sv);
+#pragma unroll
+        for (int g = 0; g < 4; ++g) {
+          const int kb = k0 + c * 32 + g * 8;
+          const uint32_t bits = a.drop.thr ? dropout_bits8(a.drop, 0, (erow + (uint64_t)kb) >> 3) : 0xFFu;
+          float pv[8];
+#pragma unroll
+          for (int t = 0; t < 8; ++t) {
+            const float x = fmaf(sv[g * 8 + t], c2, mask_log2(a, b, kb + t));
+            const float p = (x == -INFINITY || m_new == -INFINITY) ? 0.0f : exp2f(x - m_new);
+            lsum += p;
+            pv[t] = ((bits >> t) & 1u) ? p * dsc : 0.0f;
+          }
+          pair_store8<T>(sP, r, c * 4 + g, pv);
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(s_free);
+      fence_proxy_async_smem();
+      mbar_arrive(p_full);
+      l = l * alpha + lsum;
+      m = m_new;
+      alpha_prev = alpha;
+    }
+    if (ok && mbar_wait_warp(o_full, (ntiles - 1) & 1, a.err, 19)) {
+      tc_fence_after();
+      float pv[32];
+      tmem_ld32(tO + lo, pv);
+#pragma unroll
+      for (int c = 0; c < 32; ++c) o[c] = fmaf(o[c], alpha_prev, pv[c]);
+      tmem_ld32(tO + lo + 32, pv);
+#pragma unroll
+      for (int c = 0; c < 32; ++c) o[32 + c] = fmaf(o[32 + c], alpha_prev, pv[c]);
+      if (i < S) {
+        const float inv = l > 0.0f ? 1.0f / l : 0.0f;
+        T* dst = static_cast<T*>(a.ctx) + ((size_t)b * S + i) * a.H + h * HD;
+#pragma unroll
+        for (int c = 0; c < HD; c += 8) {
+          float v[8];
+#pragma unroll
+          for (int t = 0; t < 8; ++t) v[t] = o[c + t] * inv;
+          store8<T>(dst + c, v);
+        }
+        a.lse[row0 + i] = l > 0.0f ? (m + log2f(l)) * kLn2 : INFINITY;
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc(tmem, 256);
+}
+
+// ============================================================================ backward
+// Warps: 0 TMA, 1 MMA (+TMEM owner), 2-9 softmax: warp w serves TMEM lanes
+// 32*(w%4).. and key columns 64*((w-2)/4) .. +63 of each 128-key tile.
+constexpr int kBwdThreads = 320;
+constexpr int kSoftThreads = 256;
+
+// Per-thread D_i = sum_c dO[i, c] O[i, c] (from global memory).
+template <typename T>
+__device__ __forceinline__ float dvec_row(const AttnTc& a, int b, int h, int i) {
+  const size_t off = ((size_t)b * a.S + i) * a.H + h * HD;
+  const T* dO = static_cast<const T*>(a.dctx) + off;
+  const T* O = static_cast<const T*>(a.ctx_in) + off;
+  float s = 0.0f;
+#pragma unroll
+  for (int c = 0; c < HD; c += 8) {
+    float x[8], y[8];
+    load8<T>(dO + c, x);
+    load8<T>(O + c, y);
+#pragma unroll
+    for (int t = 0; t < 8; ++t) s = fmaf(x[t], y[t], s);
+  }
+  return s;
+}
+
+// Softmax-side work of one (query tile, key tile) pair for one thread: row r
+// of the tile (query i), key columns [kc0, kc0 + 64) of the tile starting at
+// key k0.  Writes Pd (if sPd) and dS rows to shared memory.
+template <typename T>
+__device__ __forceinline__ void bwd_pair_rows(const AttnTc& a, int b, int row0, int i, int r, int k0, int kc0,
+                                              uint32_t tS, uint32_t tdP, uint32_t lo, float lse2, float Di,
+                                              uint8_t* sPd, uint8_t* sdS) {
+  const float c2 = a.scale * kLog2e;
+  const float dsc = a.drop.thr ? a.drop.scale : 1.0f;
+  const uint64_t erow = ((uint64_t)row0 + (uint64_t)i) * (uint64_t)a.S;
+  const bool row_ok = i < a.S;
+#pragma unroll 1
+  for (int c = 0; c < 2; ++c) {
+    float sv[32], dv[32];
+    tmem_ld32(tS + lo + kc0 + c * 32, sv);
+    tmem_ld32(tdP + lo + kc0 + c * 32, dv);
+#pragma unroll
+    for (int g = 0; g < 4; ++g) {
+      const int kt = kc0 + c * 32 + g * 8;   // column within the key tile
+      const int kb = k0 + kt;
+      const uint32_t bits = a.drop.thr ? dropout_bits8(a.drop, 0, (erow + (uint64_t)kb) >> 3) : 0xFFu;
+      float pd[8], ds[8];
+#pragma unroll
+      for (int t = 0; t < 8; ++t) {
+        const float x = fmaf(sv[g * 8 + t], c2, mask_log2(a, b, kb + t));
+        const float p = (!row_ok || x == -INFINITY) ? 0.0f : exp2f(x - lse2);
+        const bool keep = (bits >> t) & 1u;
+        pd[t] = keep ? p * dsc : 0.0f;
+        const float dp = keep ? dv[g * 8 + t] * dsc : 0.0f;
+        ds[t] = p * (dp - Di);
+      }
+      if (sPd) pair_store8<T>(sPd, r, kt >> 3, pd);
+      pair_store8<T>(sdS, r, kt >> 3, ds);
+    }
+  }
+}
+
+// Key-tile CTA: dK, dV of 128 keys accumulated over every query tile; with
+// fuse_dq (one key tile covers the sequence) also dQ of each query tile.
+constexpr int kBwdKvSmem = 8 * TB + 1024 + 256;   // K, V, Q[2], dO... see layout below
+
+template <typename T>
+__global__ void __launch_bounds__(kBwdThreads)
+    attn_bwd_kv_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
+                   const __grid_constant__ CUtensorMap tv, const __grid_constant__ CUtensorMap tdo, AttnTc a) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* sm = align1024(smem_raw);
+  uint8_t* sK = sm;
+  uint8_t* sV = sm + TB;
+  uint8_t* sQ = sm + 2 * TB;    // one stage: Q then dO
+  uint8_t* sdO = sm + 3 * TB;
+  uint8_t* sPd = sm + 4 * TB;   // pair
+  uint8_t* sdS = sm + 6 * TB;   // pair
+  uint64_t* bar = reinterpret_cast<uint64_t*>(sm + 8 * TB);
+  uint64_t *kv_full = bar, *qd_full = bar + 1, *qd_empty = bar + 2, *s_full = bar + 3, *s_free = bar + 4,
+           *ds_full = bar + 5, *ds_free = bar + 6, *dq_full = bar + 7, *dq_free = bar + 8, *acc_full = bar + 9;
+  uint32_t* tslot = reinterpret_cast<uint32_t*>(bar + 10);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int h = blockIdx.y, b = blockIdx.z;
+  const int S = a.S;
+  const int row0 = (b * a.nh + h) * S;
+  const int k0 = blockIdx.x * TILE;
+  const int nq = (S + TILE - 1) / TILE;
+
+  if (threadIdx.x == 0) {
+    mbar_init(kv_full, 1);
+    mbar_init(qd_full, 1);
+    mbar_init(qd_empty, 1);
+    mbar_init(s_full, 1);
+    mbar_init(s_free, kSoftThreads);
+    mbar_init(ds_full, kSoftThreads);
+    mbar_init(ds_free, 1);
+    mbar_init(dq_full, 1);
+    mbar_init(dq_free, kSoftThreads);
+    mbar_init(acc_full, 1);
+    fence_barrier_init();
+  }
+  if (warp == 1) tmem_alloc(tslot, 512);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tslot;
+  const uint32_t tS = tmem, tdP = tmem + 128, tdV = tmem + 256, tdK = tmem + 320, tdQ = tmem + 384;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      bool ok = true;
+      mbar_arrive_expect_tx(kv_full, 2 * TB);
+      tma_load_2d(sK, &tk, kv_full, 0, row0 + k0);
+      tma_load_2d(sV, &tv, kv_full, 0, row0 + k0);
+      int i = 0;
+      for (; i < nq; ++i) {
+        if (!mbar_wait(qd_empty, (i & 1) ^ 1, a.err, 21)) { ok = false; break; }
+        mbar_arrive_expect_tx(qd_full, 2 * TB);
+        tma_load_2d(sQ, &tq, qd_full, 0, row0 + i * TILE);
+        tma_load_2d(sdO, &tdo, qd_full, h * HD, b * S + i * TILE);
+      }
+      if (!ok) {
+        mbar_wait(kv_full, 0, nullptr, 0);
+        if (i > 0) mbar_wait(qd_full, (i - 1) & 1, nullptr, 0);
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      const bool bf = a.bf16 != 0;
+      const uint32_t id_kk = idesc_f16(128, 128, bf, false, false);
+      const uint32_t id_mm = idesc_f16(128, 64, bf, true, true);
+      const uint32_t id_km = idesc_f16(128, 64, bf, false, true);
+      const uint32_t aK = smem_u32(sK), aV = smem_u32(sV), aQ = smem_u32(sQ), adO = smem_u32(sdO);
+      const uint32_t aPd = smem_u32(sPd), adS = smem_u32(sdS);
+      bool ok = mbar_wait(kv_full, 0, a.err, 22);
+      for (int i = 0; i < nq && ok; ++i) {
+        if (!(ok = mbar_wait(qd_full, i & 1, a.err, 23))) break;
+        if (!(ok = mbar_wait(s_free, (i & 1) ^ 1, a.err, 24))) break;
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < HD / 16; ++kk) mma_f16(tS, dk_tile(aQ, kk), dk_tile(aK, kk), id_kk, kk > 0);
+#pragma unroll
+        for (int kk = 0; kk < HD / 16; ++kk) mma_f16(tdP, dk_tile(adO, kk), dk_tile(aV, kk), id_kk, kk > 0);
+        mma_commit(s_full);
+        if (!(ok = mbar_wait(ds_full, i & 1, a.err, 25))) break;
+        tc_fence_after();
+        // dV += Pd^T dO ; dK += dS^T Q   (K runs over the 128 queries)
+#pragma unroll
+        for (int kk = 0; kk < TILE / 16; ++kk)
+          mma_f16(tdV, dmn_pair(aPd, kk), dmn_tile(adO, kk), id_mm, (i > 0 || kk > 0) ? 1u : 0u);
+#pragma unroll
+        for (int kk = 0; kk < TILE / 16; ++kk)
+          mma_f16(tdK, dmn_pair(adS, kk), dmn_tile(aQ, kk), id_mm, (i > 0 || kk > 0) ? 1u : 0u);
+        if (a.fuse_dq) {
+          if (!(ok = mbar_wait(dq_free, (i & 1) ^ 1, a.err, 26))) break;
+          tc_fence_after();
+          // dQ = dS K   (K runs over the 128 keys)
+#pragma unroll
+          for (int kk = 0; kk < TILE / 16; ++kk) mma_f16(tdQ, dk_pair(adS, kk), dmn_tile(aK, kk), id_km, kk > 0);
+          mma_commit(dq_full);
+        }
+        mma_commit(ds_free);
+        mma_commit(qd_empty);
+      }
+      if (ok) mma_commit(acc_full);
+    }
+  } else {
+    const int sw = warp - 2;
+    const int quarter = warp & 3;
+    const int half = sw >> 2;
+    const int r = quarter * 32 + lane;
+    const uint32_t lo = (uint32_t)(quarter * 32) << 16;
+    bool ok = true;
+    for (int i = 0; i < nq && ok; ++i) {
+      const int q = i * TILE + r;
+      const bool qv = q < S;
+      const float lse2 = qv ? a.lse[row0 + q] * kLog2e : INFINITY;
+      const float Di = qv ? (a.dvec ? a.dvec[row0 + q] : dvec_row<T>(a, b, h, q)) : 0.0f;
+      if (!(ok = mbar_wait_warp(s_full, i & 1, a.err, 27))) break;
+      tc_fence_after();
+      if (!(ok = mbar_wait_warp(ds_free, (i & 1) ^ 1, a.err, 28))) break;
+      bwd_pair_rows<T>(a, b, row0, q, r, k0, half * 64, tS, tdP, lo, lse2, Di, sPd, sdS);
+      tc_fence_before();
+      mbar_arrive(s_free);
+      fence_proxy_async_smem();
+      mbar_arrive(ds_full);
+      if (a.fuse_dq) {
+        if (!(ok = mbar_wait_warp(dq_full, i & 1, a.err, 29))) break;
+        tc_fence_after();
+        float v[32];
+        tmem_ld32(tdQ + lo + half * 32, v);
+        tc_fence_before();
+        mbar_arrive(dq_free);
+        if (qv) {
+          T* dst = static_cast<T*>(a.dqkv) + ((size_t)b * S + q) * 3 * a.H + h * HD + half * 32;
+#pragma unroll
+          for (int c = 0; c < 32; c += 8) {
+            float w8[8];
+#pragma unroll
+            for (int t = 0; t < 8; ++t) w8[t] = v[c + t] * a.scale;
+            store8<T>(dst + c, w8);
+          }
+        }
+      }
+    }
+    if (ok && mbar_wait_warp(acc_full, 0, a.err, 30)) {
+      tc_fence_after();
+      const int key = k0 + r;
+      float dv[32], dk[32];
+      tmem_ld32(tdV + lo + half * 32, dv);
+      tmem_ld32(tdK + lo + half * 32, dk);
+      if (key < S) {
+        T* dst = static_cast<T*>(a.dqkv) + ((size_t)b * S + key) * 3 * a.H + h * HD + half * 32;
+#pragma unroll
+        for (int c = 0; c < 32; c += 8) {
+          float w8[8], u8[8];
+#pragma unroll
+          for (int t = 0; t < 8; ++t) {
+            w8[t] = dk[c + t] * a.scale;
+            u8[t] = dv[c + t];
+          }
+          store8<T>(dst + a.H + c, w8);
+          store8<T>(dst + 2 * a.H + c, u8);
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc(tmem, 512);
+}
+
+// Query-tile CTA: dQ of 128 queries accumulated over every key tile (used
+// when the sequence spans several key tiles).
+constexpr int kBwdQSmem = 6 * TB + 1024 + 256;
+
+template <typename T>
+__global__ void __launch_bounds__(kBwdThreads)
+    attn_bwd_q_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
+                  const __grid_constant__ CUtensorMap tv, const __grid_constant__ CUtensorMap tdo, AttnTc a) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* sm = align1024(smem_raw);
+  uint8_t* sQ = sm;
+  uint8_t* sdO = sm + TB;
+  uint8_t* sK = sm + 2 * TB;
+  uint8_t* sV = sm + 3 * TB;
+  uint8_t* sdS = sm + 4 * TB;   // pair
+  uint64_t* bar = reinterpret_cast<uint64_t*>(sm + 6 * TB);
+  uint64_t *qd_full = bar, *kv_full = bar + 1, *kv_empty = bar + 2, *s_full = bar + 3, *s_free = bar + 4,
+           *ds_full = bar + 5, *ds_free = bar + 6, *acc_full = bar + 7;
+  uint32_t* tslot = reinterpret_cast<uint32_t*>(bar + 8);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int h = blockIdx.y, b = blockIdx.z;
+  const int S = a.S;
+  const int row0 = (b * a.nh + h) * S;
+  const int q0 = blockIdx.x * TILE;
+  const int nk = (S + TILE - 1) / TILE;
+
+  if (threadIdx.x == 0) {
+    mbar_init(qd_full, 1);
+    mbar_init(kv_full, 1);
+    mbar_init(kv_empty, 1);
+    mbar_init(s_full, 1);
+    mbar_init(s_free, kSoftThreads);
+    mbar_init(ds_full, kSoftThreads);
+    mbar_init(ds_free, 1);
+    mbar_init(acc_full, 1);
+    fence_barrier_init();
+  }
+  if (warp == 1) tmem_alloc(tslot, 512);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tslot;
+  const uint32_t tS = tmem, tdP = tmem + 128, tdQ = tmem + 256;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      bool ok = true;
+      mbar_arrive_expect_tx(qd_full, 2 * TB);
+      tma_load_2d(sQ, &tq, qd_full, 0, row0 + q0);
+      tma_load_2d(sdO, &tdo, qd_full, h * HD, b * S + q0);
+      int j = 0;
+      for (; j < nk; ++j) {
+        if (!mbar_wait(kv_empty, (j & 1) ^ 1, a.err, 31)) { ok = false; break; }
+        mbar_arrive_expect_tx(kv_full, 2 * TB);
+        tma_load_2d(sK, &tk, kv_full, 0, row0 + j * TILE);
+        tma_load_2d(sV, &tv, kv_full, 0, row0 + j * TILE);
+      }
+      if (!ok) {
+        mbar_wait(qd_full, 0, nullptr, 0);
+        if (j > 0) mbar_wait(kv_full, (j - 1) & 1, nullptr, 0);
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      const bool bf = a.bf16 != 0;
+      const uint32_t id_kk = idesc_f16(128, 128, bf, false, false);
+      const uint32_t id_km = idesc_f16(128, 64, bf, false, true);
+      const uint32_t aK = smem_u32(sK), aV = smem_u32(sV), aQ = smem_u32(sQ), adO = smem_u32(sdO);
+      const uint32_t adS = smem_u32(sdS);
+      bool ok = mbar_wait(qd_full, 0, a.err, 32);
+      for (int j = 0; j < nk && ok; ++j) {
+        if (!(ok = mbar_wait(kv_full, j & 1, a.err, 33))) break;
+        if (!(ok = mbar_wait(s_free, (j & 1) ^ 1, a.err, 34))) break;
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < HD / 16; ++kk) mma_f16(tS, dk_tile(aQ, kk), dk_tile(aK, kk), id_kk, kk > 0);
+#pragma unroll
+        for (int kk = 0; kk < HD / 16; ++kk) mma_f16(tdP, dk_tile(adO, kk), dk_tile(aV, kk), id_kk, kk > 0);
+        mma_commit(s_full);
+        if (!(ok = mbar_wait(ds_full, j & 1, a.err, 35))) break;
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < TILE / 16; ++kk)
+          mma_f16(tdQ, dk_pair(adS, kk), dmn_tile(aK, kk), id_km, (j > 0 || kk > 0) ? 1u : 0u);
+        mma_commit(ds_free);
+        mma_commit(kv_empty);
+      }
+      if (ok) mma_commit(acc_full);
+    }
+  } else {
+    const int sw = warp - 2;
+    const int quarter = warp & 3;
+    const int half = sw >> 2;
+    const int r = quarter * 32 + lane;
+    const uint32_t lo = (uint32_t)(quarter * 32) << 16;
+    const int q = q0 + r;
+    const bool qv = q < S;
+    const float lse2 = qv ? a.lse[row0 + q] * kLog2e : INFINITY;
+    const float Di = qv ? (a.dvec ? a.dvec[row0 + q] : dvec_row<T>(a, b, h, q)) : 0.0f;
+    bool ok = true;
+    for (int j = 0; j < nk && ok; ++j) {
+      if (!(ok = mbar_wait_warp(s_full, j & 1, a.err, 36))) break;
+      tc_fence_after();
+      if (!(ok = mbar_wait_warp(ds_free, (j & 1) ^ 1, a.err, 37))) break;
+      bwd_pair_rows<T>(a, b, row0, q, r, j * TILE, half * 64, tS, tdP, lo, lse2, Di, nullptr, sdS);
+      tc_fence_before();
+      mbar_arrive(s_free);
+      fence_proxy_async_smem();
+      mbar_arrive(ds_full);
+    }
+    if (ok && mbar_wait_warp(acc_full, 0, a.err, 38)) {
+      tc_fence_after();
+      float v[32];
+      tmem_ld32(tdQ + lo + half * 32, v);
+      if (qv) {
+        T* dst = static_cast<T*>(a.dqkv) + ((size_t)b * S + q) * 3 * a.H + h * HD + half * 32;
+#pragma unroll
+        for (int c = 0; c < 32; c += 8) {
+          float w8[8];
+#pragma unroll
+          for (int t = 0; t < 8; ++t) w8[t] = v[c + t] * a.scale;
+          store8<T>(dst + c, w8);
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc(tmem, 512);
+}
+
+// ------------------------------------------------------------------ host side
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    cudaDriverEntryPointQueryResult q;
+    void* p = nullptr;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  return fn;
+}
+
+// [rows][cols] row-major 16-bit matrix with row stride ld; box 64 x 128 rows.
+bool map_tile(CUtensorMap* m, const void* p, bool bf16, uint64_t cols, uint64_t rows, uint64_t ld) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {ld * 2};
+  cuuint32_t box[2] = {64, 128};
+  cuuint32_t es[2] = {1, 1};
+  return fn(m, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<void*>(p),
+            dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+int* attn_error_word() {
+  static int* p = nullptr;
+  if (!p) cudaMalloc(&p, sizeof(int)), cudaMemset(p, 0, sizeof(int));
+  return p;
+}
+
+AttnTc make_args(int dt, const AttnArgs& a) {
+  AttnTc t;
+  t.B = a.B; t.S = a.S; t.nh = a.nh; t.H = a.nh * a.d;
+  t.mask = a.mask;
+  t.scale = a.scale;
+  t.drop = a.drop;
+  t.ctx = a.ctx;
+  t.lse = a.lse;
+  t.ctx_in = a.ctx;
+  t.dctx = a.dctx;
+  t.dvec = nullptr;
+  t.dqkv = a.dqkv;
+  t.fuse_dq = 0;
+  t.bf16 = dt == DT_BF16;
+  t.err = attn_error_word();
+  return t;
+}
+
+template <typename T>
+void fwd_t(const AttnArgs& a, cudaStream_t s) {
+  AttnTc t = make_args(std::is_same<T, bf16_t>::value ? DT_BF16 : DT_F16, a);
+  const uint64_t rows = (uint64_t)a.B * a.nh * a.S;
+  CUtensorMap mq, mk, mv;
+  if (!map_tile(&mq, a.q, t.bf16, HD, rows, HD) || !map_tile(&mk, a.k, t.bf16, HD, rows, HD) ||
+      !map_tile(&mv, a.v, t.bf16, HD, rows, HD))
+    return;
+  static bool attr = false;
+  if (!attr) {
+    cudaFuncSetAttribute(attn_fwd_tc<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, kFwdSmem);
+    attr = true;
+  }
+  dim3 grid((a.S + TILE - 1) / TILE, a.nh, a.B);
+  attn_fwd_tc<T><<<grid, kFwdThreads, kFwdSmem, s>>>(mq, mk, mv, t);
+  count_launch();
+}
+
+template <typename T>
+void bwd_t(const AttnArgs& a, cudaStream_t s) {
+  AttnTc t = make_args(std::is_same<T, bf16_t>::value ? DT_BF16 : DT_F16, a);
+  const uint64_t rows = (uint64_t)a.B * a.nh * a.S;
+  const uint64_t tokens = (uint64_t)a.B * a.S;
+  CUtensorMap mq, mk, mv, mdo;
+  if (!map_tile(&mq, a.q, t.bf16, HD, rows, HD) || !map_tile(&mk, a.k, t.bf16, HD, rows, HD) ||
+      !map_tile(&mv, a.v, t.bf16, HD, rows, HD) || !map_tile(&mdo, a.dctx, t.bf16, t.H, tokens, t.H))
+    return;
+  const int ntile = (a.S + TILE - 1) / TILE;
+  if (ntile > 1) {
+    dvec_launch(t.bf16 ? DT_BF16 : DT_F16, a, s);
+    t.dvec = a.dvec;
+  }
+  t.fuse_dq = ntile == 1;
+  static bool attr = false;
+  if (!attr) {
+    cudaFuncSetAttribute(attn_bwd_kv_tc<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, kBwdKvSmem);
+    cudaFuncSetAttribute(attn_bwd_q_tc<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, kBwdQSmem);
+    attr = true;
+  }
+  dim3 grid(ntile, a.nh, a.B);
+  attn_bwd_kv_tc<T><<<grid, kBwdThreads, kBwdKvSmem, s>>>(mq, mk, mv, mdo, t);
+  count_launch();
+  if (!t.fuse_dq) {
+    attn_bwd_q_tc<T><<<grid, kBwdThreads, kBwdQSmem, s>>>(mq, mk, mv, mdo, t);
+    count_launch();
+  }
+}
+
+}  // namespace
+
+bool attn_tc_supports(int dt, const AttnArgs& a) {
+  if (dt == DT_F32 || a.d != HD || a.S < 8) return false;
+  // TMA row coordinates are 32-bit
+  return (uint64_t)a.B * a.nh * a.S < (1ull << 31);
+}
+
+void attn_tc_fwd_run(int dt, const AttnArgs& a, cudaStream_t s) {
+  if (dt == DT_F16) fwd_t<half_t>(a, s);
+  else fwd_t<bf16_t>(a, s);
+}
+
+void attn_tc_bwd_run(int dt, const AttnArgs& a, cudaStream_t s) {
+  if (dt == DT_F16) bwd_t<half_t>(a, s);
+  else bwd_t<bf16_t>(a, s);
+}
+
+int attn_tc_take_error() {
+  int v = 0;
+  int* p = attn_error_word();
+  cudaMemcpy(&v, p, sizeof(int), cudaMemcpyDeviceToHost);
+  if (v) cudaMemset(p, 0, sizeof(int));
+  return v;
+}
+
+}  // namespace tlp

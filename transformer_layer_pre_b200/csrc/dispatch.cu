@@ -23,10 +23,12 @@ size_t gemm_splitk_ws_floats(int dtype, int M, int N, int K) {
   return dtype == DT_F32 ? 0 : gemm_tc_splitk_ws_floats(M, N, K);
 }
 
-int device_take_error() { return gemm_tc_take_error(); }
+int attn_tc_take_error();
 
-bool attn_tc_supports(int dt, const AttnArgs& a) { (void)dt; (void)a; return false; }
-void attn_tc_fwd_run(int, const AttnArgs&, cudaStream_t) {}
-void attn_tc_bwd_run(int, const AttnArgs&, cudaStream_t) {}
+int device_take_error() {
+  const int g = gemm_tc_take_error();
+  const int a = attn_tc_take_error();
+  return g ? g : a;
+}
 
 }  // namespace tlp

@@ -6,6 +6,7 @@
 // shared memory, 256 threads with 2 rows x 8 columns each.
 #include "epilogue.cuh"
 #include "kernels.h"
+#include "profile.h"
 
 namespace tlp {
 
@@ -79,6 +80,7 @@ void launch(const GemmDesc& g, const EpiParams& e, cudaStream_t s) {
     case EPI_STORE: gemm_simt_kernel<T, EPI_STORE><<<grid, 256, 0, s>>>(g, e); break;
     case EPI_F32: gemm_simt_kernel<T, EPI_F32><<<grid, 256, 0, s>>>(g, e); break;
   }
+  count_launch();
 }
 
 }  // namespace

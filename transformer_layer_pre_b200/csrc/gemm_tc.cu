@@ -30,6 +30,7 @@
 
 #include "epilogue.cuh"
 #include "kernels.h"
+#include "profile.h"
 #include "sm100.cuh"
 
 namespace tlp {
@@ -190,7 +191,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int t = blockIdx.x; t < total; t += gridDim.x) {
       int mb, nb, sp;
       decode_tile(g, t, mb, nb, sp);
-      if (!mbar_wait(&tfull[acc], aph, g.err, 4)) break;
+      if (!mbar_wait_warp(&tfull[acc], aph, g.err, 4)) break;
       tc_fence_after();
       const int m = mb * BM + row;
       EpiParams ep = e;
@@ -314,6 +315,7 @@ int launch_tc(const GemmDesc& gd, const EpiParams& e, int splits, cudaStream_t s
     attr = true;
   }
   gemm_tc_kernel<T, BN, KIND><<<grid, kThreads, C::kSmem, s>>>(ma, mb, g, e);
+  count_launch();
   return 0;
 }
 
@@ -349,6 +351,7 @@ int run_t(const GemmDesc& g, const EpiParams& e, cudaStream_t s) {
       const size_t n4 = (size_t)g.M * g.N / 4;
       splitk_reduce_kernel<<<(int)std::min<size_t>((n4 + 255) / 256, 148 * 8), 256, 0, s>>>(
           g.splitk_ws, real, (size_t)g.M * g.N, n4, static_cast<float*>(e.out));
+      count_launch();
       return 0;
     }
     return launch_tc<T, 256, EPI_F32>(g, e, 1, s);

@@ -23,6 +23,7 @@
 
 #include "../../include/tlp.h"
 #include "kernels.h"
+#include "profile.h"
 
 namespace tlp {
 bool rowwise_supports_hidden(int H);
@@ -179,6 +180,7 @@ tl_status ensure_buffers(tl_layer* L) {
 void gemm(tl_layer* L, int M, int N, int K, const void* A, int lda, bool ak, const void* B, int ldb, bool bk,
           const EpiParams& e, cudaStream_t s) {
   GemmDesc g{M, N, K, A, lda, ak, B, ldb, bk, L->splitk, L->splitk_floats};
+  ProfScope p_(PC_GEMM, s);
   if (gemm_run(L->opt.dtype, g, e, s) != 0) L->gemm_err = 1;
 }
 
@@ -196,15 +198,18 @@ EpiParams epi(int kind, void* out, int ldo) {
 
 // Column sums of a (T, cols) stored matrix into a float32 vector.
 void bias_grad(tl_layer* L, const void* X, int cols, float* out, cudaStream_t s) {
+  ProfScope p_(PC_ROWWISE, s);
   colsum_run(L->opt.dtype, X, L->T, cols, L->part, s);
   colsum_finalize_run(L->part, colsum_parts(L->T), cols, out, s);
 }
 
 void attn_fwd(tl_layer* L, const AttnArgs& a, cudaStream_t s) {
+  ProfScope p_(PC_ATTN_FWD, s);
   if (attn_tc_supports(L->opt.dtype, a)) attn_tc_fwd_run(L->opt.dtype, a, s);
   else attn_simt_fwd_run(L->opt.dtype, a, s);
 }
 void attn_bwd(tl_layer* L, const AttnArgs& a, cudaStream_t s) {
+  ProfScope p_(PC_ATTN_BWD, s);
   if (attn_tc_supports(L->opt.dtype, a)) attn_tc_bwd_run(L->opt.dtype, a, s);
   else attn_simt_bwd_run(L->opt.dtype, a, s);
 }
@@ -340,12 +345,18 @@ tl_status layer_forward(tl_layer* L, const void* x, const float* mask, const tl_
   e2.bias = w->b2; e2.drop = make_drop(L, L->ph); e2.site = 2;
 
   if (L->pre_ln) {
-    ln_fwd_run(dt, x, w->ln1_g, w->ln1_b, L->h1, L->mean1, L->rstd1, T, H, L->opt.ln_eps, s);
+    {
+      ProfScope p_(PC_LN_FWD, s);
+      ln_fwd_run(dt, x, w->ln1_g, w->ln1_b, L->h1, L->mean1, L->rstd1, T, H, L->opt.ln_eps, s);
+    }
     gemm(L, T, 3 * H, H, L->h1, H, true, w->wqkv, H, true, eq, s);
     attn_fwd(L, aa, s);
     eo.out = L->x2;
     gemm(L, T, H, H, L->ctx, H, true, w->wo, H, true, eo, s);
-    ln_fwd_run(dt, L->x2, w->ln2_g, w->ln2_b, L->h2, L->mean2, L->rstd2, T, H, L->opt.ln_eps, s);
+    {
+      ProfScope p_(PC_LN_FWD, s);
+      ln_fwd_run(dt, L->x2, w->ln2_g, w->ln2_b, L->h2, L->mean2, L->rstd2, T, H, L->opt.ln_eps, s);
+    }
     gemm(L, T, F, H, L->h2, H, true, w->w1, H, true, e1, s);
     e2.res = L->x2; e2.out = y;
     gemm(L, T, H, F, L->g, F, true, w->w2, F, true, e2, s);
@@ -357,11 +368,17 @@ tl_status layer_forward(tl_layer* L, const void* x, const float* mask, const tl_
     attn_fwd(L, aa, s);
     eo.out = r1;
     gemm(L, T, H, H, L->ctx, H, true, w->wo, H, true, eo, s);
-    ln_fwd_run(dt, r1, w->ln1_g, w->ln1_b, L->x2, L->mean1, L->rstd1, T, H, L->opt.ln_eps, s);
+    {
+      ProfScope p_(PC_LN_FWD, s);
+      ln_fwd_run(dt, r1, w->ln1_g, w->ln1_b, L->x2, L->mean1, L->rstd1, T, H, L->opt.ln_eps, s);
+    }
     gemm(L, T, F, H, L->x2, H, true, w->w1, H, true, e1, s);
     e2.res = L->x2; e2.out = r2;
     gemm(L, T, H, F, L->g, F, true, w->w2, F, true, e2, s);
-    ln_fwd_run(dt, r2, w->ln2_g, w->ln2_b, y, L->mean2, L->rstd2, T, H, L->opt.ln_eps, s);
+    {
+      ProfScope p_(PC_LN_FWD, s);
+      ln_fwd_run(dt, r2, w->ln2_g, w->ln2_b, y, L->mean2, L->rstd2, T, H, L->opt.ln_eps, s);
+    }
     if (L->yout) cudaMemcpyAsync(L->yout, y, (size_t)T * H * dtype_size(dt), cudaMemcpyDeviceToDevice, s);
   }
   st = check_cuda(L, "layer_forward");
@@ -408,6 +425,7 @@ tl_status layer_backward(tl_layer* L, const void* x, const void* dy, const tl_we
     a.res = res; a.dx = dxo; a.drop_out = drop_out; a.drop = dh; a.site = site;
     a.part_dgamma = pa; a.part_dbeta = pb; a.part_dsum = drop_out ? pc : nullptr;
     a.rows = T; a.H = H;
+    ProfScope p_(PC_LN_BWD, s);
     ln_bwd_run(dt, a, s);
     colsum_finalize_run(pa, lnp, H, dgamma, s);
     colsum_finalize_run(pb, lnp, H, dbeta, s);
@@ -417,7 +435,10 @@ tl_status layer_backward(tl_layer* L, const void* x, const void* dy, const tl_we
   // FFN block: dZ2 -> dW2, dU (into big), db1, dW1; returns with dU in L->big
   auto ffn_bwd = [&](const void* ffn_in) {
     EpiParams ew2 = epi(EPI_F32, g->w2, F);
-    if (L->opt.gelu_checkpoint) gelu_run(dt, L->u, L->big, (size_t)T * F, s);
+    if (L->opt.gelu_checkpoint) {
+      ProfScope p_(PC_ROWWISE, s);
+      gelu_run(dt, L->u, L->big, (size_t)T * F, s);
+    }
     gemm(L, H, F, T, L->dz2, H, false, L->g, F, false, ew2, s);          // dW2 = dZ2^T G
     EpiParams edu = epi(EPI_DGELU, L->big, F);
     edu.aux = L->u;
@@ -440,8 +461,11 @@ tl_status layer_backward(tl_layer* L, const void* x, const void* dy, const tl_we
   };
 
   if (L->pre_ln) {
-    dropout_rows_run(dt, dy, L->dz2, dh, 2, T, H, pc, s);
-    colsum_finalize_run(pc, rowdrop_parts(T), H, g->b2, s);
+    {
+      ProfScope p_(PC_ROWWISE, s);
+      dropout_rows_run(dt, dy, L->dz2, dh, 2, T, H, pc, s);
+      colsum_finalize_run(pc, rowdrop_parts(T), H, g->b2, s);
+    }
     ffn_bwd(L->h2);
     EpiParams edh = epi(EPI_STORE, L->dh, H);
     gemm(L, T, H, F, L->big, F, true, w->w1, H, false, edh, s);           // dH2 = dU W1

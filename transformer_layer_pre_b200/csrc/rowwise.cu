@@ -13,6 +13,7 @@
 
 #include "common.cuh"
 #include "kernels.h"
+#include "profile.h"
 
 namespace tlp {
 
@@ -301,6 +302,7 @@ void ln_fwd_t(const void* x, const void* g, const void* b, void* y, float* mean,
   TLP_NCH_SWITCH(H, ln_fwd_kernel<T, NCH><<<blocks, kWarps * 32, 0, s>>>(
                         static_cast<const T*>(x), static_cast<const T*>(g), static_cast<const T*>(b),
                         static_cast<T*>(y), mean, rstd, rows, H, eps));
+  count_launch();
 }
 
 template <typename T, bool INV>
@@ -311,6 +313,7 @@ void ln_bwd_t(const LnBwdArgs& a, cudaStream_t s) {
     cudaFuncSetAttribute(ln_bwd_kernel<T, NCH, INV>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     ln_bwd_kernel<T, NCH, INV><<<blocks, kWarps * 32, smem, s>>>(a);
   });
+  count_launch();
 }
 
 template <typename T>
@@ -323,6 +326,7 @@ void dropout_rows_t(const void* in, void* out, const DropoutParams& dp, int site
     dropout_rows_kernel<T, NCH><<<blocks, kWarps * 32, smem, s>>>(static_cast<const T*>(in), static_cast<T*>(out),
                                                                   dp, site, rows, H, part);
   });
+  count_launch();
 }
 
 }  // namespace
@@ -364,10 +368,12 @@ void colsum_run(int dt, const void* X, int rows, int cols, float* part, cudaStre
   if (dt == DT_F32) colsum_kernel<float><<<grid, 256, 0, s>>>(static_cast<const float*>(X), rows, cols, part);
   else if (dt == DT_F16) colsum_kernel<half_t><<<grid, 256, 0, s>>>(static_cast<const half_t*>(X), rows, cols, part);
   else colsum_kernel<bf16_t><<<grid, 256, 0, s>>>(static_cast<const bf16_t*>(X), rows, cols, part);
+  count_launch();
 }
 
 void colsum_finalize_run(const float* part, int nparts, int cols, float* out, cudaStream_t s) {
   colsum_finalize_kernel<<<(cols + 255) / 256, 256, 0, s>>>(part, nparts, cols, out);
+  count_launch();
 }
 
 void gelu_run(int dt, const void* U, void* G, size_t n, cudaStream_t s) {
@@ -376,12 +382,14 @@ void gelu_run(int dt, const void* U, void* G, size_t n, cudaStream_t s) {
   if (dt == DT_F32) gelu_kernel<float><<<blocks, 256, 0, s>>>(static_cast<const float*>(U), static_cast<float*>(G), n8);
   else if (dt == DT_F16) gelu_kernel<half_t><<<blocks, 256, 0, s>>>(static_cast<const half_t*>(U), static_cast<half_t*>(G), n8);
   else gelu_kernel<bf16_t><<<blocks, 256, 0, s>>>(static_cast<const bf16_t*>(U), static_cast<bf16_t*>(G), n8);
+  count_launch();
 }
 
 void dropout_mask_run(const DropoutParams& dp, int site, uint64_t e0, uint64_t n, uint8_t* keep, cudaStream_t s) {
   const uint64_t n8 = n / 8;
   const int blocks = (int)std::min<uint64_t>((n8 + 255) / 256, 148 * 16);
   dropout_mask_kernel<<<blocks > 0 ? blocks : 1, 256, 0, s>>>(dp, site, e0, n8, keep);
+  count_launch();
 }
 
 }  // namespace tlp
