@@ -166,6 +166,24 @@ int tl_profile_read(double* ms, long long* launches, int n);
 /* Total number of kernels the library has launched since it was loaded. */
 long long tl_launch_count(void);
 
+/* Column sums that allocate nothing: db[c] = sum over r < rows of dz[r, c]
+ * (dz row-major (rows, cols) in storage dtype `dtype`, db float32 (cols)),
+ * the bias gradient of a Linear layer whose output gradient is dz.  The
+ * source pages have no counterpart: this entry point exists for callers that
+ * cannot allocate device memory (memory owned by a framework's caching
+ * allocator or a fixed budget, or code running inside a global-mode stream
+ * capture, where cudaMalloc is not allowed).
+ * Scratch: a 2 MiB array in the library's device memory, held by every GPU
+ * that loads the library until the process exits.  Limits: cols <= 8192 and a
+ * multiple of 8, rows >= 1, both pointers 16-byte aligned, else TL_EINVAL.
+ * The first call on a device looks up the array's device address
+ * (cudaGetSymbolAddress); make that first call before any stream capture.
+ * Every call shares the one array and overwrites it: calls that overlap on
+ * the GPU (other streams, other threads) race and must be serialised by the
+ * caller.  Enqueued on `stream` (a cudaStream_t); returns before the GPU
+ * finishes.  TL_ECUDA if a CUDA call fails. */
+tl_status tl_bias_grad_noalloc(int dtype, const void* dz, int rows, int cols, float* db, void* stream);
+
 const char* tl_status_string(tl_status s);
 
 #ifdef __cplusplus

@@ -29,7 +29,7 @@ EXPORTED_SYMBOLS = (
     "layer_create", "layer_default_options", "layer_set_options", "layer_get_options",
     "layer_forward", "layer_backward", "layer_workspace_bytes", "layer_last_error",
     "layer_destroy", "tl_dropout_keep_mask", "tl_device_check", "tl_profile_enable",
-    "tl_profile_read", "tl_launch_count", "tl_status_string",
+    "tl_profile_read", "tl_launch_count", "tl_bias_grad_noalloc", "tl_status_string",
 )
 PROFILE_CLASSES = ("gemm", "attn_fwd", "attn_bwd", "ln_fwd", "ln_bwd", "rowwise")
 
@@ -100,6 +100,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.tl_profile_read.restype = i
     lib.tl_launch_count.argtypes = []
     lib.tl_launch_count.restype = ctypes.c_longlong
+    lib.tl_bias_grad_noalloc.argtypes = [i, vp, i, i, vp, vp]
+    lib.tl_bias_grad_noalloc.restype = i
     lib.tl_status_string.argtypes = [i]
     lib.tl_status_string.restype = ctypes.c_char_p
     _lib = lib
