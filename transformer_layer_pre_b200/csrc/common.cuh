@@ -65,6 +65,13 @@ template <> struct Vec8Io<half_t> : Vec8Io16<__half2, half_t> {};
 template <> struct Vec8Io<bf16_t> : Vec8Io16<__nv_bfloat162, bf16_t> {};
 
 template <typename T> __device__ __forceinline__ void load8(const T* p, float (&v)[8]) { Vec8Io<T>::load(p, v); }
+
+// 8 16-bit values held in a uint4 (as loaded by a 16-byte vector load) to float.
+template <typename T> __device__ __forceinline__ void unpack8(const uint4& r, float (&v)[8]) {
+  const T* h = reinterpret_cast<const T*>(&r);
+#pragma unroll
+  for (int i = 0; i < 8; ++i) v[i] = to_f(h[i]);
+}
 template <typename T> __device__ __forceinline__ void store8(T* p, const float (&v)[8]) { Vec8Io<T>::store(p, v); }
 
 // ------------------------------------------------------------------ Philox4x32-10

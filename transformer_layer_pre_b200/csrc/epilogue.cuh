@@ -15,6 +15,9 @@
 //  EPI_DGELU          out = acc * GELU'(U).
 //  EPI_STORE          out = acc (+ res).
 //  EPI_F32            float32 out = acc.
+//
+// `aux` carries the 8 residual (EPI_BIAS_DROP_RES, EPI_STORE with res) or U
+// (EPI_DGELU) values of the chunk, loaded by the caller ahead of time.
 #pragma once
 
 #include "common.cuh"
@@ -22,17 +25,31 @@
 
 namespace tlp {
 
+// Whether a kind reads a per-element auxiliary input (and which pointer).
+template <int KIND> struct EpiAux {
+  static constexpr bool kNeeds = KIND == EPI_BIAS_DROP_RES || KIND == EPI_DGELU || KIND == EPI_STORE;
+};
+__device__ __forceinline__ const void* epi_aux_ptr(const EpiParams& e, int kind) {
+  return kind == EPI_DGELU ? e.aux : e.res;
+}
+
+// Row-dependent part of the EPI_QKV destination, computed once per row.
+__device__ __forceinline__ size_t qkv_row_base(const EpiParams& e, int m) {
+  const int bb = m / e.seq;
+  const int s = m - bb * e.seq;
+  return ((size_t)bb * e.heads * e.seq + s) * e.head_dim;
+}
+
 template <typename T, int KIND>
-__device__ __forceinline__ void epi_apply8(const EpiParams& e, int m, int n, float (&v)[8]) {
+__device__ __forceinline__ void epi_apply8(const EpiParams& e, int m, int n, float (&v)[8], const float (&aux)[8],
+                                           size_t row_base) {
   if constexpr (KIND == EPI_F32) {
     float* o = static_cast<float*>(e.out) + (size_t)m * e.ldo + n;
     store8<float>(o, v);
   } else if constexpr (KIND == EPI_STORE) {
     if (e.res) {
-      float r[8];
-      load8<T>(static_cast<const T*>(e.res) + (size_t)m * e.ldo + n, r);
 #pragma unroll
-      for (int i = 0; i < 8; ++i) v[i] += r[i];
+      for (int i = 0; i < 8; ++i) v[i] += aux[i];
     }
     store8<T>(static_cast<T*>(e.out) + (size_t)m * e.ldo + n, v);
   } else if constexpr (KIND == EPI_QKV) {
@@ -40,24 +57,22 @@ __device__ __forceinline__ void epi_apply8(const EpiParams& e, int m, int n, flo
     load8<T>(static_cast<const T*>(e.bias) + n, b);
 #pragma unroll
     for (int i = 0; i < 8; ++i) v[i] += b[i];
-    const int which = n / e.hidden;
+    // which of Q, K, V; head and lane by shifts (head_dim is a power of two)
+    const int which = (n >= e.hidden) + (n >= 2 * e.hidden);
     const int c = n - which * e.hidden;
-    const int h = c / e.head_dim;
-    const int lane = c - h * e.head_dim;
-    const int bb = m / e.seq;
-    const int s = m - bb * e.seq;
-    const size_t dst = (size_t)which * e.tokens * e.hidden +
-                       ((size_t)(bb * e.heads + h) * e.seq + s) * e.head_dim + lane;
+    const int sh = __ffs(e.head_dim) - 1;
+    const int h = c >> sh;
+    const int lane = c & (e.head_dim - 1);
+    const size_t dst = (size_t)which * e.tokens * e.hidden + row_base + ((size_t)h * e.seq << sh) + lane;
     store8<T>(static_cast<T*>(e.out) + dst, v);
   } else if constexpr (KIND == EPI_BIAS_DROP_RES) {
-    float b[8], r[8];
+    float b[8];
     load8<T>(static_cast<const T*>(e.bias) + n, b);
-    load8<T>(static_cast<const T*>(e.res) + (size_t)m * e.ldo + n, r);
     uint32_t bits = 0xFFu;
     if (e.drop.thr) bits = dropout_bits8(e.drop, e.site, ((uint64_t)m * e.ldo + n) >> 3);
     const float sc = e.drop.thr ? e.drop.scale : 1.0f;
 #pragma unroll
-    for (int i = 0; i < 8; ++i) v[i] = r[i] + (((bits >> i) & 1u) ? (v[i] + b[i]) * sc : 0.0f);
+    for (int i = 0; i < 8; ++i) v[i] = aux[i] + (((bits >> i) & 1u) ? (v[i] + b[i]) * sc : 0.0f);
     store8<T>(static_cast<T*>(e.out) + (size_t)m * e.ldo + n, v);
   } else if constexpr (KIND == EPI_BIAS_GELU) {
     float b[8];
@@ -71,12 +86,23 @@ __device__ __forceinline__ void epi_apply8(const EpiParams& e, int m, int n, flo
       store8<T>(static_cast<T*>(e.out2) + (size_t)m * e.ldo + n, v);
     }
   } else if constexpr (KIND == EPI_DGELU) {
-    float u[8];
-    load8<T>(static_cast<const T*>(e.aux) + (size_t)m * e.ldo + n, u);
 #pragma unroll
-    for (int i = 0; i < 8; ++i) v[i] *= gelu_grad_f(u[i]);
+    for (int i = 0; i < 8; ++i) v[i] *= gelu_grad_f(aux[i]);
     store8<T>(static_cast<T*>(e.out) + (size_t)m * e.ldo + n, v);
   }
+}
+
+// Convenience form that loads the auxiliary values itself (SIMT GEMM).
+template <typename T, int KIND>
+__device__ __forceinline__ void epi_apply8(const EpiParams& e, int m, int n, float (&v)[8]) {
+  float aux[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+  if constexpr (EpiAux<KIND>::kNeeds) {
+    const void* p = epi_aux_ptr(e, KIND);
+    if (p) load8<T>(static_cast<const T*>(p) + (size_t)m * e.ldo + n, aux);
+  }
+  size_t rb = 0;
+  if constexpr (KIND == EPI_QKV) rb = qkv_row_base(e, m);
+  epi_apply8<T, KIND>(e, m, n, v, aux, rb);
 }
 
 }  // namespace tlp

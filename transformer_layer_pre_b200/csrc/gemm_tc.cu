@@ -16,8 +16,10 @@
 //   warp 1   allocates TMEM (two BN-column fp32 accumulators) and issues
 //            tcgen05.mma (M=128, N=BN, K=16) from one thread, committing each
 //            stage back to the producer and each finished tile to the epilogue;
-//   warps 2-5  epilogue: tcgen05.ld 16 columns at a time from the lanes the
-//            warp may access, fused epilogue (epilogue.cuh), global stores.
+//   warps 2-9  epilogue: two warps per TMEM lane quarter split the tile's
+//            columns; tcgen05.ld 32 columns at a time, fused epilogue
+//            (epilogue.cuh), global stores.  Residual / U inputs of the
+//            epilogue are loaded before the accumulator is ready.
 // Accumulators are double-buffered so a tile's epilogue overlaps the next
 // tile's main loop.  Weight gradients (K = tokens) may split K across CTAs
 // into float32 partial tiles that a second kernel sums in a fixed order.
@@ -41,7 +43,7 @@ namespace {
 
 constexpr int BM = 128;
 constexpr int BK = 64;
-constexpr int kThreads = 192;
+constexpr int kThreads = 320;   // TMA warp, MMA warp, 8 epilogue warps
 
 template <int BN> struct TileCfg {
   static constexpr int kStages = BN == 256 ? 4 : 6;
@@ -90,7 +92,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&tfull[a], 1);
-      mbar_init(&tempty[a], 128);
+      mbar_init(&tempty[a], 256);
     }
     fence_barrier_init();
   }
@@ -184,29 +186,55 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
   } else {
-    const int quarter = warp & 3;  // this warp may access TMEM lanes 32*quarter .. +31
+    // Epilogue warps 2..9: warp w may access TMEM lanes 32*(w%4) .. +31 (one
+    // output row per thread) and takes half of the tile's columns.
+    constexpr int CW = BN / 2;
+    const int quarter = warp & 3;
+    const int half = (warp - 2) >> 2;
     const int row = quarter * 32 + lane;
     int acc = 0;
     uint32_t aph = 0;
     for (int t = blockIdx.x; t < total; t += gridDim.x) {
       int mb, nb, sp;
       decode_tile(g, t, mb, nb, sp);
+      const int m = mb * BM + row;
+      const int nbase = nb * BN + half * CW;
+      const bool mrow = m < g.M;
+      // the residual / U values of this thread's columns are fetched before
+      // the accumulator is ready, so their latency hides under the main loop
+      uint4 pre[EpiAux<KIND>::kNeeds ? CW / 8 : 1];
+      if constexpr (EpiAux<KIND>::kNeeds) {
+        const T* ap = static_cast<const T*>(epi_aux_ptr(e, KIND));
+#pragma unroll
+        for (int j = 0; j < CW / 8; ++j) {
+          const int n = nbase + j * 8;
+          pre[j] = (ap && mrow && n < g.N) ? *reinterpret_cast<const uint4*>(ap + (size_t)m * e.ldo + n)
+                                            : make_uint4(0u, 0u, 0u, 0u);
+        }
+      }
+      size_t rb = 0;
+      if constexpr (KIND == EPI_QKV) rb = mrow ? qkv_row_base(e, m) : 0;
       if (!mbar_wait_warp(&tfull[acc], aph, g.err, 4)) break;
       tc_fence_after();
-      const int m = mb * BM + row;
       EpiParams ep = e;
       if constexpr (KIND == EPI_F32) ep.out = static_cast<float*>(e.out) + (size_t)sp * g.split_stride;
-      const uint32_t tbase = tmem + ((uint32_t)(quarter * 32) << 16) + acc * BN;
-#pragma unroll 1
-      for (int c0 = 0; c0 < BN; c0 += 16) {
-        float v[16];
-        tmem_ld16(tbase + c0, v);
-        const int n = nb * BN + c0;
-        if (m < g.M) {
-          float* v0 = v;
-          float* v1 = v + 8;
-          if (n < g.N) epi_apply8<T, KIND>(ep, m, n, *reinterpret_cast<float(*)[8]>(v0));
-          if (n + 8 < g.N) epi_apply8<T, KIND>(ep, m, n + 8, *reinterpret_cast<float(*)[8]>(v1));
+      const uint32_t tbase = tmem + ((uint32_t)(quarter * 32) << 16) + acc * BN + half * CW;
+#pragma unroll
+      for (int c0 = 0; c0 < CW; c0 += 32) {
+        float v[32];
+        tmem_ld32(tbase + c0, v);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const int n = nbase + c0 + q * 8;
+          if (mrow && n < g.N) {
+            float aux[8];
+            if constexpr (EpiAux<KIND>::kNeeds) unpack8<T>(pre[(c0 >> 3) + q], aux);
+            else {
+#pragma unroll
+              for (int i = 0; i < 8; ++i) aux[i] = 0.0f;
+            }
+            epi_apply8<T, KIND>(ep, m, n, *reinterpret_cast<float(*)[8]>(v + q * 8), aux, rb);
+          }
         }
       }
       tc_fence_before();

@@ -3,12 +3,11 @@
 //
 // LayerNorm is per token over the hidden axis with the biased variance and
 // eps inside the square root; statistics are float32 ("AI-infra engineers and
-// the Transformer", section 3.2: LayerNorm kept in fp32).  One warp owns a
-// row; each lane holds chunks of 8 consecutive elements (one 16-byte load for
-// 16-bit storage), so a warp reads 512 contiguous bytes per chunk step.
-// Column sums (bias and LayerNorm-parameter gradients) are reduced in a fixed
-// order: per-warp registers, then per-block shared memory, then one partial
-// row per block, then tlp::colsum_finalize_run — the result is deterministic.
+// the Transformer", section 3.2: LayerNorm kept in fp32).  A block owns a
+// contiguous range of rows and each thread 8 consecutive columns of them, so
+// column sums (bias and LayerNorm-parameter gradients) accumulate in the
+// owning thread's registers in row order and leave as one partial row per
+// block, summed by tlp::colsum_finalize_run in block order: deterministic.
 #include <algorithm>
 
 #include "common.cuh"
@@ -19,207 +18,225 @@ namespace tlp {
 
 namespace {
 
-constexpr int kWarps = 8;  // warps per block of the row kernels
-constexpr int kMaxParts = 296;
+// Row-block kernels: a block of ceil(H/8 / 32) warps owns a contiguous range
+// of rows; thread t owns columns 8t .. 8t+7 of every row of that range (one
+// 16-byte vector for 16-bit storage) and walks the rows kRows at a time.
+// Row statistics are block reductions (one per kRows rows); column sums stay
+// in the owning thread's registers and leave as one partial row per block.
+constexpr int kRows = 4;
+constexpr int kMaxBlocks = 592;   // 4 blocks per SM
 
-// ------------------------------------------------------------------ LayerNorm forward
-template <typename T, int NCH>
-__global__ void __launch_bounds__(kWarps * 32) ln_fwd_kernel(const T* __restrict__ x, const T* __restrict__ gamma,
-                                                            const T* __restrict__ beta, T* __restrict__ y,
-                                                            float* __restrict__ mean_out, float* __restrict__ rstd_out,
-                                                            int rows, int H, float eps) {
-  const int lane = threadIdx.x & 31;
-  const int row = blockIdx.x * kWarps + (threadIdx.x >> 5);
-  if (row >= rows) return;
-  const T* xr = x + (size_t)row * H;
-  float v[NCH][8];
-  float s = 0.0f;
+__host__ __device__ inline int row_threads(int H) { return ((H / 8 + 31) / 32) * 32; }
+
+// Sums v[r] over the whole block; red holds (warps, kRows) floats.
+__device__ __forceinline__ void block_sum(float (&v)[kRows], float* red) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
 #pragma unroll
-  for (int c = 0; c < NCH; ++c) {
-    const int col = (lane + 32 * c) * 8;
-    if (col < H) {
-      load8<T>(xr + col, v[c]);
-#pragma unroll
-      for (int i = 0; i < 8; ++i) s += v[c][i];
-    }
-  }
-  const float mean = warp_sum(s) / (float)H;
-  float ss = 0.0f;
-#pragma unroll
-  for (int c = 0; c < NCH; ++c) {
-    const int col = (lane + 32 * c) * 8;
-    if (col < H) {
-#pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        const float dlt = v[c][i] - mean;
-        ss += dlt * dlt;
-      }
-    }
-  }
-  const float var = warp_sum(ss) / (float)H;
-  const float rstd = 1.0f / sqrtf(var + eps);
-  T* yr = y + (size_t)row * H;
-#pragma unroll
-  for (int c = 0; c < NCH; ++c) {
-    const int col = (lane + 32 * c) * 8;
-    if (col < H) {
-      float g[8], b[8], o[8];
-      load8<T>(gamma + col, g);
-      load8<T>(beta + col, b);
-#pragma unroll
-      for (int i = 0; i < 8; ++i) o[i] = g[i] * ((v[c][i] - mean) * rstd) + b[i];
-      store8<T>(yr + col, o);
-    }
-  }
+  for (int r = 0; r < kRows; ++r) v[r] = warp_sum(v[r]);
   if (lane == 0) {
-    mean_out[row] = mean;
-    rstd_out[row] = rstd;
+#pragma unroll
+    for (int r = 0; r < kRows; ++r) red[warp * kRows + r] = v[r];
   }
+  __syncthreads();
+#pragma unroll
+  for (int r = 0; r < kRows; ++r) {
+    float s = 0.0f;
+    for (int w = 0; w < nw; ++w) s += red[w * kRows + r];
+    v[r] = s;
+  }
+  __syncthreads();
 }
 
-// Reduce per-lane column accumulators acc[NCH][8] of every warp of the block
-// into one partial row part[blockIdx.x * H + col]; red is (kWarps, H) floats.
-template <int NCH>
-__device__ __forceinline__ void block_colsum(float (&acc)[NCH][8], float* red, float* part, int H) {
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  __syncthreads();
-#pragma unroll
-  for (int c = 0; c < NCH; ++c) {
-    const int col = (lane + 32 * c) * 8;
-    if (col < H) {
-#pragma unroll
-      for (int i = 0; i < 8; ++i) red[warp * H + col + i] = acc[c][i];
-    }
+__device__ __forceinline__ void row_range(int rows, int& r0, int& r1) {
+  const int per = (rows + gridDim.x - 1) / gridDim.x;
+  r0 = blockIdx.x * per;
+  r1 = min(rows, r0 + per);
+}
+
+__device__ __forceinline__ void store_part(float* part, int H, int col, const float (&acc)[8]) {
+  float* p = part + (size_t)blockIdx.x * H + col;
+  reinterpret_cast<float4*>(p)[0] = make_float4(acc[0], acc[1], acc[2], acc[3]);
+  reinterpret_cast<float4*>(p)[1] = make_float4(acc[4], acc[5], acc[6], acc[7]);
+}
+
+// ------------------------------------------------------------------ LayerNorm forward
+template <typename T>
+__global__ void __launch_bounds__(512) ln_fwd_kernel(const T* __restrict__ x, const T* __restrict__ gamma,
+                                                    const T* __restrict__ beta, T* __restrict__ y,
+                                                    float* __restrict__ mean_out, float* __restrict__ rstd_out,
+                                                    int rows, int H, float eps) {
+  __shared__ float red[16 * kRows];
+  const int col = threadIdx.x * 8;
+  const bool act = col < H;
+  float g[8], b[8];
+  if (act) {
+    load8<T>(gamma + col, g);
+    load8<T>(beta + col, b);
   }
-  __syncthreads();
-  for (int col = threadIdx.x; col < H; col += blockDim.x) {
-    float s = 0.0f;
-    for (int w = 0; w < kWarps; ++w) s += red[w * H + col];
-    part[(size_t)blockIdx.x * H + col] = s;
+  int r0, r1;
+  row_range(rows, r0, r1);
+  const float inv_h = 1.0f / (float)H;
+  for (int base = r0; base < r1; base += kRows) {
+    float v[kRows][8], s[kRows];
+#pragma unroll
+    for (int r = 0; r < kRows; ++r) {
+      s[r] = 0.0f;
+      if (act && base + r < r1) {
+        load8<T>(x + (size_t)(base + r) * H + col, v[r]);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) s[r] += v[r][i];
+      } else {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) v[r][i] = 0.0f;
+      }
+    }
+    block_sum(s, red);
+    float mean[kRows], ss[kRows];
+#pragma unroll
+    for (int r = 0; r < kRows; ++r) {
+      mean[r] = s[r] * inv_h;
+      ss[r] = 0.0f;
+      if (act) {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const float d = v[r][i] - mean[r];
+          ss[r] += d * d;
+        }
+      }
+    }
+    block_sum(ss, red);
+#pragma unroll
+    for (int r = 0; r < kRows; ++r) {
+      if (base + r >= r1) continue;
+      const float rstd = 1.0f / sqrtf(ss[r] * inv_h + eps);
+      if (act) {
+        float o[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) o[i] = g[i] * ((v[r][i] - mean[r]) * rstd) + b[i];
+        store8<T>(y + (size_t)(base + r) * H + col, o);
+      }
+      if (threadIdx.x == 0) {
+        mean_out[base + r] = mean[r];
+        rstd_out[base + r] = rstd;
+      }
+    }
   }
 }
 
 // ------------------------------------------------------------------ LayerNorm backward
-template <typename T, int NCH, bool INV>
-__global__ void __launch_bounds__(kWarps * 32) ln_bwd_kernel(LnBwdArgs a) {
-  extern __shared__ float red[];
-  const int lane = threadIdx.x & 31;
+template <typename T, bool INV>
+__global__ void __launch_bounds__(512) ln_bwd_kernel(LnBwdArgs a) {
+  __shared__ float red[16 * kRows];
   const int H = a.H;
-  const int nwarps = gridDim.x * kWarps;
-  float dg[NCH][8], db[NCH][8], dsum[NCH][8];
+  const int col = threadIdx.x * 8;
+  const bool act = col < H;
+  float gm[8], bt[8];
+  float dg[8], db[8], ds[8];
 #pragma unroll
-  for (int c = 0; c < NCH; ++c)
-#pragma unroll
-    for (int i = 0; i < 8; ++i) dg[c][i] = db[c][i] = dsum[c][i] = 0.0f;
-
+  for (int i = 0; i < 8; ++i) dg[i] = db[i] = ds[i] = 0.0f;
+  if (act) {
+    load8<T>(static_cast<const T*>(a.gamma) + col, gm);
+    if constexpr (INV) load8<T>(static_cast<const T*>(a.beta) + col, bt);
+  }
   const T* dyp = static_cast<const T*>(a.dy);
-  const T* gam = static_cast<const T*>(a.gamma);
-  for (int row = blockIdx.x * kWarps + (threadIdx.x >> 5); row < a.rows; row += nwarps) {
-    const size_t off = (size_t)row * H;
-    const float rstd = a.rstd[row];
-    float dy[NCH][8], xh[NCH][8];
-    float s1 = 0.0f, s2 = 0.0f;
+  const float inv_h = 1.0f / (float)H;
+  const float sc = a.drop.thr ? a.drop.scale : 1.0f;
+  int r0, r1;
+  row_range(a.rows, r0, r1);
+  for (int base = r0; base < r1; base += kRows) {
+    float g[kRows][8], xh[kRows][8], s1[kRows], s2[kRows], rs[kRows];
 #pragma unroll
-    for (int c = 0; c < NCH; ++c) {
-      const int col = (lane + 32 * c) * 8;
-      if (col < H) {
-        float g[8];
-        load8<T>(dyp + off + col, dy[c]);
-        load8<T>(gam + col, g);
+    for (int r = 0; r < kRows; ++r) {
+      s1[r] = s2[r] = 0.0f;
+      const int row = base + r;
+      rs[r] = row < r1 ? a.rstd[row] : 0.0f;
+      if (act && row < r1) {
+        const size_t off = (size_t)row * H + col;
+        float dy[8], xv[8];
+        load8<T>(dyp + off, dy);
         if constexpr (INV) {
-          float yv[8], bt[8];
-          load8<T>(static_cast<const T*>(a.y) + off + col, yv);
-          load8<T>(static_cast<const T*>(a.beta) + col, bt);
+          load8<T>(static_cast<const T*>(a.y) + off, xv);
 #pragma unroll
-          for (int i = 0; i < 8; ++i) xh[c][i] = (yv[i] - bt[i]) / g[i];
+          for (int i = 0; i < 8; ++i) xh[r][i] = (xv[i] - bt[i]) / gm[i];
         } else {
-          float xv[8];
-          load8<T>(static_cast<const T*>(a.x) + off + col, xv);
+          load8<T>(static_cast<const T*>(a.x) + off, xv);
           const float mean = a.mean[row];
 #pragma unroll
-          for (int i = 0; i < 8; ++i) xh[c][i] = (xv[i] - mean) * rstd;
+          for (int i = 0; i < 8; ++i) xh[r][i] = (xv[i] - mean) * rs[r];
         }
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
-          const float gi = dy[c][i] * g[i];
-          s1 += gi;
-          s2 += gi * xh[c][i];
-          dg[c][i] += dy[c][i] * xh[c][i];
-          db[c][i] += dy[c][i];
-          dy[c][i] = gi;  // keep g = dy * gamma
+          g[r][i] = dy[i] * gm[i];
+          s1[r] += g[r][i];
+          s2[r] += g[r][i] * xh[r][i];
+          dg[i] += dy[i] * xh[r][i];
+          db[i] += dy[i];
         }
+      } else {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) g[r][i] = xh[r][i] = 0.0f;
       }
     }
-    const float m1 = warp_sum(s1) / (float)H;
-    const float m2 = warp_sum(s2) / (float)H;
+    block_sum(s1, red);
+    block_sum(s2, red);
 #pragma unroll
-    for (int c = 0; c < NCH; ++c) {
-      const int col = (lane + 32 * c) * 8;
-      if (col < H) {
-        float o[8];
+    for (int r = 0; r < kRows; ++r) {
+      const int row = base + r;
+      if (!act || row >= r1) continue;
+      const size_t off = (size_t)row * H + col;
+      const float m1 = s1[r] * inv_h, m2 = s2[r] * inv_h;
+      float o[8];
 #pragma unroll
-        for (int i = 0; i < 8; ++i) o[i] = rstd * (dy[c][i] - m1 - xh[c][i] * m2);
-        if (a.res) {
-          float r[8];
-          load8<T>(static_cast<const T*>(a.res) + off + col, r);
+      for (int i = 0; i < 8; ++i) o[i] = rs[r] * (g[r][i] - m1 - xh[r][i] * m2);
+      if (a.res) {
+        float rv[8];
+        load8<T>(static_cast<const T*>(a.res) + off, rv);
 #pragma unroll
-          for (int i = 0; i < 8; ++i) o[i] += r[i];
+        for (int i = 0; i < 8; ++i) o[i] += rv[i];
+      }
+      store8<T>(static_cast<T*>(a.dx) + off, o);
+      if (a.drop_out) {
+        const uint32_t bits = a.drop.thr ? dropout_bits8(a.drop, a.site, off >> 3) : 0xFFu;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          o[i] = round_f<T>(((bits >> i) & 1u) ? round_f<T>(o[i]) * sc : 0.0f);
+          ds[i] += o[i];
         }
-        store8<T>(static_cast<T*>(a.dx) + off + col, o);
-        if (a.drop_out) {
-          uint32_t bits = 0xFFu;
-          if (a.drop.thr) bits = dropout_bits8(a.drop, a.site, (off + col) >> 3);
-          const float sc = a.drop.thr ? a.drop.scale : 1.0f;
-#pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            o[i] = ((bits >> i) & 1u) ? round_f<T>(o[i]) * sc : 0.0f;
-            o[i] = round_f<T>(o[i]);
-            dsum[c][i] += o[i];
-          }
-          store8<T>(static_cast<T*>(a.drop_out) + off + col, o);
-        }
+        store8<T>(static_cast<T*>(a.drop_out) + off, o);
       }
     }
   }
-  block_colsum<NCH>(dg, red, a.part_dgamma, H);
-  block_colsum<NCH>(db, red, a.part_dbeta, H);
-  if (a.part_dsum) block_colsum<NCH>(dsum, red, a.part_dsum, H);
+  if (act) {
+    store_part(a.part_dgamma, H, col, dg);
+    store_part(a.part_dbeta, H, col, db);
+    if (a.part_dsum) store_part(a.part_dsum, H, col, ds);
+  }
 }
 
 // ------------------------------------------------------------------ dropout of rows
-template <typename T, int NCH>
-__global__ void __launch_bounds__(kWarps * 32) dropout_rows_kernel(const T* __restrict__ in, T* __restrict__ out,
-                                                                  DropoutParams dp, int site, int rows, int H,
-                                                                  float* __restrict__ part) {
-  extern __shared__ float red[];
-  const int lane = threadIdx.x & 31;
-  const int nwarps = gridDim.x * kWarps;
-  float acc[NCH][8];
+template <typename T>
+__global__ void __launch_bounds__(512) dropout_rows_kernel(const T* __restrict__ in, T* __restrict__ out,
+                                                            DropoutParams dp, int site, int rows, int H,
+                                                            float* __restrict__ part) {
+  const int col = threadIdx.x * 8;
+  if (col >= H) return;
+  float acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+  const float sc = dp.thr ? dp.scale : 1.0f;
+  int r0, r1;
+  row_range(rows, r0, r1);
+  for (int row = r0; row < r1; ++row) {
+    const size_t off = (size_t)row * H + col;
+    float v[8];
+    load8<T>(in + off, v);
+    const uint32_t bits = dp.thr ? dropout_bits8(dp, site, off >> 3) : 0xFFu;
 #pragma unroll
-  for (int c = 0; c < NCH; ++c)
-#pragma unroll
-    for (int i = 0; i < 8; ++i) acc[c][i] = 0.0f;
-  for (int row = blockIdx.x * kWarps + (threadIdx.x >> 5); row < rows; row += nwarps) {
-    const size_t off = (size_t)row * H;
-#pragma unroll
-    for (int c = 0; c < NCH; ++c) {
-      const int col = (lane + 32 * c) * 8;
-      if (col < H) {
-        float v[8];
-        load8<T>(in + off + col, v);
-        uint32_t bits = 0xFFu;
-        if (dp.thr) bits = dropout_bits8(dp, site, (off + col) >> 3);
-        const float sc = dp.thr ? dp.scale : 1.0f;
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          v[i] = round_f<T>(((bits >> i) & 1u) ? v[i] * sc : 0.0f);
-          acc[c][i] += v[i];
-        }
-        store8<T>(out + off + col, v);
-      }
+    for (int i = 0; i < 8; ++i) {
+      v[i] = round_f<T>(((bits >> i) & 1u) ? v[i] * sc : 0.0f);
+      acc[i] += v[i];
     }
+    store8<T>(out + off, v);
   }
-  block_colsum<NCH>(acc, red, part, H);
+  store_part(part, H, col, acc);
 }
 
 // ------------------------------------------------------------------ column sums
@@ -251,12 +268,26 @@ __global__ void __launch_bounds__(256) colsum_kernel(const T* __restrict__ X, in
   }
 }
 
-__global__ void colsum_finalize_kernel(const float* __restrict__ part, int nparts, int cols, float* __restrict__ out) {
-  const int c = blockIdx.x * blockDim.x + threadIdx.x;
-  if (c >= cols) return;
+// out[c] = sum over p of part[p][c]: 32 columns x 32 part-lanes per block,
+// each lane sums every 32nd partial row, then a fixed-order sum over lanes.
+__global__ void __launch_bounds__(1024) colsum_finalize_kernel(const float* __restrict__ part, int nparts, int cols,
+                                                             float* __restrict__ out) {
+  __shared__ float red[32][33];
+  const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;
+  const int c = blockIdx.x * 32 + tx;
   float s = 0.0f;
-  for (int p = 0; p < nparts; ++p) s += part[(size_t)p * cols + c];
-  out[c] = s;
+  if (c < cols) {
+#pragma unroll 4
+    for (int p = ty; p < nparts; p += 32) s += part[(size_t)p * cols + c];
+  }
+  red[ty][tx] = s;
+  __syncthreads();
+  if (ty == 0 && c < cols) {
+    float t = 0.0f;
+#pragma unroll
+    for (int w = 0; w < 32; ++w) t += red[w][tx];
+    out[c] = t;
+  }
 }
 
 template <typename T>
@@ -278,68 +309,40 @@ __global__ void dropout_mask_kernel(DropoutParams dp, int site, uint64_t e0, uin
   }
 }
 
-int nch_of(int H) { return (H + 255) / 256; }
-
-#define TLP_NCH_SWITCH(H, ...)                        \
-  switch (nch_of(H)) {                                \
-    case 1: { constexpr int NCH = 1; __VA_ARGS__; } break; \
-    case 2: { constexpr int NCH = 2; __VA_ARGS__; } break; \
-    case 3: { constexpr int NCH = 3; __VA_ARGS__; } break; \
-    case 4: { constexpr int NCH = 4; __VA_ARGS__; } break; \
-    case 5: { constexpr int NCH = 5; __VA_ARGS__; } break; \
-    case 6: { constexpr int NCH = 6; __VA_ARGS__; } break; \
-    case 7: { constexpr int NCH = 7; __VA_ARGS__; } break; \
-    case 8: { constexpr int NCH = 8; __VA_ARGS__; } break; \
-    case 12: { constexpr int NCH = 12; __VA_ARGS__; } break; \
-    case 16: { constexpr int NCH = 16; __VA_ARGS__; } break; \
-    default: break;                                   \
-  }
+int row_blocks(int rows) { return std::max(1, std::min(kMaxBlocks, (rows + 4 * kRows - 1) / (4 * kRows))); }
 
 template <typename T>
 void ln_fwd_t(const void* x, const void* g, const void* b, void* y, float* mean, float* rstd, int rows, int H,
               float eps, cudaStream_t s) {
-  const int blocks = (rows + kWarps - 1) / kWarps;
-  TLP_NCH_SWITCH(H, ln_fwd_kernel<T, NCH><<<blocks, kWarps * 32, 0, s>>>(
-                        static_cast<const T*>(x), static_cast<const T*>(g), static_cast<const T*>(b),
-                        static_cast<T*>(y), mean, rstd, rows, H, eps));
+  // one group of kRows rows per block: no column sums, so maximal parallelism
+  ln_fwd_kernel<T><<<(rows + kRows - 1) / kRows, row_threads(H), 0, s>>>(static_cast<const T*>(x), static_cast<const T*>(g),
+                                                              static_cast<const T*>(b), static_cast<T*>(y), mean,
+                                                              rstd, rows, H, eps);
   count_launch();
 }
 
 template <typename T, bool INV>
 void ln_bwd_t(const LnBwdArgs& a, cudaStream_t s) {
-  const int blocks = ln_bwd_parts(a.rows);
-  const size_t smem = (size_t)kWarps * a.H * sizeof(float);
-  TLP_NCH_SWITCH(a.H, {
-    cudaFuncSetAttribute(ln_bwd_kernel<T, NCH, INV>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    ln_bwd_kernel<T, NCH, INV><<<blocks, kWarps * 32, smem, s>>>(a);
-  });
+  ln_bwd_kernel<T, INV><<<ln_bwd_parts(a.rows), row_threads(a.H), 0, s>>>(a);
   count_launch();
 }
 
 template <typename T>
 void dropout_rows_t(const void* in, void* out, const DropoutParams& dp, int site, int rows, int H, float* part,
                     cudaStream_t s) {
-  const int blocks = rowdrop_parts(rows);
-  const size_t smem = (size_t)kWarps * H * sizeof(float);
-  TLP_NCH_SWITCH(H, {
-    cudaFuncSetAttribute(dropout_rows_kernel<T, NCH>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    dropout_rows_kernel<T, NCH><<<blocks, kWarps * 32, smem, s>>>(static_cast<const T*>(in), static_cast<T*>(out),
-                                                                  dp, site, rows, H, part);
-  });
+  dropout_rows_kernel<T><<<rowdrop_parts(rows), row_threads(H), 0, s>>>(static_cast<const T*>(in),
+                                                                       static_cast<T*>(out), dp, site, rows, H, part);
   count_launch();
 }
 
 }  // namespace
 
-// Hidden sizes served by the row kernels: multiples of 8 up to 4096 whose
-// 256-column chunk count has an instantiation above.
-bool rowwise_supports_hidden(int H) {
-  const int n = nch_of(H);
-  return H % 8 == 0 && H <= 4096 && (n <= 8 || n == 12 || n == 16);
-}
+// Hidden sizes served by the row kernels: multiples of 8 up to 4096 (one
+// thread per 8 columns, at most 512 threads per block).
+bool rowwise_supports_hidden(int H) { return H % 8 == 0 && H <= 4096; }
 
-int ln_bwd_parts(int rows) { return std::max(1, std::min(kMaxParts, (rows + kWarps - 1) / kWarps)); }
-int rowdrop_parts(int rows) { return ln_bwd_parts(rows); }
+int ln_bwd_parts(int rows) { return row_blocks(rows); }
+int rowdrop_parts(int rows) { return row_blocks(rows); }
 int colsum_parts(int rows) { return std::max(1, std::min(kColParts, rows / 64)); }
 
 void ln_fwd_run(int dt, const void* x, const void* g, const void* b, void* y, float* mean, float* rstd, int rows,
@@ -372,7 +375,7 @@ void colsum_run(int dt, const void* X, int rows, int cols, float* part, cudaStre
 }
 
 void colsum_finalize_run(const float* part, int nparts, int cols, float* out, cudaStream_t s) {
-  colsum_finalize_kernel<<<(cols + 255) / 256, 256, 0, s>>>(part, nparts, cols, out);
+  colsum_finalize_kernel<<<(cols + 31) / 32, 1024, 0, s>>>(part, nparts, cols, out);
   count_launch();
 }
 
