@@ -147,6 +147,12 @@ void layer_destroy(tl_layer* layer);
 tl_status tl_dropout_keep_mask(uint64_t seed, uint64_t philox_offset, int site, float p,
                                uint64_t e0, uint64_t n, uint8_t* keep, void* stream);
 
+/* Test hook: g[i] = GELU(u[i]) and dg[i] = GELU'(u[i]) for i < n (float32
+ * device buffers), evaluated by the same device code the layer's GEMM
+ * epilogues use (erf form, CUDA's erff; the density term uses the fast
+ * exponential). */
+tl_status tl_gelu_eval(const float* u, float* g, float* dg, uint64_t n, void* stream);
+
 /* Waits for all work on the current device, then reports TL_ECUDA if a CUDA
  * error is pending, TL_ETIMEOUT if a bounded device-side wait of a
  * tensor-core kernel gave up since the last call (the flag is cleared), else

@@ -1,0 +1,23 @@
+"""The device GELU (erf form: CUDA's erff; GELU' adds u * phi(u) with the fast
+exponential) against the oracle's exact GELU and its derivative."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import transformer_layer_pre_b200 as tlp
+
+pytestmark = pytest.mark.gpu
+
+
+def test_device_gelu_matches_exact_erf_form():
+    u = np.concatenate([np.linspace(-10, 10, 200001), np.random.default_rng(3).normal(0, 3, 100000),
+                        [0.0, -0.0, 1e-30, -1e-30, 1e-6, 40.0, -40.0]]).astype(np.float32)
+    g, dg = tlp.gelu_eval(torch.from_numpy(u).cuda())
+    u64 = u.astype(np.float64)
+    ref_g, ref_dg = oracle.gelu(u64), oracle.gelu_grad(u64)
+    # erff is within a few float32 ulps: GELU error <= 0.5 |u| * 4 ulp(1) + float32 rounding of the product
+    eps = np.finfo(np.float32).eps
+    tol_g = 0.5 * np.abs(u64) * 4 * eps + 4 * eps * np.abs(ref_g)
+    assert np.all(np.abs(g.cpu().double().numpy() - ref_g) <= tol_g + 1e-30)
+    assert np.abs(dg.cpu().double().numpy() - ref_dg).max() <= 1e-6

@@ -29,7 +29,7 @@ EXPORTED_SYMBOLS = (
     "layer_create", "layer_default_options", "layer_set_options", "layer_get_options",
     "layer_forward", "layer_backward", "layer_workspace_bytes", "layer_last_error",
     "layer_destroy", "tl_dropout_keep_mask", "tl_device_check", "tl_profile_enable",
-    "tl_profile_read", "tl_launch_count", "tl_bias_grad_noalloc", "tl_status_string",
+    "tl_profile_read", "tl_launch_count", "tl_bias_grad_noalloc", "tl_gelu_eval", "tl_status_string",
 )
 PROFILE_CLASSES = ("gemm", "attn_fwd", "attn_bwd", "ln_fwd", "ln_bwd", "rowwise")
 
@@ -102,6 +102,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.tl_launch_count.restype = ctypes.c_longlong
     lib.tl_bias_grad_noalloc.argtypes = [i, vp, i, i, vp, vp]
     lib.tl_bias_grad_noalloc.restype = i
+    lib.tl_gelu_eval.argtypes = [vp, vp, vp, u64, vp]
+    lib.tl_gelu_eval.restype = i
     lib.tl_status_string.argtypes = [i]
     lib.tl_status_string.restype = ctypes.c_char_p
     _lib = lib
@@ -205,6 +207,18 @@ def device_check() -> None:
     st = lib.tl_device_check()
     if st != 0:
         raise TlError(st, lib.tl_status_string(st).decode())
+
+
+def gelu_eval(u: torch.Tensor):
+    """(GELU(u), GELU'(u)) from the library's device GELU; u float32 on the device."""
+    lib = load_library()
+    u = u.contiguous()
+    g = torch.empty_like(u)
+    dg = torch.empty_like(u)
+    st = lib.tl_gelu_eval(_ptr(u), _ptr(g), _ptr(dg), u.numel(), _stream(None))
+    if st != 0:
+        raise TlError(st, lib.tl_status_string(st).decode())
+    return g, dg
 
 
 def profile_enable(on: bool) -> None:

@@ -72,6 +72,37 @@ template <typename T> __device__ __forceinline__ void unpack8(const uint4& r, fl
 #pragma unroll
   for (int i = 0; i < 8; ++i) v[i] = to_f(h[i]);
 }
+// Raw 8-element chunk as loaded from memory (16 bytes for 16-bit types, 32
+// for float), so a load can be issued early and converted later.
+template <typename T> struct Raw8 { uint4 a; };
+template <> struct Raw8<float> { float4 a, b; };
+
+template <typename T> __device__ __forceinline__ Raw8<T> raw8_load(const T* p) {
+  Raw8<T> r;
+  r.a = *reinterpret_cast<const uint4*>(p);
+  return r;
+}
+template <> __device__ __forceinline__ Raw8<float> raw8_load<float>(const float* p) {
+  Raw8<float> r;
+  r.a = reinterpret_cast<const float4*>(p)[0];
+  r.b = reinterpret_cast<const float4*>(p)[1];
+  return r;
+}
+template <typename T> __device__ __forceinline__ Raw8<T> raw8_zero() {
+  Raw8<T> r;
+  r.a = make_uint4(0u, 0u, 0u, 0u);
+  return r;
+}
+template <> __device__ __forceinline__ Raw8<float> raw8_zero<float>() {
+  Raw8<float> r;
+  r.a = r.b = make_float4(0.f, 0.f, 0.f, 0.f);
+  return r;
+}
+template <typename T> __device__ __forceinline__ void raw8_unpack(const Raw8<T>& r, float (&v)[8]) { unpack8<T>(r.a, v); }
+template <> __device__ __forceinline__ void raw8_unpack<float>(const Raw8<float>& r, float (&v)[8]) {
+  v[0] = r.a.x; v[1] = r.a.y; v[2] = r.a.z; v[3] = r.a.w; v[4] = r.b.x; v[5] = r.b.y; v[6] = r.b.z; v[7] = r.b.w;
+}
+
 template <typename T> __device__ __forceinline__ void store8(T* p, const float (&v)[8]) { Vec8Io<T>::store(p, v); }
 
 // ------------------------------------------------------------------ Philox4x32-10
@@ -126,7 +157,7 @@ __device__ __forceinline__ uint32_t dropout_bits8(const DropoutParams& dp, int s
 // ------------------------------------------------------------------ GELU (erf form)
 __device__ __forceinline__ float gelu_f(float u) { return 0.5f * u * (1.0f + erff(u * 0.70710678118654752f)); }
 __device__ __forceinline__ float gelu_grad_f(float u) {
-  return 0.5f * (1.0f + erff(u * 0.70710678118654752f)) + u * 0.39894228040143268f * expf(-0.5f * u * u);
+  return fmaf(u * 0.39894228040143268f, __expf(-0.5f * u * u), 0.5f * (1.0f + erff(u * 0.70710678118654752f)));
 }
 
 // ------------------------------------------------------------------ warp reductions

@@ -24,11 +24,13 @@ size_t gemm_splitk_ws_floats(int dtype, int M, int N, int K) {
 }
 
 int attn_tc_take_error();
+int rowwise_take_error();
 
 int device_take_error() {
   const int g = gemm_tc_take_error();
   const int a = attn_tc_take_error();
-  return g ? g : a;
+  const int r = rowwise_take_error();
+  return g ? g : (a ? a : r);
 }
 
 }  // namespace tlp

@@ -43,7 +43,8 @@ namespace {
 
 constexpr int BM = 128;
 constexpr int BK = 64;
-constexpr int kThreads = 320;   // TMA warp, MMA warp, 8 epilogue warps
+constexpr int kEpiWarps = 8;
+constexpr int kThreads = 64 + 32 * kEpiWarps;   // TMA warp, MMA warp, epilogue warps
 
 template <int BN> struct TileCfg {
   static constexpr int kStages = BN == 256 ? 4 : 6;
@@ -92,7 +93,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&tfull[a], 1);
-      mbar_init(&tempty[a], 256);
+      mbar_init(&tempty[a], 32 * kEpiWarps);
     }
     fence_barrier_init();
   }
@@ -188,9 +189,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else {
     // Epilogue warps 2..9: warp w may access TMEM lanes 32*(w%4) .. +31 (one
     // output row per thread) and takes half of the tile's columns.
-    constexpr int CW = BN / 2;
+    constexpr int CW = BN / (kEpiWarps / 4);
     const int quarter = warp & 3;
-    const int half = (warp - 2) >> 2;
+    const int part = (warp - 2) >> 2;
     const int row = quarter * 32 + lane;
     int acc = 0;
     uint32_t aph = 0;
@@ -198,7 +199,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       int mb, nb, sp;
       decode_tile(g, t, mb, nb, sp);
       const int m = mb * BM + row;
-      const int nbase = nb * BN + half * CW;
+      const int nbase = nb * BN + part * CW;
       const bool mrow = m < g.M;
       // the residual / U values of this thread's columns are fetched before
       // the accumulator is ready, so their latency hides under the main loop
@@ -218,7 +219,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_after();
       EpiParams ep = e;
       if constexpr (KIND == EPI_F32) ep.out = static_cast<float*>(e.out) + (size_t)sp * g.split_stride;
-      const uint32_t tbase = tmem + ((uint32_t)(quarter * 32) << 16) + acc * BN + half * CW;
+      const uint32_t tbase = tmem + ((uint32_t)(quarter * 32) << 16) + acc * BN + part * CW;
 #pragma unroll
       for (int c0 = 0; c0 < CW; c0 += 32) {
         float v[32];

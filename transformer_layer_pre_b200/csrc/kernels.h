@@ -95,6 +95,11 @@ int colsum_parts(int rows);
 void colsum_run(int dtype, const void* X, int rows, int cols, float* part, cudaStream_t s);
 // out[c] = sum_p part[p*cols + c] (fixed order).
 void colsum_finalize_run(const float* part, int nparts, int cols, float* out, cudaStream_t s);
+// The same for up to three (partials, output) pairs in one launch (p1/p2 may be null).
+void colsum_finalize3_run(const float* p0, const float* p1, const float* p2, float* o0, float* o1, float* o2,
+                          int nparts, int cols, cudaStream_t s);
+// g[i] = GELU(u[i]), dg[i] = GELU'(u[i]) with the device GELU every kernel uses (float32).
+void gelu_eval_run(const float* u, float* g, float* dg, uint64_t n, cudaStream_t s);
 // G = GELU(U), elementwise, n a multiple of 8.
 void gelu_run(int dtype, const void* U, void* G, size_t n, cudaStream_t s);
 // keep[i] = dropout keep bit of element e0 + i of `site`.

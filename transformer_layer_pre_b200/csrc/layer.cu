@@ -427,9 +427,7 @@ tl_status layer_backward(tl_layer* L, const void* x, const void* dy, const tl_we
     a.rows = T; a.H = H;
     ProfScope p_(PC_LN_BWD, s);
     ln_bwd_run(dt, a, s);
-    colsum_finalize_run(pa, lnp, H, dgamma, s);
-    colsum_finalize_run(pb, lnp, H, dbeta, s);
-    if (drop_out) colsum_finalize_run(pc, lnp, H, dsum, s);
+    colsum_finalize3_run(pa, pb, drop_out ? pc : nullptr, dgamma, dbeta, drop_out ? dsum : nullptr, lnp, H, s);
   };
 
   // FFN block: dZ2 -> dW2, dU (into big), db1, dW1; returns with dU in L->big
@@ -505,6 +503,13 @@ tl_status tl_device_check(void) {
   cudaError_t e = cudaDeviceSynchronize();
   if (e != cudaSuccess) return TL_ECUDA;
   return device_take_error() ? TL_ETIMEOUT : TL_OK;
+}
+
+tl_status tl_gelu_eval(const float* u, float* g, float* dg, uint64_t n, void* stream) {
+  if (!u || !g || !dg) return TL_EINVAL;
+  if (n == 0) return TL_OK;
+  gelu_eval_run(u, g, dg, n, (cudaStream_t)stream);
+  return cudaGetLastError() == cudaSuccess ? TL_OK : TL_ECUDA;
 }
 
 tl_status tl_dropout_keep_mask(uint64_t seed, uint64_t philox_offset, int site, float p, uint64_t e0, uint64_t n,

@@ -4,44 +4,63 @@
 // LayerNorm is per token over the hidden axis with the biased variance and
 // eps inside the square root; statistics are float32 ("AI-infra engineers and
 // the Transformer", section 3.2: LayerNorm kept in fp32).  A block owns a
-// contiguous range of rows and each thread 8 consecutive columns of them, so
-// column sums (bias and LayerNorm-parameter gradients) accumulate in the
-// owning thread's registers in row order and leave as one partial row per
-// block, summed by tlp::colsum_finalize_run in block order: deterministic.
+// contiguous range of rows, streamed into shared memory by bulk asynchronous
+// copies, and each thread 8 consecutive columns of them, so column sums (bias
+// and LayerNorm-parameter gradients) accumulate in the owning thread's
+// registers in row order and leave as one partial row per block, summed by
+// tlp::colsum_finalize_run in block order: deterministic.
 #include <algorithm>
 
 #include "common.cuh"
 #include "kernels.h"
 #include "profile.h"
+#include "sm100.cuh"
 
 namespace tlp {
 
 namespace {
 
-// Row-block kernels: a block of ceil(H/8 / 32) warps owns a contiguous range
-// of rows; thread t owns columns 8t .. 8t+7 of every row of that range (one
-// 16-byte vector for 16-bit storage) and walks the rows kRows at a time.
-// Row statistics are block reductions (one per kRows rows); column sums stay
-// in the owning thread's registers and leave as one partial row per block.
-constexpr int kRows = 4;
-constexpr int kMaxBlocks = 592;   // 4 blocks per SM
+// Row-block kernels: a block owns a contiguous range of rows; thread t owns
+// columns 8t .. 8t+7 of every row of that range.  Thread 0 streams the rows
+// into shared memory kRowsPer rows at a time with bulk asynchronous copies,
+// kStages groups ahead, so DRAM stays busy while the block computes; the
+// other threads read their columns from shared memory.  Row statistics are
+// block reductions (one per group); column sums stay in the owning thread's
+// registers and leave as one partial row per block.
+constexpr int kStages = 4;
+constexpr int kMaxBlocks = 296;        // 2 blocks per SM
+__device__ int g_row_err;              // set when a bounded wait gives up
 
 __host__ __device__ inline int row_threads(int H) { return ((H / 8 + 31) / 32) * 32; }
 
-// Sums v[r] over the whole block; red holds (warps, kRows) floats.
-__device__ __forceinline__ void block_sum(float (&v)[kRows], float* red) {
+// Rows per pipeline group: a group of one tensor is at most 8 KB.
+__host__ __device__ inline int group_rows(int H, int es) {
+  const int r = 8192 / (H * es);
+  return r >= 4 ? 4 : (r >= 2 ? 2 : 1);
+}
+
+__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                   sm100::smem_u32(dst)),
+               "l"(src), "r"(bytes), "r"(sm100::smem_u32(bar))
+               : "memory");
+}
+
+// Sums v[r] over the whole block; red holds (warps, KR) floats.
+template <int KR>
+__device__ __forceinline__ void block_sum(float (&v)[KR], float* red) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
 #pragma unroll
-  for (int r = 0; r < kRows; ++r) v[r] = warp_sum(v[r]);
+  for (int r = 0; r < KR; ++r) v[r] = warp_sum(v[r]);
   if (lane == 0) {
 #pragma unroll
-    for (int r = 0; r < kRows; ++r) red[warp * kRows + r] = v[r];
+    for (int r = 0; r < KR; ++r) red[warp * KR + r] = v[r];
   }
   __syncthreads();
 #pragma unroll
-  for (int r = 0; r < kRows; ++r) {
+  for (int r = 0; r < KR; ++r) {
     float s = 0.0f;
-    for (int w = 0; w < nw; ++w) s += red[w * kRows + r];
+    for (int w = 0; w < nw; ++w) s += red[w * KR + r];
     v[r] = s;
   }
   __syncthreads();
@@ -59,74 +78,146 @@ __device__ __forceinline__ void store_part(float* part, int H, int col, const fl
   reinterpret_cast<float4*>(p)[1] = make_float4(acc[4], acc[5], acc[6], acc[7]);
 }
 
-// ------------------------------------------------------------------ LayerNorm forward
-template <typename T>
-__global__ void __launch_bounds__(512) ln_fwd_kernel(const T* __restrict__ x, const T* __restrict__ gamma,
-                                                    const T* __restrict__ beta, T* __restrict__ y,
-                                                    float* __restrict__ mean_out, float* __restrict__ rstd_out,
-                                                    int rows, int H, float eps) {
-  __shared__ float red[16 * kRows];
-  const int col = threadIdx.x * 8;
-  const bool act = col < H;
-  float g[8], b[8];
-  if (act) {
-    load8<T>(gamma + col, g);
-    load8<T>(beta + col, b);
-  }
-  int r0, r1;
-  row_range(rows, r0, r1);
-  const float inv_h = 1.0f / (float)H;
-  for (int base = r0; base < r1; base += kRows) {
-    float v[kRows][8], s[kRows];
-#pragma unroll
-    for (int r = 0; r < kRows; ++r) {
-      s[r] = 0.0f;
-      if (act && base + r < r1) {
-        load8<T>(x + (size_t)(base + r) * H + col, v[r]);
-#pragma unroll
-        for (int i = 0; i < 8; ++i) s[r] += v[r][i];
-      } else {
-#pragma unroll
-        for (int i = 0; i < 8; ++i) v[r][i] = 0.0f;
-      }
+// Pipeline of row groups: NT tensors of row stride H elements, KR rows per
+// group, kStages groups in flight.  Layout per stage: NT x [KR][H].
+template <typename T, int KR, int NT>
+struct RowPipe {
+  uint8_t* buf;
+  uint64_t* full;
+  const T* src[NT];
+  int H, r0, r1, ngroups;
+
+  __device__ size_t tensor_bytes() const { return (size_t)KR * H * sizeof(T); }
+  __device__ size_t stage_bytes() const { return NT * tensor_bytes(); }
+
+  __device__ void init(uint8_t* smem, int H_, int r0_, int r1_) {
+    H = H_; r0 = r0_; r1 = r1_;
+    ngroups = (r1 - r0 + KR - 1) / KR;
+    buf = smem;
+    full = reinterpret_cast<uint64_t*>(smem + kStages * stage_bytes());
+    if (threadIdx.x == 0) {
+      for (int s = 0; s < kStages; ++s) sm100::mbar_init(&full[s], 1);
+      sm100::fence_barrier_init();
     }
-    block_sum(s, red);
-    float mean[kRows], ss[kRows];
+    __syncthreads();
+    if (threadIdx.x == 0)
+      for (int g = 0; g < kStages && g < ngroups; ++g) issue(g);
+  }
+  // thread 0: copy group g into its stage
+  __device__ void issue(int g) {
+    const int s = g % kStages;
+    const int row = r0 + g * KR;
+    const uint32_t bytes = (uint32_t)(min(KR, r1 - row) * (size_t)H * sizeof(T));
+    uint8_t* dst = buf + s * stage_bytes();
+    sm100::mbar_arrive_expect_tx(&full[s], NT * bytes);
 #pragma unroll
-    for (int r = 0; r < kRows; ++r) {
-      mean[r] = s[r] * inv_h;
-      ss[r] = 0.0f;
-      if (act) {
+    for (int t = 0; t < NT; ++t) bulk_load(dst + t * tensor_bytes(), src[t] + (size_t)row * H, bytes, &full[s]);
+  }
+  // every thread: wait for group g; false if the wait gave up
+  __device__ bool wait(int g) {
+    return sm100::mbar_wait(&full[g % kStages], (uint32_t)((g / kStages) & 1), &g_row_err, 1);
+  }
+  __device__ const T* row(int g, int t, int r) const {
+    return reinterpret_cast<const T*>(buf + (g % kStages) * stage_bytes() + t * tensor_bytes()) + (size_t)r * H;
+  }
+  // after every thread is done with group g (block barrier): refill its stage
+  __device__ void release(int g) {
+    if (threadIdx.x == 0 && g + kStages < ngroups) {
+      sm100::fence_proxy_async_smem();
+      issue(g + kStages);
+    }
+  }
+  // an abandoned pipeline still has copies in flight: let them land
+  __device__ void drain(int g) {
+    if (threadIdx.x == 0)
+      for (int k = g; k < ngroups && k < g + kStages; ++k) sm100::mbar_wait(&full[k % kStages], (k / kStages) & 1, nullptr, 0);
+  }
+};
+
+template <typename T, int KR, int NT>
+size_t pipe_smem(int H) {
+  return (size_t)kStages * NT * KR * H * sizeof(T) + kStages * sizeof(uint64_t) + 32 * 2 * KR * sizeof(float);
+}
+
+// ------------------------------------------------------------------ LayerNorm forward
+// One warp per row, kFwdRows rows per warp loaded up front (16-byte vectors,
+// lane-interleaved chunks of 8), shuffle-only reductions, gamma/beta staged
+// in shared memory as float32.  NCH = chunks of 8 per lane (H <= 256*NCH).
+constexpr int kFwdRows = 2;
+constexpr int kFwdWarps = 8;
+
+template <typename T, int NCH>
+__global__ void __launch_bounds__(kFwdWarps * 32) ln_fwd_kernel(const T* __restrict__ x, const T* __restrict__ gamma,
+                                                                const T* __restrict__ beta, T* __restrict__ y,
+                                                                float* __restrict__ mean_out,
+                                                                float* __restrict__ rstd_out, int rows, int H,
+                                                                float eps) {
+  extern __shared__ float gb[];   // [2][H]
+  for (int c = threadIdx.x; c < H; c += blockDim.x) {
+    gb[c] = to_f(gamma[c]);
+    gb[H + c] = to_f(beta[c]);
+  }
+  __syncthreads();
+  const int lane = threadIdx.x & 31;
+  const int row0 = (blockIdx.x * kFwdWarps + (threadIdx.x >> 5)) * kFwdRows;
+  Raw8<T> raw[kFwdRows][NCH];
+#pragma unroll
+  for (int r = 0; r < kFwdRows; ++r) {
+#pragma unroll
+    for (int c = 0; c < NCH; ++c) {
+      const int col = (lane + 32 * c) * 8;
+      raw[r][c] = (row0 + r < rows && col < H) ? raw8_load<T>(x + (size_t)(row0 + r) * H + col) : raw8_zero<T>();
+    }
+  }
+  const float inv_h = 1.0f / (float)H;
+#pragma unroll
+  for (int r = 0; r < kFwdRows; ++r) {
+    const int row = row0 + r;
+    if (row >= rows) break;
+    float v[NCH][8];
+    float s = 0.0f;
+#pragma unroll
+    for (int c = 0; c < NCH; ++c) {
+      raw8_unpack<T>(raw[r][c], v[c]);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) s += v[c][i];
+    }
+    const float mean = warp_sum(s) * inv_h;
+    float ss = 0.0f;
+#pragma unroll
+    for (int c = 0; c < NCH; ++c) {
+      if ((lane + 32 * c) * 8 < H) {
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
-          const float d = v[r][i] - mean[r];
-          ss[r] += d * d;
+          const float d = v[c][i] - mean;
+          ss += d * d;
         }
       }
     }
-    block_sum(ss, red);
+    const float rstd = 1.0f / sqrtf(warp_sum(ss) * inv_h + eps);
 #pragma unroll
-    for (int r = 0; r < kRows; ++r) {
-      if (base + r >= r1) continue;
-      const float rstd = 1.0f / sqrtf(ss[r] * inv_h + eps);
-      if (act) {
+    for (int c = 0; c < NCH; ++c) {
+      const int col = (lane + 32 * c) * 8;
+      if (col < H) {
         float o[8];
 #pragma unroll
-        for (int i = 0; i < 8; ++i) o[i] = g[i] * ((v[r][i] - mean[r]) * rstd) + b[i];
-        store8<T>(y + (size_t)(base + r) * H + col, o);
+        for (int i = 0; i < 8; ++i) o[i] = gb[col + i] * ((v[c][i] - mean) * rstd) + gb[H + col + i];
+        store8<T>(y + (size_t)row * H + col, o);
       }
-      if (threadIdx.x == 0) {
-        mean_out[base + r] = mean[r];
-        rstd_out[base + r] = rstd;
-      }
+    }
+    if (lane == 0) {
+      mean_out[row] = mean;
+      rstd_out[row] = rstd;
     }
   }
 }
 
 // ------------------------------------------------------------------ LayerNorm backward
-template <typename T, bool INV>
+// Pipeline tensors: 0 dy, 1 x (or y when invertible), 2 res (when given).
+template <typename T, bool INV, bool RES, int KR>
 __global__ void __launch_bounds__(512) ln_bwd_kernel(LnBwdArgs a) {
-  __shared__ float red[16 * kRows];
+  extern __shared__ __align__(128) uint8_t smem[];
+  constexpr int NT = RES ? 3 : 2;
   const int H = a.H;
   const int col = threadIdx.x * 8;
   const bool act = col < H;
@@ -138,28 +229,34 @@ __global__ void __launch_bounds__(512) ln_bwd_kernel(LnBwdArgs a) {
     load8<T>(static_cast<const T*>(a.gamma) + col, gm);
     if constexpr (INV) load8<T>(static_cast<const T*>(a.beta) + col, bt);
   }
-  const T* dyp = static_cast<const T*>(a.dy);
   const float inv_h = 1.0f / (float)H;
   const float sc = a.drop.thr ? a.drop.scale : 1.0f;
   int r0, r1;
   row_range(a.rows, r0, r1);
-  for (int base = r0; base < r1; base += kRows) {
-    float g[kRows][8], xh[kRows][8], s1[kRows], s2[kRows], rs[kRows];
+  RowPipe<T, KR, NT> pipe;
+  pipe.src[0] = static_cast<const T*>(a.dy);
+  pipe.src[1] = static_cast<const T*>(INV ? a.y : a.x);
+  if constexpr (RES) pipe.src[2] = static_cast<const T*>(a.res);
+  pipe.init(smem, H, r0, r1);
+  float* red = reinterpret_cast<float*>(pipe.full + kStages);
+  for (int gi = 0; gi < pipe.ngroups; ++gi) {
+    const bool ok = pipe.wait(gi);
+    if (__syncthreads_or(!ok)) { pipe.drain(gi); return; }
+    const int base = r0 + gi * KR;
+    float g[KR][8], xh[KR][8], s1[KR], s2[KR], rs[KR];
 #pragma unroll
-    for (int r = 0; r < kRows; ++r) {
+    for (int r = 0; r < KR; ++r) {
       s1[r] = s2[r] = 0.0f;
       const int row = base + r;
       rs[r] = row < r1 ? a.rstd[row] : 0.0f;
       if (act && row < r1) {
-        const size_t off = (size_t)row * H + col;
         float dy[8], xv[8];
-        load8<T>(dyp + off, dy);
+        load8<T>(pipe.row(gi, 0, r) + col, dy);
+        load8<T>(pipe.row(gi, 1, r) + col, xv);
         if constexpr (INV) {
-          load8<T>(static_cast<const T*>(a.y) + off, xv);
 #pragma unroll
           for (int i = 0; i < 8; ++i) xh[r][i] = (xv[i] - bt[i]) / gm[i];
         } else {
-          load8<T>(static_cast<const T*>(a.x) + off, xv);
           const float mean = a.mean[row];
 #pragma unroll
           for (int i = 0; i < 8; ++i) xh[r][i] = (xv[i] - mean) * rs[r];
@@ -177,20 +274,25 @@ __global__ void __launch_bounds__(512) ln_bwd_kernel(LnBwdArgs a) {
         for (int i = 0; i < 8; ++i) g[r][i] = xh[r][i] = 0.0f;
       }
     }
-    block_sum(s1, red);
-    block_sum(s2, red);
+    float s12[2 * KR];
 #pragma unroll
-    for (int r = 0; r < kRows; ++r) {
+    for (int r = 0; r < KR; ++r) {
+      s12[r] = s1[r];
+      s12[KR + r] = s2[r];
+    }
+    block_sum<2 * KR>(s12, red);
+#pragma unroll
+    for (int r = 0; r < KR; ++r) {
       const int row = base + r;
       if (!act || row >= r1) continue;
       const size_t off = (size_t)row * H + col;
-      const float m1 = s1[r] * inv_h, m2 = s2[r] * inv_h;
+      const float m1 = s12[r] * inv_h, m2 = s12[KR + r] * inv_h;
       float o[8];
 #pragma unroll
       for (int i = 0; i < 8; ++i) o[i] = rs[r] * (g[r][i] - m1 - xh[r][i] * m2);
-      if (a.res) {
+      if constexpr (RES) {
         float rv[8];
-        load8<T>(static_cast<const T*>(a.res) + off, rv);
+        load8<T>(pipe.row(gi, 2, r) + col, rv);
 #pragma unroll
         for (int i = 0; i < 8; ++i) o[i] += rv[i];
       }
@@ -205,6 +307,8 @@ __global__ void __launch_bounds__(512) ln_bwd_kernel(LnBwdArgs a) {
         store8<T>(static_cast<T*>(a.drop_out) + off, o);
       }
     }
+    __syncthreads();
+    pipe.release(gi);
   }
   if (act) {
     store_part(a.part_dgamma, H, col, dg);
@@ -214,29 +318,43 @@ __global__ void __launch_bounds__(512) ln_bwd_kernel(LnBwdArgs a) {
 }
 
 // ------------------------------------------------------------------ dropout of rows
-template <typename T>
+template <typename T, int KR>
 __global__ void __launch_bounds__(512) dropout_rows_kernel(const T* __restrict__ in, T* __restrict__ out,
-                                                            DropoutParams dp, int site, int rows, int H,
-                                                            float* __restrict__ part) {
+                                                           DropoutParams dp, int site, int rows, int H,
+                                                           float* __restrict__ part) {
+  extern __shared__ __align__(128) uint8_t smem[];
   const int col = threadIdx.x * 8;
-  if (col >= H) return;
+  const bool act = col < H;
   float acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
   const float sc = dp.thr ? dp.scale : 1.0f;
   int r0, r1;
   row_range(rows, r0, r1);
-  for (int row = r0; row < r1; ++row) {
-    const size_t off = (size_t)row * H + col;
-    float v[8];
-    load8<T>(in + off, v);
-    const uint32_t bits = dp.thr ? dropout_bits8(dp, site, off >> 3) : 0xFFu;
+  RowPipe<T, KR, 1> pipe;
+  pipe.src[0] = in;
+  pipe.init(smem, H, r0, r1);
+  for (int gi = 0; gi < pipe.ngroups; ++gi) {
+    const bool ok = pipe.wait(gi);
+    if (__syncthreads_or(!ok)) { pipe.drain(gi); return; }
+    const int base = r0 + gi * KR;
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      v[i] = round_f<T>(((bits >> i) & 1u) ? v[i] * sc : 0.0f);
-      acc[i] += v[i];
+    for (int r = 0; r < KR; ++r) {
+      const int row = base + r;
+      if (!act || row >= r1) continue;
+      const size_t off = (size_t)row * H + col;
+      float v[8];
+      load8<T>(pipe.row(gi, 0, r) + col, v);
+      const uint32_t bits = dp.thr ? dropout_bits8(dp, site, off >> 3) : 0xFFu;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        v[i] = round_f<T>(((bits >> i) & 1u) ? v[i] * sc : 0.0f);
+        acc[i] += v[i];
+      }
+      store8<T>(out + off, v);
     }
-    store8<T>(out + off, v);
+    __syncthreads();
+    pipe.release(gi);
   }
-  store_part(part, H, col, acc);
+  if (act) store_part(part, H, col, acc);
 }
 
 // ------------------------------------------------------------------ column sums
@@ -270,14 +388,20 @@ __global__ void __launch_bounds__(256) colsum_kernel(const T* __restrict__ X, in
 
 // out[c] = sum over p of part[p][c]: 32 columns x 32 part-lanes per block,
 // each lane sums every 32nd partial row, then a fixed-order sum over lanes.
-__global__ void __launch_bounds__(1024) colsum_finalize_kernel(const float* __restrict__ part, int nparts, int cols,
-                                                             float* __restrict__ out) {
+// blockIdx.y selects one of up to three (partials, output) pairs.
+struct FinalizeArgs {
+  const float* part[3];
+  float* out[3];
+};
+
+__global__ void __launch_bounds__(1024) colsum_finalize_kernel(FinalizeArgs fa, int nparts, int cols) {
   __shared__ float red[32][33];
+  const float* __restrict__ part = fa.part[blockIdx.y];
   const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;
   const int c = blockIdx.x * 32 + tx;
   float s = 0.0f;
   if (c < cols) {
-#pragma unroll 4
+#pragma unroll 8
     for (int p = ty; p < nparts; p += 32) s += part[(size_t)p * cols + c];
   }
   red[ty][tx] = s;
@@ -286,7 +410,7 @@ __global__ void __launch_bounds__(1024) colsum_finalize_kernel(const float* __re
     float t = 0.0f;
 #pragma unroll
     for (int w = 0; w < 32; ++w) t += red[w][tx];
-    out[c] = t;
+    fa.out[blockIdx.y][c] = t;
   }
 }
 
@@ -309,29 +433,59 @@ __global__ void dropout_mask_kernel(DropoutParams dp, int site, uint64_t e0, uin
   }
 }
 
-int row_blocks(int rows) { return std::max(1, std::min(kMaxBlocks, (rows + 4 * kRows - 1) / (4 * kRows))); }
+int row_blocks(int rows) { return std::max(1, std::min(kMaxBlocks, (rows + 31) / 32)); }
+
+#define TLP_KR_SWITCH(H, ES, ...)                             \
+  switch (group_rows(H, ES)) {                                \
+    case 4: { constexpr int KR = 4; __VA_ARGS__; } break;     \
+    case 2: { constexpr int KR = 2; __VA_ARGS__; } break;     \
+    default: { constexpr int KR = 1; __VA_ARGS__; } break;    \
+  }
+
+#define TLP_NCH_SWITCH(H, ...)                                                  \
+  switch ((H + 255) / 256) {                                                   \
+    case 1: { constexpr int NCH = 1; __VA_ARGS__; } break;                     \
+    case 2: { constexpr int NCH = 2; __VA_ARGS__; } break;                     \
+    case 3: { constexpr int NCH = 3; __VA_ARGS__; } break;                     \
+    case 4: { constexpr int NCH = 4; __VA_ARGS__; } break;                     \
+    case 5: case 6: { constexpr int NCH = 6; __VA_ARGS__; } break;             \
+    case 7: case 8: { constexpr int NCH = 8; __VA_ARGS__; } break;             \
+    case 9: case 10: case 11: case 12: { constexpr int NCH = 12; __VA_ARGS__; } break; \
+    default: { constexpr int NCH = 16; __VA_ARGS__; } break;                   \
+  }
 
 template <typename T>
 void ln_fwd_t(const void* x, const void* g, const void* b, void* y, float* mean, float* rstd, int rows, int H,
               float eps, cudaStream_t s) {
-  // one group of kRows rows per block: no column sums, so maximal parallelism
-  ln_fwd_kernel<T><<<(rows + kRows - 1) / kRows, row_threads(H), 0, s>>>(static_cast<const T*>(x), static_cast<const T*>(g),
-                                                              static_cast<const T*>(b), static_cast<T*>(y), mean,
-                                                              rstd, rows, H, eps);
+  const int blocks = (rows + kFwdWarps * kFwdRows - 1) / (kFwdWarps * kFwdRows);
+  const size_t sm = 2 * (size_t)H * sizeof(float);
+  TLP_NCH_SWITCH(H, {
+    ln_fwd_kernel<T, NCH><<<blocks, kFwdWarps * 32, sm, s>>>(static_cast<const T*>(x), static_cast<const T*>(g),
+                                                            static_cast<const T*>(b), static_cast<T*>(y), mean, rstd,
+                                                            rows, H, eps);
+  });
   count_launch();
 }
 
-template <typename T, bool INV>
+template <typename T, bool INV, bool RES>
 void ln_bwd_t(const LnBwdArgs& a, cudaStream_t s) {
-  ln_bwd_kernel<T, INV><<<ln_bwd_parts(a.rows), row_threads(a.H), 0, s>>>(a);
+  TLP_KR_SWITCH(a.H, (int)sizeof(T), {
+    const size_t sm = pipe_smem<T, KR, RES ? 3 : 2>(a.H);
+    cudaFuncSetAttribute(ln_bwd_kernel<T, INV, RES, KR>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+    ln_bwd_kernel<T, INV, RES, KR><<<ln_bwd_parts(a.rows), row_threads(a.H), sm, s>>>(a);
+  });
   count_launch();
 }
 
 template <typename T>
 void dropout_rows_t(const void* in, void* out, const DropoutParams& dp, int site, int rows, int H, float* part,
                     cudaStream_t s) {
-  dropout_rows_kernel<T><<<rowdrop_parts(rows), row_threads(H), 0, s>>>(static_cast<const T*>(in),
-                                                                       static_cast<T*>(out), dp, site, rows, H, part);
+  TLP_KR_SWITCH(H, (int)sizeof(T), {
+    const size_t sm = pipe_smem<T, KR, 1>(H);
+    cudaFuncSetAttribute(dropout_rows_kernel<T, KR>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+    dropout_rows_kernel<T, KR><<<rowdrop_parts(rows), row_threads(H), sm, s>>>(
+        static_cast<const T*>(in), static_cast<T*>(out), dp, site, rows, H, part);
+  });
   count_launch();
 }
 
@@ -352,11 +506,24 @@ void ln_fwd_run(int dt, const void* x, const void* g, const void* b, void* y, fl
   else ln_fwd_t<bf16_t>(x, g, b, y, mean, rstd, rows, H, eps, s);
 }
 
+template <typename T>
+void ln_bwd_dispatch(const LnBwdArgs& a, cudaStream_t s) {
+  const bool inv = a.x == nullptr, res = a.res != nullptr;
+  if (inv) res ? ln_bwd_t<T, true, true>(a, s) : ln_bwd_t<T, true, false>(a, s);
+  else res ? ln_bwd_t<T, false, true>(a, s) : ln_bwd_t<T, false, false>(a, s);
+}
+
 void ln_bwd_run(int dt, const LnBwdArgs& a, cudaStream_t s) {
-  const bool inv = a.x == nullptr;
-  if (dt == DT_F32) inv ? ln_bwd_t<float, true>(a, s) : ln_bwd_t<float, false>(a, s);
-  else if (dt == DT_F16) inv ? ln_bwd_t<half_t, true>(a, s) : ln_bwd_t<half_t, false>(a, s);
-  else inv ? ln_bwd_t<bf16_t, true>(a, s) : ln_bwd_t<bf16_t, false>(a, s);
+  if (dt == DT_F32) ln_bwd_dispatch<float>(a, s);
+  else if (dt == DT_F16) ln_bwd_dispatch<half_t>(a, s);
+  else ln_bwd_dispatch<bf16_t>(a, s);
+}
+
+int rowwise_take_error() {
+  int v = 0, z = 0;
+  cudaMemcpyFromSymbol(&v, g_row_err, sizeof(int));
+  if (v) cudaMemcpyToSymbol(g_row_err, &z, sizeof(int));
+  return v;
 }
 
 void dropout_rows_run(int dt, const void* in, void* out, const DropoutParams& dp, int site, int rows, int H,
@@ -375,7 +542,30 @@ void colsum_run(int dt, const void* X, int rows, int cols, float* part, cudaStre
 }
 
 void colsum_finalize_run(const float* part, int nparts, int cols, float* out, cudaStream_t s) {
-  colsum_finalize_kernel<<<(cols + 31) / 32, 1024, 0, s>>>(part, nparts, cols, out);
+  FinalizeArgs fa = {{part, nullptr, nullptr}, {out, nullptr, nullptr}};
+  colsum_finalize_kernel<<<dim3((cols + 31) / 32, 1), 1024, 0, s>>>(fa, nparts, cols);
+  count_launch();
+}
+
+void colsum_finalize3_run(const float* p0, const float* p1, const float* p2, float* o0, float* o1, float* o2,
+                          int nparts, int cols, cudaStream_t s) {
+  FinalizeArgs fa = {{p0, p1, p2}, {o0, o1, o2}};
+  const int n = p2 ? 3 : (p1 ? 2 : 1);
+  colsum_finalize_kernel<<<dim3((cols + 31) / 32, n), 1024, 0, s>>>(fa, nparts, cols);
+  count_launch();
+}
+
+__global__ void gelu_eval_kernel(const float* __restrict__ u, float* __restrict__ g, float* __restrict__ dg,
+                                 uint64_t n) {
+  for (uint64_t i = blockIdx.x * (uint64_t)blockDim.x + threadIdx.x; i < n; i += (uint64_t)gridDim.x * blockDim.x) {
+    g[i] = gelu_f(u[i]);
+    dg[i] = gelu_grad_f(u[i]);
+  }
+}
+
+void gelu_eval_run(const float* u, float* g, float* dg, uint64_t n, cudaStream_t s) {
+  const int blocks = (int)std::min<uint64_t>((n + 255) / 256, 148 * 16);
+  gelu_eval_kernel<<<blocks > 0 ? blocks : 1, 256, 0, s>>>(u, g, dg, n);
   count_launch();
 }
 
