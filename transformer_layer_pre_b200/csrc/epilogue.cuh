@@ -92,6 +92,44 @@ __device__ __forceinline__ void epi_apply8(const EpiParams& e, int m, int n, flo
   }
 }
 
+// Epilogue arithmetic without the store: v becomes the (first) output chunk,
+// v2 the second one (EPI_BIAS_GELU's G).  Used by the tensor-core GEMM, whose
+// stores go through shared memory and TMA.
+template <typename T, int KIND>
+__device__ __forceinline__ void epi_compute8(const EpiParams& e, int m, int n, float (&v)[8], float (&v2)[8],
+                                             const float (&aux)[8]) {
+  if constexpr (KIND == EPI_STORE) {
+    if (e.res) {
+#pragma unroll
+      for (int i = 0; i < 8; ++i) v[i] += aux[i];
+    }
+  } else if constexpr (KIND == EPI_QKV) {
+    float b[8];
+    load8<T>(static_cast<const T*>(e.bias) + n, b);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) v[i] += b[i];
+  } else if constexpr (KIND == EPI_BIAS_DROP_RES) {
+    float b[8];
+    load8<T>(static_cast<const T*>(e.bias) + n, b);
+    uint32_t bits = 0xFFu;
+    if (e.drop.thr) bits = dropout_bits8(e.drop, e.site, ((uint64_t)m * e.ldo + n) >> 3);
+    const float sc = e.drop.thr ? e.drop.scale : 1.0f;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) v[i] = aux[i] + (((bits >> i) & 1u) ? (v[i] + b[i]) * sc : 0.0f);
+  } else if constexpr (KIND == EPI_BIAS_GELU) {
+    float b[8];
+    load8<T>(static_cast<const T*>(e.bias) + n, b);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      v[i] = round_f<T>(v[i] + b[i]);
+      v2[i] = gelu_f(v[i]);
+    }
+  } else if constexpr (KIND == EPI_DGELU) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) v[i] *= gelu_grad_f(aux[i]);
+  }
+}
+
 // Convenience form that loads the auxiliary values itself (SIMT GEMM).
 template <typename T, int KIND>
 __device__ __forceinline__ void epi_apply8(const EpiParams& e, int m, int n, float (&v)[8]) {

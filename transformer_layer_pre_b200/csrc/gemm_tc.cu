@@ -250,6 +250,267 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 1) tmem_dealloc(tmem, C::kTmemCols);
 }
 
+// ============================================================================
+// CTA-pair variant (cta_group::2): a cluster of two CTAs computes a 256 x 256
+// output tile.  Each CTA loads its own 128 rows of A and its own 128 rows
+// (N columns) of B into its own shared memory, signalling the leader CTA's
+// "full" barrier; the leader issues tcgen05.mma.cta_group::2 (M = 256,
+// N = 256), which reads both CTAs' operands and writes each CTA's 128 rows of
+// the accumulator into that CTA's TMEM.  Per SM this halves the B traffic
+// into shared memory (32 KB per 64-wide K block instead of 48 KB), which
+// leaves room for six pipeline stages.  Commits multicast to both CTAs'
+// barriers; both CTAs' epilogues arrive on the leader's "accumulator empty"
+// barrier.  No TMA multicast is used.
+constexpr int kPairStages = 4;
+constexpr int kPairStageBytes = 2 * 128 * BK * 2;                  // A half + B half, 32 KB
+constexpr int kPairEpiWarps = 16;
+constexpr int kPairThreads = 64 + 32 * kPairEpiWarps;
+constexpr int kStageOut = 2048;                                    // one 32-row x 64-byte store box
+constexpr int kPairOutBytes = kPairEpiWarps * 2 * kStageOut;       // two staging buffers per epilogue warp
+constexpr int kPairSmem = kPairStages * kPairStageBytes + kPairOutBytes + 1024 + 256;
+
+// Store destinations of the pair kernel's epilogue (TMA tensor maps).
+struct OutMaps {
+  CUtensorMap out;    // (rows, N) row-major, box 32 rows x 128 bytes, 128-byte swizzle
+  CUtensorMap out2;   // EPI_BIAS_GELU's G
+  int qkv_heads_rows; // EPI_QKV: rows of one of Q/K/V viewed as (B*heads*S, 64)
+  int split_rows;     // EPI_F32: rows between split partials (M rounded up to 256)
+};
+
+template <typename T, int KIND>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
+    gemm_tc_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                        const __grid_constant__ OutMaps om, TcArgs g, EpiParams e) {
+  constexpr int BN = 256;
+  constexpr int HALF = 128;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sout = smem + kPairStages * kPairStageBytes;
+  uint64_t* full = reinterpret_cast<uint64_t*>(sout + kPairOutBytes);
+  uint64_t* empty = full + kPairStages;
+  uint64_t* tfull = empty + kPairStages;
+  uint64_t* tempty = tfull + 2;
+  uint32_t* tslot = reinterpret_cast<uint32_t*>(tempty + 2);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();
+  const bool leader = rank == 0;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kPairStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&tfull[a], 1);
+      mbar_init(&tempty[a], 2 * 32 * kPairEpiWarps);
+    }
+    fence_barrier_init();
+  }
+  if (warp == 1) tmem_alloc_pair(tslot, 2 * BN);
+  tc_fence_before();
+  cluster_sync();
+  tc_fence_after();
+  const uint32_t tmem = *tslot;
+  const int cid = blockIdx.x >> 1, ncl = gridDim.x >> 1;
+  const int total = g.tiles_m * g.tiles_n * g.splits;   // tiles_m counts 256-row pair tiles
+
+  if (warp == 0) {
+    if (lane == 0) {
+      prefetch_tensormap(&tmA);
+      prefetch_tensormap(&tmB);
+      int s = 0;
+      uint32_t ph = 0;
+      bool ok = true;
+      uint32_t issued_phase[kPairStages];
+      bool issued[kPairStages];
+      for (int i = 0; i < kPairStages; ++i) issued[i] = false;
+      for (int t = cid; t < total && ok; t += ncl) {
+        int mb, nb, sp;
+        decode_tile(g, t, mb, nb, sp);
+        const int kb0 = sp * g.kb_per_split;
+        const int kb1 = min(g.kblocks, kb0 + g.kb_per_split);
+        const int m0 = mb * 256 + (int)rank * HALF;
+        const int n0 = nb * BN + (int)rank * HALF;
+        for (int kb = kb0; kb < kb1; ++kb) {
+          if (!mbar_wait(&empty[s], ph ^ 1u, g.err, 41)) { ok = false; break; }
+          uint8_t* a_dst = smem + s * kPairStageBytes;
+          uint8_t* b_dst = a_dst + 128 * BK * 2;
+          const uint32_t fb = mapa_shared(smem_u32(&full[s]), 0);
+          if (leader) mbar_arrive_expect_tx(&full[s], 2 * kPairStageBytes);
+          const int k0 = kb * BK;
+          if (!g.a_mn) {
+            tma_load_2d_pair(a_dst, &tmA, fb, k0, m0);
+          } else {
+            tma_load_2d_pair(a_dst, &tmA, fb, m0, k0);
+            tma_load_2d_pair(a_dst + 8192, &tmA, fb, m0 + 64, k0);
+          }
+          if (!g.b_mn) {
+            tma_load_2d_pair(b_dst, &tmB, fb, k0, n0);
+          } else {
+            tma_load_2d_pair(b_dst, &tmB, fb, n0, k0);
+            tma_load_2d_pair(b_dst + 8192, &tmB, fb, n0 + 64, k0);
+          }
+          issued[s] = true;
+          issued_phase[s] = ph;
+          if (++s == kPairStages) { s = 0; ph ^= 1u; }
+        }
+      }
+      if (!ok && leader) {
+        for (int i = 0; i < kPairStages; ++i)
+          if (issued[i]) mbar_wait(&full[i], issued_phase[i], nullptr, 0);
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0 && leader) {
+      const uint32_t idesc = idesc_f16(256, BN, g.bf16 != 0, g.a_mn != 0, g.b_mn != 0);
+      int s = 0;
+      uint32_t ph = 0;
+      int acc = 0;
+      uint32_t aph = 0;
+      bool ok = true;
+      for (int t = cid; t < total && ok; t += ncl) {
+        int mb, nb, sp;
+        decode_tile(g, t, mb, nb, sp);
+        const int kb0 = sp * g.kb_per_split;
+        const int kb1 = min(g.kblocks, kb0 + g.kb_per_split);
+        if (!mbar_wait_cluster(&tempty[acc], aph ^ 1u, g.err, 42)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t d = tmem + acc * BN;
+        for (int kb = kb0; kb < kb1; ++kb) {
+          if (!mbar_wait(&full[s], ph, g.err, 43)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t a_base = smem_u32(smem + s * kPairStageBytes);
+          const uint32_t b_base = a_base + 128 * BK * 2;
+#pragma unroll
+          for (int k = 0; k < BK / 16; ++k) {
+            const uint64_t ad = g.a_mn ? smem_desc_sw128(a_base + k * 2048, 8192, 1024)
+                                       : smem_desc_sw128(a_base + k * 32, 16, 1024);
+            const uint64_t bd = g.b_mn ? smem_desc_sw128(b_base + k * 2048, 8192, 1024)
+                                       : smem_desc_sw128(b_base + k * 32, 16, 1024);
+            mma_f16_pair(d, ad, bd, idesc, (kb > kb0 || k > 0) ? 1u : 0u);
+          }
+          mma_commit_pair(&empty[s]);
+          if (++s == kPairStages) { s = 0; ph ^= 1u; }
+        }
+        if (!ok) break;
+        mma_commit_pair(&tfull[acc]);
+        acc ^= 1;
+        if (acc == 0) aph ^= 1u;
+      }
+    }
+  } else {
+    // Epilogue warps 2..17: warp w reads TMEM lanes 32*(w%4) .. +31 (rows of
+    // this CTA's half tile) and a quarter of the 256 columns.  Results go
+    // through a 64-byte-swizzled staging box (32 rows x 64 bytes) and leave by
+    // TMA store, so global writes are whole lines.
+    constexpr int CW = BN / (kPairEpiWarps / 4);              // 64 columns per warp
+    constexpr int OUT_ES = KIND == EPI_F32 ? 4 : 2;
+    constexpr int SW = 64 / OUT_ES;                          // columns per staging box: 32 (16-bit) or 16 (fp32)
+    constexpr int NOUT = KIND == EPI_BIAS_GELU ? 2 : 1;
+    const int quarter = warp & 3;
+    const int part = (warp - 2) >> 2;
+    uint8_t* stage0 = sout + (warp - 2) * 2 * kStageOut;
+    const uint32_t tempty_leader[2] = {mapa_shared(smem_u32(&tempty[0]), 0), mapa_shared(smem_u32(&tempty[1]), 0)};
+    const int swz = (lane >> 1) & 3;                         // 64-byte swizzle of this lane's staging row
+    int acc = 0;
+    uint32_t aph = 0;
+    int nbuf = 0;
+    for (int t = cid; t < total; t += ncl) {
+      int mb, nb, sp;
+      decode_tile(g, t, mb, nb, sp);
+      const int mrow0 = mb * 256 + (int)rank * HALF + quarter * 32;   // first row of this warp's boxes
+      const int m = mrow0 + lane;
+      const int nbase = nb * BN + part * CW;
+      const bool mrow = m < g.M;
+      uint4 pre[EpiAux<KIND>::kNeeds ? CW / 8 : 1];
+      if constexpr (EpiAux<KIND>::kNeeds) {
+        const T* ap = static_cast<const T*>(epi_aux_ptr(e, KIND));
+#pragma unroll
+        for (int j = 0; j < CW / 8; ++j) {
+          const int n = nbase + j * 8;
+          pre[j] = (ap && mrow && n < g.N) ? *reinterpret_cast<const uint4*>(ap + (size_t)m * e.ldo + n)
+                                            : make_uint4(0u, 0u, 0u, 0u);
+        }
+      }
+      if (!mbar_wait_warp(&tfull[acc], aph, g.err, 44)) break;
+      tc_fence_after();
+      const uint32_t tbase = tmem + ((uint32_t)(quarter * 32) << 16) + acc * BN + part * CW;
+#pragma unroll
+      for (int c0 = 0; c0 < CW; c0 += SW) {
+        float v[SW];
+        if constexpr (SW == 32) tmem_ld32(tbase + c0, *reinterpret_cast<float(*)[32]>(v));
+        else tmem_ld16(tbase + c0, *reinterpret_cast<float(*)[16]>(v));
+        if (c0 + SW == CW) {
+          // last TMEM read of this tile: hand the accumulator back to the leader
+          tc_fence_before();
+          mbar_arrive_cluster(tempty_leader[acc]);
+        }
+        uint8_t* sb0 = stage0 + (NOUT == 2 ? 0 : nbuf) * kStageOut;
+        uint8_t* sb1 = stage0 + kStageOut;
+        if (lane == 0) {
+          if constexpr (NOUT == 2) bulk_wait_read<0>();
+          else bulk_wait_read<1>();
+        }
+        __syncwarp();
+        if constexpr (OUT_ES == 4) {
+          // 16 floats = four 16-byte chunks of the 64-byte row
+#pragma unroll
+          for (int q = 0; q < 4; ++q)
+            *reinterpret_cast<float4*>(sb0 + lane * 64 + ((q ^ swz) << 4)) =
+                make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+        } else {
+#pragma unroll
+          for (int q = 0; q < SW / 8; ++q) {
+            const int n = nbase + c0 + q * 8;
+            float* vq = v + q * 8;
+            float v2[8];
+            float aux[8];
+            if constexpr (EpiAux<KIND>::kNeeds) unpack8<T>(pre[(c0 >> 3) + q], aux);
+            else {
+#pragma unroll
+              for (int i = 0; i < 8; ++i) aux[i] = 0.0f;
+            }
+            if (mrow && n < g.N) epi_compute8<T, KIND>(e, m, n, *reinterpret_cast<float(*)[8]>(vq), v2, aux);
+            store8<T>(reinterpret_cast<T*>(sb0 + lane * 64 + ((q ^ swz) << 4)), *reinterpret_cast<float(*)[8]>(vq));
+            if constexpr (NOUT == 2) store8<T>(reinterpret_cast<T*>(sb1 + lane * 64 + ((q ^ swz) << 4)), v2);
+          }
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          const int x = nbase + c0;
+          if constexpr (KIND == EPI_QKV) {
+            if (mrow0 < g.M && x < g.N) {
+              const int which = (x >= e.hidden) + (x >= 2 * e.hidden);
+              const int c = x - which * e.hidden;
+              const int bb = mrow0 / e.seq, s0 = mrow0 - bb * e.seq;
+              const int y = which * om.qkv_heads_rows + (bb * e.heads + (c >> 6)) * e.seq + s0;
+              tma_store_2d(&om.out, sb0, c & 63, y);
+            }
+          } else if constexpr (KIND == EPI_F32) {
+            if (mrow0 < g.M && x < g.N) tma_store_2d(&om.out, sb0, x, sp * om.split_rows + mrow0);
+          } else if (mrow0 < g.M && x < g.N) {
+            tma_store_2d(&om.out, sb0, x, mrow0);
+            if constexpr (NOUT == 2) {
+              if (e.out2) tma_store_2d(&om.out2, sb1, x, mrow0);
+            }
+          }
+          bulk_commit();
+        }
+        if constexpr (NOUT == 1) nbuf ^= 1;
+      }
+      acc ^= 1;
+      if (acc == 0) aph ^= 1u;
+    }
+    if (lane == 0) bulk_wait_all();
+    __syncwarp();
+  }
+  tc_fence_before();
+  cluster_sync();
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc_pair(tmem, 2 * BN);
+}
+
 __global__ void splitk_reduce_kernel(const float* __restrict__ part, int splits, size_t stride, size_t n4,
                                      float* __restrict__ out) {
   for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n4; i += (size_t)gridDim.x * blockDim.x) {
@@ -280,18 +541,24 @@ EncodeTiledFn encode_fn() {
 }
 
 // 2-D map over a row-major (outer, inner) matrix with row stride ld elements;
-// box = 64 inner elements (128 bytes, swizzled) x box_outer rows.
-bool make_map(CUtensorMap* m, const void* ptr, bool bf16, uint64_t inner, uint64_t outer, uint64_t ld,
-              uint32_t box_outer) {
+// box = box_bytes of the inner dimension (swizzled to match) x box_outer rows.
+bool make_map_t(CUtensorMap* m, const void* ptr, CUtensorMapDataType dt, int es_bytes, uint64_t inner, uint64_t outer,
+                uint64_t ld, uint32_t box_outer, int box_bytes = 128) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return false;
   cuuint64_t dims[2] = {inner, outer};
-  cuuint64_t strides[1] = {ld * 2};
-  cuuint32_t box[2] = {64, box_outer};
+  cuuint64_t strides[1] = {ld * (uint64_t)es_bytes};
+  cuuint32_t box[2] = {(cuuint32_t)(box_bytes / es_bytes), box_outer};
   cuuint32_t es[2] = {1, 1};
-  return fn(m, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<void*>(ptr),
-            dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+  return fn(m, dt, 2, const_cast<void*>(ptr), dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+            box_bytes == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+bool make_map(CUtensorMap* m, const void* ptr, bool bf16, uint64_t inner, uint64_t outer, uint64_t ld,
+              uint32_t box_outer) {
+  return make_map_t(m, ptr, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, inner, outer,
+                    ld, box_outer);
 }
 
 int num_sms() {
@@ -348,64 +615,139 @@ int launch_tc(const GemmDesc& gd, const EpiParams& e, int splits, cudaStream_t s
   return 0;
 }
 
-// Weight gradients (K = tokens) split K when the output has too few tiles
-// to occupy the SMs; each split writes a float32 partial tile.
-int splitk_count(int M, int N, int K) {
-  const int tiles = ((M + BM - 1) / BM) * ((N + 255) / 256);
-  const int kblocks = (K + BK - 1) / BK;
-  if (tiles >= (3 * num_sms()) / 4) return 1;
-  return std::max(1, std::min(std::min(4, kblocks / 8), num_sms() / tiles));
-}
-
 bool aligned16(const void* p, int ld) {
   return (reinterpret_cast<uintptr_t>(p) & 15) == 0 && ((size_t)ld * 2) % 16 == 0;
+}
+
+template <typename T, int KIND>
+int launch_tc_pair(const GemmDesc& gd, const EpiParams& e, int splits, cudaStream_t s) {
+  const bool bf16 = std::is_same<T, bf16_t>::value;
+  CUtensorMap ma, mb;
+  bool ok;
+  if (gd.a_kmajor) ok = make_map(&ma, gd.A, bf16, gd.K, gd.M, gd.lda, 128);
+  else ok = make_map(&ma, gd.A, bf16, gd.M, gd.K, gd.lda, 64);
+  if (ok) {
+    if (gd.b_kmajor) ok = make_map(&mb, gd.B, bf16, gd.K, gd.N, gd.ldb, 128);
+    else ok = make_map(&mb, gd.B, bf16, gd.N, gd.K, gd.ldb, 64);
+  }
+  if (!ok) return 1;
+  TcArgs g;
+  g.M = gd.M; g.N = gd.N; g.K = gd.K;
+  g.a_mn = gd.a_kmajor ? 0 : 1;
+  g.b_mn = gd.b_kmajor ? 0 : 1;
+  g.bf16 = bf16 ? 1 : 0;
+  g.tiles_m = (gd.M + 255) / 256;
+  g.tiles_n = (gd.N + 255) / 256;
+  g.kblocks = (gd.K + BK - 1) / BK;
+  g.kb_per_split = (g.kblocks + splits - 1) / splits;
+  g.splits = (g.kblocks + g.kb_per_split - 1) / g.kb_per_split;
+  g.split_stride = (size_t)gd.M * gd.N;
+  g.err = error_word();
+  OutMaps om;
+  std::memset(&om, 0, sizeof(om));
+  om.split_rows = g.tiles_m * 256;
+  g.split_stride = (size_t)om.split_rows * gd.N;
+  bool okm;
+  const CUtensorMapDataType t16 = bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+  if constexpr (KIND == EPI_F32) {
+    // split partials live in a workspace padded to whole 256-row tiles; the
+    // unsplit output is exactly M rows, so clipping keeps stores inside it
+    const uint64_t rows = g.splits > 1 ? (uint64_t)g.splits * om.split_rows : (uint64_t)gd.M;
+    okm = make_map_t(&om.out, e.out, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, gd.N, rows, e.ldo, 32, 64);
+  } else if constexpr (KIND == EPI_QKV) {
+    om.qkv_heads_rows = e.tokens * (e.hidden / 64);
+    okm = make_map_t(&om.out, e.out, t16, 2, 64, (uint64_t)3 * om.qkv_heads_rows, 64, 32, 64);
+  } else {
+    okm = make_map_t(&om.out, e.out, t16, 2, gd.N, gd.M, e.ldo, 32, 64);
+    if (okm && KIND == EPI_BIAS_GELU && e.out2) okm = make_map_t(&om.out2, e.out2, t16, 2, gd.N, gd.M, e.ldo, 32, 64);
+  }
+  if (!okm) return 1;
+  const int total = g.tiles_m * g.tiles_n * g.splits;
+  const int grid = 2 * std::min(total, num_sms() / 2);
+  static bool attr = false;
+  if (!attr) {
+    cudaFuncSetAttribute(gemm_tc_pair_kernel<T, KIND>, cudaFuncAttributeMaxDynamicSharedMemorySize, kPairSmem);
+    attr = true;
+  }
+  gemm_tc_pair_kernel<T, KIND><<<grid, kPairThreads, kPairSmem, s>>>(ma, mb, om, g, e);
+  count_launch();
+  return 0;
+}
+
+// Split count of a weight-gradient GEMM on CTA-pair tiles (256 x 256).
+int splitk_count_pair(int M, int N, int K) {
+  const int tiles = ((M + 255) / 256) * ((N + 255) / 256);
+  const int kblocks = (K + BK - 1) / BK;
+  const int clusters = num_sms() / 2;
+  if (tiles >= (3 * clusters) / 4) return 1;
+  return std::max(1, std::min(std::min(4, kblocks / 8), clusters / tiles));
 }
 
 template <typename T>
 int run_t(const GemmDesc& g, const EpiParams& e, cudaStream_t s) {
   if (!aligned16(g.A, g.lda) || !aligned16(g.B, g.ldb)) return 2;
-  // N <= 128 keeps the 128-wide tile; otherwise 256
-  const bool wide = g.N > 128;
   if (e.kind == EPI_F32) {
-    const int kblocks = (g.K + BK - 1) / BK;
-    int splits = g.splitk_ws ? splitk_count(g.M, g.N, g.K) : 1;
-    while (splits > 1 && (size_t)splits * g.M * g.N > g.splitk_ws_floats) --splits;
+    const size_t rows_pad = (size_t)((g.M + 255) / 256) * 256;
+    int splits = g.splitk_ws ? splitk_count_pair(g.M, g.N, g.K) : 1;
+    while (splits > 1 && (size_t)splits * rows_pad * g.N > g.splitk_ws_floats) --splits;
     if (splits > 1) {
       EpiParams ep = e;
       ep.out = g.splitk_ws;
-      int rc = launch_tc<T, 256, EPI_F32>(g, ep, splits, s);
-      if (rc) return rc;
+      const int kblocks = (g.K + BK - 1) / BK;
       const int kb_per = (kblocks + splits - 1) / splits;
       const int real = (kblocks + kb_per - 1) / kb_per;
+      int rc = launch_tc_pair<T, EPI_F32>(g, ep, splits, s);
+      if (rc) return rc;
       const size_t n4 = (size_t)g.M * g.N / 4;
       splitk_reduce_kernel<<<(int)std::min<size_t>((n4 + 255) / 256, 148 * 8), 256, 0, s>>>(
-          g.splitk_ws, real, (size_t)g.M * g.N, n4, static_cast<float*>(e.out));
+          g.splitk_ws, real, rows_pad * g.N, n4, static_cast<float*>(e.out));
       count_launch();
       return 0;
     }
-    return launch_tc<T, 256, EPI_F32>(g, e, 1, s);
+    return launch_tc_pair<T, EPI_F32>(g, e, 1, s);
   }
   switch (e.kind) {
-    case EPI_QKV: return wide ? launch_tc<T, 256, EPI_QKV>(g, e, 1, s) : launch_tc<T, 128, EPI_QKV>(g, e, 1, s);
-    case EPI_BIAS_DROP_RES:
-      return wide ? launch_tc<T, 256, EPI_BIAS_DROP_RES>(g, e, 1, s) : launch_tc<T, 128, EPI_BIAS_DROP_RES>(g, e, 1, s);
-    case EPI_BIAS_GELU:
-      return wide ? launch_tc<T, 256, EPI_BIAS_GELU>(g, e, 1, s) : launch_tc<T, 128, EPI_BIAS_GELU>(g, e, 1, s);
-    case EPI_DGELU: return wide ? launch_tc<T, 256, EPI_DGELU>(g, e, 1, s) : launch_tc<T, 128, EPI_DGELU>(g, e, 1, s);
-    case EPI_STORE: return wide ? launch_tc<T, 256, EPI_STORE>(g, e, 1, s) : launch_tc<T, 128, EPI_STORE>(g, e, 1, s);
+    case EPI_QKV:
+      // the staged head-split store needs whole 64-wide heads and 32-row boxes inside one sequence
+      if (e.head_dim == 64 && e.seq % 32 == 0 && e.hidden % 64 == 0) return launch_tc_pair<T, EPI_QKV>(g, e, 1, s);
+      return g.N > 128 ? launch_tc<T, 256, EPI_QKV>(g, e, 1, s) : launch_tc<T, 128, EPI_QKV>(g, e, 1, s);
+    case EPI_BIAS_DROP_RES: return launch_tc_pair<T, EPI_BIAS_DROP_RES>(g, e, 1, s);
+    case EPI_BIAS_GELU: return launch_tc_pair<T, EPI_BIAS_GELU>(g, e, 1, s);
+    case EPI_DGELU: return launch_tc_pair<T, EPI_DGELU>(g, e, 1, s);
+    case EPI_STORE: return launch_tc_pair<T, EPI_STORE>(g, e, 1, s);
+  }
+  return 1;
+}
+
+template <typename T>
+int run_pair_t(const GemmDesc& g, const EpiParams& e, int splits, cudaStream_t s) {
+  if (!aligned16(g.A, g.lda) || !aligned16(g.B, g.ldb)) return 2;
+  switch (e.kind) {
+    case EPI_QKV: return launch_tc_pair<T, EPI_QKV>(g, e, 1, s);
+    case EPI_BIAS_DROP_RES: return launch_tc_pair<T, EPI_BIAS_DROP_RES>(g, e, 1, s);
+    case EPI_BIAS_GELU: return launch_tc_pair<T, EPI_BIAS_GELU>(g, e, 1, s);
+    case EPI_DGELU: return launch_tc_pair<T, EPI_DGELU>(g, e, 1, s);
+    case EPI_STORE: return launch_tc_pair<T, EPI_STORE>(g, e, 1, s);
+    case EPI_F32: return launch_tc_pair<T, EPI_F32>(g, e, splits, s);
   }
   return 1;
 }
 
 }  // namespace
 
+// The CTA-pair GEMM directly (splits > 1 only for EPI_F32, writing split
+// partials to e.out as laid out for splitk_reduce).
+int gemm_tc_pair_run(int dtype, const GemmDesc& g, const EpiParams& e, int splits, cudaStream_t s) {
+  return dtype == DT_F16 ? run_pair_t<half_t>(g, e, splits, s) : run_pair_t<bf16_t>(g, e, splits, s);
+}
+
 int gemm_tc_run(int dtype, const GemmDesc& g, const EpiParams& e, cudaStream_t s) {
   return dtype == DT_F16 ? run_t<half_t>(g, e, s) : run_t<bf16_t>(g, e, s);
 }
 
 size_t gemm_tc_splitk_ws_floats(int M, int N, int K) {
-  const int sp = splitk_count(M, N, K);
-  return sp > 1 ? (size_t)sp * M * N : 0;
+  const int sp = splitk_count_pair(M, N, K);
+  return sp > 1 ? (size_t)sp * ((M + 255) / 256) * 256 * N : 0;
 }
 
 // Reads and clears the bounded-wait error word of the tensor-core kernels.
