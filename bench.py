@@ -9,8 +9,9 @@ layer_backward of one layer over one batch, inputs resident in HBM.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
-For N > 1 it runs under torchrun, one rank per GPU, each rank an independent
-replica on its own batch (weak scaling); the time is the max over ranks.
+For N > 1 it runs under torchrun, one rank per GPU, each rank a data-parallel
+replica on its own batch (weak scaling) whose step ends with one NCCL
+all-reduce of the float32 gradients; the time is the max over ranks.
 Rank 0 prints one JSON line.  `--impl reference` times the float64 oracle
 (the reference arm) on the host cores instead.
 """
@@ -239,10 +240,41 @@ def workload_config(w) -> dict:
     return {"workload": w.name, "batch": w.batch, "seq": w.seq, "hidden": w.hidden, "heads": w.heads,
             "ffn": w.ffn, "attn_dropout": w.attn_dropout, "hidden_dropout": w.hidden_dropout,
             "layer_norm": "pre" if w.pre_layer_norm else "post", "padding": w.lengths is not None,
-            "l2": "flushed (256 MiB write) between timed steps", "parallelism": "replicas"}
+            "l2": "flushed (256 MiB write) between timed steps", "parallelism": "data-parallel replicas"}
 
 
 # ---------------------------------------------------------------- GPU arm
+class StepRunner:
+    """One forward + backward of the layer on fixed device buffers, replayed
+    as a captured CUDA graph of the library's launches (or eagerly)."""
+
+    def __init__(self, layer, x, mask, wt, dy, y, dx, grads, use_graph: bool):
+        self.layer, self.x, self.mask, self.wt, self.dy = layer, x, mask, wt, dy
+        self.y, self.dx, self.grads = y, dx, grads
+        self.graph = None
+        if use_graph:
+            side = torch.cuda.Stream()
+            side.wait_stream(torch.cuda.current_stream())
+            with torch.cuda.stream(side):
+                self.eager()
+            torch.cuda.current_stream().wait_stream(side)
+            torch.cuda.synchronize()
+            self.graph = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(self.graph):
+                self.eager()
+            torch.cuda.synchronize()
+
+    def eager(self):
+        self.layer.forward(self.x, self.mask, self.wt, y=self.y)
+        self.layer.backward(self.x, self.dy, self.wt, grads=self.grads, dx=self.dx)
+
+    def __call__(self):
+        if self.graph is not None:
+            self.graph.replay()
+        else:
+            self.eager()
+
+
 def run_ours(args) -> None:
     import transformer_layer_pre_b200 as tlp
     from transformer_layer_pre_b200 import Layer, WEIGHT_NAMES
@@ -261,47 +293,59 @@ def run_ours(args) -> None:
     layer = Layer(w.batch, w.seq, w.hidden, w.heads, w.ffn, w.attn_dropout, w.hidden_dropout, w.pre_layer_norm,
                   w.seed, dtype=dt, gelu_checkpoint=w.gelu_checkpoint)
     wt = {n: inp.weights[0][n].to(dev) for n in WEIGHT_NAMES}
-    x = inp.x.to(dev)
-    dy = inp.dy.to(dev)
     mask = None if inp.mask is None else inp.mask.to(dev)
-    y = torch.empty_like(x)
-    dx = torch.empty_like(x)
-    grads = {n: torch.empty(tuple(wt[n].shape), dtype=torch.float32, device=dev) for n in WEIGHT_NAMES}
+    # gradients are views of one flat buffer: data-parallel ranks average it with one all-reduce
+    from transformer_layer_pre_b200.dp import FlatGrads, allreduce_mean
+    flat = FlatGrads(w.hidden, w.ffn, dev)
+    grads = flat.as_dict()
+
+    def exchange():
+        if world > 1:
+            allreduce_mean(flat)
+    # two buffer sets, so the end-to-end run can overlap one step's copies with the other's compute
+    xs = [inp.x.to(dev) for _ in range(2)]
+    dys = [inp.dy.to(dev) for _ in range(2)]
+    ys = [torch.empty_like(xs[0]) for _ in range(2)]
+    dxs = [torch.empty_like(xs[0]) for _ in range(2)]
     flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
     stream = torch.cuda.current_stream()
 
-    def step():
-        layer.forward(x, mask, wt, y=y)
-        layer.backward(x, dy, wt, grads=grads, dx=dx)
-
-    for _ in range(max(3, args.warmup)):
-        step()
-    tlp.device_check()
-
-    # ---- timed region: per-step events, L2 flushed between steps (outside the events)
-    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
-    barrier()
+    # launches per step, counted on one eager step
+    l0 = tlp.launch_count()
+    layer.forward(xs[0], mask, wt, y=ys[0])
+    layer.backward(xs[0], dys[0], wt, grads=grads, dx=dxs[0])
+    launches_per_step = tlp.launch_count() - l0
     torch.cuda.synchronize()
-    launches0 = tlp.launch_count()
+    runners = [StepRunner(layer, xs[i], mask, wt, dys[i], ys[i], dxs[i], grads, not args.no_graph) for i in range(2)]
+
     with ClockSampler(local) as clk:
+        for _ in range(args.warmup):
+            runners[0]()
+            exchange()
+        tlp.device_check()
+        # ---- timed region: per-step events, L2 flushed between steps (outside the events)
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+        barrier()
+        torch.cuda.synchronize()
         for a, b in evs:
             flush.zero_()
             a.record(stream)
-            step()
+            runners[0]()
+            exchange()
             b.record(stream)
         torch.cuda.synchronize()
-    barrier()
-    launches = tlp.launch_count() - launches0
+        barrier()
     step_ms = [a.elapsed_time(b) for a, b in evs]
     ms = reduce_max(sum(step_ms) / len(step_ms))
     tlp.device_check()
     value = world * T / (ms / 1e3)
+    launches = launches_per_step * args.steps
 
-    # ---- kernel-class breakdown (same steps, library event profiler on)
+    # ---- kernel-class breakdown (same steps, eager, library event profiler on)
     tlp.profile_enable(True)
     for _ in range(args.steps):
         flush.zero_()
-        step()
+        runners[0].eager()
     prof = tlp.profile_read()
     tlp.profile_enable(False)
     peaks = load_peaks()
@@ -326,33 +370,55 @@ def run_ours(args) -> None:
             bound, peak, src = "alu", alu_peak_tflops(mhz), f"148 SMs x 128 FP32 lanes x 2 x {mhz:.0f} MHz"
     else:
         bound, peak, src = "hbm", peaks["hbm_gbs"], f"{peaks['source']} copy bandwidth"
-    groups = d["launch_groups_per_step"]
     roofline = {"bound": bound, "kernel": dom, "achieved": d["achieved"], "peak": peak, "unit": d["unit"],
                 "frac": d["achieved"] / peak, "traffic": None, "peak_source": src,
-                "launches_per_step": groups}
+                "launches_per_step": d["launch_groups_per_step"]}
     step_flops = (linear_flops_per_token(w.hidden, w.ffn) + attn_flops_per_token(w.seq, w.hidden)) * T
     tensor_frac = (step_flops / (ms / 1e3)) / (peaks["tflops_sustained"] * 1e12)
 
-    # ---- end to end through the public API, host buffers (pinned), copies inside the timed region
-    hx = inp.x.pin_memory()
-    hdy = inp.dy.pin_memory()
-    hy = torch.empty(x.shape, dtype=dt).pin_memory()
-    hdx = torch.empty(x.shape, dtype=dt).pin_memory()
-    e2e_ms = []
-    for i in range(args.warmup + args.steps):
-        flush.zero_()
-        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        a.record(stream)
-        x.copy_(hx, non_blocking=True)
-        dy.copy_(hdy, non_blocking=True)
-        step()
-        hy.copy_(y, non_blocking=True)
-        hdx.copy_(dx, non_blocking=True)
-        b.record(stream)
-        b.synchronize()
-        if i >= args.warmup:
-            e2e_ms.append(a.elapsed_time(b))
-    e2e = reduce_max(sum(e2e_ms) / len(e2e_ms))
+    # ---- end to end through the public API: every step copies its inputs in
+    # from pinned host memory and its results (y, dx) back; copies run on
+    # their own streams so step i+1's input copy and step i-1's output copy
+    # overlap step i's compute (double-buffered device tensors)
+    hx, hdy = inp.x.pin_memory(), inp.dy.pin_memory()
+    hys = [torch.empty(xs[0].shape, dtype=dt).pin_memory() for _ in range(2)]
+    hdxs = [torch.empty(xs[0].shape, dtype=dt).pin_memory() for _ in range(2)]
+    s_in, s_out = torch.cuda.Stream(), torch.cuda.Stream()
+    done = [torch.cuda.Event() for _ in range(2)]
+    outd = [torch.cuda.Event() for _ in range(2)]
+    for e_ in done + outd:
+        e_.record(stream)
+    torch.cuda.synchronize()
+
+    def e2e_run(nsteps: int) -> float:
+        t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        t0.record(s_in)
+        for i in range(nsteps):
+            bsel = i & 1
+            ready = torch.cuda.Event()
+            with torch.cuda.stream(s_in):
+                s_in.wait_event(done[bsel])     # compute of step i-2 is done with this buffer set
+                xs[bsel].copy_(hx, non_blocking=True)
+                dys[bsel].copy_(hdy, non_blocking=True)
+                ready.record(s_in)
+            stream.wait_event(ready)
+            stream.wait_event(outd[bsel])       # results of step i-2 have left this buffer set
+            runners[bsel]()
+            exchange()
+            done[bsel].record(stream)
+            with torch.cuda.stream(s_out):
+                s_out.wait_event(done[bsel])
+                hys[bsel].copy_(ys[bsel], non_blocking=True)
+                hdxs[bsel].copy_(dxs[bsel], non_blocking=True)
+                outd[bsel].record(s_out)
+        s_in.wait_stream(s_out)
+        s_in.wait_stream(stream)
+        t1.record(s_in)
+        torch.cuda.synchronize()
+        return t0.elapsed_time(t1)
+
+    e2e_run(args.warmup)
+    e2e = reduce_max(e2e_run(args.steps) / args.steps)
     io = T * w.hidden * elem
 
     cpu = None
@@ -363,13 +429,15 @@ def run_ours(args) -> None:
             "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": w.dtype, "data": "synthetic (seeded N(0,0.02) weights, N(0,1) x and dY)",
-            "config": workload_config(w), "tensor_peak_frac": tensor_frac,
+            "config": dict(workload_config(w), graph=not args.no_graph), "tensor_peak_frac": tensor_frac,
             "roofline": roofline, "kernel_classes": classes, "cpu_baseline": cpu,
             "e2e": {"value": world * T / (e2e / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": 2 * io,
-                    "d2h_bytes_per_step": 2 * io},
-            "gpu_launches": launches, "clocks": clocks,
+                    "d2h_bytes_per_step": 2 * io, "ms_per_step": e2e,
+                    "note": "pinned host x, dY in and y, dx out every step; copies overlap neighbouring steps"},
+            "gpu_launches": launches, "launches_per_step": launches_per_step, "clocks": clocks,
         }
         print(json.dumps(line), flush=True)
+    del runners
     layer.close()
     if world > 1:
         import torch.distributed as dist
@@ -392,6 +460,7 @@ def main() -> None:
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
     ap.add_argument("--workload", default=WORKLOAD, choices=sorted(WORKLOADS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-graph", action="store_true", help="launch every kernel eagerly instead of replaying a CUDA graph")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

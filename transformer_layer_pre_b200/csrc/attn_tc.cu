@@ -642,6 +642,351 @@ __global__ void __launch_bounds__(kBwdThreads)
   if (warp == 1) tmem_dealloc(tmem, 512);
 }
 
+// ============================================================================ forward, S <= 128 (persistent)
+// One CTA per SM walks (sequence, head) items; every item is one 128-query x
+// 128-key tile.  Q/K/V, the score accumulator S and the output accumulator O
+// are double-buffered by item parity, so item i+1's loads and Q K^T overlap
+// item i's softmax, and item i's output is written while item i+1's softmax
+// runs.  Warps: 0 TMA, 1 MMA, 2-9 softmax: warp w owns TMEM lanes 32*(w%4)
+// (one query row per thread) and key columns 64*((w-2)/4) .. +63; the two
+// threads of a row combine their maxima and sums through shared memory.
+constexpr int kPFwdThreads = 320;
+constexpr int kPFwdSmem = 10 * TB + 4096 + 1024 + 256;   // Q,K,V x2, P pair x2, row exchange
+
+template <typename T>
+__global__ void __launch_bounds__(kPFwdThreads, 1)
+    attn_fwd_tc_persist(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
+                        const __grid_constant__ CUtensorMap tv, AttnTc a) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* sm = align1024(smem_raw);
+  // per slot j: Q at j*3TB, K at +TB, V at +2TB; P pairs after the six tiles
+  uint8_t* sP0 = sm + 6 * TB;
+  // row exchange: [max | sum][2 slots][2 halves][128 rows] floats
+  float* xch = reinterpret_cast<float*>(sm + 10 * TB);
+  uint64_t* bar = reinterpret_cast<uint64_t*>(sm + 10 * TB + 4096);
+  uint64_t *in_full = bar, *in_empty = bar + 2, *s_full = bar + 4, *p_full = bar + 6, *o_full = bar + 8,
+           *o_free = bar + 10;
+  uint32_t* tslot = reinterpret_cast<uint32_t*>(bar + 12);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int S = a.S;
+  const int nitems = a.B * a.nh;
+  if (threadIdx.x == 0) {
+    for (int j = 0; j < 2; ++j) {
+      mbar_init(&in_full[j], 1);
+      mbar_init(&in_empty[j], 1);
+      mbar_init(&s_full[j], 1);
+      mbar_init(&p_full[j], 256);
+      mbar_init(&o_full[j], 1);
+      mbar_init(&o_free[j], 256);
+    }
+    fence_barrier_init();
+  }
+  if (warp == 1) tmem_alloc(tslot, 512);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tslot;   // S[j] at 128*j, O[j] at 256 + 64*j
+
+  if (warp == 0) {
+    if (lane == 0) {
+      int n = 0;
+      for (int it = blockIdx.x; it < nitems; it += gridDim.x, ++n) {
+        const int j = n & 1;
+        if (!mbar_wait(&in_empty[j], ((n >> 1) & 1) ^ 1, a.err, 51)) break;
+        uint8_t* base = sm + j * 3 * TB;
+        mbar_arrive_expect_tx(&in_full[j], 3 * TB);
+        const int row0 = it * S;
+        tma_load_2d(base, &tq, &in_full[j], 0, row0);
+        tma_load_2d(base + TB, &tk, &in_full[j], 0, row0);
+        tma_load_2d(base + 2 * TB, &tv, &in_full[j], 0, row0);
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      const uint32_t id_s = idesc_f16(128, 128, a.bf16 != 0, false, false);
+      const uint32_t id_o = idesc_f16(128, 64, a.bf16 != 0, false, true);
+      // S = Q K^T of item n into S[n&1]
+      auto mma_s = [&](int n) -> bool {
+        const int j = n & 1;
+        if (!mbar_wait(&in_full[j], (n >> 1) & 1, a.err, 52)) return false;
+        // S[j] is free once the softmax of item n-2 wrote its P (it read S first)
+        if (!mbar_wait(&p_full[j], ((n >> 1) & 1) ^ 1, a.err, 53)) return false;
+        tc_fence_after();
+        const uint32_t aQ = smem_u32(sm + j * 3 * TB), aK = aQ + TB;
+#pragma unroll
+        for (int kk = 0; kk < HD / 16; ++kk) mma_f16(tmem + 128 * j, dk_tile(aQ, kk), dk_tile(aK, kk), id_s, kk > 0);
+        mma_commit(&s_full[j]);
+        return true;
+      };
+      int n = 0;
+      bool ok = true;
+      int my_items = 0;
+      for (int it = blockIdx.x; it < nitems; it += gridDim.x) ++my_items;
+      if (my_items > 0) ok = mma_s(0);
+      for (n = 0; n < my_items && ok; ++n) {
+        const int j = n & 1;
+        if (n + 1 < my_items && !(ok = mma_s(n + 1))) break;
+        if (!(ok = mbar_wait(&p_full[j], (n >> 1) & 1, a.err, 54))) break;
+        if (!(ok = mbar_wait(&o_free[j], ((n >> 1) & 1) ^ 1, a.err, 55))) break;
+        tc_fence_after();
+        const uint32_t aV = smem_u32(sm + j * 3 * TB) + 2 * TB;
+        const uint32_t aP = smem_u32(sP0 + j * 2 * TB);
+#pragma unroll
+        for (int kk = 0; kk < TILE / 16; ++kk)
+          mma_f16(tmem + 256 + 64 * j, dk_pair(aP, kk), dmn_tile(aV, kk), id_o, kk > 0);
+        mma_commit(&o_full[j]);
+        mma_commit(&in_empty[j]);
+      }
+    }
+  } else {
+    const int quarter = warp & 3;
+    const int hf = (warp - 2) >> 2;
+    const int r = quarter * 32 + lane;
+    const uint32_t lo = (uint32_t)(quarter * 32) << 16;
+    const float c2 = a.scale * kLog2e;
+    const float dsc = a.drop.thr ? a.drop.scale : 1.0f;
+    const int kc0 = hf * 64;
+    bool ok = true;
+    int n = 0;
+    int prev_item = -1;
+    float prev_inv = 0.0f;
+    // output of item n-1 (slot jp): O rows to ctx, one 32-column half per thread
+    auto epilogue = [&](int item, int np, float inv) -> bool {
+      const int jp = np & 1;
+      if (!mbar_wait_warp(&o_full[jp], (np >> 1) & 1, a.err, 56)) return false;
+      tc_fence_after();
+      float o[32];
+      tmem_ld32(tmem + 256 + 64 * jp + lo + hf * 32, o);
+      tc_fence_before();
+      mbar_arrive(&o_free[jp]);
+      const int b = item / a.nh, h = item - (item / a.nh) * a.nh;
+      if (r < S) {
+        T* dst = static_cast<T*>(a.ctx) + ((size_t)b * S + r) * a.H + h * HD + hf * 32;
+#pragma unroll
+        for (int c = 0; c < 32; c += 8) {
+          float w8[8];
+#pragma unroll
+          for (int t = 0; t < 8; ++t) w8[t] = o[c + t] * inv;
+          store8<T>(dst + c, w8);
+        }
+      }
+      return true;
+    };
+    for (int it = blockIdx.x; it < nitems && ok; it += gridDim.x, ++n) {
+      const int j = n & 1;
+      const int b = it / a.nh;
+      const uint64_t erow = ((uint64_t)it * S + (uint64_t)r) * (uint64_t)S;
+      if (!(ok = mbar_wait_warp(&s_full[j], (n >> 1) & 1, a.err, 57))) break;
+      tc_fence_after();
+      float sv[64];
+      tmem_ld32(tmem + 128 * j + lo + kc0, *reinterpret_cast<float(*)[32]>(sv));
+      tmem_ld32(tmem + 128 * j + lo + kc0 + 32, *reinterpret_cast<float(*)[32]>(sv + 32));
+      float mx = -INFINITY;
+#pragma unroll
+      for (int t = 0; t < 64; ++t) {
+        sv[t] = fmaf(sv[t], c2, mask_log2(a, b, kc0 + t));
+        mx = fmaxf(mx, sv[t]);
+      }
+      float* xm = xch + j * 256;
+      xm[hf * 128 + r] = mx;
+      named_barrier(1, 256);
+      mx = fmaxf(mx, xm[(1 - hf) * 128 + r]);
+      float lsum = 0.0f;
+#pragma unroll
+      for (int g = 0; g < 8; ++g) {
+        const int kb = kc0 + g * 8;
+        const uint32_t bits = a.drop.thr ? dropout_bits8(a.drop, 0, (erow + (uint64_t)kb) >> 3) : 0xFFu;
+        float pv[8];
+#pragma unroll
+        for (int t = 0; t < 8; ++t) {
+          const float x = sv[g * 8 + t];
+          const float p = (x == -INFINITY) ? 0.0f : exp2f(x - mx);
+          lsum += p;
+          pv[t] = ((bits >> t) & 1u) ? p * dsc : 0.0f;
+        }
+        pair_store8<T>(sP0 + j * 2 * TB, r, hf * 8 + g, pv);
+      }
+      // P is written and S has been read: both hand-overs ride on p_full
+      tc_fence_before();
+      fence_proxy_async_smem();
+      mbar_arrive(&p_full[j]);
+      // row sum across the two halves (second exchange buffer)
+      float* xs = xch + 512 + j * 256;
+      xs[hf * 128 + r] = lsum;
+      named_barrier(1, 256);
+      const float l = lsum + xs[(1 - hf) * 128 + r];
+      if (hf == 0 && r < S) a.lse[(size_t)it * S + r] = l > 0.0f ? (mx + log2f(l)) * kLn2 : INFINITY;
+      // the previous item's output overlaps this item's softmax
+      if (prev_item >= 0 && !(ok = epilogue(prev_item, n - 1, prev_inv))) break;
+      prev_item = it;
+      prev_inv = l > 0.0f ? 1.0f / l : 0.0f;
+    }
+    if (ok && prev_item >= 0) epilogue(prev_item, n - 1, prev_inv);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc(tmem, 512);
+}
+
+// ============================================================================ backward, S <= 128 (persistent)
+// One CTA per SM walks (sequence, head) items, each one 128 x 128 tile:
+// S = Q K^T and dPd = dO V^T, then Pd and dS to shared memory, then dV, dK and
+// dQ in TMEM and out to dQKV.  Q/K/V/dO are double-buffered by item parity so
+// the next item's loads overlap this item's work.  D = rowsum(dO * O) comes
+// from the shared-memory dO tile and the stored output O.
+constexpr int kPBwdSmem = 12 * TB + 1024 + 256;   // (Q,K,V,dO) x2, Pd pair, dS pair
+
+template <typename T>
+__global__ void __launch_bounds__(kBwdThreads, 1)
+    attn_bwd_tc_persist(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
+                        const __grid_constant__ CUtensorMap tv, const __grid_constant__ CUtensorMap tdo, AttnTc a) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* sm = align1024(smem_raw);
+  uint8_t* sPd = sm + 8 * TB;
+  uint8_t* sdS = sm + 10 * TB;
+  uint64_t* bar = reinterpret_cast<uint64_t*>(sm + 12 * TB);
+  uint64_t *in_full = bar, *in_empty = bar + 2, *s_full = bar + 4, *s_free = bar + 5, *ds_full = bar + 6,
+           *g_full = bar + 7, *g_free = bar + 8;
+  uint32_t* tslot = reinterpret_cast<uint32_t*>(bar + 9);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int S = a.S;
+  const int nitems = a.B * a.nh;
+  if (threadIdx.x == 0) {
+    for (int j = 0; j < 2; ++j) {
+      mbar_init(&in_full[j], 1);
+      mbar_init(&in_empty[j], 1);
+    }
+    mbar_init(s_full, 1);
+    mbar_init(s_free, kSoftThreads);
+    mbar_init(ds_full, kSoftThreads);
+    mbar_init(g_full, 1);
+    mbar_init(g_free, kSoftThreads);
+    fence_barrier_init();
+  }
+  if (warp == 1) tmem_alloc(tslot, 512);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tslot;
+  const uint32_t tS = tmem, tdP = tmem + 128, tdV = tmem + 256, tdK = tmem + 320, tdQ = tmem + 384;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      int n = 0;
+      for (int it = blockIdx.x; it < nitems; it += gridDim.x, ++n) {
+        const int j = n & 1;
+        if (!mbar_wait(&in_empty[j], ((n >> 1) & 1) ^ 1, a.err, 61)) break;
+        uint8_t* base = sm + j * 4 * TB;
+        const int b = it / a.nh, h = it - (it / a.nh) * a.nh;
+        mbar_arrive_expect_tx(&in_full[j], 4 * TB);
+        tma_load_2d(base, &tq, &in_full[j], 0, it * S);
+        tma_load_2d(base + TB, &tk, &in_full[j], 0, it * S);
+        tma_load_2d(base + 2 * TB, &tv, &in_full[j], 0, it * S);
+        tma_load_2d(base + 3 * TB, &tdo, &in_full[j], h * HD, b * S);
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      const bool bf = a.bf16 != 0;
+      const uint32_t id_kk = idesc_f16(128, 128, bf, false, false);
+      const uint32_t id_mm = idesc_f16(128, 64, bf, true, true);
+      const uint32_t id_km = idesc_f16(128, 64, bf, false, true);
+      const uint32_t aPd = smem_u32(sPd), adS = smem_u32(sdS);
+      int n = 0;
+      for (int it = blockIdx.x; it < nitems; it += gridDim.x, ++n) {
+        const int j = n & 1;
+        const uint32_t aQ = smem_u32(sm + j * 4 * TB), aK = aQ + TB, aV = aQ + 2 * TB, adO = aQ + 3 * TB;
+        if (!mbar_wait(&in_full[j], (n >> 1) & 1, a.err, 62)) break;
+        if (!mbar_wait(s_free, (n & 1) ^ 1, a.err, 63)) break;
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < HD / 16; ++kk) mma_f16(tS, dk_tile(aQ, kk), dk_tile(aK, kk), id_kk, kk > 0);
+#pragma unroll
+        for (int kk = 0; kk < HD / 16; ++kk) mma_f16(tdP, dk_tile(adO, kk), dk_tile(aV, kk), id_kk, kk > 0);
+        mma_commit(s_full);
+        if (!mbar_wait(ds_full, n & 1, a.err, 64)) break;
+        if (!mbar_wait(g_free, (n & 1) ^ 1, a.err, 65)) break;
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < TILE / 16; ++kk) mma_f16(tdV, dmn_pair(aPd, kk), dmn_tile(adO, kk), id_mm, kk > 0);
+#pragma unroll
+        for (int kk = 0; kk < TILE / 16; ++kk) mma_f16(tdK, dmn_pair(adS, kk), dmn_tile(aQ, kk), id_mm, kk > 0);
+#pragma unroll
+        for (int kk = 0; kk < TILE / 16; ++kk) mma_f16(tdQ, dk_pair(adS, kk), dmn_tile(aK, kk), id_km, kk > 0);
+        mma_commit(g_full);
+        mma_commit(&in_empty[j]);
+      }
+    }
+  } else {
+    const int quarter = warp & 3;
+    const int hf = (warp - 2) >> 2;
+    const int r = quarter * 32 + lane;
+    const uint32_t lo = (uint32_t)(quarter * 32) << 16;
+    int n = 0;
+    for (int it = blockIdx.x; it < nitems; it += gridDim.x, ++n) {
+      const int j = n & 1;
+      const int b = it / a.nh, h = it - (it / a.nh) * a.nh;
+      const bool qv = r < S;
+      const size_t trow = (size_t)b * S + r;
+      const float lse2 = qv ? a.lse[(size_t)it * S + r] * kLog2e : INFINITY;
+      if (!mbar_wait_warp(&in_full[j], (n >> 1) & 1, a.err, 66)) break;
+      // D = rowsum(dO * O): dO from the swizzled shared tile, O from global memory
+      float Di = 0.0f;
+      if (qv) {
+        const uint8_t* drow = sm + j * 4 * TB + 3 * TB + r * 128;
+        const T* orow = static_cast<const T*>(a.ctx_in) + trow * a.H + h * HD;
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+          float x[8], y[8];
+          load8<T>(reinterpret_cast<const T*>(drow + ((c ^ (r & 7)) << 4)), x);
+          load8<T>(orow + c * 8, y);
+#pragma unroll
+          for (int t = 0; t < 8; ++t) Di = fmaf(x[t], y[t], Di);
+        }
+      }
+      if (!mbar_wait_warp(s_full, n & 1, a.err, 67)) break;
+      tc_fence_after();
+      bwd_pair_rows<T>(a, b, it * S, r, r, 0, hf * 64, tS, tdP, lo, lse2, Di, sPd, sdS);
+      tc_fence_before();
+      mbar_arrive(s_free);
+      fence_proxy_async_smem();
+      mbar_arrive(ds_full);
+      if (!mbar_wait_warp(g_full, n & 1, a.err, 68)) break;
+      tc_fence_after();
+      float dq[32], dk[32], dv[32];
+      tmem_ld32(tdQ + lo + hf * 32, dq);
+      tmem_ld32(tdK + lo + hf * 32, dk);
+      tmem_ld32(tdV + lo + hf * 32, dv);
+      tc_fence_before();
+      mbar_arrive(g_free);
+      if (qv) {
+        // row r is query r for dQ and key r for dK, dV (both < S)
+        T* dst = static_cast<T*>(a.dqkv) + trow * 3 * a.H + h * HD + hf * 32;
+#pragma unroll
+        for (int c = 0; c < 32; c += 8) {
+          float q8[8], k8[8], v8[8];
+#pragma unroll
+          for (int t = 0; t < 8; ++t) {
+            q8[t] = dq[c + t] * a.scale;
+            k8[t] = dk[c + t] * a.scale;
+            v8[t] = dv[c + t];
+          }
+          store8<T>(dst + c, q8);
+          store8<T>(dst + a.H + c, k8);
+          store8<T>(dst + 2 * a.H + c, v8);
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc(tmem, 512);
+}
+
 // ------------------------------------------------------------------ host side
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
@@ -707,10 +1052,18 @@ void fwd_t(const AttnArgs& a, cudaStream_t s) {
   static bool attr = false;
   if (!attr) {
     cudaFuncSetAttribute(attn_fwd_tc<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, kFwdSmem);
+    cudaFuncSetAttribute(attn_fwd_tc_persist<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, kPFwdSmem);
     attr = true;
   }
-  dim3 grid((a.S + TILE - 1) / TILE, a.nh, a.B);
-  attn_fwd_tc<T><<<grid, kFwdThreads, kFwdSmem, s>>>(mq, mk, mv, t);
+  if (a.S <= TILE) {
+    int nsm = 148;
+    cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, 0);
+    const int grid = std::min(a.B * a.nh, nsm);
+    attn_fwd_tc_persist<T><<<grid, kPFwdThreads, kPFwdSmem, s>>>(mq, mk, mv, t);
+  } else {
+    dim3 grid((a.S + TILE - 1) / TILE, a.nh, a.B);
+    attn_fwd_tc<T><<<grid, kFwdThreads, kFwdSmem, s>>>(mq, mk, mv, t);
+  }
   count_launch();
 }
 
@@ -724,17 +1077,23 @@ void bwd_t(const AttnArgs& a, cudaStream_t s) {
       !map_tile(&mv, a.v, t.bf16, HD, rows, HD) || !map_tile(&mdo, a.dctx, t.bf16, t.H, tokens, t.H))
     return;
   const int ntile = (a.S + TILE - 1) / TILE;
-  if (ntile > 1) {
-    dvec_launch(t.bf16 ? DT_BF16 : DT_F16, a, s);
-    t.dvec = a.dvec;
-  }
-  t.fuse_dq = ntile == 1;
   static bool attr = false;
   if (!attr) {
     cudaFuncSetAttribute(attn_bwd_kv_tc<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, kBwdKvSmem);
     cudaFuncSetAttribute(attn_bwd_q_tc<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, kBwdQSmem);
+    cudaFuncSetAttribute(attn_bwd_tc_persist<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, kPBwdSmem);
     attr = true;
   }
+  if (ntile == 1) {
+    int nsm = 148;
+    cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, 0);
+    attn_bwd_tc_persist<T><<<std::min(a.B * a.nh, nsm), kBwdThreads, kPBwdSmem, s>>>(mq, mk, mv, mdo, t);
+    count_launch();
+    return;
+  }
+  dvec_launch(t.bf16 ? DT_BF16 : DT_F16, a, s);
+  t.dvec = a.dvec;
+  t.fuse_dq = 0;
   dim3 grid(ntile, a.nh, a.B);
   attn_bwd_kv_tc<T><<<grid, kBwdThreads, kBwdKvSmem, s>>>(mq, mk, mv, mdo, t);
   count_launch();
