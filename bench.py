@@ -19,8 +19,10 @@ from __future__ import annotations
 
 import argparse
 import datetime
+import hashlib
 import json
 import os
+import re
 import statistics
 import subprocess
 import sys
@@ -73,6 +75,33 @@ def class_work(cls: str, w, tokens: int, elem: int) -> tuple[float, str]:
         return 2 * (4 * th) + th, "byte"
     # dropout backward of dY (read, write) + bias-gradient column sums of dU and dQKV
     return 2 * th + tokens * f * elem + 3 * th, "byte"
+
+
+GEMM_PROFILE = os.path.join(ROOT, "profiles", "gemm_tc_pair_bert-large-f16.txt")
+GEMM_SOURCES = ("gemm_tc.cu", "epilogue.cuh", "sm100.cuh", "common.cuh", "kernels.h")
+
+
+def gemm_sources_digest() -> str:
+    h = hashlib.sha256()
+    for n in GEMM_SOURCES:
+        with open(os.path.join(ROOT, "transformer_layer_pre_b200", "csrc", n), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()
+
+
+def recorded_gemm_traffic(workload: str) -> float | None:
+    """DRAM bytes (read + write) per GEMM launch from the committed ncu summary
+    of this workload, or None when there is none or the GEMM kernel sources
+    have changed since it was captured."""
+    if workload != WORKLOAD or not os.path.exists(GEMM_PROFILE):
+        return None
+    with open(GEMM_PROFILE) as fh:
+        text = fh.read()
+    t = re.search(r"^TRAFFIC_BYTES_PER_LAUNCH (\d+)", text, re.M)
+    d = re.search(r"^KERNEL_SOURCES_SHA256 ([0-9a-f]{64})", text, re.M)
+    if not (t and d) or d.group(1) != gemm_sources_digest():
+        return None
+    return float(t.group(1))
 
 
 def load_peaks() -> dict:
@@ -371,7 +400,10 @@ def run_ours(args) -> None:
     else:
         bound, peak, src = "hbm", peaks["hbm_gbs"], f"{peaks['source']} copy bandwidth"
     roofline = {"bound": bound, "kernel": dom, "achieved": d["achieved"], "peak": peak, "unit": d["unit"],
-                "frac": d["achieved"] / peak, "traffic": None, "peak_source": src,
+                "frac": d["achieved"] / peak,
+                "traffic": recorded_gemm_traffic(args.workload) if dom == "gemm" else None,
+                "traffic_source": "ncu dram__bytes_read.sum + dram__bytes_write.sum, mean over one step's GEMM "
+                                  "launches (profiles/gemm_tc_pair_bert-large-f16.txt)", "peak_source": src,
                 "launches_per_step": d["launch_groups_per_step"]}
     step_flops = (linear_flops_per_token(w.hidden, w.ffn) + attn_flops_per_token(w.seq, w.hidden)) * T
     tensor_frac = (step_flops / (ms / 1e3)) / (peaks["tflops_sustained"] * 1e12)
