@@ -149,8 +149,8 @@ tl_status tl_dropout_keep_mask(uint64_t seed, uint64_t philox_offset, int site, 
 
 /* Test hook: g[i] = GELU(u[i]) and dg[i] = GELU'(u[i]) for i < n (float32
  * device buffers), evaluated by the same device code the layer's GEMM
- * epilogues use (erf form, CUDA's erff; the density term uses the fast
- * exponential). */
+ * epilogues use: erf form, Phi(u) from the normal-tail approximation of
+ * Abramowitz & Stegun 26.2.17 (absolute error below 7.5e-8) in float32. */
 tl_status tl_gelu_eval(const float* u, float* g, float* dg, uint64_t n, void* stream);
 
 /* Waits for all work on the current device, then reports TL_ECUDA if a CUDA
@@ -189,6 +189,26 @@ long long tl_launch_count(void);
  * caller.  Enqueued on `stream` (a cudaStream_t); returns before the GPU
  * finishes.  TL_ECUDA if a CUDA call fails. */
 tl_status tl_bias_grad_noalloc(int dtype, const void* dz, int rows, int cols, float* db, void* stream);
+
+/* Progressive Layer Dropping for a stack of layers ("Progressive Layer
+ * Dropping" page, schedule section).  Host functions; no device work.
+ *
+ * tl_pld_theta: the keep level at global step `step`,
+ *   theta(t) = (1 - theta_bar) * exp(-gamma * t) + theta_bar,
+ * which is 1 at t = 0 and tends to theta_bar.
+ * tl_pld_keep_prob: probability that layer `layer` (0-based) of
+ * `num_layers` runs at keep level theta: 1 - (layer+1)/num_layers * (1-theta)
+ * (the depth profile is linear; the last layer is kept with probability
+ * theta).  -1 for a layer index outside [0, num_layers).
+ * tl_pld_keep: 1 if the layer runs at this step, 0 if it is skipped (the
+ * identity in forward and backward), -1 for a bad layer index.  Decided by
+ * Philox4x32-10 with counter (step mod 2^32, step div 2^32, 3, layer) and key
+ * (seed mod 2^32, seed div 2^32): kept when output word 0 < floor(p * 2^32),
+ * p the keep probability (always kept when p >= 1, never when p <= 0).
+ * Equal seeds and steps give equal decisions on every rank. */
+double tl_pld_theta(double theta_bar, double gamma, uint64_t step);
+double tl_pld_keep_prob(int layer, int num_layers, double theta);
+int tl_pld_keep(uint64_t seed, uint64_t step, int layer, int num_layers, double theta);
 
 const char* tl_status_string(tl_status s);
 

@@ -155,9 +155,79 @@ __device__ __forceinline__ uint32_t dropout_bits8(const DropoutParams& dp, int s
 }
 
 // ------------------------------------------------------------------ GELU (erf form)
-__device__ __forceinline__ float gelu_f(float u) { return 0.5f * u * (1.0f + erff(u * 0.70710678118654752f)); }
-__device__ __forceinline__ float gelu_grad_f(float u) {
-  return fmaf(u * 0.39894228040143268f, __expf(-0.5f * u * u), 0.5f * (1.0f + erff(u * 0.70710678118654752f)));
+// GELU(u) = u * Phi(u), Phi the standard normal distribution function.  Phi
+// comes from the normal upper-tail approximation of Abramowitz & Stegun,
+// "Handbook of Mathematical Functions", formula 26.2.17 (after Hastings):
+// for z >= 0
+//   Q(z) = 1 - Phi(z) = phi(z) (b1 t + b2 t^2 + b3 t^3 + b4 t^4 + b5 t^5) + e(z),
+//   t = 1 / (1 + p z),   |e(z)| < 7.5e-8,
+// phi the normal density; Phi(u) = 1 - Q(u) for u >= 0, Q(-u) otherwise, and
+// GELU'(u) = Phi(u) + u phi(u).  Lanes are evaluated in pairs with the packed
+// float32 FMA/multiply of sm_100, plus one reciprocal and one base-2
+// exponential per element on the special-function unit.  Every step is an
+// explicit single-rounded operation (nothing left to FMA contraction), so
+// each kernel that evaluates GELU gets the same bits for the same input.
+__device__ __forceinline__ float rcp_approx(float x) {
+  float r;
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(x));
+  return r;
+}
+__device__ __forceinline__ float ex2_approx(float x) {
+  float r;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(x));
+  return r;
+}
+__device__ __forceinline__ float2 f2(float a) { return make_float2(a, a); }
+
+// phi(|u|) and Q(|u|) of a pair of lanes.
+__device__ __forceinline__ void normal_tail2(float2 u, float2& phi, float2& q) {
+  constexpr float kP = 0.2316419f;
+  constexpr float kB1 = 0.319381530f, kB2 = -0.356563782f, kB3 = 1.781477937f, kB4 = -1.821255978f,
+                  kB5 = 1.330274429f;
+  constexpr float kInvSqrt2Pi = 0.398942280401432678f;
+  constexpr float kNegHalfLog2e = -0.721347520444481703f;   // exp(-z^2/2) = 2^(z^2 * kNegHalfLog2e)
+  const float2 z = make_float2(fabsf(u.x), fabsf(u.y));
+  float2 t = __ffma2_rn(z, f2(kP), f2(1.0f));
+  t = make_float2(rcp_approx(t.x), rcp_approx(t.y));
+  float2 s = __ffma2_rn(t, f2(kB5), f2(kB4));
+  s = __ffma2_rn(t, s, f2(kB3));
+  s = __ffma2_rn(t, s, f2(kB2));
+  s = __ffma2_rn(t, s, f2(kB1));
+  s = __fmul2_rn(s, t);
+  const float2 a = __fmul2_rn(__fmul2_rn(z, f2(kNegHalfLog2e)), z);
+  phi = __fmul2_rn(make_float2(ex2_approx(a.x), ex2_approx(a.y)), f2(kInvSqrt2Pi));
+  q = __fmul2_rn(phi, s);
+}
+__device__ __forceinline__ float2 normal_cdf2(float2 u, float2 q) {
+  return make_float2(u.x >= 0.0f ? __fsub_rn(1.0f, q.x) : q.x, u.y >= 0.0f ? __fsub_rn(1.0f, q.y) : q.y);
+}
+__device__ __forceinline__ float2 gelu2(float2 u) {
+  float2 phi, q;
+  normal_tail2(u, phi, q);
+  return __fmul2_rn(u, normal_cdf2(u, q));
+}
+__device__ __forceinline__ float2 gelu_grad2(float2 u) {
+  float2 phi, q;
+  normal_tail2(u, phi, q);
+  return __ffma2_rn(u, phi, normal_cdf2(u, q));
+}
+// In-place over 8 lanes.
+__device__ __forceinline__ void gelu8(float (&v)[8]) {
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float2 g = gelu2(make_float2(v[2 * i], v[2 * i + 1]));
+    v[2 * i] = g.x;
+    v[2 * i + 1] = g.y;
+  }
+}
+// v *= GELU'(u) over 8 lanes.
+__device__ __forceinline__ void mul_gelu_grad8(float (&v)[8], const float (&u)[8]) {
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float2 d = __fmul2_rn(make_float2(v[2 * i], v[2 * i + 1]), gelu_grad2(make_float2(u[2 * i], u[2 * i + 1])));
+    v[2 * i] = d.x;
+    v[2 * i + 1] = d.y;
+  }
 }
 
 // ------------------------------------------------------------------ warp reductions

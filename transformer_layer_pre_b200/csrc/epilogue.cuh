@@ -81,13 +81,11 @@ __device__ __forceinline__ void epi_apply8(const EpiParams& e, int m, int n, flo
     for (int i = 0; i < 8; ++i) v[i] = round_f<T>(v[i] + b[i]);
     store8<T>(static_cast<T*>(e.out) + (size_t)m * e.ldo + n, v);
     if (e.out2) {
-#pragma unroll
-      for (int i = 0; i < 8; ++i) v[i] = gelu_f(v[i]);
+      gelu8(v);
       store8<T>(static_cast<T*>(e.out2) + (size_t)m * e.ldo + n, v);
     }
   } else if constexpr (KIND == EPI_DGELU) {
-#pragma unroll
-    for (int i = 0; i < 8; ++i) v[i] *= gelu_grad_f(aux[i]);
+    mul_gelu_grad8(v, aux);
     store8<T>(static_cast<T*>(e.out) + (size_t)m * e.ldo + n, v);
   }
 }
@@ -122,11 +120,11 @@ __device__ __forceinline__ void epi_compute8(const EpiParams& e, int m, int n, f
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
       v[i] = round_f<T>(v[i] + b[i]);
-      v2[i] = gelu_f(v[i]);
+      v2[i] = v[i];
     }
+    gelu8(v2);
   } else if constexpr (KIND == EPI_DGELU) {
-#pragma unroll
-    for (int i = 0; i < 8; ++i) v[i] *= gelu_grad_f(aux[i]);
+    mul_gelu_grad8(v, aux);
   }
 }
 

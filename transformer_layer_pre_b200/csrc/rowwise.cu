@@ -419,8 +419,7 @@ __global__ void gelu_kernel(const T* __restrict__ U, T* __restrict__ G, size_t n
   for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n8; i += (size_t)gridDim.x * blockDim.x) {
     float v[8];
     load8<T>(U + i * 8, v);
-#pragma unroll
-    for (int k = 0; k < 8; ++k) v[k] = gelu_f(v[k]);
+    gelu8(v);
     store8<T>(G + i * 8, v);
   }
 }
@@ -558,8 +557,9 @@ void colsum_finalize3_run(const float* p0, const float* p1, const float* p2, flo
 __global__ void gelu_eval_kernel(const float* __restrict__ u, float* __restrict__ g, float* __restrict__ dg,
                                  uint64_t n) {
   for (uint64_t i = blockIdx.x * (uint64_t)blockDim.x + threadIdx.x; i < n; i += (uint64_t)gridDim.x * blockDim.x) {
-    g[i] = gelu_f(u[i]);
-    dg[i] = gelu_grad_f(u[i]);
+    const float2 v = make_float2(u[i], 0.0f);
+    g[i] = gelu2(v).x;
+    dg[i] = gelu_grad2(v).x;
   }
 }
 
