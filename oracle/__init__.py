@@ -23,9 +23,13 @@ reordered.  Citations name the page and the section they follow:
   (fused QKV Linear(D, 3D) split into heads), section 2.3 (GELU, erf form;
   keeping the GELU input), section 5.1 (inverted dropout x*mask/(1-p)).
 
+* "Progressive Layer Dropping" (page 5), schedule section: the keep level
+  theta(t) and per-step layer skipping in a stack (``oracle.pld``).
+
 Readings taken where the pages are silent (the dropout counter layout, the
 dropout site after softmax, both hidden-dropout sites, erf GELU, biased
-variance) are listed in the design doc and restated in the docstrings below.
+variance, the depth profile and random draw of layer dropping) are stated in
+the docstrings below.
 
 Pins: every function here is checked by ``tests/test_oracle_*.py`` against
 something other than itself (cuRAND's host Philox, standard-normal table values,
@@ -40,6 +44,7 @@ from .layer import (  # noqa: F401
     round_to_storage,
     layer_norm_forward,
     layer_norm_backward,
+    layer_norm_backward_from_output,
     gelu,
     gelu_grad,
     softmax_rows,
@@ -50,3 +55,4 @@ from .layer import (  # noqa: F401
     layer_forward_backward,
     WEIGHT_NAMES,
 )
+from .pld import pld_keep, pld_keep_prob, pld_theta, stack_forward_backward  # noqa: F401

@@ -170,6 +170,20 @@ def layer_norm_backward(dy: np.ndarray, x: np.ndarray, mean: np.ndarray, rstd: n
     return dx, (dy * xhat).sum(axis=red), dy.sum(axis=red)
 
 
+def layer_norm_backward_from_output(dy: np.ndarray, y: np.ndarray, rstd: np.ndarray, gamma: np.ndarray,
+                                    beta: np.ndarray):
+    """The same gradient computed from the LayerNorm output instead of its
+    input ("DeepSpeed Transformer Kernel usage guide", Step 3,
+    normalize_invertible): x-hat = (y - beta) / gamma, which needs every
+    gamma to be non-zero; only rstd of the forward statistics is used."""
+    xhat = (y - beta) / gamma
+    g = dy * gamma
+    dx = rstd[..., None] * (g - g.mean(axis=-1, keepdims=True)
+                            - xhat * (g * xhat).mean(axis=-1, keepdims=True))
+    red = tuple(range(dy.ndim - 1))
+    return dx, (dy * xhat).sum(axis=red), dy.sum(axis=red)
+
+
 def gelu(u: np.ndarray) -> np.ndarray:
     """GELU in its exact (erf) form: u * Phi(u)."""
     return 0.5 * u * (1.0 + erf(u / math.sqrt(2.0)))

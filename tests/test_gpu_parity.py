@@ -12,7 +12,7 @@ import pytest
 import torch
 
 from parity import check_layer, run_gpu, run_oracle
-from transformer_layer_pre_b200.synthetic import WORKLOADS, Workload, make_inputs
+from transformer_layer_pre_b200.synthetic import WORKLOADS, Workload, make_inputs, with_random_affine
 
 pytestmark = pytest.mark.gpu
 
@@ -26,8 +26,10 @@ MULTITILE_POST_BF16 = Workload("multitile-post-bf16", 2, 264, 192, 3, 384, "bf16
                                lengths=(130, 264))
 
 
-def _parity(w: Workload, batch=None, **kw):
+def _parity(w: Workload, batch=None, affine=False, **kw):
     inp = make_inputs(w, batch=batch)
+    if affine:
+        inp = with_random_affine(inp)
     gpu = run_gpu(inp, **kw)
     pure = run_oracle(inp)
     rounded = None if w.dtype == "f32" else run_oracle(inp, storage_rounded=True)
@@ -89,3 +91,41 @@ def test_philox_offset_changes_masks_and_matches_oracle():
     check_layer(gpu, pure, rounded, w.dtype)
     other = run_gpu(inp, philox_offset=0)
     assert not np.array_equal(gpu["y"], other["y"])
+
+
+# Non-zero biases and LayerNorm parameters away from gamma = 1, beta = 0, so
+# that every bias add and affine step of the forward is exercised.
+def test_random_affine_f16_pre_ln():
+    _parity(RAGGED_F16, affine=True)
+
+
+def test_random_affine_bf16_post_ln():
+    _parity(MULTITILE_POST_BF16, affine=True)
+
+
+def test_random_affine_f32():
+    _parity(RAGGED_F32, affine=True)
+
+
+# normalize_invertible: LayerNorm backward from the LayerNorm output
+# ("DeepSpeed Transformer Kernel usage guide", Step 3: the input of the
+# normalisation is not kept; x-hat is recovered as (y - beta) / gamma).
+def test_normalize_invertible_pre_ln_without_x():
+    _parity(RAGGED_F16, affine=True, normalize_invertible=True, keep_x=False)
+
+
+def test_normalize_invertible_pre_ln_multitile_bf16():
+    w = dataclasses.replace(MULTITILE_F16, dtype="bf16", name="multitile-bf16")
+    _parity(w, affine=True, normalize_invertible=True, keep_x=False)
+
+
+def test_normalize_invertible_post_ln():
+    _parity(MULTITILE_POST_BF16, affine=True, normalize_invertible=True)
+
+
+def test_normalize_invertible_f32():
+    _parity(RAGGED_F32, affine=True, normalize_invertible=True, keep_x=False)
+
+
+def test_normalize_invertible_bert_large_batch2():
+    _parity(WORKLOADS["bert-large-f16"], batch=2, affine=True, normalize_invertible=True, keep_x=False)

@@ -9,7 +9,7 @@ import numpy as np
 import pytest
 import torch
 
-from oracle import (gelu, gelu_grad, layer_norm_backward, layer_norm_forward,
+from oracle import (gelu, gelu_grad, layer_norm_backward, layer_norm_backward_from_output, layer_norm_forward,
                     round_to_storage, softmax_rows)
 from oracle.layer import _apply_dropout, dropout_keep
 
@@ -118,6 +118,27 @@ def test_layernorm_backward_finite_differences():
         assert abs((L(x, gp, b) - L(x, gm, b)) / (2 * h) - dg[j]) < 1e-7
         bp, bm = b.copy(), b.copy(); bp[j] += h; bm[j] -= h
         assert abs((L(x, g, bp) - L(x, g, bm)) / (2 * h) - db[j]) < 1e-7
+
+
+def test_layernorm_backward_from_output_finite_differences():
+    # the output-based form (input dropped) against central differences of the
+    # forward; gamma with mixed signs, away from zero
+    rng = np.random.default_rng(8)
+    x = rng.normal(0.5, 2.0, (4, 32))
+    g = rng.choice([-1.0, 1.0], 32) * rng.uniform(0.3, 1.5, 32)
+    b = rng.normal(0, 0.5, 32)
+    dy = rng.normal(0, 1, (4, 32))
+    y, _, rstd = layer_norm_forward(x, g, b, 1e-5)
+    dx, dg, db = layer_norm_backward_from_output(dy, y, rstd, g, b)
+    L = lambda x_, g_, b_: float((layer_norm_forward(x_, g_, b_, 1e-5)[0] * dy).sum())
+    h = 1e-6
+    for idx in [(0, 0), (2, 13), (3, 31)]:
+        xp, xm = x.copy(), x.copy(); xp[idx] += h; xm[idx] -= h
+        assert abs((L(xp, g, b) - L(xm, g, b)) / (2 * h) - dx[idx]) < 1e-7
+    for j in [0, 17, 31]:
+        gp, gm = g.copy(), g.copy(); gp[j] += h; gm[j] -= h
+        assert abs((L(x, gp, b) - L(x, gm, b)) / (2 * h) - dg[j]) < 1e-7
+    assert np.allclose(db, dy.sum(axis=0), atol=1e-13, rtol=0)
 
 
 # ---------------------------------------------------------------- GELU

@@ -112,6 +112,26 @@ def make_inputs(w: Workload, batch: int | None = None, seed: int | None = None,
     return Inputs(w, weights, x, dy, mask, lengths)
 
 
+def with_random_affine(inp: Inputs, seed: int = 4321, bias_std: float = 0.02) -> Inputs:
+    """A copy of `inp` whose biases are N(0, bias_std) and whose LayerNorm
+    parameters are gamma = 1 + N(0, 0.1), beta = N(0, 0.1) (so that no
+    parameter takes its neutral value); drawn from a separate generator, per
+    layer in the order bqkv, bo, b1, b2, ln1_g, ln1_b, ln2_g, ln2_b."""
+    rng = np.random.default_rng(seed)
+    dt = inp.workload.dtype
+    out = []
+    for w in inp.weights:
+        w = dict(w)
+        for n in ("bqkv", "bo", "b1", "b2"):
+            w[n] = _store(rng.normal(0.0, bias_std, tuple(w[n].shape)), dt)
+        for n in ("ln1", "ln2"):
+            h = tuple(w[n + "_g"].shape)
+            w[n + "_g"] = _store(1.0 + rng.normal(0.0, 0.1, h), dt)
+            w[n + "_b"] = _store(rng.normal(0.0, 0.1, h), dt)
+        out.append(w)
+    return dataclasses.replace(inp, weights=out)
+
+
 def to_f64(t: torch.Tensor | None) -> np.ndarray | None:
     """The exact values of a stored tensor, widened to float64."""
     return None if t is None else t.to(torch.float64).numpy()
