@@ -15,7 +15,8 @@ import torch
 
 __all__ = ["Layer", "Options", "TlError", "LibraryMissing", "load_library", "dropout_keep_mask",
            "WEIGHT_NAMES", "DTYPE_CODES", "EXPORTED_SYMBOLS", "device_check",
-           "profile_enable", "profile_read", "launch_count", "PROFILE_CLASSES"]
+           "profile_enable", "profile_read", "launch_count", "PROFILE_CLASSES",
+           "pld_theta", "pld_keep_prob", "pld_keep"]
 
 HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(HERE, "libtlp.so")
@@ -30,6 +31,7 @@ EXPORTED_SYMBOLS = (
     "layer_forward", "layer_backward", "layer_workspace_bytes", "layer_last_error",
     "layer_destroy", "tl_dropout_keep_mask", "tl_device_check", "tl_profile_enable",
     "tl_profile_read", "tl_launch_count", "tl_bias_grad_noalloc", "tl_gelu_eval", "tl_status_string",
+    "tl_pld_theta", "tl_pld_keep_prob", "tl_pld_keep",
 )
 PROFILE_CLASSES = ("gemm", "attn_fwd", "attn_bwd", "ln_fwd", "ln_bwd", "rowwise")
 
@@ -106,6 +108,13 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.tl_gelu_eval.restype = i
     lib.tl_status_string.argtypes = [i]
     lib.tl_status_string.restype = ctypes.c_char_p
+    d = ctypes.c_double
+    lib.tl_pld_theta.argtypes = [d, d, u64]
+    lib.tl_pld_theta.restype = d
+    lib.tl_pld_keep_prob.argtypes = [i, i, d]
+    lib.tl_pld_keep_prob.restype = d
+    lib.tl_pld_keep.argtypes = [u64, u64, i, i, d]
+    lib.tl_pld_keep.restype = i
     _lib = lib
     return lib
 
@@ -240,6 +249,23 @@ def attention_uses_tensor_cores(dtype: str, heads: int, head_dim: int, seq: int)
     (16-bit storage and head dim 64); the exact-float32 SIMT kernels serve
     the rest."""
     return dtype in ("f16", "bf16") and head_dim == 64 and seq >= 8
+
+
+def pld_theta(theta_bar: float, gamma: float, step: int) -> float:
+    """Progressive Layer Dropping keep level at a global step."""
+    return float(load_library().tl_pld_theta(theta_bar, gamma, step))
+
+
+def pld_keep_prob(layer: int, num_layers: int, theta: float) -> float:
+    return float(load_library().tl_pld_keep_prob(layer, num_layers, theta))
+
+
+def pld_keep(seed: int, step: int, layer: int, num_layers: int, theta: float) -> bool:
+    """Whether `layer` runs at `step` (False: the layer is the identity)."""
+    r = load_library().tl_pld_keep(seed, step, layer, num_layers, theta)
+    if r < 0:
+        raise ValueError(f"layer {layer} outside a stack of {num_layers}")
+    return bool(r)
 
 
 def launch_count() -> int:
