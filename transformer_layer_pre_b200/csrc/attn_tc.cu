@@ -650,8 +650,20 @@ __global__ void __launch_bounds__(kBwdThreads)
 // runs.  Warps: 0 TMA, 1 MMA, 2-9 softmax: warp w owns TMEM lanes 32*(w%4)
 // (one query row per thread) and key columns 64*((w-2)/4) .. +63; the two
 // threads of a row combine their maxima and sums through shared memory.
-constexpr int kPFwdThreads = 320;
-constexpr int kPFwdSmem = 10 * TB + 4096 + 1024 + 256;   // Q,K,V x2, P pair x2, row exchange
+// Warps 10-13 run ahead of the softmax by up to two items: per item they
+// draw the dropout keep bits of all 128 x 128 elements (thread = query row,
+// 16 Philox calls) and stage the item's additive key mask (log2 units, -inf
+// past the sequence end), so the softmax threads only read them.
+constexpr int kPFwdThreads = 448;
+constexpr int kPFwdBits = 128 * 16;                      // keep bits of one item: [row][16 bytes]
+constexpr int kPFwdMask = 128 * 4;                       // mask row of one item: [128] float
+constexpr int kPFwdSmem = 10 * TB + 4096 + 2 * kPFwdBits + 2 * kPFwdMask + 1024 + 256;
+
+__device__ __forceinline__ float ex2_fast(float x) {
+  float r;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(x));
+  return r;
+}
 
 template <typename T>
 __global__ void __launch_bounds__(kPFwdThreads, 1)
@@ -663,10 +675,12 @@ __global__ void __launch_bounds__(kPFwdThreads, 1)
   uint8_t* sP0 = sm + 6 * TB;
   // row exchange: [max | sum][2 slots][2 halves][128 rows] floats
   float* xch = reinterpret_cast<float*>(sm + 10 * TB);
-  uint64_t* bar = reinterpret_cast<uint64_t*>(sm + 10 * TB + 4096);
+  uint8_t* sbits = sm + 10 * TB + 4096;                                   // [2][128][16]
+  float* smask = reinterpret_cast<float*>(sbits + 2 * kPFwdBits);         // [2][128]
+  uint64_t* bar = reinterpret_cast<uint64_t*>(sbits + 2 * kPFwdBits + 2 * kPFwdMask);
   uint64_t *in_full = bar, *in_empty = bar + 2, *s_full = bar + 4, *p_full = bar + 6, *o_full = bar + 8,
-           *o_free = bar + 10;
-  uint32_t* tslot = reinterpret_cast<uint32_t*>(bar + 12);
+           *o_free = bar + 10, *aux_full = bar + 12, *aux_free = bar + 14;
+  uint32_t* tslot = reinterpret_cast<uint32_t*>(bar + 16);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int S = a.S;
@@ -679,6 +693,8 @@ __global__ void __launch_bounds__(kPFwdThreads, 1)
       mbar_init(&p_full[j], 256);
       mbar_init(&o_full[j], 1);
       mbar_init(&o_free[j], 256);
+      mbar_init(&aux_full[j], 128);
+      mbar_init(&aux_free[j], 256);
     }
     fence_barrier_init();
   }
@@ -739,6 +755,29 @@ __global__ void __launch_bounds__(kPFwdThreads, 1)
         mma_commit(&in_empty[j]);
       }
     }
+  } else if (warp >= 10) {
+    // keep bits and mask row of each item, two items ahead at most
+    const int r = threadIdx.x - 320;
+    int n = 0;
+    for (int it = blockIdx.x; it < nitems; it += gridDim.x, ++n) {
+      const int j = n & 1;
+      if (!mbar_wait(&aux_free[j], ((n >> 1) & 1) ^ 1, a.err, 58)) break;
+      if (a.drop.thr) {
+        const uint64_t e8 = (((uint64_t)it * S + (uint64_t)r) * (uint64_t)S) >> 3;
+        uint32_t w[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          uint32_t v = 0;
+#pragma unroll
+          for (int g = 0; g < 4; ++g) v |= dropout_bits8(a.drop, 0, e8 + (uint64_t)(q * 4 + g)) << (8 * g);
+          w[q] = v;
+        }
+        *reinterpret_cast<uint4*>(sbits + j * kPFwdBits + r * 16) = make_uint4(w[0], w[1], w[2], w[3]);
+      }
+      const int b = it / a.nh;
+      smask[j * 128 + r] = r < S ? (a.mask ? a.mask[(size_t)b * S + r] * kLog2e : 0.0f) : -INFINITY;
+      mbar_arrive(&aux_full[j]);
+    }
   } else {
     const int quarter = warp & 3;
     const int hf = (warp - 2) >> 2;
@@ -775,8 +814,9 @@ __global__ void __launch_bounds__(kPFwdThreads, 1)
     };
     for (int it = blockIdx.x; it < nitems && ok; it += gridDim.x, ++n) {
       const int j = n & 1;
-      const int b = it / a.nh;
-      const uint64_t erow = ((uint64_t)it * S + (uint64_t)r) * (uint64_t)S;
+      if (!(ok = mbar_wait_warp(&aux_full[j], (n >> 1) & 1, a.err, 59))) break;
+      const uint2 kb8 = a.drop.thr ? *reinterpret_cast<const uint2*>(sbits + j * kPFwdBits + r * 16 + hf * 8)
+                                   : make_uint2(0xFFFFFFFFu, 0xFFFFFFFFu);
       if (!(ok = mbar_wait_warp(&s_full[j], (n >> 1) & 1, a.err, 57))) break;
       tc_fence_after();
       float sv[64];
@@ -784,24 +824,29 @@ __global__ void __launch_bounds__(kPFwdThreads, 1)
       tmem_ld32(tmem + 128 * j + lo + kc0 + 32, *reinterpret_cast<float(*)[32]>(sv + 32));
       float mx = -INFINITY;
 #pragma unroll
-      for (int t = 0; t < 64; ++t) {
-        sv[t] = fmaf(sv[t], c2, mask_log2(a, b, kc0 + t));
-        mx = fmaxf(mx, sv[t]);
+      for (int t = 0; t < 64; t += 4) {
+        const float4 m4 = *reinterpret_cast<const float4*>(smask + j * 128 + kc0 + t);
+        sv[t] = fmaf(sv[t], c2, m4.x);
+        sv[t + 1] = fmaf(sv[t + 1], c2, m4.y);
+        sv[t + 2] = fmaf(sv[t + 2], c2, m4.z);
+        sv[t + 3] = fmaf(sv[t + 3], c2, m4.w);
+        mx = fmaxf(fmaxf(mx, fmaxf(sv[t], sv[t + 1])), fmaxf(sv[t + 2], sv[t + 3]));
       }
+      mbar_arrive(&aux_free[j]);
       float* xm = xch + j * 256;
       xm[hf * 128 + r] = mx;
       named_barrier(1, 256);
       mx = fmaxf(mx, xm[(1 - hf) * 128 + r]);
+      // a row whose keys are all masked has mx = -inf: every p is 0
+      const float msub = mx == -INFINITY ? 0.0f : mx;
       float lsum = 0.0f;
 #pragma unroll
       for (int g = 0; g < 8; ++g) {
-        const int kb = kc0 + g * 8;
-        const uint32_t bits = a.drop.thr ? dropout_bits8(a.drop, 0, (erow + (uint64_t)kb) >> 3) : 0xFFu;
+        const uint32_t bits = ((g < 4 ? kb8.x : kb8.y) >> (8 * (g & 3))) & 0xFFu;
         float pv[8];
 #pragma unroll
         for (int t = 0; t < 8; ++t) {
-          const float x = sv[g * 8 + t];
-          const float p = (x == -INFINITY) ? 0.0f : exp2f(x - mx);
+          const float p = ex2_fast(sv[g * 8 + t] - msub);
           lsum += p;
           pv[t] = ((bits >> t) & 1u) ? p * dsc : 0.0f;
         }
@@ -834,22 +879,27 @@ __global__ void __launch_bounds__(kPFwdThreads, 1)
 // One CTA per SM walks (sequence, head) items, each one 128 x 128 tile:
 // S = Q K^T and dPd = dO V^T, then Pd and dS to shared memory, then dV, dK and
 // dQ in TMEM and out to dQKV.  Q/K/V/dO are double-buffered by item parity so
-// the next item's loads overlap this item's work.  D = rowsum(dO * O) comes
-// from the shared-memory dO tile and the stored output O.
-constexpr int kPBwdSmem = 12 * TB + 1024 + 256;   // (Q,K,V,dO) x2, Pd pair, dS pair
+// the next item's loads overlap this item's work.  Warps 10-13 prepare each
+// item ahead of the softmax warps: D = rowsum(dO * O) (dO from the item's
+// shared tile, O from global memory), the row's log-sum-exp, the additive
+// key mask and the dropout keep bits, all into shared memory.
+constexpr int kPBwdThreads = 448;
+constexpr int kPBwdAux = 128 * 16 + 3 * 128 * 4;          // bits [128][16], mask, lse2, D [128] floats
+constexpr int kPBwdSmem = 12 * TB + 2 * kPBwdAux + 1024 + 256;   // (Q,K,V,dO) x2, Pd pair, dS pair, aux x2
 
 template <typename T>
-__global__ void __launch_bounds__(kBwdThreads, 1)
+__global__ void __launch_bounds__(kPBwdThreads, 1)
     attn_bwd_tc_persist(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
                         const __grid_constant__ CUtensorMap tv, const __grid_constant__ CUtensorMap tdo, AttnTc a) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = align1024(smem_raw);
   uint8_t* sPd = sm + 8 * TB;
   uint8_t* sdS = sm + 10 * TB;
-  uint64_t* bar = reinterpret_cast<uint64_t*>(sm + 12 * TB);
+  uint8_t* saux = sm + 12 * TB;    // per slot: bits [128][16] | mask [128] | lse2 [128] | D [128]
+  uint64_t* bar = reinterpret_cast<uint64_t*>(saux + 2 * kPBwdAux);
   uint64_t *in_full = bar, *in_empty = bar + 2, *s_full = bar + 4, *s_free = bar + 5, *ds_full = bar + 6,
-           *g_full = bar + 7, *g_free = bar + 8;
-  uint32_t* tslot = reinterpret_cast<uint32_t*>(bar + 9);
+           *g_full = bar + 7, *g_free = bar + 8, *aux_full = bar + 9, *aux_free = bar + 11;
+  uint32_t* tslot = reinterpret_cast<uint32_t*>(bar + 13);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int S = a.S;
@@ -858,6 +908,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     for (int j = 0; j < 2; ++j) {
       mbar_init(&in_full[j], 1);
       mbar_init(&in_empty[j], 1);
+      mbar_init(&aux_full[j], 128);
+      mbar_init(&aux_free[j], kSoftThreads);
     }
     mbar_init(s_full, 1);
     mbar_init(s_free, kSoftThreads);
@@ -920,36 +972,103 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         mma_commit(&in_empty[j]);
       }
     }
+  } else if (warp >= 10) {
+    // per item: keep bits, mask row, lse2 and D of every query row
+    const int r = threadIdx.x - 320;
+    int n = 0;
+    for (int it = blockIdx.x; it < nitems; it += gridDim.x, ++n) {
+      const int j = n & 1;
+      uint8_t* ax = saux + j * kPBwdAux;
+      float* smask = reinterpret_cast<float*>(ax + 2048);
+      if (!mbar_wait(&aux_free[j], ((n >> 1) & 1) ^ 1, a.err, 69)) break;
+      if (a.drop.thr) {
+        const uint64_t e8 = (((uint64_t)it * S + (uint64_t)r) * (uint64_t)S) >> 3;
+        uint32_t w[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          uint32_t v = 0;
+#pragma unroll
+          for (int g = 0; g < 4; ++g) v |= dropout_bits8(a.drop, 0, e8 + (uint64_t)(q * 4 + g)) << (8 * g);
+          w[q] = v;
+        }
+        *reinterpret_cast<uint4*>(ax + r * 16) = make_uint4(w[0], w[1], w[2], w[3]);
+      }
+      const int b = it / a.nh, h = it - (it / a.nh) * a.nh;
+      const bool qv = r < S;
+      smask[r] = qv ? (a.mask ? a.mask[(size_t)b * S + r] * kLog2e : 0.0f) : -INFINITY;
+      smask[128 + r] = qv ? a.lse[(size_t)it * S + r] * kLog2e : INFINITY;
+      float Di = 0.0f;
+      if (qv) {
+        // O row from global memory first, then dO from the item's shared tile
+        const T* orow = static_cast<const T*>(a.ctx_in) + ((size_t)b * S + r) * a.H + h * HD;
+        Raw8<T> o8[8];
+#pragma unroll
+        for (int c = 0; c < 8; ++c) o8[c] = raw8_load<T>(orow + c * 8);
+        if (!mbar_wait(&in_full[j], (n >> 1) & 1, a.err, 70)) break;
+        const uint8_t* drow = sm + j * 4 * TB + 3 * TB + r * 128;
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+          float x[8], y[8];
+          load8<T>(reinterpret_cast<const T*>(drow + ((c ^ (r & 7)) << 4)), x);
+          raw8_unpack<T>(o8[c], y);
+#pragma unroll
+          for (int t = 0; t < 8; ++t) Di = fmaf(x[t], y[t], Di);
+        }
+      }
+      smask[256 + r] = Di;
+      mbar_arrive(&aux_full[j]);
+    }
   } else {
     const int quarter = warp & 3;
     const int hf = (warp - 2) >> 2;
     const int r = quarter * 32 + lane;
     const uint32_t lo = (uint32_t)(quarter * 32) << 16;
+    const float c2 = a.scale * kLog2e;
+    const float dsc = a.drop.thr ? a.drop.scale : 1.0f;
+    const int kc0 = hf * 64;
     int n = 0;
     for (int it = blockIdx.x; it < nitems; it += gridDim.x, ++n) {
       const int j = n & 1;
       const int b = it / a.nh, h = it - (it / a.nh) * a.nh;
       const bool qv = r < S;
       const size_t trow = (size_t)b * S + r;
-      const float lse2 = qv ? a.lse[(size_t)it * S + r] * kLog2e : INFINITY;
-      if (!mbar_wait_warp(&in_full[j], (n >> 1) & 1, a.err, 66)) break;
-      // D = rowsum(dO * O): dO from the swizzled shared tile, O from global memory
-      float Di = 0.0f;
-      if (qv) {
-        const uint8_t* drow = sm + j * 4 * TB + 3 * TB + r * 128;
-        const T* orow = static_cast<const T*>(a.ctx_in) + trow * a.H + h * HD;
-#pragma unroll
-        for (int c = 0; c < 8; ++c) {
-          float x[8], y[8];
-          load8<T>(reinterpret_cast<const T*>(drow + ((c ^ (r & 7)) << 4)), x);
-          load8<T>(orow + c * 8, y);
-#pragma unroll
-          for (int t = 0; t < 8; ++t) Di = fmaf(x[t], y[t], Di);
-        }
-      }
+      const uint8_t* ax = saux + j * kPBwdAux;
+      const float* smask = reinterpret_cast<const float*>(ax + 2048);
+      if (!mbar_wait_warp(&aux_full[j], (n >> 1) & 1, a.err, 66)) break;
+      const uint2 kb8 = a.drop.thr ? *reinterpret_cast<const uint2*>(ax + r * 16 + hf * 8)
+                                   : make_uint2(0xFFFFFFFFu, 0xFFFFFFFFu);
+      const float lse2 = smask[128 + r];
+      const float Di = smask[256 + r];
       if (!mbar_wait_warp(s_full, n & 1, a.err, 67)) break;
       tc_fence_after();
-      bwd_pair_rows<T>(a, b, it * S, r, r, 0, hf * 64, tS, tdP, lo, lse2, Di, sPd, sdS);
+#pragma unroll 1
+      for (int c = 0; c < 2; ++c) {
+        float sv[32], dv[32];
+        tmem_ld32(tS + lo + kc0 + c * 32, sv);
+        tmem_ld32(tdP + lo + kc0 + c * 32, dv);
+        const uint32_t bw = c == 0 ? kb8.x : kb8.y;
+#pragma unroll
+        for (int g = 0; g < 4; ++g) {
+          const int kt = kc0 + c * 32 + g * 8;   // key column
+          const uint32_t bits = (bw >> (8 * g)) & 0xFFu;
+          const float4 m0 = *reinterpret_cast<const float4*>(smask + kt);
+          const float4 m1 = *reinterpret_cast<const float4*>(smask + kt + 4);
+          const float ml[8] = {m0.x, m0.y, m0.z, m0.w, m1.x, m1.y, m1.z, m1.w};
+          float pd[8], ds[8];
+#pragma unroll
+          for (int t = 0; t < 8; ++t) {
+            // lse2 = +inf for rows past the sequence end: p = 0
+            const float p = ex2_fast(fmaf(sv[g * 8 + t], c2, ml[t]) - lse2);
+            const bool keep = (bits >> t) & 1u;
+            pd[t] = keep ? p * dsc : 0.0f;
+            const float dp = keep ? dv[g * 8 + t] * dsc : 0.0f;
+            ds[t] = p * (dp - Di);
+          }
+          pair_store8<T>(sPd, r, kt >> 3, pd);
+          pair_store8<T>(sdS, r, kt >> 3, ds);
+        }
+      }
+      mbar_arrive(&aux_free[j]);
       tc_fence_before();
       mbar_arrive(s_free);
       fence_proxy_async_smem();
@@ -1087,7 +1206,7 @@ void bwd_t(const AttnArgs& a, cudaStream_t s) {
   if (ntile == 1) {
     int nsm = 148;
     cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, 0);
-    attn_bwd_tc_persist<T><<<std::min(a.B * a.nh, nsm), kBwdThreads, kPBwdSmem, s>>>(mq, mk, mv, mdo, t);
+    attn_bwd_tc_persist<T><<<std::min(a.B * a.nh, nsm), kPBwdThreads, kPBwdSmem, s>>>(mq, mk, mv, mdo, t);
     count_launch();
     return;
   }
