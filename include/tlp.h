@@ -83,6 +83,10 @@ typedef struct {
                                     in pre-LN form); requires every gamma != 0 */
   int training;                  /* 1 (default): forward keeps what backward needs and applies
                                     dropout; 0: inference, dropout off, no backward */
+  int gelu_tanh;                 /* 0 (default): GELU(u) = u * Phi(u), the erf form;
+                                    1: the tanh approximation 0.5 u (1 + tanh(sqrt(2/pi)
+                                    (u + 0.044715 u^3))) ("AI-infra engineers and the
+                                    Transformer", section 2.3), forward and backward */
 } tl_options;
 
 /* The twelve parameter tensors, all passed on every call (Step 2: the layer
@@ -152,6 +156,10 @@ tl_status tl_dropout_keep_mask(uint64_t seed, uint64_t philox_offset, int site, 
  * epilogues use: erf form, Phi(u) from the normal-tail approximation of
  * Abramowitz & Stegun 26.2.17 (absolute error below 7.5e-8) in float32. */
 tl_status tl_gelu_eval(const float* u, float* g, float* dg, uint64_t n, void* stream);
+
+/* Test hook: as tl_gelu_eval for the tanh form (tl_options.gelu_tanh), the
+ * same device code as the layer's epilogues with that option. */
+tl_status tl_gelu_tanh_eval(const float* u, float* g, float* dg, uint64_t n, void* stream);
 
 /* Waits for all work on the current device, then reports TL_ECUDA if a CUDA
  * error is pending, TL_ETIMEOUT if a bounded device-side wait of a

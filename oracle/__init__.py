@@ -47,6 +47,8 @@ from .layer import (  # noqa: F401
     layer_norm_backward_from_output,
     gelu,
     gelu_grad,
+    gelu_tanh,
+    gelu_tanh_grad,
     softmax_rows,
     attention_forward,
     attention_backward,

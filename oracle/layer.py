@@ -48,6 +48,7 @@ class LayerConfig:
     philox_offset: int = 0       # the layer's id in a stack
     ln_eps: float = 1e-12
     storage: str = "f32"        # 'f32' | 'f16' | 'bf16': what the GPU stores in HBM
+    gelu_form: str = "erf"      # 'erf' (exact) | 'tanh' (the approximation of section 2.3)
 
     @property
     def ffn_dim(self) -> int:
@@ -194,6 +195,27 @@ def gelu_grad(u: np.ndarray) -> np.ndarray:
     return 0.5 * (1.0 + erf(u / math.sqrt(2.0))) + u * np.exp(-0.5 * u * u) / math.sqrt(2.0 * math.pi)
 
 
+_SQRT_2_OVER_PI = math.sqrt(2.0 / math.pi)
+_TANH_CUBIC = 0.044715
+
+
+def gelu_tanh(u: np.ndarray) -> np.ndarray:
+    """GELU in the tanh approximation ("AI-infra engineers and the
+    Transformer", section 2.3): 0.5 u (1 + tanh(sqrt(2/pi) (u + 0.044715 u^3)))."""
+    return 0.5 * u * (1.0 + np.tanh(_SQRT_2_OVER_PI * (u + _TANH_CUBIC * u ** 3)))
+
+
+def gelu_tanh_grad(u: np.ndarray) -> np.ndarray:
+    """Derivative of gelu_tanh: with z = sqrt(2/pi) (u + 0.044715 u^3) and
+    t = tanh(z), 0.5 (1 + t) + 0.5 u (1 - t^2) sqrt(2/pi) (1 + 3 * 0.044715 u^2)."""
+    t = np.tanh(_SQRT_2_OVER_PI * (u + _TANH_CUBIC * u ** 3))
+    return 0.5 * (1.0 + t) + 0.5 * u * (1.0 - t * t) * _SQRT_2_OVER_PI * (1.0 + 3.0 * _TANH_CUBIC * u * u)
+
+
+def _gelu_pair(cfg):
+    return (gelu_tanh, gelu_tanh_grad) if cfg.gelu_form == "tanh" else (gelu, gelu_grad)
+
+
 def softmax_rows(s: np.ndarray) -> np.ndarray:
     """Softmax over the last axis with the row maximum subtracted; a row whose
     entries are all -inf (every key masked) is defined to be all zeros."""
@@ -332,7 +354,7 @@ def layer_forward(cfg: LayerConfig, x, mask, w, seq_index=None, storage_rounded=
         h2, m2, r2 = layer_norm_forward(x2, W["ln2_g"], W["ln2_b"], cfg.ln_eps)
         h2 = R(h2)
         u = R(h2 @ W["w1"].T + W["b1"])
-        g = R(gelu(u))
+        g = R(_gelu_pair(cfg)[0](u))
         y = R(x2 + _apply_dropout(g @ W["w2"].T + W["b2"], keep2, ph))
         sv.update(h1=h1, mean1=m1, rstd1=r1, qkv=qkv, ctx=ctx, x2=x2,
                   h2=h2, mean2=m2, rstd2=r2, u=u, g=g)
@@ -343,7 +365,7 @@ def layer_forward(cfg: LayerConfig, x, mask, w, seq_index=None, storage_rounded=
         x2, m1, r1 = layer_norm_forward(res1, W["ln1_g"], W["ln1_b"], cfg.ln_eps)
         x2 = R(x2)
         u = R(x2 @ W["w1"].T + W["b1"])
-        g = R(gelu(u))
+        g = R(_gelu_pair(cfg)[0](u))
         res2 = R(x2 + _apply_dropout(g @ W["w2"].T + W["b2"], keep2, ph))
         y, m2, r2 = layer_norm_forward(res2, W["ln2_g"], W["ln2_b"], cfg.ln_eps)
         y = R(y)
@@ -374,7 +396,7 @@ def layer_backward(cfg: LayerConfig, sv: dict, dy):
         dz2 = R(_apply_dropout(dy, sv["keep2"], ph))
         gr["b2"] = _colsum(dz2)
         gr["w2"] = _wgrad(dz2, sv["g"])
-        du = R((dz2 @ W["w2"]) * gelu_grad(sv["u"]))
+        du = R((dz2 @ W["w2"]) * _gelu_pair(cfg)[1](sv["u"]))
         gr["b1"] = _colsum(du)
         gr["w1"] = _wgrad(du, sv["h2"])
         dh2 = R(du @ W["w1"])
@@ -396,7 +418,7 @@ def layer_backward(cfg: LayerConfig, sv: dict, dy):
         dz2 = R(_apply_dropout(dres2, sv["keep2"], ph))
         gr["b2"] = _colsum(dz2)
         gr["w2"] = _wgrad(dz2, sv["g"])
-        du = R((dz2 @ W["w2"]) * gelu_grad(sv["u"]))
+        du = R((dz2 @ W["w2"]) * _gelu_pair(cfg)[1](sv["u"]))
         gr["b1"] = _colsum(du)
         gr["w1"] = _wgrad(du, sv["x2"])
         dx2 = R(du @ W["w1"] + dres2)

@@ -37,7 +37,7 @@ def oracle_config(w: Workload, batch: int, philox_offset: int = 0) -> oracle.Lay
                               attn_dropout=float(np.float32(w.attn_dropout)),
                               hidden_dropout=float(np.float32(w.hidden_dropout)),
                               pre_layer_norm=w.pre_layer_norm, seed=w.seed, philox_offset=philox_offset,
-                              storage=w.dtype)
+                              storage=w.dtype, gelu_form=w.gelu)
 
 
 def run_gpu(inp: Inputs, layer: int = 0, gelu_checkpoint: bool | None = None, normalize_invertible=False,
@@ -49,7 +49,7 @@ def run_gpu(inp: Inputs, layer: int = 0, gelu_checkpoint: bool | None = None, no
     ck = w.gelu_checkpoint if gelu_checkpoint is None else gelu_checkpoint
     L = Layer(b, w.seq, w.hidden, w.heads, w.ffn, w.attn_dropout, w.hidden_dropout, w.pre_layer_norm, w.seed,
               dtype=TORCH_DT[w.dtype], philox_offset=philox_offset, gelu_checkpoint=ck,
-              normalize_invertible=normalize_invertible)
+              normalize_invertible=normalize_invertible, gelu_tanh=w.gelu == "tanh")
     try:
         wt = {n: inp.weights[layer][n].to(dev) for n in WEIGHT_NAMES}
         x = inp.x.to(dev)

@@ -32,9 +32,18 @@ def _worker(rank: int, world: int, port: int, q):
         ptrs = sorted((g[n].data_ptr(), g[n].numel()) for n in g.views)
         aligned = all(p % 16 == 0 for p, _ in ptrs)
         disjoint = all(p1 + 4 * n1 <= p2 for (p1, n1), (p2, _) in zip(ptrs, ptrs[1:]))
+        # per-layer buckets submitted one by one (the stack's overlapped exchange)
+        from transformer_layer_pre_b200.dp import GradExchanger
+        layers = [FlatGrads(32, 64, "cpu") for _ in range(3)]
+        ex = GradExchanger()
+        for l in reversed(range(3)):
+            layers[l].flat.fill_(float(rank * 10 + l))
+            ex.submit(layers[l])
+        ex.finish()
+        ok_layers = all(torch.all(layers[l].flat == float(5 + l)) for l in range(3))
         mx = bench.reduce_max(1.0 + rank)
         bench.barrier()
-        q.put((rank, bool(ok_mean), aligned, disjoint, mx))
+        q.put((rank, bool(ok_mean) and bool(ok_layers), aligned, disjoint, mx))
     finally:
         dist.destroy_process_group()
 

@@ -25,3 +25,17 @@ def test_device_gelu_matches_exact_erf_form():
     tol_g = np.abs(u64) * (7.5e-8 + 4 * eps) + 4 * eps * np.abs(ref_g)
     assert np.all(np.abs(g.cpu().double().numpy() - ref_g) <= tol_g + 1e-30)
     assert np.abs(dg.cpu().double().numpy() - ref_dg).max() <= 1e-6
+
+
+def test_device_tanh_gelu_matches_the_tanh_form():
+    u = np.concatenate([np.linspace(-10, 10, 200001), np.random.default_rng(4).normal(0, 3, 100000),
+                        [0.0, -0.0, 1e-30, -1e-30, 1e-6, 40.0, -40.0]]).astype(np.float32)
+    g, dg = tlp.gelu_eval(torch.from_numpy(u).cuda(), tanh_form=True)
+    u64 = u.astype(np.float64)
+    ref_g, ref_dg = oracle.gelu_tanh(u64), oracle.gelu_tanh_grad(u64)
+    # tanh(|z|) = (1 - e)/(1 + e): a few float32 ulps of 1 in tanh, so the
+    # GELU error is at most |u| times that plus the rounding of the product
+    eps = np.finfo(np.float32).eps
+    tol_g = np.abs(u64) * 4 * eps + 4 * eps * np.abs(ref_g)
+    assert np.all(np.abs(g.cpu().double().numpy() - ref_g) <= tol_g + 1e-30)
+    assert np.abs(dg.cpu().double().numpy() - ref_dg).max() <= 1e-6

@@ -129,3 +129,23 @@ def test_normalize_invertible_f32():
 
 def test_normalize_invertible_bert_large_batch2():
     _parity(WORKLOADS["bert-large-f16"], batch=2, affine=True, normalize_invertible=True, keep_x=False)
+
+
+# GELU in its tanh approximation (tl_options.gelu_tanh) against the oracle's
+# tanh form, forward and backward, and bitwise under gelu_checkpoint.
+def test_gelu_tanh_f16_pre_ln():
+    _parity(dataclasses.replace(RAGGED_F16, gelu="tanh"), affine=True)
+
+
+def test_gelu_tanh_f32_post_ln():
+    _parity(dataclasses.replace(RAGGED_F32, gelu="tanh", pre_layer_norm=False), affine=True)
+
+
+def test_gelu_tanh_checkpoint_is_bitwise_identical():
+    w = dataclasses.replace(RAGGED_F16, gelu="tanh")
+    inp = make_inputs(w)
+    a = run_gpu(inp, gelu_checkpoint=False)
+    b = run_gpu(inp, gelu_checkpoint=True)
+    assert np.array_equal(a["y"], b["y"]) and np.array_equal(a["dx"], b["dx"])
+    for n in a["grads"]:
+        assert np.array_equal(a["grads"][n], b["grads"][n]), n

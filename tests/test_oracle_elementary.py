@@ -9,7 +9,7 @@ import numpy as np
 import pytest
 import torch
 
-from oracle import (gelu, gelu_grad, layer_norm_backward, layer_norm_backward_from_output, layer_norm_forward,
+from oracle import (gelu, gelu_grad, gelu_tanh, gelu_tanh_grad, layer_norm_backward, layer_norm_backward_from_output, layer_norm_forward,
                     round_to_storage, softmax_rows)
 from oracle.layer import _apply_dropout, dropout_keep
 
@@ -164,6 +164,23 @@ def test_gelu_grad_finite_differences():
     h = 1e-5
     fd = (gelu(x + h) - gelu(x - h)) / (2 * h)
     assert np.allclose(gelu_grad(x), fd, atol=1e-9)
+
+
+def test_gelu_tanh_form():
+    # the tanh approximation: odd-part identity (tanh is odd), zero at 0,
+    # close to the exact erf form everywhere (the largest gap of the
+    # approximation is a few 1e-4) but not equal to it, derivative by
+    # central differences, and the asymptotes u and 0
+    x = np.random.default_rng(10).normal(0, 3, 1000)
+    assert np.allclose(gelu_tanh(x) - gelu_tanh(-x), x, atol=1e-14)
+    assert gelu_tanh(np.array([0.0]))[0] == 0.0
+    g = np.linspace(-10, 10, 20001)
+    gap = np.abs(gelu_tanh(g) - gelu(g))
+    assert 1e-4 < gap.max() < 1e-3
+    h = 1e-5
+    xs = np.linspace(-6, 6, 241)
+    assert np.allclose(gelu_tanh_grad(xs), (gelu_tanh(xs + h) - gelu_tanh(xs - h)) / (2 * h), atol=1e-9)
+    assert gelu_tanh(np.array([30.0]))[0] == 30.0 and gelu_tanh(np.array([-30.0]))[0] == 0.0
 
 
 # ---------------------------------------------------------------- dropout

@@ -32,8 +32,9 @@ def _mask(lengths, s):
 
 def _torch_layer(cfg, w, x, mask, dy):
     h, nh, f = cfg.hidden, cfg.heads, cfg.ffn_dim
+    act = "gelu" if cfg.gelu_form == "erf" else (lambda v: torch.nn.functional.gelu(v, approximate="tanh"))
     layer = torch.nn.TransformerEncoderLayer(
-        d_model=h, nhead=nh, dim_feedforward=f, dropout=0.0, activation="gelu",
+        d_model=h, nhead=nh, dim_feedforward=f, dropout=0.0, activation=act,
         layer_norm_eps=cfg.ln_eps, batch_first=True, norm_first=cfg.pre_layer_norm,
         dtype=torch.float64)
     T = lambda a: torch.tensor(a, dtype=torch.float64)
@@ -64,9 +65,10 @@ def _torch_layer(cfg, w, x, mask, dy):
 
 @pytest.mark.parametrize("pre_ln", [True, False])
 @pytest.mark.parametrize("masked", [False, True])
-def test_matches_torch_encoder_layer_float64(pre_ln, masked):
+@pytest.mark.parametrize("gelu_form", ["erf", "tanh"])
+def test_matches_torch_encoder_layer_float64(pre_ln, masked, gelu_form):
     rng = np.random.default_rng(11)
-    cfg = LayerConfig(batch=3, seq=16, hidden=32, heads=4, ffn=48, pre_layer_norm=pre_ln)
+    cfg = LayerConfig(batch=3, seq=16, hidden=32, heads=4, ffn=48, pre_layer_norm=pre_ln, gelu_form=gelu_form)
     w = _weights(rng, 32, 48)
     x = rng.normal(0, 1, (3, 16, 32))
     dy = rng.normal(0, 1, (3, 16, 32))

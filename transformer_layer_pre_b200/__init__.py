@@ -31,7 +31,7 @@ EXPORTED_SYMBOLS = (
     "layer_forward", "layer_backward", "layer_workspace_bytes", "layer_last_error",
     "layer_destroy", "tl_dropout_keep_mask", "tl_device_check", "tl_profile_enable",
     "tl_profile_read", "tl_launch_count", "tl_bias_grad_noalloc", "tl_gelu_eval", "tl_status_string",
-    "tl_pld_theta", "tl_pld_keep_prob", "tl_pld_keep",
+    "tl_pld_theta", "tl_pld_keep_prob", "tl_pld_keep", "tl_gelu_tanh_eval",
 )
 PROFILE_CLASSES = ("gemm", "attn_fwd", "attn_bwd", "ln_fwd", "ln_bwd", "rowwise")
 
@@ -55,6 +55,7 @@ class Options(ctypes.Structure):
         ("attn_dropout_checkpoint", ctypes.c_int),
         ("normalize_invertible", ctypes.c_int),
         ("training", ctypes.c_int),
+        ("gelu_tanh", ctypes.c_int),
     ]
 
 
@@ -106,6 +107,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.tl_bias_grad_noalloc.restype = i
     lib.tl_gelu_eval.argtypes = [vp, vp, vp, u64, vp]
     lib.tl_gelu_eval.restype = i
+    lib.tl_gelu_tanh_eval.argtypes = [vp, vp, vp, u64, vp]
+    lib.tl_gelu_tanh_eval.restype = i
     lib.tl_status_string.argtypes = [i]
     lib.tl_status_string.restype = ctypes.c_char_p
     d = ctypes.c_double
@@ -139,7 +142,7 @@ class Layer:
     def __init__(self, batch, seq, hidden, heads, ffn=0, attn_dropout=0.0, hidden_dropout=0.0,
                  pre_layer_norm=True, seed=1234, dtype=torch.float16, ln_eps=1e-12, philox_offset=0,
                  gelu_checkpoint=False, attn_dropout_checkpoint=False, normalize_invertible=False,
-                 training=True):
+                 training=True, gelu_tanh=False):
         self.lib = load_library()
         self.handle = None
         h = ctypes.c_void_p()
@@ -160,6 +163,7 @@ class Layer:
         opt.attn_dropout_checkpoint = int(attn_dropout_checkpoint)
         opt.normalize_invertible = int(normalize_invertible)
         opt.training = int(training)
+        opt.gelu_tanh = int(gelu_tanh)
         self._check(self.lib.layer_set_options(self.handle, ctypes.byref(opt)))
 
     def _check(self, st: int) -> None:
@@ -218,13 +222,15 @@ def device_check() -> None:
         raise TlError(st, lib.tl_status_string(st).decode())
 
 
-def gelu_eval(u: torch.Tensor):
-    """(GELU(u), GELU'(u)) from the library's device GELU; u float32 on the device."""
+def gelu_eval(u: torch.Tensor, tanh_form: bool = False):
+    """(GELU(u), GELU'(u)) from the library's device GELU (erf form, or the
+    tanh approximation); u float32 on the device."""
     lib = load_library()
     u = u.contiguous()
     g = torch.empty_like(u)
     dg = torch.empty_like(u)
-    st = lib.tl_gelu_eval(_ptr(u), _ptr(g), _ptr(dg), u.numel(), _stream(None))
+    fn = lib.tl_gelu_tanh_eval if tanh_form else lib.tl_gelu_eval
+    st = fn(_ptr(u), _ptr(g), _ptr(dg), u.numel(), _stream(None))
     if st != 0:
         raise TlError(st, lib.tl_status_string(st).decode())
     return g, dg

@@ -230,6 +230,62 @@ __device__ __forceinline__ void mul_gelu_grad8(float (&v)[8], const float (&u)[8
   }
 }
 
+// GELU in its tanh approximation ("AI-infra engineers and the Transformer",
+// section 2.3): GELU(u) = u (1 + tanh(z)) / 2 with z = sqrt(2/pi) (u + 0.044715 u^3),
+// GELU'(u) = (1 + t)/2 + u (1 - t^2) sqrt(2/pi) (1 + 3 * 0.044715 u^2) / 2, t = tanh(z).
+// tanh(|z|) = (1 - e) / (1 + e) with e = exp(-2|z|) (one base-2 exponential and
+// one reciprocal per element), the sign restored from z.
+__device__ __forceinline__ float2 tanh_gelu_arg2(float2 u) {
+  constexpr float kS = 0.797884560802865356f;      // sqrt(2/pi)
+  constexpr float kC = 0.044715f;
+  constexpr float kM2Log2e = -2.88539008177792682f;   // exp(-2a) = 2^(a * kM2Log2e)
+  const float2 z = __fmul2_rn(__fmul2_rn(u, f2(kS)), __ffma2_rn(__fmul2_rn(u, u), f2(kC), f2(1.0f)));
+  const float2 a = __fmul2_rn(make_float2(fabsf(z.x), fabsf(z.y)), f2(kM2Log2e));
+  const float2 e = make_float2(ex2_approx(a.x), ex2_approx(a.y));
+  const float2 den = __fadd2_rn(e, f2(1.0f));
+  const float2 t = __fmul2_rn(__ffma2_rn(e, f2(-1.0f), f2(1.0f)), make_float2(rcp_approx(den.x), rcp_approx(den.y)));
+  return make_float2(copysignf(t.x, z.x), copysignf(t.y, z.y));
+}
+__device__ __forceinline__ float2 gelu_tanh2(float2 u) {
+  const float2 t = tanh_gelu_arg2(u);
+  return __fmul2_rn(__fmul2_rn(u, f2(0.5f)), __fadd2_rn(t, f2(1.0f)));
+}
+__device__ __forceinline__ float2 gelu_tanh_grad2(float2 u) {
+  constexpr float kS = 0.797884560802865356f;
+  constexpr float kC3 = 3.0f * 0.044715f;
+  const float2 t = tanh_gelu_arg2(u);
+  const float2 sech2 = __ffma2_rn(t, make_float2(-t.x, -t.y), f2(1.0f));                  // 1 - t^2
+  const float2 dz = __fmul2_rn(__ffma2_rn(__fmul2_rn(u, u), f2(kC3), f2(1.0f)), f2(kS));  // dz/du
+  const float2 half_u = __fmul2_rn(u, f2(0.5f));
+  return __ffma2_rn(__fmul2_rn(half_u, sech2), dz, __fmul2_rn(__fadd2_rn(t, f2(1.0f)), f2(0.5f)));
+}
+// In-place over 8 lanes, either form.
+__device__ __forceinline__ void gelu8_form(float (&v)[8], bool tanh_form) {
+  if (!tanh_form) {
+    gelu8(v);
+    return;
+  }
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float2 g = gelu_tanh2(make_float2(v[2 * i], v[2 * i + 1]));
+    v[2 * i] = g.x;
+    v[2 * i + 1] = g.y;
+  }
+}
+__device__ __forceinline__ void mul_gelu_grad8_form(float (&v)[8], const float (&u)[8], bool tanh_form) {
+  if (!tanh_form) {
+    mul_gelu_grad8(v, u);
+    return;
+  }
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float2 d =
+        __fmul2_rn(make_float2(v[2 * i], v[2 * i + 1]), gelu_tanh_grad2(make_float2(u[2 * i], u[2 * i + 1])));
+    v[2 * i] = d.x;
+    v[2 * i + 1] = d.y;
+  }
+}
+
 // ------------------------------------------------------------------ warp reductions
 __device__ __forceinline__ float warp_sum(float v) {
 #pragma unroll

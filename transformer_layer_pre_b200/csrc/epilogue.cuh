@@ -11,7 +11,8 @@
 //                     and FFN2 sites, "DeepSpeed Transformer Kernel usage
 //                     guide", Step 2 hidden_dropout_ratio).
 //  EPI_BIAS_GELU      U = acc + bias stored; G = GELU(U as stored) so that a
-//                     backward that recomputes G from U gets identical bits.
+//                     backward that recomputes G from U gets identical bits
+//                     (erf form, or the tanh form when e.gelu_tanh).
 //  EPI_DGELU          out = acc * GELU'(U).
 //  EPI_STORE          out = acc (+ res).
 //  EPI_F32            float32 out = acc.
@@ -81,11 +82,11 @@ __device__ __forceinline__ void epi_apply8(const EpiParams& e, int m, int n, flo
     for (int i = 0; i < 8; ++i) v[i] = round_f<T>(v[i] + b[i]);
     store8<T>(static_cast<T*>(e.out) + (size_t)m * e.ldo + n, v);
     if (e.out2) {
-      gelu8(v);
+      gelu8_form(v, e.gelu_tanh != 0);
       store8<T>(static_cast<T*>(e.out2) + (size_t)m * e.ldo + n, v);
     }
   } else if constexpr (KIND == EPI_DGELU) {
-    mul_gelu_grad8(v, aux);
+    mul_gelu_grad8_form(v, aux, e.gelu_tanh != 0);
     store8<T>(static_cast<T*>(e.out) + (size_t)m * e.ldo + n, v);
   }
 }
@@ -122,9 +123,9 @@ __device__ __forceinline__ void epi_compute8(const EpiParams& e, int m, int n, f
       v[i] = round_f<T>(v[i] + b[i]);
       v2[i] = v[i];
     }
-    gelu8(v2);
+    gelu8_form(v2, e.gelu_tanh != 0);
   } else if constexpr (KIND == EPI_DGELU) {
-    mul_gelu_grad8(v, aux);
+    mul_gelu_grad8_form(v, aux, e.gelu_tanh != 0);
   }
 }
 

@@ -45,6 +45,8 @@ struct EpiParams {
   int site;
   // head split (EPI_QKV)
   int seq, hidden, head_dim, heads, tokens;
+  // EPI_BIAS_GELU / EPI_DGELU: 1 for the tanh approximation of GELU
+  int gelu_tanh;
 };
 
 // Returns 0, or non-zero when an operand cannot be described to the TMA unit
@@ -82,8 +84,10 @@ struct LnBwdArgs {
   float* part_dsum;     // column sums of drop_out, or null
   int rows, H;
 };
+// Upper bound of the partial rows ln_bwd_run writes (size of the part_* buffers).
 int ln_bwd_parts(int rows);
-void ln_bwd_run(int dtype, const LnBwdArgs& a, cudaStream_t s);
+// Returns the number of partial rows written (to pass to the finalize).
+int ln_bwd_run(int dtype, const LnBwdArgs& a, cudaStream_t s);
 
 // ------------------------------------------------------------------ elementwise / reductions
 // out = dropout(in) (site, element t*H + c) with column partial sums of out.
@@ -99,9 +103,9 @@ void colsum_finalize_run(const float* part, int nparts, int cols, float* out, cu
 void colsum_finalize3_run(const float* p0, const float* p1, const float* p2, float* o0, float* o1, float* o2,
                           int nparts, int cols, cudaStream_t s);
 // g[i] = GELU(u[i]), dg[i] = GELU'(u[i]) with the device GELU every kernel uses (float32).
-void gelu_eval_run(const float* u, float* g, float* dg, uint64_t n, cudaStream_t s);
+void gelu_eval_run(const float* u, float* g, float* dg, uint64_t n, int tanh_form, cudaStream_t s);
 // G = GELU(U), elementwise, n a multiple of 8.
-void gelu_run(int dtype, const void* U, void* G, size_t n, cudaStream_t s);
+void gelu_run(int dtype, const void* U, void* G, size_t n, int tanh_form, cudaStream_t s);
 // keep[i] = dropout keep bit of element e0 + i of `site`.
 void dropout_mask_run(const DropoutParams& dp, int site, uint64_t e0, uint64_t n, uint8_t* keep, cudaStream_t s);
 

@@ -293,6 +293,7 @@ tl_status layer_set_options(tl_layer* L, const tl_options* o) {
   free_buffers(L);
   L->opt = *o;
   L->opt.training = o->training ? 1 : 0;
+  L->opt.gelu_tanh = o->gelu_tanh ? 1 : 0;
   return ensure_buffers(L);
 }
 
@@ -340,7 +341,7 @@ tl_status layer_forward(tl_layer* L, const void* x, const float* mask, const tl_
   EpiParams eo = epi(EPI_BIAS_DROP_RES, nullptr, H);
   eo.bias = w->bo; eo.res = x; eo.drop = make_drop(L, L->ph); eo.site = 1;
   EpiParams e1 = epi(EPI_BIAS_GELU, L->u, F);
-  e1.bias = w->b1; e1.out2 = L->g;
+  e1.bias = w->b1; e1.out2 = L->g; e1.gelu_tanh = L->opt.gelu_tanh ? 1 : 0;
   EpiParams e2 = epi(EPI_BIAS_DROP_RES, nullptr, H);
   e2.bias = w->b2; e2.drop = make_drop(L, L->ph); e2.site = 2;
 
@@ -409,7 +410,6 @@ tl_status layer_backward(tl_layer* L, const void* x, const void* dy, const tl_we
   cudaStream_t s = (cudaStream_t)stream;
   const int dt = L->opt.dtype, T = L->T, H = L->H, F = L->F;
   const size_t es = dtype_size(dt);
-  const int lnp = ln_bwd_parts(T);
   float* pa = L->part;
   float* pb = L->part + L->part_floats;
   float* pc = L->part + 2 * L->part_floats;
@@ -426,8 +426,8 @@ tl_status layer_backward(tl_layer* L, const void* x, const void* dy, const tl_we
     a.part_dgamma = pa; a.part_dbeta = pb; a.part_dsum = drop_out ? pc : nullptr;
     a.rows = T; a.H = H;
     ProfScope p_(PC_LN_BWD, s);
-    ln_bwd_run(dt, a, s);
-    colsum_finalize3_run(pa, pb, drop_out ? pc : nullptr, dgamma, dbeta, drop_out ? dsum : nullptr, lnp, H, s);
+    const int parts = ln_bwd_run(dt, a, s);
+    colsum_finalize3_run(pa, pb, drop_out ? pc : nullptr, dgamma, dbeta, drop_out ? dsum : nullptr, parts, H, s);
   };
 
   // FFN block: dZ2 -> dW2, dU (into big), db1, dW1; returns with dU in L->big
@@ -435,11 +435,12 @@ tl_status layer_backward(tl_layer* L, const void* x, const void* dy, const tl_we
     EpiParams ew2 = epi(EPI_F32, g->w2, F);
     if (L->opt.gelu_checkpoint) {
       ProfScope p_(PC_ROWWISE, s);
-      gelu_run(dt, L->u, L->big, (size_t)T * F, s);
+      gelu_run(dt, L->u, L->big, (size_t)T * F, L->opt.gelu_tanh ? 1 : 0, s);
     }
     gemm(L, H, F, T, L->dz2, H, false, L->g, F, false, ew2, s);          // dW2 = dZ2^T G
     EpiParams edu = epi(EPI_DGELU, L->big, F);
     edu.aux = L->u;
+    edu.gelu_tanh = L->opt.gelu_tanh ? 1 : 0;
     gemm(L, T, F, H, L->dz2, H, true, w->w2, F, false, edu, s);          // dU = (dZ2 W2) GELU'(U)
     bias_grad(L, L->big, F, g->b1, s);                                     // db1
     EpiParams ew1 = epi(EPI_F32, g->w1, H);
@@ -508,7 +509,14 @@ tl_status tl_device_check(void) {
 tl_status tl_gelu_eval(const float* u, float* g, float* dg, uint64_t n, void* stream) {
   if (!u || !g || !dg) return TL_EINVAL;
   if (n == 0) return TL_OK;
-  gelu_eval_run(u, g, dg, n, (cudaStream_t)stream);
+  gelu_eval_run(u, g, dg, n, 0, (cudaStream_t)stream);
+  return cudaGetLastError() == cudaSuccess ? TL_OK : TL_ECUDA;
+}
+
+tl_status tl_gelu_tanh_eval(const float* u, float* g, float* dg, uint64_t n, void* stream) {
+  if (!u || !g || !dg) return TL_EINVAL;
+  if (n == 0) return TL_OK;
+  gelu_eval_run(u, g, dg, n, 1, (cudaStream_t)stream);
   return cudaGetLastError() == cudaSuccess ? TL_OK : TL_ECUDA;
 }
 

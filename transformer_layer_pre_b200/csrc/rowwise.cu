@@ -140,11 +140,40 @@ size_t pipe_smem(int H) {
 }
 
 // ------------------------------------------------------------------ LayerNorm forward
-// One warp per row, kFwdRows rows per warp loaded up front (16-byte vectors,
-// lane-interleaved chunks of 8), shuffle-only reductions, gamma/beta staged
-// in shared memory as float32.  NCH = chunks of 8 per lane (H <= 256*NCH).
-constexpr int kFwdRows = 2;
-constexpr int kFwdWarps = 8;
+// One warp per row, lane-interleaved chunks of 8 columns (16-byte vectors),
+// shuffle-only reductions, no shared memory and no block barrier: a warp
+// issues its row's loads first (streaming, not kept in L1) and gamma/beta
+// through the read-only path (every warp reads the same H values, so they
+// stay cached).  NCH = chunks of 8 per lane (H <= 256*NCH).
+constexpr int kFwdWarps = 4;
+
+__device__ __forceinline__ uint4 ldg_stream16(const void* p) {
+  uint4 r;
+  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w) : "l"(p));
+  return r;
+}
+template <typename T> __device__ __forceinline__ Raw8<T> raw8_stream(const T* p) {
+  Raw8<T> r;
+  r.a = ldg_stream16(p);
+  return r;
+}
+template <> __device__ __forceinline__ Raw8<float> raw8_stream<float>(const float* p) {
+  Raw8<float> r;
+  const uint4 a = ldg_stream16(p), b = ldg_stream16(p + 4);
+  r.a = make_float4(__uint_as_float(a.x), __uint_as_float(a.y), __uint_as_float(a.z), __uint_as_float(a.w));
+  r.b = make_float4(__uint_as_float(b.x), __uint_as_float(b.y), __uint_as_float(b.z), __uint_as_float(b.w));
+  return r;
+}
+template <typename T> __device__ __forceinline__ void load8_ro(const T* p, float (&v)[8]) {
+  Raw8<T> r;
+  r.a = __ldg(reinterpret_cast<const uint4*>(p));
+  raw8_unpack<T>(r, v);
+}
+template <> __device__ __forceinline__ void load8_ro<float>(const float* p, float (&v)[8]) {
+  const float4 a = __ldg(reinterpret_cast<const float4*>(p)), b = __ldg(reinterpret_cast<const float4*>(p) + 1);
+  v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w; v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+}
 
 template <typename T, int NCH>
 __global__ void __launch_bounds__(kFwdWarps * 32) ln_fwd_kernel(const T* __restrict__ x, const T* __restrict__ gamma,
@@ -152,63 +181,52 @@ __global__ void __launch_bounds__(kFwdWarps * 32) ln_fwd_kernel(const T* __restr
                                                                 float* __restrict__ mean_out,
                                                                 float* __restrict__ rstd_out, int rows, int H,
                                                                 float eps) {
-  extern __shared__ float gb[];   // [2][H]
-  for (int c = threadIdx.x; c < H; c += blockDim.x) {
-    gb[c] = to_f(gamma[c]);
-    gb[H + c] = to_f(beta[c]);
-  }
-  __syncthreads();
   const int lane = threadIdx.x & 31;
-  const int row0 = (blockIdx.x * kFwdWarps + (threadIdx.x >> 5)) * kFwdRows;
-  Raw8<T> raw[kFwdRows][NCH];
+  const int row = blockIdx.x * kFwdWarps + (threadIdx.x >> 5);
+  if (row >= rows) return;
+  Raw8<T> raw[NCH];
 #pragma unroll
-  for (int r = 0; r < kFwdRows; ++r) {
-#pragma unroll
-    for (int c = 0; c < NCH; ++c) {
-      const int col = (lane + 32 * c) * 8;
-      raw[r][c] = (row0 + r < rows && col < H) ? raw8_load<T>(x + (size_t)(row0 + r) * H + col) : raw8_zero<T>();
-    }
+  for (int c = 0; c < NCH; ++c) {
+    const int col = (lane + 32 * c) * 8;
+    raw[c] = col < H ? raw8_stream<T>(x + (size_t)row * H + col) : raw8_zero<T>();
   }
   const float inv_h = 1.0f / (float)H;
+  float v[NCH][8];
+  float s = 0.0f;
 #pragma unroll
-  for (int r = 0; r < kFwdRows; ++r) {
-    const int row = row0 + r;
-    if (row >= rows) break;
-    float v[NCH][8];
-    float s = 0.0f;
+  for (int c = 0; c < NCH; ++c) {
+    raw8_unpack<T>(raw[c], v[c]);
 #pragma unroll
-    for (int c = 0; c < NCH; ++c) {
-      raw8_unpack<T>(raw[r][c], v[c]);
+    for (int i = 0; i < 8; ++i) s += v[c][i];
+  }
+  const float mean = warp_sum(s) * inv_h;
+  float ss = 0.0f;
 #pragma unroll
-      for (int i = 0; i < 8; ++i) s += v[c][i];
-    }
-    const float mean = warp_sum(s) * inv_h;
-    float ss = 0.0f;
+  for (int c = 0; c < NCH; ++c) {
+    if ((lane + 32 * c) * 8 < H) {
 #pragma unroll
-    for (int c = 0; c < NCH; ++c) {
-      if ((lane + 32 * c) * 8 < H) {
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          const float d = v[c][i] - mean;
-          ss += d * d;
-        }
+      for (int i = 0; i < 8; ++i) {
+        const float d = v[c][i] - mean;
+        ss += d * d;
       }
     }
-    const float rstd = 1.0f / sqrtf(warp_sum(ss) * inv_h + eps);
+  }
+  const float rstd = 1.0f / sqrtf(warp_sum(ss) * inv_h + eps);
 #pragma unroll
-    for (int c = 0; c < NCH; ++c) {
-      const int col = (lane + 32 * c) * 8;
-      if (col < H) {
-        float o[8];
+  for (int c = 0; c < NCH; ++c) {
+    const int col = (lane + 32 * c) * 8;
+    if (col < H) {
+      float g[8], b[8], o[8];
+      load8_ro<T>(gamma + col, g);
+      load8_ro<T>(beta + col, b);
 #pragma unroll
-        for (int i = 0; i < 8; ++i) o[i] = gb[col + i] * ((v[c][i] - mean) * rstd) + gb[H + col + i];
-        store8<T>(y + (size_t)row * H + col, o);
-      }
+      for (int i = 0; i < 8; ++i) o[i] = g[i] * ((v[c][i] - mean) * rstd) + b[i];
+      store8<T>(y + (size_t)row * H + col, o);
     }
-    if (lane == 0) {
-      mean_out[row] = mean;
-      rstd_out[row] = rstd;
-    }
+  }
+  if (lane == 0) {
+    mean_out[row] = mean;
+    rstd_out[row] = rstd;
   }
 }
 
@@ -317,6 +335,155 @@ __global__ void __launch_bounds__(512) ln_bwd_kernel(LnBwdArgs a) {
   }
 }
 
+// LayerNorm backward for H <= 1024: two warps per row (64 lanes, lane L owns
+// the 8-column chunks L, L+64, ...; NC chunks), no block-wide barrier inside
+// the row loop.  A block owns a contiguous range of rows; its kLnbPairs warp
+// pairs take every kLnbPairs-th row and load the pair's next row before
+// working on the current one.  The row sums of the two warps meet in shared
+// memory behind a 64-thread named barrier.  Each lane keeps the column sums
+// (dgamma, dbeta and, with a dropout copy, the dropped gradient) of its own
+// columns in registers; at the end the block adds its pairs' sums in shared
+// memory in pair order, leaving one partial row per block.
+constexpr int kLnbPairs = 4;
+
+template <typename T, bool INV, bool RES, bool DROP, int NC>
+__global__ void __launch_bounds__(kLnbPairs * 64, (sizeof(T) == 4 || (INV && DROP)) ? 1 : 2) ln_bwd_warp_kernel(LnBwdArgs a) {
+  extern __shared__ __align__(16) float red[];   // [kLnbPairs][H]; row exchange after it
+  float* xch = red + kLnbPairs * a.H;            // [pair][row parity][half][2]
+  const int H = a.H;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int pair = warp >> 1, half = warp & 1;
+  const int L = half * 32 + lane;
+  const float inv_h = 1.0f / (float)H;
+  const float sc = a.drop.thr ? a.drop.scale : 1.0f;
+  const T* dyp = static_cast<const T*>(a.dy);
+  const T* xp = static_cast<const T*>(INV ? a.y : a.x);
+  const T* rp = static_cast<const T*>(a.res);
+  float dg[NC][8], db[NC][8], ds[DROP ? NC : 1][8];
+#pragma unroll
+  for (int c = 0; c < NC; ++c)
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      dg[c][i] = db[c][i] = 0.0f;
+      if constexpr (DROP) ds[c][i] = 0.0f;
+    }
+  int r0, r1;
+  row_range(a.rows, r0, r1);
+  Raw8<T> rdy[NC], rx[NC];
+  auto fetch = [&](int row) {
+#pragma unroll
+    for (int c = 0; c < NC; ++c) {
+      const int col = (L + 64 * c) * 8;
+      const bool in = row < r1 && col < H;
+      const size_t off = (size_t)row * H + col;
+      rdy[c] = in ? raw8_stream<T>(dyp + off) : raw8_zero<T>();
+      rx[c] = in ? raw8_stream<T>(xp + off) : raw8_zero<T>();
+    }
+  };
+  int row = r0 + pair;
+  fetch(row);
+  for (int k = 0; row < r1; row += kLnbPairs, ++k) {
+    float dy[NC][8], xh[NC][8];
+#pragma unroll
+    for (int c = 0; c < NC; ++c) {
+      raw8_unpack<T>(rdy[c], dy[c]);
+      raw8_unpack<T>(rx[c], xh[c]);
+    }
+    const float rs = a.rstd[row];
+    const float mean = INV ? 0.0f : a.mean[row];
+    fetch(row + kLnbPairs);
+    Raw8<T> rr[RES ? NC : 1];
+    if constexpr (RES) {
+#pragma unroll
+      for (int c = 0; c < NC; ++c) {
+        const int col = (L + 64 * c) * 8;
+        rr[c] = col < H ? raw8_stream<T>(rp + (size_t)row * H + col) : raw8_zero<T>();
+      }
+    }
+    float s1 = 0.0f, s2 = 0.0f;
+#pragma unroll
+    for (int c = 0; c < NC; ++c) {
+      const int col = (L + 64 * c) * 8;
+      if (col >= H) continue;
+      float gm[8];
+      load8_ro<T>(static_cast<const T*>(a.gamma) + col, gm);
+      if constexpr (INV) {
+        float bt[8];
+        load8_ro<T>(static_cast<const T*>(a.beta) + col, bt);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) xh[c][i] = (xh[c][i] - bt[i]) / gm[i];
+      } else {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) xh[c][i] = (xh[c][i] - mean) * rs;
+      }
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        dg[c][i] += dy[c][i] * xh[c][i];
+        db[c][i] += dy[c][i];
+        dy[c][i] *= gm[i];                 // g = dy * gamma from here on
+        s1 += dy[c][i];
+        s2 += dy[c][i] * xh[c][i];
+      }
+    }
+    s1 = warp_sum(s1);
+    s2 = warp_sum(s2);
+    float* xr = xch + (pair * 2 + (k & 1)) * 4;
+    if (lane == 0) {
+      xr[half * 2] = s1;
+      xr[half * 2 + 1] = s2;
+    }
+    sm100::named_barrier(1 + pair, 64);
+    const float m1 = (xr[0] + xr[2]) * inv_h, m2 = (xr[1] + xr[3]) * inv_h;
+#pragma unroll
+    for (int c = 0; c < NC; ++c) {
+      const int col = (L + 64 * c) * 8;
+      if (col >= H) continue;
+      const size_t off = (size_t)row * H + col;
+      float o[8];
+      float rv[8];
+      if constexpr (RES) raw8_unpack<T>(rr[c], rv);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        o[i] = rs * (dy[c][i] - m1 - xh[c][i] * m2);
+        if constexpr (RES) o[i] += rv[i];
+      }
+      store8<T>(static_cast<T*>(a.dx) + off, o);
+      if constexpr (DROP) {
+        const uint32_t bits = a.drop.thr ? dropout_bits8(a.drop, a.site, off >> 3) : 0xFFu;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          o[i] = round_f<T>(((bits >> i) & 1u) ? round_f<T>(o[i]) * sc : 0.0f);
+          ds[c][i] += o[i];
+        }
+        store8<T>(static_cast<T*>(a.drop_out) + off, o);
+      }
+    }
+  }
+  // block sums in pair order, one tensor at a time
+  auto reduce = [&](float (*acc)[8], float* part) {
+    __syncthreads();
+#pragma unroll
+    for (int c = 0; c < NC; ++c) {
+      const int col = (L + 64 * c) * 8;
+      if (col < H) {
+        float* d = red + pair * H + col;
+        reinterpret_cast<float4*>(d)[0] = make_float4(acc[c][0], acc[c][1], acc[c][2], acc[c][3]);
+        reinterpret_cast<float4*>(d)[1] = make_float4(acc[c][4], acc[c][5], acc[c][6], acc[c][7]);
+      }
+    }
+    __syncthreads();
+    for (int col = threadIdx.x; col < H; col += blockDim.x) {
+      float t = 0.0f;
+#pragma unroll
+      for (int w = 0; w < kLnbPairs; ++w) t += red[w * H + col];
+      part[(size_t)blockIdx.x * H + col] = t;
+    }
+  };
+  reduce(dg, a.part_dgamma);
+  reduce(db, a.part_dbeta);
+  if constexpr (DROP) reduce(ds, a.part_dsum);
+}
+
 // ------------------------------------------------------------------ dropout of rows
 template <typename T, int KR>
 __global__ void __launch_bounds__(512) dropout_rows_kernel(const T* __restrict__ in, T* __restrict__ out,
@@ -415,11 +582,11 @@ __global__ void __launch_bounds__(1024) colsum_finalize_kernel(FinalizeArgs fa, 
 }
 
 template <typename T>
-__global__ void gelu_kernel(const T* __restrict__ U, T* __restrict__ G, size_t n8) {
+__global__ void gelu_kernel(const T* __restrict__ U, T* __restrict__ G, size_t n8, int tanh_form) {
   for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n8; i += (size_t)gridDim.x * blockDim.x) {
     float v[8];
     load8<T>(U + i * 8, v);
-    gelu8(v);
+    gelu8_form(v, tanh_form != 0);
     store8<T>(G + i * 8, v);
   }
 }
@@ -456,24 +623,41 @@ int row_blocks(int rows) { return std::max(1, std::min(kMaxBlocks, (rows + 31) /
 template <typename T>
 void ln_fwd_t(const void* x, const void* g, const void* b, void* y, float* mean, float* rstd, int rows, int H,
               float eps, cudaStream_t s) {
-  const int blocks = (rows + kFwdWarps * kFwdRows - 1) / (kFwdWarps * kFwdRows);
-  const size_t sm = 2 * (size_t)H * sizeof(float);
+  const int blocks = (rows + kFwdWarps - 1) / kFwdWarps;
   TLP_NCH_SWITCH(H, {
-    ln_fwd_kernel<T, NCH><<<blocks, kFwdWarps * 32, sm, s>>>(static_cast<const T*>(x), static_cast<const T*>(g),
+    ln_fwd_kernel<T, NCH><<<blocks, kFwdWarps * 32, 0, s>>>(static_cast<const T*>(x), static_cast<const T*>(g),
                                                             static_cast<const T*>(b), static_cast<T*>(y), mean, rstd,
                                                             rows, H, eps);
   });
   count_launch();
 }
 
+template <typename T, bool INV, bool RES, bool DROP, int NC>
+void ln_bwd_warp_launch(const LnBwdArgs& a, int parts, cudaStream_t s) {
+  const size_t sm = ((size_t)kLnbPairs * a.H + kLnbPairs * 8) * sizeof(float);
+  cudaFuncSetAttribute(ln_bwd_warp_kernel<T, INV, RES, DROP, NC>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                       (int)sm);
+  ln_bwd_warp_kernel<T, INV, RES, DROP, NC><<<parts, kLnbPairs * 64, sm, s>>>(a);
+}
+
 template <typename T, bool INV, bool RES>
-void ln_bwd_t(const LnBwdArgs& a, cudaStream_t s) {
-  TLP_KR_SWITCH(a.H, (int)sizeof(T), {
-    const size_t sm = pipe_smem<T, KR, RES ? 3 : 2>(a.H);
-    cudaFuncSetAttribute(ln_bwd_kernel<T, INV, RES, KR>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
-    ln_bwd_kernel<T, INV, RES, KR><<<ln_bwd_parts(a.rows), row_threads(a.H), sm, s>>>(a);
-  });
+int ln_bwd_t(const LnBwdArgs& a, cudaStream_t s) {
+  const int parts = ln_bwd_parts(a.rows);
+  if (a.H <= 512) {
+    a.drop_out ? ln_bwd_warp_launch<T, INV, RES, true, 1>(a, parts, s)
+               : ln_bwd_warp_launch<T, INV, RES, false, 1>(a, parts, s);
+  } else if (a.H <= 1024) {
+    a.drop_out ? ln_bwd_warp_launch<T, INV, RES, true, 2>(a, parts, s)
+               : ln_bwd_warp_launch<T, INV, RES, false, 2>(a, parts, s);
+  } else {
+    TLP_KR_SWITCH(a.H, (int)sizeof(T), {
+      const size_t sm = pipe_smem<T, KR, RES ? 3 : 2>(a.H);
+      cudaFuncSetAttribute(ln_bwd_kernel<T, INV, RES, KR>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+      ln_bwd_kernel<T, INV, RES, KR><<<parts, row_threads(a.H), sm, s>>>(a);
+    });
+  }
   count_launch();
+  return parts;
 }
 
 template <typename T>
@@ -506,16 +690,16 @@ void ln_fwd_run(int dt, const void* x, const void* g, const void* b, void* y, fl
 }
 
 template <typename T>
-void ln_bwd_dispatch(const LnBwdArgs& a, cudaStream_t s) {
+int ln_bwd_dispatch(const LnBwdArgs& a, cudaStream_t s) {
   const bool inv = a.x == nullptr, res = a.res != nullptr;
-  if (inv) res ? ln_bwd_t<T, true, true>(a, s) : ln_bwd_t<T, true, false>(a, s);
-  else res ? ln_bwd_t<T, false, true>(a, s) : ln_bwd_t<T, false, false>(a, s);
+  if (inv) return res ? ln_bwd_t<T, true, true>(a, s) : ln_bwd_t<T, true, false>(a, s);
+  return res ? ln_bwd_t<T, false, true>(a, s) : ln_bwd_t<T, false, false>(a, s);
 }
 
-void ln_bwd_run(int dt, const LnBwdArgs& a, cudaStream_t s) {
-  if (dt == DT_F32) ln_bwd_dispatch<float>(a, s);
-  else if (dt == DT_F16) ln_bwd_dispatch<half_t>(a, s);
-  else ln_bwd_dispatch<bf16_t>(a, s);
+int ln_bwd_run(int dt, const LnBwdArgs& a, cudaStream_t s) {
+  if (dt == DT_F32) return ln_bwd_dispatch<float>(a, s);
+  if (dt == DT_F16) return ln_bwd_dispatch<half_t>(a, s);
+  return ln_bwd_dispatch<bf16_t>(a, s);
 }
 
 int rowwise_take_error() {
@@ -555,26 +739,29 @@ void colsum_finalize3_run(const float* p0, const float* p1, const float* p2, flo
 }
 
 __global__ void gelu_eval_kernel(const float* __restrict__ u, float* __restrict__ g, float* __restrict__ dg,
-                                 uint64_t n) {
+                                 uint64_t n, int tanh_form) {
   for (uint64_t i = blockIdx.x * (uint64_t)blockDim.x + threadIdx.x; i < n; i += (uint64_t)gridDim.x * blockDim.x) {
     const float2 v = make_float2(u[i], 0.0f);
-    g[i] = gelu2(v).x;
-    dg[i] = gelu_grad2(v).x;
+    g[i] = tanh_form ? gelu_tanh2(v).x : gelu2(v).x;
+    dg[i] = tanh_form ? gelu_tanh_grad2(v).x : gelu_grad2(v).x;
   }
 }
 
-void gelu_eval_run(const float* u, float* g, float* dg, uint64_t n, cudaStream_t s) {
+void gelu_eval_run(const float* u, float* g, float* dg, uint64_t n, int tanh_form, cudaStream_t s) {
   const int blocks = (int)std::min<uint64_t>((n + 255) / 256, 148 * 16);
-  gelu_eval_kernel<<<blocks > 0 ? blocks : 1, 256, 0, s>>>(u, g, dg, n);
+  gelu_eval_kernel<<<blocks > 0 ? blocks : 1, 256, 0, s>>>(u, g, dg, n, tanh_form);
   count_launch();
 }
 
-void gelu_run(int dt, const void* U, void* G, size_t n, cudaStream_t s) {
+void gelu_run(int dt, const void* U, void* G, size_t n, int tanh_form, cudaStream_t s) {
   const size_t n8 = n / 8;
   const int blocks = (int)std::min<size_t>((n8 + 255) / 256, 148 * 16);
-  if (dt == DT_F32) gelu_kernel<float><<<blocks, 256, 0, s>>>(static_cast<const float*>(U), static_cast<float*>(G), n8);
-  else if (dt == DT_F16) gelu_kernel<half_t><<<blocks, 256, 0, s>>>(static_cast<const half_t*>(U), static_cast<half_t*>(G), n8);
-  else gelu_kernel<bf16_t><<<blocks, 256, 0, s>>>(static_cast<const bf16_t*>(U), static_cast<bf16_t*>(G), n8);
+  if (dt == DT_F32)
+    gelu_kernel<float><<<blocks, 256, 0, s>>>(static_cast<const float*>(U), static_cast<float*>(G), n8, tanh_form);
+  else if (dt == DT_F16)
+    gelu_kernel<half_t><<<blocks, 256, 0, s>>>(static_cast<const half_t*>(U), static_cast<half_t*>(G), n8, tanh_form);
+  else
+    gelu_kernel<bf16_t><<<blocks, 256, 0, s>>>(static_cast<const bf16_t*>(U), static_cast<bf16_t*>(G), n8, tanh_form);
   count_launch();
 }
 

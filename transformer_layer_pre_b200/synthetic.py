@@ -44,6 +44,7 @@ class Workload:
     layers: int = 1
     gelu_checkpoint: bool = False
     seed: int = 1234
+    gelu: str = "erf"              # 'erf' | 'tanh' (the approximation)
 
     @property
     def tokens(self) -> int:
