@@ -24,9 +24,7 @@ import json
 import os
 import re
 import statistics
-import subprocess
 import sys
-import tempfile
 import time
 
 import numpy as np
@@ -41,10 +39,6 @@ from transformer_layer_pre_b200.synthetic import WORKLOADS, make_inputs  # noqa:
 METRIC = "fwd+bwd tokens/s per BERT-Large layer (B64,S128,fp16); % of tensor peak"
 WORKLOAD = "bert-large-f16"
 L2_FLUSH_BYTES = 256 << 20   # > 126 MB of L2
-CLOCK_FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-                "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-                "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
-
 
 # ---------------------------------------------------------------- algorithmic work
 def linear_flops_per_token(h: int, f: int) -> float:
@@ -143,57 +137,72 @@ def barrier() -> None:
 
 # ---------------------------------------------------------------- clocks
 class ClockSampler:
-    """nvidia-smi sampling of SM clocks and throttle reasons in the background."""
+    """Samples the GPU's SM clock, power and clock-event (throttle) reasons
+    through NVML every few milliseconds on a background thread (read-only
+    queries; no setting is touched).  Samples taken while `timed` is set
+    form the timed-region summary."""
 
-    def __init__(self, index: int):
-        self.index = index
-        self.proc = None
-        self.path = None
+    REASONS = (("nvmlClocksEventReasonHwSlowdown", "hw_slowdown"),
+               ("nvmlClocksEventReasonHwThermalSlowdown", "hw_thermal_slowdown"),
+               ("nvmlClocksEventReasonSwThermalSlowdown", "sw_thermal_slowdown"),
+               ("nvmlClocksEventReasonSwPowerCap", "sw_power_cap"))
+
+    def __init__(self, index: int, period_s: float = 0.002):
+        self.index, self.period = index, period_s
+        self.timed = False
+        self.rows: list = []
+        self.smax = None
+        self._stop = None
+        self._thread = None
+
+    def _handle(self, pynvml):
+        """The NVML handle of CUDA device `index`, matched by PCI address
+        (NVML numbers every GPU of the machine, CUDA only the visible ones)."""
+        try:
+            p = torch.cuda.get_device_properties(self.index)
+            return pynvml.nvmlDeviceGetHandleByPciBusId(
+                f"{p.pci_domain_id:08x}:{p.pci_bus_id:02x}:{p.pci_device_id:02x}.0".encode())
+        except Exception:
+            return pynvml.nvmlDeviceGetHandleByIndex(self.index)
 
     def __enter__(self):
+        import threading
         try:
-            fd, self.path = tempfile.mkstemp(suffix=".csv")
-            os.close(fd)
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={CLOCK_FIELDS}", "--format=csv,noheader,nounits",
-                 "-lms", "200"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
-        except (OSError, FileNotFoundError):
-            self.proc = None
+            import pynvml
+            pynvml.nvmlInit()
+            h = self._handle(pynvml)
+            self.smax = float(pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM))
+        except Exception:   # no NVML: no clock record
+            return self
+        masks = [(getattr(pynvml, n), name) for n, name in self.REASONS]
+        self._stop = threading.Event()
+
+        def loop():
+            while not self._stop.is_set():
+                if self.timed:
+                    try:
+                        sm = pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM)
+                        r = pynvml.nvmlDeviceGetCurrentClocksEventReasons(h)
+                        self.rows.append((float(sm), [name for m, name in masks if r & m]))
+                    except Exception:
+                        pass
+                self._stop.wait(self.period)
+
+        self._thread = threading.Thread(target=loop, daemon=True)
+        self._thread.start()
         return self
 
     def __exit__(self, *exc):
-        if self.proc is not None:
-            self.proc.terminate()
-            try:
-                self.proc.wait(timeout=5)
-            except subprocess.TimeoutExpired:
-                self.proc.kill()
+        if self._thread is not None:
+            self._stop.set()
+            self._thread.join(timeout=5)
 
     def summary(self) -> dict | None:
-        if self.proc is None or not self.path or not os.path.exists(self.path):
+        if not self.rows:
             return None
-        rows = []
-        for ln in open(self.path):
-            parts = [p.strip() for p in ln.split(",")]
-            if len(parts) < 9:
-                continue
-            try:
-                rows.append(dict(sm=float(parts[1]), smax=float(parts[2]), power=float(parts[3]),
-                                 hw=parts[5], hwt=parts[6], swt=parts[7], cap=parts[8]))
-            except ValueError:
-                continue
-        os.unlink(self.path)
-        if not rows:
-            return None
-        load = [r for r in rows if r["power"] > 300.0] or rows
-        reasons = set()
-        for r in load:
-            for k, name in (("hw", "hw_slowdown"), ("hwt", "hw_thermal_slowdown"), ("swt", "sw_thermal_slowdown"),
-                            ("cap", "sw_power_cap")):
-                if r[k].lower().startswith("active"):
-                    reasons.add(name)
-        return {"sm_mhz": statistics.median(r["sm"] for r in load), "sm_max_mhz": max(r["smax"] for r in rows),
-                "reasons": sorted(reasons), "samples": len(rows), "samples_under_load": len(load)}
+        reasons = sorted({n for _, rs in self.rows for n in rs})
+        return {"sm_mhz": statistics.median(sm for sm, _ in self.rows), "sm_max_mhz": self.smax,
+                "reasons": reasons, "samples": len(self.rows), "source": "NVML, every 2 ms over the timed region"}
 
 
 # ---------------------------------------------------------------- oracle (reference arm / CPU baseline)
@@ -356,6 +365,7 @@ def run_ours(args) -> None:
         evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
         barrier()
         torch.cuda.synchronize()
+        clk.timed = True
         for a, b in evs:
             flush.zero_()
             a.record(stream)
@@ -363,6 +373,7 @@ def run_ours(args) -> None:
             exchange()
             b.record(stream)
         torch.cuda.synchronize()
+        clk.timed = False
         barrier()
     step_ms = [a.elapsed_time(b) for a, b in evs]
     ms = reduce_max(sum(step_ms) / len(step_ms))
@@ -487,8 +498,8 @@ def tlp_uses_tensor_attention(cls: str, w) -> bool:
 def main() -> None:
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
-    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
     ap.add_argument("--workload", default=WORKLOAD, choices=sorted(WORKLOADS))
     ap.add_argument("--no-cpu-baseline", action="store_true")

@@ -57,3 +57,47 @@ def allreduce_mean(grads: FlatGrads, group=None) -> None:
         return
     dist.all_reduce(grads.flat, op=dist.ReduceOp.SUM, group=group)
     grads.flat.mul_(1.0 / world)
+
+
+class GradExchanger:
+    """Per-layer gradient all-reduce overlapped with the rest of a backward
+    pass: `submit(grads)` right after a layer's backward enqueues the mean
+    over ranks of that layer's flat buffer on a side stream that first waits
+    for the layer's kernels, so the collective runs while the next (lower)
+    layer's backward computes; `finish()` makes the caller's stream wait for
+    every submitted exchange.  Every rank must submit the same buffers in the
+    same order (in a stack with layer dropping the decisions are equal on all
+    ranks).  Without a process group of size > 1 both calls do nothing; CPU
+    tensors (gloo) are reduced synchronously."""
+
+    def __init__(self, group=None):
+        self.group = group
+        self.world = (dist.get_world_size(group) if dist.is_available() and dist.is_initialized() else 1)
+        self.stream = None
+        self.pending = 0
+
+    def submit(self, grads: FlatGrads, stream=None) -> None:
+        """`stream`: the stream the layer's backward was enqueued on (None:
+        the current stream)."""
+        if self.world == 1:
+            return
+        t = grads.flat
+        if t.device.type != "cuda":
+            dist.all_reduce(t, op=dist.ReduceOp.SUM, group=self.group)
+            t.mul_(1.0 / self.world)
+            return
+        if self.stream is None:
+            self.stream = torch.cuda.Stream(device=t.device)
+        ev = torch.cuda.Event()
+        ev.record(stream if stream is not None else torch.cuda.current_stream(t.device))
+        self.stream.wait_event(ev)
+        with torch.cuda.stream(self.stream):
+            dist.all_reduce(t, op=dist.ReduceOp.SUM, group=self.group)
+            t.mul_(1.0 / self.world)
+        self.pending += 1
+
+    def finish(self, stream=None) -> None:
+        """Makes `stream` (None: the current stream) wait for the exchanges."""
+        if self.stream is not None and self.pending:
+            (stream if stream is not None else torch.cuda.current_stream(self.stream.device)).wait_stream(self.stream)
+        self.pending = 0

@@ -14,12 +14,19 @@ shares the seed and the step.  A skipped layer gets no gradients (None).
 
 Every layer's output and input gradient live in buffers of their own, so
 the inputs each layer's backward needs stay valid through the step.
+
+Data parallelism: with a process group of size > 1, `backward(...,
+exchange=True)` averages each layer's gradients over the ranks as soon as
+that layer's backward is enqueued, on a side stream, so the collective
+overlaps the backward of the layers below it (one bucket per layer, the
+layer's flat float32 gradient buffer).
 """
 from __future__ import annotations
 
 import torch
 
 from . import Layer, pld_keep, pld_theta
+from .dp import FlatGrads, GradExchanger
 
 
 class EncoderStack:
@@ -38,6 +45,8 @@ class EncoderStack:
         self.pre_layer_norm = pre_layer_norm
         self.layers = [Layer(batch, seq, hidden, heads, ffn, attn_dropout, hidden_dropout, pre_layer_norm, seed,
                              dtype=dtype, philox_offset=l, **options) for l in range(num_layers)]
+        self.ffn = self.layers[0].ffn
+        self.grads = [FlatGrads(hidden, self.ffn, self.device) for _ in range(num_layers)]
         self.ys = [torch.empty(self.shape, dtype=dtype, device=self.device) for _ in range(num_layers)]
         self.dxs = [torch.empty(self.shape, dtype=dtype, device=self.device) for _ in range(num_layers)]
         self.inputs: list = [None] * num_layers
@@ -64,20 +73,28 @@ class EncoderStack:
                 h = layer.forward(h, mask, weights[l], y=self.ys[l], stream=stream)
         return h
 
-    def backward(self, dy: torch.Tensor, weights: list, grads: list | None = None, stream=None):
+    def backward(self, dy: torch.Tensor, weights: list, exchange: bool = False, stream=None):
         """Backward of the last forward, layers in reverse.  Returns (dx,
-        grads) with grads[l] a dict of float32 gradients for a layer that ran
-        and None for a skipped one.  `grads`, when given, holds the
-        destination dicts (entries of skipped layers are left untouched)."""
+        grads) with grads[l] a dict of float32 gradients (views of the stack's
+        per-layer flat buffer, overwritten by the next backward) for a layer
+        that ran and None for a skipped one.  With `exchange`, each layer's
+        gradients are averaged over the data-parallel ranks (see the module
+        docstring); they are final once the caller's stream reaches the end
+        of this call's work."""
         out = [None] * self.num_layers
+        ex = GradExchanger() if exchange else None
         g = dy
         for l in reversed(range(self.num_layers)):
             self.dys[l] = g
             if not self.keep[l]:
                 continue
             x_in = None if (self.normalize_invertible and self.pre_layer_norm) else self.inputs[l]
-            dst = None if grads is None else grads[l]
-            g, out[l] = self.layers[l].backward(x_in, g, weights[l], grads=dst, dx=self.dxs[l], stream=stream)
+            g, out[l] = self.layers[l].backward(x_in, g, weights[l], grads=self.grads[l].as_dict(), dx=self.dxs[l],
+                                                stream=stream)
+            if ex is not None:
+                ex.submit(self.grads[l], stream)
+        if ex is not None:
+            ex.finish(stream)
         return g, out
 
     def close(self) -> None:
