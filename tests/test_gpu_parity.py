@@ -149,3 +149,25 @@ def test_gelu_tanh_checkpoint_is_bitwise_identical():
     assert np.array_equal(a["y"], b["y"]) and np.array_equal(a["dx"], b["dx"])
     for n in a["grads"]:
         assert np.array_equal(a["grads"][n], b["grads"][n]), n
+
+
+def _sampled_full_size(w: Workload, idx):
+    """Whole-batch run on the GPU at the workload's full size; y and dx of the
+    sampled sequences against the oracle run on those sequences alone (their
+    global indices fix their dropout bits)."""
+    inp = make_inputs(w)
+    gpu = run_gpu(inp)
+    idx = np.asarray(idx)
+    pure = run_oracle(inp, seq_index=idx)
+    rounded = run_oracle(inp, storage_rounded=True, seq_index=idx)
+    from parity import check_tensor
+    check_tensor("y", gpu["y"][idx], pure["y"], rounded["y"], w.dtype, True)
+    check_tensor("dx", gpu["dx"][idx], pure["dx"], rounded["dx"], w.dtype, True)
+
+
+def test_bert_large_f16_full_batch_sampled_sequences():
+    _sampled_full_size(WORKLOADS["bert-large-f16"], [0, 37, 63])
+
+
+def test_long_post_ln_bf16_full_batch_sampled_sequences():
+    _sampled_full_size(WORKLOADS["long-postln-bf16"], [1, 3])

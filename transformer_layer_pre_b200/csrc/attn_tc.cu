@@ -133,6 +133,8 @@ __global__ void __launch_bounds__(kFwdThreads)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tslot;
+  pdl_wait();
+  pdl_launch_dependents();
   const uint32_t tS = tmem, tO = tmem + 128;
 
   if (warp == 0) {
@@ -382,6 +384,8 @@ __global__ void __launch_bounds__(kBwdThreads)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tslot;
+  pdl_wait();
+  pdl_launch_dependents();
   const uint32_t tS = tmem, tdP = tmem + 128, tdV = tmem + 256, tdK = tmem + 320, tdQ = tmem + 384;
 
   if (warp == 0) {
@@ -552,6 +556,8 @@ __global__ void __launch_bounds__(kBwdThreads)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tslot;
+  pdl_wait();
+  pdl_launch_dependents();
   const uint32_t tS = tmem, tdP = tmem + 128, tdQ = tmem + 256;
 
   if (warp == 0) {
@@ -702,7 +708,9 @@ __global__ void __launch_bounds__(kPFwdThreads, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  const uint32_t tmem = *tslot;   // S[j] at 128*j, O[j] at 256 + 64*j
+  const uint32_t tmem = *tslot;
+  pdl_wait();
+  pdl_launch_dependents();   // S[j] at 128*j, O[j] at 256 + 64*j
 
   if (warp == 0) {
     if (lane == 0) {
@@ -923,6 +931,8 @@ __global__ void __launch_bounds__(kPBwdThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tslot;
+  pdl_wait();
+  pdl_launch_dependents();
   const uint32_t tS = tmem, tdP = tmem + 128, tdV = tmem + 256, tdK = tmem + 320, tdQ = tmem + 384;
 
   if (warp == 0) {
@@ -1178,10 +1188,10 @@ void fwd_t(const AttnArgs& a, cudaStream_t s) {
     int nsm = 148;
     cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, 0);
     const int grid = std::min(a.B * a.nh, nsm);
-    attn_fwd_tc_persist<T><<<grid, kPFwdThreads, kPFwdSmem, s>>>(mq, mk, mv, t);
+    launch_pdl(attn_fwd_tc_persist<T>, grid, kPFwdThreads, kPFwdSmem, s, mq, mk, mv, t);
   } else {
     dim3 grid((a.S + TILE - 1) / TILE, a.nh, a.B);
-    attn_fwd_tc<T><<<grid, kFwdThreads, kFwdSmem, s>>>(mq, mk, mv, t);
+    launch_pdl(attn_fwd_tc<T>, grid, kFwdThreads, kFwdSmem, s, mq, mk, mv, t);
   }
   count_launch();
 }
@@ -1206,7 +1216,7 @@ void bwd_t(const AttnArgs& a, cudaStream_t s) {
   if (ntile == 1) {
     int nsm = 148;
     cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, 0);
-    attn_bwd_tc_persist<T><<<std::min(a.B * a.nh, nsm), kPBwdThreads, kPBwdSmem, s>>>(mq, mk, mv, mdo, t);
+    launch_pdl(attn_bwd_tc_persist<T>, std::min(a.B * a.nh, nsm), kPBwdThreads, kPBwdSmem, s, mq, mk, mv, mdo, t);
     count_launch();
     return;
   }
@@ -1214,10 +1224,10 @@ void bwd_t(const AttnArgs& a, cudaStream_t s) {
   t.dvec = a.dvec;
   t.fuse_dq = 0;
   dim3 grid(ntile, a.nh, a.B);
-  attn_bwd_kv_tc<T><<<grid, kBwdThreads, kBwdKvSmem, s>>>(mq, mk, mv, mdo, t);
+  launch_pdl(attn_bwd_kv_tc<T>, grid, kBwdThreads, kBwdKvSmem, s, mq, mk, mv, mdo, t);
   count_launch();
   if (!t.fuse_dq) {
-    attn_bwd_q_tc<T><<<grid, kBwdThreads, kBwdQSmem, s>>>(mq, mk, mv, mdo, t);
+    launch_pdl(attn_bwd_q_tc<T>, grid, kBwdThreads, kBwdQSmem, s, mq, mk, mv, mdo, t);
     count_launch();
   }
 }

@@ -14,6 +14,18 @@ namespace tlp {
 typedef __half half_t;
 typedef __nv_bfloat16 bf16_t;
 
+// ------------------------------------------------------------------ programmatic dependent launch
+// Kernels of the layer are launched with programmatic stream serialization
+// (launch_pdl in kernels.h): a kernel may be scheduled while the previous
+// kernel of the stream is still finishing, runs its local setup (barriers,
+// tensor memory, descriptor prefetch), and then pdl_wait() blocks until that
+// previous kernel has completed and its memory is visible.  No global memory
+// is read or written before pdl_wait().  pdl_launch_dependents() lets the
+// next kernel start being scheduled (it still waits for this one to finish).
+// Both are no-ops for an ordinary launch.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 // ------------------------------------------------------------------ scalar conversion
 __device__ __forceinline__ float to_f(float v) { return v; }
 __device__ __forceinline__ float to_f(half_t v) { return __half2float(v); }
@@ -291,6 +303,24 @@ __device__ __forceinline__ float warp_sum(float v) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
   return v;
+}
+// Column sums of a warp's 32 x 32 block: v holds 32 values of this lane's
+// row; lane l returns the sum over the 32 lanes of v[l].  Recursive halving:
+// at each step a lane keeps one half of its values and adds the partner
+// lane's copy of that half (31 shuffles), in a fixed order.
+__device__ __forceinline__ float warp_colsum32(float (&v)[32]) {
+  const int lane = threadIdx.x & 31;
+#pragma unroll
+  for (int k = 16; k >= 1; k >>= 1) {
+    const bool upper = (lane & k) != 0;
+#pragma unroll
+    for (int i = 0; i < k; ++i) {
+      const float send = upper ? v[i] : v[i + k];
+      const float keep = upper ? v[i + k] : v[i];
+      v[i] = keep + __shfl_xor_sync(0xffffffffu, send, k);
+    }
+  }
+  return v[0];
 }
 __device__ __forceinline__ float warp_max(float v) {
 #pragma unroll

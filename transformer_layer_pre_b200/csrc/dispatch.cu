@@ -6,6 +6,8 @@ namespace tlp {
 
 void gemm_simt_run(int dtype, const GemmDesc& g, const EpiParams& e, cudaStream_t s);
 int gemm_tc_run(int dtype, const GemmDesc& g, const EpiParams& e, cudaStream_t s);
+int gemm_tc_run2(int dtype, const GemmDesc& ga, const EpiParams& ea, const GemmDesc& gb, const EpiParams& eb,
+                 cudaStream_t s);
 size_t gemm_tc_splitk_ws_floats(int M, int N, int K);
 int gemm_tc_take_error();
 
@@ -17,6 +19,16 @@ int gemm_run(int dtype, const GemmDesc& g, const EpiParams& e, cudaStream_t s) {
     return 0;
   }
   return gemm_tc_run(dtype, g, e, s);
+}
+
+int gemm_run2(int dtype, const GemmDesc& ga, const EpiParams& ea, const GemmDesc& gb, const EpiParams& eb,
+              cudaStream_t s) {
+  if (dtype == DT_F32) {
+    gemm_simt_run(dtype, ga, ea, s);
+    gemm_simt_run(dtype, gb, eb, s);
+    return 0;
+  }
+  return gemm_tc_run2(dtype, ga, ea, gb, eb, s);
 }
 
 size_t gemm_splitk_ws_floats(int dtype, int M, int N, int K) {

@@ -12,7 +12,7 @@
 //                     guide", Step 2 hidden_dropout_ratio).
 //  EPI_BIAS_GELU      U = acc + bias stored; G = GELU(U as stored) so that a
 //                     backward that recomputes G from U gets identical bits
-//                     (erf form, or the tanh form when e.gelu_tanh).
+//                     (erf form, or the tanh form for KIND | EPI_TANH).
 //  EPI_DGELU          out = acc * GELU'(U).
 //  EPI_STORE          out = acc (+ res).
 //  EPI_F32            float32 out = acc.
@@ -26,9 +26,16 @@
 
 namespace tlp {
 
+// Flag bit on a kernel's compile-time epilogue kind: GELU (EPI_BIAS_GELU,
+// EPI_DGELU) in its tanh form (EpiParams.gelu_tanh at run time).  The low
+// bits are the EpiKind.
+constexpr int EPI_TANH = 16;
+constexpr int epi_base(int kind) { return kind & (EPI_TANH - 1); }
+
 // Whether a kind reads a per-element auxiliary input (and which pointer).
 template <int KIND> struct EpiAux {
-  static constexpr bool kNeeds = KIND == EPI_BIAS_DROP_RES || KIND == EPI_DGELU || KIND == EPI_STORE;
+  static constexpr bool kNeeds =
+      epi_base(KIND) == EPI_BIAS_DROP_RES || epi_base(KIND) == EPI_DGELU || epi_base(KIND) == EPI_STORE;
 };
 __device__ __forceinline__ const void* epi_aux_ptr(const EpiParams& e, int kind) {
   return kind == EPI_DGELU ? e.aux : e.res;
@@ -44,16 +51,16 @@ __device__ __forceinline__ size_t qkv_row_base(const EpiParams& e, int m) {
 template <typename T, int KIND>
 __device__ __forceinline__ void epi_apply8(const EpiParams& e, int m, int n, float (&v)[8], const float (&aux)[8],
                                            size_t row_base) {
-  if constexpr (KIND == EPI_F32) {
+  if constexpr (epi_base(KIND) == EPI_F32) {
     float* o = static_cast<float*>(e.out) + (size_t)m * e.ldo + n;
     store8<float>(o, v);
-  } else if constexpr (KIND == EPI_STORE) {
+  } else if constexpr (epi_base(KIND) == EPI_STORE) {
     if (e.res) {
 #pragma unroll
       for (int i = 0; i < 8; ++i) v[i] += aux[i];
     }
     store8<T>(static_cast<T*>(e.out) + (size_t)m * e.ldo + n, v);
-  } else if constexpr (KIND == EPI_QKV) {
+  } else if constexpr (epi_base(KIND) == EPI_QKV) {
     float b[8];
     load8<T>(static_cast<const T*>(e.bias) + n, b);
 #pragma unroll
@@ -66,7 +73,7 @@ __device__ __forceinline__ void epi_apply8(const EpiParams& e, int m, int n, flo
     const int lane = c & (e.head_dim - 1);
     const size_t dst = (size_t)which * e.tokens * e.hidden + row_base + ((size_t)h * e.seq << sh) + lane;
     store8<T>(static_cast<T*>(e.out) + dst, v);
-  } else if constexpr (KIND == EPI_BIAS_DROP_RES) {
+  } else if constexpr (epi_base(KIND) == EPI_BIAS_DROP_RES) {
     float b[8];
     load8<T>(static_cast<const T*>(e.bias) + n, b);
     uint32_t bits = 0xFFu;
@@ -75,18 +82,18 @@ __device__ __forceinline__ void epi_apply8(const EpiParams& e, int m, int n, flo
 #pragma unroll
     for (int i = 0; i < 8; ++i) v[i] = aux[i] + (((bits >> i) & 1u) ? (v[i] + b[i]) * sc : 0.0f);
     store8<T>(static_cast<T*>(e.out) + (size_t)m * e.ldo + n, v);
-  } else if constexpr (KIND == EPI_BIAS_GELU) {
+  } else if constexpr (epi_base(KIND) == EPI_BIAS_GELU) {
     float b[8];
     load8<T>(static_cast<const T*>(e.bias) + n, b);
 #pragma unroll
     for (int i = 0; i < 8; ++i) v[i] = round_f<T>(v[i] + b[i]);
     store8<T>(static_cast<T*>(e.out) + (size_t)m * e.ldo + n, v);
     if (e.out2) {
-      gelu8_form(v, e.gelu_tanh != 0);
+      gelu8_form(v, (KIND & EPI_TANH) != 0);
       store8<T>(static_cast<T*>(e.out2) + (size_t)m * e.ldo + n, v);
     }
-  } else if constexpr (KIND == EPI_DGELU) {
-    mul_gelu_grad8_form(v, aux, e.gelu_tanh != 0);
+  } else if constexpr (epi_base(KIND) == EPI_DGELU) {
+    mul_gelu_grad8_form(v, aux, (KIND & EPI_TANH) != 0);
     store8<T>(static_cast<T*>(e.out) + (size_t)m * e.ldo + n, v);
   }
 }
@@ -97,17 +104,17 @@ __device__ __forceinline__ void epi_apply8(const EpiParams& e, int m, int n, flo
 template <typename T, int KIND>
 __device__ __forceinline__ void epi_compute8(const EpiParams& e, int m, int n, float (&v)[8], float (&v2)[8],
                                              const float (&aux)[8]) {
-  if constexpr (KIND == EPI_STORE) {
+  if constexpr (epi_base(KIND) == EPI_STORE) {
     if (e.res) {
 #pragma unroll
       for (int i = 0; i < 8; ++i) v[i] += aux[i];
     }
-  } else if constexpr (KIND == EPI_QKV) {
+  } else if constexpr (epi_base(KIND) == EPI_QKV) {
     float b[8];
     load8<T>(static_cast<const T*>(e.bias) + n, b);
 #pragma unroll
     for (int i = 0; i < 8; ++i) v[i] += b[i];
-  } else if constexpr (KIND == EPI_BIAS_DROP_RES) {
+  } else if constexpr (epi_base(KIND) == EPI_BIAS_DROP_RES) {
     float b[8];
     load8<T>(static_cast<const T*>(e.bias) + n, b);
     uint32_t bits = 0xFFu;
@@ -115,7 +122,7 @@ __device__ __forceinline__ void epi_compute8(const EpiParams& e, int m, int n, f
     const float sc = e.drop.thr ? e.drop.scale : 1.0f;
 #pragma unroll
     for (int i = 0; i < 8; ++i) v[i] = aux[i] + (((bits >> i) & 1u) ? (v[i] + b[i]) * sc : 0.0f);
-  } else if constexpr (KIND == EPI_BIAS_GELU) {
+  } else if constexpr (epi_base(KIND) == EPI_BIAS_GELU) {
     float b[8];
     load8<T>(static_cast<const T*>(e.bias) + n, b);
 #pragma unroll
@@ -123,9 +130,9 @@ __device__ __forceinline__ void epi_compute8(const EpiParams& e, int m, int n, f
       v[i] = round_f<T>(v[i] + b[i]);
       v2[i] = v[i];
     }
-    gelu8_form(v2, e.gelu_tanh != 0);
-  } else if constexpr (KIND == EPI_DGELU) {
-    mul_gelu_grad8_form(v, aux, e.gelu_tanh != 0);
+    gelu8_form(v2, (KIND & EPI_TANH) != 0);
+  } else if constexpr (epi_base(KIND) == EPI_DGELU) {
+    mul_gelu_grad8_form(v, aux, (KIND & EPI_TANH) != 0);
   }
 }
 
@@ -134,11 +141,11 @@ template <typename T, int KIND>
 __device__ __forceinline__ void epi_apply8(const EpiParams& e, int m, int n, float (&v)[8]) {
   float aux[8] = {0, 0, 0, 0, 0, 0, 0, 0};
   if constexpr (EpiAux<KIND>::kNeeds) {
-    const void* p = epi_aux_ptr(e, KIND);
+    const void* p = epi_aux_ptr(e, epi_base(KIND));
     if (p) load8<T>(static_cast<const T*>(p) + (size_t)m * e.ldo + n, aux);
   }
   size_t rb = 0;
-  if constexpr (KIND == EPI_QKV) rb = qkv_row_base(e, m);
+  if constexpr (epi_base(KIND) == EPI_QKV) rb = qkv_row_base(e, m);
   epi_apply8<T, KIND>(e, m, n, v, aux, rb);
 }
 

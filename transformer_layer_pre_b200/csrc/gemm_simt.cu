@@ -75,8 +75,14 @@ void launch(const GemmDesc& g, const EpiParams& e, cudaStream_t s) {
   switch (e.kind) {
     case EPI_QKV: gemm_simt_kernel<T, EPI_QKV><<<grid, 256, 0, s>>>(g, e); break;
     case EPI_BIAS_DROP_RES: gemm_simt_kernel<T, EPI_BIAS_DROP_RES><<<grid, 256, 0, s>>>(g, e); break;
-    case EPI_BIAS_GELU: gemm_simt_kernel<T, EPI_BIAS_GELU><<<grid, 256, 0, s>>>(g, e); break;
-    case EPI_DGELU: gemm_simt_kernel<T, EPI_DGELU><<<grid, 256, 0, s>>>(g, e); break;
+    case EPI_BIAS_GELU:
+      if (e.gelu_tanh) gemm_simt_kernel<T, EPI_BIAS_GELU | EPI_TANH><<<grid, 256, 0, s>>>(g, e);
+      else gemm_simt_kernel<T, EPI_BIAS_GELU><<<grid, 256, 0, s>>>(g, e);
+      break;
+    case EPI_DGELU:
+      if (e.gelu_tanh) gemm_simt_kernel<T, EPI_DGELU | EPI_TANH><<<grid, 256, 0, s>>>(g, e);
+      else gemm_simt_kernel<T, EPI_DGELU><<<grid, 256, 0, s>>>(g, e);
+      break;
     case EPI_STORE: gemm_simt_kernel<T, EPI_STORE><<<grid, 256, 0, s>>>(g, e); break;
     case EPI_F32: gemm_simt_kernel<T, EPI_F32><<<grid, 256, 0, s>>>(g, e); break;
   }

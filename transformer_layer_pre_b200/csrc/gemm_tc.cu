@@ -29,6 +29,7 @@
 #include <algorithm>
 #include <cstring>
 #include <type_traits>
+#include <vector>
 
 #include "epilogue.cuh"
 #include "kernels.h"
@@ -103,6 +104,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tslot;
   const int total = g.tiles_m * g.tiles_n * g.splits;
+  pdl_wait();
+  pdl_launch_dependents();
 
   if (warp == 0) {
     if (lane == 0) {
@@ -205,7 +208,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       // the accumulator is ready, so their latency hides under the main loop
       uint4 pre[EpiAux<KIND>::kNeeds ? CW / 8 : 1];
       if constexpr (EpiAux<KIND>::kNeeds) {
-        const T* ap = static_cast<const T*>(epi_aux_ptr(e, KIND));
+        const T* ap = static_cast<const T*>(epi_aux_ptr(e, epi_base(KIND)));
 #pragma unroll
         for (int j = 0; j < CW / 8; ++j) {
           const int n = nbase + j * 8;
@@ -214,11 +217,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       size_t rb = 0;
-      if constexpr (KIND == EPI_QKV) rb = mrow ? qkv_row_base(e, m) : 0;
+      if constexpr (epi_base(KIND) == EPI_QKV) rb = mrow ? qkv_row_base(e, m) : 0;
       if (!mbar_wait_warp(&tfull[acc], aph, g.err, 4)) break;
       tc_fence_after();
       EpiParams ep = e;
-      if constexpr (KIND == EPI_F32) ep.out = static_cast<float*>(e.out) + (size_t)sp * g.split_stride;
+      if constexpr (epi_base(KIND) == EPI_F32) ep.out = static_cast<float*>(e.out) + (size_t)sp * g.split_stride;
       const uint32_t tbase = tmem + ((uint32_t)(quarter * 32) << 16) + acc * BN + part * CW;
 #pragma unroll
       for (int c0 = 0; c0 < CW; c0 += 32) {
@@ -277,10 +280,197 @@ struct OutMaps {
   int split_rows;     // EPI_F32: rows between split partials (M rounded up to 256)
 };
 
+// One GEMM of a pair launch: operand maps, output maps, sizes, epilogue.
+struct PairGemm {
+  CUtensorMap tmA, tmB;
+  OutMaps om;
+  TcArgs g;
+  EpiParams e;
+};
+
+// Which output tiles each CTA pair computes, in order.  Round-robin (one
+// GEMM): pair c takes tiles c, c + pairs, ...  Table (two GEMMs in one
+// launch, e.g. a weight gradient and an input gradient that read the same
+// operand): entry = gemm * 32768 + tile, planned on the host so that every
+// pair gets about the same number of K blocks (longest tiles first, each to
+// the pair that frees up first), which fills the pairs a lone GEMM would
+// leave idle in its last wave.
+constexpr int kMaxPairs = 80;
+constexpr int kMaxItems = 24;
+struct PairSched {
+  int table;
+  uint16_t n[kMaxPairs];
+  uint16_t item[kMaxPairs][kMaxItems];
+};
+
+template <bool GROUP>
+struct SchedIter {
+  const PairSched& s;
+  int cid, i, t, step, total;
+  __device__ SchedIter(const PairSched& s_, const TcArgs& g0, int cid_, int ncl)
+      : s(s_), cid(cid_), i(0), t(cid_), step(ncl), total(g0.tiles_m * g0.tiles_n * g0.splits) {}
+  __device__ bool next(int& gi, int& tile) {
+    if (!GROUP || !s.table) {
+      if (t >= total) return false;
+      gi = 0;
+      tile = t;
+      t += step;
+      return true;
+    }
+    if (i >= s.n[cid]) return false;
+    const int v = s.item[cid][i++];
+    gi = v >> 15;
+    tile = v & 32767;
+    return true;
+  }
+};
+
+// Epilogue of one tile for epilogue warp (quarter, part) of this CTA:
+// TMEM accumulator `acc` -> fused epilogue -> staging box -> TMA store.
 template <typename T, int KIND>
+__device__ __forceinline__ bool pair_epilogue_tile(const OutMaps& om, const TcArgs& g, const EpiParams& e, int t,
+                                                   int rank, int quarter, int part, int lane, uint32_t tmem, int acc,
+                                                   uint32_t aph, uint64_t* tfull,
+                                                   const uint32_t (&tempty_leader)[2], uint8_t* stage0, int& nbuf) {
+  constexpr int BN = 256;
+  constexpr int HALF = 128;
+  constexpr int CW = BN / (kPairEpiWarps / 4);              // 64 columns per warp
+  constexpr int OUT_ES = epi_base(KIND) == EPI_F32 ? 4 : 2;
+  constexpr int SW = 64 / OUT_ES;                          // columns per staging box: 32 (16-bit) or 16 (fp32)
+  constexpr int NOUT = epi_base(KIND) == EPI_BIAS_GELU ? 2 : 1;
+  const int swz = (lane >> 1) & 3;                         // 64-byte swizzle of this lane's staging row
+  int mb, nb, sp;
+  decode_tile(g, t, mb, nb, sp);
+  const int mrow0 = mb * 256 + rank * HALF + quarter * 32;   // first row of this warp's boxes
+  const int m = mrow0 + lane;
+  const int nbase = nb * BN + part * CW;
+  const bool mrow = m < g.M;
+  uint4 pre[EpiAux<KIND>::kNeeds ? CW / 8 : 1];
+  if constexpr (EpiAux<KIND>::kNeeds) {
+    const T* ap = static_cast<const T*>(epi_aux_ptr(e, epi_base(KIND)));
+#pragma unroll
+    for (int j = 0; j < CW / 8; ++j) {
+      const int n = nbase + j * 8;
+      pre[j] = (ap && mrow && n < g.N) ? *reinterpret_cast<const uint4*>(ap + (size_t)m * e.ldo + n)
+                                        : make_uint4(0u, 0u, 0u, 0u);
+    }
+  }
+  if (!mbar_wait_warp(&tfull[acc], aph, g.err, 44)) return false;
+  tc_fence_after();
+  const uint32_t tbase = tmem + ((uint32_t)(quarter * 32) << 16) + acc * BN + part * CW;
+#pragma unroll
+  for (int c0 = 0; c0 < CW; c0 += SW) {
+    float v[SW];
+    if constexpr (SW == 32) tmem_ld32(tbase + c0, *reinterpret_cast<float(*)[32]>(v));
+    else tmem_ld16(tbase + c0, *reinterpret_cast<float(*)[16]>(v));
+    if (c0 + SW == CW) {
+      // last TMEM read of this tile: hand the accumulator back to the leader
+      tc_fence_before();
+      mbar_arrive_cluster(tempty_leader[acc]);
+    }
+    uint8_t* sb0 = stage0 + (NOUT == 2 ? 0 : nbuf) * kStageOut;
+    uint8_t* sb1 = stage0 + kStageOut;
+    if (lane == 0) {
+      if constexpr (NOUT == 2) bulk_wait_read<0>();
+      else bulk_wait_read<1>();
+    }
+    __syncwarp();
+    if constexpr (OUT_ES == 4) {
+      // 16 floats = four 16-byte chunks of the 64-byte row
+#pragma unroll
+      for (int q = 0; q < 4; ++q)
+        *reinterpret_cast<float4*>(sb0 + lane * 64 + ((q ^ swz) << 4)) =
+            make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+    } else {
+#pragma unroll
+      for (int q = 0; q < SW / 8; ++q) {
+        const int n = nbase + c0 + q * 8;
+        float* vq = v + q * 8;
+        float v2[8];
+        float aux[8];
+        if constexpr (EpiAux<KIND>::kNeeds) unpack8<T>(pre[(c0 >> 3) + q], aux);
+        else {
+#pragma unroll
+          for (int i = 0; i < 8; ++i) aux[i] = 0.0f;
+        }
+        if (mrow && n < g.N) epi_compute8<T, KIND>(e, m, n, *reinterpret_cast<float(*)[8]>(vq), v2, aux);
+        store8<T>(reinterpret_cast<T*>(sb0 + lane * 64 + ((q ^ swz) << 4)), *reinterpret_cast<float(*)[8]>(vq));
+        if constexpr (NOUT == 2) store8<T>(reinterpret_cast<T*>(sb1 + lane * 64 + ((q ^ swz) << 4)), v2);
+      }
+      if constexpr (epi_base(KIND) == EPI_DGELU && SW == 32) {
+        // bias gradient of the FFN1 Linear fused in: column sums of the
+        // stored (rounded) values of this warp's 32 rows
+        if (e.colsum) {
+          float cs[32];
+#pragma unroll
+          for (int i = 0; i < 32; ++i) cs[i] = (mrow && nbase + c0 + i < g.N) ? round_f<T>(v[i]) : 0.0f;
+          const float tot = warp_colsum32(cs);
+          const int col = nbase + c0 + lane;
+          if (col < g.N) e.colsum[(size_t)((mb * 2 + rank) * 4 + quarter) * g.N + col] = tot;
+        }
+      }
+    }
+    fence_proxy_async_smem();
+    __syncwarp();
+    if (lane == 0) {
+      const int x = nbase + c0;
+      if constexpr (epi_base(KIND) == EPI_QKV) {
+        if (mrow0 < g.M && x < g.N) {
+          const int which = (x >= e.hidden) + (x >= 2 * e.hidden);
+          const int c = x - which * e.hidden;
+          const int bb = mrow0 / e.seq, s0 = mrow0 - bb * e.seq;
+          const int y = which * om.qkv_heads_rows + (bb * e.heads + (c >> 6)) * e.seq + s0;
+          tma_store_2d(&om.out, sb0, c & 63, y);
+        }
+      } else if constexpr (epi_base(KIND) == EPI_F32) {
+        if (mrow0 < g.M && x < g.N) tma_store_2d(&om.out, sb0, x, sp * om.split_rows + mrow0);
+      } else if (mrow0 < g.M && x < g.N) {
+        tma_store_2d(&om.out, sb0, x, mrow0);
+        if constexpr (NOUT == 2) {
+          if (e.out2) tma_store_2d(&om.out2, sb1, x, mrow0);
+        }
+      }
+      bulk_commit();
+    }
+    if constexpr (NOUT == 1) nbuf ^= 1;
+  }
+  return true;
+}
+
+// Per-item scalars of whichever GEMM a scheduled tile belongs to.
+struct ItemArgs {
+  int tiles_m, tiles_n, kb_per_split, kblocks, a_mn, b_mn, bf16;
+};
+__device__ __forceinline__ ItemArgs item_args(const TcArgs& g0, const TcArgs& g1, int gi) {
+  ItemArgs a;
+  a.tiles_m = gi ? g1.tiles_m : g0.tiles_m;
+  a.tiles_n = gi ? g1.tiles_n : g0.tiles_n;
+  a.kb_per_split = gi ? g1.kb_per_split : g0.kb_per_split;
+  a.kblocks = gi ? g1.kblocks : g0.kblocks;
+  a.a_mn = gi ? g1.a_mn : g0.a_mn;
+  a.b_mn = gi ? g1.b_mn : g0.b_mn;
+  a.bf16 = gi ? g1.bf16 : g0.bf16;
+  return a;
+}
+__device__ __forceinline__ void decode_item(const ItemArgs& a, int t, int& mb, int& nb, int& kb0, int& kb1) {
+  const int per = a.tiles_m * a.tiles_n;
+  const int sp = t / per;
+  const int r = t - sp * per;
+  mb = r / a.tiles_n;
+  nb = r - mb * a.tiles_n;
+  kb0 = sp * a.kb_per_split;
+  kb1 = min(a.kblocks, kb0 + a.kb_per_split);
+}
+
+// Kernel parameters are per GEMM and by value (the scheduled item selects
+// scalars from them), so every access stays a parameter-space load.
+template <typename T, int KA, int KB>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
-    gemm_tc_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                        const __grid_constant__ OutMaps om, TcArgs g, EpiParams e) {
+    gemm_tc_pair_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUtensorMap tmB0,
+                        const __grid_constant__ OutMaps om0, const TcArgs g0, const EpiParams e0,
+                        const __grid_constant__ CUtensorMap tmA1, const __grid_constant__ CUtensorMap tmB1,
+                        const __grid_constant__ OutMaps om1, const TcArgs g1, const EpiParams e1,
+                        const __grid_constant__ PairSched sch) {
   constexpr int BN = 256;
   constexpr int HALF = 128;
   extern __shared__ uint8_t smem_raw[];
@@ -295,6 +485,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t rank = cluster_ctarank();
   const bool leader = rank == 0;
+  int* const err = g0.err;
   if (threadIdx.x == 0) {
     for (int s = 0; s < kPairStages; ++s) {
       mbar_init(&full[s], 1);
@@ -311,44 +502,52 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
   cluster_sync();
   tc_fence_after();
   const uint32_t tmem = *tslot;
-  const int cid = blockIdx.x >> 1, ncl = gridDim.x >> 1;
-  const int total = g.tiles_m * g.tiles_n * g.splits;   // tiles_m counts 256-row pair tiles
+  pdl_wait();
+  pdl_launch_dependents();
+  const int cid = blockIdx.x >> 1, ncl = gridDim.x >> 1;   // tiles_m counts 256-row pair tiles
 
   if (warp == 0) {
     if (lane == 0) {
-      prefetch_tensormap(&tmA);
-      prefetch_tensormap(&tmB);
+      prefetch_tensormap(&tmA0);
+      prefetch_tensormap(&tmB0);
+      if (sch.table) {
+        prefetch_tensormap(&tmA1);
+        prefetch_tensormap(&tmB1);
+      }
       int s = 0;
       uint32_t ph = 0;
       bool ok = true;
       uint32_t issued_phase[kPairStages];
       bool issued[kPairStages];
       for (int i = 0; i < kPairStages; ++i) issued[i] = false;
-      for (int t = cid; t < total && ok; t += ncl) {
-        int mb, nb, sp;
-        decode_tile(g, t, mb, nb, sp);
-        const int kb0 = sp * g.kb_per_split;
-        const int kb1 = min(g.kblocks, kb0 + g.kb_per_split);
+      SchedIter<KA != KB> it(sch, g0, cid, ncl);
+      int gi, t;
+      while (ok && it.next(gi, t)) {
+        const ItemArgs g = item_args(g0, g1, gi);
+        const CUtensorMap* mA = gi ? &tmA1 : &tmA0;
+        const CUtensorMap* mB = gi ? &tmB1 : &tmB0;
+        int mb, nb, kb0, kb1;
+        decode_item(g, t, mb, nb, kb0, kb1);
         const int m0 = mb * 256 + (int)rank * HALF;
         const int n0 = nb * BN + (int)rank * HALF;
         for (int kb = kb0; kb < kb1; ++kb) {
-          if (!mbar_wait(&empty[s], ph ^ 1u, g.err, 41)) { ok = false; break; }
+          if (!mbar_wait(&empty[s], ph ^ 1u, err, 41)) { ok = false; break; }
           uint8_t* a_dst = smem + s * kPairStageBytes;
           uint8_t* b_dst = a_dst + 128 * BK * 2;
           const uint32_t fb = mapa_shared(smem_u32(&full[s]), 0);
           if (leader) mbar_arrive_expect_tx(&full[s], 2 * kPairStageBytes);
           const int k0 = kb * BK;
           if (!g.a_mn) {
-            tma_load_2d_pair(a_dst, &tmA, fb, k0, m0);
+            tma_load_2d_pair(a_dst, mA, fb, k0, m0);
           } else {
-            tma_load_2d_pair(a_dst, &tmA, fb, m0, k0);
-            tma_load_2d_pair(a_dst + 8192, &tmA, fb, m0 + 64, k0);
+            tma_load_2d_pair(a_dst, mA, fb, m0, k0);
+            tma_load_2d_pair(a_dst + 8192, mA, fb, m0 + 64, k0);
           }
           if (!g.b_mn) {
-            tma_load_2d_pair(b_dst, &tmB, fb, k0, n0);
+            tma_load_2d_pair(b_dst, mB, fb, k0, n0);
           } else {
-            tma_load_2d_pair(b_dst, &tmB, fb, n0, k0);
-            tma_load_2d_pair(b_dst + 8192, &tmB, fb, n0 + 64, k0);
+            tma_load_2d_pair(b_dst, mB, fb, n0, k0);
+            tma_load_2d_pair(b_dst + 8192, mB, fb, n0 + 64, k0);
           }
           issued[s] = true;
           issued_phase[s] = ph;
@@ -362,22 +561,23 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
     }
   } else if (warp == 1) {
     if (lane == 0 && leader) {
-      const uint32_t idesc = idesc_f16(256, BN, g.bf16 != 0, g.a_mn != 0, g.b_mn != 0);
       int s = 0;
       uint32_t ph = 0;
       int acc = 0;
       uint32_t aph = 0;
       bool ok = true;
-      for (int t = cid; t < total && ok; t += ncl) {
-        int mb, nb, sp;
-        decode_tile(g, t, mb, nb, sp);
-        const int kb0 = sp * g.kb_per_split;
-        const int kb1 = min(g.kblocks, kb0 + g.kb_per_split);
-        if (!mbar_wait_cluster(&tempty[acc], aph ^ 1u, g.err, 42)) { ok = false; break; }
+      SchedIter<KA != KB> it(sch, g0, cid, ncl);
+      int gi, t;
+      while (ok && it.next(gi, t)) {
+        const ItemArgs g = item_args(g0, g1, gi);
+        const uint32_t idesc = idesc_f16(256, BN, g.bf16 != 0, g.a_mn != 0, g.b_mn != 0);
+        int mb, nb, kb0, kb1;
+        decode_item(g, t, mb, nb, kb0, kb1);
+        if (!mbar_wait_cluster(&tempty[acc], aph ^ 1u, err, 42)) { ok = false; break; }
         tc_fence_after();
         const uint32_t d = tmem + acc * BN;
         for (int kb = kb0; kb < kb1; ++kb) {
-          if (!mbar_wait(&full[s], ph, g.err, 43)) { ok = false; break; }
+          if (!mbar_wait(&full[s], ph, err, 43)) { ok = false; break; }
           tc_fence_after();
           const uint32_t a_base = smem_u32(smem + s * kPairStageBytes);
           const uint32_t b_base = a_base + 128 * BK * 2;
@@ -403,102 +603,26 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
     // this CTA's half tile) and a quarter of the 256 columns.  Results go
     // through a 64-byte-swizzled staging box (32 rows x 64 bytes) and leave by
     // TMA store, so global writes are whole lines.
-    constexpr int CW = BN / (kPairEpiWarps / 4);              // 64 columns per warp
-    constexpr int OUT_ES = KIND == EPI_F32 ? 4 : 2;
-    constexpr int SW = 64 / OUT_ES;                          // columns per staging box: 32 (16-bit) or 16 (fp32)
-    constexpr int NOUT = KIND == EPI_BIAS_GELU ? 2 : 1;
     const int quarter = warp & 3;
     const int part = (warp - 2) >> 2;
     uint8_t* stage0 = sout + (warp - 2) * 2 * kStageOut;
     const uint32_t tempty_leader[2] = {mapa_shared(smem_u32(&tempty[0]), 0), mapa_shared(smem_u32(&tempty[1]), 0)};
-    const int swz = (lane >> 1) & 3;                         // 64-byte swizzle of this lane's staging row
     int acc = 0;
     uint32_t aph = 0;
     int nbuf = 0;
-    for (int t = cid; t < total; t += ncl) {
-      int mb, nb, sp;
-      decode_tile(g, t, mb, nb, sp);
-      const int mrow0 = mb * 256 + (int)rank * HALF + quarter * 32;   // first row of this warp's boxes
-      const int m = mrow0 + lane;
-      const int nbase = nb * BN + part * CW;
-      const bool mrow = m < g.M;
-      uint4 pre[EpiAux<KIND>::kNeeds ? CW / 8 : 1];
-      if constexpr (EpiAux<KIND>::kNeeds) {
-        const T* ap = static_cast<const T*>(epi_aux_ptr(e, KIND));
-#pragma unroll
-        for (int j = 0; j < CW / 8; ++j) {
-          const int n = nbase + j * 8;
-          pre[j] = (ap && mrow && n < g.N) ? *reinterpret_cast<const uint4*>(ap + (size_t)m * e.ldo + n)
-                                            : make_uint4(0u, 0u, 0u, 0u);
-        }
-      }
-      if (!mbar_wait_warp(&tfull[acc], aph, g.err, 44)) break;
-      tc_fence_after();
-      const uint32_t tbase = tmem + ((uint32_t)(quarter * 32) << 16) + acc * BN + part * CW;
-#pragma unroll
-      for (int c0 = 0; c0 < CW; c0 += SW) {
-        float v[SW];
-        if constexpr (SW == 32) tmem_ld32(tbase + c0, *reinterpret_cast<float(*)[32]>(v));
-        else tmem_ld16(tbase + c0, *reinterpret_cast<float(*)[16]>(v));
-        if (c0 + SW == CW) {
-          // last TMEM read of this tile: hand the accumulator back to the leader
-          tc_fence_before();
-          mbar_arrive_cluster(tempty_leader[acc]);
-        }
-        uint8_t* sb0 = stage0 + (NOUT == 2 ? 0 : nbuf) * kStageOut;
-        uint8_t* sb1 = stage0 + kStageOut;
-        if (lane == 0) {
-          if constexpr (NOUT == 2) bulk_wait_read<0>();
-          else bulk_wait_read<1>();
-        }
-        __syncwarp();
-        if constexpr (OUT_ES == 4) {
-          // 16 floats = four 16-byte chunks of the 64-byte row
-#pragma unroll
-          for (int q = 0; q < 4; ++q)
-            *reinterpret_cast<float4*>(sb0 + lane * 64 + ((q ^ swz) << 4)) =
-                make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
-        } else {
-#pragma unroll
-          for (int q = 0; q < SW / 8; ++q) {
-            const int n = nbase + c0 + q * 8;
-            float* vq = v + q * 8;
-            float v2[8];
-            float aux[8];
-            if constexpr (EpiAux<KIND>::kNeeds) unpack8<T>(pre[(c0 >> 3) + q], aux);
-            else {
-#pragma unroll
-              for (int i = 0; i < 8; ++i) aux[i] = 0.0f;
-            }
-            if (mrow && n < g.N) epi_compute8<T, KIND>(e, m, n, *reinterpret_cast<float(*)[8]>(vq), v2, aux);
-            store8<T>(reinterpret_cast<T*>(sb0 + lane * 64 + ((q ^ swz) << 4)), *reinterpret_cast<float(*)[8]>(vq));
-            if constexpr (NOUT == 2) store8<T>(reinterpret_cast<T*>(sb1 + lane * 64 + ((q ^ swz) << 4)), v2);
-          }
-        }
-        fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) {
-          const int x = nbase + c0;
-          if constexpr (KIND == EPI_QKV) {
-            if (mrow0 < g.M && x < g.N) {
-              const int which = (x >= e.hidden) + (x >= 2 * e.hidden);
-              const int c = x - which * e.hidden;
-              const int bb = mrow0 / e.seq, s0 = mrow0 - bb * e.seq;
-              const int y = which * om.qkv_heads_rows + (bb * e.heads + (c >> 6)) * e.seq + s0;
-              tma_store_2d(&om.out, sb0, c & 63, y);
-            }
-          } else if constexpr (KIND == EPI_F32) {
-            if (mrow0 < g.M && x < g.N) tma_store_2d(&om.out, sb0, x, sp * om.split_rows + mrow0);
-          } else if (mrow0 < g.M && x < g.N) {
-            tma_store_2d(&om.out, sb0, x, mrow0);
-            if constexpr (NOUT == 2) {
-              if (e.out2) tma_store_2d(&om.out2, sb1, x, mrow0);
-            }
-          }
-          bulk_commit();
-        }
-        if constexpr (NOUT == 1) nbuf ^= 1;
-      }
+    SchedIter<KA != KB> it(sch, g0, cid, ncl);
+    int gi, t;
+    while (it.next(gi, t)) {
+      bool ok;
+      if constexpr (KA == KB)
+        ok = pair_epilogue_tile<T, KA>(om0, g0, e0, t, (int)rank, quarter, part, lane, tmem, acc, aph, tfull,
+                                       tempty_leader, stage0, nbuf);
+      else
+        ok = gi ? pair_epilogue_tile<T, KB>(om1, g1, e1, t, (int)rank, quarter, part, lane, tmem, acc, aph, tfull,
+                                            tempty_leader, stage0, nbuf)
+                : pair_epilogue_tile<T, KA>(om0, g0, e0, t, (int)rank, quarter, part, lane, tmem, acc, aph, tfull,
+                                            tempty_leader, stage0, nbuf);
+      if (!ok) break;
       acc ^= 1;
       if (acc == 0) aph ^= 1u;
     }
@@ -513,6 +637,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
 
 __global__ void splitk_reduce_kernel(const float* __restrict__ part, int splits, size_t stride, size_t n4,
                                      float* __restrict__ out) {
+  pdl_wait();
+  pdl_launch_dependents();
   for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n4; i += (size_t)gridDim.x * blockDim.x) {
     float4 s = reinterpret_cast<const float4*>(part)[i];
     for (int k = 1; k < splits; ++k) {
@@ -610,7 +736,7 @@ int launch_tc(const GemmDesc& gd, const EpiParams& e, int splits, cudaStream_t s
     cudaFuncSetAttribute(gemm_tc_kernel<T, BN, KIND>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
     attr = true;
   }
-  gemm_tc_kernel<T, BN, KIND><<<grid, kThreads, C::kSmem, s>>>(ma, mb, g, e);
+  launch_pdl(gemm_tc_kernel<T, BN, KIND>, grid, kThreads, C::kSmem, s, ma, mb, g, e);
   count_launch();
   return 0;
 }
@@ -619,19 +745,20 @@ bool aligned16(const void* p, int ld) {
   return (reinterpret_cast<uintptr_t>(p) & 15) == 0 && ((size_t)ld * 2) % 16 == 0;
 }
 
+// Fills the operand maps, output maps and sizes of one pair-kernel GEMM.
 template <typename T, int KIND>
-int launch_tc_pair(const GemmDesc& gd, const EpiParams& e, int splits, cudaStream_t s) {
+bool build_pair_gemm(PairGemm& P, const GemmDesc& gd, const EpiParams& e, int splits) {
   const bool bf16 = std::is_same<T, bf16_t>::value;
-  CUtensorMap ma, mb;
+  std::memset(&P, 0, sizeof(P));
   bool ok;
-  if (gd.a_kmajor) ok = make_map(&ma, gd.A, bf16, gd.K, gd.M, gd.lda, 128);
-  else ok = make_map(&ma, gd.A, bf16, gd.M, gd.K, gd.lda, 64);
+  if (gd.a_kmajor) ok = make_map(&P.tmA, gd.A, bf16, gd.K, gd.M, gd.lda, 128);
+  else ok = make_map(&P.tmA, gd.A, bf16, gd.M, gd.K, gd.lda, 64);
   if (ok) {
-    if (gd.b_kmajor) ok = make_map(&mb, gd.B, bf16, gd.K, gd.N, gd.ldb, 128);
-    else ok = make_map(&mb, gd.B, bf16, gd.N, gd.K, gd.ldb, 64);
+    if (gd.b_kmajor) ok = make_map(&P.tmB, gd.B, bf16, gd.K, gd.N, gd.ldb, 128);
+    else ok = make_map(&P.tmB, gd.B, bf16, gd.N, gd.K, gd.ldb, 64);
   }
-  if (!ok) return 1;
-  TcArgs g;
+  if (!ok) return false;
+  TcArgs& g = P.g;
   g.M = gd.M; g.N = gd.N; g.K = gd.K;
   g.a_mn = gd.a_kmajor ? 0 : 1;
   g.b_mn = gd.b_kmajor ? 0 : 1;
@@ -641,36 +768,96 @@ int launch_tc_pair(const GemmDesc& gd, const EpiParams& e, int splits, cudaStrea
   g.kblocks = (gd.K + BK - 1) / BK;
   g.kb_per_split = (g.kblocks + splits - 1) / splits;
   g.splits = (g.kblocks + g.kb_per_split - 1) / g.kb_per_split;
-  g.split_stride = (size_t)gd.M * gd.N;
   g.err = error_word();
-  OutMaps om;
-  std::memset(&om, 0, sizeof(om));
+  OutMaps& om = P.om;
   om.split_rows = g.tiles_m * 256;
   g.split_stride = (size_t)om.split_rows * gd.N;
-  bool okm;
   const CUtensorMapDataType t16 = bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
-  if constexpr (KIND == EPI_F32) {
+  if constexpr (epi_base(KIND) == EPI_F32) {
     // split partials live in a workspace padded to whole 256-row tiles; the
     // unsplit output is exactly M rows, so clipping keeps stores inside it
     const uint64_t rows = g.splits > 1 ? (uint64_t)g.splits * om.split_rows : (uint64_t)gd.M;
-    okm = make_map_t(&om.out, e.out, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, gd.N, rows, e.ldo, 32, 64);
-  } else if constexpr (KIND == EPI_QKV) {
+    ok = make_map_t(&om.out, e.out, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, gd.N, rows, e.ldo, 32, 64);
+  } else if constexpr (epi_base(KIND) == EPI_QKV) {
     om.qkv_heads_rows = e.tokens * (e.hidden / 64);
-    okm = make_map_t(&om.out, e.out, t16, 2, 64, (uint64_t)3 * om.qkv_heads_rows, 64, 32, 64);
+    ok = make_map_t(&om.out, e.out, t16, 2, 64, (uint64_t)3 * om.qkv_heads_rows, 64, 32, 64);
   } else {
-    okm = make_map_t(&om.out, e.out, t16, 2, gd.N, gd.M, e.ldo, 32, 64);
-    if (okm && KIND == EPI_BIAS_GELU && e.out2) okm = make_map_t(&om.out2, e.out2, t16, 2, gd.N, gd.M, e.ldo, 32, 64);
+    ok = make_map_t(&om.out, e.out, t16, 2, gd.N, gd.M, e.ldo, 32, 64);
+    if (ok && epi_base(KIND) == EPI_BIAS_GELU && e.out2) ok = make_map_t(&om.out2, e.out2, t16, 2, gd.N, gd.M, e.ldo, 32, 64);
   }
-  if (!okm) return 1;
-  const int total = g.tiles_m * g.tiles_n * g.splits;
-  const int grid = 2 * std::min(total, num_sms() / 2);
+  P.e = e;
+  return ok;
+}
+
+// Plans a table schedule for two GEMMs on `pairs` CTA pairs: tiles sorted by
+// their K blocks (longest first, then GEMM and tile order), each given to
+// the pair with the least work so far (lowest index on ties).  False if a
+// pair would get more than kMaxItems tiles.
+bool plan_pair_table(PairSched& sch, const TcArgs& g0, const TcArgs& g1, int pairs) {
+  struct Item { int kb, gi, tile; };
+  std::vector<Item> items;
+  for (int gi = 0; gi < 2; ++gi) {
+    const TcArgs& g = gi ? g1 : g0;
+    const int total = g.tiles_m * g.tiles_n * g.splits;
+    for (int t = 0; t < total; ++t) {
+      const int sp = t / (g.tiles_m * g.tiles_n);
+      const int kb0 = sp * g.kb_per_split;
+      items.push_back({std::min(g.kblocks, kb0 + g.kb_per_split) - kb0, gi, t});
+    }
+  }
+  if (items.empty() || items.size() > (size_t)pairs * kMaxItems) return false;
+  std::stable_sort(items.begin(), items.end(), [](const Item& a, const Item& b) { return a.kb > b.kb; });
+  std::memset(&sch, 0, sizeof(sch));
+  sch.table = 1;
+  std::vector<long long> load(pairs, 0);
+  for (const Item& it : items) {
+    int best = 0;
+    for (int p = 1; p < pairs; ++p)
+      if (load[p] < load[best]) best = p;
+    if (sch.n[best] >= kMaxItems || it.tile >= 32768) return false;
+    sch.item[best][sch.n[best]++] = (uint16_t)(it.gi * 32768 + it.tile);
+    load[best] += it.kb;
+  }
+  return true;
+}
+
+template <typename T, int KA, int KB>
+void launch_pair(const PairGemm& pa, const PairGemm& pb, const PairSched& sch, int grid, cudaStream_t s) {
   static bool attr = false;
   if (!attr) {
-    cudaFuncSetAttribute(gemm_tc_pair_kernel<T, KIND>, cudaFuncAttributeMaxDynamicSharedMemorySize, kPairSmem);
+    cudaFuncSetAttribute(gemm_tc_pair_kernel<T, KA, KB>, cudaFuncAttributeMaxDynamicSharedMemorySize, kPairSmem);
     attr = true;
   }
-  gemm_tc_pair_kernel<T, KIND><<<grid, kPairThreads, kPairSmem, s>>>(ma, mb, om, g, e);
+  launch_pdl(gemm_tc_pair_kernel<T, KA, KB>, grid, kPairThreads, kPairSmem, s, pa.tmA, pa.tmB, pa.om, pa.g, pa.e,
+             pb.tmA, pb.tmB, pb.om, pb.g, pb.e, sch);
   count_launch();
+}
+
+template <typename T, int KIND>
+int launch_tc_pair(const GemmDesc& gd, const EpiParams& e, int splits, cudaStream_t s) {
+  PairGemm P;
+  PairSched sch;
+  if (!build_pair_gemm<T, KIND>(P, gd, e, splits)) return 1;
+  std::memset(&sch, 0, sizeof(sch));   // round-robin
+  const int total = P.g.tiles_m * P.g.tiles_n * P.g.splits;
+  launch_pair<T, KIND, KIND>(P, P, sch, 2 * std::min(total, num_sms() / 2), s);
+  return 0;
+}
+
+// Two independent GEMMs in one launch on a planned table (falls back to two
+// launches when the plan does not fit the table).
+template <typename T, int KA, int KB>
+int launch_tc_pair_group(const GemmDesc& ga, const EpiParams& ea, int splits_a, const GemmDesc& gb,
+                         const EpiParams& eb, cudaStream_t s) {
+  PairGemm A, B;
+  PairSched sch;
+  if (!build_pair_gemm<T, KA>(A, ga, ea, splits_a) || !build_pair_gemm<T, KB>(B, gb, eb, 1)) return 1;
+  const int pairs = std::min(num_sms() / 2, kMaxPairs);
+  if (!plan_pair_table(sch, A.g, B.g, pairs)) {
+    int rc = launch_tc_pair<T, KA>(ga, ea, splits_a, s);
+    return rc ? rc : launch_tc_pair<T, KB>(gb, eb, 1, s);
+  }
+  launch_pair<T, KA, KB>(A, B, sch, 2 * pairs, s);
   return 0;
 }
 
@@ -683,25 +870,37 @@ int splitk_count_pair(int M, int N, int K) {
   return std::max(1, std::min(std::min(4, kblocks / 8), clusters / tiles));
 }
 
+// Split count and workspace use of a float32 weight-gradient GEMM.
+int f32_splits(const GemmDesc& g) {
+  const size_t rows_pad = (size_t)((g.M + 255) / 256) * 256;
+  int splits = g.splitk_ws ? splitk_count_pair(g.M, g.N, g.K) : 1;
+  while (splits > 1 && (size_t)splits * rows_pad * g.N > g.splitk_ws_floats) --splits;
+  return splits;
+}
+
+// Sums the split partials of a float32 GEMM in split order into e.out.
+void f32_split_reduce(const GemmDesc& g, const EpiParams& e, int splits, cudaStream_t s) {
+  const size_t rows_pad = (size_t)((g.M + 255) / 256) * 256;
+  const int kblocks = (g.K + BK - 1) / BK;
+  const int kb_per = (kblocks + splits - 1) / splits;
+  const int real = (kblocks + kb_per - 1) / kb_per;
+  const size_t n4 = (size_t)g.M * g.N / 4;
+  launch_pdl(splitk_reduce_kernel, (int)std::min<size_t>((n4 + 255) / 256, 148 * 8), 256, 0, s,
+             static_cast<const float*>(g.splitk_ws), real, rows_pad * g.N, n4, static_cast<float*>(e.out));
+  count_launch();
+}
+
 template <typename T>
 int run_t(const GemmDesc& g, const EpiParams& e, cudaStream_t s) {
   if (!aligned16(g.A, g.lda) || !aligned16(g.B, g.ldb)) return 2;
   if (e.kind == EPI_F32) {
-    const size_t rows_pad = (size_t)((g.M + 255) / 256) * 256;
-    int splits = g.splitk_ws ? splitk_count_pair(g.M, g.N, g.K) : 1;
-    while (splits > 1 && (size_t)splits * rows_pad * g.N > g.splitk_ws_floats) --splits;
+    const int splits = f32_splits(g);
     if (splits > 1) {
       EpiParams ep = e;
       ep.out = g.splitk_ws;
-      const int kblocks = (g.K + BK - 1) / BK;
-      const int kb_per = (kblocks + splits - 1) / splits;
-      const int real = (kblocks + kb_per - 1) / kb_per;
       int rc = launch_tc_pair<T, EPI_F32>(g, ep, splits, s);
       if (rc) return rc;
-      const size_t n4 = (size_t)g.M * g.N / 4;
-      splitk_reduce_kernel<<<(int)std::min<size_t>((n4 + 255) / 256, 148 * 8), 256, 0, s>>>(
-          g.splitk_ws, real, rows_pad * g.N, n4, static_cast<float*>(e.out));
-      count_launch();
+      f32_split_reduce(g, e, splits, s);
       return 0;
     }
     return launch_tc_pair<T, EPI_F32>(g, e, 1, s);
@@ -712,11 +911,37 @@ int run_t(const GemmDesc& g, const EpiParams& e, cudaStream_t s) {
       if (e.head_dim == 64 && e.seq % 32 == 0 && e.hidden % 64 == 0) return launch_tc_pair<T, EPI_QKV>(g, e, 1, s);
       return g.N > 128 ? launch_tc<T, 256, EPI_QKV>(g, e, 1, s) : launch_tc<T, 128, EPI_QKV>(g, e, 1, s);
     case EPI_BIAS_DROP_RES: return launch_tc_pair<T, EPI_BIAS_DROP_RES>(g, e, 1, s);
-    case EPI_BIAS_GELU: return launch_tc_pair<T, EPI_BIAS_GELU>(g, e, 1, s);
-    case EPI_DGELU: return launch_tc_pair<T, EPI_DGELU>(g, e, 1, s);
+    case EPI_BIAS_GELU:
+      return e.gelu_tanh ? launch_tc_pair<T, EPI_BIAS_GELU | EPI_TANH>(g, e, 1, s)
+                         : launch_tc_pair<T, EPI_BIAS_GELU>(g, e, 1, s);
+    case EPI_DGELU:
+      return e.gelu_tanh ? launch_tc_pair<T, EPI_DGELU | EPI_TANH>(g, e, 1, s) : launch_tc_pair<T, EPI_DGELU>(g, e, 1, s);
     case EPI_STORE: return launch_tc_pair<T, EPI_STORE>(g, e, 1, s);
   }
   return 1;
+}
+
+// A float32 weight gradient (ga) and an input gradient (gb, EPI_DGELU or
+// EPI_STORE) in one launch.
+template <typename T>
+int run2_t(const GemmDesc& ga, const EpiParams& ea, const GemmDesc& gb, const EpiParams& eb, cudaStream_t s) {
+  const bool groupable = ea.kind == EPI_F32 && (eb.kind == EPI_DGELU || eb.kind == EPI_STORE) &&
+                         aligned16(ga.A, ga.lda) && aligned16(ga.B, ga.ldb) && aligned16(gb.A, gb.lda) &&
+                         aligned16(gb.B, gb.ldb);
+  if (!groupable) {
+    const int rc = run_t<T>(ga, ea, s);
+    return rc ? rc : run_t<T>(gb, eb, s);
+  }
+  const int splits = f32_splits(ga);
+  EpiParams ep = ea;
+  if (splits > 1) ep.out = ga.splitk_ws;
+  const int rc =
+      eb.kind == EPI_STORE   ? launch_tc_pair_group<T, EPI_F32, EPI_STORE>(ga, ep, splits, gb, eb, s)
+      : eb.gelu_tanh         ? launch_tc_pair_group<T, EPI_F32, EPI_DGELU | EPI_TANH>(ga, ep, splits, gb, eb, s)
+                             : launch_tc_pair_group<T, EPI_F32, EPI_DGELU>(ga, ep, splits, gb, eb, s);
+  if (rc) return rc;
+  if (splits > 1) f32_split_reduce(ga, ea, splits, s);
+  return 0;
 }
 
 template <typename T>
@@ -725,8 +950,11 @@ int run_pair_t(const GemmDesc& g, const EpiParams& e, int splits, cudaStream_t s
   switch (e.kind) {
     case EPI_QKV: return launch_tc_pair<T, EPI_QKV>(g, e, 1, s);
     case EPI_BIAS_DROP_RES: return launch_tc_pair<T, EPI_BIAS_DROP_RES>(g, e, 1, s);
-    case EPI_BIAS_GELU: return launch_tc_pair<T, EPI_BIAS_GELU>(g, e, 1, s);
-    case EPI_DGELU: return launch_tc_pair<T, EPI_DGELU>(g, e, 1, s);
+    case EPI_BIAS_GELU:
+      return e.gelu_tanh ? launch_tc_pair<T, EPI_BIAS_GELU | EPI_TANH>(g, e, 1, s)
+                         : launch_tc_pair<T, EPI_BIAS_GELU>(g, e, 1, s);
+    case EPI_DGELU:
+      return e.gelu_tanh ? launch_tc_pair<T, EPI_DGELU | EPI_TANH>(g, e, 1, s) : launch_tc_pair<T, EPI_DGELU>(g, e, 1, s);
     case EPI_STORE: return launch_tc_pair<T, EPI_STORE>(g, e, 1, s);
     case EPI_F32: return launch_tc_pair<T, EPI_F32>(g, e, splits, s);
   }
@@ -743,6 +971,11 @@ int gemm_tc_pair_run(int dtype, const GemmDesc& g, const EpiParams& e, int split
 
 int gemm_tc_run(int dtype, const GemmDesc& g, const EpiParams& e, cudaStream_t s) {
   return dtype == DT_F16 ? run_t<half_t>(g, e, s) : run_t<bf16_t>(g, e, s);
+}
+
+int gemm_tc_run2(int dtype, const GemmDesc& ga, const EpiParams& ea, const GemmDesc& gb, const EpiParams& eb,
+                 cudaStream_t s) {
+  return dtype == DT_F16 ? run2_t<half_t>(ga, ea, gb, eb, s) : run2_t<bf16_t>(ga, ea, gb, eb, s);
 }
 
 size_t gemm_tc_splitk_ws_floats(int M, int N, int K) {

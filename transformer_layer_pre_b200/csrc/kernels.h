@@ -10,6 +10,24 @@
 namespace tlp {
 
 enum Dtype { DT_F32 = 0, DT_F16 = 1, DT_BF16 = 2 };
+
+// Launches `kernel` with programmatic stream serialization (see pdl_wait in
+// common.cuh); the kernel must call pdl_wait() before touching global memory.
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                              Args... args) {
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  at[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cfg.attrs = at;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, args...);
+}
 inline size_t dtype_size(int dt) { return dt == DT_F32 ? 4 : 2; }
 
 // ------------------------------------------------------------------ GEMM
@@ -47,11 +65,20 @@ struct EpiParams {
   int seq, hidden, head_dim, heads, tokens;
   // EPI_BIAS_GELU / EPI_DGELU: 1 for the tanh approximation of GELU
   int gelu_tanh;
+  // EPI_DGELU on the tensor-core GEMM: column sums of the stored output, one
+  // partial row per (256-row tile, CTA of the pair, TMEM lane quarter), i.e.
+  // row (m / 256) * 8 + ((m % 256) / 128) * 4 + (m % 128) / 32; or null
+  float* colsum;
 };
 
 // Returns 0, or non-zero when an operand cannot be described to the TMA unit
 // (unaligned base address or row stride).
 int gemm_run(int dtype, const GemmDesc& g, const EpiParams& e, cudaStream_t s);
+// Two independent GEMMs (a float32 weight gradient `ga` and an input
+// gradient `gb` that reads the same operands), in one launch where the
+// tensor-core kernel can plan them together; same results as two gemm_run.
+int gemm_run2(int dtype, const GemmDesc& ga, const EpiParams& ea, const GemmDesc& gb, const EpiParams& eb,
+              cudaStream_t s);
 // 1 when the tensor-core (tcgen05) GEMM serves this dtype, 0 for the SIMT one.
 int gemm_uses_tensor_cores(int dtype);
 // Split-K scratch (floats) the tensor-core GEMM would use for an EPI_F32 GEMM of this shape.

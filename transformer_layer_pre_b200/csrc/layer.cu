@@ -146,7 +146,8 @@ size_t carve(tl_layer* L, char* base) {
   L->dres = c.take(TH * es);
   L->dqkv = c.take(3 * TH * es);
   L->dvec = (float*)c.take((size_t)L->B * L->nh * L->S * 4);
-  const int np = std::max(std::max(ln_bwd_parts(L->T), rowdrop_parts(L->T)), colsum_parts(L->T));
+  const int np = std::max(std::max(std::max(ln_bwd_parts(L->T), rowdrop_parts(L->T)), colsum_parts(L->T)),
+                          (L->T + 255) / 256 * 8);   // + partial rows of the GEMM-fused column sums
   const int maxc = std::max(3 * L->H, L->F);
   L->part_floats = (size_t)np * maxc;
   L->part = (float*)c.take(3 * L->part_floats * 4);
@@ -177,11 +178,23 @@ tl_status ensure_buffers(tl_layer* L) {
   return TL_OK;
 }
 
+GemmDesc gdesc(tl_layer* L, int M, int N, int K, const void* A, int lda, bool ak, const void* B, int ldb, bool bk) {
+  return GemmDesc{M, N, K, A, lda, ak, B, ldb, bk, L->splitk, L->splitk_floats};
+}
+
 void gemm(tl_layer* L, int M, int N, int K, const void* A, int lda, bool ak, const void* B, int ldb, bool bk,
           const EpiParams& e, cudaStream_t s) {
-  GemmDesc g{M, N, K, A, lda, ak, B, ldb, bk, L->splitk, L->splitk_floats};
+  const GemmDesc g = gdesc(L, M, N, K, A, lda, ak, B, ldb, bk);
   ProfScope p_(PC_GEMM, s);
   if (gemm_run(L->opt.dtype, g, e, s) != 0) L->gemm_err = 1;
+}
+
+// A weight gradient and an input gradient that read the same operand, in one
+// launch (they must not write what the other reads).
+void gemm2(tl_layer* L, const GemmDesc& ga, const EpiParams& ea, const GemmDesc& gb, const EpiParams& eb,
+           cudaStream_t s) {
+  ProfScope p_(PC_GEMM, s);
+  if (gemm_run2(L->opt.dtype, ga, ea, gb, eb, s) != 0) L->gemm_err = 1;
 }
 
 // Tensor pointers must be 16-byte aligned (vector loads and TMA).
@@ -430,33 +443,52 @@ tl_status layer_backward(tl_layer* L, const void* x, const void* dy, const tl_we
     colsum_finalize3_run(pa, pb, drop_out ? pc : nullptr, dgamma, dbeta, drop_out ? dsum : nullptr, parts, H, s);
   };
 
-  // FFN block: dZ2 -> dW2, dU (into big), db1, dW1; returns with dU in L->big
-  auto ffn_bwd = [&](const void* ffn_in) {
+  // FFN block: dZ2 -> dW2, dU (into big), db1, then dW1 with the FFN input
+  // gradient dU W1 (epilogue `edin`, output (T, H))
+  auto ffn_bwd = [&](const void* ffn_in, const EpiParams& edin) {
     EpiParams ew2 = epi(EPI_F32, g->w2, F);
     if (L->opt.gelu_checkpoint) {
       ProfScope p_(PC_ROWWISE, s);
       gelu_run(dt, L->u, L->big, (size_t)T * F, L->opt.gelu_tanh ? 1 : 0, s);
     }
-    gemm(L, H, F, T, L->dz2, H, false, L->g, F, false, ew2, s);          // dW2 = dZ2^T G
     EpiParams edu = epi(EPI_DGELU, L->big, F);
     edu.aux = L->u;
     edu.gelu_tanh = L->opt.gelu_tanh ? 1 : 0;
-    gemm(L, T, F, H, L->dz2, H, true, w->w2, F, false, edu, s);          // dU = (dZ2 W2) GELU'(U)
-    bias_grad(L, L->big, F, g->b1, s);                                     // db1
+    // the tensor-core GEMM sums dU's columns in its epilogue (db1)
+    const bool fused_db1 = gemm_uses_tensor_cores(dt) != 0;
+    if (fused_db1) edu.colsum = L->part;
+    const GemmDesc gw2 = gdesc(L, H, F, T, L->dz2, H, false, L->g, F, false);   // dW2 = dZ2^T G
+    const GemmDesc gdu = gdesc(L, T, F, H, L->dz2, H, true, w->w2, F, false);   // dU = (dZ2 W2) GELU'(U)
+    if (L->g != L->big) {
+      gemm2(L, gw2, ew2, gdu, edu, s);
+    } else {
+      // recompute mode: G lives where dU goes, so dW2 must finish first
+      gemm(L, H, F, T, L->dz2, H, false, L->g, F, false, ew2, s);
+      gemm(L, T, F, H, L->dz2, H, true, w->w2, F, false, edu, s);
+    }
+    if (fused_db1) {
+      ProfScope p_(PC_ROWWISE, s);
+      colsum_finalize_run(L->part, (T + 255) / 256 * 8, F, g->b1, s);     // db1 from the GEMM's partials
+    } else {
+      bias_grad(L, L->big, F, g->b1, s);                                   // db1
+    }
     EpiParams ew1 = epi(EPI_F32, g->w1, H);
-    gemm(L, F, H, T, L->big, F, false, ffn_in, H, false, ew1, s);         // dW1 = dU^T in
+    gemm2(L, gdesc(L, F, H, T, L->big, F, false, ffn_in, H, false), ew1,   // dW1 = dU^T in
+          gdesc(L, T, H, F, L->big, F, true, w->w1, H, false), edin, s);   // dU W1
   };
-  // attention block from dA: dWo, dctx, attention backward, dbqkv, dWqkv
-  auto attn_bwd_block = [&](const void* attn_in) {
+  // attention block from dA: dWo with dctx, attention backward, dbqkv, then
+  // dWqkv with the attention input gradient dQKV Wqkv (epilogue `edin`)
+  auto attn_bwd_block = [&](const void* attn_in, const EpiParams& edin) {
     EpiParams ewo = epi(EPI_F32, g->wo, H);
-    gemm(L, H, H, T, L->da, H, false, L->ctx, H, false, ewo, s);          // dWo = dA^T ctx
     EpiParams edc = epi(EPI_STORE, L->dctx, H);
-    gemm(L, T, H, H, L->da, H, true, w->wo, H, false, edc, s);            // dctx = dA Wo
+    gemm2(L, gdesc(L, H, H, T, L->da, H, false, L->ctx, H, false), ewo,    // dWo = dA^T ctx
+          gdesc(L, T, H, H, L->da, H, true, w->wo, H, false), edc, s);     // dctx = dA Wo
     AttnArgs aa = attn_args(L, L->mask);
     attn_bwd(L, aa, s);
     bias_grad(L, L->dqkv, 3 * H, g->bqkv, s);
     EpiParams ewq = epi(EPI_F32, g->wqkv, H);
-    gemm(L, 3 * H, H, T, L->dqkv, 3 * H, false, attn_in, H, false, ewq, s);  // dWqkv = dQKV^T in
+    gemm2(L, gdesc(L, 3 * H, H, T, L->dqkv, 3 * H, false, attn_in, H, false), ewq,   // dWqkv = dQKV^T in
+          gdesc(L, T, H, 3 * H, L->dqkv, 3 * H, true, w->wqkv, H, false), edin, s);  // dQKV Wqkv
   };
 
   if (L->pre_ln) {
@@ -465,14 +497,10 @@ tl_status layer_backward(tl_layer* L, const void* x, const void* dy, const tl_we
       dropout_rows_run(dt, dy, L->dz2, dh, 2, T, H, pc, s);
       colsum_finalize_run(pc, rowdrop_parts(T), H, g->b2, s);
     }
-    ffn_bwd(L->h2);
-    EpiParams edh = epi(EPI_STORE, L->dh, H);
-    gemm(L, T, H, F, L->big, F, true, w->w1, H, false, edh, s);           // dH2 = dU W1
+    ffn_bwd(L->h2, epi(EPI_STORE, L->dh, H));                            // dH2 = dU W1
     ln_bwd(L->dh, L->x2, L->h2, L->mean2, L->rstd2, w->ln2_g, w->ln2_b, dy, L->dx2, L->da, 1,
            g->ln2_g, g->ln2_b, g->bo);
-    attn_bwd_block(L->h1);
-    EpiParams edh1 = epi(EPI_STORE, L->dh, H);
-    gemm(L, T, H, 3 * H, L->dqkv, 3 * H, true, w->wqkv, H, false, edh1, s);  // dH1 = dQKV Wqkv
+    attn_bwd_block(L->h1, epi(EPI_STORE, L->dh, H));                     // dH1 = dQKV Wqkv
     ln_bwd(L->dh, x, L->h1, L->mean1, L->rstd1, w->ln1_g, w->ln1_b, L->dx2, dx, nullptr, 0,
            g->ln1_g, g->ln1_b, nullptr);
   } else {
@@ -480,16 +508,14 @@ tl_status layer_backward(tl_layer* L, const void* x, const void* dy, const tl_we
     const void* r1 = L->res1;
     ln_bwd(dy, r2, L->yout, L->mean2, L->rstd2, w->ln2_g, w->ln2_b, nullptr, L->dres, L->dz2, 2,
            g->ln2_g, g->ln2_b, g->b2);
-    ffn_bwd(L->x2);
     EpiParams edx2 = epi(EPI_STORE, L->dx2, H);
     edx2.res = L->dres;
-    gemm(L, T, H, F, L->big, F, true, w->w1, H, false, edx2, s);          // dx2 = dU W1 + dres2
+    ffn_bwd(L->x2, edx2);                                                 // dx2 = dU W1 + dres2
     ln_bwd(L->dx2, r1, L->x2, L->mean1, L->rstd1, w->ln1_g, w->ln1_b, nullptr, L->dres, L->da, 1,
            g->ln1_g, g->ln1_b, g->bo);
-    attn_bwd_block(x);
     EpiParams edx = epi(EPI_STORE, dx, H);
     edx.res = L->dres;
-    gemm(L, T, H, 3 * H, L->dqkv, 3 * H, true, w->wqkv, H, false, edx, s);  // dx = dQKV Wqkv + dres1
+    attn_bwd_block(x, edx);                                               // dx = dQKV Wqkv + dres1
   }
   (void)es;
   st = check_cuda(L, "layer_backward");

@@ -181,6 +181,8 @@ __global__ void __launch_bounds__(kFwdWarps * 32) ln_fwd_kernel(const T* __restr
                                                                 float* __restrict__ mean_out,
                                                                 float* __restrict__ rstd_out, int rows, int H,
                                                                 float eps) {
+  pdl_wait();
+  pdl_launch_dependents();
   const int lane = threadIdx.x & 31;
   const int row = blockIdx.x * kFwdWarps + (threadIdx.x >> 5);
   if (row >= rows) return;
@@ -234,6 +236,8 @@ __global__ void __launch_bounds__(kFwdWarps * 32) ln_fwd_kernel(const T* __restr
 // Pipeline tensors: 0 dy, 1 x (or y when invertible), 2 res (when given).
 template <typename T, bool INV, bool RES, int KR>
 __global__ void __launch_bounds__(512) ln_bwd_kernel(LnBwdArgs a) {
+  pdl_wait();
+  pdl_launch_dependents();
   extern __shared__ __align__(128) uint8_t smem[];
   constexpr int NT = RES ? 3 : 2;
   const int H = a.H;
@@ -348,6 +352,8 @@ constexpr int kLnbPairs = 4;
 
 template <typename T, bool INV, bool RES, bool DROP, int NC>
 __global__ void __launch_bounds__(kLnbPairs * 64, (sizeof(T) == 4 || (INV && DROP)) ? 1 : 2) ln_bwd_warp_kernel(LnBwdArgs a) {
+  pdl_wait();
+  pdl_launch_dependents();
   extern __shared__ __align__(16) float red[];   // [kLnbPairs][H]; row exchange after it
   float* xch = red + kLnbPairs * a.H;            // [pair][row parity][half][2]
   const int H = a.H;
@@ -489,6 +495,8 @@ template <typename T, int KR>
 __global__ void __launch_bounds__(512) dropout_rows_kernel(const T* __restrict__ in, T* __restrict__ out,
                                                            DropoutParams dp, int site, int rows, int H,
                                                            float* __restrict__ part) {
+  pdl_wait();
+  pdl_launch_dependents();
   extern __shared__ __align__(128) uint8_t smem[];
   const int col = threadIdx.x * 8;
   const bool act = col < H;
@@ -530,6 +538,8 @@ constexpr int kColParts = 64;
 template <typename T>
 __global__ void __launch_bounds__(256) colsum_kernel(const T* __restrict__ X, int rows, int cols,
                                                      float* __restrict__ part) {
+  pdl_wait();
+  pdl_launch_dependents();
   __shared__ float red[8][256 + 8];
   const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;
   const int c0 = (blockIdx.x * 32 + tx) * 8;
@@ -562,6 +572,8 @@ struct FinalizeArgs {
 };
 
 __global__ void __launch_bounds__(1024) colsum_finalize_kernel(FinalizeArgs fa, int nparts, int cols) {
+  pdl_wait();
+  pdl_launch_dependents();
   __shared__ float red[32][33];
   const float* __restrict__ part = fa.part[blockIdx.y];
   const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;
@@ -583,6 +595,8 @@ __global__ void __launch_bounds__(1024) colsum_finalize_kernel(FinalizeArgs fa, 
 
 template <typename T>
 __global__ void gelu_kernel(const T* __restrict__ U, T* __restrict__ G, size_t n8, int tanh_form) {
+  pdl_wait();
+  pdl_launch_dependents();
   for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n8; i += (size_t)gridDim.x * blockDim.x) {
     float v[8];
     load8<T>(U + i * 8, v);
@@ -625,7 +639,7 @@ void ln_fwd_t(const void* x, const void* g, const void* b, void* y, float* mean,
               float eps, cudaStream_t s) {
   const int blocks = (rows + kFwdWarps - 1) / kFwdWarps;
   TLP_NCH_SWITCH(H, {
-    ln_fwd_kernel<T, NCH><<<blocks, kFwdWarps * 32, 0, s>>>(static_cast<const T*>(x), static_cast<const T*>(g),
+    launch_pdl(ln_fwd_kernel<T, NCH>, blocks, kFwdWarps * 32, 0, s, static_cast<const T*>(x), static_cast<const T*>(g),
                                                             static_cast<const T*>(b), static_cast<T*>(y), mean, rstd,
                                                             rows, H, eps);
   });
@@ -637,7 +651,7 @@ void ln_bwd_warp_launch(const LnBwdArgs& a, int parts, cudaStream_t s) {
   const size_t sm = ((size_t)kLnbPairs * a.H + kLnbPairs * 8) * sizeof(float);
   cudaFuncSetAttribute(ln_bwd_warp_kernel<T, INV, RES, DROP, NC>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                        (int)sm);
-  ln_bwd_warp_kernel<T, INV, RES, DROP, NC><<<parts, kLnbPairs * 64, sm, s>>>(a);
+  launch_pdl(ln_bwd_warp_kernel<T, INV, RES, DROP, NC>, parts, kLnbPairs * 64, sm, s, a);
 }
 
 template <typename T, bool INV, bool RES>
@@ -653,7 +667,7 @@ int ln_bwd_t(const LnBwdArgs& a, cudaStream_t s) {
     TLP_KR_SWITCH(a.H, (int)sizeof(T), {
       const size_t sm = pipe_smem<T, KR, RES ? 3 : 2>(a.H);
       cudaFuncSetAttribute(ln_bwd_kernel<T, INV, RES, KR>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
-      ln_bwd_kernel<T, INV, RES, KR><<<parts, row_threads(a.H), sm, s>>>(a);
+      launch_pdl(ln_bwd_kernel<T, INV, RES, KR>, parts, row_threads(a.H), sm, s, a);
     });
   }
   count_launch();
@@ -666,7 +680,7 @@ void dropout_rows_t(const void* in, void* out, const DropoutParams& dp, int site
   TLP_KR_SWITCH(H, (int)sizeof(T), {
     const size_t sm = pipe_smem<T, KR, 1>(H);
     cudaFuncSetAttribute(dropout_rows_kernel<T, KR>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
-    dropout_rows_kernel<T, KR><<<rowdrop_parts(rows), row_threads(H), sm, s>>>(
+    launch_pdl(dropout_rows_kernel<T, KR>, rowdrop_parts(rows), row_threads(H), sm, s, 
         static_cast<const T*>(in), static_cast<T*>(out), dp, site, rows, H, part);
   });
   count_launch();
@@ -718,15 +732,15 @@ void dropout_rows_run(int dt, const void* in, void* out, const DropoutParams& dp
 
 void colsum_run(int dt, const void* X, int rows, int cols, float* part, cudaStream_t s) {
   dim3 grid((cols + 255) / 256, colsum_parts(rows));
-  if (dt == DT_F32) colsum_kernel<float><<<grid, 256, 0, s>>>(static_cast<const float*>(X), rows, cols, part);
-  else if (dt == DT_F16) colsum_kernel<half_t><<<grid, 256, 0, s>>>(static_cast<const half_t*>(X), rows, cols, part);
-  else colsum_kernel<bf16_t><<<grid, 256, 0, s>>>(static_cast<const bf16_t*>(X), rows, cols, part);
+  if (dt == DT_F32) launch_pdl(colsum_kernel<float>, grid, 256, 0, s, static_cast<const float*>(X), rows, cols, part);
+  else if (dt == DT_F16) launch_pdl(colsum_kernel<half_t>, grid, 256, 0, s, static_cast<const half_t*>(X), rows, cols, part);
+  else launch_pdl(colsum_kernel<bf16_t>, grid, 256, 0, s, static_cast<const bf16_t*>(X), rows, cols, part);
   count_launch();
 }
 
 void colsum_finalize_run(const float* part, int nparts, int cols, float* out, cudaStream_t s) {
   FinalizeArgs fa = {{part, nullptr, nullptr}, {out, nullptr, nullptr}};
-  colsum_finalize_kernel<<<dim3((cols + 31) / 32, 1), 1024, 0, s>>>(fa, nparts, cols);
+  launch_pdl(colsum_finalize_kernel, dim3((cols + 31) / 32, 1), 1024, 0, s, fa, nparts, cols);
   count_launch();
 }
 
@@ -734,7 +748,7 @@ void colsum_finalize3_run(const float* p0, const float* p1, const float* p2, flo
                           int nparts, int cols, cudaStream_t s) {
   FinalizeArgs fa = {{p0, p1, p2}, {o0, o1, o2}};
   const int n = p2 ? 3 : (p1 ? 2 : 1);
-  colsum_finalize_kernel<<<dim3((cols + 31) / 32, n), 1024, 0, s>>>(fa, nparts, cols);
+  launch_pdl(colsum_finalize_kernel, dim3((cols + 31) / 32, n), 1024, 0, s, fa, nparts, cols);
   count_launch();
 }
 
@@ -757,11 +771,11 @@ void gelu_run(int dt, const void* U, void* G, size_t n, int tanh_form, cudaStrea
   const size_t n8 = n / 8;
   const int blocks = (int)std::min<size_t>((n8 + 255) / 256, 148 * 16);
   if (dt == DT_F32)
-    gelu_kernel<float><<<blocks, 256, 0, s>>>(static_cast<const float*>(U), static_cast<float*>(G), n8, tanh_form);
+    launch_pdl(gelu_kernel<float>, blocks, 256, 0, s, static_cast<const float*>(U), static_cast<float*>(G), n8, tanh_form);
   else if (dt == DT_F16)
-    gelu_kernel<half_t><<<blocks, 256, 0, s>>>(static_cast<const half_t*>(U), static_cast<half_t*>(G), n8, tanh_form);
+    launch_pdl(gelu_kernel<half_t>, blocks, 256, 0, s, static_cast<const half_t*>(U), static_cast<half_t*>(G), n8, tanh_form);
   else
-    gelu_kernel<bf16_t><<<blocks, 256, 0, s>>>(static_cast<const bf16_t*>(U), static_cast<bf16_t*>(G), n8, tanh_form);
+    launch_pdl(gelu_kernel<bf16_t>, blocks, 256, 0, s, static_cast<const bf16_t*>(U), static_cast<bf16_t*>(G), n8, tanh_form);
   count_launch();
 }
 
