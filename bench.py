@@ -72,7 +72,7 @@ def class_work(cls: str, w, tokens: int, elem: int) -> tuple[float, str]:
 
 
 GEMM_PROFILE = os.path.join(ROOT, "profiles", "gemm_tc_pair_bert-large-f16.txt")
-GEMM_SOURCES = ("gemm_tc.cu", "epilogue.cuh", "sm100.cuh", "common.cuh", "kernels.h")
+GEMM_SOURCES = ("gemm_tc.cu", "epilogue.cuh", "sm100.cuh", "common.cuh", "kernels.h", "dispatch.cu", "layer.cu")
 
 
 def gemm_sources_digest() -> str:
@@ -86,7 +86,8 @@ def gemm_sources_digest() -> str:
 def recorded_gemm_traffic(workload: str) -> float | None:
     """DRAM bytes (read + write) per GEMM launch from the committed ncu summary
     of this workload, or None when there is none or the GEMM kernel sources
-    have changed since it was captured."""
+    (or the layer code that decides which GEMM launches a step makes) have
+    changed since it was captured."""
     if workload != WORKLOAD or not os.path.exists(GEMM_PROFILE):
         return None
     with open(GEMM_PROFILE) as fh:

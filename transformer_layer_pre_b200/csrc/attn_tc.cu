@@ -56,6 +56,7 @@ struct AttnTc {
   const void* dctx;
   const float* dvec;    // precomputed D, or null to compute it in-kernel
   void* dqkv;
+  float* colsum;        // fused QKV bias-gradient partials (persistent backward), or null
   int fuse_dq;
   int bf16;
   int* err;
@@ -1091,22 +1092,34 @@ __global__ void __launch_bounds__(kPBwdThreads, 1)
       tmem_ld32(tdV + lo + hf * 32, dv);
       tc_fence_before();
       mbar_arrive(g_free);
+#pragma unroll
+      for (int c = 0; c < 32; ++c) {
+        dq[c] *= a.scale;
+        dk[c] *= a.scale;
+      }
       if (qv) {
         // row r is query r for dQ and key r for dK, dV (both < S)
         T* dst = static_cast<T*>(a.dqkv) + trow * 3 * a.H + h * HD + hf * 32;
 #pragma unroll
         for (int c = 0; c < 32; c += 8) {
-          float q8[8], k8[8], v8[8];
-#pragma unroll
-          for (int t = 0; t < 8; ++t) {
-            q8[t] = dq[c + t] * a.scale;
-            k8[t] = dk[c + t] * a.scale;
-            v8[t] = dv[c + t];
-          }
-          store8<T>(dst + c, q8);
-          store8<T>(dst + a.H + c, k8);
-          store8<T>(dst + 2 * a.H + c, v8);
+          store8<T>(dst + c, *reinterpret_cast<float(*)[8]>(dq + c));
+          store8<T>(dst + a.H + c, *reinterpret_cast<float(*)[8]>(dk + c));
+          store8<T>(dst + 2 * a.H + c, *reinterpret_cast<float(*)[8]>(dv + c));
         }
+      }
+      if (a.colsum) {
+        // QKV bias gradient fused in: column sums of the stored values over
+        // this warp's 32 rows (rows past the sequence end count as zero)
+        float* cs = a.colsum + (size_t)(b * 4 + quarter) * 3 * a.H + h * HD + hf * 32 + lane;
+#pragma unroll
+        for (int c = 0; c < 32; ++c) {
+          dq[c] = qv ? round_f<T>(dq[c]) : 0.0f;
+          dk[c] = qv ? round_f<T>(dk[c]) : 0.0f;
+          dv[c] = qv ? round_f<T>(dv[c]) : 0.0f;
+        }
+        cs[0] = warp_colsum32(dq);
+        cs[a.H] = warp_colsum32(dk);
+        cs[2 * a.H] = warp_colsum32(dv);
       }
     }
   }
@@ -1164,6 +1177,7 @@ AttnTc make_args(int dt, const AttnArgs& a) {
   t.dctx = a.dctx;
   t.dvec = nullptr;
   t.dqkv = a.dqkv;
+  t.colsum = a.colsum;
   t.fuse_dq = 0;
   t.bf16 = dt == DT_BF16;
   t.err = attn_error_word();
@@ -1233,6 +1247,9 @@ void bwd_t(const AttnArgs& a, cudaStream_t s) {
 }
 
 }  // namespace
+
+// Whether attn_tc_bwd_run writes the QKV bias-gradient partials (AttnArgs.colsum).
+bool attn_tc_fuses_colsum(int dt, const AttnArgs& a) { return dt != DT_F32 && a.d == HD && a.S <= TILE; }
 
 bool attn_tc_supports(int dt, const AttnArgs& a) {
   if (dt == DT_F32 || a.d != HD || a.S < 8) return false;

@@ -126,6 +126,18 @@ int colsum_parts(int rows);
 void colsum_run(int dtype, const void* X, int rows, int cols, float* part, cudaStream_t s);
 // out[c] = sum_p part[p*cols + c] (fixed order).
 void colsum_finalize_run(const float* part, int nparts, int cols, float* out, cudaStream_t s);
+// Several finalizes in one launch: out[c] = sum over p < nparts of part[p * cols + c] per job.
+constexpr int kMaxFinalize = 8;
+struct FinalizeJob {
+  const float* part;
+  float* out;
+  int nparts, cols;
+};
+struct FinalizeList {
+  FinalizeJob job[kMaxFinalize];
+  int n;
+};
+void colsum_finalize_list_run(const FinalizeList& fl, cudaStream_t s);
 // The same for up to three (partials, output) pairs in one launch (p1/p2 may be null).
 void colsum_finalize3_run(const float* p0, const float* p1, const float* p2, float* o0, float* o1, float* o2,
                           int nparts, int cols, cudaStream_t s);
@@ -151,6 +163,11 @@ struct AttnArgs {
   const void* dctx;     // (B*S, nh*d)
   float* dvec;          // (B, nh, S) rowsum(dctx * ctx)
   void* dqkv;           // (B*S, 3*nh*d): [dQ | dK | dV]
+  // column sums of the stored dQKV (the QKV bias gradient), one partial row
+  // per (sequence b, 32-query block q): row b*4 + q of a (B*4, 3*nh*d)
+  // float32 matrix; written only by kernels that fuse it (see
+  // attn_tc_fuses_colsum), else untouched
+  float* colsum;
 };
 void attn_fwd_run(int dtype, const AttnArgs& a, cudaStream_t s);
 void attn_bwd_run(int dtype, const AttnArgs& a, cudaStream_t s);

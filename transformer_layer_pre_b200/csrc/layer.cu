@@ -32,6 +32,7 @@ void attn_simt_bwd_run(int dt, const AttnArgs& a, cudaStream_t s);
 void attn_tc_fwd_run(int dt, const AttnArgs& a, cudaStream_t s);
 void attn_tc_bwd_run(int dt, const AttnArgs& a, cudaStream_t s);
 bool attn_tc_supports(int dt, const AttnArgs& a);
+bool attn_tc_fuses_colsum(int dt, const AttnArgs& a);
 }  // namespace tlp
 
 using namespace tlp;
@@ -147,10 +148,10 @@ size_t carve(tl_layer* L, char* base) {
   L->dqkv = c.take(3 * TH * es);
   L->dvec = (float*)c.take((size_t)L->B * L->nh * L->S * 4);
   const int np = std::max(std::max(std::max(ln_bwd_parts(L->T), rowdrop_parts(L->T)), colsum_parts(L->T)),
-                          (L->T + 255) / 256 * 8);   // + partial rows of the GEMM-fused column sums
+                          std::max((L->T + 255) / 256 * 8, L->B * 4));   // + partial rows of fused column sums
   const int maxc = std::max(3 * L->H, L->F);
   L->part_floats = (size_t)np * maxc;
-  L->part = (float*)c.take(3 * L->part_floats * 4);
+  L->part = (float*)c.take((size_t)kMaxFinalize * L->part_floats * 4);   // one slot per parameter column sum
   const int dt = L->opt.dtype, T = L->T, H = L->H, F = L->F;
   L->splitk_floats = std::max(std::max(gemm_splitk_ws_floats(dt, H, F, T), gemm_splitk_ws_floats(dt, F, H, T)),
                               std::max(gemm_splitk_ws_floats(dt, H, H, T), gemm_splitk_ws_floats(dt, 3 * H, H, T)));
@@ -209,11 +210,13 @@ EpiParams epi(int kind, void* out, int ldo) {
   return e;
 }
 
-// Column sums of a (T, cols) stored matrix into a float32 vector.
-void bias_grad(tl_layer* L, const void* X, int cols, float* out, cudaStream_t s) {
+// Column partial sums of a (T, cols) stored matrix into partial slot `slot`,
+// summed into `out` by the backward's closing finalize.
+void bias_grad(tl_layer* L, const void* X, int cols, int slot, float* out, FinalizeList& fin, cudaStream_t s) {
   ProfScope p_(PC_ROWWISE, s);
-  colsum_run(L->opt.dtype, X, L->T, cols, L->part, s);
-  colsum_finalize_run(L->part, colsum_parts(L->T), cols, out, s);
+  float* part = L->part + (size_t)slot * L->part_floats;
+  colsum_run(L->opt.dtype, X, L->T, cols, part, s);
+  fin.job[fin.n++] = {part, out, colsum_parts(L->T), cols};
 }
 
 void attn_fwd(tl_layer* L, const AttnArgs& a, cudaStream_t s) {
@@ -423,29 +426,33 @@ tl_status layer_backward(tl_layer* L, const void* x, const void* dy, const tl_we
   cudaStream_t s = (cudaStream_t)stream;
   const int dt = L->opt.dtype, T = L->T, H = L->H, F = L->F;
   const size_t es = dtype_size(dt);
-  float* pa = L->part;
-  float* pb = L->part + L->part_floats;
-  float* pc = L->part + 2 * L->part_floats;
   const DropoutParams dh = make_drop(L, L->ph);
+  // every parameter column sum (bias, gamma, beta gradients) leaves its
+  // producer as partial rows in a slot of its own; one launch at the end sums them
+  FinalizeList fin;
+  fin.n = 0;
+  auto slot = [&](int i) { return L->part + (size_t)i * L->part_floats; };
 
   auto ln_bwd = [&](const void* dyln, const void* xin, const void* yln, const float* mean, const float* rstd,
                     const void* gamma, const void* beta, const void* res, void* dxo, void* drop_out, int site,
-                    float* dgamma, float* dbeta, float* dsum) {
+                    float* dgamma, float* dbeta, float* dsum, int slot0) {
     LnBwdArgs a;
     std::memset(&a, 0, sizeof(a));
     a.dy = dyln; a.x = inv ? nullptr : xin; a.y = inv ? yln : nullptr;
     a.mean = mean; a.rstd = rstd; a.gamma = gamma; a.beta = beta;
     a.res = res; a.dx = dxo; a.drop_out = drop_out; a.drop = dh; a.site = site;
-    a.part_dgamma = pa; a.part_dbeta = pb; a.part_dsum = drop_out ? pc : nullptr;
+    a.part_dgamma = slot(slot0); a.part_dbeta = slot(slot0 + 1); a.part_dsum = drop_out ? slot(slot0 + 2) : nullptr;
     a.rows = T; a.H = H;
     ProfScope p_(PC_LN_BWD, s);
     const int parts = ln_bwd_run(dt, a, s);
-    colsum_finalize3_run(pa, pb, drop_out ? pc : nullptr, dgamma, dbeta, drop_out ? dsum : nullptr, parts, H, s);
+    fin.job[fin.n++] = {a.part_dgamma, dgamma, parts, H};
+    fin.job[fin.n++] = {a.part_dbeta, dbeta, parts, H};
+    if (drop_out) fin.job[fin.n++] = {a.part_dsum, dsum, parts, H};
   };
 
   // FFN block: dZ2 -> dW2, dU (into big), db1, then dW1 with the FFN input
   // gradient dU W1 (epilogue `edin`, output (T, H))
-  auto ffn_bwd = [&](const void* ffn_in, const EpiParams& edin) {
+  auto ffn_bwd = [&](const void* ffn_in, const EpiParams& edin, int db1_slot) {
     EpiParams ew2 = epi(EPI_F32, g->w2, F);
     if (L->opt.gelu_checkpoint) {
       ProfScope p_(PC_ROWWISE, s);
@@ -456,36 +463,35 @@ tl_status layer_backward(tl_layer* L, const void* x, const void* dy, const tl_we
     edu.gelu_tanh = L->opt.gelu_tanh ? 1 : 0;
     // the tensor-core GEMM sums dU's columns in its epilogue (db1)
     const bool fused_db1 = gemm_uses_tensor_cores(dt) != 0;
-    if (fused_db1) edu.colsum = L->part;
+    if (fused_db1) edu.colsum = slot(db1_slot);
     const GemmDesc gw2 = gdesc(L, H, F, T, L->dz2, H, false, L->g, F, false);   // dW2 = dZ2^T G
     const GemmDesc gdu = gdesc(L, T, F, H, L->dz2, H, true, w->w2, F, false);   // dU = (dZ2 W2) GELU'(U)
-    if (L->g != L->big) {
-      gemm2(L, gw2, ew2, gdu, edu, s);
-    } else {
-      // recompute mode: G lives where dU goes, so dW2 must finish first
-      gemm(L, H, F, T, L->dz2, H, false, L->g, F, false, ew2, s);
-      gemm(L, T, F, H, L->dz2, H, true, w->w2, F, false, edu, s);
+    // two launches: the dGELU epilogue makes dU's tiles slower than their
+    // K blocks say, which the grouped plan does not model (and in recompute
+    // mode G lives where dU goes, so dW2 must finish first anyway)
+    {
+      ProfScope p_(PC_GEMM, s);
+      if (gemm_run(dt, gw2, ew2, s) != 0 || gemm_run(dt, gdu, edu, s) != 0) L->gemm_err = 1;
     }
-    if (fused_db1) {
-      ProfScope p_(PC_ROWWISE, s);
-      colsum_finalize_run(L->part, (T + 255) / 256 * 8, F, g->b1, s);     // db1 from the GEMM's partials
-    } else {
-      bias_grad(L, L->big, F, g->b1, s);                                   // db1
-    }
+    if (fused_db1) fin.job[fin.n++] = {slot(db1_slot), g->b1, (T + 255) / 256 * 8, F};   // db1 from the GEMM
+    else bias_grad(L, L->big, F, db1_slot, g->b1, fin, s);                                  // db1
     EpiParams ew1 = epi(EPI_F32, g->w1, H);
     gemm2(L, gdesc(L, F, H, T, L->big, F, false, ffn_in, H, false), ew1,   // dW1 = dU^T in
           gdesc(L, T, H, F, L->big, F, true, w->w1, H, false), edin, s);   // dU W1
   };
   // attention block from dA: dWo with dctx, attention backward, dbqkv, then
   // dWqkv with the attention input gradient dQKV Wqkv (epilogue `edin`)
-  auto attn_bwd_block = [&](const void* attn_in, const EpiParams& edin) {
+  auto attn_bwd_block = [&](const void* attn_in, const EpiParams& edin, int dbqkv_slot) {
     EpiParams ewo = epi(EPI_F32, g->wo, H);
     EpiParams edc = epi(EPI_STORE, L->dctx, H);
     gemm2(L, gdesc(L, H, H, T, L->da, H, false, L->ctx, H, false), ewo,    // dWo = dA^T ctx
           gdesc(L, T, H, H, L->da, H, true, w->wo, H, false), edc, s);     // dctx = dA Wo
     AttnArgs aa = attn_args(L, L->mask);
+    const bool fused_dbqkv = attn_tc_supports(dt, aa) && attn_tc_fuses_colsum(dt, aa);
+    if (fused_dbqkv) aa.colsum = slot(dbqkv_slot);
     attn_bwd(L, aa, s);
-    bias_grad(L, L->dqkv, 3 * H, g->bqkv, s);
+    if (fused_dbqkv) fin.job[fin.n++] = {slot(dbqkv_slot), g->bqkv, L->B * 4, 3 * H};   // from the attention
+    else bias_grad(L, L->dqkv, 3 * H, dbqkv_slot, g->bqkv, fin, s);
     EpiParams ewq = epi(EPI_F32, g->wqkv, H);
     gemm2(L, gdesc(L, 3 * H, H, T, L->dqkv, 3 * H, false, attn_in, H, false), ewq,   // dWqkv = dQKV^T in
           gdesc(L, T, H, 3 * H, L->dqkv, 3 * H, true, w->wqkv, H, false), edin, s);  // dQKV Wqkv
@@ -494,28 +500,32 @@ tl_status layer_backward(tl_layer* L, const void* x, const void* dy, const tl_we
   if (L->pre_ln) {
     {
       ProfScope p_(PC_ROWWISE, s);
-      dropout_rows_run(dt, dy, L->dz2, dh, 2, T, H, pc, s);
-      colsum_finalize_run(pc, rowdrop_parts(T), H, g->b2, s);
+      dropout_rows_run(dt, dy, L->dz2, dh, 2, T, H, slot(0), s);
+      fin.job[fin.n++] = {slot(0), g->b2, rowdrop_parts(T), H};
     }
-    ffn_bwd(L->h2, epi(EPI_STORE, L->dh, H));                            // dH2 = dU W1
+    ffn_bwd(L->h2, epi(EPI_STORE, L->dh, H), 1);                         // dH2 = dU W1
     ln_bwd(L->dh, L->x2, L->h2, L->mean2, L->rstd2, w->ln2_g, w->ln2_b, dy, L->dx2, L->da, 1,
-           g->ln2_g, g->ln2_b, g->bo);
-    attn_bwd_block(L->h1, epi(EPI_STORE, L->dh, H));                     // dH1 = dQKV Wqkv
+           g->ln2_g, g->ln2_b, g->bo, 2);
+    attn_bwd_block(L->h1, epi(EPI_STORE, L->dh, H), 5);                  // dH1 = dQKV Wqkv
     ln_bwd(L->dh, x, L->h1, L->mean1, L->rstd1, w->ln1_g, w->ln1_b, L->dx2, dx, nullptr, 0,
-           g->ln1_g, g->ln1_b, nullptr);
+           g->ln1_g, g->ln1_b, nullptr, 6);
   } else {
     const void* r2 = L->res2;
     const void* r1 = L->res1;
     ln_bwd(dy, r2, L->yout, L->mean2, L->rstd2, w->ln2_g, w->ln2_b, nullptr, L->dres, L->dz2, 2,
-           g->ln2_g, g->ln2_b, g->b2);
+           g->ln2_g, g->ln2_b, g->b2, 0);
     EpiParams edx2 = epi(EPI_STORE, L->dx2, H);
     edx2.res = L->dres;
-    ffn_bwd(L->x2, edx2);                                                 // dx2 = dU W1 + dres2
+    ffn_bwd(L->x2, edx2, 3);                                              // dx2 = dU W1 + dres2
     ln_bwd(L->dx2, r1, L->x2, L->mean1, L->rstd1, w->ln1_g, w->ln1_b, nullptr, L->dres, L->da, 1,
-           g->ln1_g, g->ln1_b, g->bo);
+           g->ln1_g, g->ln1_b, g->bo, 4);
     EpiParams edx = epi(EPI_STORE, dx, H);
     edx.res = L->dres;
-    attn_bwd_block(x, edx);                                               // dx = dQKV Wqkv + dres1
+    attn_bwd_block(x, edx, 7);                                            // dx = dQKV Wqkv + dres1
+  }
+  {
+    ProfScope p_(PC_ROWWISE, s);
+    colsum_finalize_list_run(fin, s);                                     // every bias / LayerNorm gradient
   }
   (void)es;
   st = check_cuda(L, "layer_backward");

@@ -566,16 +566,18 @@ __global__ void __launch_bounds__(256) colsum_kernel(const T* __restrict__ X, in
 // out[c] = sum over p of part[p][c]: 32 columns x 32 part-lanes per block,
 // each lane sums every 32nd partial row, then a fixed-order sum over lanes.
 // blockIdx.y selects one of up to three (partials, output) pairs.
-struct FinalizeArgs {
-  const float* part[3];
-  float* out[3];
-};
-
-__global__ void __launch_bounds__(1024) colsum_finalize_kernel(FinalizeArgs fa, int nparts, int cols) {
+// Column sums of partial rows, for up to kMaxFinalize (partials, output)
+// jobs in one launch: blockIdx.y picks the job, 32 x 32 threads sum 32
+// columns of it (partial rows strided over the 32 warps, then the 32 warp
+// sums in warp order: a fixed order).
+__global__ void __launch_bounds__(1024) colsum_finalize_kernel(FinalizeList fl) {
   pdl_wait();
   pdl_launch_dependents();
   __shared__ float red[32][33];
-  const float* __restrict__ part = fa.part[blockIdx.y];
+  const FinalizeJob& job = fl.job[blockIdx.y];
+  const int cols = job.cols, nparts = job.nparts;
+  if (blockIdx.x * 32 >= cols) return;
+  const float* __restrict__ part = job.part;
   const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;
   const int c = blockIdx.x * 32 + tx;
   float s = 0.0f;
@@ -589,7 +591,7 @@ __global__ void __launch_bounds__(1024) colsum_finalize_kernel(FinalizeArgs fa, 
     float t = 0.0f;
 #pragma unroll
     for (int w = 0; w < 32; ++w) t += red[w][tx];
-    fa.out[blockIdx.y][c] = t;
+    job.out[c] = t;
   }
 }
 
@@ -738,18 +740,29 @@ void colsum_run(int dt, const void* X, int rows, int cols, float* part, cudaStre
   count_launch();
 }
 
-void colsum_finalize_run(const float* part, int nparts, int cols, float* out, cudaStream_t s) {
-  FinalizeArgs fa = {{part, nullptr, nullptr}, {out, nullptr, nullptr}};
-  launch_pdl(colsum_finalize_kernel, dim3((cols + 31) / 32, 1), 1024, 0, s, fa, nparts, cols);
+void colsum_finalize_list_run(const FinalizeList& fl, cudaStream_t s) {
+  if (fl.n <= 0) return;
+  int maxc = 0;
+  for (int i = 0; i < fl.n; ++i) maxc = std::max(maxc, fl.job[i].cols);
+  launch_pdl(colsum_finalize_kernel, dim3((maxc + 31) / 32, fl.n), 1024, 0, s, fl);
   count_launch();
+}
+
+void colsum_finalize_run(const float* part, int nparts, int cols, float* out, cudaStream_t s) {
+  FinalizeList fl;
+  fl.n = 1;
+  fl.job[0] = {part, out, nparts, cols};
+  colsum_finalize_list_run(fl, s);
 }
 
 void colsum_finalize3_run(const float* p0, const float* p1, const float* p2, float* o0, float* o1, float* o2,
                           int nparts, int cols, cudaStream_t s) {
-  FinalizeArgs fa = {{p0, p1, p2}, {o0, o1, o2}};
-  const int n = p2 ? 3 : (p1 ? 2 : 1);
-  launch_pdl(colsum_finalize_kernel, dim3((cols + 31) / 32, n), 1024, 0, s, fa, nparts, cols);
-  count_launch();
+  FinalizeList fl;
+  fl.n = 0;
+  fl.job[fl.n++] = {p0, o0, nparts, cols};
+  if (p1) fl.job[fl.n++] = {p1, o1, nparts, cols};
+  if (p2) fl.job[fl.n++] = {p2, o2, nparts, cols};
+  colsum_finalize_list_run(fl, s);
 }
 
 __global__ void gelu_eval_kernel(const float* __restrict__ u, float* __restrict__ g, float* __restrict__ dg,
