@@ -77,7 +77,8 @@ __device__ __forceinline__ void epi_apply8(const EpiParams& e, int m, int n, flo
     float b[8];
     load8<T>(static_cast<const T*>(e.bias) + n, b);
     uint32_t bits = 0xFFu;
-    if (e.drop.thr) bits = dropout_bits8(e.drop, e.site, ((uint64_t)m * e.ldo + n) >> 3);
+    if (e.keep8) bits = e.keep8[((uint64_t)m * e.ldo + n) >> 3];
+    else if (e.drop.thr) bits = dropout_bits8(e.drop, e.site, ((uint64_t)m * e.ldo + n) >> 3);
     const float sc = e.drop.thr ? e.drop.scale : 1.0f;
 #pragma unroll
     for (int i = 0; i < 8; ++i) v[i] = aux[i] + (((bits >> i) & 1u) ? (v[i] + b[i]) * sc : 0.0f);
@@ -101,9 +102,11 @@ __device__ __forceinline__ void epi_apply8(const EpiParams& e, int m, int n, flo
 // Epilogue arithmetic without the store: v becomes the (first) output chunk,
 // v2 the second one (EPI_BIAS_GELU's G).  Used by the tensor-core GEMM, whose
 // stores go through shared memory and TMA.
+// kbits: the 8 dropout keep bits of this chunk when the caller already has
+// them (EPI_BIAS_DROP_RES), or a value above 0xFF to look them up here.
 template <typename T, int KIND>
 __device__ __forceinline__ void epi_compute8(const EpiParams& e, int m, int n, float (&v)[8], float (&v2)[8],
-                                             const float (&aux)[8]) {
+                                             const float (&aux)[8], uint32_t kbits = 0x100u) {
   if constexpr (epi_base(KIND) == EPI_STORE) {
     if (e.res) {
 #pragma unroll
@@ -118,7 +121,9 @@ __device__ __forceinline__ void epi_compute8(const EpiParams& e, int m, int n, f
     float b[8];
     load8<T>(static_cast<const T*>(e.bias) + n, b);
     uint32_t bits = 0xFFu;
-    if (e.drop.thr) bits = dropout_bits8(e.drop, e.site, ((uint64_t)m * e.ldo + n) >> 3);
+    if (kbits <= 0xFFu) bits = kbits;
+    else if (e.keep8) bits = e.keep8[((uint64_t)m * e.ldo + n) >> 3];
+    else if (e.drop.thr) bits = dropout_bits8(e.drop, e.site, ((uint64_t)m * e.ldo + n) >> 3);
     const float sc = e.drop.thr ? e.drop.scale : 1.0f;
 #pragma unroll
     for (int i = 0; i < 8; ++i) v[i] = aux[i] + (((bits >> i) & 1u) ? (v[i] + b[i]) * sc : 0.0f);

@@ -355,6 +355,16 @@ __device__ __forceinline__ bool pair_epilogue_tile(const OutMaps& om, const TcAr
                                         : make_uint4(0u, 0u, 0u, 0u);
     }
   }
+  // precomputed dropout keep bits of this thread's 64 columns (one byte per 8), loaded early
+  uint2 kpre = make_uint2(0u, 0u);
+  bool kvalid = false;
+  if constexpr (epi_base(KIND) == EPI_BIAS_DROP_RES) {
+    const size_t e0 = (size_t)m * e.ldo + nbase;
+    if (e.keep8 && mrow && (e0 & 63) == 0 && nbase + CW <= g.N) {
+      kpre = *reinterpret_cast<const uint2*>(e.keep8 + (e0 >> 3));
+      kvalid = true;
+    }
+  }
   if (!mbar_wait_warp(&tfull[acc], aph, g.err, 44)) return false;
   tc_fence_after();
   const uint32_t tbase = tmem + ((uint32_t)(quarter * 32) << 16) + acc * BN + part * CW;
@@ -393,7 +403,12 @@ __device__ __forceinline__ bool pair_epilogue_tile(const OutMaps& om, const TcAr
 #pragma unroll
           for (int i = 0; i < 8; ++i) aux[i] = 0.0f;
         }
-        if (mrow && n < g.N) epi_compute8<T, KIND>(e, m, n, *reinterpret_cast<float(*)[8]>(vq), v2, aux);
+        uint32_t kb = 0x100u;
+        if constexpr (epi_base(KIND) == EPI_BIAS_DROP_RES) {
+          const int j = (c0 >> 3) + q;
+          if (kvalid) kb = ((j < 4 ? kpre.x : kpre.y) >> (8 * (j & 3))) & 0xFFu;
+        }
+        if (mrow && n < g.N) epi_compute8<T, KIND>(e, m, n, *reinterpret_cast<float(*)[8]>(vq), v2, aux, kb);
         store8<T>(reinterpret_cast<T*>(sb0 + lane * 64 + ((q ^ swz) << 4)), *reinterpret_cast<float(*)[8]>(vq));
         if constexpr (NOUT == 2) store8<T>(reinterpret_cast<T*>(sb1 + lane * 64 + ((q ^ swz) << 4)), v2);
       }

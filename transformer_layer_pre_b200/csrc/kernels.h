@@ -61,6 +61,7 @@ struct EpiParams {
   // dropout (EPI_BIAS_DROP_RES)
   DropoutParams drop;
   int site;
+  const uint8_t* keep8;   // EPI_BIAS_DROP_RES: precomputed keep bits (byte per 8 elements), or null
   // head split (EPI_QKV)
   int seq, hidden, head_dim, heads, tokens;
   // EPI_BIAS_GELU / EPI_DGELU: 1 for the tanh approximation of GELU
@@ -87,8 +88,14 @@ size_t gemm_splitk_ws_floats(int dtype, int M, int N, int K);
 int device_take_error();
 
 // ------------------------------------------------------------------ LayerNorm
+// LayerNorm forward.  With keep_out, also writes the dropout keep bits of
+// site `site` for the (rows, H) elements: byte e/8 holds elements e..e+7
+// (bit k = element e+k), the same bits dropout_bits8 gives; the row kernels
+// have idle arithmetic units, so the downstream kernels read the bits
+// instead of drawing Philox themselves.
 void ln_fwd_run(int dtype, const void* x, const void* gamma, const void* beta, void* y, float* mean,
-                float* rstd, int rows, int H, float eps, cudaStream_t s);
+                float* rstd, int rows, int H, float eps, cudaStream_t s, uint8_t* keep_out = nullptr,
+                const DropoutParams* dp = nullptr, int site = 0);
 
 // LayerNorm backward of one row block + residual-gradient add + optional
 // dropout of the result, with column partial sums for dgamma, dbeta and the
@@ -106,6 +113,7 @@ struct LnBwdArgs {
   void* drop_out;       // dropout(dx) (rows, H), or null
   DropoutParams drop;
   int site;
+  const uint8_t* keep8;   // keep bits of the dropout copy (byte per 8 elements), or null: draw them
   float* part_dgamma;
   float* part_dbeta;
   float* part_dsum;     // column sums of drop_out, or null
@@ -120,7 +128,7 @@ int ln_bwd_run(int dtype, const LnBwdArgs& a, cudaStream_t s);
 // out = dropout(in) (site, element t*H + c) with column partial sums of out.
 int rowdrop_parts(int rows);
 void dropout_rows_run(int dtype, const void* in, void* out, const DropoutParams& dp, int site, int rows, int H,
-                      float* part_sum, cudaStream_t s);
+                      float* part_sum, cudaStream_t s, const uint8_t* keep8 = nullptr);
 // Column partial sums of a (rows, cols) storage-typed matrix: (colsum_parts(rows), cols) floats.
 int colsum_parts(int rows);
 void colsum_run(int dtype, const void* X, int rows, int cols, float* part, cudaStream_t s);

@@ -60,6 +60,8 @@ struct tl_layer {
   void *dqkv = nullptr;
   float *dvec = nullptr, *part = nullptr;
   size_t part_floats = 0;
+  // hidden-dropout keep bits of sites 1 and 2 (one byte per 8 elements)
+  uint8_t *keep1 = nullptr, *keep2 = nullptr;
   float* splitk = nullptr;
   size_t splitk_floats = 0;
   int gemm_err = 0;
@@ -147,6 +149,8 @@ size_t carve(tl_layer* L, char* base) {
   L->dres = c.take(TH * es);
   L->dqkv = c.take(3 * TH * es);
   L->dvec = (float*)c.take((size_t)L->B * L->nh * L->S * 4);
+  L->keep1 = (uint8_t*)c.take((size_t)L->T * L->H / 8);
+  L->keep2 = (uint8_t*)c.take((size_t)L->T * L->H / 8);
   const int np = std::max(std::max(std::max(ln_bwd_parts(L->T), rowdrop_parts(L->T)), colsum_parts(L->T)),
                           std::max((L->T + 255) / 256 * 8, L->B * 4));   // + partial rows of fused column sums
   const int maxc = std::max(3 * L->H, L->F);
@@ -361,19 +365,27 @@ tl_status layer_forward(tl_layer* L, const void* x, const float* mask, const tl_
   EpiParams e2 = epi(EPI_BIAS_DROP_RES, nullptr, H);
   e2.bias = w->b2; e2.drop = make_drop(L, L->ph); e2.site = 2;
 
+  // hidden-dropout keep bits come from the LayerNorm forward kernels that
+  // run before their consumers (pre-LN: LN1 for site 1, LN2 for site 2;
+  // post-LN: LN1 for site 2); the consumers read them instead of drawing Philox
+  const bool keepbits = eo.drop.thr != 0;
   if (L->pre_ln) {
     {
       ProfScope p_(PC_LN_FWD, s);
-      ln_fwd_run(dt, x, w->ln1_g, w->ln1_b, L->h1, L->mean1, L->rstd1, T, H, L->opt.ln_eps, s);
+      ln_fwd_run(dt, x, w->ln1_g, w->ln1_b, L->h1, L->mean1, L->rstd1, T, H, L->opt.ln_eps, s,
+                 keepbits ? L->keep1 : nullptr, &eo.drop, 1);
     }
+    if (keepbits) eo.keep8 = L->keep1;
     gemm(L, T, 3 * H, H, L->h1, H, true, w->wqkv, H, true, eq, s);
     attn_fwd(L, aa, s);
     eo.out = L->x2;
     gemm(L, T, H, H, L->ctx, H, true, w->wo, H, true, eo, s);
     {
       ProfScope p_(PC_LN_FWD, s);
-      ln_fwd_run(dt, L->x2, w->ln2_g, w->ln2_b, L->h2, L->mean2, L->rstd2, T, H, L->opt.ln_eps, s);
+      ln_fwd_run(dt, L->x2, w->ln2_g, w->ln2_b, L->h2, L->mean2, L->rstd2, T, H, L->opt.ln_eps, s,
+                 keepbits ? L->keep2 : nullptr, &e2.drop, 2);
     }
+    if (keepbits) e2.keep8 = L->keep2;
     gemm(L, T, F, H, L->h2, H, true, w->w1, H, true, e1, s);
     e2.res = L->x2; e2.out = y;
     gemm(L, T, H, F, L->g, F, true, w->w2, F, true, e2, s);
@@ -387,8 +399,10 @@ tl_status layer_forward(tl_layer* L, const void* x, const float* mask, const tl_
     gemm(L, T, H, H, L->ctx, H, true, w->wo, H, true, eo, s);
     {
       ProfScope p_(PC_LN_FWD, s);
-      ln_fwd_run(dt, r1, w->ln1_g, w->ln1_b, L->x2, L->mean1, L->rstd1, T, H, L->opt.ln_eps, s);
+      ln_fwd_run(dt, r1, w->ln1_g, w->ln1_b, L->x2, L->mean1, L->rstd1, T, H, L->opt.ln_eps, s,
+                 keepbits ? L->keep2 : nullptr, &e2.drop, 2);
     }
+    if (keepbits) e2.keep8 = L->keep2;
     gemm(L, T, F, H, L->x2, H, true, w->w1, H, true, e1, s);
     e2.res = L->x2; e2.out = r2;
     gemm(L, T, H, F, L->g, F, true, w->w2, F, true, e2, s);
@@ -427,6 +441,7 @@ tl_status layer_backward(tl_layer* L, const void* x, const void* dy, const tl_we
   const int dt = L->opt.dtype, T = L->T, H = L->H, F = L->F;
   const size_t es = dtype_size(dt);
   const DropoutParams dh = make_drop(L, L->ph);
+  const bool keepbits = dh.thr != 0;   // the forward left the hidden-dropout keep bits
   // every parameter column sum (bias, gamma, beta gradients) leaves its
   // producer as partial rows in a slot of its own; one launch at the end sums them
   FinalizeList fin;
@@ -435,12 +450,12 @@ tl_status layer_backward(tl_layer* L, const void* x, const void* dy, const tl_we
 
   auto ln_bwd = [&](const void* dyln, const void* xin, const void* yln, const float* mean, const float* rstd,
                     const void* gamma, const void* beta, const void* res, void* dxo, void* drop_out, int site,
-                    float* dgamma, float* dbeta, float* dsum, int slot0) {
+                    float* dgamma, float* dbeta, float* dsum, int slot0, const uint8_t* keep8) {
     LnBwdArgs a;
     std::memset(&a, 0, sizeof(a));
     a.dy = dyln; a.x = inv ? nullptr : xin; a.y = inv ? yln : nullptr;
     a.mean = mean; a.rstd = rstd; a.gamma = gamma; a.beta = beta;
-    a.res = res; a.dx = dxo; a.drop_out = drop_out; a.drop = dh; a.site = site;
+    a.res = res; a.dx = dxo; a.drop_out = drop_out; a.drop = dh; a.site = site; a.keep8 = keep8;
     a.part_dgamma = slot(slot0); a.part_dbeta = slot(slot0 + 1); a.part_dsum = drop_out ? slot(slot0 + 2) : nullptr;
     a.rows = T; a.H = H;
     ProfScope p_(PC_LN_BWD, s);
@@ -500,25 +515,27 @@ tl_status layer_backward(tl_layer* L, const void* x, const void* dy, const tl_we
   if (L->pre_ln) {
     {
       ProfScope p_(PC_ROWWISE, s);
+      // draws its own bits: its rows stream through shared memory and a byte load per
+      // chunk would sit in that pipeline's critical path
       dropout_rows_run(dt, dy, L->dz2, dh, 2, T, H, slot(0), s);
       fin.job[fin.n++] = {slot(0), g->b2, rowdrop_parts(T), H};
     }
     ffn_bwd(L->h2, epi(EPI_STORE, L->dh, H), 1);                         // dH2 = dU W1
     ln_bwd(L->dh, L->x2, L->h2, L->mean2, L->rstd2, w->ln2_g, w->ln2_b, dy, L->dx2, L->da, 1,
-           g->ln2_g, g->ln2_b, g->bo, 2);
+           g->ln2_g, g->ln2_b, g->bo, 2, keepbits ? L->keep1 : nullptr);
     attn_bwd_block(L->h1, epi(EPI_STORE, L->dh, H), 5);                  // dH1 = dQKV Wqkv
     ln_bwd(L->dh, x, L->h1, L->mean1, L->rstd1, w->ln1_g, w->ln1_b, L->dx2, dx, nullptr, 0,
-           g->ln1_g, g->ln1_b, nullptr, 6);
+           g->ln1_g, g->ln1_b, nullptr, 6, nullptr);
   } else {
     const void* r2 = L->res2;
     const void* r1 = L->res1;
     ln_bwd(dy, r2, L->yout, L->mean2, L->rstd2, w->ln2_g, w->ln2_b, nullptr, L->dres, L->dz2, 2,
-           g->ln2_g, g->ln2_b, g->b2, 0);
+           g->ln2_g, g->ln2_b, g->b2, 0, keepbits ? L->keep2 : nullptr);
     EpiParams edx2 = epi(EPI_STORE, L->dx2, H);
     edx2.res = L->dres;
     ffn_bwd(L->x2, edx2, 3);                                              // dx2 = dU W1 + dres2
     ln_bwd(L->dx2, r1, L->x2, L->mean1, L->rstd1, w->ln1_g, w->ln1_b, nullptr, L->dres, L->da, 1,
-           g->ln1_g, g->ln1_b, g->bo, 4);
+           g->ln1_g, g->ln1_b, g->bo, 4, nullptr);
     EpiParams edx = epi(EPI_STORE, dx, H);
     edx.res = L->dres;
     attn_bwd_block(x, edx, 7);                                            // dx = dQKV Wqkv + dres1

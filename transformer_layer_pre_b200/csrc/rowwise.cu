@@ -180,7 +180,8 @@ __global__ void __launch_bounds__(kFwdWarps * 32) ln_fwd_kernel(const T* __restr
                                                                 const T* __restrict__ beta, T* __restrict__ y,
                                                                 float* __restrict__ mean_out,
                                                                 float* __restrict__ rstd_out, int rows, int H,
-                                                                float eps) {
+                                                                float eps, uint8_t* __restrict__ keep_out,
+                                                                DropoutParams dp, int site) {
   pdl_wait();
   pdl_launch_dependents();
   const int lane = threadIdx.x & 31;
@@ -229,6 +230,17 @@ __global__ void __launch_bounds__(kFwdWarps * 32) ln_fwd_kernel(const T* __restr
   if (lane == 0) {
     mean_out[row] = mean;
     rstd_out[row] = rstd;
+  }
+  if (keep_out) {
+    // dropout keep bits of this row for a downstream kernel (element index row*H + col)
+#pragma unroll
+    for (int c = 0; c < NCH; ++c) {
+      const int col = (lane + 32 * c) * 8;
+      if (col < H) {
+        const uint64_t e8 = ((uint64_t)row * H + col) >> 3;
+        keep_out[e8] = (uint8_t)dropout_bits8(dp, site, e8);
+      }
+    }
   }
 }
 
@@ -320,7 +332,8 @@ __global__ void __launch_bounds__(512) ln_bwd_kernel(LnBwdArgs a) {
       }
       store8<T>(static_cast<T*>(a.dx) + off, o);
       if (a.drop_out) {
-        const uint32_t bits = a.drop.thr ? dropout_bits8(a.drop, a.site, off >> 3) : 0xFFu;
+        const uint32_t bits = a.keep8 ? (uint32_t)a.keep8[off >> 3]
+                                      : (a.drop.thr ? dropout_bits8(a.drop, a.site, off >> 3) : 0xFFu);
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
           o[i] = round_f<T>(((bits >> i) & 1u) ? round_f<T>(o[i]) * sc : 0.0f);
@@ -455,7 +468,8 @@ __global__ void __launch_bounds__(kLnbPairs * 64, (sizeof(T) == 4 || (INV && DRO
       }
       store8<T>(static_cast<T*>(a.dx) + off, o);
       if constexpr (DROP) {
-        const uint32_t bits = a.drop.thr ? dropout_bits8(a.drop, a.site, off >> 3) : 0xFFu;
+        const uint32_t bits = a.keep8 ? (uint32_t)a.keep8[off >> 3]
+                                      : (a.drop.thr ? dropout_bits8(a.drop, a.site, off >> 3) : 0xFFu);
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
           o[i] = round_f<T>(((bits >> i) & 1u) ? round_f<T>(o[i]) * sc : 0.0f);
@@ -494,7 +508,8 @@ __global__ void __launch_bounds__(kLnbPairs * 64, (sizeof(T) == 4 || (INV && DRO
 template <typename T, int KR>
 __global__ void __launch_bounds__(512) dropout_rows_kernel(const T* __restrict__ in, T* __restrict__ out,
                                                            DropoutParams dp, int site, int rows, int H,
-                                                           float* __restrict__ part) {
+                                                           float* __restrict__ part,
+                                                           const uint8_t* __restrict__ keep8) {
   pdl_wait();
   pdl_launch_dependents();
   extern __shared__ __align__(128) uint8_t smem[];
@@ -518,7 +533,7 @@ __global__ void __launch_bounds__(512) dropout_rows_kernel(const T* __restrict__
       const size_t off = (size_t)row * H + col;
       float v[8];
       load8<T>(pipe.row(gi, 0, r) + col, v);
-      const uint32_t bits = dp.thr ? dropout_bits8(dp, site, off >> 3) : 0xFFu;
+      const uint32_t bits = keep8 ? (uint32_t)keep8[off >> 3] : (dp.thr ? dropout_bits8(dp, site, off >> 3) : 0xFFu);
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
         v[i] = round_f<T>(((bits >> i) & 1u) ? v[i] * sc : 0.0f);
@@ -638,12 +653,12 @@ int row_blocks(int rows) { return std::max(1, std::min(kMaxBlocks, (rows + 31) /
 
 template <typename T>
 void ln_fwd_t(const void* x, const void* g, const void* b, void* y, float* mean, float* rstd, int rows, int H,
-              float eps, cudaStream_t s) {
+              float eps, cudaStream_t s, uint8_t* keep_out, const DropoutParams& dp, int site) {
   const int blocks = (rows + kFwdWarps - 1) / kFwdWarps;
   TLP_NCH_SWITCH(H, {
-    launch_pdl(ln_fwd_kernel<T, NCH>, blocks, kFwdWarps * 32, 0, s, static_cast<const T*>(x), static_cast<const T*>(g),
-                                                            static_cast<const T*>(b), static_cast<T*>(y), mean, rstd,
-                                                            rows, H, eps);
+    launch_pdl(ln_fwd_kernel<T, NCH>, blocks, kFwdWarps * 32, 0, s, static_cast<const T*>(x),
+               static_cast<const T*>(g), static_cast<const T*>(b), static_cast<T*>(y), mean, rstd, rows, H, eps,
+               keep_out, dp, site);
   });
   count_launch();
 }
@@ -678,12 +693,12 @@ int ln_bwd_t(const LnBwdArgs& a, cudaStream_t s) {
 
 template <typename T>
 void dropout_rows_t(const void* in, void* out, const DropoutParams& dp, int site, int rows, int H, float* part,
-                    cudaStream_t s) {
+                    cudaStream_t s, const uint8_t* keep8) {
   TLP_KR_SWITCH(H, (int)sizeof(T), {
     const size_t sm = pipe_smem<T, KR, 1>(H);
     cudaFuncSetAttribute(dropout_rows_kernel<T, KR>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
-    launch_pdl(dropout_rows_kernel<T, KR>, rowdrop_parts(rows), row_threads(H), sm, s, 
-        static_cast<const T*>(in), static_cast<T*>(out), dp, site, rows, H, part);
+    launch_pdl(dropout_rows_kernel<T, KR>, rowdrop_parts(rows), row_threads(H), sm, s,
+               static_cast<const T*>(in), static_cast<T*>(out), dp, site, rows, H, part, keep8);
   });
   count_launch();
 }
@@ -699,10 +714,13 @@ int rowdrop_parts(int rows) { return row_blocks(rows); }
 int colsum_parts(int rows) { return std::max(1, std::min(kColParts, rows / 64)); }
 
 void ln_fwd_run(int dt, const void* x, const void* g, const void* b, void* y, float* mean, float* rstd, int rows,
-                int H, float eps, cudaStream_t s) {
-  if (dt == DT_F32) ln_fwd_t<float>(x, g, b, y, mean, rstd, rows, H, eps, s);
-  else if (dt == DT_F16) ln_fwd_t<half_t>(x, g, b, y, mean, rstd, rows, H, eps, s);
-  else ln_fwd_t<bf16_t>(x, g, b, y, mean, rstd, rows, H, eps, s);
+                int H, float eps, cudaStream_t s, uint8_t* keep_out, const DropoutParams* dp, int site) {
+  DropoutParams d = {};
+  if (keep_out && dp && dp->thr) d = *dp;
+  else keep_out = nullptr;
+  if (dt == DT_F32) ln_fwd_t<float>(x, g, b, y, mean, rstd, rows, H, eps, s, keep_out, d, site);
+  else if (dt == DT_F16) ln_fwd_t<half_t>(x, g, b, y, mean, rstd, rows, H, eps, s, keep_out, d, site);
+  else ln_fwd_t<bf16_t>(x, g, b, y, mean, rstd, rows, H, eps, s, keep_out, d, site);
 }
 
 template <typename T>
@@ -726,10 +744,10 @@ int rowwise_take_error() {
 }
 
 void dropout_rows_run(int dt, const void* in, void* out, const DropoutParams& dp, int site, int rows, int H,
-                      float* part, cudaStream_t s) {
-  if (dt == DT_F32) dropout_rows_t<float>(in, out, dp, site, rows, H, part, s);
-  else if (dt == DT_F16) dropout_rows_t<half_t>(in, out, dp, site, rows, H, part, s);
-  else dropout_rows_t<bf16_t>(in, out, dp, site, rows, H, part, s);
+                      float* part, cudaStream_t s, const uint8_t* keep8) {
+  if (dt == DT_F32) dropout_rows_t<float>(in, out, dp, site, rows, H, part, s, keep8);
+  else if (dt == DT_F16) dropout_rows_t<half_t>(in, out, dp, site, rows, H, part, s, keep8);
+  else dropout_rows_t<bf16_t>(in, out, dp, site, rows, H, part, s, keep8);
 }
 
 void colsum_run(int dt, const void* X, int rows, int cols, float* part, cudaStream_t s) {
