@@ -653,10 +653,12 @@ __global__ void __launch_bounds__(kBwdThreads)
 // One CTA per SM walks (sequence, head) items; every item is one 128-query x
 // 128-key tile.  Q/K/V, the score accumulator S and the output accumulator O
 // are double-buffered by item parity, so item i+1's loads and Q K^T overlap
-// item i's softmax, and item i's output is written while item i+1's softmax
-// runs.  Warps: 0 TMA, 1 MMA, 2-9 softmax: warp w owns TMEM lanes 32*(w%4)
-// (one query row per thread) and key columns 64*((w-2)/4) .. +63; the two
-// threads of a row combine their maxima and sums through shared memory.
+// item i's softmax.  Warps: 0 TMA, 1 MMA, 2-9 softmax in two groups of four
+// (warps 2-5 take the even items of this CTA, warps 6-9 the odd ones, so two
+// items are in their softmax at once); warp w owns TMEM lanes 32*(w%4), one
+// thread per query row and all 128 keys of it (a first pass over the
+// accumulator for the row maximum, a second for P), so no thread waits for
+// another; the same group then writes the item's output rows.
 // Warps 10-13 run ahead of the softmax by up to two items: per item they
 // draw the dropout keep bits of all 128 x 128 elements (thread = query row,
 // 16 Philox calls) and stage the item's additive key mask (log2 units, -inf
@@ -664,7 +666,7 @@ __global__ void __launch_bounds__(kBwdThreads)
 constexpr int kPFwdThreads = 448;
 constexpr int kPFwdBits = 128 * 16;                      // keep bits of one item: [row][16 bytes]
 constexpr int kPFwdMask = 128 * 4;                       // mask row of one item: [128] float
-constexpr int kPFwdSmem = 10 * TB + 4096 + 2 * kPFwdBits + 2 * kPFwdMask + 1024 + 256;
+constexpr int kPFwdSmem = 10 * TB + 4096 + 2 * kPFwdBits + 2 * kPFwdMask + 1024 + 256;   // 4 KB after the tiles unused
 
 __device__ __forceinline__ float ex2_fast(float x) {
   float r;
@@ -680,8 +682,6 @@ __global__ void __launch_bounds__(kPFwdThreads, 1)
   uint8_t* sm = align1024(smem_raw);
   // per slot j: Q at j*3TB, K at +TB, V at +2TB; P pairs after the six tiles
   uint8_t* sP0 = sm + 6 * TB;
-  // row exchange: [max | sum][2 slots][2 halves][128 rows] floats
-  float* xch = reinterpret_cast<float*>(sm + 10 * TB);
   uint8_t* sbits = sm + 10 * TB + 4096;                                   // [2][128][16]
   float* smask = reinterpret_cast<float*>(sbits + 2 * kPFwdBits);         // [2][128]
   uint64_t* bar = reinterpret_cast<uint64_t*>(sbits + 2 * kPFwdBits + 2 * kPFwdMask);
@@ -697,11 +697,11 @@ __global__ void __launch_bounds__(kPFwdThreads, 1)
       mbar_init(&in_full[j], 1);
       mbar_init(&in_empty[j], 1);
       mbar_init(&s_full[j], 1);
-      mbar_init(&p_full[j], 256);
+      mbar_init(&p_full[j], 128);
       mbar_init(&o_full[j], 1);
-      mbar_init(&o_free[j], 256);
+      mbar_init(&o_free[j], 128);
       mbar_init(&aux_full[j], 128);
-      mbar_init(&aux_free[j], 256);
+      mbar_init(&aux_free[j], 128);
     }
     fence_barrier_init();
   }
@@ -788,95 +788,91 @@ __global__ void __launch_bounds__(kPFwdThreads, 1)
       mbar_arrive(&aux_full[j]);
     }
   } else {
+    // softmax group grp (0: warps 2-5, 1: warps 6-9) owns the items n with n % 2 == grp, slot j = grp
     const int quarter = warp & 3;
-    const int hf = (warp - 2) >> 2;
+    const int grp = (warp - 2) >> 2;
+    const int j = grp;
     const int r = quarter * 32 + lane;
     const uint32_t lo = (uint32_t)(quarter * 32) << 16;
     const float c2 = a.scale * kLog2e;
     const float dsc = a.drop.thr ? a.drop.scale : 1.0f;
-    const int kc0 = hf * 64;
-    bool ok = true;
-    int n = 0;
-    int prev_item = -1;
-    float prev_inv = 0.0f;
-    // output of item n-1 (slot jp): O rows to ctx, one 32-column half per thread
-    auto epilogue = [&](int item, int np, float inv) -> bool {
-      const int jp = np & 1;
-      if (!mbar_wait_warp(&o_full[jp], (np >> 1) & 1, a.err, 56)) return false;
+    const float* mrow = smask + j * 128;
+    int k = 0;   // this group's item count: item n = 2k + grp
+    for (int it = blockIdx.x + grp * gridDim.x; it < nitems; it += 2 * gridDim.x, ++k) {
+      const uint32_t par = k & 1;
+      if (!mbar_wait_warp(&aux_full[j], par, a.err, 59)) break;
+      const uint4 kb16 = a.drop.thr ? *reinterpret_cast<const uint4*>(sbits + j * kPFwdBits + r * 16)
+                                    : make_uint4(~0u, ~0u, ~0u, ~0u);
+      if (!mbar_wait_warp(&s_full[j], par, a.err, 57)) break;
       tc_fence_after();
-      float o[32];
-      tmem_ld32(tmem + 256 + 64 * jp + lo + hf * 32, o);
-      tc_fence_before();
-      mbar_arrive(&o_free[jp]);
-      const int b = item / a.nh, h = item - (item / a.nh) * a.nh;
-      if (r < S) {
-        T* dst = static_cast<T*>(a.ctx) + ((size_t)b * S + r) * a.H + h * HD + hf * 32;
+      const uint32_t ts = tmem + 128 * j + lo;
+      // pass 1: row maximum over the 128 keys (scaled scores + mask, log2 units)
+      float mx = -INFINITY;
+#pragma unroll 1
+      for (int c = 0; c < 4; ++c) {
+        float sv[32];
+        tmem_ld32(ts + c * 32, sv);
 #pragma unroll
-        for (int c = 0; c < 32; c += 8) {
+        for (int t = 0; t < 32; t += 4) {
+          const float4 m4 = *reinterpret_cast<const float4*>(mrow + c * 32 + t);
+          mx = fmaxf(mx, fmaxf(fmaxf(fmaf(sv[t], c2, m4.x), fmaf(sv[t + 1], c2, m4.y)),
+                               fmaxf(fmaf(sv[t + 2], c2, m4.z), fmaf(sv[t + 3], c2, m4.w))));
+        }
+      }
+      // a row whose keys are all masked has mx = -inf: every p is 0
+      const float msub = mx == -INFINITY ? 0.0f : mx;
+      // pass 2: P = 2^(x - max), dropped and scaled, into the P tile; row sum of the undropped P
+      float lsum = 0.0f, lsum2 = 0.0f;
+#pragma unroll 1
+      for (int c = 0; c < 4; ++c) {
+        float sv[32];
+        tmem_ld32(ts + c * 32, sv);
+        const uint32_t bw = c == 0 ? kb16.x : (c == 1 ? kb16.y : (c == 2 ? kb16.z : kb16.w));
+#pragma unroll
+        for (int g = 0; g < 4; ++g) {
+          const uint32_t bits = (bw >> (8 * g)) & 0xFFu;
+          const float4 m0 = *reinterpret_cast<const float4*>(mrow + c * 32 + g * 8);
+          const float4 m1 = *reinterpret_cast<const float4*>(mrow + c * 32 + g * 8 + 4);
+          const float ml[8] = {m0.x, m0.y, m0.z, m0.w, m1.x, m1.y, m1.z, m1.w};
+          float pv[8];
+#pragma unroll
+          for (int t = 0; t < 8; ++t) {
+            const float p = ex2_fast(fmaf(sv[g * 8 + t], c2, ml[t]) - msub);
+            if (t & 1) lsum2 += p;
+            else lsum += p;
+            pv[t] = ((bits >> t) & 1u) ? p * dsc : 0.0f;
+          }
+          pair_store8<T>(sP0 + j * 2 * TB, r, c * 4 + g, pv);
+        }
+      }
+      lsum += lsum2;
+      mbar_arrive(&aux_free[j]);
+      // P is written and S has been read: both hand-overs ride on p_full
+      tc_fence_before();
+      fence_proxy_async_smem();
+      mbar_arrive(&p_full[j]);
+      if (r < S) a.lse[(size_t)it * S + r] = lsum > 0.0f ? (mx + log2f(lsum)) * kLn2 : INFINITY;
+      // this item's output rows once P V is in TMEM
+      const float inv = lsum > 0.0f ? 1.0f / lsum : 0.0f;
+      if (!mbar_wait_warp(&o_full[j], par, a.err, 56)) break;
+      tc_fence_after();
+      float o[64];
+      tmem_ld32(tmem + 256 + 64 * j + lo, *reinterpret_cast<float(*)[32]>(o));
+      tmem_ld32(tmem + 256 + 64 * j + lo + 32, *reinterpret_cast<float(*)[32]>(o + 32));
+      tc_fence_before();
+      mbar_arrive(&o_free[j]);
+      const int b = it / a.nh, h = it - (it / a.nh) * a.nh;
+      if (r < S) {
+        T* dst = static_cast<T*>(a.ctx) + ((size_t)b * S + r) * a.H + h * HD;
+#pragma unroll
+        for (int c = 0; c < 64; c += 8) {
           float w8[8];
 #pragma unroll
           for (int t = 0; t < 8; ++t) w8[t] = o[c + t] * inv;
           store8<T>(dst + c, w8);
         }
       }
-      return true;
-    };
-    for (int it = blockIdx.x; it < nitems && ok; it += gridDim.x, ++n) {
-      const int j = n & 1;
-      if (!(ok = mbar_wait_warp(&aux_full[j], (n >> 1) & 1, a.err, 59))) break;
-      const uint2 kb8 = a.drop.thr ? *reinterpret_cast<const uint2*>(sbits + j * kPFwdBits + r * 16 + hf * 8)
-                                   : make_uint2(0xFFFFFFFFu, 0xFFFFFFFFu);
-      if (!(ok = mbar_wait_warp(&s_full[j], (n >> 1) & 1, a.err, 57))) break;
-      tc_fence_after();
-      float sv[64];
-      tmem_ld32(tmem + 128 * j + lo + kc0, *reinterpret_cast<float(*)[32]>(sv));
-      tmem_ld32(tmem + 128 * j + lo + kc0 + 32, *reinterpret_cast<float(*)[32]>(sv + 32));
-      float mx = -INFINITY;
-#pragma unroll
-      for (int t = 0; t < 64; t += 4) {
-        const float4 m4 = *reinterpret_cast<const float4*>(smask + j * 128 + kc0 + t);
-        sv[t] = fmaf(sv[t], c2, m4.x);
-        sv[t + 1] = fmaf(sv[t + 1], c2, m4.y);
-        sv[t + 2] = fmaf(sv[t + 2], c2, m4.z);
-        sv[t + 3] = fmaf(sv[t + 3], c2, m4.w);
-        mx = fmaxf(fmaxf(mx, fmaxf(sv[t], sv[t + 1])), fmaxf(sv[t + 2], sv[t + 3]));
-      }
-      mbar_arrive(&aux_free[j]);
-      float* xm = xch + j * 256;
-      xm[hf * 128 + r] = mx;
-      named_barrier(1, 256);
-      mx = fmaxf(mx, xm[(1 - hf) * 128 + r]);
-      // a row whose keys are all masked has mx = -inf: every p is 0
-      const float msub = mx == -INFINITY ? 0.0f : mx;
-      float lsum = 0.0f;
-#pragma unroll
-      for (int g = 0; g < 8; ++g) {
-        const uint32_t bits = ((g < 4 ? kb8.x : kb8.y) >> (8 * (g & 3))) & 0xFFu;
-        float pv[8];
-#pragma unroll
-        for (int t = 0; t < 8; ++t) {
-          const float p = ex2_fast(sv[g * 8 + t] - msub);
-          lsum += p;
-          pv[t] = ((bits >> t) & 1u) ? p * dsc : 0.0f;
-        }
-        pair_store8<T>(sP0 + j * 2 * TB, r, hf * 8 + g, pv);
-      }
-      // P is written and S has been read: both hand-overs ride on p_full
-      tc_fence_before();
-      fence_proxy_async_smem();
-      mbar_arrive(&p_full[j]);
-      // row sum across the two halves (second exchange buffer)
-      float* xs = xch + 512 + j * 256;
-      xs[hf * 128 + r] = lsum;
-      named_barrier(1, 256);
-      const float l = lsum + xs[(1 - hf) * 128 + r];
-      if (hf == 0 && r < S) a.lse[(size_t)it * S + r] = l > 0.0f ? (mx + log2f(l)) * kLn2 : INFINITY;
-      // the previous item's output overlaps this item's softmax
-      if (prev_item >= 0 && !(ok = epilogue(prev_item, n - 1, prev_inv))) break;
-      prev_item = it;
-      prev_inv = l > 0.0f ? 1.0f / l : 0.0f;
     }
-    if (ok && prev_item >= 0) epilogue(prev_item, n - 1, prev_inv);
   }
   tc_fence_before();
   __syncthreads();

@@ -805,10 +805,16 @@ bool build_pair_gemm(PairGemm& P, const GemmDesc& gd, const EpiParams& e, int sp
 }
 
 // Plans a table schedule for two GEMMs on `pairs` CTA pairs: tiles sorted by
-// their K blocks (longest first, then GEMM and tile order), each given to
+// estimated cost (longest first, then GEMM and tile order), each given to
 // the pair with the least work so far (lowest index on ties).  False if a
 // pair would get more than kMaxItems tiles.
-bool plan_pair_table(PairSched& sch, const TcArgs& g0, const TcArgs& g1, int pairs) {
+// Estimated cost of a tile in tenths of a 64-wide K block of main loop:
+// its K blocks, weighted by the epilogue (the dGELU epilogue keeps the
+// epilogue warps busier than the main loop of its K = 1024 tiles, measured
+// ~1.45x per K block), plus a fixed per-tile fill/drain of ~4 K blocks.
+int tile_cost10(int kb, int kind) { return (epi_base(kind) == EPI_DGELU ? 145 : 100) * kb / 10 + 40; }
+
+bool plan_pair_table(PairSched& sch, const TcArgs& g0, int kind0, const TcArgs& g1, int kind1, int pairs) {
   struct Item { int kb, gi, tile; };
   std::vector<Item> items;
   for (int gi = 0; gi < 2; ++gi) {
@@ -817,7 +823,7 @@ bool plan_pair_table(PairSched& sch, const TcArgs& g0, const TcArgs& g1, int pai
     for (int t = 0; t < total; ++t) {
       const int sp = t / (g.tiles_m * g.tiles_n);
       const int kb0 = sp * g.kb_per_split;
-      items.push_back({std::min(g.kblocks, kb0 + g.kb_per_split) - kb0, gi, t});
+      items.push_back({tile_cost10(std::min(g.kblocks, kb0 + g.kb_per_split) - kb0, gi ? kind1 : kind0), gi, t});
     }
   }
   if (items.empty() || items.size() > (size_t)pairs * kMaxItems) return false;
@@ -868,7 +874,7 @@ int launch_tc_pair_group(const GemmDesc& ga, const EpiParams& ea, int splits_a, 
   PairSched sch;
   if (!build_pair_gemm<T, KA>(A, ga, ea, splits_a) || !build_pair_gemm<T, KB>(B, gb, eb, 1)) return 1;
   const int pairs = std::min(num_sms() / 2, kMaxPairs);
-  if (!plan_pair_table(sch, A.g, B.g, pairs)) {
+  if (!plan_pair_table(sch, A.g, KA, B.g, KB, pairs)) {
     int rc = launch_tc_pair<T, KA>(ga, ea, splits_a, s);
     return rc ? rc : launch_tc_pair<T, KB>(gb, eb, 1, s);
   }

@@ -481,10 +481,10 @@ tl_status layer_backward(tl_layer* L, const void* x, const void* dy, const tl_we
     if (fused_db1) edu.colsum = slot(db1_slot);
     const GemmDesc gw2 = gdesc(L, H, F, T, L->dz2, H, false, L->g, F, false);   // dW2 = dZ2^T G
     const GemmDesc gdu = gdesc(L, T, F, H, L->dz2, H, true, w->w2, F, false);   // dU = (dZ2 W2) GELU'(U)
-    // two launches: the dGELU epilogue makes dU's tiles slower than their
-    // K blocks say, which the grouped plan does not model (and in recompute
-    // mode G lives where dU goes, so dW2 must finish first anyway)
-    {
+    if (L->g != L->big) {
+      gemm2(L, gw2, ew2, gdu, edu, s);
+    } else {
+      // recompute mode: G lives where dU goes, so dW2 must finish first
       ProfScope p_(PC_GEMM, s);
       if (gemm_run(dt, gw2, ew2, s) != 0 || gemm_run(dt, gdu, edu, s) != 0) L->gemm_err = 1;
     }
