@@ -515,9 +515,7 @@ tl_status layer_backward(tl_layer* L, const void* x, const void* dy, const tl_we
   if (L->pre_ln) {
     {
       ProfScope p_(PC_ROWWISE, s);
-      // draws its own bits: its rows stream through shared memory and a byte load per
-      // chunk would sit in that pipeline's critical path
-      dropout_rows_run(dt, dy, L->dz2, dh, 2, T, H, slot(0), s);
+      dropout_rows_run(dt, dy, L->dz2, dh, 2, T, H, slot(0), s, keepbits ? L->keep2 : nullptr);
       fin.job[fin.n++] = {slot(0), g->b2, rowdrop_parts(T), H};
     }
     ffn_bwd(L->h2, epi(EPI_STORE, L->dh, H), 1);                         // dH2 = dU W1

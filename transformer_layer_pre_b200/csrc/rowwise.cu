@@ -547,6 +547,82 @@ __global__ void __launch_bounds__(512) dropout_rows_kernel(const T* __restrict__
   if (act) store_part(part, H, col, acc);
 }
 
+// Dropout backward for H <= 1024 with precomputed keep bits: one warp per
+// row (lane-interleaved 8-column chunks, NCH per lane), the next row's data
+// and keep bytes loaded before the current row is written; column sums in
+// registers, added over the block's 8 warps in warp order at the end (one
+// partial row per block, like the row-block kernel above).
+constexpr int kDropWarps = 8;
+
+template <typename T, int NCH>
+__global__ void __launch_bounds__(kDropWarps * 32) dropout_rows_warp_kernel(const T* __restrict__ in,
+                                                                            T* __restrict__ out, float scale,
+                                                                            int rows, int H, float* __restrict__ part,
+                                                                            const uint8_t* __restrict__ keep8) {
+  pdl_wait();
+  pdl_launch_dependents();
+  extern __shared__ __align__(16) float dred[];   // [kDropWarps][H]
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  float acc[NCH][8];
+#pragma unroll
+  for (int c = 0; c < NCH; ++c)
+#pragma unroll
+    for (int i = 0; i < 8; ++i) acc[c][i] = 0.0f;
+  int r0, r1;
+  row_range(rows, r0, r1);
+  Raw8<T> rv[NCH];
+  uint32_t kb[NCH];
+  auto fetch = [&](int row) {
+#pragma unroll
+    for (int c = 0; c < NCH; ++c) {
+      const int col = (lane + 32 * c) * 8;
+      const bool ok = row < r1 && col < H;
+      const size_t off = (size_t)row * H + col;
+      rv[c] = ok ? raw8_stream<T>(in + off) : raw8_zero<T>();
+      kb[c] = ok ? (uint32_t)keep8[off >> 3] : 0u;
+    }
+  };
+  int row = r0 + warp;
+  fetch(row);
+  for (; row < r1; row += kDropWarps) {
+    float v[NCH][8];
+    uint32_t bits[NCH];
+#pragma unroll
+    for (int c = 0; c < NCH; ++c) {
+      raw8_unpack<T>(rv[c], v[c]);
+      bits[c] = kb[c];
+    }
+    fetch(row + kDropWarps);
+#pragma unroll
+    for (int c = 0; c < NCH; ++c) {
+      const int col = (lane + 32 * c) * 8;
+      if (col >= H) continue;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        v[c][i] = round_f<T>(((bits[c] >> i) & 1u) ? v[c][i] * scale : 0.0f);
+        acc[c][i] += v[c][i];
+      }
+      store8<T>(out + (size_t)row * H + col, v[c]);
+    }
+  }
+#pragma unroll
+  for (int c = 0; c < NCH; ++c) {
+    const int col = (lane + 32 * c) * 8;
+    if (col < H) {
+      float* d = dred + warp * H + col;
+      reinterpret_cast<float4*>(d)[0] = make_float4(acc[c][0], acc[c][1], acc[c][2], acc[c][3]);
+      reinterpret_cast<float4*>(d)[1] = make_float4(acc[c][4], acc[c][5], acc[c][6], acc[c][7]);
+    }
+  }
+  __syncthreads();
+  for (int col = threadIdx.x; col < H; col += blockDim.x) {
+    float t = 0.0f;
+#pragma unroll
+    for (int w = 0; w < kDropWarps; ++w) t += dred[w * H + col];
+    part[(size_t)blockIdx.x * H + col] = t;
+  }
+}
+
 // ------------------------------------------------------------------ column sums
 constexpr int kColParts = 64;
 
@@ -743,8 +819,29 @@ int rowwise_take_error() {
   return v;
 }
 
+template <typename T>
+void dropout_rows_warp_t(const void* in, void* out, float scale, int rows, int H, float* part, cudaStream_t s,
+                         const uint8_t* keep8) {
+  const size_t sm = (size_t)kDropWarps * H * sizeof(float);
+  TLP_NCH_SWITCH(H, {
+    if constexpr (NCH <= 4) {
+      cudaFuncSetAttribute(dropout_rows_warp_kernel<T, NCH>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+      launch_pdl(dropout_rows_warp_kernel<T, NCH>, rowdrop_parts(rows), kDropWarps * 32, sm, s,
+                 static_cast<const T*>(in), static_cast<T*>(out), scale, rows, H, part, keep8);
+    }
+  });
+  count_launch();
+}
+
 void dropout_rows_run(int dt, const void* in, void* out, const DropoutParams& dp, int site, int rows, int H,
                       float* part, cudaStream_t s, const uint8_t* keep8) {
+  if (keep8 && dp.thr && H <= 1024) {
+    // keep bits at hand: the warp-per-row form (no Philox, no shared-memory pipeline)
+    if (dt == DT_F32) dropout_rows_warp_t<float>(in, out, dp.scale, rows, H, part, s, keep8);
+    else if (dt == DT_F16) dropout_rows_warp_t<half_t>(in, out, dp.scale, rows, H, part, s, keep8);
+    else dropout_rows_warp_t<bf16_t>(in, out, dp.scale, rows, H, part, s, keep8);
+    return;
+  }
   if (dt == DT_F32) dropout_rows_t<float>(in, out, dp, site, rows, H, part, s, keep8);
   else if (dt == DT_F16) dropout_rows_t<half_t>(in, out, dp, site, rows, H, part, s, keep8);
   else dropout_rows_t<bf16_t>(in, out, dp, site, rows, H, part, s, keep8);
