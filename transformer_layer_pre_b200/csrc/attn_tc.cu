@@ -666,7 +666,8 @@ __global__ void __launch_bounds__(kBwdThreads)
 constexpr int kPFwdThreads = 448;
 constexpr int kPFwdBits = 128 * 16;                      // keep bits of one item: [row][16 bytes]
 constexpr int kPFwdMask = 128 * 4;                       // mask row of one item: [128] float
-constexpr int kPFwdSmem = 10 * TB + 4096 + 2 * kPFwdBits + 2 * kPFwdMask + 1024 + 256;   // 4 KB after the tiles unused
+constexpr int kPFwdIn = 3;                               // Q/K/V input slots (loads run up to 3 items ahead)
+constexpr int kPFwdSmem = (3 * kPFwdIn + 4) * TB + 2 * kPFwdBits + 2 * kPFwdMask + 1024 + 256;
 
 __device__ __forceinline__ float ex2_fast(float x) {
   float r;
@@ -680,22 +681,24 @@ __global__ void __launch_bounds__(kPFwdThreads, 1)
                         const __grid_constant__ CUtensorMap tv, AttnTc a) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = align1024(smem_raw);
-  // per slot j: Q at j*3TB, K at +TB, V at +2TB; P pairs after the six tiles
-  uint8_t* sP0 = sm + 6 * TB;
-  uint8_t* sbits = sm + 10 * TB + 4096;                                   // [2][128][16]
+  // input slot i: Q at i*3TB, K at +TB, V at +2TB; then the two P pairs (by item parity)
+  uint8_t* sP0 = sm + 3 * kPFwdIn * TB;
+  uint8_t* sbits = sP0 + 4 * TB;                                          // [2][128][16]
   float* smask = reinterpret_cast<float*>(sbits + 2 * kPFwdBits);         // [2][128]
   uint64_t* bar = reinterpret_cast<uint64_t*>(sbits + 2 * kPFwdBits + 2 * kPFwdMask);
-  uint64_t *in_full = bar, *in_empty = bar + 2, *s_full = bar + 4, *p_full = bar + 6, *o_full = bar + 8,
-           *o_free = bar + 10, *aux_full = bar + 12, *aux_free = bar + 14;
-  uint32_t* tslot = reinterpret_cast<uint32_t*>(bar + 16);
+  uint64_t *in_full = bar, *in_empty = bar + kPFwdIn, *s_full = bar + 2 * kPFwdIn, *p_full = s_full + 2,
+           *o_full = s_full + 4, *o_free = s_full + 6, *aux_full = s_full + 8, *aux_free = s_full + 10;
+  uint32_t* tslot = reinterpret_cast<uint32_t*>(s_full + 12);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int S = a.S;
   const int nitems = a.B * a.nh;
   if (threadIdx.x == 0) {
+    for (int i = 0; i < kPFwdIn; ++i) {
+      mbar_init(&in_full[i], 1);
+      mbar_init(&in_empty[i], 1);
+    }
     for (int j = 0; j < 2; ++j) {
-      mbar_init(&in_full[j], 1);
-      mbar_init(&in_empty[j], 1);
       mbar_init(&s_full[j], 1);
       mbar_init(&p_full[j], 128);
       mbar_init(&o_full[j], 1);
@@ -717,14 +720,14 @@ __global__ void __launch_bounds__(kPFwdThreads, 1)
     if (lane == 0) {
       int n = 0;
       for (int it = blockIdx.x; it < nitems; it += gridDim.x, ++n) {
-        const int j = n & 1;
-        if (!mbar_wait(&in_empty[j], ((n >> 1) & 1) ^ 1, a.err, 51)) break;
-        uint8_t* base = sm + j * 3 * TB;
-        mbar_arrive_expect_tx(&in_full[j], 3 * TB);
+        const int i = n % kPFwdIn;
+        if (!mbar_wait(&in_empty[i], ((n / kPFwdIn) & 1) ^ 1, a.err, 51)) break;
+        uint8_t* base = sm + i * 3 * TB;
+        mbar_arrive_expect_tx(&in_full[i], 3 * TB);
         const int row0 = it * S;
-        tma_load_2d(base, &tq, &in_full[j], 0, row0);
-        tma_load_2d(base + TB, &tk, &in_full[j], 0, row0);
-        tma_load_2d(base + 2 * TB, &tv, &in_full[j], 0, row0);
+        tma_load_2d(base, &tq, &in_full[i], 0, row0);
+        tma_load_2d(base + TB, &tk, &in_full[i], 0, row0);
+        tma_load_2d(base + 2 * TB, &tv, &in_full[i], 0, row0);
       }
     }
   } else if (warp == 1) {
@@ -733,12 +736,12 @@ __global__ void __launch_bounds__(kPFwdThreads, 1)
       const uint32_t id_o = idesc_f16(128, 64, a.bf16 != 0, false, true);
       // S = Q K^T of item n into S[n&1]
       auto mma_s = [&](int n) -> bool {
-        const int j = n & 1;
-        if (!mbar_wait(&in_full[j], (n >> 1) & 1, a.err, 52)) return false;
+        const int j = n & 1, i = n % kPFwdIn;
+        if (!mbar_wait(&in_full[i], (n / kPFwdIn) & 1, a.err, 52)) return false;
         // S[j] is free once the softmax of item n-2 wrote its P (it read S first)
         if (!mbar_wait(&p_full[j], ((n >> 1) & 1) ^ 1, a.err, 53)) return false;
         tc_fence_after();
-        const uint32_t aQ = smem_u32(sm + j * 3 * TB), aK = aQ + TB;
+        const uint32_t aQ = smem_u32(sm + i * 3 * TB), aK = aQ + TB;
 #pragma unroll
         for (int kk = 0; kk < HD / 16; ++kk) mma_f16(tmem + 128 * j, dk_tile(aQ, kk), dk_tile(aK, kk), id_s, kk > 0);
         mma_commit(&s_full[j]);
@@ -755,13 +758,13 @@ __global__ void __launch_bounds__(kPFwdThreads, 1)
         if (!(ok = mbar_wait(&p_full[j], (n >> 1) & 1, a.err, 54))) break;
         if (!(ok = mbar_wait(&o_free[j], ((n >> 1) & 1) ^ 1, a.err, 55))) break;
         tc_fence_after();
-        const uint32_t aV = smem_u32(sm + j * 3 * TB) + 2 * TB;
+        const uint32_t aV = smem_u32(sm + (n % kPFwdIn) * 3 * TB) + 2 * TB;
         const uint32_t aP = smem_u32(sP0 + j * 2 * TB);
 #pragma unroll
         for (int kk = 0; kk < TILE / 16; ++kk)
           mma_f16(tmem + 256 + 64 * j, dk_pair(aP, kk), dmn_tile(aV, kk), id_o, kk > 0);
         mma_commit(&o_full[j]);
-        mma_commit(&in_empty[j]);
+        mma_commit(&in_empty[n % kPFwdIn]);
       }
     }
   } else if (warp >= 10) {
