@@ -387,7 +387,9 @@ def layer_backward(cfg: LayerConfig, sv: dict, dy):
     """Backward pass of layer_forward: returns (dx, grads) where grads holds
     the gradient of every weight in WEIGHT_NAMES, summed over the sequences
     of the forward.  Bias gradients are column sums of the stored output
-    gradient of their Linear."""
+    gradient of their Linear.  In storage-rounded mode GELU'(U) is rounded
+    to the storage type before it scales dU (the CUDA path keeps it in HBM
+    from the forward, or rounds it so when it recomputes it from U)."""
     dy = np.asarray(dy, dtype=np.float64)
     R, W, mask, seq_index = sv["R"], sv["W"], sv["mask"], sv["seq_index"]
     ph = cfg.hidden_dropout
@@ -396,7 +398,7 @@ def layer_backward(cfg: LayerConfig, sv: dict, dy):
         dz2 = R(_apply_dropout(dy, sv["keep2"], ph))
         gr["b2"] = _colsum(dz2)
         gr["w2"] = _wgrad(dz2, sv["g"])
-        du = R((dz2 @ W["w2"]) * _gelu_pair(cfg)[1](sv["u"]))
+        du = R((dz2 @ W["w2"]) * R(_gelu_pair(cfg)[1](sv["u"])))
         gr["b1"] = _colsum(du)
         gr["w1"] = _wgrad(du, sv["h2"])
         dh2 = R(du @ W["w1"])
@@ -418,7 +420,7 @@ def layer_backward(cfg: LayerConfig, sv: dict, dy):
         dz2 = R(_apply_dropout(dres2, sv["keep2"], ph))
         gr["b2"] = _colsum(dz2)
         gr["w2"] = _wgrad(dz2, sv["g"])
-        du = R((dz2 @ W["w2"]) * _gelu_pair(cfg)[1](sv["u"]))
+        du = R((dz2 @ W["w2"]) * R(_gelu_pair(cfg)[1](sv["u"])))
         gr["b1"] = _colsum(du)
         gr["w1"] = _wgrad(du, sv["x2"])
         dx2 = R(du @ W["w1"] + dres2)

@@ -58,6 +58,7 @@ struct AttnTc {
   void* dqkv;
   float* colsum;        // fused QKV bias-gradient partials (persistent backward), or null
   int fuse_dq;
+  int ctx_tma;          // persistent forward: ctx rows leave by TMA store (S % 32 == 0)
   int bf16;
   int* err;
 };
@@ -678,7 +679,8 @@ __device__ __forceinline__ float ex2_fast(float x) {
 template <typename T>
 __global__ void __launch_bounds__(kPFwdThreads, 1)
     attn_fwd_tc_persist(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
-                        const __grid_constant__ CUtensorMap tv, AttnTc a) {
+                        const __grid_constant__ CUtensorMap tv, const __grid_constant__ CUtensorMap tctx,
+                        AttnTc a) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = align1024(smem_raw);
   // input slot i: Q at i*3TB, K at +TB, V at +2TB; then the two P pairs (by item parity)
@@ -800,6 +802,9 @@ __global__ void __launch_bounds__(kPFwdThreads, 1)
     const float c2 = a.scale * kLog2e;
     const float dsc = a.drop.thr ? a.drop.scale : 1.0f;
     const float* mrow = smask + j * 128;
+    // this warp's 32 output rows staged as one 32 x 128-byte swizzled box
+    // inside the group's P pair (free between P V and the next item's P)
+    uint8_t* ostage = sP0 + j * 2 * TB + quarter * 4096;
     int k = 0;   // this group's item count: item n = 2k + grp
     for (int it = blockIdx.x + grp * gridDim.x; it < nitems; it += 2 * gridDim.x, ++k) {
       const uint32_t par = k & 1;
@@ -808,6 +813,10 @@ __global__ void __launch_bounds__(kPFwdThreads, 1)
                                     : make_uint4(~0u, ~0u, ~0u, ~0u);
       if (!mbar_wait_warp(&s_full[j], par, a.err, 57)) break;
       tc_fence_after();
+      if (a.ctx_tma) {
+        if (lane == 0) bulk_wait_read<0>();
+        __syncwarp();
+      }
       const uint32_t ts = tmem + 128 * j + lo;
       // pass 1: row maximum over the 128 keys (scaled scores + mask, log2 units)
       float mx = -INFINITY;
@@ -843,7 +852,7 @@ __global__ void __launch_bounds__(kPFwdThreads, 1)
             const float p = ex2_fast(fmaf(sv[g * 8 + t], c2, ml[t]) - msub);
             if (t & 1) lsum2 += p;
             else lsum += p;
-            pv[t] = ((bits >> t) & 1u) ? p * dsc : 0.0f;
+            pv[t] = ((bits >> t) & 1u) ? p : 0.0f;
           }
           pair_store8<T>(sP0 + j * 2 * TB, r, c * 4 + g, pv);
         }
@@ -855,8 +864,9 @@ __global__ void __launch_bounds__(kPFwdThreads, 1)
       fence_proxy_async_smem();
       mbar_arrive(&p_full[j]);
       if (r < S) a.lse[(size_t)it * S + r] = lsum > 0.0f ? (mx + log2f(lsum)) * kLn2 : INFINITY;
-      // this item's output rows once P V is in TMEM
-      const float inv = lsum > 0.0f ? 1.0f / lsum : 0.0f;
+      // this item's output rows once P V is in TMEM (P carried the keep
+      // mask only; the dropout scale joins the normalisation here)
+      const float inv = lsum > 0.0f ? dsc / lsum : 0.0f;
       if (!mbar_wait_warp(&o_full[j], par, a.err, 56)) break;
       tc_fence_after();
       float o[64];
@@ -865,7 +875,24 @@ __global__ void __launch_bounds__(kPFwdThreads, 1)
       tc_fence_before();
       mbar_arrive(&o_free[j]);
       const int b = it / a.nh, h = it - (it / a.nh) * a.nh;
-      if (r < S) {
+      if (a.ctx_tma) {
+        // whole 32-row boxes (S % 32 == 0): swizzled smem rows, one TMA store per warp
+        if (quarter * 32 < S) {
+#pragma unroll
+          for (int c = 0; c < 8; ++c) {
+            float w8[8];
+#pragma unroll
+            for (int t = 0; t < 8; ++t) w8[t] = o[c * 8 + t] * inv;
+            store8<T>(reinterpret_cast<T*>(ostage + lane * 128 + ((c ^ (lane & 7)) << 4)), w8);
+          }
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            tma_store_2d(&tctx, ostage, h * HD, b * S + quarter * 32);
+            bulk_commit();
+          }
+        }
+      } else if (r < S) {
         T* dst = static_cast<T*>(a.ctx) + ((size_t)b * S + r) * a.H + h * HD;
 #pragma unroll
         for (int c = 0; c < 64; c += 8) {
@@ -876,6 +903,8 @@ __global__ void __launch_bounds__(kPFwdThreads, 1)
         }
       }
     }
+    if (a.ctx_tma && lane == 0) bulk_wait_all();
+    __syncwarp();
   }
   tc_fence_before();
   __syncthreads();
@@ -1145,13 +1174,14 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-// [rows][cols] row-major 16-bit matrix with row stride ld; box 64 x 128 rows.
-bool map_tile(CUtensorMap* m, const void* p, bool bf16, uint64_t cols, uint64_t rows, uint64_t ld) {
+// [rows][cols] row-major 16-bit matrix with row stride ld; box 64 x box_rows.
+bool map_tile(CUtensorMap* m, const void* p, bool bf16, uint64_t cols, uint64_t rows, uint64_t ld,
+              uint32_t box_rows = 128) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return false;
   cuuint64_t dims[2] = {cols, rows};
   cuuint64_t strides[1] = {ld * 2};
-  cuuint32_t box[2] = {64, 128};
+  cuuint32_t box[2] = {64, box_rows};
   cuuint32_t es[2] = {1, 1};
   return fn(m, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<void*>(p),
             dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -1178,6 +1208,7 @@ AttnTc make_args(int dt, const AttnArgs& a) {
   t.dqkv = a.dqkv;
   t.colsum = a.colsum;
   t.fuse_dq = 0;
+  t.ctx_tma = 0;
   t.bf16 = dt == DT_BF16;
   t.err = attn_error_word();
   return t;
@@ -1201,7 +1232,11 @@ void fwd_t(const AttnArgs& a, cudaStream_t s) {
     int nsm = 148;
     cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, 0);
     const int grid = std::min(a.B * a.nh, nsm);
-    launch_pdl(attn_fwd_tc_persist<T>, grid, kPFwdThreads, kPFwdSmem, s, mq, mk, mv, t);
+    // ctx (B*S, H) in 32-row boxes of one head; rows of a box stay inside one sequence when S % 32 == 0
+    CUtensorMap mc;
+    t.ctx_tma = a.S % 32 == 0 && map_tile(&mc, a.ctx, t.bf16, t.H, (uint64_t)a.B * a.S, t.H, 32) ? 1 : 0;
+    if (!t.ctx_tma) mc = mq;   // unused
+    launch_pdl(attn_fwd_tc_persist<T>, grid, kPFwdThreads, kPFwdSmem, s, mq, mk, mv, mc, t);
   } else {
     dim3 grid((a.S + TILE - 1) / TILE, a.nh, a.B);
     launch_pdl(attn_fwd_tc<T>, grid, kFwdThreads, kFwdSmem, s, mq, mk, mv, t);

@@ -232,15 +232,6 @@ __device__ __forceinline__ void gelu8(float (&v)[8]) {
     v[2 * i + 1] = g.y;
   }
 }
-// v *= GELU'(u) over 8 lanes.
-__device__ __forceinline__ void mul_gelu_grad8(float (&v)[8], const float (&u)[8]) {
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const float2 d = __fmul2_rn(make_float2(v[2 * i], v[2 * i + 1]), gelu_grad2(make_float2(u[2 * i], u[2 * i + 1])));
-    v[2 * i] = d.x;
-    v[2 * i + 1] = d.y;
-  }
-}
 
 // GELU in its tanh approximation ("AI-infra engineers and the Transformer",
 // section 2.3): GELU(u) = u (1 + tanh(z)) / 2 with z = sqrt(2/pi) (u + 0.044715 u^3),
@@ -271,6 +262,34 @@ __device__ __forceinline__ float2 gelu_tanh_grad2(float2 u) {
   const float2 half_u = __fmul2_rn(u, f2(0.5f));
   return __ffma2_rn(__fmul2_rn(half_u, sech2), dz, __fmul2_rn(__fadd2_rn(t, f2(1.0f)), f2(0.5f)));
 }
+// GELU(u) and GELU'(u) of 8 lanes from one evaluation of phi and Q (erf form)
+// or of tanh (tanh form): g = GELU(u), d = GELU'(u).
+__device__ __forceinline__ void gelu_and_grad8_form(const float (&u)[8], float (&g)[8], float (&d)[8], bool tanh_form) {
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float2 x = make_float2(u[2 * i], u[2 * i + 1]);
+    float2 gv, dv;
+    if (!tanh_form) {
+      float2 phi, q;
+      normal_tail2(x, phi, q);
+      const float2 cdf = normal_cdf2(x, q);
+      gv = __fmul2_rn(x, cdf);
+      dv = __ffma2_rn(x, phi, cdf);
+    } else {
+      constexpr float kS = 0.797884560802865356f;
+      constexpr float kC3 = 3.0f * 0.044715f;
+      const float2 t = tanh_gelu_arg2(x);
+      const float2 half_u = __fmul2_rn(x, f2(0.5f));
+      const float2 onep = __fadd2_rn(t, f2(1.0f));
+      gv = __fmul2_rn(half_u, onep);
+      const float2 sech2 = __ffma2_rn(t, make_float2(-t.x, -t.y), f2(1.0f));
+      const float2 dz = __fmul2_rn(__ffma2_rn(__fmul2_rn(x, x), f2(kC3), f2(1.0f)), f2(kS));
+      dv = __ffma2_rn(__fmul2_rn(half_u, sech2), dz, __fmul2_rn(onep, f2(0.5f)));
+    }
+    g[2 * i] = gv.x; g[2 * i + 1] = gv.y;
+    d[2 * i] = dv.x; d[2 * i + 1] = dv.y;
+  }
+}
 // In-place over 8 lanes, either form.
 __device__ __forceinline__ void gelu8_form(float (&v)[8], bool tanh_form) {
   if (!tanh_form) {
@@ -282,19 +301,6 @@ __device__ __forceinline__ void gelu8_form(float (&v)[8], bool tanh_form) {
     const float2 g = gelu_tanh2(make_float2(v[2 * i], v[2 * i + 1]));
     v[2 * i] = g.x;
     v[2 * i + 1] = g.y;
-  }
-}
-__device__ __forceinline__ void mul_gelu_grad8_form(float (&v)[8], const float (&u)[8], bool tanh_form) {
-  if (!tanh_form) {
-    mul_gelu_grad8(v, u);
-    return;
-  }
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const float2 d =
-        __fmul2_rn(make_float2(v[2 * i], v[2 * i + 1]), gelu_tanh_grad2(make_float2(u[2 * i], u[2 * i + 1])));
-    v[2 * i] = d.x;
-    v[2 * i + 1] = d.y;
   }
 }
 

@@ -13,12 +13,20 @@
 //  EPI_BIAS_GELU      U = acc + bias stored; G = GELU(U as stored) so that a
 //                     backward that recomputes G from U gets identical bits
 //                     (erf form, or the tanh form for KIND | EPI_TANH).
-//  EPI_DGELU          out = acc * GELU'(U).
+//  EPI_DGELU          out = acc * GELU'(U), GELU'(U) rounded to the storage type
+//                     first, as EPI_BIAS_GELU_D stores it (both paths give the
+//                     same bits).
+//  EPI_BIAS_GELU_D    U = acc + bias rounded to storage (not stored);
+//                     out = GELU'(U), out2 = G = GELU(U), both from one
+//                     evaluation of the normal density and tail (or of tanh).
+//                     The backward then needs no special function:
+//  EPI_MUL            out = acc * aux (aux = the stored GELU'(U)).
 //  EPI_STORE          out = acc (+ res).
 //  EPI_F32            float32 out = acc.
 //
-// `aux` carries the 8 residual (EPI_BIAS_DROP_RES, EPI_STORE with res) or U
-// (EPI_DGELU) values of the chunk, loaded by the caller ahead of time.
+// `aux` carries the 8 residual (EPI_BIAS_DROP_RES, EPI_STORE with res), U
+// (EPI_DGELU) or factor (EPI_MUL) values of the chunk, loaded by the caller
+// ahead of time.
 #pragma once
 
 #include "common.cuh"
@@ -27,7 +35,7 @@
 namespace tlp {
 
 // Flag bit on a kernel's compile-time epilogue kind: GELU (EPI_BIAS_GELU,
-// EPI_DGELU) in its tanh form (EpiParams.gelu_tanh at run time).  The low
+// EPI_BIAS_GELU_D, EPI_DGELU) in its tanh form (EpiParams.gelu_tanh at run time).  The low
 // bits are the EpiKind.
 constexpr int EPI_TANH = 16;
 constexpr int epi_base(int kind) { return kind & (EPI_TANH - 1); }
@@ -35,10 +43,27 @@ constexpr int epi_base(int kind) { return kind & (EPI_TANH - 1); }
 // Whether a kind reads a per-element auxiliary input (and which pointer).
 template <int KIND> struct EpiAux {
   static constexpr bool kNeeds =
-      epi_base(KIND) == EPI_BIAS_DROP_RES || epi_base(KIND) == EPI_DGELU || epi_base(KIND) == EPI_STORE;
+      epi_base(KIND) == EPI_BIAS_DROP_RES || epi_base(KIND) == EPI_DGELU || epi_base(KIND) == EPI_STORE ||
+      epi_base(KIND) == EPI_MUL;
 };
 __device__ __forceinline__ const void* epi_aux_ptr(const EpiParams& e, int kind) {
-  return kind == EPI_DGELU ? e.aux : e.res;
+  return kind == EPI_DGELU || kind == EPI_MUL ? e.aux : e.res;
+}
+// Kinds with two stored outputs (out and out2).
+constexpr bool epi_two_outputs(int kind) {
+  return epi_base(kind) == EPI_BIAS_GELU || epi_base(kind) == EPI_BIAS_GELU_D;
+}
+// Kinds whose tensor-core epilogue can also sum the stored output's columns.
+constexpr bool epi_sums_columns(int kind) { return epi_base(kind) == EPI_DGELU || epi_base(kind) == EPI_MUL; }
+
+// v *= GELU'(u) with GELU'(u) rounded to the storage type T (the value
+// EPI_BIAS_GELU_D stores for EPI_MUL), over 8 lanes.
+template <typename T>
+__device__ __forceinline__ void mul_stored_gelu_grad8(float (&v)[8], const float (&u)[8], bool tanh_form) {
+  float g[8], d[8];
+  gelu_and_grad8_form(u, g, d, tanh_form);
+#pragma unroll
+  for (int i = 0; i < 8; ++i) v[i] *= round_f<T>(d[i]);
 }
 
 // Row-dependent part of the EPI_QKV destination, computed once per row.
@@ -94,13 +119,25 @@ __device__ __forceinline__ void epi_apply8(const EpiParams& e, int m, int n, flo
       store8<T>(static_cast<T*>(e.out2) + (size_t)m * e.ldo + n, v);
     }
   } else if constexpr (epi_base(KIND) == EPI_DGELU) {
-    mul_gelu_grad8_form(v, aux, (KIND & EPI_TANH) != 0);
+    mul_stored_gelu_grad8<T>(v, aux, (KIND & EPI_TANH) != 0);
+    store8<T>(static_cast<T*>(e.out) + (size_t)m * e.ldo + n, v);
+  } else if constexpr (epi_base(KIND) == EPI_BIAS_GELU_D) {
+    float b[8], g[8], d[8];
+    load8<T>(static_cast<const T*>(e.bias) + n, b);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) v[i] = round_f<T>(v[i] + b[i]);
+    gelu_and_grad8_form(v, g, d, (KIND & EPI_TANH) != 0);
+    store8<T>(static_cast<T*>(e.out) + (size_t)m * e.ldo + n, d);
+    store8<T>(static_cast<T*>(e.out2) + (size_t)m * e.ldo + n, g);
+  } else if constexpr (epi_base(KIND) == EPI_MUL) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) v[i] *= aux[i];
     store8<T>(static_cast<T*>(e.out) + (size_t)m * e.ldo + n, v);
   }
 }
 
 // Epilogue arithmetic without the store: v becomes the (first) output chunk,
-// v2 the second one (EPI_BIAS_GELU's G).  Used by the tensor-core GEMM, whose
+// v2 the second one (the G of EPI_BIAS_GELU and EPI_BIAS_GELU_D).  Used by the tensor-core GEMM, whose
 // stores go through shared memory and TMA.
 // kbits: the 8 dropout keep bits of this chunk when the caller already has
 // them (EPI_BIAS_DROP_RES), or a value above 0xFF to look them up here.
@@ -137,7 +174,16 @@ __device__ __forceinline__ void epi_compute8(const EpiParams& e, int m, int n, f
     }
     gelu8_form(v2, (KIND & EPI_TANH) != 0);
   } else if constexpr (epi_base(KIND) == EPI_DGELU) {
-    mul_gelu_grad8_form(v, aux, (KIND & EPI_TANH) != 0);
+    mul_stored_gelu_grad8<T>(v, aux, (KIND & EPI_TANH) != 0);
+  } else if constexpr (epi_base(KIND) == EPI_BIAS_GELU_D) {
+    float b[8], u[8];
+    load8<T>(static_cast<const T*>(e.bias) + n, b);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) u[i] = round_f<T>(v[i] + b[i]);
+    gelu_and_grad8_form(u, v2, v, (KIND & EPI_TANH) != 0);
+  } else if constexpr (epi_base(KIND) == EPI_MUL) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) v[i] *= aux[i];
   }
 }
 

@@ -83,6 +83,11 @@ void launch(const GemmDesc& g, const EpiParams& e, cudaStream_t s) {
       if (e.gelu_tanh) gemm_simt_kernel<T, EPI_DGELU | EPI_TANH><<<grid, 256, 0, s>>>(g, e);
       else gemm_simt_kernel<T, EPI_DGELU><<<grid, 256, 0, s>>>(g, e);
       break;
+    case EPI_BIAS_GELU_D:
+      if (e.gelu_tanh) gemm_simt_kernel<T, EPI_BIAS_GELU_D | EPI_TANH><<<grid, 256, 0, s>>>(g, e);
+      else gemm_simt_kernel<T, EPI_BIAS_GELU_D><<<grid, 256, 0, s>>>(g, e);
+      break;
+    case EPI_MUL: gemm_simt_kernel<T, EPI_MUL><<<grid, 256, 0, s>>>(g, e); break;
     case EPI_STORE: gemm_simt_kernel<T, EPI_STORE><<<grid, 256, 0, s>>>(g, e); break;
     case EPI_F32: gemm_simt_kernel<T, EPI_F32><<<grid, 256, 0, s>>>(g, e); break;
   }

@@ -337,7 +337,7 @@ __device__ __forceinline__ bool pair_epilogue_tile(const OutMaps& om, const TcAr
   constexpr int CW = BN / (kPairEpiWarps / 4);              // 64 columns per warp
   constexpr int OUT_ES = epi_base(KIND) == EPI_F32 ? 4 : 2;
   constexpr int SW = 64 / OUT_ES;                          // columns per staging box: 32 (16-bit) or 16 (fp32)
-  constexpr int NOUT = epi_base(KIND) == EPI_BIAS_GELU ? 2 : 1;
+  constexpr int NOUT = epi_two_outputs(KIND) ? 2 : 1;
   const int swz = (lane >> 1) & 3;                         // 64-byte swizzle of this lane's staging row
   int mb, nb, sp;
   decode_tile(g, t, mb, nb, sp);
@@ -412,7 +412,7 @@ __device__ __forceinline__ bool pair_epilogue_tile(const OutMaps& om, const TcAr
         store8<T>(reinterpret_cast<T*>(sb0 + lane * 64 + ((q ^ swz) << 4)), *reinterpret_cast<float(*)[8]>(vq));
         if constexpr (NOUT == 2) store8<T>(reinterpret_cast<T*>(sb1 + lane * 64 + ((q ^ swz) << 4)), v2);
       }
-      if constexpr (epi_base(KIND) == EPI_DGELU && SW == 32) {
+      if constexpr (epi_sums_columns(KIND) && SW == 32) {
         // bias gradient of the FFN1 Linear fused in: column sums of the
         // stored (rounded) values of this warp's 32 rows
         if (e.colsum) {
@@ -798,7 +798,7 @@ bool build_pair_gemm(PairGemm& P, const GemmDesc& gd, const EpiParams& e, int sp
     ok = make_map_t(&om.out, e.out, t16, 2, 64, (uint64_t)3 * om.qkv_heads_rows, 64, 32, 64);
   } else {
     ok = make_map_t(&om.out, e.out, t16, 2, gd.N, gd.M, e.ldo, 32, 64);
-    if (ok && epi_base(KIND) == EPI_BIAS_GELU && e.out2) ok = make_map_t(&om.out2, e.out2, t16, 2, gd.N, gd.M, e.ldo, 32, 64);
+    if (ok && epi_two_outputs(KIND) && e.out2) ok = make_map_t(&om.out2, e.out2, t16, 2, gd.N, gd.M, e.ldo, 32, 64);
   }
   P.e = e;
   return ok;
@@ -811,8 +811,12 @@ bool build_pair_gemm(PairGemm& P, const GemmDesc& gd, const EpiParams& e, int sp
 // Estimated cost of a tile in tenths of a 64-wide K block of main loop:
 // its K blocks, weighted by the epilogue (the dGELU epilogue keeps the
 // epilogue warps busier than the main loop of its K = 1024 tiles, measured
-// ~1.45x per K block), plus a fixed per-tile fill/drain of ~4 K blocks.
-int tile_cost10(int kb, int kind) { return (epi_base(kind) == EPI_DGELU ? 145 : 100) * kb / 10 + 40; }
+// ~1.45x per K block; the multiply-and-column-sum epilogue ~1.1x), plus a
+// fixed per-tile fill/drain of ~4 K blocks.
+int tile_cost10(int kb, int kind) {
+  const int w = epi_base(kind) == EPI_DGELU ? 145 : epi_base(kind) == EPI_MUL ? 110 : 100;
+  return w * kb / 10 + 40;
+}
 
 bool plan_pair_table(PairSched& sch, const TcArgs& g0, int kind0, const TcArgs& g1, int kind1, int pairs) {
   struct Item { int kb, gi, tile; };
@@ -937,16 +941,20 @@ int run_t(const GemmDesc& g, const EpiParams& e, cudaStream_t s) {
                          : launch_tc_pair<T, EPI_BIAS_GELU>(g, e, 1, s);
     case EPI_DGELU:
       return e.gelu_tanh ? launch_tc_pair<T, EPI_DGELU | EPI_TANH>(g, e, 1, s) : launch_tc_pair<T, EPI_DGELU>(g, e, 1, s);
+    case EPI_BIAS_GELU_D:
+      return e.gelu_tanh ? launch_tc_pair<T, EPI_BIAS_GELU_D | EPI_TANH>(g, e, 1, s)
+                         : launch_tc_pair<T, EPI_BIAS_GELU_D>(g, e, 1, s);
+    case EPI_MUL: return launch_tc_pair<T, EPI_MUL>(g, e, 1, s);
     case EPI_STORE: return launch_tc_pair<T, EPI_STORE>(g, e, 1, s);
   }
   return 1;
 }
 
-// A float32 weight gradient (ga) and an input gradient (gb, EPI_DGELU or
-// EPI_STORE) in one launch.
+// A float32 weight gradient (ga) and an input gradient (gb, EPI_DGELU,
+// EPI_MUL or EPI_STORE) in one launch.
 template <typename T>
 int run2_t(const GemmDesc& ga, const EpiParams& ea, const GemmDesc& gb, const EpiParams& eb, cudaStream_t s) {
-  const bool groupable = ea.kind == EPI_F32 && (eb.kind == EPI_DGELU || eb.kind == EPI_STORE) &&
+  const bool groupable = ea.kind == EPI_F32 && (eb.kind == EPI_DGELU || eb.kind == EPI_MUL || eb.kind == EPI_STORE) &&
                          aligned16(ga.A, ga.lda) && aligned16(ga.B, ga.ldb) && aligned16(gb.A, gb.lda) &&
                          aligned16(gb.B, gb.ldb);
   if (!groupable) {
@@ -958,6 +966,7 @@ int run2_t(const GemmDesc& ga, const EpiParams& ea, const GemmDesc& gb, const Ep
   if (splits > 1) ep.out = ga.splitk_ws;
   const int rc =
       eb.kind == EPI_STORE   ? launch_tc_pair_group<T, EPI_F32, EPI_STORE>(ga, ep, splits, gb, eb, s)
+      : eb.kind == EPI_MUL   ? launch_tc_pair_group<T, EPI_F32, EPI_MUL>(ga, ep, splits, gb, eb, s)
       : eb.gelu_tanh         ? launch_tc_pair_group<T, EPI_F32, EPI_DGELU | EPI_TANH>(ga, ep, splits, gb, eb, s)
                              : launch_tc_pair_group<T, EPI_F32, EPI_DGELU>(ga, ep, splits, gb, eb, s);
   if (rc) return rc;
@@ -976,6 +985,10 @@ int run_pair_t(const GemmDesc& g, const EpiParams& e, int splits, cudaStream_t s
                          : launch_tc_pair<T, EPI_BIAS_GELU>(g, e, 1, s);
     case EPI_DGELU:
       return e.gelu_tanh ? launch_tc_pair<T, EPI_DGELU | EPI_TANH>(g, e, 1, s) : launch_tc_pair<T, EPI_DGELU>(g, e, 1, s);
+    case EPI_BIAS_GELU_D:
+      return e.gelu_tanh ? launch_tc_pair<T, EPI_BIAS_GELU_D | EPI_TANH>(g, e, 1, s)
+                         : launch_tc_pair<T, EPI_BIAS_GELU_D>(g, e, 1, s);
+    case EPI_MUL: return launch_tc_pair<T, EPI_MUL>(g, e, 1, s);
     case EPI_STORE: return launch_tc_pair<T, EPI_STORE>(g, e, 1, s);
     case EPI_F32: return launch_tc_pair<T, EPI_F32>(g, e, splits, s);
   }

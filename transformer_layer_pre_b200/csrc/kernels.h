@@ -45,18 +45,20 @@ enum EpiKind {
   EPI_QKV = 0,        // + bias, scattered into Q, K, V laid out (B, heads, S, d)
   EPI_BIAS_DROP_RES,  // out = res + dropout(acc + bias); element index m*N + n
   EPI_BIAS_GELU,      // U = acc + bias (stored), G = GELU(stored U) (stored if out2)
-  EPI_DGELU,          // out = acc * GELU'(U)
+  EPI_DGELU,          // out = acc * GELU'(U) (GELU'(U) rounded to storage first)
   EPI_STORE,          // out = acc (+ res if given)
-  EPI_F32             // float32 out = acc
+  EPI_F32,            // float32 out = acc
+  EPI_BIAS_GELU_D,    // U = acc + bias rounded to storage; out = GELU'(U), out2 = G = GELU(U)
+  EPI_MUL             // out = acc * aux (aux = the GELU'(U) that EPI_BIAS_GELU_D stored)
 };
 
 struct EpiParams {
   int kind;
   const void* bias;   // N entries, storage type
   const void* res;    // residual (M, N) storage type, or null
-  const void* aux;    // EPI_DGELU: U (M, N)
+  const void* aux;    // EPI_DGELU: U (M, N); EPI_MUL: the factor (M, N)
   void* out;          // (M, N) with row stride ldo (EPI_QKV: Q|K|V base)
-  void* out2;         // EPI_BIAS_GELU: G, may be null
+  void* out2;         // EPI_BIAS_GELU: G, may be null; EPI_BIAS_GELU_D: G
   int ldo;
   // dropout (EPI_BIAS_DROP_RES)
   DropoutParams drop;
@@ -64,9 +66,9 @@ struct EpiParams {
   const uint8_t* keep8;   // EPI_BIAS_DROP_RES: precomputed keep bits (byte per 8 elements), or null
   // head split (EPI_QKV)
   int seq, hidden, head_dim, heads, tokens;
-  // EPI_BIAS_GELU / EPI_DGELU: 1 for the tanh approximation of GELU
+  // EPI_BIAS_GELU / EPI_BIAS_GELU_D / EPI_DGELU: 1 for the tanh approximation of GELU
   int gelu_tanh;
-  // EPI_DGELU on the tensor-core GEMM: column sums of the stored output, one
+  // EPI_DGELU / EPI_MUL on the tensor-core GEMM: column sums of the stored output, one
   // partial row per (256-row tile, CTA of the pair, TMEM lane quarter), i.e.
   // row (m / 256) * 8 + ((m % 256) / 128) * 4 + (m % 128) / 32; or null
   float* colsum;

@@ -128,6 +128,9 @@ size_t carve(tl_layer* L, char* base) {
   L->mean2 = (float*)c.take((size_t)L->T * 4);
   L->rstd2 = (float*)c.take((size_t)L->T * 4);
   L->x2 = c.take(TH * es);
+  // u: the FFN1 output U when G is recomputed in backward (checkpoint mode),
+  // else GELU'(U), written by the FFN1 epilogue next to G so that the
+  // backward's dU needs no special function
   L->u = c.take(TF * es);
   L->big = c.take(TF * es);
   L->g = ckpt ? L->big : c.take(TF * es);
@@ -360,7 +363,7 @@ tl_status layer_forward(tl_layer* L, const void* x, const float* mask, const tl_
 
   EpiParams eo = epi(EPI_BIAS_DROP_RES, nullptr, H);
   eo.bias = w->bo; eo.res = x; eo.drop = make_drop(L, L->ph); eo.site = 1;
-  EpiParams e1 = epi(EPI_BIAS_GELU, L->u, F);
+  EpiParams e1 = epi(L->opt.gelu_checkpoint ? EPI_BIAS_GELU : EPI_BIAS_GELU_D, L->u, F);
   e1.bias = w->b1; e1.out2 = L->g; e1.gelu_tanh = L->opt.gelu_tanh ? 1 : 0;
   EpiParams e2 = epi(EPI_BIAS_DROP_RES, nullptr, H);
   e2.bias = w->b2; e2.drop = make_drop(L, L->ph); e2.site = 2;
@@ -473,7 +476,8 @@ tl_status layer_backward(tl_layer* L, const void* x, const void* dy, const tl_we
       ProfScope p_(PC_ROWWISE, s);
       gelu_run(dt, L->u, L->big, (size_t)T * F, L->opt.gelu_tanh ? 1 : 0, s);
     }
-    EpiParams edu = epi(EPI_DGELU, L->big, F);
+    // dU = (dZ2 W2) * GELU'(U): GELU' from U (checkpoint mode) or as stored by the forward
+    EpiParams edu = epi(L->opt.gelu_checkpoint ? EPI_DGELU : EPI_MUL, L->big, F);
     edu.aux = L->u;
     edu.gelu_tanh = L->opt.gelu_tanh ? 1 : 0;
     // the tensor-core GEMM sums dU's columns in its epilogue (db1)
