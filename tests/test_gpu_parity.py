@@ -20,6 +20,8 @@ RAGGED_F16 = Workload("ragged-f16", 3, 72, 192, 3, 520, "f16", 0.1, 0.1, lengths
 RAGGED_POST_BF16 = Workload("ragged-post-bf16", 2, 40, 128, 2, 264, "bf16", 0.1, 0.1, pre_layer_norm=False,
                             lengths=(17, 40))
 RAGGED_F32 = Workload("ragged-f32", 2, 24, 96, 6, 200, "f32", 0.1, 0.2, lengths=(9, 24))
+# S = 96: whole 32-row output boxes, the last query quarter of the 128-row tile empty
+RAGGED96_F16 = Workload("ragged96-f16", 3, 96, 128, 2, 256, "f16", 0.1, 0.1, lengths=(50, 96))
 # sequences spanning two 128-key tiles with a ragged second tile
 MULTITILE_F16 = Workload("multitile-f16", 2, 200, 128, 2, 256, "f16", 0.1, 0.1, lengths=(150, 200))
 MULTITILE_POST_BF16 = Workload("multitile-post-bf16", 2, 264, 192, 3, 384, "bf16", 0.1, 0.1, pre_layer_norm=False,
@@ -46,6 +48,10 @@ def test_ragged_f32_with_dropout_and_mask():
 
 def test_ragged_f16_pre_ln():
     _parity(RAGGED_F16)
+
+
+def test_ragged96_f16_pre_ln():
+    _parity(RAGGED96_F16)
 
 
 def test_ragged_bf16_post_ln():

@@ -58,7 +58,8 @@ struct AttnTc {
   void* dqkv;
   float* colsum;        // fused QKV bias-gradient partials (persistent backward), or null
   int fuse_dq;
-  int ctx_tma;          // persistent forward: ctx rows leave by TMA store (S % 32 == 0)
+  int ctx_tma;          // persistent kernels: ctx (forward) or dQKV (backward) rows leave by TMA store (S % 32 == 0)
+  uint8_t* keep;        // persistent path: attention keep bits [B*nh][128][16] (forward writes, backward reads)
   int bf16;
   int* err;
 };
@@ -786,7 +787,9 @@ __global__ void __launch_bounds__(kPFwdThreads, 1)
           for (int g = 0; g < 4; ++g) v |= dropout_bits8(a.drop, 0, e8 + (uint64_t)(q * 4 + g)) << (8 * g);
           w[q] = v;
         }
-        *reinterpret_cast<uint4*>(sbits + j * kPFwdBits + r * 16) = make_uint4(w[0], w[1], w[2], w[3]);
+        const uint4 kv = make_uint4(w[0], w[1], w[2], w[3]);
+        *reinterpret_cast<uint4*>(sbits + j * kPFwdBits + r * 16) = kv;
+        if (a.keep) *reinterpret_cast<uint4*>(a.keep + ((size_t)it * 128 + r) * 16) = kv;
       }
       const int b = it / a.nh;
       smask[j * 128 + r] = r < S ? (a.mask ? a.mask[(size_t)b * S + r] * kLog2e : 0.0f) : -INFINITY;
@@ -927,7 +930,8 @@ constexpr int kPBwdSmem = 12 * TB + 2 * kPBwdAux + 1024 + 256;   // (Q,K,V,dO) x
 template <typename T>
 __global__ void __launch_bounds__(kPBwdThreads, 1)
     attn_bwd_tc_persist(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
-                        const __grid_constant__ CUtensorMap tv, const __grid_constant__ CUtensorMap tdo, AttnTc a) {
+                        const __grid_constant__ CUtensorMap tv, const __grid_constant__ CUtensorMap tdo,
+                        const __grid_constant__ CUtensorMap tdqkv, AttnTc a) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = align1024(smem_raw);
   uint8_t* sPd = sm + 8 * TB;
@@ -1020,7 +1024,11 @@ __global__ void __launch_bounds__(kPBwdThreads, 1)
       uint8_t* ax = saux + j * kPBwdAux;
       float* smask = reinterpret_cast<float*>(ax + 2048);
       if (!mbar_wait(&aux_free[j], ((n >> 1) & 1) ^ 1, a.err, 69)) break;
-      if (a.drop.thr) {
+      if (a.drop.thr && a.keep) {
+        // the forward's keep bits of this item
+        *reinterpret_cast<uint4*>(ax + r * 16) =
+            __ldg(reinterpret_cast<const uint4*>(a.keep + ((size_t)it * 128 + r) * 16));
+      } else if (a.drop.thr) {
         const uint64_t e8 = (((uint64_t)it * S + (uint64_t)r) * (uint64_t)S) >> 3;
         uint32_t w[4];
 #pragma unroll
@@ -1065,6 +1073,12 @@ __global__ void __launch_bounds__(kPBwdThreads, 1)
     const float c2 = a.scale * kLog2e;
     const float dsc = a.drop.thr ? a.drop.scale : 1.0f;
     const int kc0 = hf * 64;
+    // dQ, dK, dV rows of this warp staged as 32 x 64-byte swizzled boxes in
+    // the warp's own rows of Pd and dS (free between the dV/dK/dQ products
+    // and the next item's Pd, dS)
+    uint8_t* stq = sPd + hf * 16384 + quarter * 4096;
+    uint8_t* stv = sdS + hf * 16384 + quarter * 4096;
+    const int swz = (lane >> 1) & 3;
     int n = 0;
     for (int it = blockIdx.x; it < nitems; it += gridDim.x, ++n) {
       const int j = n & 1;
@@ -1080,6 +1094,11 @@ __global__ void __launch_bounds__(kPBwdThreads, 1)
       const float Di = smask[256 + r];
       if (!mbar_wait_warp(s_full, n & 1, a.err, 67)) break;
       tc_fence_after();
+      if (a.ctx_tma) {
+        // the previous item's dQKV stores have read the staging rows
+        if (lane == 0) bulk_wait_read<0>();
+        __syncwarp();
+      }
 #pragma unroll 1
       for (int c = 0; c < 2; ++c) {
         float sv[32], dv[32];
@@ -1114,42 +1133,55 @@ __global__ void __launch_bounds__(kPBwdThreads, 1)
       mbar_arrive(ds_full);
       if (!mbar_wait_warp(g_full, n & 1, a.err, 68)) break;
       tc_fence_after();
-      float dq[32], dk[32], dv[32];
-      tmem_ld32(tdQ + lo + hf * 32, dq);
-      tmem_ld32(tdK + lo + hf * 32, dk);
-      tmem_ld32(tdV + lo + hf * 32, dv);
-      tc_fence_before();
-      mbar_arrive(g_free);
+      // dQ, dK, dV one after another (w3 = 0, 1, 2): TMEM -> scale -> store
+      // (staged for TMA, or direct) -> fused column sums
+      const bool staged = a.ctx_tma && quarter * 32 < S;
+#pragma unroll 1
+      for (int w3 = 0; w3 < 3; ++w3) {
+        float x[32];
+        tmem_ld32(tdQ - 64 * w3 + lo + hf * 32, x);
+        if (w3 == 2) {
+          tc_fence_before();
+          mbar_arrive(g_free);
+        }
+        if (w3 < 2) {
 #pragma unroll
-      for (int c = 0; c < 32; ++c) {
-        dq[c] *= a.scale;
-        dk[c] *= a.scale;
-      }
-      if (qv) {
-        // row r is query r for dQ and key r for dK, dV (both < S)
-        T* dst = static_cast<T*>(a.dqkv) + trow * 3 * a.H + h * HD + hf * 32;
+          for (int c = 0; c < 32; ++c) x[c] *= a.scale;
+        }
+        if (staged) {
+          uint8_t* st = w3 == 0 ? stq : (w3 == 1 ? stq + 2048 : stv);
 #pragma unroll
-        for (int c = 0; c < 32; c += 8) {
-          store8<T>(dst + c, *reinterpret_cast<float(*)[8]>(dq + c));
-          store8<T>(dst + a.H + c, *reinterpret_cast<float(*)[8]>(dk + c));
-          store8<T>(dst + 2 * a.H + c, *reinterpret_cast<float(*)[8]>(dv + c));
+          for (int c = 0; c < 4; ++c)
+            store8<T>(reinterpret_cast<T*>(st + lane * 64 + ((c ^ swz) << 4)), *reinterpret_cast<float(*)[8]>(x + c * 8));
+        } else if (!a.ctx_tma && qv) {
+          // row r is query r for dQ and key r for dK, dV (both < S)
+          T* dst = static_cast<T*>(a.dqkv) + trow * 3 * a.H + w3 * a.H + h * HD + hf * 32;
+#pragma unroll
+          for (int c = 0; c < 32; c += 8) store8<T>(dst + c, *reinterpret_cast<float(*)[8]>(x + c));
+        }
+        if (a.colsum) {
+          // QKV bias gradient fused in: column sums of the stored values over
+          // this warp's 32 rows (rows past the sequence end count as zero)
+#pragma unroll
+          for (int c = 0; c < 32; ++c) x[c] = qv ? round_f<T>(x[c]) : 0.0f;
+          a.colsum[(size_t)(b * 4 + quarter) * 3 * a.H + w3 * a.H + h * HD + hf * 32 + lane] = warp_colsum32(x);
         }
       }
-      if (a.colsum) {
-        // QKV bias gradient fused in: column sums of the stored values over
-        // this warp's 32 rows (rows past the sequence end count as zero)
-        float* cs = a.colsum + (size_t)(b * 4 + quarter) * 3 * a.H + h * HD + hf * 32 + lane;
-#pragma unroll
-        for (int c = 0; c < 32; ++c) {
-          dq[c] = qv ? round_f<T>(dq[c]) : 0.0f;
-          dk[c] = qv ? round_f<T>(dk[c]) : 0.0f;
-          dv[c] = qv ? round_f<T>(dv[c]) : 0.0f;
+      if (staged) {
+        // three TMA stores per warp of whole 32-row boxes (S % 32 == 0)
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          const int x = h * HD + hf * 32, y = b * S + quarter * 32;
+          tma_store_2d(&tdqkv, stq, x, y);
+          tma_store_2d(&tdqkv, stq + 2048, x + a.H, y);
+          tma_store_2d(&tdqkv, stv, x + 2 * a.H, y);
+          bulk_commit();
         }
-        cs[0] = warp_colsum32(dq);
-        cs[a.H] = warp_colsum32(dk);
-        cs[2 * a.H] = warp_colsum32(dv);
       }
     }
+    if (a.ctx_tma && lane == 0) bulk_wait_all();
+    __syncwarp();
   }
   tc_fence_before();
   __syncthreads();
@@ -1174,17 +1206,19 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-// [rows][cols] row-major 16-bit matrix with row stride ld; box 64 x box_rows.
+// [rows][cols] row-major 16-bit matrix with row stride ld; box 64 x box_rows
+// (128-byte swizzle), or 32 x box_rows (64-byte swizzle) with narrow.
 bool map_tile(CUtensorMap* m, const void* p, bool bf16, uint64_t cols, uint64_t rows, uint64_t ld,
-              uint32_t box_rows = 128) {
+              uint32_t box_rows = 128, bool narrow = false) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return false;
   cuuint64_t dims[2] = {cols, rows};
   cuuint64_t strides[1] = {ld * 2};
-  cuuint32_t box[2] = {64, box_rows};
+  cuuint32_t box[2] = {narrow ? 32u : 64u, box_rows};
   cuuint32_t es[2] = {1, 1};
   return fn(m, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<void*>(p),
-            dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+            narrow ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B,
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
@@ -1209,6 +1243,7 @@ AttnTc make_args(int dt, const AttnArgs& a) {
   t.colsum = a.colsum;
   t.fuse_dq = 0;
   t.ctx_tma = 0;
+  t.keep = a.S <= TILE ? a.keep : nullptr;
   t.bf16 = dt == DT_BF16;
   t.err = attn_error_word();
   return t;
@@ -1264,7 +1299,13 @@ void bwd_t(const AttnArgs& a, cudaStream_t s) {
   if (ntile == 1) {
     int nsm = 148;
     cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, 0);
-    launch_pdl(attn_bwd_tc_persist<T>, std::min(a.B * a.nh, nsm), kPBwdThreads, kPBwdSmem, s, mq, mk, mv, mdo, t);
+    // dQKV (B*S, 3H) in 32 x 32 boxes; a box's rows stay inside one sequence when S % 32 == 0
+    CUtensorMap mdq;
+    t.ctx_tma = a.S % 32 == 0 && map_tile(&mdq, a.dqkv, t.bf16, 3 * (uint64_t)t.H, tokens, 3 * (uint64_t)t.H, 32, true)
+                    ? 1 : 0;
+    if (!t.ctx_tma) mdq = mq;   // unused
+    launch_pdl(attn_bwd_tc_persist<T>, std::min(a.B * a.nh, nsm), kPBwdThreads, kPBwdSmem, s, mq, mk, mv, mdo, mdq,
+               t);
     count_launch();
     return;
   }

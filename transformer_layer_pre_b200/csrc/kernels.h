@@ -169,6 +169,11 @@ struct AttnArgs {
   DropoutParams drop;   // site 0
   void* ctx;            // (B*S, nh*d)
   float* lse;           // (B, nh, S); +inf marks a row with every key masked
+  // attention dropout keep bits of the S <= 128 tensor-core path, laid out
+  // [B*nh][128 query rows][16 bytes] (bit k of byte c = key 8c + k): the
+  // forward writes them, the backward reads them instead of drawing Philox
+  // again; null to draw them in both
+  uint8_t* keep;
   // backward
   const void* dctx;     // (B*S, nh*d)
   float* dvec;          // (B, nh, S) rowsum(dctx * ctx)

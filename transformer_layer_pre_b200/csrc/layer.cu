@@ -62,6 +62,8 @@ struct tl_layer {
   size_t part_floats = 0;
   // hidden-dropout keep bits of sites 1 and 2 (one byte per 8 elements)
   uint8_t *keep1 = nullptr, *keep2 = nullptr;
+  // attention dropout keep bits (site 0), [B*nh][128][16] bytes, or null
+  uint8_t* akeep = nullptr;
   float* splitk = nullptr;
   size_t splitk_floats = 0;
   int gemm_err = 0;
@@ -154,6 +156,7 @@ size_t carve(tl_layer* L, char* base) {
   L->dvec = (float*)c.take((size_t)L->B * L->nh * L->S * 4);
   L->keep1 = (uint8_t*)c.take((size_t)L->T * L->H / 8);
   L->keep2 = (uint8_t*)c.take((size_t)L->T * L->H / 8);
+  L->akeep = L->pa > 0.0f && L->S <= 128 ? (uint8_t*)c.take((size_t)L->B * L->nh * 128 * 16) : nullptr;
   const int np = std::max(std::max(std::max(ln_bwd_parts(L->T), rowdrop_parts(L->T)), colsum_parts(L->T)),
                           std::max((L->T + 255) / 256 * 8, L->B * 4));   // + partial rows of fused column sums
   const int maxc = std::max(3 * L->H, L->F);
@@ -254,6 +257,7 @@ AttnArgs attn_args(tl_layer* L, const float* mask) {
   a.dctx = L->dctx;
   a.dvec = L->dvec;
   a.dqkv = L->dqkv;
+  a.keep = L->akeep;
   return a;
 }
 
