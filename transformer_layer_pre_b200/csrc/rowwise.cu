@@ -193,6 +193,18 @@ __global__ void __launch_bounds__(kFwdWarps * 32) ln_fwd_kernel(const T* __restr
     const int col = (lane + 32 * c) * 8;
     raw[c] = col < H ? raw8_stream<T>(x + (size_t)row * H + col) : raw8_zero<T>();
   }
+  if (keep_out) {
+    // dropout keep bits of this row for a downstream kernel (element index
+    // row*H + col), drawn while the row's loads are in flight
+#pragma unroll
+    for (int c = 0; c < NCH; ++c) {
+      const int col = (lane + 32 * c) * 8;
+      if (col < H) {
+        const uint64_t e8 = ((uint64_t)row * H + col) >> 3;
+        keep_out[e8] = (uint8_t)dropout_bits8(dp, site, e8);
+      }
+    }
+  }
   const float inv_h = 1.0f / (float)H;
   float v[NCH][8];
   float s = 0.0f;
@@ -230,17 +242,6 @@ __global__ void __launch_bounds__(kFwdWarps * 32) ln_fwd_kernel(const T* __restr
   if (lane == 0) {
     mean_out[row] = mean;
     rstd_out[row] = rstd;
-  }
-  if (keep_out) {
-    // dropout keep bits of this row for a downstream kernel (element index row*H + col)
-#pragma unroll
-    for (int c = 0; c < NCH; ++c) {
-      const int col = (lane + 32 * c) * 8;
-      if (col < H) {
-        const uint64_t e8 = ((uint64_t)row * H + col) >> 3;
-        keep_out[e8] = (uint8_t)dropout_bits8(dp, site, e8);
-      }
-    }
   }
 }
 
@@ -419,6 +420,15 @@ __global__ void __launch_bounds__(kLnbPairs * 64, (sizeof(T) == 4 || (INV && DRO
         rr[c] = col < H ? raw8_stream<T>(rp + (size_t)row * H + col) : raw8_zero<T>();
       }
     }
+    // keep bits of the dropout copy, loaded with the residual (consumed after the row sums)
+    uint32_t kb[DROP ? NC : 1];
+    if constexpr (DROP) {
+#pragma unroll
+      for (int c = 0; c < NC; ++c) {
+        const int col = (L + 64 * c) * 8;
+        kb[c] = a.keep8 && col < H ? (uint32_t)__ldg(a.keep8 + (((size_t)row * H + col) >> 3)) : 0xFFu;
+      }
+    }
     float s1 = 0.0f, s2 = 0.0f;
 #pragma unroll
     for (int c = 0; c < NC; ++c) {
@@ -468,8 +478,7 @@ __global__ void __launch_bounds__(kLnbPairs * 64, (sizeof(T) == 4 || (INV && DRO
       }
       store8<T>(static_cast<T*>(a.dx) + off, o);
       if constexpr (DROP) {
-        const uint32_t bits = a.keep8 ? (uint32_t)a.keep8[off >> 3]
-                                      : (a.drop.thr ? dropout_bits8(a.drop, a.site, off >> 3) : 0xFFu);
+        const uint32_t bits = a.keep8 ? kb[c] : (a.drop.thr ? dropout_bits8(a.drop, a.site, off >> 3) : 0xFFu);
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
           o[i] = round_f<T>(((bits >> i) & 1u) ? round_f<T>(o[i]) * sc : 0.0f);
@@ -706,7 +715,10 @@ __global__ void dropout_mask_kernel(DropoutParams dp, int site, uint64_t e0, uin
   }
 }
 
-int row_blocks(int rows) { return std::max(1, std::min(kMaxBlocks, (rows + 31) / 32)); }
+// Blocks of the row kernels that keep per-block column sums: at least 16 rows
+// a block, at most two blocks per SM, so a large batch fills every SM evenly
+// (8192 rows: 296 blocks of <= 28 rows, not 256 blocks of 32 on 148 SMs).
+int row_blocks(int rows) { return std::max(1, std::min(kMaxBlocks, (rows + 15) / 16)); }
 
 #define TLP_KR_SWITCH(H, ES, ...)                             \
   switch (group_rows(H, ES)) {                                \
