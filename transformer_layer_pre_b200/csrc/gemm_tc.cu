@@ -910,6 +910,12 @@ void f32_split_reduce(const GemmDesc& g, const EpiParams& e, int splits, cudaStr
   const int kb_per = (kblocks + splits - 1) / splits;
   const int real = (kblocks + kb_per - 1) / kb_per;
   const size_t n4 = (size_t)g.M * g.N / 4;
+  const size_t n = (size_t)g.M * g.N;
+  if (g.defer && g.defer->n < kMaxFinalizeJobs && n % 4 == 0 && n < (1ull << 31) &&
+      (reinterpret_cast<uintptr_t>(e.out) & 15) == 0) {
+    g.defer->job[g.defer->n++] = {g.splitk_ws, static_cast<float*>(e.out), real, (int)n, rows_pad * g.N};
+    return;
+  }
   launch_pdl(splitk_reduce_kernel, (int)std::min<size_t>((n4 + 255) / 256, 148 * 8), 256, 0, s,
              static_cast<const float*>(g.splitk_ws), real, rows_pad * g.N, n4, static_cast<float*>(e.out));
   count_launch();

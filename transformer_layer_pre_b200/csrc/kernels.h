@@ -33,12 +33,18 @@ inline size_t dtype_size(int dt) { return dt == DT_F32 ? 4 : 2; }
 // ------------------------------------------------------------------ GEMM
 // C[m, n] = sum_k A(m, k) * B(n, k), float32 accumulation, then an epilogue.
 // A(m, k) = A[m*lda + k] when a_kmajor, else A[k*lda + m]; B likewise.
+struct FinalizeList;
+
 struct GemmDesc {
   int M, N, K;
   const void* A; int lda; bool a_kmajor;
   const void* B; int ldb; bool b_kmajor;
   float* splitk_ws;          // float32 scratch for split-K weight gradients, or null
   size_t splitk_ws_floats;
+  // when set (and it has room), a split-K float32 GEMM appends the sum of its
+  // partials to this list (summed by a later colsum_finalize_list_run; the
+  // scratch must stay untouched until then) instead of launching the sum
+  FinalizeList* defer = nullptr;
 };
 
 enum EpiKind {
@@ -136,15 +142,23 @@ int colsum_parts(int rows);
 void colsum_run(int dtype, const void* X, int rows, int cols, float* part, cudaStream_t s);
 // out[c] = sum_p part[p*cols + c] (fixed order).
 void colsum_finalize_run(const float* part, int nparts, int cols, float* out, cudaStream_t s);
-// Several finalizes in one launch: out[c] = sum over p < nparts of part[p * cols + c] per job.
-constexpr int kMaxFinalize = 8;
+// Several finalizes in one launch, each job either
+//   stride == 0: out[c] = sum over p < nparts of part[p * cols + c] (column
+//                sums of partial rows), or
+//   stride != 0: out[i] = sum over p < nparts of part[p * stride + i] for
+//                i < cols (the split-K partials of a float32 weight gradient;
+//                cols a multiple of 4, 16-byte aligned pointers),
+// always summed in increasing p.
+constexpr int kMaxFinalize = 8;        // partial-row slots a layer keeps
+constexpr int kMaxFinalizeJobs = 12;   // + the split-K weight gradients
 struct FinalizeJob {
   const float* part;
   float* out;
   int nparts, cols;
+  size_t stride;
 };
 struct FinalizeList {
-  FinalizeJob job[kMaxFinalize];
+  FinalizeJob job[kMaxFinalizeJobs];
   int n;
 };
 void colsum_finalize_list_run(const FinalizeList& fl, cudaStream_t s);

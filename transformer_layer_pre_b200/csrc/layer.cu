@@ -64,8 +64,10 @@ struct tl_layer {
   uint8_t *keep1 = nullptr, *keep2 = nullptr;
   // attention dropout keep bits (site 0), [B*nh][128][16] bytes, or null
   uint8_t* akeep = nullptr;
-  float* splitk = nullptr;
-  size_t splitk_floats = 0;
+  // split-K scratch of the four weight gradients (W2, W1, Wo, Wqkv), each its
+  // own, so every split sum can wait for the closing finalize launch
+  float* splitk[4] = {nullptr, nullptr, nullptr, nullptr};
+  size_t splitk_floats[4] = {0, 0, 0, 0};
   int gemm_err = 0;
 };
 
@@ -163,9 +165,12 @@ size_t carve(tl_layer* L, char* base) {
   L->part_floats = (size_t)np * maxc;
   L->part = (float*)c.take((size_t)kMaxFinalize * L->part_floats * 4);   // one slot per parameter column sum
   const int dt = L->opt.dtype, T = L->T, H = L->H, F = L->F;
-  L->splitk_floats = std::max(std::max(gemm_splitk_ws_floats(dt, H, F, T), gemm_splitk_ws_floats(dt, F, H, T)),
-                              std::max(gemm_splitk_ws_floats(dt, H, H, T), gemm_splitk_ws_floats(dt, 3 * H, H, T)));
-  L->splitk = L->splitk_floats ? (float*)c.take(L->splitk_floats * 4) : nullptr;
+  const size_t wsf[4] = {gemm_splitk_ws_floats(dt, H, F, T), gemm_splitk_ws_floats(dt, F, H, T),
+                         gemm_splitk_ws_floats(dt, H, H, T), gemm_splitk_ws_floats(dt, 3 * H, H, T)};
+  for (int i = 0; i < 4; ++i) {
+    L->splitk_floats[i] = wsf[i];
+    L->splitk[i] = wsf[i] ? (float*)c.take(wsf[i] * 4) : nullptr;
+  }
   return c.off;
 }
 
@@ -190,7 +195,16 @@ tl_status ensure_buffers(tl_layer* L) {
 }
 
 GemmDesc gdesc(tl_layer* L, int M, int N, int K, const void* A, int lda, bool ak, const void* B, int ldb, bool bk) {
-  return GemmDesc{M, N, K, A, lda, ak, B, ldb, bk, L->splitk, L->splitk_floats};
+  return GemmDesc{M, N, K, A, lda, ak, B, ldb, bk, nullptr, 0};
+}
+
+// A weight-gradient GEMM (float32 out) with split-K scratch `which` (0 W2,
+// 1 W1, 2 Wo, 3 Wqkv) whose split sum joins the closing finalize list.
+GemmDesc wdesc(tl_layer* L, int which, FinalizeList* fin, int M, int N, int K, const void* A, int lda, const void* B,
+               int ldb) {
+  GemmDesc g{M, N, K, A, lda, false, B, ldb, false, L->splitk[which], L->splitk_floats[which]};
+  g.defer = fin;
+  return g;
 }
 
 void gemm(tl_layer* L, int M, int N, int K, const void* A, int lda, bool ak, const void* B, int ldb, bool bk,
@@ -487,7 +501,7 @@ tl_status layer_backward(tl_layer* L, const void* x, const void* dy, const tl_we
     // the tensor-core GEMM sums dU's columns in its epilogue (db1)
     const bool fused_db1 = gemm_uses_tensor_cores(dt) != 0;
     if (fused_db1) edu.colsum = slot(db1_slot);
-    const GemmDesc gw2 = gdesc(L, H, F, T, L->dz2, H, false, L->g, F, false);   // dW2 = dZ2^T G
+    const GemmDesc gw2 = wdesc(L, 0, &fin, H, F, T, L->dz2, H, L->g, F);          // dW2 = dZ2^T G
     const GemmDesc gdu = gdesc(L, T, F, H, L->dz2, H, true, w->w2, F, false);   // dU = (dZ2 W2) GELU'(U)
     if (L->g != L->big) {
       gemm2(L, gw2, ew2, gdu, edu, s);
@@ -499,7 +513,7 @@ tl_status layer_backward(tl_layer* L, const void* x, const void* dy, const tl_we
     if (fused_db1) fin.job[fin.n++] = {slot(db1_slot), g->b1, (T + 255) / 256 * 8, F};   // db1 from the GEMM
     else bias_grad(L, L->big, F, db1_slot, g->b1, fin, s);                                  // db1
     EpiParams ew1 = epi(EPI_F32, g->w1, H);
-    gemm2(L, gdesc(L, F, H, T, L->big, F, false, ffn_in, H, false), ew1,   // dW1 = dU^T in
+    gemm2(L, wdesc(L, 1, &fin, F, H, T, L->big, F, ffn_in, H), ew1,          // dW1 = dU^T in
           gdesc(L, T, H, F, L->big, F, true, w->w1, H, false), edin, s);   // dU W1
   };
   // attention block from dA: dWo with dctx, attention backward, dbqkv, then
@@ -507,7 +521,7 @@ tl_status layer_backward(tl_layer* L, const void* x, const void* dy, const tl_we
   auto attn_bwd_block = [&](const void* attn_in, const EpiParams& edin, int dbqkv_slot) {
     EpiParams ewo = epi(EPI_F32, g->wo, H);
     EpiParams edc = epi(EPI_STORE, L->dctx, H);
-    gemm2(L, gdesc(L, H, H, T, L->da, H, false, L->ctx, H, false), ewo,    // dWo = dA^T ctx
+    gemm2(L, wdesc(L, 2, &fin, H, H, T, L->da, H, L->ctx, H), ewo,           // dWo = dA^T ctx
           gdesc(L, T, H, H, L->da, H, true, w->wo, H, false), edc, s);     // dctx = dA Wo
     AttnArgs aa = attn_args(L, L->mask);
     const bool fused_dbqkv = attn_tc_supports(dt, aa) && attn_tc_fuses_colsum(dt, aa);
@@ -516,7 +530,7 @@ tl_status layer_backward(tl_layer* L, const void* x, const void* dy, const tl_we
     if (fused_dbqkv) fin.job[fin.n++] = {slot(dbqkv_slot), g->bqkv, L->B * 4, 3 * H};   // from the attention
     else bias_grad(L, L->dqkv, 3 * H, dbqkv_slot, g->bqkv, fin, s);
     EpiParams ewq = epi(EPI_F32, g->wqkv, H);
-    gemm2(L, gdesc(L, 3 * H, H, T, L->dqkv, 3 * H, false, attn_in, H, false), ewq,   // dWqkv = dQKV^T in
+    gemm2(L, wdesc(L, 3, &fin, 3 * H, H, T, L->dqkv, 3 * H, attn_in, H), ewq,           // dWqkv = dQKV^T in
           gdesc(L, T, H, 3 * H, L->dqkv, 3 * H, true, w->wqkv, H, false), edin, s);  // dQKV Wqkv
   };
 

@@ -663,14 +663,70 @@ __global__ void __launch_bounds__(256) colsum_kernel(const T* __restrict__ X, in
   }
 }
 
-// out[c] = sum over p of part[p][c]: 32 columns x 32 part-lanes per block,
-// each lane sums every 32nd partial row, then a fixed-order sum over lanes.
-// blockIdx.y selects one of up to three (partials, output) pairs.
-// Column sums of partial rows, for up to kMaxFinalize (partials, output)
-// jobs in one launch: blockIdx.y picks the job, 32 x 32 threads sum 32
-// columns of it (partial rows strided over the 32 warps, then the 32 warp
-// sums in warp order: a fixed order).
-__global__ void __launch_bounds__(1024) colsum_finalize_kernel(FinalizeList fl) {
+// The closing sums of a backward pass, in one launch.  Blocks are numbered
+// over all jobs (first[j] = the first block of job j).  A column-sum job
+// gives each block 64 columns: 16 column groups of 4 (float4 loads) x 16
+// part lanes, lane l summing partial rows l, l+16, ..., then the 16 lane sums
+// in lane order (a fixed order).  A split-K job sums its partial matrices
+// element-wise, four floats a thread, partials in increasing order.
+constexpr int kFinCols = 64;
+constexpr int kFinThreads = 256;
+
+struct FinalizeGrid {
+  FinalizeList fl;
+  int first[kMaxFinalizeJobs + 1];
+};
+
+__global__ void __launch_bounds__(kFinThreads) colsum_finalize_kernel(const __grid_constant__ FinalizeGrid fg) {
+  pdl_wait();
+  pdl_launch_dependents();
+  __shared__ float4 red[16][17];
+  int j = 0;
+  while (j + 1 < fg.fl.n && (int)blockIdx.x >= fg.first[j + 1]) ++j;
+  const FinalizeJob& job = fg.fl.job[j];
+  const int b = (int)blockIdx.x - fg.first[j];
+  const int cols = job.cols, nparts = job.nparts;
+  if (job.stride) {
+    const float4* p = reinterpret_cast<const float4*>(job.part);
+    const size_t n4 = (size_t)cols / 4, st4 = job.stride / 4;
+    const size_t step = (size_t)(fg.first[j + 1] - fg.first[j]) * kFinThreads;
+    for (size_t i = (size_t)b * kFinThreads + threadIdx.x; i < n4; i += step) {
+      float4 sum = p[i];
+      for (int k = 1; k < nparts; ++k) {
+        const float4 v = p[k * st4 + i];
+        sum.x += v.x; sum.y += v.y; sum.z += v.z; sum.w += v.w;
+      }
+      reinterpret_cast<float4*>(job.out)[i] = sum;
+    }
+    return;
+  }
+  const int cg = threadIdx.x & 15, pl = threadIdx.x >> 4;
+  const int c = b * kFinCols + cg * 4;
+  float4 s = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+  if (c < cols) {
+    const float* __restrict__ part = job.part + c;
+#pragma unroll 4
+    for (int p = pl; p < nparts; p += 16) {
+      const float4 v = *reinterpret_cast<const float4*>(part + (size_t)p * cols);
+      s.x += v.x; s.y += v.y; s.z += v.z; s.w += v.w;
+    }
+  }
+  red[pl][cg] = s;
+  __syncthreads();
+  if (pl == 0 && c < cols) {
+    float4 t = red[0][cg];
+#pragma unroll
+    for (int w = 1; w < 16; ++w) {
+      const float4 v = red[w][cg];
+      t.x += v.x; t.y += v.y; t.z += v.z; t.w += v.w;
+    }
+    *reinterpret_cast<float4*>(job.out + c) = t;
+  }
+}
+
+// Scalar column sums for column counts that are not a multiple of 4: 32
+// columns x 32 part lanes per block, blockIdx.y the job.
+__global__ void __launch_bounds__(1024) colsum_finalize_scalar_kernel(FinalizeList fl) {
   pdl_wait();
   pdl_launch_dependents();
   __shared__ float red[32][33];
@@ -869,9 +925,46 @@ void colsum_run(int dt, const void* X, int rows, int cols, float* part, cudaStre
 
 void colsum_finalize_list_run(const FinalizeList& fl, cudaStream_t s) {
   if (fl.n <= 0) return;
-  int maxc = 0;
-  for (int i = 0; i < fl.n; ++i) maxc = std::max(maxc, fl.job[i].cols);
-  launch_pdl(colsum_finalize_kernel, dim3((maxc + 31) / 32, fl.n), 1024, 0, s, fl);
+  bool vec = true;
+  for (int i = 0; i < fl.n; ++i) {
+    const FinalizeJob& j = fl.job[i];
+    if (!j.stride && (j.cols % 4 != 0 || (reinterpret_cast<uintptr_t>(j.part) & 15) != 0 ||
+                      (reinterpret_cast<uintptr_t>(j.out) & 15) != 0))
+      vec = false;
+  }
+  if (!vec) {
+    // scalar column sums; split-K jobs (always 4-aligned) then go one by one
+    FinalizeList cs = fl;
+    cs.n = 0;
+    int maxc = 0;
+    for (int i = 0; i < fl.n; ++i)
+      if (!fl.job[i].stride) {
+        cs.job[cs.n++] = fl.job[i];
+        maxc = std::max(maxc, fl.job[i].cols);
+      }
+    if (cs.n) {
+      launch_pdl(colsum_finalize_scalar_kernel, dim3((maxc + 31) / 32, cs.n), 1024, 0, s, cs);
+      count_launch();
+    }
+    for (int i = 0; i < fl.n; ++i)
+      if (fl.job[i].stride) {
+        FinalizeList one;
+        one.n = 1;
+        one.job[0] = fl.job[i];
+        colsum_finalize_list_run(one, s);
+      }
+    return;
+  }
+  FinalizeGrid fg;
+  fg.fl = fl;
+  fg.first[0] = 0;
+  for (int i = 0; i < fl.n; ++i) {
+    const FinalizeJob& j = fl.job[i];
+    const int nb = j.stride ? (int)std::min<size_t>(((size_t)j.cols / 4 + kFinThreads - 1) / kFinThreads, 296)
+                            : (j.cols + kFinCols - 1) / kFinCols;
+    fg.first[i + 1] = fg.first[i] + std::max(nb, 1);
+  }
+  launch_pdl(colsum_finalize_kernel, fg.first[fl.n], kFinThreads, 0, s, fg);
   count_launch();
 }
 
