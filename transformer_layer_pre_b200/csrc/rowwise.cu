@@ -390,6 +390,7 @@ __global__ void __launch_bounds__(kLnbPairs * 64, (sizeof(T) == 4 || (INV && DRO
   int r0, r1;
   row_range(a.rows, r0, r1);
   Raw8<T> rdy[NC], rx[NC];
+  float rs_n = 0.0f, mean_n = 0.0f;   // the fetched row's rstd and mean
   auto fetch = [&](int row) {
 #pragma unroll
     for (int c = 0; c < NC; ++c) {
@@ -398,6 +399,10 @@ __global__ void __launch_bounds__(kLnbPairs * 64, (sizeof(T) == 4 || (INV && DRO
       const size_t off = (size_t)row * H + col;
       rdy[c] = in ? raw8_stream<T>(dyp + off) : raw8_zero<T>();
       rx[c] = in ? raw8_stream<T>(xp + off) : raw8_zero<T>();
+    }
+    if (row < r1) {
+      rs_n = __ldg(a.rstd + row);
+      if constexpr (!INV) mean_n = __ldg(a.mean + row);
     }
   };
   int row = r0 + pair;
@@ -409,8 +414,8 @@ __global__ void __launch_bounds__(kLnbPairs * 64, (sizeof(T) == 4 || (INV && DRO
       raw8_unpack<T>(rdy[c], dy[c]);
       raw8_unpack<T>(rx[c], xh[c]);
     }
-    const float rs = a.rstd[row];
-    const float mean = INV ? 0.0f : a.mean[row];
+    const float rs = rs_n;
+    const float mean = INV ? 0.0f : mean_n;
     fetch(row + kLnbPairs);
     Raw8<T> rr[RES ? NC : 1];
     if constexpr (RES) {
