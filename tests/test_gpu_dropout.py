@@ -33,15 +33,19 @@ def _zero_weights(h, f, dtype, dev):
                 ln2_b=z(h))
 
 
-@pytest.mark.parametrize("dtype", [torch.float16, torch.bfloat16, torch.float32])
-def test_hidden_site_masks_through_layer(dtype):
+@pytest.mark.parametrize("dtype,B,S,H,heads,F", [
+    (torch.float16, 2, 64, 256, 4, 512), (torch.bfloat16, 2, 64, 256, 4, 512), (torch.float32, 2, 64, 256, 4, 512),
+    # BERT-Large shape: the QKV and out-projection GEMMs have CTA pairs without
+    # a tile in their last round, which draw the keep bits of sites 1 and 2
+    (torch.float16, 64, 128, 1024, 16, 1024)])
+def test_hidden_site_masks_through_layer(dtype, B, S, H, heads, F):
     # x = 0, Wqkv = Wo = W2 = 0, bo = 1, b2 = 2: y = keep1 * 1/(1-p) + keep2 * 2/(1-p)
-    B, S, H, F, p, seed, off = 2, 64, 256, 512, 0.1, 4321, 3
+    p, seed, off = 0.1, 4321, 3
     dev = torch.device("cuda", 0)
     w = _zero_weights(H, F, dtype, dev)
     w["bo"].fill_(1.0)
     w["b2"].fill_(2.0)
-    L = Layer(B, S, H, 4, F, 0.0, p, True, seed, dtype=dtype, philox_offset=off)
+    L = Layer(B, S, H, heads, F, 0.0, p, True, seed, dtype=dtype, philox_offset=off)
     try:
         x = torch.zeros(B, S, H, dtype=dtype, device=dev)
         y = L.forward(x, None, w).double().cpu().numpy().reshape(-1)

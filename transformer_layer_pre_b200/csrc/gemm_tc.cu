@@ -641,6 +641,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
       acc ^= 1;
       if (acc == 0) aph ^= 1u;
     }
+    if constexpr (KA == KB) {
+      if (e0.gen_keep) {
+        // pairs without a tile in the last round draw dropout keep bits
+        // while the other pairs finish it (consecutive lanes, consecutive bytes)
+        const int total = g0.tiles_m * g0.tiles_n * g0.splits;
+        const int rem = total % ncl;
+        if (rem != 0 && cid >= rem) {
+          const uint64_t nthr = (uint64_t)(ncl - rem) * 2 * 32 * kPairEpiWarps;
+          for (uint64_t u = ((uint64_t)((cid - rem) * 2 + (int)rank) * kPairEpiWarps + (warp - 2)) * 32 + lane;
+               u < e0.gen_n8; u += nthr)
+            e0.gen_keep[u] = (uint8_t)dropout_bits8(e0.gen_drop, e0.gen_site, u);
+        }
+      }
+    }
     if (lane == 0) bulk_wait_all();
     __syncwarp();
   }
@@ -1002,6 +1016,16 @@ int run_pair_t(const GemmDesc& g, const EpiParams& e, int splits, cudaStream_t s
 }
 
 }  // namespace
+
+int gemm_tc_bubble_pairs(int dtype, int M, int N, const EpiParams& e) {
+  if (dtype == DT_F32) return 0;
+  if (e.kind == EPI_QKV && !(e.head_dim == 64 && e.seq % 32 == 0 && e.hidden % 64 == 0)) return 0;
+  if (e.kind != EPI_QKV && e.kind != EPI_BIAS_DROP_RES) return 0;
+  const int total = ((M + 255) / 256) * ((N + 255) / 256);   // launch_tc_pair's round-robin grid
+  const int ncl = std::min(total, num_sms() / 2);
+  const int rem = total % ncl;
+  return rem ? ncl - rem : 0;
+}
 
 // The CTA-pair GEMM directly (splits > 1 only for EPI_F32, writing split
 // partials to e.out as laid out for splitk_reduce).

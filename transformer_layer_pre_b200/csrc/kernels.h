@@ -74,11 +74,24 @@ struct EpiParams {
   int seq, hidden, head_dim, heads, tokens;
   // EPI_BIAS_GELU / EPI_BIAS_GELU_D / EPI_DGELU: 1 for the tanh approximation of GELU
   int gelu_tanh;
+  // EPI_QKV / EPI_BIAS_DROP_RES on the tensor-core pair kernel: the CTA
+  // pairs left without a tile in the last round (gemm_tc_bubble_pairs) draw
+  // the keep bits of dropout site gen_site with gen_drop (gen_n8 bytes, one
+  // per 8 elements) into gen_keep meanwhile; or null
+  uint8_t* gen_keep;
+  int gen_site;
+  uint64_t gen_n8;
+  DropoutParams gen_drop;
   // EPI_DGELU / EPI_MUL on the tensor-core GEMM: column sums of the stored output, one
   // partial row per (256-row tile, CTA of the pair, TMEM lane quarter), i.e.
   // row (m / 256) * 8 + ((m % 256) / 128) * 4 + (m % 128) / 32; or null
   float* colsum;
 };
+
+// CTA pairs of the tensor-core pair kernel that have no tile in its last
+// round for an M x N GEMM with this epilogue (0 when it runs elsewhere or the
+// last round is full): the pairs that honour EpiParams.gen_keep.
+int gemm_tc_bubble_pairs(int dtype, int M, int N, const EpiParams& e);
 
 // Returns 0, or non-zero when an operand cannot be described to the TMA unit
 // (unaligned base address or row stride).

@@ -386,15 +386,25 @@ tl_status layer_forward(tl_layer* L, const void* x, const float* mask, const tl_
   EpiParams e2 = epi(EPI_BIAS_DROP_RES, nullptr, H);
   e2.bias = w->b2; e2.drop = make_drop(L, L->ph); e2.site = 2;
 
-  // hidden-dropout keep bits come from the LayerNorm forward kernels that
-  // run before their consumers (pre-LN: LN1 for site 1, LN2 for site 2;
-  // post-LN: LN1 for site 2); the consumers read them instead of drawing Philox
+  // hidden-dropout keep bits are drawn once, ahead of their consumers, which
+  // read them instead of drawing Philox: site 1 by the QKV GEMM's pairs that
+  // sit out its last round, site 2 likewise by the out-projection GEMM's;
+  // where a GEMM has no such pairs, by the LayerNorm forward before the
+  // consumer (pre-LN: LN1 for site 1, LN2 for site 2; post-LN: LN1 for site 2)
   const bool keepbits = eo.drop.thr != 0;
+  const bool k1_gemm = keepbits && gemm_tc_bubble_pairs(dt, T, 3 * H, eq) >= 8;
+  const bool k2_gemm = keepbits && gemm_tc_bubble_pairs(dt, T, H, eo) >= 8;
+  if (k1_gemm) {
+    eq.gen_keep = L->keep1; eq.gen_site = 1; eq.gen_n8 = (uint64_t)T * H / 8; eq.gen_drop = eo.drop;
+  }
+  if (k2_gemm) {
+    eo.gen_keep = L->keep2; eo.gen_site = 2; eo.gen_n8 = (uint64_t)T * H / 8; eo.gen_drop = e2.drop;
+  }
   if (L->pre_ln) {
     {
       ProfScope p_(PC_LN_FWD, s);
       ln_fwd_run(dt, x, w->ln1_g, w->ln1_b, L->h1, L->mean1, L->rstd1, T, H, L->opt.ln_eps, s,
-                 keepbits ? L->keep1 : nullptr, &eo.drop, 1);
+                 keepbits && !k1_gemm ? L->keep1 : nullptr, &eo.drop, 1);
     }
     if (keepbits) eo.keep8 = L->keep1;
     gemm(L, T, 3 * H, H, L->h1, H, true, w->wqkv, H, true, eq, s);
@@ -404,7 +414,7 @@ tl_status layer_forward(tl_layer* L, const void* x, const float* mask, const tl_
     {
       ProfScope p_(PC_LN_FWD, s);
       ln_fwd_run(dt, L->x2, w->ln2_g, w->ln2_b, L->h2, L->mean2, L->rstd2, T, H, L->opt.ln_eps, s,
-                 keepbits ? L->keep2 : nullptr, &e2.drop, 2);
+                 keepbits && !k2_gemm ? L->keep2 : nullptr, &e2.drop, 2);
     }
     if (keepbits) e2.keep8 = L->keep2;
     gemm(L, T, F, H, L->h2, H, true, w->w1, H, true, e1, s);
@@ -416,12 +426,13 @@ tl_status layer_forward(tl_layer* L, const void* x, const float* mask, const tl_
     void* r2 = L->res2 ? L->res2 : L->dres;
     gemm(L, T, 3 * H, H, x, H, true, w->wqkv, H, true, eq, s);
     attn_fwd(L, aa, s);
+    if (k1_gemm) eo.keep8 = L->keep1;
     eo.out = r1;
     gemm(L, T, H, H, L->ctx, H, true, w->wo, H, true, eo, s);
     {
       ProfScope p_(PC_LN_FWD, s);
       ln_fwd_run(dt, r1, w->ln1_g, w->ln1_b, L->x2, L->mean1, L->rstd1, T, H, L->opt.ln_eps, s,
-                 keepbits ? L->keep2 : nullptr, &e2.drop, 2);
+                 keepbits && !k2_gemm ? L->keep2 : nullptr, &e2.drop, 2);
     }
     if (keepbits) e2.keep8 = L->keep2;
     gemm(L, T, F, H, L->x2, H, true, w->w1, H, true, e1, s);
