@@ -35,8 +35,8 @@ def _zero_weights(h, f, dtype, dev):
 
 @pytest.mark.parametrize("dtype,B,S,H,heads,F", [
     (torch.float16, 2, 64, 256, 4, 512), (torch.bfloat16, 2, 64, 256, 4, 512), (torch.float32, 2, 64, 256, 4, 512),
-    # BERT-Large shape: the QKV and out-projection GEMMs have CTA pairs without
-    # a tile in their last round, which draw the keep bits of sites 1 and 2
+    # BERT-Large shape: the QKV GEMM has CTA pairs without a tile in its last
+    # round, which draw the keep bits of sites 1 and 2
     (torch.float16, 64, 128, 1024, 16, 1024)])
 def test_hidden_site_masks_through_layer(dtype, B, S, H, heads, F):
     # x = 0, Wqkv = Wo = W2 = 0, bo = 1, b2 = 2: y = keep1 * 1/(1-p) + keep2 * 2/(1-p)

@@ -649,9 +649,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
         const int rem = total % ncl;
         if (rem != 0 && cid >= rem) {
           const uint64_t nthr = (uint64_t)(ncl - rem) * 2 * 32 * kPairEpiWarps;
+          const uint64_t n = e0.gen_keep2 ? 2 * e0.gen_n8 : e0.gen_n8;
           for (uint64_t u = ((uint64_t)((cid - rem) * 2 + (int)rank) * kPairEpiWarps + (warp - 2)) * 32 + lane;
-               u < e0.gen_n8; u += nthr)
-            e0.gen_keep[u] = (uint8_t)dropout_bits8(e0.gen_drop, e0.gen_site, u);
+               u < n; u += nthr) {
+            const bool second = u >= e0.gen_n8;
+            const uint64_t e8 = second ? u - e0.gen_n8 : u;
+            (second ? e0.gen_keep2 : e0.gen_keep)[e8] =
+                (uint8_t)dropout_bits8(e0.gen_drop, e0.gen_site + (second ? 1 : 0), e8);
+          }
         }
       }
     }

@@ -77,8 +77,10 @@ struct EpiParams {
   // EPI_QKV / EPI_BIAS_DROP_RES on the tensor-core pair kernel: the CTA
   // pairs left without a tile in the last round (gemm_tc_bubble_pairs) draw
   // the keep bits of dropout site gen_site with gen_drop (gen_n8 bytes, one
-  // per 8 elements) into gen_keep meanwhile; or null
+  // per 8 elements) into gen_keep meanwhile, and those of site gen_site + 1
+  // into gen_keep2 when it is set; or null
   uint8_t* gen_keep;
+  uint8_t* gen_keep2;
   int gen_site;
   uint64_t gen_n8;
   DropoutParams gen_drop;

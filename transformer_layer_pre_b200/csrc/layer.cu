@@ -387,18 +387,16 @@ tl_status layer_forward(tl_layer* L, const void* x, const float* mask, const tl_
   e2.bias = w->b2; e2.drop = make_drop(L, L->ph); e2.site = 2;
 
   // hidden-dropout keep bits are drawn once, ahead of their consumers, which
-  // read them instead of drawing Philox: site 1 by the QKV GEMM's pairs that
-  // sit out its last round, site 2 likewise by the out-projection GEMM's;
-  // where a GEMM has no such pairs, by the LayerNorm forward before the
-  // consumer (pre-LN: LN1 for site 1, LN2 for site 2; post-LN: LN1 for site 2)
+  // read them instead of drawing Philox: both sites by the QKV GEMM's CTA
+  // pairs that sit out its last round; where it has none (small batches), by
+  // the LayerNorm forward before the consumer (pre-LN: LN1 for site 1, LN2 for
+  // site 2; post-LN: LN1 for site 2)
   const bool keepbits = eo.drop.thr != 0;
-  const bool k1_gemm = keepbits && gemm_tc_bubble_pairs(dt, T, 3 * H, eq) >= 8;
-  const bool k2_gemm = keepbits && gemm_tc_bubble_pairs(dt, T, H, eo) >= 8;
+  const bool k1_gemm = keepbits && gemm_tc_bubble_pairs(dt, T, 3 * H, eq) >= 16;
+  const bool k2_gemm = k1_gemm;
   if (k1_gemm) {
-    eq.gen_keep = L->keep1; eq.gen_site = 1; eq.gen_n8 = (uint64_t)T * H / 8; eq.gen_drop = eo.drop;
-  }
-  if (k2_gemm) {
-    eo.gen_keep = L->keep2; eo.gen_site = 2; eo.gen_n8 = (uint64_t)T * H / 8; eo.gen_drop = e2.drop;
+    eq.gen_keep = L->keep1; eq.gen_keep2 = L->keep2; eq.gen_site = 1; eq.gen_n8 = (uint64_t)T * H / 8;
+    eq.gen_drop = eo.drop;
   }
   if (L->pre_ln) {
     {
