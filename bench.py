@@ -245,9 +245,14 @@ def size_sample(w, inp, target_s: float) -> tuple[int, float]:
 def cpu_baseline(w, inp, target_s: float = 15.0) -> dict:
     nseq, _ = size_sample(w, inp, target_s)
     t = oracle_step(w, inp, nseq)
-    return {"value": nseq * w.seq / t, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
+    reps = 1
+    # the whole batch can take less than the target: repeat it (at most 4 times)
+    while t < 0.67 * target_s and reps < 4:
+        t += oracle_step(w, inp, nseq)
+        reps += 1
+    return {"value": reps * nseq * w.seq / t, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
             "sample": f"float64 oracle forward+backward of {nseq} of the {w.batch} sequences "
-                      f"({nseq * w.seq} tokens), {t:.1f} s"}
+                      f"({nseq * w.seq} tokens) x {reps}, {t:.1f} s"}
 
 
 def run_reference(args) -> None:
