@@ -74,10 +74,13 @@ typedef struct {
   int dtype;                     /* tl_dtype; default TL_F32 (fp16 = False) */
   float ln_eps;                  /* default 1e-12 */
   uint64_t philox_offset;        /* 4th Philox counter word; the layer id in a stack (default 0) */
-  int gelu_checkpoint;           /* 1: keep only the FFN1 pre-activation U; GELU(U) is
-                                    recomputed in backward.  Results are bitwise identical. */
+  int gelu_checkpoint;           /* 1: keep only the FFN1 pre-activation U; GELU(U) and
+                                    GELU'(U) are recomputed in backward (0: the forward
+                                    keeps G = GELU(U) and GELU'(U)).  Results are bitwise
+                                    identical. */
   int attn_dropout_checkpoint;   /* accepted; the attention kernels never store the
-                                    dropped probabilities, so this is always in effect */
+                                    dropped probabilities (only their keep bits, one bit
+                                    per element), so this is always in effect */
   int normalize_invertible;      /* 1: LayerNorm backward from its output, the LayerNorm
                                     input is not needed (layer_backward may get x = NULL
                                     in pre-LN form); requires every gamma != 0 */
