@@ -345,14 +345,35 @@ __device__ __forceinline__ bool pair_epilogue_tile(const OutMaps& om, const TcAr
   const int m = mrow0 + lane;
   const int nbase = nb * BN + part * CW;
   const bool mrow = m < g.M;
-  uint4 pre[EpiAux<KIND>::kNeeds ? CW / 8 : 1];
+  // The epilogue's (M, N) input (residual, U or GELU'(U)) of this warp's 32
+  // rows x 64 columns is loaded row-contiguously (8 lanes per 128-byte row
+  // segment, 4 rows per load) into the warp's two staging boxes, in the
+  // swizzled layout the outputs use; each lane then reads its own row from
+  // there and the outputs overwrite it in place.  (Row-per-lane 16-byte
+  // loads touched 32 lines per instruction.)
+  static_assert(!EpiAux<KIND>::kNeeds || (NOUT == 1 && OUT_ES == 2 && CW == 2 * SW), "aux staging layout");
+  bool aux_on = false;
   if constexpr (EpiAux<KIND>::kNeeds) {
     const T* ap = static_cast<const T*>(epi_aux_ptr(e, epi_base(KIND)));
+    aux_on = ap != nullptr;
+    if (aux_on) {
+      if (lane == 0) bulk_wait_read<0>();   // both boxes free: earlier stores from them have read them
+      __syncwarp();
+      const int ch = lane & 7;              // 16-byte chunk of the row's 128 bytes
+      const int n = nbase + ch * 8;
+      uint4 v[8];
 #pragma unroll
-    for (int j = 0; j < CW / 8; ++j) {
-      const int n = nbase + j * 8;
-      pre[j] = (ap && mrow && n < g.N) ? *reinterpret_cast<const uint4*>(ap + (size_t)m * e.ldo + n)
-                                        : make_uint4(0u, 0u, 0u, 0u);
+      for (int k = 0; k < 8; ++k) {
+        const int mm = mrow0 + k * 4 + (lane >> 3);
+        v[k] = (mm < g.M && n < g.N) ? *reinterpret_cast<const uint4*>(ap + (size_t)mm * e.ldo + n)
+                                      : make_uint4(0u, 0u, 0u, 0u);
+      }
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        const int rl = k * 4 + (lane >> 3);   // row within the warp's 32
+        *reinterpret_cast<uint4*>(stage0 + (ch >> 2) * kStageOut + rl * 64 + (((ch & 3) ^ ((rl >> 1) & 3)) << 4)) = v[k];
+      }
+      __syncwarp();
     }
   }
   // precomputed dropout keep bits of this thread's 64 columns (one byte per 8), loaded early
@@ -380,11 +401,13 @@ __device__ __forceinline__ bool pair_epilogue_tile(const OutMaps& om, const TcAr
     }
     uint8_t* sb0 = stage0 + (NOUT == 2 ? 0 : nbuf) * kStageOut;
     uint8_t* sb1 = stage0 + kStageOut;
-    if (lane == 0) {
-      if constexpr (NOUT == 2) bulk_wait_read<0>();
-      else bulk_wait_read<1>();
+    if (!aux_on) {
+      if (lane == 0) {
+        if constexpr (NOUT == 2) bulk_wait_read<0>();
+        else bulk_wait_read<1>();
+      }
+      __syncwarp();
     }
-    __syncwarp();
     if constexpr (OUT_ES == 4) {
       // 16 floats = four 16-byte chunks of the 64-byte row
 #pragma unroll
@@ -398,8 +421,13 @@ __device__ __forceinline__ bool pair_epilogue_tile(const OutMaps& om, const TcAr
         float* vq = v + q * 8;
         float v2[8];
         float aux[8];
-        if constexpr (EpiAux<KIND>::kNeeds) unpack8<T>(pre[(c0 >> 3) + q], aux);
-        else {
+        if constexpr (EpiAux<KIND>::kNeeds) {
+          if (aux_on) unpack8<T>(*reinterpret_cast<const uint4*>(sb0 + lane * 64 + ((q ^ swz) << 4)), aux);
+          else {
+#pragma unroll
+            for (int i = 0; i < 8; ++i) aux[i] = 0.0f;
+          }
+        } else {
 #pragma unroll
           for (int i = 0; i < 8; ++i) aux[i] = 0.0f;
         }
