@@ -139,8 +139,27 @@ tl_status layer_forward(tl_layer* layer, const void* x, const float* mask,
 tl_status layer_backward(tl_layer* layer, const void* x, const void* dy,
                          const tl_weights* w, tl_grads* g, void* dx, void* stream);
 
-/* Device bytes the layer holds (saved activations + scratch). */
+/* Device bytes the layer holds: its saved activations, plus its own scratch
+ * unless it uses a shared one (layer_share_scratch). */
 size_t layer_workspace_bytes(const tl_layer* layer);
+
+/* Scratch sharing ("DeepSpeed Transformer Kernel usage guide", Step 3: the
+ * memory switches exist so that larger micro-batches fit).  A layer's
+ * scratch holds what lives only within one layer_forward or layer_backward
+ * call (the backward's intermediate gradients, GELU(U) between the two FFN
+ * GEMMs in recompute mode, column-sum partials, split-K partials); nothing
+ * in it is needed from one call to the next.  Layers of a stack that never
+ * run at the same time can therefore share one scratch.
+ * layer_scratch_bytes: the size this layer's scratch needs (its options
+ * included).  layer_share_scratch: the layer frees its own scratch and uses
+ * `scratch` (a device buffer of `bytes` >= layer_scratch_bytes, 256-byte
+ * aligned, owned by the caller and valid for the layer's lifetime) instead;
+ * TL_EINVAL if it is null, unaligned or too small.  Calls of layers that
+ * share a scratch must not overlap on the GPU (enqueue them on one stream,
+ * or order the streams).  layer_set_options keeps a shared scratch while it
+ * is large enough for the new options, else the layer allocates its own. */
+size_t layer_scratch_bytes(const tl_layer* layer);
+tl_status layer_share_scratch(tl_layer* layer, void* scratch, size_t bytes);
 
 /* Text of the last error on this layer ("" if none).  Valid until the next call. */
 const char* layer_last_error(const tl_layer* layer);
@@ -170,6 +189,22 @@ tl_status tl_gelu_tanh_eval(const float* u, float* g, float* dg, uint64_t n, voi
  * TL_OK.  Blocks the host. */
 tl_status tl_device_check(void);
 
+/* Failure detection.  Every wait of the tensor-core and row kernels on an
+ * mbarrier (for a copy, an MMA or another warp) is bounded: once it has
+ * waited longer than the limit it records an error, lets the copies it has
+ * issued land, frees its tensor memory and returns, and tl_device_check
+ * reports TL_ETIMEOUT.  tl_set_wait_limit_ns sets that limit for the
+ * current device (ns; 0 restores the default of 2 s); it is synchronous
+ * and applies to launches enqueued after it.  A limit shorter than the
+ * longest legitimate wait (microseconds in these kernels) makes healthy
+ * kernels give up.
+ * tl_wait_probe enqueues a one-thread kernel whose single bounded wait
+ * nothing ever satisfies: it gives up after the current limit with nothing
+ * else in flight, so the next tl_device_check reports TL_ETIMEOUT and the
+ * context stays usable (a test of the detection path). */
+tl_status tl_set_wait_limit_ns(uint64_t ns);
+tl_status tl_wait_probe(void* stream);
+
 /* Profiling (off by default).  While enabled, the library brackets each of
  * its kernel launches with a pair of CUDA events on the launching stream.
  * tl_profile_read synchronises the device, fills ms[c] (summed elapsed
@@ -195,10 +230,14 @@ long long tl_launch_count(void);
  * multiple of 8, rows >= 1, both pointers 16-byte aligned, else TL_EINVAL.
  * The first call on a device looks up the array's device address
  * (cudaGetSymbolAddress); make that first call before any stream capture.
+ * The address is kept per device together with the CUDA context it belongs
+ * to; after a device reset (a new context) the next call looks it up again
+ * and, like a first call, belongs before any capture.
  * Every call shares the one array and overwrites it: calls that overlap on
  * the GPU (other streams, other threads) race and must be serialised by the
  * caller.  Enqueued on `stream` (a cudaStream_t); returns before the GPU
- * finishes.  TL_ECUDA if a CUDA call fails. */
+ * finishes.  TL_ECUDA if a CUDA call fails, including an error that an
+ * earlier call left pending when this one starts (it is cleared). */
 tl_status tl_bias_grad_noalloc(int dtype, const void* dz, int rows, int cols, float* db, void* stream);
 
 /* Progressive Layer Dropping for a stack of layers ("Progressive Layer

@@ -6,6 +6,9 @@ import pytest
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
+HERE = os.path.dirname(os.path.abspath(__file__))
+if HERE not in sys.path:
+    sys.path.insert(0, HERE)
 
 
 def pytest_configure(config):
@@ -21,3 +24,14 @@ def pytest_collection_modifyitems(config, items):
     for it in items:
         if "gpu" in it.keywords:
             it.add_marker(skip)
+
+
+def pytest_terminal_summary(terminalreporter, exitstatus, config):
+    """Prints the parity margins recorded by tests/parity.py (one line per
+    test: the worst error against each bar and the tensor it comes from)."""
+    mod = sys.modules.get("parity")
+    if mod is None or not getattr(mod, "REPORT", None):
+        return
+    terminalreporter.write_sep("-", "parity margins")
+    for line in mod.summary_lines():
+        terminalreporter.write_line(line)

@@ -3,23 +3,34 @@ and the oracle on the same seeded inputs, and compare with the stated bars.
 
 Bars (what the layer must meet against the float64 oracle):
   * float32 storage: max|gpu - oracle| / max|oracle| <= 1e-5 per tensor;
-  * float16 / bfloat16 storage: relative Frobenius error <= 1e-2 against the
-    pure float64 oracle for every tensor, and a max-abs bar of 2e-2 against
-    the oracle in storage-rounded mode (float64 arithmetic, rounded to the
-    storage type where the CUDA path stores a tensor):
-      - y and dx (unit-scale tensors): max |gpu - oracle| <= 2e-2 plus two
-        units in the last place of their own 16-bit storage at the value: one
-        for the output's own rounding and one for a one-unit flip of the
-        stored tensor that feeds the last step (a residual sum or a LayerNorm
-        input of similar magnitude).  Both sides round values that can fall
-        on either side of a rounding boundary; for bfloat16 magnitudes >= 4
-        one such unit, 2^-5, exceeds 2e-2 by itself;
-      - weight and bias gradients (float32 sums over all T tokens, whose
-        magnitude and rounding noise grow like sqrt(T)): max |gpu - oracle|
-        <= 2e-2 * max(1, max |oracle|), i.e. the bar relative to the
-        tensor's own scale.
+  * float16 / bfloat16 storage, every tensor: relative Frobenius error
+    <= 1e-2 against the pure float64 oracle; and a max-abs bar against the
+    oracle in storage-rounded mode (float64 arithmetic, rounded to the
+    storage type exactly where the CUDA path stores a tensor in HBM):
+      - y and dx: float16: max |gpu - oracle| <= 2e-2.  bfloat16: 2e-2
+        plus two units in the last place of bfloat16 at the value (one for
+        the output's own rounding, one for a one-unit flip of the stored
+        tensor feeding the last step; one unit, 2^-5 at magnitudes >= 4, is
+        above 2e-2 by itself);
+      - weight and bias gradients: max |gpu - oracle| <= 2e-2, or one unit
+        in the last place of the storage type at the tensor's largest
+        magnitude when that unit is larger (float16 from magnitude 32 on,
+        bfloat16 from 4 on).  These gradients are float32 sums over all T
+        tokens of products of stored 16-bit values; two equally valid
+        implementations that round at the same points but accumulate in a
+        different order (the storage-rounded oracle in float32 and in
+        float64) already differ by more than 2e-2 once the sums are that
+        large (BERT-Large B64: up to 0.061 at |bqkv| <= 224; BERT-base bf16
+        B8: up to 0.11 at |bo| <= 134).
+Every comparison also records the literal reading of the 2e-2 bar: max-abs
+error against the PURE float64 oracle (inputs rounded, nothing else), and
+the ratio of the storage-rounded max-abs error to a flat 2e-2.  They are
+reported, not asserted.  The records of a test session are printed at its
+end (see conftest.py).
 """
 from __future__ import annotations
+
+import os
 
 import numpy as np
 import torch
@@ -30,6 +41,12 @@ from transformer_layer_pre_b200.synthetic import Inputs, Workload, to_f64
 
 TORCH_DT = {"f32": torch.float32, "f16": torch.float16, "bf16": torch.bfloat16}
 ULP_BITS = {"f16": 10, "bf16": 7}
+MAX_ABS = 2e-2
+REL_FROB = 1e-2
+REL_MAX_F32 = 1e-5
+
+# (test id, tensor name, dtype, error record) of every check_tensor call
+REPORT: list = []
 
 
 def oracle_config(w: Workload, batch: int, philox_offset: int = 0) -> oracle.LayerConfig:
@@ -85,30 +102,42 @@ def ulp(ref: np.ndarray, dtype: str) -> np.ndarray:
     return np.ldexp(1.0, e - 1 - ULP_BITS[dtype])
 
 
+def allowance(rounded: np.ndarray, dtype: str, stored: bool):
+    """The max-abs allowance against the storage-rounded oracle (scalar or
+    per element); see the module docstring."""
+    if stored:
+        return MAX_ABS if dtype == "f16" else MAX_ABS + 2.0 * ulp(rounded, dtype)
+    return max(MAX_ABS, float(ulp(np.asarray(np.abs(rounded).max()), dtype)))
+
+
 def errors(gpu: np.ndarray, pure: np.ndarray, rounded: np.ndarray | None, dtype: str, stored: bool) -> dict:
     gpu, pure = np.asarray(gpu), np.asarray(pure)
     assert gpu.shape == pure.shape
     assert np.all(np.isfinite(gpu)), "non-finite values"
-    out = {"rel_max": float(np.abs(gpu - pure).max() / max(np.abs(pure).max(), 1e-300)),
-           "rel_frob": float(np.linalg.norm(gpu - pure) / max(np.linalg.norm(pure), 1e-300))}
+    dp = np.abs(gpu - pure)
+    out = {"rel_max": float(dp.max() / max(np.abs(pure).max(), 1e-300)),
+           "rel_frob": float(np.linalg.norm(gpu - pure) / max(np.linalg.norm(pure), 1e-300)),
+           "max_abs_pure": float(dp.max()), "max_ref": float(np.abs(pure).max())}
     if rounded is not None:
         d = np.abs(gpu - rounded)
+        allow = allowance(rounded, dtype, stored)
         out["max_abs"] = float(d.max())
-        if stored:
-            allow = 2e-2 + 2.0 * ulp(rounded, dtype)
-        else:
-            allow = 2e-2 * max(1.0, float(np.abs(rounded).max()))
+        out["flat_ratio"] = float(d.max() / MAX_ABS)
         out["excess"] = float((d - allow).max())
+        # the worst ratio error / allowance (1.0 = at the bar)
+        out["bar_ratio"] = float((d / allow).max())
     return out
 
 
 def check_tensor(name: str, gpu, pure, rounded, dtype: str, stored: bool) -> dict:
     e = errors(gpu, pure, rounded, dtype, stored)
+    REPORT.append((os.environ.get("PYTEST_CURRENT_TEST", "?").split(" ")[0], name, dtype, e))
     if dtype == "f32":
-        assert e["rel_max"] <= 1e-5, (name, e)
+        assert e["rel_max"] <= REL_MAX_F32, (name, e)
     else:
-        assert e["rel_frob"] <= 1e-2, (name, e)
-        assert e["excess"] <= 0.0, (name, e)
+        assert e["rel_frob"] <= REL_FROB, (name, e)
+        if rounded is not None:
+            assert e["excess"] <= 0.0, (name, e)
     return e
 
 
@@ -120,3 +149,31 @@ def check_layer(gpu: dict, pure: dict, rounded: dict | None, dtype: str) -> dict
         report[n] = check_tensor(n, gpu["grads"][n], pure["grads"][n],
                                  None if rounded is None else rounded["grads"][n], dtype, False)
     return report
+
+
+def summary_lines() -> list:
+    """One line per test: the worst bar ratios and the literal pure-oracle
+    max-abs error, with the tensors they come from."""
+    by_test: dict = {}
+    for test, name, dtype, e in REPORT:
+        by_test.setdefault(test, []).append((name, dtype, e))
+    lines = []
+    for test, rows in by_test.items():
+        dtype = rows[0][1]
+        short = test.split("::")[-1]
+        if dtype == "f32":
+            n, _, e = max(rows, key=lambda r: r[2]["rel_max"])
+            lines.append(f"{short} [f32] rel_max {e['rel_max']:.1e} ({n}) / bar {REL_MAX_F32:.0e}")
+            continue
+        nf, _, ef = max(rows, key=lambda r: r[2]["rel_frob"])
+        np_, _, ep = max(rows, key=lambda r: r[2]["max_abs_pure"])
+        s = f"{short} [{dtype}] rel_frob {ef['rel_frob']:.1e} ({nf}) / bar {REL_FROB:.0e}"
+        rr = [r for r in rows if "bar_ratio" in r[2]]
+        if rr:
+            nb, _, eb = max(rr, key=lambda r: r[2]["bar_ratio"])
+            s += f"; max_abs vs rounded {eb['max_abs']:.1e} ({nb}, {eb['bar_ratio']:.2f} of its bar)"
+            nl, _, el = max(rr, key=lambda r: r[2]["flat_ratio"])
+            s += f", {el['flat_ratio']:.2f} of a flat 2e-2 ({nl})"
+        s += f"; max_abs vs pure {ep['max_abs_pure']:.1e} ({np_})"
+        lines.append(s)
+    return lines

@@ -4,7 +4,9 @@ the same seeded inputs, element by element.
 Cases: the tiny float32 layer; ragged shapes (token counts, widths and FFN
 sizes that are not multiples of any tile) in both layer orders; the
 BERT-base bf16 workload at full size; the BERT-Large fp16 workload at a
-reduced batch; the long-sequence post-LN bf16 workload at batch 1."""
+reduced batch and at its full batch of 64 (every gradient); the
+long-sequence post-LN bf16 workload at batch 1 and, on sampled sequences,
+at its full batch."""
 import dataclasses
 
 import numpy as np
@@ -157,6 +159,26 @@ def test_gelu_tanh_checkpoint_is_bitwise_identical():
         assert np.array_equal(a["grads"][n], b["grads"][n]), n
 
 
+# Valid lengths that end well before the sequence does: the long-sequence
+# attention kernels skip key tiles past the last unmasked key (forward,
+# dQ) and write zero dK, dV for key tiles that hold only masked keys; the
+# result must not change (2^-inf = 0 exactly).  Lengths 37 (one partly valid
+# tile of three), 128 (exactly one tile), 129 (one key into the second) and
+# 384 (no padding).
+SHORT_LEN_F16 = Workload("short-lengths-f16", 4, 384, 128, 2, 256, "f16", 0.1, 0.1)
+
+
+@pytest.mark.parametrize("pre_ln", [True, False])
+def test_long_sequence_skips_padded_key_tiles_exactly(pre_ln):
+    from transformer_layer_pre_b200.synthetic import make_mask
+    w = dataclasses.replace(SHORT_LEN_F16, pre_layer_norm=pre_ln)
+    inp = make_inputs(w)
+    lengths = np.array([37, 128, 129, 384])
+    inp = dataclasses.replace(inp, mask=make_mask(lengths, w.seq), lengths=lengths)
+    gpu = run_gpu(inp)
+    check_layer(gpu, run_oracle(inp), run_oracle(inp, storage_rounded=True), w.dtype)
+
+
 def _sampled_full_size(w: Workload, idx):
     """Whole-batch run on the GPU at the workload's full size; y and dx of the
     sampled sequences against the oracle run on those sequences alone (their
@@ -171,8 +193,16 @@ def _sampled_full_size(w: Workload, idx):
     check_tensor("dx", gpu["dx"][idx], pure["dx"], rounded["dx"], w.dtype, True)
 
 
-def test_bert_large_f16_full_batch_sampled_sequences():
-    _sampled_full_size(WORKLOADS["bert-large-f16"], [0, 37, 63])
+def test_bert_large_f16_full_batch_every_gradient():
+    """The benchmarked workload itself (B64 S128 H1024, fp16, dropout 0.1;
+    "DeepSpeed Transformer Kernel usage guide", Step 1's BERT-Large) at its
+    full batch, in the launch configuration the benchmark times: y, dx and
+    all twelve parameter gradients element by element against the oracle,
+    pure and storage-rounded.  This is where the GEMM tile plans, the
+    split-K weight gradients, the keep bits drawn by the idle CTA pairs of
+    the QKV GEMM and the persistent attention's multi-round schedule run at
+    the sizes the benchmark uses."""
+    _parity(WORKLOADS["bert-large-f16"])
 
 
 def test_long_post_ln_bf16_full_batch_sampled_sequences():

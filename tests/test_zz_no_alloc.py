@@ -4,7 +4,8 @@ It serves callers that cannot allocate device memory: its partial sums live
 in a fixed array inside the library.  Its result must equal what the
 existing entry point computes for the same quantity: layer_backward's
 gradient of the FFN output bias, which in pre-LN form with hidden dropout 0
-is the column sum of dY.  Two calls in a row check that the shared array's
+is the column sum of dY; and it must equal that column sum computed in
+float64 on the host from the stored dY.  Two calls in a row check that the shared array's
 leftover contents do not leak into the next result.  This file is collected
 last so that a run stopping at its first failure has run everything else.
 """
@@ -57,6 +58,9 @@ def test_noalloc_bias_grad_matches_layer_backward(dtype):
         a, r = out.double().cpu().numpy(), ref.double().cpu().numpy()
         assert np.all(np.isfinite(a))
         assert np.abs(a - r).max() <= 1e-5 * max(1.0, np.abs(r).max()), (call, np.abs(a - r).max())
+        # and the column sum itself, in float64 on the host from the stored values
+        exact = dy.double().cpu().numpy().reshape(B * S, H).sum(axis=0)
+        assert np.abs(a - exact).max() <= 1e-5 * max(1.0, np.abs(exact).max()), (call, np.abs(a - exact).max())
 
 
 def test_noalloc_rejects_sizes_beyond_its_array():

@@ -16,7 +16,7 @@ import torch
 __all__ = ["Layer", "Options", "TlError", "LibraryMissing", "load_library", "dropout_keep_mask",
            "WEIGHT_NAMES", "DTYPE_CODES", "EXPORTED_SYMBOLS", "device_check",
            "profile_enable", "profile_read", "launch_count", "PROFILE_CLASSES",
-           "pld_theta", "pld_keep_prob", "pld_keep"]
+           "pld_theta", "pld_keep_prob", "pld_keep", "set_wait_limit", "wait_probe"]
 
 HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(HERE, "libtlp.so")
@@ -32,6 +32,7 @@ EXPORTED_SYMBOLS = (
     "layer_destroy", "tl_dropout_keep_mask", "tl_device_check", "tl_profile_enable",
     "tl_profile_read", "tl_launch_count", "tl_bias_grad_noalloc", "tl_gelu_eval", "tl_status_string",
     "tl_pld_theta", "tl_pld_keep_prob", "tl_pld_keep", "tl_gelu_tanh_eval",
+    "tl_set_wait_limit_ns", "tl_wait_probe", "layer_scratch_bytes", "layer_share_scratch",
 )
 PROFILE_CLASSES = ("gemm", "attn_fwd", "attn_bwd", "ln_fwd", "ln_bwd", "rowwise")
 
@@ -89,6 +90,10 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.layer_backward.restype = i
     lib.layer_workspace_bytes.argtypes = [vp]
     lib.layer_workspace_bytes.restype = ctypes.c_size_t
+    lib.layer_scratch_bytes.argtypes = [vp]
+    lib.layer_scratch_bytes.restype = ctypes.c_size_t
+    lib.layer_share_scratch.argtypes = [vp, vp, ctypes.c_size_t]
+    lib.layer_share_scratch.restype = i
     lib.layer_last_error.argtypes = [vp]
     lib.layer_last_error.restype = ctypes.c_char_p
     lib.layer_destroy.argtypes = [vp]
@@ -118,6 +123,10 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.tl_pld_keep_prob.restype = d
     lib.tl_pld_keep.argtypes = [u64, u64, i, i, d]
     lib.tl_pld_keep.restype = i
+    lib.tl_set_wait_limit_ns.argtypes = [u64]
+    lib.tl_set_wait_limit_ns.restype = i
+    lib.tl_wait_probe.argtypes = [vp]
+    lib.tl_wait_probe.restype = i
     _lib = lib
     return lib
 
@@ -199,7 +208,20 @@ class Layer:
 
     @property
     def workspace_bytes(self) -> int:
+        """Device bytes the layer holds (saved activations + its own scratch)."""
         return int(self.lib.layer_workspace_bytes(self.handle))
+
+    @property
+    def scratch_bytes(self) -> int:
+        """Bytes of the per-call scratch this layer needs."""
+        return int(self.lib.layer_scratch_bytes(self.handle))
+
+    def share_scratch(self, buf: torch.Tensor) -> None:
+        """Use `buf` (a device tensor of >= scratch_bytes bytes, 256-byte
+        aligned; the caller keeps it alive) as this layer's scratch; layers
+        sharing one must not run concurrently."""
+        self._check(self.lib.layer_share_scratch(self.handle, _ptr(buf), buf.numel() * buf.element_size()))
+        self._scratch_ref = buf
 
     def close(self) -> None:
         if self.handle:
@@ -218,6 +240,24 @@ def device_check() -> None:
     bounded device-side wait that gave up."""
     lib = load_library()
     st = lib.tl_device_check()
+    if st != 0:
+        raise TlError(st, lib.tl_status_string(st).decode())
+
+
+def set_wait_limit(ns: int) -> None:
+    """Limit (ns; 0 = the default 2 s) of every bounded device-side wait on
+    the current device."""
+    lib = load_library()
+    st = lib.tl_set_wait_limit_ns(int(ns))
+    if st != 0:
+        raise TlError(st, lib.tl_status_string(st).decode())
+
+
+def wait_probe(stream=None) -> None:
+    """Enqueues a kernel whose one bounded wait is never satisfied; the next
+    device_check raises TlError with status 5 (TL_ETIMEOUT)."""
+    lib = load_library()
+    st = lib.tl_wait_probe(_stream(stream))
     if st != 0:
         raise TlError(st, lib.tl_status_string(st).decode())
 

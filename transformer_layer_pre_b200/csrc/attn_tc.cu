@@ -59,7 +59,8 @@ struct AttnTc {
   float* colsum;        // fused QKV bias-gradient partials (persistent backward), or null
   int fuse_dq;
   int ctx_tma;          // persistent kernels: ctx (forward) or dQKV (backward) rows leave by TMA store (S % 32 == 0)
-  uint8_t* keep;        // persistent path: attention keep bits [B*nh][128][16] (forward writes, backward reads)
+  uint8_t* keep;        // attention keep bits (forward writes, backward reads) or null: persistent path
+                        // [B*nh][128][16]; longer sequences flat, byte e/8 for element e of site 0
   int bf16;
   int* err;
 };
@@ -92,6 +93,42 @@ __device__ __forceinline__ float mask_log2(const AttnTc& a, int b, int key) {
   if (key >= a.S) return -INFINITY;
   return a.mask ? a.mask[(size_t)b * a.S + key] * kLog2e : 0.0f;
 }
+// The additive mask of keys key0 .. key0+7 (key0 % 8 == 0, S % 8 == 0), in
+// log2 units: two 16-byte loads that every lane of a warp shares.
+__device__ __forceinline__ void mask8_log2(const AttnTc& a, int b, int key0, float (&m)[8]) {
+  if (key0 >= a.S) {
+#pragma unroll
+    for (int t = 0; t < 8; ++t) m[t] = -INFINITY;
+  } else if (!a.mask) {
+#pragma unroll
+    for (int t = 0; t < 8; ++t) m[t] = 0.0f;
+  } else {
+    const float4* p = reinterpret_cast<const float4*>(a.mask + (size_t)b * a.S + key0);
+    const float4 u = __ldg(p), v = __ldg(p + 1);
+    m[0] = u.x * kLog2e; m[1] = u.y * kLog2e; m[2] = u.z * kLog2e; m[3] = u.w * kLog2e;
+    m[4] = v.x * kLog2e; m[5] = v.y * kLog2e; m[6] = v.z * kLog2e; m[7] = v.w * kLog2e;
+  }
+}
+
+// One past the last key of sequence b whose additive mask is not -inf (S
+// without a mask), found by the whole block.  Key tiles at or beyond it hold
+// only masked keys: their probabilities are exactly 0 (2^-inf), so they add
+// nothing to any row sum, output or gradient, and the long-sequence kernels
+// skip them ("AI-infra engineers and the Transformer", section 2.1 Step 4:
+// dynamic padding keeps padded positions out of the work).  Call after
+// pdl_wait, from every thread of the block.
+__device__ __forceinline__ int key_extent(const AttnTc& a, int b) {
+  if (!a.mask) return a.S;
+  __shared__ int ext;
+  if (threadIdx.x == 0) ext = 0;
+  __syncthreads();
+  int e = 0;
+  for (int j = threadIdx.x; j < a.S; j += blockDim.x)
+    if (a.mask[(size_t)b * a.S + j] != -INFINITY) e = j + 1;
+  if (e) atomicMax(&ext, e);
+  __syncthreads();
+  return ext;
+}
 
 // ============================================================================ forward
 // Warps: 0 TMA, 1 MMA (+TMEM owner), 2-5 softmax (thread = query row).
@@ -118,7 +155,7 @@ __global__ void __launch_bounds__(kFwdThreads)
   const int S = a.S;
   const int row0 = (b * a.nh + h) * S;
   const int q0 = blockIdx.x * TILE;
-  const int ntiles = (S + TILE - 1) / TILE;
+  const int ntiles_all = (S + TILE - 1) / TILE;
 
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
@@ -139,6 +176,9 @@ __global__ void __launch_bounds__(kFwdThreads)
   pdl_wait();
   pdl_launch_dependents();
   const uint32_t tS = tmem, tO = tmem + 128;
+  // key tiles past the last unmasked key are skipped (at least one is run,
+  // so a fully masked row still ends with its zero output)
+  const int ntiles = max(1, min(ntiles_all, (key_extent(a, b) + TILE - 1) / TILE));
 
   if (warp == 0) {
     if (lane == 0) {
@@ -188,6 +228,7 @@ __global__ void __launch_bounds__(kFwdThreads)
     const float c2 = a.scale * kLog2e;
     const float dsc = a.drop.thr ? a.drop.scale : 1.0f;
     const uint64_t erow = ((uint64_t)row0 + (uint64_t)i) * (uint64_t)S;
+    const bool row_ok = i < S;
     float o[HD];
 #pragma unroll
     for (int c = 0; c < HD; ++c) o[c] = 0.0f;
@@ -204,7 +245,12 @@ __global__ void __launch_bounds__(kFwdThreads)
         float sv[32];
         tmem_ld32(tS + lo + c * 32, sv);
 #pragma unroll
-        for (int t = 0; t < 32; ++t) mx = fmaxf(mx, fmaf(sv[t], c2, mask_log2(a, b, k0 + c * 32 + t)));
+        for (int g = 0; g < 4; ++g) {
+          float ml[8];
+          mask8_log2(a, b, k0 + c * 32 + g * 8, ml);
+#pragma unroll
+          for (int t = 0; t < 8; ++t) mx = fmaxf(mx, fmaf(sv[g * 8 + t], c2, ml[t]));
+        }
       }
       const float m_new = fmaxf(m, mx);
       const float alpha = (m == -INFINITY) ? 0.0f : exp2f(m - m_new);
@@ -222,21 +268,40 @@ __global__ void __launch_bounds__(kFwdThreads)
         tc_fence_before();
         mbar_arrive(o_free);
       }
-      // pass 2: probabilities, dropout, P to shared memory
+      // pass 2: probabilities, dropout, P to shared memory; the keep bits are
+      // also written out for the backward (byte e/8 of site 0, e the flat index)
       float lsum = 0.0f;
+      const float msub = m_new == -INFINITY ? 0.0f : m_new;   // 2^(-inf - msub) = 0
 #pragma unroll 1
       for (int c = 0; c < 4; ++c) {
         float sv[32];
         tmem_ld32(tS + lo + c * 32, sv);
+        uint32_t kw = 0xFFFFFFFFu;
+        if (a.drop.thr) {
+          const uint64_t e8 = (erow + (uint64_t)(k0 + c * 32)) >> 3;
+          kw = 0;
+#pragma unroll
+          for (int g = 0; g < 4; ++g) kw |= dropout_bits8(a.drop, 0, e8 + g) << (8 * g);
+          if (a.keep && row_ok) {
+            // a 32-bit word when it is 4-byte aligned (S % 32 == 0), else bytes
+            if ((e8 & 3) == 0) {
+              *reinterpret_cast<uint32_t*>(a.keep + e8) = kw;
+            } else {
+#pragma unroll
+              for (int g = 0; g < 4; ++g) a.keep[e8 + g] = (uint8_t)(kw >> (8 * g));
+            }
+          }
+        }
 #pragma unroll
         for (int g = 0; g < 4; ++g) {
           const int kb = k0 + c * 32 + g * 8;
-          const uint32_t bits = a.drop.thr ? dropout_bits8(a.drop, 0, (erow + (uint64_t)kb) >> 3) : 0xFFu;
+          const uint32_t bits = (kw >> (8 * g)) & 0xFFu;
+          float ml[8];
+          mask8_log2(a, b, kb, ml);
           float pv[8];
 #pragma unroll
           for (int t = 0; t < 8; ++t) {
-            const float x = fmaf(sv[g * 8 + t], c2, mask_log2(a, b, kb + t));
-            const float p = (x == -INFINITY || m_new == -INFINITY) ? 0.0f : exp2f(x - m_new);
+            const float p = ex2_approx(fmaf(sv[g * 8 + t], c2, ml[t]) - msub);
             lsum += p;
             pv[t] = ((bits >> t) & 1u) ? p * dsc : 0.0f;
           }
@@ -320,16 +385,38 @@ __device__ __forceinline__ void bwd_pair_rows(const AttnTc& a, int b, int row0, 
     float sv[32], dv[32];
     tmem_ld32(tS + lo + kc0 + c * 32, sv);
     tmem_ld32(tdP + lo + kc0 + c * 32, dv);
+    // the forward's keep bits of these 32 keys (one 32-bit word), or drawn again
+    uint32_t kw = 0xFFFFFFFFu;
+    if (a.drop.thr) {
+      const uint64_t e8 = (erow + (uint64_t)(k0 + kc0 + c * 32)) >> 3;
+      if (a.keep) {
+        if (!row_ok) {
+          kw = 0u;
+        } else if ((e8 & 3) == 0) {
+          kw = __ldg(reinterpret_cast<const uint32_t*>(a.keep + e8));
+        } else {
+          kw = 0u;
+#pragma unroll
+          for (int g = 0; g < 4; ++g) kw |= (uint32_t)__ldg(a.keep + e8 + g) << (8 * g);
+        }
+      } else {
+        kw = 0;
+#pragma unroll
+        for (int g = 0; g < 4; ++g) kw |= dropout_bits8(a.drop, 0, e8 + g) << (8 * g);
+      }
+    }
 #pragma unroll
     for (int g = 0; g < 4; ++g) {
       const int kt = kc0 + c * 32 + g * 8;   // column within the key tile
       const int kb = k0 + kt;
-      const uint32_t bits = a.drop.thr ? dropout_bits8(a.drop, 0, (erow + (uint64_t)kb) >> 3) : 0xFFu;
+      const uint32_t bits = (kw >> (8 * g)) & 0xFFu;
+      float ml[8];
+      mask8_log2(a, b, kb, ml);
       float pd[8], ds[8];
 #pragma unroll
       for (int t = 0; t < 8; ++t) {
-        const float x = fmaf(sv[g * 8 + t], c2, mask_log2(a, b, kb + t));
-        const float p = (!row_ok || x == -INFINITY) ? 0.0f : exp2f(x - lse2);
+        // lse2 = +inf for rows past the sequence end: 2^-inf = 0
+        const float p = ex2_approx(fmaf(sv[g * 8 + t], c2, ml[t]) - lse2);
         const bool keep = (bits >> t) & 1u;
         pd[t] = keep ? p * dsc : 0.0f;
         const float dp = keep ? dv[g * 8 + t] * dsc : 0.0f;
@@ -367,7 +454,7 @@ __global__ void __launch_bounds__(kBwdThreads)
   const int S = a.S;
   const int row0 = (b * a.nh + h) * S;
   const int k0 = blockIdx.x * TILE;
-  const int nq = (S + TILE - 1) / TILE;
+  const int nq_all = (S + TILE - 1) / TILE;
 
   if (threadIdx.x == 0) {
     mbar_init(kv_full, 1);
@@ -390,8 +477,28 @@ __global__ void __launch_bounds__(kBwdThreads)
   pdl_wait();
   pdl_launch_dependents();
   const uint32_t tS = tmem, tdP = tmem + 128, tdV = tmem + 256, tdK = tmem + 320, tdQ = tmem + 384;
+  // every key of this tile masked: no query attends to them, dK = dV = 0
+  // exactly (this CTA runs no product; dQ never comes from here then, since
+  // fuse_dq needs one key tile that covers the sequence)
+  const bool keys_masked = !a.fuse_dq && k0 >= key_extent(a, b);
+  const int nq = keys_masked ? 0 : nq_all;
+  if (keys_masked && warp >= 2) {
+    const int sw = warp - 2, quarter = warp & 3, half = sw >> 2;
+    const int key = k0 + quarter * 32 + lane;
+    if (key < S) {
+      T* dst = static_cast<T*>(a.dqkv) + ((size_t)b * S + key) * 3 * a.H + h * HD + half * 32;
+      const float z[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+#pragma unroll
+      for (int c = 0; c < 32; c += 8) {
+        store8<T>(dst + a.H + c, z);
+        store8<T>(dst + 2 * a.H + c, z);
+      }
+    }
+  }
 
-  if (warp == 0) {
+  if (keys_masked) {
+    // nothing is loaded or multiplied
+  } else if (warp == 0) {
     if (lane == 0) {
       bool ok = true;
       mbar_arrive_expect_tx(kv_full, 2 * TB);
@@ -541,7 +648,7 @@ __global__ void __launch_bounds__(kBwdThreads)
   const int S = a.S;
   const int row0 = (b * a.nh + h) * S;
   const int q0 = blockIdx.x * TILE;
-  const int nk = (S + TILE - 1) / TILE;
+  const int nk_all = (S + TILE - 1) / TILE;
 
   if (threadIdx.x == 0) {
     mbar_init(qd_full, 1);
@@ -562,6 +669,8 @@ __global__ void __launch_bounds__(kBwdThreads)
   pdl_wait();
   pdl_launch_dependents();
   const uint32_t tS = tmem, tdP = tmem + 128, tdQ = tmem + 256;
+  // key tiles past the last unmasked key add nothing to dQ (at least one runs)
+  const int nk = max(1, min(nk_all, (key_extent(a, b) + TILE - 1) / TILE));
 
   if (warp == 0) {
     if (lane == 0) {
@@ -675,6 +784,27 @@ __device__ __forceinline__ float ex2_fast(float x) {
   float r;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(x));
   return r;
+}
+__device__ __forceinline__ float max3f(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+// Packed pairs of float32 (one instruction for both lanes on sm_100).
+__device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) {
+  unsigned long long d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;"
+      : "=l"(d)
+      : "l"(*reinterpret_cast<unsigned long long*>(&a)), "l"(*reinterpret_cast<unsigned long long*>(&b)),
+        "l"(*reinterpret_cast<unsigned long long*>(&c)));
+  return *reinterpret_cast<float2*>(&d);
+}
+__device__ __forceinline__ float2 add2(float2 a, float2 b) {
+  unsigned long long d;
+  asm("add.rn.f32x2 %0, %1, %2;"
+      : "=l"(d)
+      : "l"(*reinterpret_cast<unsigned long long*>(&a)), "l"(*reinterpret_cast<unsigned long long*>(&b)));
+  return *reinterpret_cast<float2*>(&d);
 }
 
 template <typename T>
@@ -805,6 +935,8 @@ __global__ void __launch_bounds__(kPFwdThreads, 1)
     const float c2 = a.scale * kLog2e;
     const float dsc = a.drop.thr ? a.drop.scale : 1.0f;
     const float* mrow = smask + j * 128;
+    // no mask and a full tile of keys: every mask value is 0
+    const bool plain = a.mask == nullptr && S == TILE;
     // this warp's 32 output rows staged as one 32 x 128-byte swizzled box
     // inside the group's P pair (free between P V and the next item's P)
     uint8_t* ostage = sP0 + j * 2 * TB + quarter * 4096;
@@ -821,46 +953,61 @@ __global__ void __launch_bounds__(kPFwdThreads, 1)
         __syncwarp();
       }
       const uint32_t ts = tmem + 128 * j + lo;
-      // pass 1: row maximum over the 128 keys (scaled scores + mask, log2 units)
+      // pass 1: row maximum over the 128 keys (scaled scores + mask, log2
+      // units); without a mask (and S = 128) the maximum of the raw scores,
+      // scaled once (c2 > 0)
       float mx = -INFINITY;
 #pragma unroll 1
-      for (int c = 0; c < 4; ++c) {
-        float sv[32];
-        tmem_ld32(ts + c * 32, sv);
+      for (int hh = 0; hh < 2; ++hh) {
+        float sv[64];
+        tmem_ld64(ts + hh * 64, sv);
+        if (plain) {
 #pragma unroll
-        for (int t = 0; t < 32; t += 4) {
-          const float4 m4 = *reinterpret_cast<const float4*>(mrow + c * 32 + t);
-          mx = fmaxf(mx, fmaxf(fmaxf(fmaf(sv[t], c2, m4.x), fmaf(sv[t + 1], c2, m4.y)),
-                               fmaxf(fmaf(sv[t + 2], c2, m4.z), fmaf(sv[t + 3], c2, m4.w))));
+          for (int t = 0; t < 64; t += 2) mx = max3f(mx, sv[t], sv[t + 1]);
+        } else {
+#pragma unroll
+          for (int t = 0; t < 64; t += 4) {
+            const float4 m4 = *reinterpret_cast<const float4*>(mrow + hh * 64 + t);
+            const float2 x0 = fma2(make_float2(sv[t], sv[t + 1]), make_float2(c2, c2), make_float2(m4.x, m4.y));
+            const float2 x1 = fma2(make_float2(sv[t + 2], sv[t + 3]), make_float2(c2, c2), make_float2(m4.z, m4.w));
+            mx = max3f(mx, max3f(x0.x, x0.y, x1.x), x1.y);
+          }
         }
       }
+      if (plain) mx *= c2;
       // a row whose keys are all masked has mx = -inf: every p is 0
       const float msub = mx == -INFINITY ? 0.0f : mx;
-      // pass 2: P = 2^(x - max), dropped and scaled, into the P tile; row sum of the undropped P
-      float lsum = 0.0f, lsum2 = 0.0f;
+      // pass 2: P = 2^(x - max), dropped, into the P tile; row sum of the undropped P
+      float2 ls2 = make_float2(0.0f, 0.0f);
 #pragma unroll 1
-      for (int c = 0; c < 4; ++c) {
-        float sv[32];
-        tmem_ld32(ts + c * 32, sv);
-        const uint32_t bw = c == 0 ? kb16.x : (c == 1 ? kb16.y : (c == 2 ? kb16.z : kb16.w));
+      for (int hh = 0; hh < 2; ++hh) {
+        float sv[64];
+        tmem_ld64(ts + hh * 64, sv);
+        const uint32_t bw0 = hh == 0 ? kb16.x : kb16.z, bw1 = hh == 0 ? kb16.y : kb16.w;
 #pragma unroll
-        for (int g = 0; g < 4; ++g) {
-          const uint32_t bits = (bw >> (8 * g)) & 0xFFu;
-          const float4 m0 = *reinterpret_cast<const float4*>(mrow + c * 32 + g * 8);
-          const float4 m1 = *reinterpret_cast<const float4*>(mrow + c * 32 + g * 8 + 4);
-          const float ml[8] = {m0.x, m0.y, m0.z, m0.w, m1.x, m1.y, m1.z, m1.w};
+        for (int g = 0; g < 8; ++g) {
+          const uint32_t bits = ((g < 4 ? bw0 : bw1) >> (8 * (g & 3))) & 0xFFu;
           float pv[8];
 #pragma unroll
-          for (int t = 0; t < 8; ++t) {
-            const float p = ex2_fast(fmaf(sv[g * 8 + t], c2, ml[t]) - msub);
-            if (t & 1) lsum2 += p;
-            else lsum += p;
-            pv[t] = ((bits >> t) & 1u) ? p : 0.0f;
+          for (int t = 0; t < 8; t += 2) {
+            const int k = hh * 64 + g * 8 + t;
+            float2 x;
+            if (plain) {
+              x = fma2(make_float2(sv[g * 8 + t], sv[g * 8 + t + 1]), make_float2(c2, c2), make_float2(-msub, -msub));
+            } else {
+              const float2 m2 = *reinterpret_cast<const float2*>(mrow + k);
+              x = add2(fma2(make_float2(sv[g * 8 + t], sv[g * 8 + t + 1]), make_float2(c2, c2), m2),
+                       make_float2(-msub, -msub));
+            }
+            const float2 p = make_float2(ex2_fast(x.x), ex2_fast(x.y));
+            ls2 = add2(ls2, p);
+            pv[t] = ((bits >> t) & 1u) ? p.x : 0.0f;
+            pv[t + 1] = ((bits >> (t + 1)) & 1u) ? p.y : 0.0f;
           }
-          pair_store8<T>(sP0 + j * 2 * TB, r, c * 4 + g, pv);
+          pair_store8<T>(sP0 + j * 2 * TB, r, hh * 8 + g, pv);
         }
       }
-      lsum += lsum2;
+      float lsum = ls2.x + ls2.y;
       mbar_arrive(&aux_free[j]);
       // P is written and S has been read: both hand-overs ride on p_full
       tc_fence_before();
@@ -1222,9 +1369,10 @@ bool map_tile(CUtensorMap* m, const void* p, bool bf16, uint64_t cols, uint64_t 
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// Error word of the attention kernels' bounded waits (layout in sm100.cuh).
 int* attn_error_word() {
   static int* p = nullptr;
-  if (!p) cudaMalloc(&p, sizeof(int)), cudaMemset(p, 0, sizeof(int));
+  if (!p) cudaMalloc(&p, 4 * sizeof(int)), cudaMemset(p, 0, 4 * sizeof(int));
   return p;
 }
 
@@ -1243,7 +1391,7 @@ AttnTc make_args(int dt, const AttnArgs& a) {
   t.colsum = a.colsum;
   t.fuse_dq = 0;
   t.ctx_tma = 0;
-  t.keep = a.S <= TILE ? a.keep : nullptr;
+  t.keep = a.keep;
   t.bf16 = dt == DT_BF16;
   t.err = attn_error_word();
   return t;
@@ -1340,6 +1488,10 @@ void attn_tc_fwd_run(int dt, const AttnArgs& a, cudaStream_t s) {
 void attn_tc_bwd_run(int dt, const AttnArgs& a, cudaStream_t s) {
   if (dt == DT_F16) bwd_t<half_t>(a, s);
   else bwd_t<bf16_t>(a, s);
+}
+
+void attn_tc_set_wait_limit(uint64_t ns) {
+  cudaMemcpy(attn_error_word() + 2, &ns, sizeof(ns), cudaMemcpyHostToDevice);
 }
 
 int attn_tc_take_error() {

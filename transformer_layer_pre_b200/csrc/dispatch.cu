@@ -37,6 +37,15 @@ size_t gemm_splitk_ws_floats(int dtype, int M, int N, int K) {
 
 int attn_tc_take_error();
 int rowwise_take_error();
+void gemm_tc_set_wait_limit(uint64_t ns);
+void attn_tc_set_wait_limit(uint64_t ns);
+void rowwise_set_wait_limit(uint64_t ns);
+
+void device_set_wait_limit(uint64_t ns) {
+  gemm_tc_set_wait_limit(ns);
+  attn_tc_set_wait_limit(ns);
+  rowwise_set_wait_limit(ns);
+}
 
 int device_take_error() {
   const int g = gemm_tc_take_error();

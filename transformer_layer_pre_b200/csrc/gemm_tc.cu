@@ -28,7 +28,10 @@
 
 #include <algorithm>
 #include <cstring>
+#include <mutex>
+#include <string>
 #include <type_traits>
+#include <unordered_map>
 #include <vector>
 
 #include "epilogue.cuh"
@@ -760,9 +763,11 @@ int num_sms() {
   return n;
 }
 
+// Error word of the GEMM kernels' bounded waits: four ints, [0] the error
+// code, [2..3] the host-set wait limit in ns (0 = the default; sm100.cuh).
 int* error_word() {
   static int* p = nullptr;
-  if (!p) cudaMalloc(&p, sizeof(int)), cudaMemset(p, 0, sizeof(int));
+  if (!p) cudaMalloc(&p, 4 * sizeof(int)), cudaMemset(p, 0, 4 * sizeof(int));
   return p;
 }
 
@@ -905,14 +910,97 @@ void launch_pair(const PairGemm& pa, const PairGemm& pb, const PairSched& sch, i
   count_launch();
 }
 
+// Launch cache.  The tensor maps, sizes and tile table of a pair launch
+// depend only on its operands, outputs, sizes and epilogue parameters; a
+// call that repeats them (every training step of a layer) reuses what the
+// first one built instead of encoding the tensor maps and planning the tile
+// table again.  Keyed by every field of the GEMM descriptors and epilogue
+// parameters (and the device); bounded, emptied when full.
+struct PairLaunch {
+  PairGemm a, b;
+  PairSched sch;
+  int grid;
+  bool grouped;   // false: a group whose table did not fit runs as two launches
+};
+
+struct LaunchKey {
+  uint64_t w[96];
+  int n = 0;
+  void add(uint64_t v) { w[n++] = v; }
+  void addp(const void* p) { add(static_cast<uint64_t>(reinterpret_cast<uintptr_t>(p))); }
+  void addf(float f) {
+    uint32_t u;
+    std::memcpy(&u, &f, 4);
+    add(u);
+  }
+  std::string str() const { return std::string(reinterpret_cast<const char*>(w), n * sizeof(uint64_t)); }
+};
+
+static_assert(sizeof(EpiParams) == 184 && sizeof(GemmDesc) == 72 && sizeof(DropoutParams) == 24,
+              "a field was added: the launch-cache key must list it");
+
+void key_drop(LaunchKey& k, const DropoutParams& d) {
+  k.add(d.seed);
+  k.add(d.offset);
+  k.add(d.thr);
+  k.addf(d.scale);
+}
+
+void key_gemm(LaunchKey& k, const GemmDesc& g, const EpiParams& e, int kind, int splits) {
+  k.add(kind); k.add(splits);
+  k.add(g.M); k.add(g.N); k.add(g.K);
+  k.addp(g.A); k.add(g.lda); k.add(g.a_kmajor);
+  k.addp(g.B); k.add(g.ldb); k.add(g.b_kmajor);
+  k.add(e.kind); k.addp(e.bias); k.addp(e.res); k.addp(e.aux); k.addp(e.out); k.addp(e.out2); k.add(e.ldo);
+  key_drop(k, e.drop);
+  k.add(e.site); k.addp(e.keep8);
+  k.add(e.seq); k.add(e.hidden); k.add(e.head_dim); k.add(e.heads); k.add(e.tokens); k.add(e.gelu_tanh);
+  k.addp(e.gen_keep); k.addp(e.gen_keep2); k.add(e.gen_site); k.add(e.gen_n8);
+  key_drop(k, e.gen_drop);
+  k.addp(e.colsum);
+}
+
+std::mutex g_launch_mu;
+std::unordered_map<std::string, PairLaunch>& launch_cache() {
+  static std::unordered_map<std::string, PairLaunch> m;
+  return m;
+}
+constexpr size_t kLaunchCacheMax = 4096;
+
+// The cached launch for `key`, built by `build` on a miss (nullptr if the
+// build fails).  Call with g_launch_mu held.
+template <typename Build>
+const PairLaunch* cached_launch(LaunchKey& key, Build build) {
+  int dev = 0;
+  cudaGetDevice(&dev);
+  key.add(dev);
+  auto& m = launch_cache();
+  const std::string ks = key.str();
+  auto it = m.find(ks);
+  if (it != m.end()) return &it->second;
+  PairLaunch pl;
+  if (!build(pl)) return nullptr;
+  if (m.size() >= kLaunchCacheMax) m.clear();
+  return &m.emplace(ks, pl).first->second;
+}
+
 template <typename T, int KIND>
 int launch_tc_pair(const GemmDesc& gd, const EpiParams& e, int splits, cudaStream_t s) {
-  PairGemm P;
-  PairSched sch;
-  if (!build_pair_gemm<T, KIND>(P, gd, e, splits)) return 1;
-  std::memset(&sch, 0, sizeof(sch));   // round-robin
-  const int total = P.g.tiles_m * P.g.tiles_n * P.g.splits;
-  launch_pair<T, KIND, KIND>(P, P, sch, 2 * std::min(total, num_sms() / 2), s);
+  LaunchKey key;
+  key.add(1);
+  key.add(std::is_same<T, bf16_t>::value);
+  key_gemm(key, gd, e, KIND, splits);
+  std::lock_guard<std::mutex> lk(g_launch_mu);
+  const PairLaunch* pl = cached_launch(key, [&](PairLaunch& L) {
+    if (!build_pair_gemm<T, KIND>(L.a, gd, e, splits)) return false;
+    std::memset(&L.sch, 0, sizeof(L.sch));   // round-robin
+    const int total = L.a.g.tiles_m * L.a.g.tiles_n * L.a.g.splits;
+    L.grid = 2 * std::min(total, num_sms() / 2);
+    L.grouped = false;
+    return true;
+  });
+  if (!pl) return 1;
+  launch_pair<T, KIND, KIND>(pl->a, pl->a, pl->sch, pl->grid, s);
   return 0;
 }
 
@@ -921,15 +1009,29 @@ int launch_tc_pair(const GemmDesc& gd, const EpiParams& e, int splits, cudaStrea
 template <typename T, int KA, int KB>
 int launch_tc_pair_group(const GemmDesc& ga, const EpiParams& ea, int splits_a, const GemmDesc& gb,
                          const EpiParams& eb, cudaStream_t s) {
-  PairGemm A, B;
-  PairSched sch;
-  if (!build_pair_gemm<T, KA>(A, ga, ea, splits_a) || !build_pair_gemm<T, KB>(B, gb, eb, 1)) return 1;
-  const int pairs = std::min(num_sms() / 2, kMaxPairs);
-  if (!plan_pair_table(sch, A.g, KA, B.g, KB, pairs)) {
+  LaunchKey key;
+  key.add(2);
+  key.add(std::is_same<T, bf16_t>::value);
+  key_gemm(key, ga, ea, KA, splits_a);
+  key_gemm(key, gb, eb, KB, 1);
+  bool grouped = false;
+  {
+    std::lock_guard<std::mutex> lk(g_launch_mu);
+    const PairLaunch* pl = cached_launch(key, [&](PairLaunch& L) {
+      if (!build_pair_gemm<T, KA>(L.a, ga, ea, splits_a) || !build_pair_gemm<T, KB>(L.b, gb, eb, 1)) return false;
+      const int pairs = std::min(num_sms() / 2, kMaxPairs);
+      L.grouped = plan_pair_table(L.sch, L.a.g, KA, L.b.g, KB, pairs);
+      L.grid = 2 * pairs;
+      return true;
+    });
+    if (!pl) return 1;
+    grouped = pl->grouped;
+    if (grouped) launch_pair<T, KA, KB>(pl->a, pl->b, pl->sch, pl->grid, s);
+  }
+  if (!grouped) {
     int rc = launch_tc_pair<T, KA>(ga, ea, splits_a, s);
     return rc ? rc : launch_tc_pair<T, KB>(gb, eb, 1, s);
   }
-  launch_pair<T, KA, KB>(A, B, sch, 2 * pairs, s);
   return 0;
 }
 
@@ -1078,6 +1180,30 @@ int gemm_tc_run2(int dtype, const GemmDesc& ga, const EpiParams& ea, const GemmD
 size_t gemm_tc_splitk_ws_floats(int M, int N, int K) {
   const int sp = splitk_count_pair(M, N, K);
   return sp > 1 ? (size_t)sp * ((M + 255) / 256) * 256 * N : 0;
+}
+
+// Sets the wait limit (ns, 0 = default) the GEMM kernels' waits read.
+void gemm_tc_set_wait_limit(uint64_t ns) {
+  cudaMemcpy(error_word() + 2, &ns, sizeof(ns), cudaMemcpyHostToDevice);
+}
+
+// One thread waits, with the library's bounded wait and the GEMM error word,
+// on an mbarrier that nothing ever arrives on: the wait runs out after the
+// limit and records code 99.  Nothing asynchronous is in flight meanwhile.
+__global__ void wait_probe_kernel(int* err) {
+  __shared__ __align__(8) uint64_t bar;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    fence_barrier_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) mbar_wait(&bar, 0, err, 99);
+  __syncthreads();
+}
+
+void gemm_tc_wait_probe(cudaStream_t s) {
+  wait_probe_kernel<<<1, 32, 0, s>>>(error_word());
+  count_launch();
 }
 
 // Reads and clears the bounded-wait error word of the tensor-core kernels.

@@ -109,6 +109,12 @@ int gemm_uses_tensor_cores(int dtype);
 size_t gemm_splitk_ws_floats(int dtype, int M, int N, int K);
 // Reads and clears the error word set by a bounded device-side wait that gave up.
 int device_take_error();
+// Sets the limit (ns; 0 = the default 2 s) of every kernel's bounded waits on
+// the current device.  Synchronous.
+void device_set_wait_limit(uint64_t ns);
+// Launches a kernel whose one bounded wait nothing ever satisfies (it gives
+// up after the limit and sets the error word of the GEMM kernels).
+void gemm_tc_wait_probe(cudaStream_t s);
 
 // ------------------------------------------------------------------ LayerNorm
 // LayerNorm forward.  With keep_out, also writes the dropout keep bits of
@@ -198,10 +204,11 @@ struct AttnArgs {
   DropoutParams drop;   // site 0
   void* ctx;            // (B*S, nh*d)
   float* lse;           // (B, nh, S); +inf marks a row with every key masked
-  // attention dropout keep bits of the S <= 128 tensor-core path, laid out
-  // [B*nh][128 query rows][16 bytes] (bit k of byte c = key 8c + k): the
-  // forward writes them, the backward reads them instead of drawing Philox
-  // again; null to draw them in both
+  // attention dropout keep bits of the tensor-core path (bit k of byte c =
+  // key 8c + k of a query row): the forward writes them, the backward reads
+  // them instead of drawing Philox again; null to draw them in both.  Laid
+  // out [B*nh][128 query rows][16 bytes] for S <= 128, else [B*nh][S][S/8]
+  // (byte e/8 for the flat element index e of site 0)
   uint8_t* keep;
   // backward
   const void* dctx;     // (B*S, nh*d)

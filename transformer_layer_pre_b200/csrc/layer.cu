@@ -44,8 +44,11 @@ struct tl_layer {
   uint64_t seed;
   tl_options opt;
   int device = -1;
-  char* arena = nullptr;
+  char* arena = nullptr;          // saved activations (forward -> backward)
   size_t arena_bytes = 0;
+  char* scratch = nullptr;        // scratch of one call: the layer's own, or the caller's
+  size_t scratch_bytes = 0;
+  bool scratch_owned = false;
   bool have_fwd = false;
   const float* mask = nullptr;
   std::string err;
@@ -62,7 +65,8 @@ struct tl_layer {
   size_t part_floats = 0;
   // hidden-dropout keep bits of sites 1 and 2 (one byte per 8 elements)
   uint8_t *keep1 = nullptr, *keep2 = nullptr;
-  // attention dropout keep bits (site 0), [B*nh][128][16] bytes, or null
+  // attention dropout keep bits (site 0), written by the forward for the
+  // backward: [B*nh][128][16] bytes for S <= 128, else [B*nh][S][S/8]; or null
   uint8_t* akeep = nullptr;
   // split-K scratch of the four weight gradients (W2, W1, Wo, Wqkv), each its
   // own, so every split sum can wait for the closing finalize launch
@@ -97,6 +101,16 @@ DropoutParams make_drop(const tl_layer* L, float p) {
   return d;
 }
 
+void free_scratch(tl_layer* L) {
+  if (L->scratch && L->scratch_owned) {
+    cudaDeviceSynchronize();
+    cudaFree(L->scratch);
+  }
+  L->scratch = nullptr;
+  L->scratch_bytes = 0;
+  L->scratch_owned = false;
+}
+
 void free_buffers(tl_layer* L) {
   if (L->arena) {
     cudaDeviceSynchronize();
@@ -104,6 +118,7 @@ void free_buffers(tl_layer* L) {
   }
   L->arena = nullptr;
   L->arena_bytes = 0;
+  free_scratch(L);
   L->have_fwd = false;
 }
 
@@ -118,7 +133,8 @@ struct Carver {
   }
 };
 
-// Lays out every buffer; with base == nullptr it only measures.
+// Lays out the buffers that live from a forward to its backward; with
+// base == nullptr it only measures.
 size_t carve(tl_layer* L, char* base) {
   Carver c(base);
   const size_t es = dtype_size(L->opt.dtype);
@@ -136,8 +152,7 @@ size_t carve(tl_layer* L, char* base) {
   // else GELU'(U), written by the FFN1 epilogue next to G so that the
   // backward's dU needs no special function
   L->u = c.take(TF * es);
-  L->big = c.take(TF * es);
-  L->g = ckpt ? L->big : c.take(TF * es);
+  if (!ckpt) L->g = c.take(TF * es);   // recompute mode: G lives in the scratch's `big` (carve_scratch)
   if (L->pre_ln) {
     L->h1 = c.take(TH * es);
     L->h2 = c.take(TH * es);
@@ -148,6 +163,26 @@ size_t carve(tl_layer* L, char* base) {
     L->res2 = L->opt.normalize_invertible ? nullptr : c.take(TH * es);
     L->yout = L->opt.normalize_invertible ? c.take(TH * es) : nullptr;
   }
+  L->keep1 = (uint8_t*)c.take((size_t)L->T * L->H / 8);
+  L->keep2 = (uint8_t*)c.take((size_t)L->T * L->H / 8);
+  // attention keep bits (site 0), one bit per element: [B*nh][128][16] bytes
+  // for S <= 128, the flat [B*nh][S][S/8] otherwise
+  const size_t akeep_bytes = L->S <= 128 ? (size_t)L->B * L->nh * 128 * 16 : (size_t)L->B * L->nh * L->S * (L->S / 8);
+  L->akeep = L->pa > 0.0f ? (uint8_t*)c.take(akeep_bytes) : nullptr;
+  return c.off;
+}
+
+// Lays out the scratch of one call (nothing in it outlives a forward or a
+// backward: layers that never run at the same time may share it); with
+// base == nullptr it only measures.
+size_t carve_scratch(tl_layer* L, char* base) {
+  Carver c(base);
+  const size_t es = dtype_size(L->opt.dtype);
+  const size_t TH = (size_t)L->T * L->H, TF = (size_t)L->T * L->F;
+  // (T, F): dU in backward; in recompute mode also G, from FFN1 to FFN2 in
+  // the forward and recomputed from U in the backward
+  L->big = c.take(TF * es);
+  if (L->opt.gelu_checkpoint) L->g = L->big;
   L->dz2 = c.take(TH * es);
   L->dh = c.take(TH * es);
   L->dx2 = c.take(TH * es);
@@ -156,9 +191,6 @@ size_t carve(tl_layer* L, char* base) {
   L->dres = c.take(TH * es);
   L->dqkv = c.take(3 * TH * es);
   L->dvec = (float*)c.take((size_t)L->B * L->nh * L->S * 4);
-  L->keep1 = (uint8_t*)c.take((size_t)L->T * L->H / 8);
-  L->keep2 = (uint8_t*)c.take((size_t)L->T * L->H / 8);
-  L->akeep = L->pa > 0.0f && L->S <= 128 ? (uint8_t*)c.take((size_t)L->B * L->nh * 128 * 16) : nullptr;
   const int np = std::max(std::max(std::max(ln_bwd_parts(L->T), rowdrop_parts(L->T)), colsum_parts(L->T)),
                           std::max((L->T + 255) / 256 * 8, L->B * 4));   // + partial rows of fused column sums
   const int maxc = std::max(3 * L->H, L->F);
@@ -174,23 +206,43 @@ size_t carve(tl_layer* L, char* base) {
   return c.off;
 }
 
+// Bytes of the scratch (measured on a copy: measuring lays out null pointers).
+size_t scratch_size(const tl_layer* L) {
+  tl_layer tmp = *L;
+  return carve_scratch(&tmp, nullptr);
+}
+
 tl_status ensure_buffers(tl_layer* L) {
-  if (L->arena) {
+  if (L->arena && L->scratch) {
     int dev = -1;
     cudaGetDevice(&dev);
     if (dev != L->device) return fail(L, TL_EINVAL, "layer used on a different device than it was allocated on");
     return TL_OK;
   }
-  const size_t bytes = carve(L, nullptr);
-  cudaGetDevice(&L->device);
-  void* p = nullptr;
-  if (cudaMalloc(&p, bytes) != cudaSuccess) {
-    cudaGetLastError();
-    return fail(L, TL_ENOMEM, "cudaMalloc of the layer workspace failed");
+  if (!L->arena) {
+    const size_t bytes = carve(L, nullptr);
+    cudaGetDevice(&L->device);
+    void* p = nullptr;
+    if (cudaMalloc(&p, bytes) != cudaSuccess) {
+      cudaGetLastError();
+      return fail(L, TL_ENOMEM, "cudaMalloc of the layer workspace failed");
+    }
+    L->arena = (char*)p;
+    L->arena_bytes = bytes;
+    carve(L, L->arena);
   }
-  L->arena = (char*)p;
-  L->arena_bytes = bytes;
-  carve(L, L->arena);
+  if (!L->scratch) {
+    const size_t bytes = carve_scratch(L, nullptr);
+    void* p = nullptr;
+    if (cudaMalloc(&p, bytes) != cudaSuccess) {
+      cudaGetLastError();
+      return fail(L, TL_ENOMEM, "cudaMalloc of the layer scratch failed");
+    }
+    L->scratch = (char*)p;
+    L->scratch_bytes = bytes;
+    L->scratch_owned = true;
+    carve_scratch(L, L->scratch);
+  }
   return TL_OK;
 }
 
@@ -331,10 +383,19 @@ tl_status layer_set_options(tl_layer* L, const tl_options* o) {
   if (!L || !o) return TL_EINVAL;
   if (o->dtype < TL_F32 || o->dtype > TL_BF16) return fail(L, TL_EINVAL, "unknown dtype");
   if (!(o->ln_eps > 0.0f)) return fail(L, TL_EINVAL, "ln_eps must be positive");
+  // shared scratch stays shared if it still fits the new options
+  char* shared = (L->scratch && !L->scratch_owned) ? L->scratch : nullptr;
+  const size_t shared_bytes = shared ? L->scratch_bytes : 0;
   free_buffers(L);
   L->opt = *o;
   L->opt.training = o->training ? 1 : 0;
   L->opt.gelu_tanh = o->gelu_tanh ? 1 : 0;
+  if (shared && shared_bytes >= scratch_size(L)) {
+    L->scratch = shared;
+    L->scratch_bytes = shared_bytes;
+    L->scratch_owned = false;
+    carve_scratch(L, L->scratch);
+  }
   return ensure_buffers(L);
 }
 
@@ -344,7 +405,26 @@ tl_status layer_get_options(const tl_layer* L, tl_options* o) {
   return TL_OK;
 }
 
-size_t layer_workspace_bytes(const tl_layer* L) { return L ? L->arena_bytes : 0; }
+size_t layer_workspace_bytes(const tl_layer* L) {
+  return L ? L->arena_bytes + (L->scratch_owned ? L->scratch_bytes : 0) : 0;
+}
+
+size_t layer_scratch_bytes(const tl_layer* L) { return L ? scratch_size(L) : 0; }
+
+tl_status layer_share_scratch(tl_layer* L, void* scratch, size_t bytes) {
+  if (!L) return TL_EINVAL;
+  L->err.clear();
+  if (!scratch) return fail(L, TL_EINVAL, "null scratch pointer");
+  if (reinterpret_cast<uintptr_t>(scratch) & 255) return fail(L, TL_EINVAL, "scratch must be 256-byte aligned");
+  const size_t need = scratch_size(L);
+  if (bytes < need) return fail(L, TL_EINVAL, "scratch smaller than layer_scratch_bytes");
+  free_scratch(L);
+  L->scratch = (char*)scratch;
+  L->scratch_bytes = bytes;
+  L->scratch_owned = false;
+  carve_scratch(L, L->scratch);
+  return TL_OK;
+}
 
 const char* layer_last_error(const tl_layer* L) { return L ? L->err.c_str() : "null layer"; }
 
@@ -586,6 +666,16 @@ tl_status tl_device_check(void) {
   cudaError_t e = cudaDeviceSynchronize();
   if (e != cudaSuccess) return TL_ECUDA;
   return device_take_error() ? TL_ETIMEOUT : TL_OK;
+}
+
+tl_status tl_set_wait_limit_ns(uint64_t ns) {
+  device_set_wait_limit(ns);
+  return cudaGetLastError() == cudaSuccess ? TL_OK : TL_ECUDA;
+}
+
+tl_status tl_wait_probe(void* stream) {
+  gemm_tc_wait_probe((cudaStream_t)stream);
+  return cudaPeekAtLastError() == cudaSuccess ? TL_OK : TL_ECUDA;
 }
 
 tl_status tl_gelu_eval(const float* u, float* g, float* dg, uint64_t n, void* stream) {

@@ -29,7 +29,8 @@ namespace {
 // registers and leave as one partial row per block.
 constexpr int kStages = 4;
 constexpr int kMaxBlocks = 296;        // 2 blocks per SM
-__device__ int g_row_err;              // set when a bounded wait gives up
+// error word of the row kernels' bounded waits (layout in sm100.cuh)
+__device__ __align__(16) int g_row_err[4];
 
 __host__ __device__ inline int row_threads(int H) { return ((H / 8 + 31) / 32) * 32; }
 
@@ -115,7 +116,7 @@ struct RowPipe {
   }
   // every thread: wait for group g; false if the wait gave up
   __device__ bool wait(int g) {
-    return sm100::mbar_wait(&full[g % kStages], (uint32_t)((g / kStages) & 1), &g_row_err, 1);
+    return sm100::mbar_wait(&full[g % kStages], (uint32_t)((g / kStages) & 1), g_row_err, 1);
   }
   __device__ const T* row(int g, int t, int r) const {
     return reinterpret_cast<const T*>(buf + (g % kStages) * stage_bytes() + t * tensor_bytes()) + (size_t)r * H;
@@ -142,7 +143,7 @@ size_t pipe_smem(int H) {
 // ------------------------------------------------------------------ LayerNorm forward
 // One warp per row, lane-interleaved chunks of 8 columns (16-byte vectors),
 // shuffle-only reductions, no shared memory and no block barrier: a warp
-// issues its row's loads first (streaming, not kept in L1) and gamma/beta
+// issues its rows' loads first (streaming, not kept in L1) and gamma/beta
 // through the read-only path (every warp reads the same H values, so they
 // stay cached).  NCH = chunks of 8 per lane (H <= 256*NCH).
 constexpr int kFwdWarps = 4;
@@ -175,7 +176,7 @@ template <> __device__ __forceinline__ void load8_ro<float>(const float* p, floa
   v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w; v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
 }
 
-template <typename T, int NCH>
+template <typename T, int NCH, int RPW>
 __global__ void __launch_bounds__(kFwdWarps * 32) ln_fwd_kernel(const T* __restrict__ x, const T* __restrict__ gamma,
                                                                 const T* __restrict__ beta, T* __restrict__ y,
                                                                 float* __restrict__ mean_out,
@@ -185,63 +186,77 @@ __global__ void __launch_bounds__(kFwdWarps * 32) ln_fwd_kernel(const T* __restr
   pdl_wait();
   pdl_launch_dependents();
   const int lane = threadIdx.x & 31;
-  const int row = blockIdx.x * kFwdWarps + (threadIdx.x >> 5);
-  if (row >= rows) return;
-  Raw8<T> raw[NCH];
+  // a warp owns RPW consecutive rows; every load of all of them is issued
+  // before the first row's arithmetic, so RPW rows' bytes are in flight
+  const int row0 = (blockIdx.x * kFwdWarps + (threadIdx.x >> 5)) * RPW;
+  if (row0 >= rows) return;
+  Raw8<T> raw[RPW][NCH];
 #pragma unroll
-  for (int c = 0; c < NCH; ++c) {
-    const int col = (lane + 32 * c) * 8;
-    raw[c] = col < H ? raw8_stream<T>(x + (size_t)row * H + col) : raw8_zero<T>();
-  }
-  if (keep_out) {
-    // dropout keep bits of this row for a downstream kernel (element index
-    // row*H + col), drawn while the row's loads are in flight
+  for (int q = 0; q < RPW; ++q) {
+    const int row = row0 + q;
 #pragma unroll
     for (int c = 0; c < NCH; ++c) {
       const int col = (lane + 32 * c) * 8;
-      if (col < H) {
-        const uint64_t e8 = ((uint64_t)row * H + col) >> 3;
-        keep_out[e8] = (uint8_t)dropout_bits8(dp, site, e8);
+      raw[q][c] = (row < rows && col < H) ? raw8_stream<T>(x + (size_t)row * H + col) : raw8_zero<T>();
+    }
+  }
+  if (keep_out) {
+    // dropout keep bits of these rows for a downstream kernel (element index
+    // row*H + col), drawn while the rows' loads are in flight
+#pragma unroll
+    for (int q = 0; q < RPW; ++q) {
+#pragma unroll
+      for (int c = 0; c < NCH; ++c) {
+        const int col = (lane + 32 * c) * 8;
+        if (row0 + q < rows && col < H) {
+          const uint64_t e8 = ((uint64_t)(row0 + q) * H + col) >> 3;
+          keep_out[e8] = (uint8_t)dropout_bits8(dp, site, e8);
+        }
       }
     }
   }
   const float inv_h = 1.0f / (float)H;
-  float v[NCH][8];
-  float s = 0.0f;
 #pragma unroll
-  for (int c = 0; c < NCH; ++c) {
-    raw8_unpack<T>(raw[c], v[c]);
+  for (int q = 0; q < RPW; ++q) {
+    const int row = row0 + q;
+    if (row >= rows) break;
+    float v[NCH][8];
+    float s = 0.0f;
 #pragma unroll
-    for (int i = 0; i < 8; ++i) s += v[c][i];
-  }
-  const float mean = warp_sum(s) * inv_h;
-  float ss = 0.0f;
+    for (int c = 0; c < NCH; ++c) {
+      raw8_unpack<T>(raw[q][c], v[c]);
 #pragma unroll
-  for (int c = 0; c < NCH; ++c) {
-    if ((lane + 32 * c) * 8 < H) {
+      for (int i = 0; i < 8; ++i) s += v[c][i];
+    }
+    const float mean = warp_sum(s) * inv_h;
+    float ss = 0.0f;
 #pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        const float d = v[c][i] - mean;
-        ss += d * d;
+    for (int c = 0; c < NCH; ++c) {
+      if ((lane + 32 * c) * 8 < H) {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const float d = v[c][i] - mean;
+          ss += d * d;
+        }
       }
     }
-  }
-  const float rstd = 1.0f / sqrtf(warp_sum(ss) * inv_h + eps);
+    const float rstd = 1.0f / sqrtf(warp_sum(ss) * inv_h + eps);
 #pragma unroll
-  for (int c = 0; c < NCH; ++c) {
-    const int col = (lane + 32 * c) * 8;
-    if (col < H) {
-      float g[8], b[8], o[8];
-      load8_ro<T>(gamma + col, g);
-      load8_ro<T>(beta + col, b);
+    for (int c = 0; c < NCH; ++c) {
+      const int col = (lane + 32 * c) * 8;
+      if (col < H) {
+        float g[8], b[8], o[8];
+        load8_ro<T>(gamma + col, g);
+        load8_ro<T>(beta + col, b);
 #pragma unroll
-      for (int i = 0; i < 8; ++i) o[i] = g[i] * ((v[c][i] - mean) * rstd) + b[i];
-      store8<T>(y + (size_t)row * H + col, o);
+        for (int i = 0; i < 8; ++i) o[i] = g[i] * ((v[c][i] - mean) * rstd) + b[i];
+        store8<T>(y + (size_t)row * H + col, o);
+      }
     }
-  }
-  if (lane == 0) {
-    mean_out[row] = mean;
-    rstd_out[row] = rstd;
+    if (lane == 0) {
+      mean_out[row] = mean;
+      rstd_out[row] = rstd;
+    }
   }
 }
 
@@ -803,9 +818,11 @@ int row_blocks(int rows) { return std::max(1, std::min(kMaxBlocks, (rows + 15) /
 template <typename T>
 void ln_fwd_t(const void* x, const void* g, const void* b, void* y, float* mean, float* rstd, int rows, int H,
               float eps, cudaStream_t s, uint8_t* keep_out, const DropoutParams& dp, int site) {
-  const int blocks = (rows + kFwdWarps - 1) / kFwdWarps;
   TLP_NCH_SWITCH(H, {
-    launch_pdl(ln_fwd_kernel<T, NCH>, blocks, kFwdWarps * 32, 0, s, static_cast<const T*>(x),
+    // two rows per warp up to 1024 16-bit columns (8 KB of loads in flight per warp)
+    constexpr int RPW = NCH * sizeof(T) <= 8 ? 2 : 1;
+    const int blocks = (rows + kFwdWarps * RPW - 1) / (kFwdWarps * RPW);
+    launch_pdl(ln_fwd_kernel<T, NCH, RPW>, blocks, kFwdWarps * 32, 0, s, static_cast<const T*>(x),
                static_cast<const T*>(g), static_cast<const T*>(b), static_cast<T*>(y), mean, rstd, rows, H, eps,
                keep_out, dp, site);
   });
@@ -884,6 +901,8 @@ int ln_bwd_run(int dt, const LnBwdArgs& a, cudaStream_t s) {
   if (dt == DT_F16) return ln_bwd_dispatch<half_t>(a, s);
   return ln_bwd_dispatch<bf16_t>(a, s);
 }
+
+void rowwise_set_wait_limit(uint64_t ns) { cudaMemcpyToSymbol(g_row_err, &ns, sizeof(ns), 2 * sizeof(int)); }
 
 int rowwise_take_error() {
   int v = 0, z = 0;

@@ -68,11 +68,22 @@ class GradExchanger:
     every submitted exchange.  Every rank must submit the same buffers in the
     same order (in a stack with layer dropping the decisions are equal on all
     ranks).  Without a process group of size > 1 both calls do nothing; CPU
-    tensors (gloo) are reduced synchronously."""
+    tensors (gloo) are reduced synchronously.
 
-    def __init__(self, group=None):
+    `allreduce` (with `world`) replaces the collective: a callable that sums
+    a tensor over `world` ranks in place, enqueued on the current stream (by
+    default torch.distributed's all_reduce over `group`)."""
+
+    def __init__(self, group=None, allreduce=None, world: int | None = None):
         self.group = group
-        self.world = (dist.get_world_size(group) if dist.is_available() and dist.is_initialized() else 1)
+        if allreduce is not None:
+            if world is None:
+                raise ValueError("a replacement collective needs the world size")
+            self.world = int(world)
+            self.allreduce = allreduce
+        else:
+            self.world = (dist.get_world_size(group) if dist.is_available() and dist.is_initialized() else 1)
+            self.allreduce = lambda t: dist.all_reduce(t, op=dist.ReduceOp.SUM, group=self.group)
         self.stream = None
         self.pending = 0
 
@@ -83,7 +94,7 @@ class GradExchanger:
             return
         t = grads.flat
         if t.device.type != "cuda":
-            dist.all_reduce(t, op=dist.ReduceOp.SUM, group=self.group)
+            self.allreduce(t)
             t.mul_(1.0 / self.world)
             return
         if self.stream is None:
@@ -92,7 +103,7 @@ class GradExchanger:
         ev.record(stream if stream is not None else torch.cuda.current_stream(t.device))
         self.stream.wait_event(ev)
         with torch.cuda.stream(self.stream):
-            dist.all_reduce(t, op=dist.ReduceOp.SUM, group=self.group)
+            self.allreduce(t)
             t.mul_(1.0 / self.world)
         self.pending += 1
 

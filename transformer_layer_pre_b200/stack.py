@@ -13,7 +13,10 @@ decisions come from the library (tl_pld_keep), equal on every rank that
 shares the seed and the step.  A skipped layer gets no gradients (None).
 
 Every layer's output and input gradient live in buffers of their own, so
-the inputs each layer's backward needs stay valid through the step.
+the inputs each layer's backward needs stay valid through the step.  The
+layers' per-call scratch (Step 3's memory concern: what lives only within
+one layer's forward or backward) is one buffer shared by all of them, since
+they run one at a time (share_scratch=False gives each its own).
 
 Data parallelism: with a process group of size > 1, `backward(...,
 exchange=True)` averages each layer's gradients over the ranks as soon as
@@ -43,8 +46,16 @@ class EncoderStack:
         self.device = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
         self.normalize_invertible = bool(options.get("normalize_invertible", False))
         self.pre_layer_norm = pre_layer_norm
+        share = bool(options.pop("share_scratch", True))
         self.layers = [Layer(batch, seq, hidden, heads, ffn, attn_dropout, hidden_dropout, pre_layer_norm, seed,
                              dtype=dtype, philox_offset=l, **options) for l in range(num_layers)]
+        # the layers run one at a time on one stream: one scratch serves them all
+        self.scratch = None
+        if share and num_layers > 1:
+            need = max(layer.scratch_bytes for layer in self.layers)
+            self.scratch = torch.empty(need, dtype=torch.uint8, device=self.device)
+            for layer in self.layers:
+                layer.share_scratch(self.scratch)
         self.ffn = self.layers[0].ffn
         self.grads = [FlatGrads(hidden, self.ffn, self.device) for _ in range(num_layers)]
         self.ys = [torch.empty(self.shape, dtype=dtype, device=self.device) for _ in range(num_layers)]
@@ -73,16 +84,17 @@ class EncoderStack:
                 h = layer.forward(h, mask, weights[l], y=self.ys[l], stream=stream)
         return h
 
-    def backward(self, dy: torch.Tensor, weights: list, exchange: bool = False, stream=None):
+    def backward(self, dy: torch.Tensor, weights: list, exchange=False, stream=None):
         """Backward of the last forward, layers in reverse.  Returns (dx,
         grads) with grads[l] a dict of float32 gradients (views of the stack's
         per-layer flat buffer, overwritten by the next backward) for a layer
         that ran and None for a skipped one.  With `exchange`, each layer's
         gradients are averaged over the data-parallel ranks (see the module
         docstring); they are final once the caller's stream reaches the end
-        of this call's work."""
+        of this call's work.  `exchange` may also be a GradExchanger to use
+        (e.g. one with its own collective)."""
         out = [None] * self.num_layers
-        ex = GradExchanger() if exchange else None
+        ex = exchange if isinstance(exchange, GradExchanger) else (GradExchanger() if exchange else None)
         g = dy
         for l in reversed(range(self.num_layers)):
             self.dys[l] = g
@@ -96,6 +108,12 @@ class EncoderStack:
         if ex is not None:
             ex.finish(stream)
         return g, out
+
+    @property
+    def workspace_bytes(self) -> int:
+        """Device bytes the stack's layers hold, the shared scratch included."""
+        shared = 0 if self.scratch is None else self.scratch.numel()
+        return sum(layer.workspace_bytes for layer in self.layers) + shared
 
     def close(self) -> None:
         for layer in self.layers:
