@@ -8,13 +8,16 @@
 // ("Transformer deployment", section 1 pseudo-code: softmax(Q K^T / sqrt(d_k))
 // then the product with V; "DeepSpeed Transformer Kernel usage guide", Step 3:
 // the attention-dropout input is not stored, backward regenerates it.)
-// Backward regenerates P from LSE and the dropout bits from Philox:
+// Backward regenerates P from LSE and reads the forward's dropout keep bits
+// (one bit per element, written by the forward next to its output):
 //   dV = Pd^T dO; dPd = dO V^T; dP = dPd * keep / (1 - p);
 //   dS = P * (dP - D) with D = rowsum(dO * O); dQ = dS K c; dK = dS^T Q c.
 //
 // Tiles are 128 queries x 128 keys.  One elected thread issues every MMA
-// (M = 128) into TMEM; softmax warps own one TMEM lane (one query row) each,
-// so each thread's dropout bits are its own row's Philox draws.  P and dS go
+// (M = 128) into TMEM; softmax warps own one TMEM lane (one query row) each;
+// helper warps draw the dropout bits of a row (forward) ahead of the softmax
+// warps, or stage the stored ones (backward).  Every kernel is persistent
+// (one CTA per SM walking work items).  P and dS go
 // back to shared memory in the 128-byte-swizzled layout TMA uses for a
 // [rows][64] tile, which serves as a K-major operand (rows x keys) and as an
 // MN-major operand (keys x rows) alike; Q, K, V and dO tiles likewise serve
@@ -59,6 +62,7 @@ struct AttnTc {
   float* colsum;        // fused QKV bias-gradient partials (persistent backward), or null
   int fuse_dq;
   int ctx_tma;          // persistent kernels: ctx (forward) or dQKV (backward) rows leave by TMA store (S % 32 == 0)
+  const int* kv_ext;    // per sequence, one past its last unmasked key (long forward), or null
   uint8_t* keep;        // attention keep bits (forward writes, backward reads) or null: persistent path
                         // [B*nh][128][16]; longer sequences flat, byte e/8 for element e of site 0
   int bf16;
@@ -89,384 +93,576 @@ __device__ __forceinline__ void pair_store8(uint8_t* pair, int r, int k8, const 
   store8<T>(reinterpret_cast<T*>(pair + region * 16384 + r * 128 + ((c ^ (r & 7)) << 4)), v);
 }
 
-__device__ __forceinline__ float mask_log2(const AttnTc& a, int b, int key) {
-  if (key >= a.S) return -INFINITY;
-  return a.mask ? a.mask[(size_t)b * a.S + key] * kLog2e : 0.0f;
+
+__device__ __forceinline__ float ex2_fast(float x) {
+  float r;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(x));
+  return r;
 }
-// The additive mask of keys key0 .. key0+7 (key0 % 8 == 0, S % 8 == 0), in
-// log2 units: two 16-byte loads that every lane of a warp shares.
-__device__ __forceinline__ void mask8_log2(const AttnTc& a, int b, int key0, float (&m)[8]) {
-  if (key0 >= a.S) {
-#pragma unroll
-    for (int t = 0; t < 8; ++t) m[t] = -INFINITY;
-  } else if (!a.mask) {
-#pragma unroll
-    for (int t = 0; t < 8; ++t) m[t] = 0.0f;
-  } else {
-    const float4* p = reinterpret_cast<const float4*>(a.mask + (size_t)b * a.S + key0);
-    const float4 u = __ldg(p), v = __ldg(p + 1);
-    m[0] = u.x * kLog2e; m[1] = u.y * kLog2e; m[2] = u.z * kLog2e; m[3] = u.w * kLog2e;
-    m[4] = v.x * kLog2e; m[5] = v.y * kLog2e; m[6] = v.z * kLog2e; m[7] = v.w * kLog2e;
-  }
+__device__ __forceinline__ float max3f(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+// Packed pairs of float32 (one instruction for both lanes on sm_100).
+__device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) {
+  unsigned long long d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;"
+      : "=l"(d)
+      : "l"(*reinterpret_cast<unsigned long long*>(&a)), "l"(*reinterpret_cast<unsigned long long*>(&b)),
+        "l"(*reinterpret_cast<unsigned long long*>(&c)));
+  return *reinterpret_cast<float2*>(&d);
+}
+__device__ __forceinline__ float2 add2(float2 a, float2 b) {
+  unsigned long long d;
+  asm("add.rn.f32x2 %0, %1, %2;"
+      : "=l"(d)
+      : "l"(*reinterpret_cast<unsigned long long*>(&a)), "l"(*reinterpret_cast<unsigned long long*>(&b)));
+  return *reinterpret_cast<float2*>(&d);
 }
 
-// One past the last key of sequence b whose additive mask is not -inf (S
-// without a mask), found by the whole block.  Key tiles at or beyond it hold
-// only masked keys: their probabilities are exactly 0 (2^-inf), so they add
-// nothing to any row sum, output or gradient, and the long-sequence kernels
-// skip them ("AI-infra engineers and the Transformer", section 2.1 Step 4:
-// dynamic padding keeps padded positions out of the work).  Call after
-// pdl_wait, from every thread of the block.
-__device__ __forceinline__ int key_extent(const AttnTc& a, int b) {
-  if (!a.mask) return a.S;
+// ============================================================================ backward
+// Softmax-side threads of the backward kernels: warps 2-9, two threads per
+// query row (TMEM lane), each 64 of the 128 key columns.
+constexpr int kSoftThreads = 256;
+
+// ============================================================================ forward, S > 128 (persistent)
+// One CTA per SM walks items (sequence b, head h, 128-query tile), each over
+// the key tiles up to the sequence's last unmasked key.  Warps: 0 TMA (Q of
+// the item, K/V tiles into a three-slot ring, running ahead across items),
+// 1 MMA, 2-5 softmax (thread = query row), 6-9 helpers (per key tile: the
+// dropout keep bits of the 128 x 128 elements, also written out for the
+// backward, and the key mask row, up to two tiles ahead).  The score
+// accumulator S and the probability tile P are double-buffered by the
+// running tile count g, so Q K^T of tile g+1 and the helpers' work overlap
+// the softmax of tile g; O accumulates in TMEM over the item's key tiles.
+// Online softmax with a lazy reference: P = 2^(x - m_ref) where m_ref is the
+// running row maximum at the last rescale; O and the row sum are rescaled
+// (in TMEM) only when the maximum has grown by more than 2^8 since then, so
+// P stays below 256 (exact in fp16/bf16 range) and most tiles skip the
+// rescale.  The result is the same softmax: every term carries the same
+// reference until the final normalisation.
+constexpr int kLThreads = 320;
+constexpr int kLKv = 3;                                     // K/V ring slots
+constexpr int kLAux = 128 * 16 + 128 * 4;                   // per slot: keep bits [128][16], mask [128]
+constexpr int kLSmem = 2 * TB + kLKv * 2 * TB + 4 * TB + 2 * kLAux + 1024 + 256;
+constexpr float kLRescale = 8.0f;                           // log2 units: P < 2^8
+
+// One past the last unmasked key of each sequence (kv_ext[b]), or S when the
+// mask leaves the last key valid; one block per sequence.
+__global__ void key_extent_kernel(const float* __restrict__ mask, int S, int* __restrict__ kv_ext) {
+  pdl_wait();
+  pdl_launch_dependents();
   __shared__ int ext;
   if (threadIdx.x == 0) ext = 0;
   __syncthreads();
+  const int b = blockIdx.x;
   int e = 0;
-  for (int j = threadIdx.x; j < a.S; j += blockDim.x)
-    if (a.mask[(size_t)b * a.S + j] != -INFINITY) e = j + 1;
+  for (int j = threadIdx.x; j < S; j += blockDim.x)
+    if (mask[(size_t)b * S + j] != -INFINITY) e = j + 1;
   if (e) atomicMax(&ext, e);
   __syncthreads();
-  return ext;
+  if (threadIdx.x == 0) kv_ext[b] = ext;
 }
 
-// ============================================================================ forward
-// Warps: 0 TMA, 1 MMA (+TMEM owner), 2-5 softmax (thread = query row).
-constexpr int kFwdThreads = 192;
-constexpr int kFwdSmem = 5 * TB + 1024 + 256;   // Q, K, V, P pair
+// Writes 32 x 32-bit registers to 32 consecutive TMEM columns of this warp's lanes.
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const float (&v)[32]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
+      "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
+      "r"(__float_as_uint(v[0])), "r"(__float_as_uint(v[1])), "r"(__float_as_uint(v[2])), "r"(__float_as_uint(v[3])),
+      "r"(__float_as_uint(v[4])), "r"(__float_as_uint(v[5])), "r"(__float_as_uint(v[6])), "r"(__float_as_uint(v[7])),
+      "r"(__float_as_uint(v[8])), "r"(__float_as_uint(v[9])), "r"(__float_as_uint(v[10])), "r"(__float_as_uint(v[11])),
+      "r"(__float_as_uint(v[12])), "r"(__float_as_uint(v[13])), "r"(__float_as_uint(v[14])), "r"(__float_as_uint(v[15])),
+      "r"(__float_as_uint(v[16])), "r"(__float_as_uint(v[17])), "r"(__float_as_uint(v[18])), "r"(__float_as_uint(v[19])),
+      "r"(__float_as_uint(v[20])), "r"(__float_as_uint(v[21])), "r"(__float_as_uint(v[22])), "r"(__float_as_uint(v[23])),
+      "r"(__float_as_uint(v[24])), "r"(__float_as_uint(v[25])), "r"(__float_as_uint(v[26])), "r"(__float_as_uint(v[27])),
+      "r"(__float_as_uint(v[28])), "r"(__float_as_uint(v[29])), "r"(__float_as_uint(v[30])), "r"(__float_as_uint(v[31]))
+      : "memory");
+}
+__device__ __forceinline__ void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
+// Key tiles item `it` runs over (at least one).
+__device__ __forceinline__ int long_item_tiles(const AttnTc& a, int b, int ntiles_all) {
+  if (!a.kv_ext) return ntiles_all;
+  return max(1, min(ntiles_all, (a.kv_ext[b] + TILE - 1) / TILE));
+}
 
 template <typename T>
-__global__ void __launch_bounds__(kFwdThreads)
-    attn_fwd_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
-                const __grid_constant__ CUtensorMap tv, AttnTc a) {
+__global__ void __launch_bounds__(kLThreads, 1)
+    attn_fwd_tc_long(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
+                     const __grid_constant__ CUtensorMap tv, const __grid_constant__ CUtensorMap tctx, AttnTc a) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = align1024(smem_raw);
-  uint8_t* sQ = sm;
-  uint8_t* sK = sm + TB;
-  uint8_t* sV = sm + 2 * TB;
-  uint8_t* sP = sm + 3 * TB;
-  uint64_t* bar = reinterpret_cast<uint64_t*>(sm + 5 * TB);
-  uint64_t *q_full = bar, *kv_full = bar + 1, *kv_empty = bar + 2, *s_full = bar + 3, *s_free = bar + 4,
-           *p_full = bar + 5, *o_full = bar + 6, *o_free = bar + 7;
-  uint32_t* tslot = reinterpret_cast<uint32_t*>(bar + 8);
+  uint8_t* sQ = sm;                                   // [2] Q tiles
+  uint8_t* sKV = sm + 2 * TB;                         // [kLKv] x (K, V)
+  uint8_t* sP = sKV + kLKv * 2 * TB;                  // [2] P pairs (also output staging)
+  uint8_t* saux = sP + 4 * TB;                        // [2] x (bits [128][16], mask [128])
+  uint64_t* bar = reinterpret_cast<uint64_t*>(saux + 2 * kLAux);
+  uint64_t *q_full = bar, *q_empty = bar + 2, *kv_full = bar + 4, *kv_empty = kv_full + kLKv;
+  uint64_t *s_full = kv_empty + kLKv, *s_free = s_full + 2, *p_full = s_free + 2, *pv_done = p_full + 2;
+  uint64_t *aux_full = pv_done + 2, *aux_free = aux_full + 2;
+  uint32_t* tslot = reinterpret_cast<uint32_t*>(aux_free + 2);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int h = blockIdx.y, b = blockIdx.z;
   const int S = a.S;
-  const int row0 = (b * a.nh + h) * S;
-  const int q0 = blockIdx.x * TILE;
-  const int ntiles_all = (S + TILE - 1) / TILE;
-
+  const int nq = (S + TILE - 1) / TILE;
+  const int nitems = a.B * a.nh * nq;
   if (threadIdx.x == 0) {
-    mbar_init(q_full, 1);
-    mbar_init(kv_full, 1);
-    mbar_init(kv_empty, 1);
-    mbar_init(s_full, 1);
-    mbar_init(s_free, 128);
-    mbar_init(p_full, 128);
-    mbar_init(o_full, 1);
-    mbar_init(o_free, 128);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&q_full[i], 1);
+      mbar_init(&q_empty[i], 1);
+      mbar_init(&s_full[i], 1);
+      mbar_init(&s_free[i], 128);
+      mbar_init(&p_full[i], 128);
+      mbar_init(&pv_done[i], 1);
+      mbar_init(&aux_full[i], 128);
+      mbar_init(&aux_free[i], 128);
+    }
+    for (int i = 0; i < kLKv; ++i) {
+      mbar_init(&kv_full[i], 1);
+      mbar_init(&kv_empty[i], 1);
+    }
     fence_barrier_init();
   }
-  if (warp == 1) tmem_alloc(tslot, 256);
+  if (warp == 1) tmem_alloc(tslot, 512);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  const uint32_t tmem = *tslot;
+  const uint32_t tmem = *tslot;   // S[0] at 0, S[1] at 128, O at 256
   pdl_wait();
   pdl_launch_dependents();
-  const uint32_t tS = tmem, tO = tmem + 128;
-  // key tiles past the last unmasked key are skipped (at least one is run,
-  // so a fully masked row still ends with its zero output)
-  const int ntiles = max(1, min(ntiles_all, (key_extent(a, b) + TILE - 1) / TILE));
 
   if (warp == 0) {
     if (lane == 0) {
+      uint32_t g = 0;
+      int n = 0;
       bool ok = true;
-      mbar_arrive_expect_tx(q_full, TB);
-      tma_load_2d(sQ, &tq, q_full, 0, row0 + q0);
-      int j = 0;
-      for (; j < ntiles; ++j) {
-        if (!mbar_wait(kv_empty, (j & 1) ^ 1, a.err, 11)) { ok = false; break; }
-        mbar_arrive_expect_tx(kv_full, 2 * TB);
-        tma_load_2d(sK, &tk, kv_full, 0, row0 + j * TILE);
-        tma_load_2d(sV, &tv, kv_full, 0, row0 + j * TILE);
+      for (int it = blockIdx.x; it < nitems && ok; it += gridDim.x, ++n) {
+        const int bh = it / nq, q0 = (it - bh * nq) * TILE;
+        const int nt = long_item_tiles(a, bh / a.nh, nq);
+        const int row0 = bh * S;
+        const int qs = n & 1;
+        if (!(ok = mbar_wait(&q_empty[qs], ((n >> 1) & 1) ^ 1, a.err, 81))) break;
+        mbar_arrive_expect_tx(&q_full[qs], TB);
+        tma_load_2d(sQ + qs * TB, &tq, &q_full[qs], 0, row0 + q0);
+        for (int j = 0; j < nt; ++j, ++g) {
+          const int ks = g % kLKv;
+          if (!(ok = mbar_wait(&kv_empty[ks], ((g / kLKv) & 1) ^ 1, a.err, 82))) break;
+          mbar_arrive_expect_tx(&kv_full[ks], 2 * TB);
+          tma_load_2d(sKV + ks * 2 * TB, &tk, &kv_full[ks], 0, row0 + j * TILE);
+          tma_load_2d(sKV + ks * 2 * TB + TB, &tv, &kv_full[ks], 0, row0 + j * TILE);
+        }
       }
+      // a wait that gave up: the loads already issued land before the CTA exits
       if (!ok) {
-        mbar_wait(q_full, 0, nullptr, 0);
-        if (j > 0) mbar_wait(kv_full, (j - 1) & 1, nullptr, 0);
+        for (int i = 0; i < 2; ++i) mbar_wait(&q_full[i], 0, nullptr, 0);
       }
     }
   } else if (warp == 1) {
     if (lane == 0) {
       const uint32_t id_s = idesc_f16(128, 128, a.bf16 != 0, false, false);
       const uint32_t id_o = idesc_f16(128, 64, a.bf16 != 0, false, true);
-      const uint32_t aQ = smem_u32(sQ), aK = smem_u32(sK), aV = smem_u32(sV), aP = smem_u32(sP);
-      if (mbar_wait(q_full, 0, a.err, 12)) {
-        for (int j = 0; j < ntiles; ++j) {
-          if (!mbar_wait(kv_full, j & 1, a.err, 13)) break;
-          if (!mbar_wait(s_free, (j & 1) ^ 1, a.err, 14)) break;
-          tc_fence_after();
+      uint32_t g = 0;
+      int n = 0;
+      bool ok = true;
+      // O += P(gp) V(gp); the first product of an item overwrites O
+      auto pv = [&](uint32_t gp, bool acc) -> bool {
+        const int ps = gp & 1, ks = gp % kLKv;
+        if (!mbar_wait(&p_full[ps], (gp >> 1) & 1, a.err, 83)) return false;
+        tc_fence_after();
+        const uint32_t aP = smem_u32(sP + ps * 2 * TB), aV = smem_u32(sKV + ks * 2 * TB + TB);
 #pragma unroll
-          for (int kk = 0; kk < HD / 16; ++kk) mma_f16(tS, dk_tile(aQ, kk), dk_tile(aK, kk), id_s, kk > 0);
-          mma_commit(s_full);
-          if (!mbar_wait(p_full, j & 1, a.err, 15)) break;
-          if (!mbar_wait(o_free, (j & 1) ^ 1, a.err, 16)) break;
+        for (int kk = 0; kk < TILE / 16; ++kk)
+          mma_f16(tmem + 256, dk_pair(aP, kk), dmn_tile(aV, kk), id_o, (acc || kk > 0) ? 1u : 0u);
+        mma_commit(&pv_done[ps]);
+        mma_commit(&kv_empty[ks]);
+        return true;
+      };
+      for (int it = blockIdx.x; it < nitems && ok; it += gridDim.x, ++n) {
+        const int bh = it / nq;
+        const int nt = long_item_tiles(a, bh / a.nh, nq);
+        const int qs = n & 1;
+        if (!(ok = mbar_wait(&q_full[qs], (n >> 1) & 1, a.err, 84))) break;
+        const uint32_t aQ = smem_u32(sQ + qs * TB);
+        for (int j = 0; j < nt; ++j, ++g) {
+          const int ks = g % kLKv, ss = g & 1;
+          if (!(ok = mbar_wait(&kv_full[ks], (g / kLKv) & 1, a.err, 85))) break;
+          if (!(ok = mbar_wait(&s_free[ss], ((g >> 1) & 1) ^ 1, a.err, 86))) break;
           tc_fence_after();
+          const uint32_t aK = smem_u32(sKV + ks * 2 * TB);
 #pragma unroll
-          for (int kk = 0; kk < TILE / 16; ++kk) mma_f16(tO, dk_pair(aP, kk), dmn_tile(aV, kk), id_o, kk > 0);
-          mma_commit(o_full);
-          mma_commit(kv_empty);
+          for (int kk = 0; kk < HD / 16; ++kk)
+            mma_f16(tmem + 128 * ss, dk_tile(aQ, kk), dk_tile(aK, kk), id_s, kk > 0);
+          mma_commit(&s_full[ss]);
+          if (j == nt - 1) mma_commit(&q_empty[qs]);
+          if (j > 0 && !(ok = pv(g - 1, j > 1))) break;
         }
+        if (ok) ok = pv(g - 1, nt > 1);
       }
     }
-  } else {
-    const int quarter = warp & 3;
-    const int r = quarter * 32 + lane;
-    const int i = q0 + r;
-    const uint32_t lo = (uint32_t)(quarter * 32) << 16;
-    const float c2 = a.scale * kLog2e;
-    const float dsc = a.drop.thr ? a.drop.scale : 1.0f;
-    const uint64_t erow = ((uint64_t)row0 + (uint64_t)i) * (uint64_t)S;
-    const bool row_ok = i < S;
-    float o[HD];
-#pragma unroll
-    for (int c = 0; c < HD; ++c) o[c] = 0.0f;
-    float m = -INFINITY, l = 0.0f, alpha_prev = 0.0f;
-    bool ok = true;
-    for (int j = 0; j < ntiles && ok; ++j) {
-      const int k0 = j * TILE;
-      if (!mbar_wait_warp(s_full, j & 1, a.err, 17)) { ok = false; break; }
-      tc_fence_after();
-      // pass 1: row maximum of the scaled, masked scores (log2 domain)
-      float mx = -INFINITY;
-#pragma unroll 1
-      for (int c = 0; c < 4; ++c) {
-        float sv[32];
-        tmem_ld32(tS + lo + c * 32, sv);
-#pragma unroll
-        for (int g = 0; g < 4; ++g) {
-          float ml[8];
-          mask8_log2(a, b, k0 + c * 32 + g * 8, ml);
-#pragma unroll
-          for (int t = 0; t < 8; ++t) mx = fmaxf(mx, fmaf(sv[g * 8 + t], c2, ml[t]));
-        }
-      }
-      const float m_new = fmaxf(m, mx);
-      const float alpha = (m == -INFINITY) ? 0.0f : exp2f(m - m_new);
-      // the P buffer and O_part of the previous tile must be consumed first
-      if (j > 0) {
-        if (!mbar_wait_warp(o_full, (j - 1) & 1, a.err, 18)) { ok = false; break; }
-        tc_fence_after();
-        float pv[32];
-        tmem_ld32(tO + lo, pv);
-#pragma unroll
-        for (int c = 0; c < 32; ++c) o[c] = fmaf(o[c], alpha_prev, pv[c]);
-        tmem_ld32(tO + lo + 32, pv);
-#pragma unroll
-        for (int c = 0; c < 32; ++c) o[32 + c] = fmaf(o[32 + c], alpha_prev, pv[c]);
-        tc_fence_before();
-        mbar_arrive(o_free);
-      }
-      // pass 2: probabilities, dropout, P to shared memory; the keep bits are
-      // also written out for the backward (byte e/8 of site 0, e the flat index)
-      float lsum = 0.0f;
-      const float msub = m_new == -INFINITY ? 0.0f : m_new;   // 2^(-inf - msub) = 0
-#pragma unroll 1
-      for (int c = 0; c < 4; ++c) {
-        float sv[32];
-        tmem_ld32(tS + lo + c * 32, sv);
-        uint32_t kw = 0xFFFFFFFFu;
+  } else if (warp >= 6) {
+    // helpers: keep bits and mask row of each key tile, two tiles ahead at most
+    const int r = threadIdx.x - 192;
+    uint32_t g = 0;
+    for (int it = blockIdx.x; it < nitems; it += gridDim.x) {
+      const int bh = it / nq, q0 = (it - bh * nq) * TILE;
+      const int b = bh / a.nh;
+      const int nt = long_item_tiles(a, b, nq);
+      const bool row_ok = q0 + r < S;
+      bool ok = true;
+      for (int j = 0; j < nt; ++j, ++g) {
+        const int as = g & 1;
+        if (!(ok = mbar_wait(&aux_free[as], ((g >> 1) & 1) ^ 1, a.err, 87))) break;
+        uint8_t* ax = saux + as * kLAux;
+        const int k0 = j * TILE;
         if (a.drop.thr) {
-          const uint64_t e8 = (erow + (uint64_t)(k0 + c * 32)) >> 3;
-          kw = 0;
+          const uint64_t e8 = (((uint64_t)bh * S + (uint64_t)(q0 + r)) * (uint64_t)S + (uint64_t)k0) >> 3;
+          uint32_t w[4];
 #pragma unroll
-          for (int g = 0; g < 4; ++g) kw |= dropout_bits8(a.drop, 0, e8 + g) << (8 * g);
+          for (int q = 0; q < 4; ++q) {
+            uint32_t v = 0;
+#pragma unroll
+            for (int gg = 0; gg < 4; ++gg) v |= dropout_bits8(a.drop, 0, e8 + (uint64_t)(q * 4 + gg)) << (8 * gg);
+            w[q] = v;
+          }
+          *reinterpret_cast<uint4*>(ax + r * 16) = make_uint4(w[0], w[1], w[2], w[3]);
           if (a.keep && row_ok) {
-            // a 32-bit word when it is 4-byte aligned (S % 32 == 0), else bytes
-            if ((e8 & 3) == 0) {
-              *reinterpret_cast<uint32_t*>(a.keep + e8) = kw;
+            // 16 bytes when they are 16-byte aligned (S % 128 == 0), else words or bytes
+            if ((e8 & 15) == 0) {
+              *reinterpret_cast<uint4*>(a.keep + e8) = make_uint4(w[0], w[1], w[2], w[3]);
+            } else if ((e8 & 3) == 0) {
+#pragma unroll
+              for (int q = 0; q < 4; ++q) reinterpret_cast<uint32_t*>(a.keep + e8)[q] = w[q];
             } else {
 #pragma unroll
-              for (int g = 0; g < 4; ++g) a.keep[e8 + g] = (uint8_t)(kw >> (8 * g));
+              for (int q = 0; q < 16; ++q) a.keep[e8 + q] = (uint8_t)(w[q >> 2] >> (8 * (q & 3)));
             }
           }
         }
-#pragma unroll
-        for (int g = 0; g < 4; ++g) {
-          const int kb = k0 + c * 32 + g * 8;
-          const uint32_t bits = (kw >> (8 * g)) & 0xFFu;
-          float ml[8];
-          mask8_log2(a, b, kb, ml);
-          float pv[8];
-#pragma unroll
-          for (int t = 0; t < 8; ++t) {
-            const float p = ex2_approx(fmaf(sv[g * 8 + t], c2, ml[t]) - msub);
-            lsum += p;
-            pv[t] = ((bits >> t) & 1u) ? p * dsc : 0.0f;
-          }
-          pair_store8<T>(sP, r, c * 4 + g, pv);
-        }
+        const int key = k0 + r;
+        reinterpret_cast<float*>(ax + 2048)[r] =
+            key < S ? (a.mask ? a.mask[(size_t)b * S + key] * kLog2e : 0.0f) : -INFINITY;
+        mbar_arrive(&aux_full[as]);
       }
-      tc_fence_before();
-      mbar_arrive(s_free);
-      fence_proxy_async_smem();
-      mbar_arrive(p_full);
-      l = l * alpha + lsum;
-      m = m_new;
-      alpha_prev = alpha;
+      if (!ok) break;
     }
-    if (ok && mbar_wait_warp(o_full, (ntiles - 1) & 1, a.err, 19)) {
+  } else {
+    // softmax: warp w owns TMEM lanes 32*(w%4), thread = query row
+    const int quarter = warp & 3;
+    const int r = quarter * 32 + lane;
+    const uint32_t lo = (uint32_t)(quarter * 32) << 16;
+    const float c2 = a.scale * kLog2e;
+    const float dsc = a.drop.thr ? a.drop.scale : 1.0f;
+    uint32_t g = 0;
+    bool ok = true;
+    for (int it = blockIdx.x; it < nitems && ok; it += gridDim.x) {
+      const int bh = it / nq, q0 = (it - bh * nq) * TILE;
+      const int b = bh / a.nh, h = bh - b * a.nh;
+      const int nt = long_item_tiles(a, b, nq);
+      const int i = q0 + r;
+      float mref = -INFINITY, l = 0.0f;
+      for (int j = 0; j < nt; ++j, ++g) {
+        const int ss = g & 1;
+        const uint8_t* ax = saux + ss * kLAux;
+        const float* mrow = reinterpret_cast<const float*>(ax + 2048);
+        if (!(ok = mbar_wait_warp(&aux_full[ss], (g >> 1) & 1, a.err, 88))) break;
+        const uint4 kb16 = a.drop.thr ? *reinterpret_cast<const uint4*>(ax + r * 16) : make_uint4(~0u, ~0u, ~0u, ~0u);
+        if (!(ok = mbar_wait_warp(&s_full[ss], (g >> 1) & 1, a.err, 89))) break;
+        tc_fence_after();
+        const uint32_t ts = tmem + 128 * ss + lo;
+        // pass 1: the tile's row maximum (scaled scores + mask, log2 units)
+        float mx = -INFINITY;
+#pragma unroll 1
+        for (int hh = 0; hh < 2; ++hh) {
+          float sv[64];
+          tmem_ld64(ts + hh * 64, sv);
+#pragma unroll
+          for (int t = 0; t < 64; t += 4) {
+            const float4 m4 = *reinterpret_cast<const float4*>(mrow + hh * 64 + t);
+            const float2 x0 = fma2(make_float2(sv[t], sv[t + 1]), make_float2(c2, c2), make_float2(m4.x, m4.y));
+            const float2 x1 = fma2(make_float2(sv[t + 2], sv[t + 3]), make_float2(c2, c2), make_float2(m4.z, m4.w));
+            mx = max3f(mx, max3f(x0.x, x0.y, x1.x), x1.y);
+          }
+        }
+        const float mnew = fmaxf(mref, mx);
+        if (j == 0) {
+          mref = mnew;   // the item's first product overwrites O
+        } else {
+          const bool need = mnew > mref + kLRescale;
+          if (__any_sync(0xffffffffu, need)) {
+            // O (and the row sum) to the new reference, once the previous product is in
+            if (!(ok = mbar_wait_warp(&pv_done[(g - 1) & 1], ((g - 1) >> 1) & 1, a.err, 90))) break;
+            tc_fence_after();
+            const float alpha = need ? ex2_approx(mref - mnew) : 1.0f;
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh) {
+              float o[32];
+              tmem_ld32(tmem + 256 + lo + hh * 32, o);
+#pragma unroll
+              for (int c = 0; c < 32; ++c) o[c] *= alpha;
+              tmem_st32(tmem + 256 + lo + hh * 32, o);
+            }
+            tmem_st_wait();
+            if (need) {
+              l *= alpha;
+              mref = mnew;
+            }
+          }
+        }
+        const float msub = mref == -INFINITY ? 0.0f : mref;   // 2^(-inf - msub) = 0
+        // the P slot is free once the product of tile g-2 is done
+        if (g >= 2 && !(ok = mbar_wait_warp(&pv_done[ss], ((g - 2) >> 1) & 1, a.err, 91))) break;
+        if (lane == 0) bulk_wait_read<0>();   // an earlier item's output staged in this slot has left
+        __syncwarp();
+        // pass 2: P = 2^(x - m_ref), dropped, into the P tile; row sum of the undropped P
+        float2 ls2 = make_float2(0.0f, 0.0f);
+#pragma unroll 1
+        for (int hh = 0; hh < 2; ++hh) {
+          float sv[64];
+          tmem_ld64(ts + hh * 64, sv);
+          const uint32_t bw0 = hh == 0 ? kb16.x : kb16.z, bw1 = hh == 0 ? kb16.y : kb16.w;
+#pragma unroll
+          for (int gg = 0; gg < 8; ++gg) {
+            const uint32_t bits = ((gg < 4 ? bw0 : bw1) >> (8 * (gg & 3))) & 0xFFu;
+            float pv[8];
+#pragma unroll
+            for (int t = 0; t < 8; t += 2) {
+              const float2 m2 = *reinterpret_cast<const float2*>(mrow + hh * 64 + gg * 8 + t);
+              const float2 x = add2(fma2(make_float2(sv[gg * 8 + t], sv[gg * 8 + t + 1]), make_float2(c2, c2), m2),
+                                    make_float2(-msub, -msub));
+              const float2 p = make_float2(ex2_approx(x.x), ex2_approx(x.y));
+              ls2 = add2(ls2, p);
+              pv[t] = ((bits >> t) & 1u) ? p.x : 0.0f;
+              pv[t + 1] = ((bits >> (t + 1)) & 1u) ? p.y : 0.0f;
+            }
+            pair_store8<T>(sP + ss * 2 * TB, r, hh * 8 + gg, pv);
+          }
+        }
+        l += ls2.x + ls2.y;
+        mbar_arrive(&aux_free[ss]);
+        tc_fence_before();
+        mbar_arrive(&s_free[ss]);
+        fence_proxy_async_smem();
+        mbar_arrive(&p_full[ss]);
+      }
+      if (!ok) break;
+      // the item's output once its last product is in
+      const uint32_t gl = g - 1;
+      if (!(ok = mbar_wait_warp(&pv_done[gl & 1], (gl >> 1) & 1, a.err, 92))) break;
       tc_fence_after();
-      float pv[32];
-      tmem_ld32(tO + lo, pv);
+      float o[64];
+      tmem_ld64(tmem + 256 + lo, o);
+      const float inv = l > 0.0f ? dsc / l : 0.0f;
+      if (i < S) a.lse[(size_t)bh * S + i] = l > 0.0f ? (mref + log2f(l)) * kLn2 : INFINITY;
+      if (a.ctx_tma) {
+        // whole 32-row boxes (S % 32 == 0), staged in this warp's rows of the last P slot
+        if (q0 + quarter * 32 < S) {
+          uint8_t* ostage = sP + (gl & 1) * 2 * TB + quarter * 4096;
 #pragma unroll
-      for (int c = 0; c < 32; ++c) o[c] = fmaf(o[c], alpha_prev, pv[c]);
-      tmem_ld32(tO + lo + 32, pv);
+          for (int c = 0; c < 8; ++c) {
+            float w8[8];
 #pragma unroll
-      for (int c = 0; c < 32; ++c) o[32 + c] = fmaf(o[32 + c], alpha_prev, pv[c]);
-      if (i < S) {
-        const float inv = l > 0.0f ? 1.0f / l : 0.0f;
+            for (int t = 0; t < 8; ++t) w8[t] = o[c * 8 + t] * inv;
+            store8<T>(reinterpret_cast<T*>(ostage + lane * 128 + ((c ^ (lane & 7)) << 4)), w8);
+          }
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            tma_store_2d(&tctx, ostage, h * HD, b * S + q0 + quarter * 32);
+            bulk_commit();
+          }
+        }
+      } else if (i < S) {
         T* dst = static_cast<T*>(a.ctx) + ((size_t)b * S + i) * a.H + h * HD;
 #pragma unroll
-        for (int c = 0; c < HD; c += 8) {
-          float v[8];
+        for (int c = 0; c < 64; c += 8) {
+          float w8[8];
 #pragma unroll
-          for (int t = 0; t < 8; ++t) v[t] = o[c + t] * inv;
-          store8<T>(dst + c, v);
+          for (int t = 0; t < 8; ++t) w8[t] = o[c + t] * inv;
+          store8<T>(dst + c, w8);
         }
-        a.lse[row0 + i] = l > 0.0f ? (m + log2f(l)) * kLn2 : INFINITY;
       }
     }
+    if (lane == 0) bulk_wait_all();
+    __syncwarp();
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (warp == 1) tmem_dealloc(tmem, 256);
+  if (warp == 1) tmem_dealloc(tmem, 512);
 }
 
-// ============================================================================ backward
-// Warps: 0 TMA, 1 MMA (+TMEM owner), 2-9 softmax: warp w serves TMEM lanes
-// 32*(w%4).. and key columns 64*((w-2)/4) .. +63 of each 128-key tile.
-constexpr int kBwdThreads = 320;
-constexpr int kSoftThreads = 256;
+// ============================================================================ backward, S > 128 (persistent)
+// Two persistent kernels.  attn_bwd_kv_long walks items (key tile, b, h): K
+// and V stay in shared memory while every query tile of the sequence passes
+// (Q, dO through a two-slot ring); per query tile S = Q K^T and dPd = dO V^T
+// go to TMEM, the softmax warps turn them into Pd and dS in shared memory,
+// and dV += Pd^T dO, dK += dS^T Q accumulate in TMEM.  attn_bwd_q_long walks
+// items (query tile, b, h) over the key tiles up to the sequence's last
+// unmasked key and accumulates dQ += dS K.  In both, the products of the next
+// tile are issued as soon as the softmax has read the current S and dPd, so
+// they run while the softmax finishes; keep bits come from the forward (no
+// Philox), the log-sum-exp, D = rowsum(dO O) and the key mask are staged by
+// helper warps one tile ahead.  Key tiles holding only masked keys get dK =
+// dV = 0 without any product (their probabilities are all exactly 0).
+constexpr int kBLThreads = 448;                              // 0 TMA, 1 MMA, 2-9 softmax, 10-13 helpers
+constexpr int kBLAux = 128 * 16 + 3 * 128 * 4;               // bits [128][16], mask, lse2, D [128]
+constexpr int kBLKvSmem = 4 * TB + 4 * TB + 4 * TB + 2 * kBLAux + 1024 + 256;   // K/V x2, Q/dO x2, Pd+dS pairs
+constexpr int kBLQSmem = 4 * TB + 4 * TB + 2 * TB + 2 * kBLAux + 1024 + 256;    // Q/dO x2, K/V x2, dS pair
 
-// Per-thread D_i = sum_c dO[i, c] O[i, c] (from global memory).
-template <typename T>
-__device__ __forceinline__ float dvec_row(const AttnTc& a, int b, int h, int i) {
-  const size_t off = ((size_t)b * a.S + i) * a.H + h * HD;
-  const T* dO = static_cast<const T*>(a.dctx) + off;
-  const T* O = static_cast<const T*>(a.ctx_in) + off;
-  float s = 0.0f;
-#pragma unroll
-  for (int c = 0; c < HD; c += 8) {
-    float x[8], y[8];
-    load8<T>(dO + c, x);
-    load8<T>(O + c, y);
-#pragma unroll
-    for (int t = 0; t < 8; ++t) s = fmaf(x[t], y[t], s);
-  }
-  return s;
-}
-
-// Softmax-side work of one (query tile, key tile) pair for one thread: row r
-// of the tile (query i), key columns [kc0, kc0 + 64) of the tile starting at
-// key k0.  Writes Pd (if sPd) and dS rows to shared memory.
-template <typename T>
-__device__ __forceinline__ void bwd_pair_rows(const AttnTc& a, int b, int row0, int i, int r, int k0, int kc0,
-                                              uint32_t tS, uint32_t tdP, uint32_t lo, float lse2, float Di,
-                                              uint8_t* sPd, uint8_t* sdS) {
-  const float c2 = a.scale * kLog2e;
-  const float dsc = a.drop.thr ? a.drop.scale : 1.0f;
-  const uint64_t erow = ((uint64_t)row0 + (uint64_t)i) * (uint64_t)a.S;
-  const bool row_ok = i < a.S;
-#pragma unroll 1
-  for (int c = 0; c < 2; ++c) {
-    float sv[32], dv[32];
-    tmem_ld32(tS + lo + kc0 + c * 32, sv);
-    tmem_ld32(tdP + lo + kc0 + c * 32, dv);
-    // the forward's keep bits of these 32 keys (one 32-bit word), or drawn again
-    uint32_t kw = 0xFFFFFFFFu;
-    if (a.drop.thr) {
-      const uint64_t e8 = (erow + (uint64_t)(k0 + kc0 + c * 32)) >> 3;
+// Helper-warp staging of one (query tile q0, key tile k0) pair of item bh:
+// lse2, D and the 16 keep-bit bytes of query row q0 + r, and the mask of key k0 + r.
+__device__ __forceinline__ void bl_stage_aux(const AttnTc& a, uint8_t* ax, int bh, int b, int q0, int k0, int r) {
+  const int S = a.S;
+  float* smask = reinterpret_cast<float*>(ax + 2048);
+  const int q = q0 + r;
+  const bool qv = q < S;
+  uint4 kb = make_uint4(~0u, ~0u, ~0u, ~0u);
+  if (a.drop.thr) {
+    if (!qv) {
+      kb = make_uint4(0u, 0u, 0u, 0u);
+    } else {
+      const uint64_t e8 = (((uint64_t)bh * S + (uint64_t)q) * (uint64_t)S + (uint64_t)k0) >> 3;
       if (a.keep) {
-        if (!row_ok) {
-          kw = 0u;
-        } else if ((e8 & 3) == 0) {
-          kw = __ldg(reinterpret_cast<const uint32_t*>(a.keep + e8));
+        if ((e8 & 15) == 0) {
+          kb = __ldg(reinterpret_cast<const uint4*>(a.keep + e8));
         } else {
-          kw = 0u;
+          uint32_t w[4] = {0u, 0u, 0u, 0u};
 #pragma unroll
-          for (int g = 0; g < 4; ++g) kw |= (uint32_t)__ldg(a.keep + e8 + g) << (8 * g);
+          for (int t = 0; t < 16; ++t) w[t >> 2] |= (uint32_t)__ldg(a.keep + e8 + t) << (8 * (t & 3));
+          kb = make_uint4(w[0], w[1], w[2], w[3]);
         }
       } else {
-        kw = 0;
+        uint32_t w[4];
 #pragma unroll
-        for (int g = 0; g < 4; ++g) kw |= dropout_bits8(a.drop, 0, e8 + g) << (8 * g);
+        for (int qq = 0; qq < 4; ++qq) {
+          uint32_t v = 0;
+#pragma unroll
+          for (int gg = 0; gg < 4; ++gg) v |= dropout_bits8(a.drop, 0, e8 + (uint64_t)(qq * 4 + gg)) << (8 * gg);
+          w[qq] = v;
+        }
+        kb = make_uint4(w[0], w[1], w[2], w[3]);
       }
-    }
-#pragma unroll
-    for (int g = 0; g < 4; ++g) {
-      const int kt = kc0 + c * 32 + g * 8;   // column within the key tile
-      const int kb = k0 + kt;
-      const uint32_t bits = (kw >> (8 * g)) & 0xFFu;
-      float ml[8];
-      mask8_log2(a, b, kb, ml);
-      float pd[8], ds[8];
-#pragma unroll
-      for (int t = 0; t < 8; ++t) {
-        // lse2 = +inf for rows past the sequence end: 2^-inf = 0
-        const float p = ex2_approx(fmaf(sv[g * 8 + t], c2, ml[t]) - lse2);
-        const bool keep = (bits >> t) & 1u;
-        pd[t] = keep ? p * dsc : 0.0f;
-        const float dp = keep ? dv[g * 8 + t] * dsc : 0.0f;
-        ds[t] = p * (dp - Di);
-      }
-      if (sPd) pair_store8<T>(sPd, r, kt >> 3, pd);
-      pair_store8<T>(sdS, r, kt >> 3, ds);
     }
   }
+  *reinterpret_cast<uint4*>(ax + r * 16) = kb;
+  const int key = k0 + r;
+  smask[r] = key < S ? (a.mask ? a.mask[(size_t)b * S + key] * kLog2e : 0.0f) : -INFINITY;
+  smask[128 + r] = qv ? a.lse[(size_t)bh * S + q] * kLog2e : INFINITY;
+  smask[256 + r] = qv ? a.dvec[(size_t)bh * S + q] : 0.0f;
 }
 
-// Key-tile CTA: dK, dV of 128 keys accumulated over every query tile; with
-// fuse_dq (one key tile covers the sequence) also dQ of each query tile.
-constexpr int kBwdKvSmem = 8 * TB + 1024 + 256;   // K, V, Q[2], dO... see layout below
+// Softmax-side work of one (query tile, key tile) pair for one thread: query
+// row r, key columns [kc0, kc0 + 64).  Reads S and dPd from TMEM (then
+// releases them on s_free), waits until the previous pair's products have
+// read the shared tiles (ds_free), writes Pd (when sPd) and dS.
+template <typename T>
+__device__ __forceinline__ bool bl_softmax_pair(const AttnTc& a, const uint8_t* ax, int r, int kc0, uint32_t tS,
+                                                uint32_t tdP, uint32_t lo, uint64_t* s_free, uint64_t* ds_free,
+                                                uint32_t ds_parity, uint8_t* sPd, uint8_t* sdS) {
+  const float c2 = a.scale * kLog2e;
+  const float dsc = a.drop.thr ? a.drop.scale : 1.0f;
+  const float* smask = reinterpret_cast<const float*>(ax + 2048);
+  const float lse2 = smask[128 + r], Di = smask[256 + r];
+  const uint2 kb8 = *reinterpret_cast<const uint2*>(ax + r * 16 + (kc0 >> 3));
+  // first 32 columns: computed while the previous pair's products may still
+  // read the shared tiles, held packed; the shared tiles are written once
+  // those products are done (ds_free); the second 32 columns go straight there
+  uint4 pdp[4], dsp[4];
+  auto compute = [&](int c, const float (&sv)[32], const float (&dv)[32], int g, float (&pd)[8], float (&ds)[8]) {
+    const uint32_t bits = ((c == 0 ? kb8.x : kb8.y) >> (8 * g)) & 0xFFu;
+    const int kt = kc0 + c * 32 + g * 8;
+    const float4 m0 = *reinterpret_cast<const float4*>(smask + kt);
+    const float4 m1 = *reinterpret_cast<const float4*>(smask + kt + 4);
+    const float ml[8] = {m0.x - lse2, m0.y - lse2, m0.z - lse2, m0.w - lse2,
+                         m1.x - lse2, m1.y - lse2, m1.z - lse2, m1.w - lse2};
+#pragma unroll
+    for (int t = 0; t < 8; ++t) {
+      // lse2 = +inf for query rows past the sequence end: p = 0
+      const float p = ex2_approx(fmaf(sv[g * 8 + t], c2, ml[t]));
+      const bool keep = (bits >> t) & 1u;
+      pd[t] = keep ? p * dsc : 0.0f;
+      const float dp = keep ? dv[g * 8 + t] * dsc : 0.0f;
+      ds[t] = p * (dp - Di);
+    }
+  };
+  auto put = [&](int k8, const uint4& pdv, const uint4& dsv) {
+    const int region = k8 >> 3, cc = k8 & 7;
+    if (sPd) *reinterpret_cast<uint4*>(sPd + region * 16384 + r * 128 + ((cc ^ (r & 7)) << 4)) = pdv;
+    *reinterpret_cast<uint4*>(sdS + region * 16384 + r * 128 + ((cc ^ (r & 7)) << 4)) = dsv;
+  };
+  {
+    float sv[32], dv[32];
+    tmem_ld32x2(tS + lo + kc0, sv, tdP + lo + kc0, dv);
+#pragma unroll
+    for (int g = 0; g < 4; ++g) {
+      float pd[8], ds[8];
+      compute(0, sv, dv, g, pd, ds);
+      pdp[g] = pack8<T>(pd);
+      dsp[g] = pack8<T>(ds);
+    }
+  }
+  if (!mbar_wait_warp(ds_free, ds_parity, a.err, 95)) return false;
+#pragma unroll
+  for (int g = 0; g < 4; ++g) put((kc0 >> 3) + g, pdp[g], dsp[g]);
+  {
+    float sv[32], dv[32];
+    tmem_ld32x2(tS + lo + kc0 + 32, sv, tdP + lo + kc0 + 32, dv);
+    // every TMEM read of this pair is done: S and dPd may be overwritten
+    tc_fence_before();
+    mbar_arrive(s_free);
+#pragma unroll
+    for (int g = 0; g < 4; ++g) {
+      float pd[8], ds[8];
+      compute(1, sv, dv, g, pd, ds);
+      put((kc0 >> 3) + 4 + g, pack8<T>(pd), pack8<T>(ds));
+    }
+  }
+  return true;
+}
+
+__device__ __forceinline__ int bl_key_tiles(const AttnTc& a, int b, int nk) {
+  if (!a.kv_ext) return nk;
+  return max(1, min(nk, (a.kv_ext[b] + TILE - 1) / TILE));
+}
 
 template <typename T>
-__global__ void __launch_bounds__(kBwdThreads)
-    attn_bwd_kv_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
-                   const __grid_constant__ CUtensorMap tv, const __grid_constant__ CUtensorMap tdo, AttnTc a) {
+__global__ void __launch_bounds__(kBLThreads, 1)
+    attn_bwd_kv_long(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
+                     const __grid_constant__ CUtensorMap tv, const __grid_constant__ CUtensorMap tdo, AttnTc a) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = align1024(smem_raw);
-  uint8_t* sK = sm;
-  uint8_t* sV = sm + TB;
-  uint8_t* sQ = sm + 2 * TB;    // one stage: Q then dO
-  uint8_t* sdO = sm + 3 * TB;
-  uint8_t* sPd = sm + 4 * TB;   // pair
-  uint8_t* sdS = sm + 6 * TB;   // pair
-  uint64_t* bar = reinterpret_cast<uint64_t*>(sm + 8 * TB);
-  uint64_t *kv_full = bar, *qd_full = bar + 1, *qd_empty = bar + 2, *s_full = bar + 3, *s_free = bar + 4,
-           *ds_full = bar + 5, *ds_free = bar + 6, *dq_full = bar + 7, *dq_free = bar + 8, *acc_full = bar + 9;
-  uint32_t* tslot = reinterpret_cast<uint32_t*>(bar + 10);
+  uint8_t* sKV = sm;                      // [2] x (K, V)
+  uint8_t* sQD = sm + 4 * TB;             // [2] x (Q, dO)
+  uint8_t* sPd = sm + 8 * TB;             // pair
+  uint8_t* sdS = sm + 10 * TB;            // pair
+  uint8_t* saux = sm + 12 * TB;           // [2]
+  uint64_t* bar = reinterpret_cast<uint64_t*>(saux + 2 * kBLAux);
+  uint64_t *kv_full = bar, *kv_empty = bar + 2, *qd_full = bar + 4, *qd_empty = bar + 6, *aux_full = bar + 8,
+           *aux_free = bar + 10, *s_full = bar + 12, *s_free = bar + 13, *ds_full = bar + 14, *ds_free = bar + 15,
+           *acc_full = bar + 16, *acc_free = bar + 17;
+  uint32_t* tslot = reinterpret_cast<uint32_t*>(bar + 18);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int h = blockIdx.y, b = blockIdx.z;
   const int S = a.S;
-  const int row0 = (b * a.nh + h) * S;
-  const int k0 = blockIdx.x * TILE;
-  const int nq_all = (S + TILE - 1) / TILE;
-
+  const int nk = (S + TILE - 1) / TILE, nq = nk;
+  const int nitems = a.B * a.nh * nk;
   if (threadIdx.x == 0) {
-    mbar_init(kv_full, 1);
-    mbar_init(qd_full, 1);
-    mbar_init(qd_empty, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&kv_full[i], 1);
+      mbar_init(&kv_empty[i], 1);
+      mbar_init(&qd_full[i], 1);
+      mbar_init(&qd_empty[i], 1);
+      mbar_init(&aux_full[i], 128);
+      mbar_init(&aux_free[i], kSoftThreads);
+    }
     mbar_init(s_full, 1);
     mbar_init(s_free, kSoftThreads);
     mbar_init(ds_full, kSoftThreads);
     mbar_init(ds_free, 1);
-    mbar_init(dq_full, 1);
-    mbar_init(dq_free, kSoftThreads);
     mbar_init(acc_full, 1);
+    mbar_init(acc_free, kSoftThreads);
     fence_barrier_init();
   }
   if (warp == 1) tmem_alloc(tslot, 512);
@@ -476,44 +672,31 @@ __global__ void __launch_bounds__(kBwdThreads)
   const uint32_t tmem = *tslot;
   pdl_wait();
   pdl_launch_dependents();
-  const uint32_t tS = tmem, tdP = tmem + 128, tdV = tmem + 256, tdK = tmem + 320, tdQ = tmem + 384;
-  // every key of this tile masked: no query attends to them, dK = dV = 0
-  // exactly (this CTA runs no product; dQ never comes from here then, since
-  // fuse_dq needs one key tile that covers the sequence)
-  const bool keys_masked = !a.fuse_dq && k0 >= key_extent(a, b);
-  const int nq = keys_masked ? 0 : nq_all;
-  if (keys_masked && warp >= 2) {
-    const int sw = warp - 2, quarter = warp & 3, half = sw >> 2;
-    const int key = k0 + quarter * 32 + lane;
-    if (key < S) {
-      T* dst = static_cast<T*>(a.dqkv) + ((size_t)b * S + key) * 3 * a.H + h * HD + half * 32;
-      const float z[8] = {0, 0, 0, 0, 0, 0, 0, 0};
-#pragma unroll
-      for (int c = 0; c < 32; c += 8) {
-        store8<T>(dst + a.H + c, z);
-        store8<T>(dst + 2 * a.H + c, z);
-      }
-    }
-  }
+  const uint32_t tS = tmem, tdP = tmem + 128, tdV = tmem + 256, tdK = tmem + 320;
+  // an item (key tile j of sequence b, head h) whose keys are all masked
+  auto masked = [&](int b, int j) { return j >= bl_key_tiles(a, b, nk) || (a.kv_ext && j * TILE >= a.kv_ext[b]); };
 
-  if (keys_masked) {
-    // nothing is loaded or multiplied
-  } else if (warp == 0) {
+  if (warp == 0) {
     if (lane == 0) {
+      int n = 0;
+      uint32_t g = 0;
       bool ok = true;
-      mbar_arrive_expect_tx(kv_full, 2 * TB);
-      tma_load_2d(sK, &tk, kv_full, 0, row0 + k0);
-      tma_load_2d(sV, &tv, kv_full, 0, row0 + k0);
-      int i = 0;
-      for (; i < nq; ++i) {
-        if (!mbar_wait(qd_empty, (i & 1) ^ 1, a.err, 21)) { ok = false; break; }
-        mbar_arrive_expect_tx(qd_full, 2 * TB);
-        tma_load_2d(sQ, &tq, qd_full, 0, row0 + i * TILE);
-        tma_load_2d(sdO, &tdo, qd_full, h * HD, b * S + i * TILE);
-      }
-      if (!ok) {
-        mbar_wait(kv_full, 0, nullptr, 0);
-        if (i > 0) mbar_wait(qd_full, (i - 1) & 1, nullptr, 0);
+      for (int it = blockIdx.x; it < nitems && ok; it += gridDim.x) {
+        const int bh = it / nk, j = it - bh * nk, b = bh / a.nh, h = bh - b * a.nh;
+        if (masked(b, j)) continue;
+        const int ks = n & 1;
+        if (!(ok = mbar_wait(&kv_empty[ks], ((n >> 1) & 1) ^ 1, a.err, 101))) break;
+        mbar_arrive_expect_tx(&kv_full[ks], 2 * TB);
+        tma_load_2d(sKV + ks * 2 * TB, &tk, &kv_full[ks], 0, bh * S + j * TILE);
+        tma_load_2d(sKV + ks * 2 * TB + TB, &tv, &kv_full[ks], 0, bh * S + j * TILE);
+        for (int i = 0; i < nq; ++i, ++g) {
+          const int qs = g & 1;
+          if (!(ok = mbar_wait(&qd_empty[qs], ((g >> 1) & 1) ^ 1, a.err, 102))) break;
+          mbar_arrive_expect_tx(&qd_full[qs], 2 * TB);
+          tma_load_2d(sQD + qs * 2 * TB, &tq, &qd_full[qs], 0, bh * S + i * TILE);
+          tma_load_2d(sQD + qs * 2 * TB + TB, &tdo, &qd_full[qs], h * HD, b * S + i * TILE);
+        }
+        ++n;
       }
     }
   } else if (warp == 1) {
@@ -521,88 +704,111 @@ __global__ void __launch_bounds__(kBwdThreads)
       const bool bf = a.bf16 != 0;
       const uint32_t id_kk = idesc_f16(128, 128, bf, false, false);
       const uint32_t id_mm = idesc_f16(128, 64, bf, true, true);
-      const uint32_t id_km = idesc_f16(128, 64, bf, false, true);
-      const uint32_t aK = smem_u32(sK), aV = smem_u32(sV), aQ = smem_u32(sQ), adO = smem_u32(sdO);
       const uint32_t aPd = smem_u32(sPd), adS = smem_u32(sdS);
-      bool ok = mbar_wait(kv_full, 0, a.err, 22);
-      for (int i = 0; i < nq && ok; ++i) {
-        if (!(ok = mbar_wait(qd_full, i & 1, a.err, 23))) break;
-        if (!(ok = mbar_wait(s_free, (i & 1) ^ 1, a.err, 24))) break;
+      int n = 0;
+      uint32_t g = 0;
+      bool ok = true;
+      // dV += Pd^T dO, dK += dS^T Q of pair gp; the first pair of an item overwrites
+      auto dvdk = [&](uint32_t gp, bool acc, int nn) -> bool {
+        if (!acc && !mbar_wait(acc_free, (nn & 1) ^ 1, a.err, 103)) return false;
+        if (!mbar_wait(ds_full, gp & 1, a.err, 104)) return false;
         tc_fence_after();
-#pragma unroll
-        for (int kk = 0; kk < HD / 16; ++kk) mma_f16(tS, dk_tile(aQ, kk), dk_tile(aK, kk), id_kk, kk > 0);
-#pragma unroll
-        for (int kk = 0; kk < HD / 16; ++kk) mma_f16(tdP, dk_tile(adO, kk), dk_tile(aV, kk), id_kk, kk > 0);
-        mma_commit(s_full);
-        if (!(ok = mbar_wait(ds_full, i & 1, a.err, 25))) break;
-        tc_fence_after();
-        // dV += Pd^T dO ; dK += dS^T Q   (K runs over the 128 queries)
+        const uint32_t aQ = smem_u32(sQD + (gp & 1) * 2 * TB), adO = aQ + TB;
 #pragma unroll
         for (int kk = 0; kk < TILE / 16; ++kk)
-          mma_f16(tdV, dmn_pair(aPd, kk), dmn_tile(adO, kk), id_mm, (i > 0 || kk > 0) ? 1u : 0u);
+          mma_f16(tdV, dmn_pair(aPd, kk), dmn_tile(adO, kk), id_mm, (acc || kk > 0) ? 1u : 0u);
 #pragma unroll
         for (int kk = 0; kk < TILE / 16; ++kk)
-          mma_f16(tdK, dmn_pair(adS, kk), dmn_tile(aQ, kk), id_mm, (i > 0 || kk > 0) ? 1u : 0u);
-        if (a.fuse_dq) {
-          if (!(ok = mbar_wait(dq_free, (i & 1) ^ 1, a.err, 26))) break;
-          tc_fence_after();
-          // dQ = dS K   (K runs over the 128 keys)
-#pragma unroll
-          for (int kk = 0; kk < TILE / 16; ++kk) mma_f16(tdQ, dk_pair(adS, kk), dmn_tile(aK, kk), id_km, kk > 0);
-          mma_commit(dq_full);
-        }
+          mma_f16(tdK, dmn_pair(adS, kk), dmn_tile(aQ, kk), id_mm, (acc || kk > 0) ? 1u : 0u);
         mma_commit(ds_free);
-        mma_commit(qd_empty);
+        mma_commit(&qd_empty[gp & 1]);
+        return true;
+      };
+      for (int it = blockIdx.x; it < nitems && ok; it += gridDim.x) {
+        const int bh = it / nk, j = it - bh * nk, b = bh / a.nh;
+        if (masked(b, j)) continue;
+        const int ks = n & 1;
+        if (!(ok = mbar_wait(&kv_full[ks], (n >> 1) & 1, a.err, 105))) break;
+        const uint32_t aK = smem_u32(sKV + ks * 2 * TB), aV = aK + TB;
+        for (int i = 0; i < nq; ++i, ++g) {
+          const int qs = g & 1;
+          if (!(ok = mbar_wait(&qd_full[qs], (g >> 1) & 1, a.err, 106))) break;
+          if (!(ok = mbar_wait(s_free, (g & 1) ^ 1, a.err, 107))) break;
+          tc_fence_after();
+          const uint32_t aQ = smem_u32(sQD + qs * 2 * TB), adO = aQ + TB;
+#pragma unroll
+          for (int kk = 0; kk < HD / 16; ++kk) mma_f16(tS, dk_tile(aQ, kk), dk_tile(aK, kk), id_kk, kk > 0);
+#pragma unroll
+          for (int kk = 0; kk < HD / 16; ++kk) mma_f16(tdP, dk_tile(adO, kk), dk_tile(aV, kk), id_kk, kk > 0);
+          mma_commit(s_full);
+          if (i > 0 && !(ok = dvdk(g - 1, i > 1, n))) break;
+        }
+        if (ok) ok = dvdk(g - 1, nq > 1, n);
+        if (!ok) break;
+        mma_commit(acc_full);
+        mma_commit(&kv_empty[ks]);
+        ++n;
       }
-      if (ok) mma_commit(acc_full);
+    }
+  } else if (warp >= 10) {
+    const int r = threadIdx.x - 320;
+    uint32_t g = 0;
+    bool ok = true;
+    for (int it = blockIdx.x; it < nitems && ok; it += gridDim.x) {
+      const int bh = it / nk, j = it - bh * nk, b = bh / a.nh;
+      if (masked(b, j)) continue;
+      for (int i = 0; i < nq; ++i, ++g) {
+        const int as = g & 1;
+        if (!(ok = mbar_wait(&aux_free[as], ((g >> 1) & 1) ^ 1, a.err, 108))) break;
+        bl_stage_aux(a, saux + as * kBLAux, bh, b, i * TILE, j * TILE, r);
+        mbar_arrive(&aux_full[as]);
+      }
     }
   } else {
-    const int sw = warp - 2;
     const int quarter = warp & 3;
-    const int half = sw >> 2;
+    const int hf = (warp - 2) >> 2;
     const int r = quarter * 32 + lane;
     const uint32_t lo = (uint32_t)(quarter * 32) << 16;
+    int n = 0;
+    uint32_t g = 0;
     bool ok = true;
-    for (int i = 0; i < nq && ok; ++i) {
-      const int q = i * TILE + r;
-      const bool qv = q < S;
-      const float lse2 = qv ? a.lse[row0 + q] * kLog2e : INFINITY;
-      const float Di = qv ? (a.dvec ? a.dvec[row0 + q] : dvec_row<T>(a, b, h, q)) : 0.0f;
-      if (!(ok = mbar_wait_warp(s_full, i & 1, a.err, 27))) break;
-      tc_fence_after();
-      if (!(ok = mbar_wait_warp(ds_free, (i & 1) ^ 1, a.err, 28))) break;
-      bwd_pair_rows<T>(a, b, row0, q, r, k0, half * 64, tS, tdP, lo, lse2, Di, sPd, sdS);
-      tc_fence_before();
-      mbar_arrive(s_free);
-      fence_proxy_async_smem();
-      mbar_arrive(ds_full);
-      if (a.fuse_dq) {
-        if (!(ok = mbar_wait_warp(dq_full, i & 1, a.err, 29))) break;
-        tc_fence_after();
-        float v[32];
-        tmem_ld32(tdQ + lo + half * 32, v);
-        tc_fence_before();
-        mbar_arrive(dq_free);
-        if (qv) {
-          T* dst = static_cast<T*>(a.dqkv) + ((size_t)b * S + q) * 3 * a.H + h * HD + half * 32;
+    for (int it = blockIdx.x; it < nitems && ok; it += gridDim.x) {
+      const int bh = it / nk, j = it - bh * nk, b = bh / a.nh, h = bh - b * a.nh;
+      const int key = j * TILE + r;   // TMEM lane r of dV, dK = key row
+      if (masked(b, j)) {
+        // no query attends to these keys: dK = dV = 0
+        if (key < S) {
+          T* dst = static_cast<T*>(a.dqkv) + ((size_t)b * S + key) * 3 * a.H + h * HD + hf * 32;
+          const float z[8] = {0, 0, 0, 0, 0, 0, 0, 0};
 #pragma unroll
           for (int c = 0; c < 32; c += 8) {
-            float w8[8];
-#pragma unroll
-            for (int t = 0; t < 8; ++t) w8[t] = v[c + t] * a.scale;
-            store8<T>(dst + c, w8);
+            store8<T>(dst + a.H + c, z);
+            store8<T>(dst + 2 * a.H + c, z);
           }
         }
+        continue;
       }
-    }
-    if (ok && mbar_wait_warp(acc_full, 0, a.err, 30)) {
+      for (int i = 0; i < nq; ++i, ++g) {
+        const int as = g & 1;
+        if (!(ok = mbar_wait_warp(&aux_full[as], (g >> 1) & 1, a.err, 109))) break;
+        if (!(ok = mbar_wait_warp(s_full, g & 1, a.err, 110))) break;
+        tc_fence_after();
+        if (!(ok = bl_softmax_pair<T>(a, saux + as * kBLAux, r, hf * 64, tS, tdP, lo, s_free, ds_free, (g & 1) ^ 1,
+                                      sPd, sdS)))
+          break;
+        mbar_arrive(&aux_free[as]);
+        fence_proxy_async_smem();
+        mbar_arrive(ds_full);
+      }
+      if (!ok) break;
+      if (!(ok = mbar_wait_warp(acc_full, n & 1, a.err, 111))) break;
       tc_fence_after();
-      const int key = k0 + r;
       float dv[32], dk[32];
-      tmem_ld32(tdV + lo + half * 32, dv);
-      tmem_ld32(tdK + lo + half * 32, dk);
+      tmem_ld32x2(tdV + lo + hf * 32, dv, tdK + lo + hf * 32, dk);
+      tc_fence_before();
+      mbar_arrive(acc_free);
       if (key < S) {
-        T* dst = static_cast<T*>(a.dqkv) + ((size_t)b * S + key) * 3 * a.H + h * HD + half * 32;
+        T* dst = static_cast<T*>(a.dqkv) + ((size_t)b * S + key) * 3 * a.H + h * HD + hf * 32;
 #pragma unroll
         for (int c = 0; c < 32; c += 8) {
           float w8[8], u8[8];
@@ -615,6 +821,7 @@ __global__ void __launch_bounds__(kBwdThreads)
           store8<T>(dst + 2 * a.H + c, u8);
         }
       }
+      ++n;
     }
   }
   tc_fence_before();
@@ -623,42 +830,41 @@ __global__ void __launch_bounds__(kBwdThreads)
   if (warp == 1) tmem_dealloc(tmem, 512);
 }
 
-// Query-tile CTA: dQ of 128 queries accumulated over every key tile (used
-// when the sequence spans several key tiles).
-constexpr int kBwdQSmem = 6 * TB + 1024 + 256;
-
 template <typename T>
-__global__ void __launch_bounds__(kBwdThreads)
-    attn_bwd_q_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
-                  const __grid_constant__ CUtensorMap tv, const __grid_constant__ CUtensorMap tdo, AttnTc a) {
+__global__ void __launch_bounds__(kBLThreads, 1)
+    attn_bwd_q_long(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
+                    const __grid_constant__ CUtensorMap tv, const __grid_constant__ CUtensorMap tdo, AttnTc a) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = align1024(smem_raw);
-  uint8_t* sQ = sm;
-  uint8_t* sdO = sm + TB;
-  uint8_t* sK = sm + 2 * TB;
-  uint8_t* sV = sm + 3 * TB;
-  uint8_t* sdS = sm + 4 * TB;   // pair
-  uint64_t* bar = reinterpret_cast<uint64_t*>(sm + 6 * TB);
-  uint64_t *qd_full = bar, *kv_full = bar + 1, *kv_empty = bar + 2, *s_full = bar + 3, *s_free = bar + 4,
-           *ds_full = bar + 5, *ds_free = bar + 6, *acc_full = bar + 7;
-  uint32_t* tslot = reinterpret_cast<uint32_t*>(bar + 8);
+  uint8_t* sQD = sm;                      // [2] x (Q, dO)
+  uint8_t* sKV = sm + 4 * TB;             // [2] x (K, V)
+  uint8_t* sdS = sm + 8 * TB;             // pair
+  uint8_t* saux = sm + 10 * TB;           // [2]
+  uint64_t* bar = reinterpret_cast<uint64_t*>(saux + 2 * kBLAux);
+  uint64_t *qd_full = bar, *qd_empty = bar + 2, *kv_full = bar + 4, *kv_empty = bar + 6, *aux_full = bar + 8,
+           *aux_free = bar + 10, *s_full = bar + 12, *s_free = bar + 13, *ds_full = bar + 14, *ds_free = bar + 15,
+           *acc_full = bar + 16, *acc_free = bar + 17;
+  uint32_t* tslot = reinterpret_cast<uint32_t*>(bar + 18);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int h = blockIdx.y, b = blockIdx.z;
   const int S = a.S;
-  const int row0 = (b * a.nh + h) * S;
-  const int q0 = blockIdx.x * TILE;
-  const int nk_all = (S + TILE - 1) / TILE;
-
+  const int nq = (S + TILE - 1) / TILE, nk_all = nq;
+  const int nitems = a.B * a.nh * nq;
   if (threadIdx.x == 0) {
-    mbar_init(qd_full, 1);
-    mbar_init(kv_full, 1);
-    mbar_init(kv_empty, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&qd_full[i], 1);
+      mbar_init(&qd_empty[i], 1);
+      mbar_init(&kv_full[i], 1);
+      mbar_init(&kv_empty[i], 1);
+      mbar_init(&aux_full[i], 128);
+      mbar_init(&aux_free[i], kSoftThreads);
+    }
     mbar_init(s_full, 1);
     mbar_init(s_free, kSoftThreads);
     mbar_init(ds_full, kSoftThreads);
     mbar_init(ds_free, 1);
     mbar_init(acc_full, 1);
+    mbar_init(acc_free, kSoftThreads);
     fence_barrier_init();
   }
   if (warp == 1) tmem_alloc(tslot, 512);
@@ -669,25 +875,27 @@ __global__ void __launch_bounds__(kBwdThreads)
   pdl_wait();
   pdl_launch_dependents();
   const uint32_t tS = tmem, tdP = tmem + 128, tdQ = tmem + 256;
-  // key tiles past the last unmasked key add nothing to dQ (at least one runs)
-  const int nk = max(1, min(nk_all, (key_extent(a, b) + TILE - 1) / TILE));
 
   if (warp == 0) {
     if (lane == 0) {
+      int n = 0;
+      uint32_t g = 0;
       bool ok = true;
-      mbar_arrive_expect_tx(qd_full, 2 * TB);
-      tma_load_2d(sQ, &tq, qd_full, 0, row0 + q0);
-      tma_load_2d(sdO, &tdo, qd_full, h * HD, b * S + q0);
-      int j = 0;
-      for (; j < nk; ++j) {
-        if (!mbar_wait(kv_empty, (j & 1) ^ 1, a.err, 31)) { ok = false; break; }
-        mbar_arrive_expect_tx(kv_full, 2 * TB);
-        tma_load_2d(sK, &tk, kv_full, 0, row0 + j * TILE);
-        tma_load_2d(sV, &tv, kv_full, 0, row0 + j * TILE);
-      }
-      if (!ok) {
-        mbar_wait(qd_full, 0, nullptr, 0);
-        if (j > 0) mbar_wait(kv_full, (j - 1) & 1, nullptr, 0);
+      for (int it = blockIdx.x; it < nitems && ok; it += gridDim.x, ++n) {
+        const int bh = it / nq, i = it - bh * nq, b = bh / a.nh, h = bh - b * a.nh;
+        const int nk = bl_key_tiles(a, b, nk_all);
+        const int qs = n & 1;
+        if (!(ok = mbar_wait(&qd_empty[qs], ((n >> 1) & 1) ^ 1, a.err, 121))) break;
+        mbar_arrive_expect_tx(&qd_full[qs], 2 * TB);
+        tma_load_2d(sQD + qs * 2 * TB, &tq, &qd_full[qs], 0, bh * S + i * TILE);
+        tma_load_2d(sQD + qs * 2 * TB + TB, &tdo, &qd_full[qs], h * HD, b * S + i * TILE);
+        for (int j = 0; j < nk; ++j, ++g) {
+          const int ks = g & 1;
+          if (!(ok = mbar_wait(&kv_empty[ks], ((g >> 1) & 1) ^ 1, a.err, 122))) break;
+          mbar_arrive_expect_tx(&kv_full[ks], 2 * TB);
+          tma_load_2d(sKV + ks * 2 * TB, &tk, &kv_full[ks], 0, bh * S + j * TILE);
+          tma_load_2d(sKV + ks * 2 * TB + TB, &tv, &kv_full[ks], 0, bh * S + j * TILE);
+        }
       }
     }
   } else if (warp == 1) {
@@ -695,55 +903,95 @@ __global__ void __launch_bounds__(kBwdThreads)
       const bool bf = a.bf16 != 0;
       const uint32_t id_kk = idesc_f16(128, 128, bf, false, false);
       const uint32_t id_km = idesc_f16(128, 64, bf, false, true);
-      const uint32_t aK = smem_u32(sK), aV = smem_u32(sV), aQ = smem_u32(sQ), adO = smem_u32(sdO);
       const uint32_t adS = smem_u32(sdS);
-      bool ok = mbar_wait(qd_full, 0, a.err, 32);
-      for (int j = 0; j < nk && ok; ++j) {
-        if (!(ok = mbar_wait(kv_full, j & 1, a.err, 33))) break;
-        if (!(ok = mbar_wait(s_free, (j & 1) ^ 1, a.err, 34))) break;
+      int n = 0;
+      uint32_t g = 0;
+      bool ok = true;
+      // dQ += dS K of pair gp; the first pair of an item overwrites
+      auto dq = [&](uint32_t gp, bool acc, int nn) -> bool {
+        if (!acc && !mbar_wait(acc_free, (nn & 1) ^ 1, a.err, 123)) return false;
+        if (!mbar_wait(ds_full, gp & 1, a.err, 124)) return false;
         tc_fence_after();
-#pragma unroll
-        for (int kk = 0; kk < HD / 16; ++kk) mma_f16(tS, dk_tile(aQ, kk), dk_tile(aK, kk), id_kk, kk > 0);
-#pragma unroll
-        for (int kk = 0; kk < HD / 16; ++kk) mma_f16(tdP, dk_tile(adO, kk), dk_tile(aV, kk), id_kk, kk > 0);
-        mma_commit(s_full);
-        if (!(ok = mbar_wait(ds_full, j & 1, a.err, 35))) break;
-        tc_fence_after();
+        const uint32_t aK = smem_u32(sKV + (gp & 1) * 2 * TB);
 #pragma unroll
         for (int kk = 0; kk < TILE / 16; ++kk)
-          mma_f16(tdQ, dk_pair(adS, kk), dmn_tile(aK, kk), id_km, (j > 0 || kk > 0) ? 1u : 0u);
+          mma_f16(tdQ, dk_pair(adS, kk), dmn_tile(aK, kk), id_km, (acc || kk > 0) ? 1u : 0u);
         mma_commit(ds_free);
-        mma_commit(kv_empty);
+        mma_commit(&kv_empty[gp & 1]);
+        return true;
+      };
+      for (int it = blockIdx.x; it < nitems && ok; it += gridDim.x, ++n) {
+        const int bh = it / nq, b = bh / a.nh;
+        const int nk = bl_key_tiles(a, b, nk_all);
+        const int qs = n & 1;
+        if (!(ok = mbar_wait(&qd_full[qs], (n >> 1) & 1, a.err, 125))) break;
+        const uint32_t aQ = smem_u32(sQD + qs * 2 * TB), adO = aQ + TB;
+        for (int j = 0; j < nk; ++j, ++g) {
+          const int ks = g & 1;
+          if (!(ok = mbar_wait(&kv_full[ks], (g >> 1) & 1, a.err, 126))) break;
+          if (!(ok = mbar_wait(s_free, (g & 1) ^ 1, a.err, 127))) break;
+          tc_fence_after();
+          const uint32_t aK = smem_u32(sKV + ks * 2 * TB), aV = aK + TB;
+#pragma unroll
+          for (int kk = 0; kk < HD / 16; ++kk) mma_f16(tS, dk_tile(aQ, kk), dk_tile(aK, kk), id_kk, kk > 0);
+#pragma unroll
+          for (int kk = 0; kk < HD / 16; ++kk) mma_f16(tdP, dk_tile(adO, kk), dk_tile(aV, kk), id_kk, kk > 0);
+          mma_commit(s_full);
+          if (j > 0 && !(ok = dq(g - 1, j > 1, n))) break;
+        }
+        if (ok) ok = dq(g - 1, nk > 1, n);
+        if (!ok) break;
+        mma_commit(acc_full);
+        mma_commit(&qd_empty[qs]);
       }
-      if (ok) mma_commit(acc_full);
+    }
+  } else if (warp >= 10) {
+    const int r = threadIdx.x - 320;
+    uint32_t g = 0;
+    bool ok = true;
+    for (int it = blockIdx.x; it < nitems && ok; it += gridDim.x) {
+      const int bh = it / nq, i = it - bh * nq, b = bh / a.nh;
+      const int nk = bl_key_tiles(a, b, nk_all);
+      for (int j = 0; j < nk; ++j, ++g) {
+        const int as = g & 1;
+        if (!(ok = mbar_wait(&aux_free[as], ((g >> 1) & 1) ^ 1, a.err, 128))) break;
+        bl_stage_aux(a, saux + as * kBLAux, bh, b, i * TILE, j * TILE, r);
+        mbar_arrive(&aux_full[as]);
+      }
     }
   } else {
-    const int sw = warp - 2;
     const int quarter = warp & 3;
-    const int half = sw >> 2;
+    const int hf = (warp - 2) >> 2;
     const int r = quarter * 32 + lane;
     const uint32_t lo = (uint32_t)(quarter * 32) << 16;
-    const int q = q0 + r;
-    const bool qv = q < S;
-    const float lse2 = qv ? a.lse[row0 + q] * kLog2e : INFINITY;
-    const float Di = qv ? (a.dvec ? a.dvec[row0 + q] : dvec_row<T>(a, b, h, q)) : 0.0f;
+    int n = 0;
+    uint32_t g = 0;
     bool ok = true;
-    for (int j = 0; j < nk && ok; ++j) {
-      if (!(ok = mbar_wait_warp(s_full, j & 1, a.err, 36))) break;
-      tc_fence_after();
-      if (!(ok = mbar_wait_warp(ds_free, (j & 1) ^ 1, a.err, 37))) break;
-      bwd_pair_rows<T>(a, b, row0, q, r, j * TILE, half * 64, tS, tdP, lo, lse2, Di, nullptr, sdS);
-      tc_fence_before();
-      mbar_arrive(s_free);
-      fence_proxy_async_smem();
-      mbar_arrive(ds_full);
-    }
-    if (ok && mbar_wait_warp(acc_full, 0, a.err, 38)) {
+    for (int it = blockIdx.x; it < nitems && ok; it += gridDim.x, ++n) {
+      const int bh = it / nq, i = it - bh * nq, b = bh / a.nh, h = bh - b * a.nh;
+      const int nk = bl_key_tiles(a, b, nk_all);
+      for (int j = 0; j < nk; ++j, ++g) {
+        const int as = g & 1;
+        if (!(ok = mbar_wait_warp(&aux_full[as], (g >> 1) & 1, a.err, 129))) break;
+        if (!(ok = mbar_wait_warp(s_full, g & 1, a.err, 130))) break;
+        tc_fence_after();
+        if (!(ok = bl_softmax_pair<T>(a, saux + as * kBLAux, r, hf * 64, tS, tdP, lo, s_free, ds_free, (g & 1) ^ 1,
+                                      nullptr, sdS)))
+          break;
+        mbar_arrive(&aux_free[as]);
+        fence_proxy_async_smem();
+        mbar_arrive(ds_full);
+      }
+      if (!ok) break;
+      if (!(ok = mbar_wait_warp(acc_full, n & 1, a.err, 131))) break;
       tc_fence_after();
       float v[32];
-      tmem_ld32(tdQ + lo + half * 32, v);
-      if (qv) {
-        T* dst = static_cast<T*>(a.dqkv) + ((size_t)b * S + q) * 3 * a.H + h * HD + half * 32;
+      tmem_ld32(tdQ + lo + hf * 32, v);
+      tc_fence_before();
+      mbar_arrive(acc_free);
+      const int q = i * TILE + r;
+      if (q < S) {
+        T* dst = static_cast<T*>(a.dqkv) + ((size_t)b * S + q) * 3 * a.H + h * HD + hf * 32;
 #pragma unroll
         for (int c = 0; c < 32; c += 8) {
           float w8[8];
@@ -779,33 +1027,6 @@ constexpr int kPFwdBits = 128 * 16;                      // keep bits of one ite
 constexpr int kPFwdMask = 128 * 4;                       // mask row of one item: [128] float
 constexpr int kPFwdIn = 3;                               // Q/K/V input slots (loads run up to 3 items ahead)
 constexpr int kPFwdSmem = (3 * kPFwdIn + 4) * TB + 2 * kPFwdBits + 2 * kPFwdMask + 1024 + 256;
-
-__device__ __forceinline__ float ex2_fast(float x) {
-  float r;
-  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(x));
-  return r;
-}
-__device__ __forceinline__ float max3f(float a, float b, float c) {
-  float r;
-  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
-  return r;
-}
-// Packed pairs of float32 (one instruction for both lanes on sm_100).
-__device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) {
-  unsigned long long d;
-  asm("fma.rn.f32x2 %0, %1, %2, %3;"
-      : "=l"(d)
-      : "l"(*reinterpret_cast<unsigned long long*>(&a)), "l"(*reinterpret_cast<unsigned long long*>(&b)),
-        "l"(*reinterpret_cast<unsigned long long*>(&c)));
-  return *reinterpret_cast<float2*>(&d);
-}
-__device__ __forceinline__ float2 add2(float2 a, float2 b) {
-  unsigned long long d;
-  asm("add.rn.f32x2 %0, %1, %2;"
-      : "=l"(d)
-      : "l"(*reinterpret_cast<unsigned long long*>(&a)), "l"(*reinterpret_cast<unsigned long long*>(&b)));
-  return *reinterpret_cast<float2*>(&d);
-}
 
 template <typename T>
 __global__ void __launch_bounds__(kPFwdThreads, 1)
@@ -1226,6 +1447,8 @@ __global__ void __launch_bounds__(kPBwdThreads, 1)
     uint8_t* stq = sPd + hf * 16384 + quarter * 4096;
     uint8_t* stv = sdS + hf * 16384 + quarter * 4096;
     const int swz = (lane >> 1) & 3;
+    // no mask and a full tile of keys: every mask value is 0
+    const bool plain = a.mask == nullptr && S == TILE;
     int n = 0;
     for (int it = blockIdx.x; it < nitems; it += gridDim.x, ++n) {
       const int j = n & 1;
@@ -1249,21 +1472,27 @@ __global__ void __launch_bounds__(kPBwdThreads, 1)
 #pragma unroll 1
       for (int c = 0; c < 2; ++c) {
         float sv[32], dv[32];
-        tmem_ld32(tS + lo + kc0 + c * 32, sv);
-        tmem_ld32(tdP + lo + kc0 + c * 32, dv);
+        tmem_ld32x2(tS + lo + kc0 + c * 32, sv, tdP + lo + kc0 + c * 32, dv);
         const uint32_t bw = c == 0 ? kb8.x : kb8.y;
 #pragma unroll
         for (int g = 0; g < 4; ++g) {
           const int kt = kc0 + c * 32 + g * 8;   // key column
           const uint32_t bits = (bw >> (8 * g)) & 0xFFu;
-          const float4 m0 = *reinterpret_cast<const float4*>(smask + kt);
-          const float4 m1 = *reinterpret_cast<const float4*>(smask + kt + 4);
-          const float ml[8] = {m0.x, m0.y, m0.z, m0.w, m1.x, m1.y, m1.z, m1.w};
+          float ml[8];
+          if (plain) {
+#pragma unroll
+            for (int t = 0; t < 8; ++t) ml[t] = -lse2;
+          } else {
+            const float4 m0 = *reinterpret_cast<const float4*>(smask + kt);
+            const float4 m1 = *reinterpret_cast<const float4*>(smask + kt + 4);
+            ml[0] = m0.x - lse2; ml[1] = m0.y - lse2; ml[2] = m0.z - lse2; ml[3] = m0.w - lse2;
+            ml[4] = m1.x - lse2; ml[5] = m1.y - lse2; ml[6] = m1.z - lse2; ml[7] = m1.w - lse2;
+          }
           float pd[8], ds[8];
 #pragma unroll
           for (int t = 0; t < 8; ++t) {
             // lse2 = +inf for rows past the sequence end: p = 0
-            const float p = ex2_fast(fmaf(sv[g * 8 + t], c2, ml[t]) - lse2);
+            const float p = ex2_fast(fmaf(sv[g * 8 + t], c2, ml[t]));
             const bool keep = (bits >> t) & 1u;
             pd[t] = keep ? p * dsc : 0.0f;
             const float dp = keep ? dv[g * 8 + t] * dsc : 0.0f;
@@ -1392,6 +1621,7 @@ AttnTc make_args(int dt, const AttnArgs& a) {
   t.fuse_dq = 0;
   t.ctx_tma = 0;
   t.keep = a.keep;
+  t.kv_ext = a.mask ? a.kv_ext : nullptr;
   t.bf16 = dt == DT_BF16;
   t.err = attn_error_word();
   return t;
@@ -1407,7 +1637,6 @@ void fwd_t(const AttnArgs& a, cudaStream_t s) {
     return;
   static bool attr = false;
   if (!attr) {
-    cudaFuncSetAttribute(attn_fwd_tc<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, kFwdSmem);
     cudaFuncSetAttribute(attn_fwd_tc_persist<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, kPFwdSmem);
     attr = true;
   }
@@ -1421,8 +1650,23 @@ void fwd_t(const AttnArgs& a, cudaStream_t s) {
     if (!t.ctx_tma) mc = mq;   // unused
     launch_pdl(attn_fwd_tc_persist<T>, grid, kPFwdThreads, kPFwdSmem, s, mq, mk, mv, mc, t);
   } else {
-    dim3 grid((a.S + TILE - 1) / TILE, a.nh, a.B);
-    launch_pdl(attn_fwd_tc<T>, grid, kFwdThreads, kFwdSmem, s, mq, mk, mv, t);
+    static bool lattr = false;
+    if (!lattr) {
+      cudaFuncSetAttribute(attn_fwd_tc_long<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, kLSmem);
+      lattr = true;
+    }
+    if (t.kv_ext) {
+      // each sequence's key extent, so items skip key tiles past it
+      launch_pdl(key_extent_kernel, a.B, 256, 0, s, a.mask, a.S, a.kv_ext);
+      count_launch();
+    }
+    int nsm = 148;
+    cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, 0);
+    const int nitems = a.B * a.nh * ((a.S + TILE - 1) / TILE);
+    CUtensorMap mc;
+    t.ctx_tma = a.S % 32 == 0 && map_tile(&mc, a.ctx, t.bf16, t.H, (uint64_t)a.B * a.S, t.H, 32) ? 1 : 0;
+    if (!t.ctx_tma) mc = mq;   // unused
+    launch_pdl(attn_fwd_tc_long<T>, std::min(nitems, nsm), kLThreads, kLSmem, s, mq, mk, mv, mc, t);
   }
   count_launch();
 }
@@ -1439,8 +1683,6 @@ void bwd_t(const AttnArgs& a, cudaStream_t s) {
   const int ntile = (a.S + TILE - 1) / TILE;
   static bool attr = false;
   if (!attr) {
-    cudaFuncSetAttribute(attn_bwd_kv_tc<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, kBwdKvSmem);
-    cudaFuncSetAttribute(attn_bwd_q_tc<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, kBwdQSmem);
     cudaFuncSetAttribute(attn_bwd_tc_persist<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, kPBwdSmem);
     attr = true;
   }
@@ -1460,13 +1702,18 @@ void bwd_t(const AttnArgs& a, cudaStream_t s) {
   dvec_launch(t.bf16 ? DT_BF16 : DT_F16, a, s);
   t.dvec = a.dvec;
   t.fuse_dq = 0;
-  dim3 grid(ntile, a.nh, a.B);
-  launch_pdl(attn_bwd_kv_tc<T>, grid, kBwdThreads, kBwdKvSmem, s, mq, mk, mv, mdo, t);
-  count_launch();
-  if (!t.fuse_dq) {
-    launch_pdl(attn_bwd_q_tc<T>, grid, kBwdThreads, kBwdQSmem, s, mq, mk, mv, mdo, t);
-    count_launch();
+  static bool lattr = false;
+  if (!lattr) {
+    cudaFuncSetAttribute(attn_bwd_kv_long<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, kBLKvSmem);
+    cudaFuncSetAttribute(attn_bwd_q_long<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, kBLQSmem);
+    lattr = true;
   }
+  int nsm = 148;
+  cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, 0);
+  const int nitems = a.B * a.nh * ntile;
+  launch_pdl(attn_bwd_kv_long<T>, std::min(nitems, nsm), kBLThreads, kBLKvSmem, s, mq, mk, mv, mdo, t);
+  launch_pdl(attn_bwd_q_long<T>, std::min(nitems, nsm), kBLThreads, kBLQSmem, s, mq, mk, mv, mdo, t);
+  count_launch(2);
 }
 
 }  // namespace

@@ -84,6 +84,15 @@ template <typename T> __device__ __forceinline__ void unpack8(const uint4& r, fl
 #pragma unroll
   for (int i = 0; i < 8; ++i) v[i] = to_f(h[i]);
 }
+// 8 floats rounded to the 16-bit type T, packed as a 16-byte vector (the
+// inverse of unpack8).
+template <typename T> __device__ __forceinline__ uint4 pack8(const float (&v)[8]) {
+  uint4 r;
+  T* h = reinterpret_cast<T*>(&r);
+#pragma unroll
+  for (int i = 0; i < 8; ++i) h[i] = from_f<T>(v[i]);
+  return r;
+}
 // Raw 8-element chunk as loaded from memory (16 bytes for 16-bit types, 32
 // for float), so a load can be issued early and converted later.
 template <typename T> struct Raw8 { uint4 a; };

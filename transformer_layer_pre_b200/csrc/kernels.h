@@ -210,6 +210,10 @@ struct AttnArgs {
   // out [B*nh][128 query rows][16 bytes] for S <= 128, else [B*nh][S][S/8]
   // (byte e/8 for the flat element index e of site 0)
   uint8_t* keep;
+  // (B) ints the forward of sequences longer than 128 fills with one past
+  // each sequence's last unmasked key (key tiles beyond it are skipped), or
+  // null to run every key tile
+  int* kv_ext;
   // backward
   const void* dctx;     // (B*S, nh*d)
   float* dvec;          // (B, nh, S) rowsum(dctx * ctx)

@@ -68,6 +68,8 @@ struct tl_layer {
   // attention dropout keep bits (site 0), written by the forward for the
   // backward: [B*nh][128][16] bytes for S <= 128, else [B*nh][S][S/8]; or null
   uint8_t* akeep = nullptr;
+  // per sequence: one past its last unmasked key (filled by the long-sequence forward)
+  int* kv_ext = nullptr;
   // split-K scratch of the four weight gradients (W2, W1, Wo, Wqkv), each its
   // own, so every split sum can wait for the closing finalize launch
   float* splitk[4] = {nullptr, nullptr, nullptr, nullptr};
@@ -169,6 +171,7 @@ size_t carve(tl_layer* L, char* base) {
   // for S <= 128, the flat [B*nh][S][S/8] otherwise
   const size_t akeep_bytes = L->S <= 128 ? (size_t)L->B * L->nh * 128 * 16 : (size_t)L->B * L->nh * L->S * (L->S / 8);
   L->akeep = L->pa > 0.0f ? (uint8_t*)c.take(akeep_bytes) : nullptr;
+  L->kv_ext = (int*)c.take((size_t)L->B * 4);
   return c.off;
 }
 
@@ -324,6 +327,7 @@ AttnArgs attn_args(tl_layer* L, const float* mask) {
   a.dvec = L->dvec;
   a.dqkv = L->dqkv;
   a.keep = L->akeep;
+  a.kv_ext = L->kv_ext;
   return a;
 }
 
