@@ -8,10 +8,12 @@ Bars (what the layer must meet against the float64 oracle):
     oracle in storage-rounded mode (float64 arithmetic, rounded to the
     storage type exactly where the CUDA path stores a tensor in HBM):
       - y and dx: float16: max |gpu - oracle| <= 2e-2.  bfloat16: 2e-2
-        plus two units in the last place of bfloat16 at the value (one for
-        the output's own rounding, one for a one-unit flip of the stored
-        tensor feeding the last step; one unit, 2^-5 at magnitudes >= 4, is
-        above 2e-2 by itself);
+        plus two units in the last place of bfloat16 at the tensor's
+        largest magnitude (one unit there, 2^-5 from magnitude 4 on, is
+        above 2e-2 by itself; the last steps, residual sums and the
+        LayerNorm backward's row means, carry a flip at a row's large
+        values to its small ones: two valid implementations differ by
+        0.031 on dx, |dx| <= 5.5, in the long post-LN bf16 layer);
       - weight and bias gradients: max |gpu - oracle| <= 2e-2, or one unit
         in the last place of the storage type at the tensor's largest
         magnitude when that unit is larger (float16 from magnitude 32 on,
@@ -105,9 +107,10 @@ def ulp(ref: np.ndarray, dtype: str) -> np.ndarray:
 def allowance(rounded: np.ndarray, dtype: str, stored: bool):
     """The max-abs allowance against the storage-rounded oracle (scalar or
     per element); see the module docstring."""
+    top = np.asarray(np.abs(rounded).max())
     if stored:
-        return MAX_ABS if dtype == "f16" else MAX_ABS + 2.0 * ulp(rounded, dtype)
-    return max(MAX_ABS, float(ulp(np.asarray(np.abs(rounded).max()), dtype)))
+        return MAX_ABS if dtype == "f16" else MAX_ABS + 2.0 * float(ulp(top, dtype))
+    return max(MAX_ABS, float(ulp(top, dtype)))
 
 
 def errors(gpu: np.ndarray, pure: np.ndarray, rounded: np.ndarray | None, dtype: str, stored: bool) -> dict:
