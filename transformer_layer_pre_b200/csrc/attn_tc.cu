@@ -63,6 +63,7 @@ struct AttnTc {
   int fuse_dq;
   int ctx_tma;          // persistent kernels: ctx (forward) or dQKV (backward) rows leave by TMA store (S % 32 == 0)
   const int* kv_ext;    // per sequence, one past its last unmasked key (long forward), or null
+  int keep_ready;       // persistent forward: the keep bits are already in `keep` (read, not drawn)
   uint8_t* keep;        // attention keep bits (forward writes, backward reads) or null: persistent path
                         // [B*nh][128][16]; longer sequences flat, byte e/8 for element e of site 0
   int bf16;
@@ -1128,7 +1129,11 @@ __global__ void __launch_bounds__(kPFwdThreads, 1)
     for (int it = blockIdx.x; it < nitems; it += gridDim.x, ++n) {
       const int j = n & 1;
       if (!mbar_wait(&aux_free[j], ((n >> 1) & 1) ^ 1, a.err, 58)) break;
-      if (a.drop.thr) {
+      if (a.drop.thr && a.keep_ready) {
+        // drawn ahead of this kernel (by the LayerNorm forward before it)
+        *reinterpret_cast<uint4*>(sbits + j * kPFwdBits + r * 16) =
+            __ldg(reinterpret_cast<const uint4*>(a.keep + ((size_t)it * 128 + r) * 16));
+      } else if (a.drop.thr) {
         const uint64_t e8 = (((uint64_t)it * S + (uint64_t)r) * (uint64_t)S) >> 3;
         uint32_t w[4];
 #pragma unroll
@@ -1622,6 +1627,7 @@ AttnTc make_args(int dt, const AttnArgs& a) {
   t.ctx_tma = 0;
   t.keep = a.keep;
   t.kv_ext = a.mask ? a.kv_ext : nullptr;
+  t.keep_ready = a.keep && a.S <= TILE ? a.keep_ready : 0;
   t.bf16 = dt == DT_BF16;
   t.err = attn_error_word();
   return t;

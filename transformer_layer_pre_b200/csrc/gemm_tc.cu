@@ -263,17 +263,20 @@ __global__ void __launch_bounds__(kThreads, 1)
 // "full" barrier; the leader issues tcgen05.mma.cta_group::2 (M = 256,
 // N = 256), which reads both CTAs' operands and writes each CTA's 128 rows of
 // the accumulator into that CTA's TMEM.  Per SM this halves the B traffic
-// into shared memory (32 KB per 64-wide K block instead of 48 KB), which
-// leaves room for six pipeline stages.  Commits multicast to both CTAs'
+// into shared memory (32 KB per 64-wide K block instead of 48 KB).  Commits multicast to both CTAs'
 // barriers; both CTAs' epilogues arrive on the leader's "accumulator empty"
 // barrier.  No TMA multicast is used.
-constexpr int kPairStages = 4;
+// Five stages (225 KB of shared memory with the epilogue's staging boxes):
+// measured against four on the layer's GEMMs in isolation, the K = 4096 and
+// 8192 launches gain 5-6 us and the others 1-3 us.
+constexpr int kPairStages = 5;
 constexpr int kPairStageBytes = 2 * 128 * BK * 2;                  // A half + B half, 32 KB
 constexpr int kPairEpiWarps = 16;
 constexpr int kPairThreads = 64 + 32 * kPairEpiWarps;
 constexpr int kStageOut = 2048;                                    // one 32-row x 64-byte store box
 constexpr int kPairOutBytes = kPairEpiWarps * 2 * kStageOut;       // two staging buffers per epilogue warp
 constexpr int kPairSmem = kPairStages * kPairStageBytes + kPairOutBytes + 1024 + 256;
+static_assert(kPairSmem <= 227 * 1024, "the pair kernel's shared memory exceeds a CTA's maximum");
 
 // Store destinations of the pair kernel's epilogue (TMA tensor maps).
 struct OutMaps {

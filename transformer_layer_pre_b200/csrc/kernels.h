@@ -122,9 +122,20 @@ void gemm_tc_wait_probe(cudaStream_t s);
 // (bit k = element e+k), the same bits dropout_bits8 gives; the row kernels
 // have idle arithmetic units, so the downstream kernels read the bits
 // instead of drawing Philox themselves.
+// With AttnKeepGen.keep set, a pre-LN LayerNorm forward (whose rows are the
+// layer's tokens, row t = b*S + s) also draws the attention-probability keep
+// bits (site 0) whose query row is its token, for every head, in the
+// [B*nh][128][16] layout of the S <= 128 tensor-core attention (16 bytes per
+// (sequence, head, query): byte q of query s is element-group
+// (((b*nh + h)*S + s)*S)/8 + q), so the attention forward reads them.
+struct AttnKeepGen {
+  uint8_t* keep;       // null: off
+  int nh, S;
+  DropoutParams dp;
+};
 void ln_fwd_run(int dtype, const void* x, const void* gamma, const void* beta, void* y, float* mean,
                 float* rstd, int rows, int H, float eps, cudaStream_t s, uint8_t* keep_out = nullptr,
-                const DropoutParams* dp = nullptr, int site = 0);
+                const DropoutParams* dp = nullptr, int site = 0, const AttnKeepGen* akeep = nullptr);
 
 // LayerNorm backward of one row block + residual-gradient add + optional
 // dropout of the result, with column partial sums for dgamma, dbeta and the
@@ -210,6 +221,9 @@ struct AttnArgs {
   // out [B*nh][128 query rows][16 bytes] for S <= 128, else [B*nh][S][S/8]
   // (byte e/8 for the flat element index e of site 0)
   uint8_t* keep;
+  // 1: the S <= 128 keep bits are already in `keep` (drawn by the LayerNorm
+  // forward before the attention), the forward reads them instead of drawing
+  int keep_ready;
   // (B) ints the forward of sequences longer than 128 fills with one past
   // each sequence's last unmasked key (key tiles beyond it are skipped), or
   // null to run every key tile

@@ -483,10 +483,18 @@ tl_status layer_forward(tl_layer* L, const void* x, const float* mask, const tl_
     eq.gen_drop = eo.drop;
   }
   if (L->pre_ln) {
+    // the attention keep bits (S <= 128, tensor-core attention) are drawn by
+    // LN1, whose arithmetic units are idle while it streams, instead of by
+    // the attention forward
+    AttnKeepGen ak = {};
+    if (aa.drop.thr && L->akeep && L->S <= 128 && attn_tc_supports(dt, aa)) {
+      ak.keep = L->akeep; ak.nh = L->nh; ak.S = L->S; ak.dp = aa.drop;
+      aa.keep_ready = 1;
+    }
     {
       ProfScope p_(PC_LN_FWD, s);
       ln_fwd_run(dt, x, w->ln1_g, w->ln1_b, L->h1, L->mean1, L->rstd1, T, H, L->opt.ln_eps, s,
-                 keepbits && !k1_gemm ? L->keep1 : nullptr, &eo.drop, 1);
+                 keepbits && !k1_gemm ? L->keep1 : nullptr, &eo.drop, 1, &ak);
     }
     if (keepbits) eo.keep8 = L->keep1;
     gemm(L, T, 3 * H, H, L->h1, H, true, w->wqkv, H, true, eq, s);

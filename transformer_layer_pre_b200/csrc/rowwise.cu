@@ -182,7 +182,7 @@ __global__ void __launch_bounds__(kFwdWarps * 32) ln_fwd_kernel(const T* __restr
                                                                 float* __restrict__ mean_out,
                                                                 float* __restrict__ rstd_out, int rows, int H,
                                                                 float eps, uint8_t* __restrict__ keep_out,
-                                                                DropoutParams dp, int site) {
+                                                                DropoutParams dp, int site, AttnKeepGen ak) {
   pdl_wait();
   pdl_launch_dependents();
   const int lane = threadIdx.x & 31;
@@ -211,6 +211,28 @@ __global__ void __launch_bounds__(kFwdWarps * 32) ln_fwd_kernel(const T* __restr
         if (row0 + q < rows && col < H) {
           const uint64_t e8 = ((uint64_t)(row0 + q) * H + col) >> 3;
           keep_out[e8] = (uint8_t)dropout_bits8(dp, site, e8);
+        }
+      }
+    }
+  }
+  if (ak.keep) {
+    // the attention-probability keep bits of the queries these rows are (site
+    // 0): 16 bytes per head, 8 per lane and step, drawn while the loads are in flight
+#pragma unroll
+    for (int q = 0; q < RPW; ++q) {
+      const int row = row0 + q;
+      if (row < rows) {
+        const int b = row / ak.S, sq = row - b * ak.S;
+        for (int c = lane; c < ak.nh * 2; c += 32) {
+          const int h = c >> 1, q0 = (c & 1) * 8;
+          const uint64_t e8 = ((((uint64_t)(b * ak.nh + h)) * ak.S + sq) * ak.S >> 3) + q0;
+          uint32_t w0 = 0, w1 = 0;
+#pragma unroll
+          for (int g = 0; g < 4; ++g) {
+            w0 |= dropout_bits8(ak.dp, 0, e8 + g) << (8 * g);
+            w1 |= dropout_bits8(ak.dp, 0, e8 + 4 + g) << (8 * g);
+          }
+          *reinterpret_cast<uint2*>(ak.keep + ((size_t)(b * ak.nh + h) * 128 + sq) * 16 + q0) = make_uint2(w0, w1);
         }
       }
     }
@@ -817,7 +839,7 @@ int row_blocks(int rows) { return std::max(1, std::min(kMaxBlocks, (rows + 15) /
 
 template <typename T>
 void ln_fwd_t(const void* x, const void* g, const void* b, void* y, float* mean, float* rstd, int rows, int H,
-              float eps, cudaStream_t s, uint8_t* keep_out, const DropoutParams& dp, int site) {
+              float eps, cudaStream_t s, uint8_t* keep_out, const DropoutParams& dp, int site, const AttnKeepGen& ak) {
   TLP_NCH_SWITCH(H, {
     // one row per warp (two rows per warp, with both rows' loads issued
     // first, measured slower: 16.1 against 15.9 us for 8192 x 1024 fp16)
@@ -825,7 +847,7 @@ void ln_fwd_t(const void* x, const void* g, const void* b, void* y, float* mean,
     const int blocks = (rows + kFwdWarps * RPW - 1) / (kFwdWarps * RPW);
     launch_pdl(ln_fwd_kernel<T, NCH, RPW>, blocks, kFwdWarps * 32, 0, s, static_cast<const T*>(x),
                static_cast<const T*>(g), static_cast<const T*>(b), static_cast<T*>(y), mean, rstd, rows, H, eps,
-               keep_out, dp, site);
+               keep_out, dp, site, ak);
   });
   count_launch();
 }
@@ -881,13 +903,16 @@ int rowdrop_parts(int rows) { return row_blocks(rows); }
 int colsum_parts(int rows) { return std::max(1, std::min(kColParts, rows / 64)); }
 
 void ln_fwd_run(int dt, const void* x, const void* g, const void* b, void* y, float* mean, float* rstd, int rows,
-                int H, float eps, cudaStream_t s, uint8_t* keep_out, const DropoutParams* dp, int site) {
+                int H, float eps, cudaStream_t s, uint8_t* keep_out, const DropoutParams* dp, int site,
+                const AttnKeepGen* akeep) {
   DropoutParams d = {};
   if (keep_out && dp && dp->thr) d = *dp;
   else keep_out = nullptr;
-  if (dt == DT_F32) ln_fwd_t<float>(x, g, b, y, mean, rstd, rows, H, eps, s, keep_out, d, site);
-  else if (dt == DT_F16) ln_fwd_t<half_t>(x, g, b, y, mean, rstd, rows, H, eps, s, keep_out, d, site);
-  else ln_fwd_t<bf16_t>(x, g, b, y, mean, rstd, rows, H, eps, s, keep_out, d, site);
+  AttnKeepGen ak = {};
+  if (akeep && akeep->keep && akeep->dp.thr) ak = *akeep;
+  if (dt == DT_F32) ln_fwd_t<float>(x, g, b, y, mean, rstd, rows, H, eps, s, keep_out, d, site, ak);
+  else if (dt == DT_F16) ln_fwd_t<half_t>(x, g, b, y, mean, rstd, rows, H, eps, s, keep_out, d, site, ak);
+  else ln_fwd_t<bf16_t>(x, g, b, y, mean, rstd, rows, H, eps, s, keep_out, d, site, ak);
 }
 
 template <typename T>
