@@ -143,10 +143,10 @@ constexpr int kSoftThreads = 256;
 // P stays below 256 (exact in fp16/bf16 range) and most tiles skip the
 // rescale.  The result is the same softmax: every term carries the same
 // reference until the final normalisation.
-constexpr int kLThreads = 320;
+constexpr int kLThreads = 448;
 constexpr int kLKv = 3;                                     // K/V ring slots
 constexpr int kLAux = 128 * 16 + 128 * 4;                   // per slot: keep bits [128][16], mask [128]
-constexpr int kLSmem = 2 * TB + kLKv * 2 * TB + 4 * TB + 2 * kLAux + 1024 + 256;
+constexpr int kLSmem = 2 * TB + kLKv * 2 * TB + 4 * TB + 2 * kLAux + 1024 + 256 + 4096;   // + row exchange
 constexpr float kLRescale = 8.0f;                           // log2 units: P < 2^8
 
 // One past the last unmasked key of each sequence (kv_ext[b]), or S when the
@@ -214,11 +214,11 @@ __global__ void __launch_bounds__(kLThreads, 1)
       mbar_init(&q_full[i], 1);
       mbar_init(&q_empty[i], 1);
       mbar_init(&s_full[i], 1);
-      mbar_init(&s_free[i], 128);
-      mbar_init(&p_full[i], 128);
+      mbar_init(&s_free[i], kSoftThreads);
+      mbar_init(&p_full[i], kSoftThreads);
       mbar_init(&pv_done[i], 1);
       mbar_init(&aux_full[i], 128);
-      mbar_init(&aux_free[i], 128);
+      mbar_init(&aux_free[i], kSoftThreads);
     }
     for (int i = 0; i < kLKv; ++i) {
       mbar_init(&kv_full[i], 1);
@@ -302,9 +302,9 @@ __global__ void __launch_bounds__(kLThreads, 1)
         if (ok) ok = pv(g - 1, nt > 1);
       }
     }
-  } else if (warp >= 6) {
+  } else if (warp >= 10) {
     // helpers: keep bits and mask row of each key tile, two tiles ahead at most
-    const int r = threadIdx.x - 192;
+    const int r = threadIdx.x - 320;
     uint32_t g = 0;
     for (int it = blockIdx.x; it < nitems; it += gridDim.x) {
       const int bh = it / nq, q0 = (it - bh * nq) * TILE;
@@ -349,12 +349,17 @@ __global__ void __launch_bounds__(kLThreads, 1)
       if (!ok) break;
     }
   } else {
-    // softmax: warp w owns TMEM lanes 32*(w%4), thread = query row
+    // softmax: warp w owns TMEM lanes 32*(w%4) (query rows) and key columns
+    // 64*hf .. +63 of each tile, hf = (w-2)/4: two threads per query row,
+    // warps w and w+4 meet at a named barrier to combine their row maxima
     const int quarter = warp & 3;
+    const int hf = (warp - 2) >> 2;
     const int r = quarter * 32 + lane;
+    const int bar_id = 1 + quarter;
     const uint32_t lo = (uint32_t)(quarter * 32) << 16;
     const float c2 = a.scale * kLog2e;
     const float dsc = a.drop.thr ? a.drop.scale : 1.0f;
+    float* xch = reinterpret_cast<float*>(tslot + 4);   // [2 tiles][2 halves][128] row maxima, then row sums
     uint32_t g = 0;
     bool ok = true;
     for (int it = blockIdx.x; it < nitems && ok; it += gridDim.x) {
@@ -366,26 +371,27 @@ __global__ void __launch_bounds__(kLThreads, 1)
       for (int j = 0; j < nt; ++j, ++g) {
         const int ss = g & 1;
         const uint8_t* ax = saux + ss * kLAux;
-        const float* mrow = reinterpret_cast<const float*>(ax + 2048);
+        const float* mrow = reinterpret_cast<const float*>(ax + 2048) + hf * 64;
         if (!(ok = mbar_wait_warp(&aux_full[ss], (g >> 1) & 1, a.err, 88))) break;
-        const uint4 kb16 = a.drop.thr ? *reinterpret_cast<const uint4*>(ax + r * 16) : make_uint4(~0u, ~0u, ~0u, ~0u);
+        const uint2 kb8 = a.drop.thr ? *reinterpret_cast<const uint2*>(ax + r * 16 + hf * 8) : make_uint2(~0u, ~0u);
         if (!(ok = mbar_wait_warp(&s_full[ss], (g >> 1) & 1, a.err, 89))) break;
         tc_fence_after();
-        const uint32_t ts = tmem + 128 * ss + lo;
-        // pass 1: the tile's row maximum (scaled scores + mask, log2 units)
+        const uint32_t ts = tmem + 128 * ss + lo + hf * 64;
+        float sv[64];
+        // pass 1: this half's row maximum (scaled scores + mask, log2 units),
+        // combined with the other half's
+        tmem_ld64(ts, sv);
         float mx = -INFINITY;
-#pragma unroll 1
-        for (int hh = 0; hh < 2; ++hh) {
-          float sv[64];
-          tmem_ld64(ts + hh * 64, sv);
 #pragma unroll
-          for (int t = 0; t < 64; t += 4) {
-            const float4 m4 = *reinterpret_cast<const float4*>(mrow + hh * 64 + t);
-            const float2 x0 = fma2(make_float2(sv[t], sv[t + 1]), make_float2(c2, c2), make_float2(m4.x, m4.y));
-            const float2 x1 = fma2(make_float2(sv[t + 2], sv[t + 3]), make_float2(c2, c2), make_float2(m4.z, m4.w));
-            mx = max3f(mx, max3f(x0.x, x0.y, x1.x), x1.y);
-          }
+        for (int t = 0; t < 64; t += 4) {
+          const float4 m4 = *reinterpret_cast<const float4*>(mrow + t);
+          const float2 x0 = fma2(make_float2(sv[t], sv[t + 1]), make_float2(c2, c2), make_float2(m4.x, m4.y));
+          const float2 x1 = fma2(make_float2(sv[t + 2], sv[t + 3]), make_float2(c2, c2), make_float2(m4.z, m4.w));
+          mx = max3f(mx, max3f(x0.x, x0.y, x1.x), x1.y);
         }
+        xch[(ss * 2 + hf) * 128 + r] = mx;
+        named_barrier(bar_id, 64);
+        mx = fmaxf(xch[(ss * 2) * 128 + r], xch[(ss * 2 + 1) * 128 + r]);
         const float mnew = fmaxf(mref, mx);
         if (j == 0) {
           mref = mnew;   // the item's first product overwrites O
@@ -396,14 +402,11 @@ __global__ void __launch_bounds__(kLThreads, 1)
             if (!(ok = mbar_wait_warp(&pv_done[(g - 1) & 1], ((g - 1) >> 1) & 1, a.err, 90))) break;
             tc_fence_after();
             const float alpha = need ? ex2_approx(mref - mnew) : 1.0f;
+            float o[32];
+            tmem_ld32(tmem + 256 + lo + hf * 32, o);
 #pragma unroll
-            for (int hh = 0; hh < 2; ++hh) {
-              float o[32];
-              tmem_ld32(tmem + 256 + lo + hh * 32, o);
-#pragma unroll
-              for (int c = 0; c < 32; ++c) o[c] *= alpha;
-              tmem_st32(tmem + 256 + lo + hh * 32, o);
-            }
+            for (int c = 0; c < 32; ++c) o[c] *= alpha;
+            tmem_st32(tmem + 256 + lo + hf * 32, o);
             tmem_st_wait();
             if (need) {
               l *= alpha;
@@ -414,31 +417,24 @@ __global__ void __launch_bounds__(kLThreads, 1)
         const float msub = mref == -INFINITY ? 0.0f : mref;   // 2^(-inf - msub) = 0
         // the P slot is free once the product of tile g-2 is done
         if (g >= 2 && !(ok = mbar_wait_warp(&pv_done[ss], ((g - 2) >> 1) & 1, a.err, 91))) break;
-        if (lane == 0) bulk_wait_read<0>();   // an earlier item's output staged in this slot has left
-        __syncwarp();
-        // pass 2: P = 2^(x - m_ref), dropped, into the P tile; row sum of the undropped P
+        // pass 2: P = 2^(x - m_ref), dropped, into this half of the P tile;
+        // row sum of the undropped P (the S values are still in registers)
         float2 ls2 = make_float2(0.0f, 0.0f);
-#pragma unroll 1
-        for (int hh = 0; hh < 2; ++hh) {
-          float sv[64];
-          tmem_ld64(ts + hh * 64, sv);
-          const uint32_t bw0 = hh == 0 ? kb16.x : kb16.z, bw1 = hh == 0 ? kb16.y : kb16.w;
 #pragma unroll
-          for (int gg = 0; gg < 8; ++gg) {
-            const uint32_t bits = ((gg < 4 ? bw0 : bw1) >> (8 * (gg & 3))) & 0xFFu;
-            float pv[8];
+        for (int gg = 0; gg < 8; ++gg) {
+          const uint32_t bits = ((gg < 4 ? kb8.x : kb8.y) >> (8 * (gg & 3))) & 0xFFu;
+          float pv[8];
 #pragma unroll
-            for (int t = 0; t < 8; t += 2) {
-              const float2 m2 = *reinterpret_cast<const float2*>(mrow + hh * 64 + gg * 8 + t);
-              const float2 x = add2(fma2(make_float2(sv[gg * 8 + t], sv[gg * 8 + t + 1]), make_float2(c2, c2), m2),
-                                    make_float2(-msub, -msub));
-              const float2 p = make_float2(ex2_approx(x.x), ex2_approx(x.y));
-              ls2 = add2(ls2, p);
-              pv[t] = ((bits >> t) & 1u) ? p.x : 0.0f;
-              pv[t + 1] = ((bits >> (t + 1)) & 1u) ? p.y : 0.0f;
-            }
-            pair_store8<T>(sP + ss * 2 * TB, r, hh * 8 + gg, pv);
+          for (int t = 0; t < 8; t += 2) {
+            const float2 m2 = *reinterpret_cast<const float2*>(mrow + gg * 8 + t);
+            const float2 x = add2(fma2(make_float2(sv[gg * 8 + t], sv[gg * 8 + t + 1]), make_float2(c2, c2), m2),
+                                  make_float2(-msub, -msub));
+            const float2 p = make_float2(ex2_approx(x.x), ex2_approx(x.y));
+            ls2 = add2(ls2, p);
+            pv[t] = ((bits >> t) & 1u) ? p.x : 0.0f;
+            pv[t + 1] = ((bits >> (t + 1)) & 1u) ? p.y : 0.0f;
           }
+          pair_store8<T>(sP + ss * 2 * TB, r, hf * 8 + gg, pv);
         }
         l += ls2.x + ls2.y;
         mbar_arrive(&aux_free[ss]);
@@ -448,36 +444,23 @@ __global__ void __launch_bounds__(kLThreads, 1)
         mbar_arrive(&p_full[ss]);
       }
       if (!ok) break;
-      // the item's output once its last product is in
+      // the item's output once its last product is in: this thread's 32
+      // columns of the row; the row sum is the two halves' sums
       const uint32_t gl = g - 1;
       if (!(ok = mbar_wait_warp(&pv_done[gl & 1], (gl >> 1) & 1, a.err, 92))) break;
       tc_fence_after();
-      float o[64];
-      tmem_ld64(tmem + 256 + lo, o);
-      const float inv = l > 0.0f ? dsc / l : 0.0f;
-      if (i < S) a.lse[(size_t)bh * S + i] = l > 0.0f ? (mref + log2f(l)) * kLn2 : INFINITY;
-      if (a.ctx_tma) {
-        // whole 32-row boxes (S % 32 == 0), staged in this warp's rows of the last P slot
-        if (q0 + quarter * 32 < S) {
-          uint8_t* ostage = sP + (gl & 1) * 2 * TB + quarter * 4096;
+      float o[32];
+      tmem_ld32(tmem + 256 + lo + hf * 32, o);
+      xch[(512 + hf * 128) + r] = l;
+      named_barrier(bar_id, 64);
+      const float lt = xch[512 + r] + xch[640 + r];
+      named_barrier(bar_id, 64);   // both have read the sums before the next item's tile maxima land
+      const float inv = lt > 0.0f ? dsc / lt : 0.0f;
+      if (i < S) {
+        if (hf == 0) a.lse[(size_t)bh * S + i] = lt > 0.0f ? (mref + log2f(lt)) * kLn2 : INFINITY;
+        T* dst = static_cast<T*>(a.ctx) + ((size_t)b * S + i) * a.H + h * HD + hf * 32;
 #pragma unroll
-          for (int c = 0; c < 8; ++c) {
-            float w8[8];
-#pragma unroll
-            for (int t = 0; t < 8; ++t) w8[t] = o[c * 8 + t] * inv;
-            store8<T>(reinterpret_cast<T*>(ostage + lane * 128 + ((c ^ (lane & 7)) << 4)), w8);
-          }
-          fence_proxy_async_smem();
-          __syncwarp();
-          if (lane == 0) {
-            tma_store_2d(&tctx, ostage, h * HD, b * S + q0 + quarter * 32);
-            bulk_commit();
-          }
-        }
-      } else if (i < S) {
-        T* dst = static_cast<T*>(a.ctx) + ((size_t)b * S + i) * a.H + h * HD;
-#pragma unroll
-        for (int c = 0; c < 64; c += 8) {
+        for (int c = 0; c < 32; c += 8) {
           float w8[8];
 #pragma unroll
           for (int t = 0; t < 8; ++t) w8[t] = o[c + t] * inv;
@@ -485,8 +468,6 @@ __global__ void __launch_bounds__(kLThreads, 1)
         }
       }
     }
-    if (lane == 0) bulk_wait_all();
-    __syncwarp();
   }
   tc_fence_before();
   __syncthreads();

@@ -124,10 +124,10 @@ void gemm_tc_wait_probe(cudaStream_t s);
 // instead of drawing Philox themselves.
 // With AttnKeepGen.keep set, a pre-LN LayerNorm forward (whose rows are the
 // layer's tokens, row t = b*S + s) also draws the attention-probability keep
-// bits (site 0) whose query row is its token, for every head, in the
-// [B*nh][128][16] layout of the S <= 128 tensor-core attention (16 bytes per
-// (sequence, head, query): byte q of query s is element-group
-// (((b*nh + h)*S + s)*S)/8 + q), so the attention forward reads them.
+// bits (site 0) whose query row is its token, for every head, in the S <= 128
+// layout of AttnArgs.keep (byte q of query s of item (b, h), at
+// ((b*nh + h)*128 + s)*16 + q, is element group (((b*nh + h)*S + s)*S)/8 + q),
+// so the attention forward reads them.
 struct AttnKeepGen {
   uint8_t* keep;       // null: off
   int nh, S;

@@ -482,12 +482,18 @@ tl_status layer_forward(tl_layer* L, const void* x, const float* mask, const tl_
     eq.gen_keep = L->keep1; eq.gen_keep2 = L->keep2; eq.gen_site = 1; eq.gen_n8 = (uint64_t)T * H / 8;
     eq.gen_drop = eo.drop;
   }
+  // The attention keep bits of the S <= 128 tensor-core attention are drawn
+  // ahead of it by LN1 (pre-LN), whose arithmetic units idle while its row
+  // loads stream, and the forward copies them in.  (Adding them to the idle
+  // QKV pairs' share instead made the step 4.7 us slower at B64 S128: those
+  // pairs then outlast the last round.  For longer sequences, S/8 bytes per
+  // head and token, LN1 itself became compute-bound: at S = 512 it took 58
+  // instead of 27 us while the attention forward saved 14 us, so there the
+  // forward's helper warps draw them.)
+  const bool attn_bits = aa.drop.thr && L->akeep && L->S <= 128 && attn_tc_supports(dt, aa);
   if (L->pre_ln) {
-    // the attention keep bits (S <= 128, tensor-core attention) are drawn by
-    // LN1, whose arithmetic units are idle while it streams, instead of by
-    // the attention forward
     AttnKeepGen ak = {};
-    if (aa.drop.thr && L->akeep && L->S <= 128 && attn_tc_supports(dt, aa)) {
+    if (attn_bits) {
       ak.keep = L->akeep; ak.nh = L->nh; ak.S = L->S; ak.dp = aa.drop;
       aa.keep_ready = 1;
     }
