@@ -707,12 +707,16 @@ __global__ void __launch_bounds__(256) colsum_kernel(const T* __restrict__ X, in
 
 // The closing sums of a backward pass, in one launch.  Blocks are numbered
 // over all jobs (first[j] = the first block of job j).  A column-sum job
-// gives each block 64 columns: 16 column groups of 4 (float4 loads) x 16
-// part lanes, lane l summing partial rows l, l+16, ..., then the 16 lane sums
-// in lane order (a fixed order).  A split-K job sums its partial matrices
-// element-wise, four floats a thread, partials in increasing order.
-constexpr int kFinCols = 64;
+// gives each block 32 columns: 8 column groups of 4 (float4 loads) x 32
+// part lanes, lane l summing partial rows l, l+32, ..., then the 32 lane sums
+// in lane order (a fixed order).  (Up to ten loads per thread, all issued
+// before the first add, so a block waits about one memory latency, not one
+// per load.)  A split-K job sums its partial matrices element-wise, four
+// floats a thread, partials in increasing order.
+constexpr int kFinCols = 32;
+constexpr int kFinLanes = 32;
 constexpr int kFinThreads = 256;
+static_assert(kFinLanes * (kFinCols / 4) == kFinThreads, "one thread per (part lane, column group)");
 
 struct FinalizeGrid {
   FinalizeList fl;
@@ -722,7 +726,7 @@ struct FinalizeGrid {
 __global__ void __launch_bounds__(kFinThreads) colsum_finalize_kernel(const __grid_constant__ FinalizeGrid fg) {
   pdl_wait();
   pdl_launch_dependents();
-  __shared__ float4 red[16][17];
+  __shared__ float4 red[kFinLanes][kFinCols / 4 + 1];
   int j = 0;
   while (j + 1 < fg.fl.n && (int)blockIdx.x >= fg.first[j + 1]) ++j;
   const FinalizeJob& job = fg.fl.job[j];
@@ -742,13 +746,20 @@ __global__ void __launch_bounds__(kFinThreads) colsum_finalize_kernel(const __gr
     }
     return;
   }
-  const int cg = threadIdx.x & 15, pl = threadIdx.x >> 4;
+  const int cg = threadIdx.x % (kFinCols / 4), pl = threadIdx.x / (kFinCols / 4);
   const int c = b * kFinCols + cg * 4;
   float4 s = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
   if (c < cols) {
     const float* __restrict__ part = job.part + c;
-#pragma unroll 4
-    for (int p = pl; p < nparts; p += 16) {
+    int p = pl;
+    for (; p + 7 * kFinLanes < nparts; p += 8 * kFinLanes) {
+      float4 v[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) v[i] = *reinterpret_cast<const float4*>(part + (size_t)(p + i * kFinLanes) * cols);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) { s.x += v[i].x; s.y += v[i].y; s.z += v[i].z; s.w += v[i].w; }
+    }
+    for (; p < nparts; p += kFinLanes) {
       const float4 v = *reinterpret_cast<const float4*>(part + (size_t)p * cols);
       s.x += v.x; s.y += v.y; s.z += v.z; s.w += v.w;
     }
@@ -758,7 +769,7 @@ __global__ void __launch_bounds__(kFinThreads) colsum_finalize_kernel(const __gr
   if (pl == 0 && c < cols) {
     float4 t = red[0][cg];
 #pragma unroll
-    for (int w = 1; w < 16; ++w) {
+    for (int w = 1; w < kFinLanes; ++w) {
       const float4 v = red[w][cg];
       t.x += v.x; t.y += v.y; t.z += v.z; t.w += v.w;
     }
