@@ -27,6 +27,9 @@
 #include <math.h>
 
 #include <algorithm>
+#include <map>
+#include <mutex>
+#include <tuple>
 #include <type_traits>
 
 #include "kernels.h"
@@ -1570,8 +1573,8 @@ EncodeTiledFn encode_fn() {
 
 // [rows][cols] row-major 16-bit matrix with row stride ld; box 64 x box_rows
 // (128-byte swizzle), or 32 x box_rows (64-byte swizzle) with narrow.
-bool map_tile(CUtensorMap* m, const void* p, bool bf16, uint64_t cols, uint64_t rows, uint64_t ld,
-              uint32_t box_rows = 128, bool narrow = false) {
+bool encode_tile(CUtensorMap* m, const void* p, bool bf16, uint64_t cols, uint64_t rows, uint64_t ld,
+                 uint32_t box_rows, bool narrow) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return false;
   cuuint64_t dims[2] = {cols, rows};
@@ -1582,6 +1585,27 @@ bool map_tile(CUtensorMap* m, const void* p, bool bf16, uint64_t cols, uint64_t 
             dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
             narrow ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B,
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// The same, from a cache keyed on every argument: a tensor map is a pure
+// function of them (address, shape, box), so a call with the buffers of an
+// earlier call encodes nothing.  Bounded: cleared when it reaches 1024 maps.
+std::mutex g_map_mu;
+std::map<std::tuple<uintptr_t, uint64_t, uint64_t, uint64_t, uint32_t, int, int>, CUtensorMap> g_maps;
+
+bool map_tile(CUtensorMap* m, const void* p, bool bf16, uint64_t cols, uint64_t rows, uint64_t ld,
+              uint32_t box_rows = 128, bool narrow = false) {
+  const auto key = std::make_tuple(reinterpret_cast<uintptr_t>(p), cols, rows, ld, box_rows, (int)narrow, (int)bf16);
+  std::lock_guard<std::mutex> lk(g_map_mu);
+  const auto it = g_maps.find(key);
+  if (it != g_maps.end()) {
+    *m = it->second;
+    return true;
+  }
+  if (!encode_tile(m, p, bf16, cols, rows, ld, box_rows, narrow)) return false;
+  if (g_maps.size() >= 1024) g_maps.clear();
+  g_maps.emplace(key, *m);
+  return true;
 }
 
 // Error word of the attention kernels' bounded waits (layout in sm100.cuh).
