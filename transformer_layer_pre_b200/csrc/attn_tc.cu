@@ -1280,21 +1280,29 @@ __global__ void __launch_bounds__(kPFwdThreads, 1)
 // item ahead of the softmax warps: D = rowsum(dO * O) (dO from the item's
 // shared tile, O from global memory), the row's log-sum-exp, the additive
 // key mask and the dropout keep bits, all into shared memory.
+// The softmax warps take item n's softmax and then item n-1's epilogue, and
+// the MMA issuer puts item n+1's S and dPd ahead of item n's dV, dK, dQ: the
+// gradient products of one item run while the epilogue of the one before it
+// drains, so no warp waits for them.  The epilogue goes through a staging
+// box of its own (dQ, dK, dV in turn), since Pd and dS already hold the next
+// item by then.
 constexpr int kPBwdThreads = 448;
 constexpr int kPBwdAux = 128 * 16 + 3 * 128 * 4;          // bits [128][16], mask, lse2, D [128] floats
-constexpr int kPBwdSmem = 12 * TB + 2 * kPBwdAux + 1024 + 256;   // (Q,K,V,dO) x2, Pd pair, dS pair, aux x2
+constexpr int kPBwdStage = 8 * 2048;                      // per softmax warp: one 32 x 64-byte box
+constexpr int kPBwdSmem = 12 * TB + 2 * kPBwdAux + kPBwdStage + 1024 + 256;   // (Q,K,V,dO) x2, Pd, dS, aux x2, stage
+static_assert(kPBwdSmem <= 227 * 1024, "the persistent backward's shared memory exceeds a CTA's maximum");
 
 template <typename T>
 __global__ void __launch_bounds__(kPBwdThreads, 1)
     attn_bwd_tc_persist(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
-                        const __grid_constant__ CUtensorMap tv, const __grid_constant__ CUtensorMap tdo,
-                        const __grid_constant__ CUtensorMap tdqkv, AttnTc a) {
+                        const __grid_constant__ CUtensorMap tv, const __grid_constant__ CUtensorMap tdo, AttnTc a) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = align1024(smem_raw);
   uint8_t* sPd = sm + 8 * TB;
   uint8_t* sdS = sm + 10 * TB;
   uint8_t* saux = sm + 12 * TB;    // per slot: bits [128][16] | mask [128] | lse2 [128] | D [128]
-  uint64_t* bar = reinterpret_cast<uint64_t*>(saux + 2 * kPBwdAux);
+  uint8_t* sstage = saux + 2 * kPBwdAux;
+  uint64_t* bar = reinterpret_cast<uint64_t*>(sstage + kPBwdStage);
   uint64_t *in_full = bar, *in_empty = bar + 2, *s_full = bar + 4, *s_free = bar + 5, *ds_full = bar + 6,
            *g_full = bar + 7, *g_free = bar + 8, *aux_full = bar + 9, *aux_free = bar + 11;
   uint32_t* tslot = reinterpret_cast<uint32_t*>(bar + 13);
@@ -1347,20 +1355,30 @@ __global__ void __launch_bounds__(kPBwdThreads, 1)
       const uint32_t id_mm = idesc_f16(128, 64, bf, true, true);
       const uint32_t id_km = idesc_f16(128, 64, bf, false, true);
       const uint32_t aPd = smem_u32(sPd), adS = smem_u32(sdS);
-      int n = 0;
-      for (int it = blockIdx.x; it < nitems; it += gridDim.x, ++n) {
+      int my_items = 0;
+      for (int it = blockIdx.x; it < nitems; it += gridDim.x) ++my_items;
+      // S and dPd of item n (TMEM free once the softmax of item n-1 read it)
+      auto mma_s = [&](int n) -> bool {
         const int j = n & 1;
         const uint32_t aQ = smem_u32(sm + j * 4 * TB), aK = aQ + TB, aV = aQ + 2 * TB, adO = aQ + 3 * TB;
-        if (!mbar_wait(&in_full[j], (n >> 1) & 1, a.err, 62)) break;
-        if (!mbar_wait(s_free, (n & 1) ^ 1, a.err, 63)) break;
+        if (!mbar_wait(&in_full[j], (n >> 1) & 1, a.err, 62)) return false;
+        if (!mbar_wait(s_free, (n & 1) ^ 1, a.err, 63)) return false;
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < HD / 16; ++kk) mma_f16(tS, dk_tile(aQ, kk), dk_tile(aK, kk), id_kk, kk > 0);
 #pragma unroll
         for (int kk = 0; kk < HD / 16; ++kk) mma_f16(tdP, dk_tile(adO, kk), dk_tile(aV, kk), id_kk, kk > 0);
         mma_commit(s_full);
-        if (!mbar_wait(ds_full, n & 1, a.err, 64)) break;
-        if (!mbar_wait(g_free, (n & 1) ^ 1, a.err, 65)) break;
+        return true;
+      };
+      bool ok = my_items > 0 ? mma_s(0) : true;
+      for (int n = 0; n < my_items && ok; ++n) {
+        const int j = n & 1;
+        const uint32_t aQ = smem_u32(sm + j * 4 * TB), aK = aQ + TB, adO = aQ + 3 * TB;
+        if (!(ok = mbar_wait(ds_full, n & 1, a.err, 64))) break;
+        if (n + 1 < my_items && !(ok = mma_s(n + 1))) break;
+        // dV, dK, dQ TMEM free once the epilogue of item n-1 read it
+        if (!(ok = mbar_wait(g_free, (n & 1) ^ 1, a.err, 65))) break;
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < TILE / 16; ++kk) mma_f16(tdV, dmn_pair(aPd, kk), dmn_tile(adO, kk), id_mm, kk > 0);
@@ -1401,25 +1419,35 @@ __global__ void __launch_bounds__(kPBwdThreads, 1)
       const bool qv = r < S;
       smask[r] = qv ? (a.mask ? a.mask[(size_t)b * S + r] * kLog2e : 0.0f) : -INFINITY;
       smask[128 + r] = qv ? a.lse[(size_t)it * S + r] * kLog2e : INFINITY;
-      float Di = 0.0f;
-      if (qv) {
-        // O row from global memory first, then dO from the item's shared tile
-        const T* orow = static_cast<const T*>(a.ctx_in) + ((size_t)b * S + r) * a.H + h * HD;
+      // D = rowsum(dO * O): O from global memory with whole-line loads (8
+      // lanes per 128-byte row, 4 rows per load, 32 rows per warp), then dO
+      // from the item's shared tile, the 8 lanes of a row reduced by shuffles
+      {
+        const int ch = lane & 7, sub = lane >> 3, r0 = (warp - 10) * 32;
+        const T* obase = static_cast<const T*>(a.ctx_in) + (size_t)b * S * a.H + h * HD + ch * 8;
         Raw8<T> o8[8];
 #pragma unroll
-        for (int c = 0; c < 8; ++c) o8[c] = raw8_load<T>(orow + c * 8);
+        for (int k = 0; k < 8; ++k) {
+          const int rr = r0 + k * 4 + sub;
+          o8[k] = rr < S ? raw8_load<T>(obase + (size_t)rr * a.H) : raw8_zero<T>();
+        }
         if (!mbar_wait(&in_full[j], (n >> 1) & 1, a.err, 70)) break;
-        const uint8_t* drow = sm + j * 4 * TB + 3 * TB + r * 128;
+        const uint8_t* dtile = sm + j * 4 * TB + 3 * TB;
 #pragma unroll
-        for (int c = 0; c < 8; ++c) {
+        for (int k = 0; k < 8; ++k) {
+          const int rr = r0 + k * 4 + sub;
           float x[8], y[8];
-          load8<T>(reinterpret_cast<const T*>(drow + ((c ^ (r & 7)) << 4)), x);
-          raw8_unpack<T>(o8[c], y);
+          load8<T>(reinterpret_cast<const T*>(dtile + rr * 128 + ((ch ^ (rr & 7)) << 4)), x);
+          raw8_unpack<T>(o8[k], y);
+          float d = 0.0f;
 #pragma unroll
-          for (int t = 0; t < 8; ++t) Di = fmaf(x[t], y[t], Di);
+          for (int t = 0; t < 8; ++t) d = fmaf(x[t], y[t], d);
+          d += __shfl_xor_sync(0xffffffffu, d, 1);
+          d += __shfl_xor_sync(0xffffffffu, d, 2);
+          d += __shfl_xor_sync(0xffffffffu, d, 4);
+          if (ch == 0) smask[256 + rr] = rr < S ? d : 0.0f;
         }
       }
-      smask[256 + r] = Di;
       mbar_arrive(&aux_full[j]);
     }
   } else {
@@ -1430,123 +1458,131 @@ __global__ void __launch_bounds__(kPBwdThreads, 1)
     const float c2 = a.scale * kLog2e;
     const float dsc = a.drop.thr ? a.drop.scale : 1.0f;
     const int kc0 = hf * 64;
-    // dQ, dK, dV rows of this warp staged as 32 x 64-byte swizzled boxes in
-    // the warp's own rows of Pd and dS (free between the dV/dK/dQ products
-    // and the next item's Pd, dS)
-    uint8_t* stq = sPd + hf * 16384 + quarter * 4096;
-    uint8_t* stv = sdS + hf * 16384 + quarter * 4096;
+    // this warp's staging box: dQ, dK, dV rows (32 x 64 bytes, 64-byte swizzle) in turn
+    uint8_t* stg = sstage + (warp - 2) * 2048;
     const int swz = (lane >> 1) & 3;
     // no mask and a full tile of keys: every mask value is 0
     const bool plain = a.mask == nullptr && S == TILE;
-    int n = 0;
-    for (int it = blockIdx.x; it < nitems; it += gridDim.x, ++n) {
-      const int j = n & 1;
-      const int b = it / a.nh, h = it - (it / a.nh) * a.nh;
-      const bool qv = r < S;
-      const size_t trow = (size_t)b * S + r;
-      const uint8_t* ax = saux + j * kPBwdAux;
-      const float* smask = reinterpret_cast<const float*>(ax + 2048);
-      if (!mbar_wait_warp(&aux_full[j], (n >> 1) & 1, a.err, 66)) break;
-      const uint2 kb8 = a.drop.thr ? *reinterpret_cast<const uint2*>(ax + r * 16 + hf * 8)
-                                   : make_uint2(0xFFFFFFFFu, 0xFFFFFFFFu);
-      const float lse2 = smask[128 + r];
-      const float Di = smask[256 + r];
-      if (!mbar_wait_warp(s_full, n & 1, a.err, 67)) break;
-      tc_fence_after();
-      if (a.ctx_tma) {
-        // the previous item's dQKV stores have read the staging rows
-        if (lane == 0) bulk_wait_read<0>();
-        __syncwarp();
-      }
+    int my_items = 0;
+    for (int it = blockIdx.x; it < nitems; it += gridDim.x) ++my_items;
+    for (int n = 0; n <= my_items; ++n) {
+      if (n < my_items) {
+        // ---- softmax of item n: Pd and dS into shared memory
+        const int j = n & 1;
+        const uint8_t* ax = saux + j * kPBwdAux;
+        const float* smask = reinterpret_cast<const float*>(ax + 2048);
+        if (!mbar_wait_warp(&aux_full[j], (n >> 1) & 1, a.err, 66)) break;
+        const uint2 kb8 = a.drop.thr ? *reinterpret_cast<const uint2*>(ax + r * 16 + hf * 8)
+                                     : make_uint2(0xFFFFFFFFu, 0xFFFFFFFFu);
+        const float lse2 = smask[128 + r];
+        const float Di = smask[256 + r];
+        if (!mbar_wait_warp(s_full, n & 1, a.err, 67)) break;
+        // the previous item's products have read its Pd and dS
+        if (n > 0 && !mbar_wait_warp(g_full, (n - 1) & 1, a.err, 71)) break;
+        tc_fence_after();
 #pragma unroll 1
-      for (int c = 0; c < 2; ++c) {
-        float sv[32], dv[32];
-        tmem_ld32x2(tS + lo + kc0 + c * 32, sv, tdP + lo + kc0 + c * 32, dv);
-        const uint32_t bw = c == 0 ? kb8.x : kb8.y;
+        for (int c = 0; c < 2; ++c) {
+          float sv[32], dv[32];
+          tmem_ld32x2(tS + lo + kc0 + c * 32, sv, tdP + lo + kc0 + c * 32, dv);
+          const uint32_t bw = c == 0 ? kb8.x : kb8.y;
 #pragma unroll
-        for (int g = 0; g < 4; ++g) {
-          const int kt = kc0 + c * 32 + g * 8;   // key column
-          const uint32_t bits = (bw >> (8 * g)) & 0xFFu;
-          float ml[8];
-          if (plain) {
+          for (int g = 0; g < 4; ++g) {
+            const int kt = kc0 + c * 32 + g * 8;   // key column
+            const uint32_t bits = (bw >> (8 * g)) & 0xFFu;
+            float ml[8];
+            if (plain) {
 #pragma unroll
-            for (int t = 0; t < 8; ++t) ml[t] = -lse2;
-          } else {
-            const float4 m0 = *reinterpret_cast<const float4*>(smask + kt);
-            const float4 m1 = *reinterpret_cast<const float4*>(smask + kt + 4);
-            ml[0] = m0.x - lse2; ml[1] = m0.y - lse2; ml[2] = m0.z - lse2; ml[3] = m0.w - lse2;
-            ml[4] = m1.x - lse2; ml[5] = m1.y - lse2; ml[6] = m1.z - lse2; ml[7] = m1.w - lse2;
+              for (int t = 0; t < 8; ++t) ml[t] = -lse2;
+            } else {
+              const float4 m0 = *reinterpret_cast<const float4*>(smask + kt);
+              const float4 m1 = *reinterpret_cast<const float4*>(smask + kt + 4);
+              ml[0] = m0.x - lse2; ml[1] = m0.y - lse2; ml[2] = m0.z - lse2; ml[3] = m0.w - lse2;
+              ml[4] = m1.x - lse2; ml[5] = m1.y - lse2; ml[6] = m1.z - lse2; ml[7] = m1.w - lse2;
+            }
+            float pd[8], ds[8];
+#pragma unroll
+            for (int t = 0; t < 8; ++t) {
+              // lse2 = +inf for rows past the sequence end: p = 0
+              const float p = ex2_fast(fmaf(sv[g * 8 + t], c2, ml[t]));
+              const bool keep = (bits >> t) & 1u;
+              pd[t] = keep ? p * dsc : 0.0f;
+              const float dp = keep ? dv[g * 8 + t] * dsc : 0.0f;
+              ds[t] = p * (dp - Di);
+            }
+            pair_store8<T>(sPd, r, kt >> 3, pd);
+            pair_store8<T>(sdS, r, kt >> 3, ds);
           }
-          float pd[8], ds[8];
-#pragma unroll
-          for (int t = 0; t < 8; ++t) {
-            // lse2 = +inf for rows past the sequence end: p = 0
-            const float p = ex2_fast(fmaf(sv[g * 8 + t], c2, ml[t]));
-            const bool keep = (bits >> t) & 1u;
-            pd[t] = keep ? p * dsc : 0.0f;
-            const float dp = keep ? dv[g * 8 + t] * dsc : 0.0f;
-            ds[t] = p * (dp - Di);
-          }
-          pair_store8<T>(sPd, r, kt >> 3, pd);
-          pair_store8<T>(sdS, r, kt >> 3, ds);
         }
+        mbar_arrive(&aux_free[j]);
+        tc_fence_before();
+        mbar_arrive(s_free);
+        fence_proxy_async_smem();
+        mbar_arrive(ds_full);
       }
-      mbar_arrive(&aux_free[j]);
-      tc_fence_before();
-      mbar_arrive(s_free);
-      fence_proxy_async_smem();
-      mbar_arrive(ds_full);
-      if (!mbar_wait_warp(g_full, n & 1, a.err, 68)) break;
-      tc_fence_after();
-      // dQ, dK, dV one after another (w3 = 0, 1, 2): TMEM -> scale -> store
-      // (staged for TMA, or direct) -> fused column sums
-      const bool staged = a.ctx_tma && quarter * 32 < S;
+      if (n > 0) {
+        // ---- epilogue of item n-1: TMEM -> scale -> staging box -> fused
+        // column sums and whole-row-segment stores, dQ, dK, dV in turn
+        const int pn = n - 1, pit = blockIdx.x + pn * gridDim.x;
+        const int b = pit / a.nh, h = pit - b * a.nh;
+        if (!mbar_wait_warp(g_full, pn & 1, a.err, 68)) break;
+        tc_fence_after();
 #pragma unroll 1
-      for (int w3 = 0; w3 < 3; ++w3) {
-        float x[32];
-        tmem_ld32(tdQ - 64 * w3 + lo + hf * 32, x);
-        if (w3 == 2) {
-          tc_fence_before();
-          mbar_arrive(g_free);
-        }
-        if (w3 < 2) {
+        for (int w3 = 0; w3 < 3; ++w3) {
+          float x[32];
+          tmem_ld32(tdQ - 64 * w3 + lo + hf * 32, x);
+          if (w3 == 2) {
+            tc_fence_before();
+            mbar_arrive(g_free);
+          }
+          if (w3 < 2) {
 #pragma unroll
-          for (int c = 0; c < 32; ++c) x[c] *= a.scale;
-        }
-        if (staged) {
-          uint8_t* st = w3 == 0 ? stq : (w3 == 1 ? stq + 2048 : stv);
+            for (int c = 0; c < 32; ++c) x[c] *= a.scale;
+          }
 #pragma unroll
           for (int c = 0; c < 4; ++c)
-            store8<T>(reinterpret_cast<T*>(st + lane * 64 + ((c ^ swz) << 4)), *reinterpret_cast<float(*)[8]>(x + c * 8));
-        } else if (!a.ctx_tma && qv) {
-          // row r is query r for dQ and key r for dK, dV (both < S)
-          T* dst = static_cast<T*>(a.dqkv) + trow * 3 * a.H + w3 * a.H + h * HD + hf * 32;
+            store8<T>(reinterpret_cast<T*>(stg + lane * 64 + ((c ^ swz) << 4)), *reinterpret_cast<float(*)[8]>(x + c * 8));
+          __syncwarp();
+          if (a.colsum) {
+            // QKV bias gradient fused in: column sums of the stored values
+            // over this warp's rows inside the sequence.  Lane l sums
+            // columns 2p, 2p+1 (p = l % 16) over rows 16*(l / 16) .. +15 (the
+            // upper half in the other bank half's row order), then the halves
+            const int p = lane & 15, rh = lane >> 4;
+            float s0 = 0.0f, s1 = 0.0f;
+#pragma unroll 4
+            for (int i = 0; i < 16; ++i) {
+              const int rr = rh * 16 + (i ^ rh);
+              if (quarter * 32 + rr < S) {
+                const uint32_t w = *reinterpret_cast<const uint32_t*>(
+                    stg + rr * 64 + ((((p >> 2) ^ ((rr >> 1) & 3))) << 4) + (p & 3) * 4);
+                const T* hv = reinterpret_cast<const T*>(&w);
+                s0 += to_f(hv[0]);
+                s1 += to_f(hv[1]);
+              }
+            }
+            s0 += __shfl_xor_sync(0xffffffffu, s0, 16);
+            s1 += __shfl_xor_sync(0xffffffffu, s1, 16);
+            float* cs = a.colsum + (size_t)(b * 4 + quarter) * 3 * a.H + w3 * a.H + h * HD + hf * 32;
+            if (lane < 16) {
+              cs[2 * p] = s0;
+              cs[2 * p + 1] = s1;
+            }
+          }
+          // rows r of the box: query r for dQ, key r for dK and dV; 4 lanes
+          // per row's 64 bytes, 8 rows per store
+          const int ch = lane & 3;
 #pragma unroll
-          for (int c = 0; c < 32; c += 8) store8<T>(dst + c, *reinterpret_cast<float(*)[8]>(x + c));
-        }
-        if (a.colsum) {
-          // QKV bias gradient fused in: column sums of the stored values over
-          // this warp's 32 rows (rows past the sequence end count as zero)
-#pragma unroll
-          for (int c = 0; c < 32; ++c) x[c] = qv ? round_f<T>(x[c]) : 0.0f;
-          a.colsum[(size_t)(b * 4 + quarter) * 3 * a.H + w3 * a.H + h * HD + hf * 32 + lane] = warp_colsum32(x);
-        }
-      }
-      if (staged) {
-        // three TMA stores per warp of whole 32-row boxes (S % 32 == 0)
-        fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) {
-          const int x = h * HD + hf * 32, y = b * S + quarter * 32;
-          tma_store_2d(&tdqkv, stq, x, y);
-          tma_store_2d(&tdqkv, stq + 2048, x + a.H, y);
-          tma_store_2d(&tdqkv, stv, x + 2 * a.H, y);
-          bulk_commit();
+          for (int i = 0; i < 4; ++i) {
+            const int rr = i * 8 + (lane >> 2);
+            const uint4 v = *reinterpret_cast<const uint4*>(stg + rr * 64 + ((ch ^ ((rr >> 1) & 3)) << 4));
+            if (quarter * 32 + rr < S)
+              *reinterpret_cast<uint4*>(static_cast<T*>(a.dqkv) + ((size_t)b * S + quarter * 32 + rr) * 3 * a.H +
+                                        w3 * a.H + h * HD + hf * 32 + ch * 8) = v;
+          }
+          __syncwarp();
         }
       }
     }
-    if (a.ctx_tma && lane == 0) bulk_wait_all();
-    __syncwarp();
   }
   tc_fence_before();
   __syncthreads();
@@ -1700,13 +1736,7 @@ void bwd_t(const AttnArgs& a, cudaStream_t s) {
   if (ntile == 1) {
     int nsm = 148;
     cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, 0);
-    // dQKV (B*S, 3H) in 32 x 32 boxes; a box's rows stay inside one sequence when S % 32 == 0
-    CUtensorMap mdq;
-    t.ctx_tma = a.S % 32 == 0 && map_tile(&mdq, a.dqkv, t.bf16, 3 * (uint64_t)t.H, tokens, 3 * (uint64_t)t.H, 32, true)
-                    ? 1 : 0;
-    if (!t.ctx_tma) mdq = mq;   // unused
-    launch_pdl(attn_bwd_tc_persist<T>, std::min(a.B * a.nh, nsm), kPBwdThreads, kPBwdSmem, s, mq, mk, mv, mdo, mdq,
-               t);
+    launch_pdl(attn_bwd_tc_persist<T>, std::min(a.B * a.nh, nsm), kPBwdThreads, kPBwdSmem, s, mq, mk, mv, mdo, t);
     count_launch();
     return;
   }
