@@ -1284,8 +1284,8 @@ __global__ void __launch_bounds__(kPFwdThreads, 1)
 // the MMA issuer puts item n+1's S and dPd ahead of item n's dV, dK, dQ: the
 // gradient products of one item run while the epilogue of the one before it
 // drains, so no warp waits for them.  The epilogue goes through a staging
-// box of its own (dQ, dK, dV in turn), since Pd and dS already hold the next
-// item by then.
+// box of each warp's own (dQ, dK, dV in turn, each leaving by TMA store),
+// since Pd and dS already hold the next item by then.
 constexpr int kPBwdThreads = 448;
 constexpr int kPBwdAux = 128 * 16 + 3 * 128 * 4;          // bits [128][16], mask, lse2, D [128] floats
 constexpr int kPBwdStage = 8 * 2048;                      // per softmax warp: one 32 x 64-byte box
@@ -1295,7 +1295,8 @@ static_assert(kPBwdSmem <= 227 * 1024, "the persistent backward's shared memory 
 template <typename T>
 __global__ void __launch_bounds__(kPBwdThreads, 1)
     attn_bwd_tc_persist(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
-                        const __grid_constant__ CUtensorMap tv, const __grid_constant__ CUtensorMap tdo, AttnTc a) {
+                        const __grid_constant__ CUtensorMap tv, const __grid_constant__ CUtensorMap tdo,
+                        const __grid_constant__ CUtensorMap tdqkv, AttnTc a) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = align1024(smem_raw);
   uint8_t* sPd = sm + 8 * TB;
@@ -1526,6 +1527,8 @@ __global__ void __launch_bounds__(kPBwdThreads, 1)
         const int b = pit / a.nh, h = pit - b * a.nh;
         if (!mbar_wait_warp(g_full, pn & 1, a.err, 68)) break;
         tc_fence_after();
+        // whole 32-row boxes inside the sequence leave by TMA store
+        const bool tma = a.ctx_tma && quarter * 32 + 32 <= S;
 #pragma unroll 1
         for (int w3 = 0; w3 < 3; ++w3) {
           float x[32];
@@ -1538,10 +1541,20 @@ __global__ void __launch_bounds__(kPBwdThreads, 1)
 #pragma unroll
             for (int c = 0; c < 32; ++c) x[c] *= a.scale;
           }
+          // the box's previous store has read it
+          if (a.ctx_tma) {
+            if (lane == 0) bulk_wait_read<0>();
+            __syncwarp();
+          }
 #pragma unroll
           for (int c = 0; c < 4; ++c)
             store8<T>(reinterpret_cast<T*>(stg + lane * 64 + ((c ^ swz) << 4)), *reinterpret_cast<float(*)[8]>(x + c * 8));
+          if (tma) fence_proxy_async_smem();
           __syncwarp();
+          if (tma && lane == 0) {
+            tma_store_2d(&tdqkv, stg, w3 * a.H + h * HD + hf * 32, b * S + quarter * 32);
+            bulk_commit();
+          }
           if (a.colsum) {
             // QKV bias gradient fused in: column sums of the stored values
             // over this warp's rows inside the sequence.  Lane l sums
@@ -1568,21 +1581,25 @@ __global__ void __launch_bounds__(kPBwdThreads, 1)
               cs[2 * p + 1] = s1;
             }
           }
-          // rows r of the box: query r for dQ, key r for dK and dV; 4 lanes
-          // per row's 64 bytes, 8 rows per store
-          const int ch = lane & 3;
+          if (!tma) {
+            // rows r of the box: query r for dQ, key r for dK and dV; 4 lanes
+            // per row's 64 bytes, 8 rows per store
+            const int ch = lane & 3;
 #pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            const int rr = i * 8 + (lane >> 2);
-            const uint4 v = *reinterpret_cast<const uint4*>(stg + rr * 64 + ((ch ^ ((rr >> 1) & 3)) << 4));
-            if (quarter * 32 + rr < S)
-              *reinterpret_cast<uint4*>(static_cast<T*>(a.dqkv) + ((size_t)b * S + quarter * 32 + rr) * 3 * a.H +
-                                        w3 * a.H + h * HD + hf * 32 + ch * 8) = v;
+            for (int i = 0; i < 4; ++i) {
+              const int rr = i * 8 + (lane >> 2);
+              const uint4 v = *reinterpret_cast<const uint4*>(stg + rr * 64 + ((ch ^ ((rr >> 1) & 3)) << 4));
+              if (quarter * 32 + rr < S)
+                *reinterpret_cast<uint4*>(static_cast<T*>(a.dqkv) + ((size_t)b * S + quarter * 32 + rr) * 3 * a.H +
+                                          w3 * a.H + h * HD + hf * 32 + ch * 8) = v;
+            }
           }
           __syncwarp();
         }
       }
     }
+    if (a.ctx_tma && lane == 0) bulk_wait_all();
+    __syncwarp();
   }
   tc_fence_before();
   __syncthreads();
@@ -1736,7 +1753,13 @@ void bwd_t(const AttnArgs& a, cudaStream_t s) {
   if (ntile == 1) {
     int nsm = 148;
     cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, 0);
-    launch_pdl(attn_bwd_tc_persist<T>, std::min(a.B * a.nh, nsm), kPBwdThreads, kPBwdSmem, s, mq, mk, mv, mdo, t);
+    // dQKV (B*S, 3H) in 32 x 32 boxes; a box's rows stay inside one sequence when S % 32 == 0
+    CUtensorMap mdq;
+    t.ctx_tma = a.S % 32 == 0 && map_tile(&mdq, a.dqkv, t.bf16, 3 * (uint64_t)t.H, tokens, 3 * (uint64_t)t.H, 32, true)
+                    ? 1 : 0;
+    if (!t.ctx_tma) mdq = mq;   // unused
+    launch_pdl(attn_bwd_tc_persist<T>, std::min(a.B * a.nh, nsm), kPBwdThreads, kPBwdSmem, s, mq, mk, mv, mdo, mdq,
+               t);
     count_launch();
     return;
   }
