@@ -1280,15 +1280,15 @@ __global__ void __launch_bounds__(kPFwdThreads, 1)
 // item ahead of the softmax warps: D = rowsum(dO * O) (dO from the item's
 // shared tile, O from global memory), the row's log-sum-exp, the additive
 // key mask and the dropout keep bits, all into shared memory.
-// The softmax warps take item n's softmax and then item n-1's epilogue, and
-// the MMA issuer puts item n+1's S and dPd ahead of item n's dV, dK, dQ: the
-// gradient products of one item run while the epilogue of the one before it
-// drains, so no warp waits for them.  The epilogue goes through a staging
-// box of each warp's own (dQ, dK, dV in turn, each leaving by TMA store),
-// since Pd and dS already hold the next item by then.
-constexpr int kPBwdThreads = 448;
+// Warps 2-9 (softmax) turn item n's S and dPd into Pd and dS while warps
+// 14-21 (epilogue) drain item n-1's dV, dK, dQ, and the MMA issuer puts item
+// n+1's S and dPd ahead of item n's gradient products: the tensor core, the
+// softmax and the epilogue each work on a different item.  Each epilogue warp
+// stages its rows through a box of its own (dQ, dK, dV in turn, each leaving
+// by TMA store).
+constexpr int kPBwdThreads = 704;                        // 0 TMA, 1 MMA, 2-9 softmax, 10-13 helpers, 14-21 epilogue
 constexpr int kPBwdAux = 128 * 16 + 3 * 128 * 4;          // bits [128][16], mask, lse2, D [128] floats
-constexpr int kPBwdStage = 8 * 2048;                      // per softmax warp: one 32 x 64-byte box
+constexpr int kPBwdStage = 8 * 2048;                      // per epilogue warp: one 32 x 64-byte box
 constexpr int kPBwdSmem = 12 * TB + 2 * kPBwdAux + kPBwdStage + 1024 + 256;   // (Q,K,V,dO) x2, Pd, dS, aux x2, stage
 static_assert(kPBwdSmem <= 227 * 1024, "the persistent backward's shared memory exceeds a CTA's maximum");
 
@@ -1391,7 +1391,7 @@ __global__ void __launch_bounds__(kPBwdThreads, 1)
         mma_commit(&in_empty[j]);
       }
     }
-  } else if (warp >= 10) {
+  } else if (warp >= 10 && warp < 14) {
     // per item: keep bits, mask row, lse2 and D of every query row
     const int r = threadIdx.x - 320;
     int n = 0;
@@ -1451,7 +1451,7 @@ __global__ void __launch_bounds__(kPBwdThreads, 1)
       }
       mbar_arrive(&aux_full[j]);
     }
-  } else {
+  } else if (warp < 10) {
     const int quarter = warp & 3;
     const int hf = (warp - 2) >> 2;
     const int r = quarter * 32 + lane;
@@ -1459,143 +1459,146 @@ __global__ void __launch_bounds__(kPBwdThreads, 1)
     const float c2 = a.scale * kLog2e;
     const float dsc = a.drop.thr ? a.drop.scale : 1.0f;
     const int kc0 = hf * 64;
-    // this warp's staging box: dQ, dK, dV rows (32 x 64 bytes, 64-byte swizzle) in turn
-    uint8_t* stg = sstage + (warp - 2) * 2048;
-    const int swz = (lane >> 1) & 3;
     // no mask and a full tile of keys: every mask value is 0
     const bool plain = a.mask == nullptr && S == TILE;
     int my_items = 0;
     for (int it = blockIdx.x; it < nitems; it += gridDim.x) ++my_items;
-    for (int n = 0; n <= my_items; ++n) {
-      if (n < my_items) {
-        // ---- softmax of item n: Pd and dS into shared memory
-        const int j = n & 1;
-        const uint8_t* ax = saux + j * kPBwdAux;
-        const float* smask = reinterpret_cast<const float*>(ax + 2048);
-        if (!mbar_wait_warp(&aux_full[j], (n >> 1) & 1, a.err, 66)) break;
-        const uint2 kb8 = a.drop.thr ? *reinterpret_cast<const uint2*>(ax + r * 16 + hf * 8)
-                                     : make_uint2(0xFFFFFFFFu, 0xFFFFFFFFu);
-        const float lse2 = smask[128 + r];
-        const float Di = smask[256 + r];
-        if (!mbar_wait_warp(s_full, n & 1, a.err, 67)) break;
-        // the previous item's products have read its Pd and dS
-        if (n > 0 && !mbar_wait_warp(g_full, (n - 1) & 1, a.err, 71)) break;
-        tc_fence_after();
+    for (int n = 0; n < my_items; ++n) {
+      // ---- softmax of item n: Pd and dS into shared memory
+      const int j = n & 1;
+      const uint8_t* ax = saux + j * kPBwdAux;
+      const float* smask = reinterpret_cast<const float*>(ax + 2048);
+      if (!mbar_wait_warp(&aux_full[j], (n >> 1) & 1, a.err, 66)) break;
+      const uint2 kb8 = a.drop.thr ? *reinterpret_cast<const uint2*>(ax + r * 16 + hf * 8)
+                                   : make_uint2(0xFFFFFFFFu, 0xFFFFFFFFu);
+      const float lse2 = smask[128 + r];
+      const float Di = smask[256 + r];
+      if (!mbar_wait_warp(s_full, n & 1, a.err, 67)) break;
+      // the previous item's products have read its Pd and dS
+      if (n > 0 && !mbar_wait_warp(g_full, (n - 1) & 1, a.err, 71)) break;
+      tc_fence_after();
 #pragma unroll 1
-        for (int c = 0; c < 2; ++c) {
-          float sv[32], dv[32];
-          tmem_ld32x2(tS + lo + kc0 + c * 32, sv, tdP + lo + kc0 + c * 32, dv);
-          const uint32_t bw = c == 0 ? kb8.x : kb8.y;
+      for (int c = 0; c < 4; ++c) {
+        float sv[16], dv[16];
+        tmem_ld16x2(tS + lo + kc0 + c * 16, sv, tdP + lo + kc0 + c * 16, dv);
+        const uint32_t bw = (c < 2 ? kb8.x : kb8.y) >> (16 * (c & 1));
 #pragma unroll
-          for (int g = 0; g < 4; ++g) {
-            const int kt = kc0 + c * 32 + g * 8;   // key column
-            const uint32_t bits = (bw >> (8 * g)) & 0xFFu;
-            float ml[8];
-            if (plain) {
+        for (int g = 0; g < 2; ++g) {
+          const int kt = kc0 + c * 16 + g * 8;   // key column
+          const uint32_t bits = (bw >> (8 * g)) & 0xFFu;
+          float ml[8];
+          if (plain) {
 #pragma unroll
-              for (int t = 0; t < 8; ++t) ml[t] = -lse2;
-            } else {
-              const float4 m0 = *reinterpret_cast<const float4*>(smask + kt);
-              const float4 m1 = *reinterpret_cast<const float4*>(smask + kt + 4);
-              ml[0] = m0.x - lse2; ml[1] = m0.y - lse2; ml[2] = m0.z - lse2; ml[3] = m0.w - lse2;
-              ml[4] = m1.x - lse2; ml[5] = m1.y - lse2; ml[6] = m1.z - lse2; ml[7] = m1.w - lse2;
-            }
-            float pd[8], ds[8];
-#pragma unroll
-            for (int t = 0; t < 8; ++t) {
-              // lse2 = +inf for rows past the sequence end: p = 0
-              const float p = ex2_fast(fmaf(sv[g * 8 + t], c2, ml[t]));
-              const bool keep = (bits >> t) & 1u;
-              pd[t] = keep ? p * dsc : 0.0f;
-              const float dp = keep ? dv[g * 8 + t] * dsc : 0.0f;
-              ds[t] = p * (dp - Di);
-            }
-            pair_store8<T>(sPd, r, kt >> 3, pd);
-            pair_store8<T>(sdS, r, kt >> 3, ds);
+            for (int t = 0; t < 8; ++t) ml[t] = -lse2;
+          } else {
+            const float4 m0 = *reinterpret_cast<const float4*>(smask + kt);
+            const float4 m1 = *reinterpret_cast<const float4*>(smask + kt + 4);
+            ml[0] = m0.x - lse2; ml[1] = m0.y - lse2; ml[2] = m0.z - lse2; ml[3] = m0.w - lse2;
+            ml[4] = m1.x - lse2; ml[5] = m1.y - lse2; ml[6] = m1.z - lse2; ml[7] = m1.w - lse2;
           }
+          float pd[8], ds[8];
+#pragma unroll
+          for (int t = 0; t < 8; ++t) {
+            // lse2 = +inf for rows past the sequence end: p = 0
+            const float p = ex2_fast(fmaf(sv[g * 8 + t], c2, ml[t]));
+            const bool keep = (bits >> t) & 1u;
+            pd[t] = keep ? p * dsc : 0.0f;
+            const float dp = keep ? dv[g * 8 + t] * dsc : 0.0f;
+            ds[t] = p * (dp - Di);
+          }
+          pair_store8<T>(sPd, r, kt >> 3, pd);
+          pair_store8<T>(sdS, r, kt >> 3, ds);
         }
-        mbar_arrive(&aux_free[j]);
-        tc_fence_before();
-        mbar_arrive(s_free);
-        fence_proxy_async_smem();
-        mbar_arrive(ds_full);
       }
-      if (n > 0) {
-        // ---- epilogue of item n-1: TMEM -> scale -> staging box -> fused
-        // column sums and whole-row-segment stores, dQ, dK, dV in turn
-        const int pn = n - 1, pit = blockIdx.x + pn * gridDim.x;
-        const int b = pit / a.nh, h = pit - b * a.nh;
-        if (!mbar_wait_warp(g_full, pn & 1, a.err, 68)) break;
-        tc_fence_after();
-        // whole 32-row boxes inside the sequence leave by TMA store
-        const bool tma = a.ctx_tma && quarter * 32 + 32 <= S;
+      mbar_arrive(&aux_free[j]);
+      tc_fence_before();
+      mbar_arrive(s_free);
+      fence_proxy_async_smem();
+      mbar_arrive(ds_full);
+    }
+  } else {
+    // ---- epilogue warps: item n's dV, dK, dQ out of TMEM -> scale -> staging
+    // box -> fused column sums and TMA store (whole-row-segment stores at a
+    // sequence's ragged end), dQ, dK, dV in turn
+    const int quarter = warp & 3;
+    const int hf = (warp - 14) >> 2;
+    const uint32_t lo = (uint32_t)(quarter * 32) << 16;
+    // this warp's staging box: dQ, dK, dV rows (32 x 64 bytes, 64-byte swizzle) in turn
+    uint8_t* stg = sstage + (warp - 14) * 2048;
+    const int swz = (lane >> 1) & 3;
+    // whole 32-row boxes inside the sequence leave by TMA store
+    const bool tma = a.ctx_tma && quarter * 32 + 32 <= S;
+    int n = 0;
+    for (int it = blockIdx.x; it < nitems; it += gridDim.x, ++n) {
+      const int b = it / a.nh, h = it - b * a.nh;
+      if (!mbar_wait_warp(g_full, n & 1, a.err, 68)) break;
+      tc_fence_after();
 #pragma unroll 1
-        for (int w3 = 0; w3 < 3; ++w3) {
-          float x[32];
-          tmem_ld32(tdQ - 64 * w3 + lo + hf * 32, x);
-          if (w3 == 2) {
-            tc_fence_before();
-            mbar_arrive(g_free);
-          }
-          if (w3 < 2) {
+      for (int w3 = 0; w3 < 3; ++w3) {
+        float x[32];
+        tmem_ld32(tdQ - 64 * w3 + lo + hf * 32, x);
+        if (w3 == 2) {
+          tc_fence_before();
+          mbar_arrive(g_free);
+        }
+        if (w3 < 2) {
 #pragma unroll
-            for (int c = 0; c < 32; ++c) x[c] *= a.scale;
-          }
-          // the box's previous store has read it
-          if (a.ctx_tma) {
-            if (lane == 0) bulk_wait_read<0>();
-            __syncwarp();
-          }
-#pragma unroll
-          for (int c = 0; c < 4; ++c)
-            store8<T>(reinterpret_cast<T*>(stg + lane * 64 + ((c ^ swz) << 4)), *reinterpret_cast<float(*)[8]>(x + c * 8));
-          if (tma) fence_proxy_async_smem();
-          __syncwarp();
-          if (tma && lane == 0) {
-            tma_store_2d(&tdqkv, stg, w3 * a.H + h * HD + hf * 32, b * S + quarter * 32);
-            bulk_commit();
-          }
-          if (a.colsum) {
-            // QKV bias gradient fused in: column sums of the stored values
-            // over this warp's rows inside the sequence.  Lane l sums
-            // columns 2p, 2p+1 (p = l % 16) over rows 16*(l / 16) .. +15 (the
-            // upper half in the other bank half's row order), then the halves
-            const int p = lane & 15, rh = lane >> 4;
-            float s0 = 0.0f, s1 = 0.0f;
-#pragma unroll 4
-            for (int i = 0; i < 16; ++i) {
-              const int rr = rh * 16 + (i ^ rh);
-              if (quarter * 32 + rr < S) {
-                const uint32_t w = *reinterpret_cast<const uint32_t*>(
-                    stg + rr * 64 + ((((p >> 2) ^ ((rr >> 1) & 3))) << 4) + (p & 3) * 4);
-                const T* hv = reinterpret_cast<const T*>(&w);
-                s0 += to_f(hv[0]);
-                s1 += to_f(hv[1]);
-              }
-            }
-            s0 += __shfl_xor_sync(0xffffffffu, s0, 16);
-            s1 += __shfl_xor_sync(0xffffffffu, s1, 16);
-            float* cs = a.colsum + (size_t)(b * 4 + quarter) * 3 * a.H + w3 * a.H + h * HD + hf * 32;
-            if (lane < 16) {
-              cs[2 * p] = s0;
-              cs[2 * p + 1] = s1;
-            }
-          }
-          if (!tma) {
-            // rows r of the box: query r for dQ, key r for dK and dV; 4 lanes
-            // per row's 64 bytes, 8 rows per store
-            const int ch = lane & 3;
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-              const int rr = i * 8 + (lane >> 2);
-              const uint4 v = *reinterpret_cast<const uint4*>(stg + rr * 64 + ((ch ^ ((rr >> 1) & 3)) << 4));
-              if (quarter * 32 + rr < S)
-                *reinterpret_cast<uint4*>(static_cast<T*>(a.dqkv) + ((size_t)b * S + quarter * 32 + rr) * 3 * a.H +
-                                          w3 * a.H + h * HD + hf * 32 + ch * 8) = v;
-            }
-          }
+          for (int c = 0; c < 32; ++c) x[c] *= a.scale;
+        }
+        // the box's previous store has read it
+        if (a.ctx_tma) {
+          if (lane == 0) bulk_wait_read<0>();
           __syncwarp();
         }
+#pragma unroll
+        for (int c = 0; c < 4; ++c)
+          store8<T>(reinterpret_cast<T*>(stg + lane * 64 + ((c ^ swz) << 4)), *reinterpret_cast<float(*)[8]>(x + c * 8));
+        if (tma) fence_proxy_async_smem();
+        __syncwarp();
+        if (tma && lane == 0) {
+          tma_store_2d(&tdqkv, stg, w3 * a.H + h * HD + hf * 32, b * S + quarter * 32);
+          bulk_commit();
+        }
+        if (a.colsum) {
+          // QKV bias gradient fused in: column sums of the stored values over
+          // this warp's rows inside the sequence.  Lane l sums columns 2p,
+          // 2p+1 (p = l % 16) over rows 16*(l / 16) .. +15 (the upper half in
+          // the other bank half's row order), then the halves
+          const int p = lane & 15, rh = lane >> 4;
+          float s0 = 0.0f, s1 = 0.0f;
+#pragma unroll 4
+          for (int i = 0; i < 16; ++i) {
+            const int rr = rh * 16 + (i ^ rh);
+            if (quarter * 32 + rr < S) {
+              const uint32_t w = *reinterpret_cast<const uint32_t*>(
+                  stg + rr * 64 + ((((p >> 2) ^ ((rr >> 1) & 3))) << 4) + (p & 3) * 4);
+              const T* hv = reinterpret_cast<const T*>(&w);
+              s0 += to_f(hv[0]);
+              s1 += to_f(hv[1]);
+            }
+          }
+          s0 += __shfl_xor_sync(0xffffffffu, s0, 16);
+          s1 += __shfl_xor_sync(0xffffffffu, s1, 16);
+          float* cs = a.colsum + (size_t)(b * 4 + quarter) * 3 * a.H + w3 * a.H + h * HD + hf * 32;
+          if (lane < 16) {
+            cs[2 * p] = s0;
+            cs[2 * p + 1] = s1;
+          }
+        }
+        if (!tma) {
+          // rows r of the box: query r for dQ, key r for dK and dV; 4 lanes
+          // per row's 64 bytes, 8 rows per store
+          const int ch = lane & 3;
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const int rr = i * 8 + (lane >> 2);
+            const uint4 v = *reinterpret_cast<const uint4*>(stg + rr * 64 + ((ch ^ ((rr >> 1) & 3)) << 4));
+            if (quarter * 32 + rr < S)
+              *reinterpret_cast<uint4*>(static_cast<T*>(a.dqkv) + ((size_t)b * S + quarter * 32 + rr) * 3 * a.H +
+                                        w3 * a.H + h * HD + hf * 32 + ch * 8) = v;
+          }
+        }
+        __syncwarp();
       }
     }
     if (a.ctx_tma && lane == 0) bulk_wait_all();
