@@ -1283,7 +1283,9 @@ __global__ void __launch_bounds__(kPFwdThreads, 1)
 // Warps 2-9 (softmax) turn item n's S and dPd into Pd and dS while warps
 // 14-21 (epilogue) drain item n-1's dV, dK, dQ, and the MMA issuer puts item
 // n+1's S and dPd ahead of item n's gradient products: the tensor core, the
-// softmax and the epilogue each work on a different item.  Each epilogue warp
+// softmax and the epilogue each work on a different item.  dV, dK and dQ each
+// have their own full/free barrier pair, so each product starts as soon as
+// the epilogue has read its accumulator.  Each epilogue warp
 // stages its rows through a box of its own (dQ, dK, dV in turn, each leaving
 // by TMA store).
 constexpr int kPBwdThreads = 704;                        // 0 TMA, 1 MMA, 2-9 softmax, 10-13 helpers, 14-21 epilogue
@@ -1305,8 +1307,8 @@ __global__ void __launch_bounds__(kPBwdThreads, 1)
   uint8_t* sstage = saux + 2 * kPBwdAux;
   uint64_t* bar = reinterpret_cast<uint64_t*>(sstage + kPBwdStage);
   uint64_t *in_full = bar, *in_empty = bar + 2, *s_full = bar + 4, *s_free = bar + 5, *ds_full = bar + 6,
-           *g_full = bar + 7, *g_free = bar + 8, *aux_full = bar + 9, *aux_free = bar + 11;
-  uint32_t* tslot = reinterpret_cast<uint32_t*>(bar + 13);
+           *aux_full = bar + 7, *aux_free = bar + 9, *g_full = bar + 11, *g_free = bar + 14;
+  uint32_t* tslot = reinterpret_cast<uint32_t*>(bar + 17);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int S = a.S;
@@ -1321,8 +1323,10 @@ __global__ void __launch_bounds__(kPBwdThreads, 1)
     mbar_init(s_full, 1);
     mbar_init(s_free, kSoftThreads);
     mbar_init(ds_full, kSoftThreads);
-    mbar_init(g_full, 1);
-    mbar_init(g_free, kSoftThreads);
+    for (int q = 0; q < 3; ++q) {
+      mbar_init(&g_full[q], 1);
+      mbar_init(&g_free[q], kSoftThreads);
+    }
     fence_barrier_init();
   }
   if (warp == 1) tmem_alloc(tslot, 512);
@@ -1378,33 +1382,56 @@ __global__ void __launch_bounds__(kPBwdThreads, 1)
         const uint32_t aQ = smem_u32(sm + j * 4 * TB), aK = aQ + TB, adO = aQ + 3 * TB;
         if (!(ok = mbar_wait(ds_full, n & 1, a.err, 64))) break;
         if (n + 1 < my_items && !(ok = mma_s(n + 1))) break;
-        // dV, dK, dQ TMEM free once the epilogue of item n-1 read it
-        if (!(ok = mbar_wait(g_free, (n & 1) ^ 1, a.err, 65))) break;
+        // dV, dK, dQ one by one, each as soon as the epilogue of item n-1
+        // has read that accumulator (g_free[0..2]), each with its own commit
+        if (!(ok = mbar_wait(&g_free[0], (n & 1) ^ 1, a.err, 65))) break;
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < TILE / 16; ++kk) mma_f16(tdV, dmn_pair(aPd, kk), dmn_tile(adO, kk), id_mm, kk > 0);
+        mma_commit(&g_full[0]);
+        if (!(ok = mbar_wait(&g_free[1], (n & 1) ^ 1, a.err, 72))) break;
+        tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < TILE / 16; ++kk) mma_f16(tdK, dmn_pair(adS, kk), dmn_tile(aQ, kk), id_mm, kk > 0);
+        mma_commit(&g_full[1]);
+        if (!(ok = mbar_wait(&g_free[2], (n & 1) ^ 1, a.err, 73))) break;
+        tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < TILE / 16; ++kk) mma_f16(tdQ, dk_pair(adS, kk), dmn_tile(aK, kk), id_km, kk > 0);
-        mma_commit(g_full);
+        mma_commit(&g_full[2]);
         mma_commit(&in_empty[j]);
       }
     }
   } else if (warp >= 10 && warp < 14) {
-    // per item: keep bits, mask row, lse2 and D of every query row
+    // per item: keep bits, mask row, lse2 and D of every query row.  Every
+    // global load of an item (keep bits, mask, LSE, O) is issued before the
+    // wait for its shared-memory slot, so their latencies overlap one another
+    // and the wait.
     const int r = threadIdx.x - 320;
+    const int ch = lane & 7, sub = lane >> 3, r0 = (warp - 10) * 32;
+    const bool qv = r < S;
     int n = 0;
     for (int it = blockIdx.x; it < nitems; it += gridDim.x, ++n) {
       const int j = n & 1;
+      const int b = it / a.nh, h = it - (it / a.nh) * a.nh;
+      uint4 kb = make_uint4(0u, 0u, 0u, 0u);
+      if (a.drop.thr && a.keep) kb = __ldg(reinterpret_cast<const uint4*>(a.keep + ((size_t)it * 128 + r) * 16));
+      const float mv = qv && a.mask ? a.mask[(size_t)b * S + r] : 0.0f;
+      const float lv = qv ? a.lse[(size_t)it * S + r] : 0.0f;
+      // O for D = rowsum(dO * O) with whole-line loads: 8 lanes per 128-byte
+      // row, 4 rows per load, 32 rows per warp
+      const T* obase = static_cast<const T*>(a.ctx_in) + (size_t)b * S * a.H + h * HD + ch * 8;
+      Raw8<T> o8[8];
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        const int rr = r0 + k * 4 + sub;
+        o8[k] = rr < S ? raw8_load<T>(obase + (size_t)rr * a.H) : raw8_zero<T>();
+      }
       uint8_t* ax = saux + j * kPBwdAux;
       float* smask = reinterpret_cast<float*>(ax + 2048);
       if (!mbar_wait(&aux_free[j], ((n >> 1) & 1) ^ 1, a.err, 69)) break;
-      if (a.drop.thr && a.keep) {
-        // the forward's keep bits of this item
-        *reinterpret_cast<uint4*>(ax + r * 16) =
-            __ldg(reinterpret_cast<const uint4*>(a.keep + ((size_t)it * 128 + r) * 16));
-      } else if (a.drop.thr) {
+      if (a.drop.thr && !a.keep) {
+        // no stored forward bits: draw them again
         const uint64_t e8 = (((uint64_t)it * S + (uint64_t)r) * (uint64_t)S) >> 3;
         uint32_t w[4];
 #pragma unroll
@@ -1414,40 +1441,27 @@ __global__ void __launch_bounds__(kPBwdThreads, 1)
           for (int g = 0; g < 4; ++g) v |= dropout_bits8(a.drop, 0, e8 + (uint64_t)(q * 4 + g)) << (8 * g);
           w[q] = v;
         }
-        *reinterpret_cast<uint4*>(ax + r * 16) = make_uint4(w[0], w[1], w[2], w[3]);
+        kb = make_uint4(w[0], w[1], w[2], w[3]);
       }
-      const int b = it / a.nh, h = it - (it / a.nh) * a.nh;
-      const bool qv = r < S;
-      smask[r] = qv ? (a.mask ? a.mask[(size_t)b * S + r] * kLog2e : 0.0f) : -INFINITY;
-      smask[128 + r] = qv ? a.lse[(size_t)it * S + r] * kLog2e : INFINITY;
-      // D = rowsum(dO * O): O from global memory with whole-line loads (8
-      // lanes per 128-byte row, 4 rows per load, 32 rows per warp), then dO
-      // from the item's shared tile, the 8 lanes of a row reduced by shuffles
-      {
-        const int ch = lane & 7, sub = lane >> 3, r0 = (warp - 10) * 32;
-        const T* obase = static_cast<const T*>(a.ctx_in) + (size_t)b * S * a.H + h * HD + ch * 8;
-        Raw8<T> o8[8];
+      if (a.drop.thr) *reinterpret_cast<uint4*>(ax + r * 16) = kb;
+      smask[r] = qv ? mv * kLog2e : -INFINITY;
+      smask[128 + r] = qv ? lv * kLog2e : INFINITY;
+      // D: dO from the item's shared tile, the 8 lanes of a row reduced by shuffles
+      if (!mbar_wait(&in_full[j], (n >> 1) & 1, a.err, 70)) break;
+      const uint8_t* dtile = sm + j * 4 * TB + 3 * TB;
 #pragma unroll
-        for (int k = 0; k < 8; ++k) {
-          const int rr = r0 + k * 4 + sub;
-          o8[k] = rr < S ? raw8_load<T>(obase + (size_t)rr * a.H) : raw8_zero<T>();
-        }
-        if (!mbar_wait(&in_full[j], (n >> 1) & 1, a.err, 70)) break;
-        const uint8_t* dtile = sm + j * 4 * TB + 3 * TB;
+      for (int k = 0; k < 8; ++k) {
+        const int rr = r0 + k * 4 + sub;
+        float x[8], y[8];
+        load8<T>(reinterpret_cast<const T*>(dtile + rr * 128 + ((ch ^ (rr & 7)) << 4)), x);
+        raw8_unpack<T>(o8[k], y);
+        float d = 0.0f;
 #pragma unroll
-        for (int k = 0; k < 8; ++k) {
-          const int rr = r0 + k * 4 + sub;
-          float x[8], y[8];
-          load8<T>(reinterpret_cast<const T*>(dtile + rr * 128 + ((ch ^ (rr & 7)) << 4)), x);
-          raw8_unpack<T>(o8[k], y);
-          float d = 0.0f;
-#pragma unroll
-          for (int t = 0; t < 8; ++t) d = fmaf(x[t], y[t], d);
-          d += __shfl_xor_sync(0xffffffffu, d, 1);
-          d += __shfl_xor_sync(0xffffffffu, d, 2);
-          d += __shfl_xor_sync(0xffffffffu, d, 4);
-          if (ch == 0) smask[256 + rr] = rr < S ? d : 0.0f;
-        }
+        for (int t = 0; t < 8; ++t) d = fmaf(x[t], y[t], d);
+        d += __shfl_xor_sync(0xffffffffu, d, 1);
+        d += __shfl_xor_sync(0xffffffffu, d, 2);
+        d += __shfl_xor_sync(0xffffffffu, d, 4);
+        if (ch == 0) smask[256 + rr] = rr < S ? d : 0.0f;
       }
       mbar_arrive(&aux_full[j]);
     }
@@ -1475,7 +1489,8 @@ __global__ void __launch_bounds__(kPBwdThreads, 1)
       const float Di = smask[256 + r];
       if (!mbar_wait_warp(s_full, n & 1, a.err, 67)) break;
       // the previous item's products have read its Pd and dS
-      if (n > 0 && !mbar_wait_warp(g_full, (n - 1) & 1, a.err, 71)) break;
+      // (dQ, the last of them, is done: MMAs complete in issue order)
+      if (n > 0 && !mbar_wait_warp(&g_full[2], (n - 1) & 1, a.err, 71)) break;
       tc_fence_after();
 #pragma unroll 1
       for (int c = 0; c < 4; ++c) {
@@ -1531,16 +1546,17 @@ __global__ void __launch_bounds__(kPBwdThreads, 1)
     int n = 0;
     for (int it = blockIdx.x; it < nitems; it += gridDim.x, ++n) {
       const int b = it / a.nh, h = it - b * a.nh;
-      if (!mbar_wait_warp(g_full, n & 1, a.err, 68)) break;
-      tc_fence_after();
+      // dV, dK, dQ in the order the MMA issuer produces them (w3 = 2, 1, 0),
+      // each accumulator handed back right after its read
+      bool ok = true;
 #pragma unroll 1
-      for (int w3 = 0; w3 < 3; ++w3) {
+      for (int w3 = 2; w3 >= 0; --w3) {
+        if (!(ok = mbar_wait_warp(&g_full[2 - w3], n & 1, a.err, 68))) break;
+        tc_fence_after();
         float x[32];
         tmem_ld32(tdQ - 64 * w3 + lo + hf * 32, x);
-        if (w3 == 2) {
-          tc_fence_before();
-          mbar_arrive(g_free);
-        }
+        tc_fence_before();
+        mbar_arrive(&g_free[2 - w3]);
         if (w3 < 2) {
 #pragma unroll
           for (int c = 0; c < 32; ++c) x[c] *= a.scale;
@@ -1560,30 +1576,13 @@ __global__ void __launch_bounds__(kPBwdThreads, 1)
           bulk_commit();
         }
         if (a.colsum) {
-          // QKV bias gradient fused in: column sums of the stored values over
-          // this warp's rows inside the sequence.  Lane l sums columns 2p,
-          // 2p+1 (p = l % 16) over rows 16*(l / 16) .. +15 (the upper half in
-          // the other bank half's row order), then the halves
-          const int p = lane & 15, rh = lane >> 4;
-          float s0 = 0.0f, s1 = 0.0f;
-#pragma unroll 4
-          for (int i = 0; i < 16; ++i) {
-            const int rr = rh * 16 + (i ^ rh);
-            if (quarter * 32 + rr < S) {
-              const uint32_t w = *reinterpret_cast<const uint32_t*>(
-                  stg + rr * 64 + ((((p >> 2) ^ ((rr >> 1) & 3))) << 4) + (p & 3) * 4);
-              const T* hv = reinterpret_cast<const T*>(&w);
-              s0 += to_f(hv[0]);
-              s1 += to_f(hv[1]);
-            }
-          }
-          s0 += __shfl_xor_sync(0xffffffffu, s0, 16);
-          s1 += __shfl_xor_sync(0xffffffffu, s1, 16);
-          float* cs = a.colsum + (size_t)(b * 4 + quarter) * 3 * a.H + w3 * a.H + h * HD + hf * 32;
-          if (lane < 16) {
-            cs[2 * p] = s0;
-            cs[2 * p + 1] = s1;
-          }
+          // QKV bias gradient fused in: column sums of the stored (rounded)
+          // values over this warp's rows inside the sequence, by a shuffle
+          // reduction in registers (shared memory is the contended path here)
+          const bool rv = quarter * 32 + lane < S;
+#pragma unroll
+          for (int c = 0; c < 32; ++c) x[c] = rv ? round_f<T>(x[c]) : 0.0f;
+          a.colsum[(size_t)(b * 4 + quarter) * 3 * a.H + w3 * a.H + h * HD + hf * 32 + lane] = warp_colsum32(x);
         }
         if (!tma) {
           // rows r of the box: query r for dQ, key r for dK and dV; 4 lanes
@@ -1600,6 +1599,7 @@ __global__ void __launch_bounds__(kPBwdThreads, 1)
         }
         __syncwarp();
       }
+      if (!ok) break;
     }
     if (a.ctx_tma && lane == 0) bulk_wait_all();
     __syncwarp();
