@@ -1032,6 +1032,13 @@ __global__ void __launch_bounds__(kPFwdThreads, 1)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int S = a.S;
   const int nitems = a.B * a.nh;
+  if (threadIdx.x == 32) {
+    // kernel parameters, not the previous kernel's output
+    prefetch_tensormap(&tq);
+    prefetch_tensormap(&tk);
+    prefetch_tensormap(&tv);
+    if (a.ctx_tma) prefetch_tensormap(&tctx);
+  }
   if (threadIdx.x == 0) {
     for (int i = 0; i < kPFwdIn; ++i) {
       mbar_init(&in_full[i], 1);
@@ -1313,6 +1320,14 @@ __global__ void __launch_bounds__(kPBwdThreads, 1)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int S = a.S;
   const int nitems = a.B * a.nh;
+  if (threadIdx.x == 32) {
+    // kernel parameters, not the previous kernel's output
+    prefetch_tensormap(&tq);
+    prefetch_tensormap(&tk);
+    prefetch_tensormap(&tv);
+    prefetch_tensormap(&tdo);
+    if (a.ctx_tma) prefetch_tensormap(&tdqkv);
+  }
   if (threadIdx.x == 0) {
     for (int j = 0; j < 2; ++j) {
       mbar_init(&in_full[j], 1);

@@ -554,6 +554,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
   const uint32_t rank = cluster_ctarank();
   const bool leader = rank == 0;
   int* const err = g0.err;
+  if (threadIdx.x == 32) {
+    // the tensor maps are kernel parameters, not the previous kernel's
+    // output: fetch them while the setup and the dependency wait run
+    prefetch_tensormap(&tmA0);
+    prefetch_tensormap(&tmB0);
+    prefetch_tensormap(&om0.out);
+    if (sch.table) {
+      prefetch_tensormap(&tmA1);
+      prefetch_tensormap(&tmB1);
+      prefetch_tensormap(&om1.out);
+    }
+  }
   if (threadIdx.x == 0) {
     for (int s = 0; s < kPairStages; ++s) {
       mbar_init(&full[s], 1);
@@ -576,12 +588,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
 
   if (warp == 0) {
     if (lane == 0) {
-      prefetch_tensormap(&tmA0);
-      prefetch_tensormap(&tmB0);
-      if (sch.table) {
-        prefetch_tensormap(&tmA1);
-        prefetch_tensormap(&tmB1);
-      }
       int s = 0;
       uint32_t ph = 0;
       bool ok = true;
