@@ -448,33 +448,17 @@ __device__ __forceinline__ bool pair_epilogue_tile(const OutMaps& om, const TcAr
       }
       if constexpr (epi_sums_columns(KIND) && SW == 32) {
         // bias gradient of the FFN1 Linear fused in: column sums of the
-        // stored (rounded) values of this warp's 32 rows, read back from the
-        // staging box: lane l sums columns 2p, 2p+1 (p = l % 16) over rows
-        // 16*(l / 16) .. +15 (the upper half in the other bank half's row
-        // order), then the two halves
+        // stored (rounded) values of this warp's 32 rows, by a shuffle
+        // reduction in registers (a read-back from the staging box instead
+        // made the dW2|dU launch 3.5 us slower: it competes with the main
+        // loop for shared-memory bandwidth)
         if (e.colsum) {
-          __syncwarp();
-          const int p = lane & 15, rh = lane >> 4;
-          float s0 = 0.0f, s1 = 0.0f;
+          float cs[32];
 #pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            const int rr = rh * 16 + (i ^ rh);
-            if (mrow0 + rr < g.M) {
-              const uint32_t w = *reinterpret_cast<const uint32_t*>(
-                  sb0 + rr * 64 + ((((p >> 2) ^ ((rr >> 1) & 3))) << 4) + (p & 3) * 4);
-              const T* hv = reinterpret_cast<const T*>(&w);
-              s0 += to_f(hv[0]);
-              s1 += to_f(hv[1]);
-            }
-          }
-          s0 += __shfl_xor_sync(0xffffffffu, s0, 16);
-          s1 += __shfl_xor_sync(0xffffffffu, s1, 16);
-          const int col = nbase + c0 + 2 * p;
-          float* cs = e.colsum + (size_t)((mb * 2 + rank) * 4 + quarter) * g.N;
-          if (lane < 16) {
-            if (col < g.N) cs[col] = s0;
-            if (col + 1 < g.N) cs[col + 1] = s1;
-          }
+          for (int i = 0; i < 32; ++i) cs[i] = (mrow && nbase + c0 + i < g.N) ? round_f<T>(v[i]) : 0.0f;
+          const float tot = warp_colsum32(cs);
+          const int col = nbase + c0 + lane;
+          if (col < g.N) e.colsum[(size_t)((mb * 2 + rank) * 4 + quarter) * g.N + col] = tot;
         }
       }
     }
