@@ -1119,11 +1119,16 @@ __global__ void __launch_bounds__(kPFwdThreads, 1)
     int n = 0;
     for (int it = blockIdx.x; it < nitems; it += gridDim.x, ++n) {
       const int j = n & 1;
+      // the item's global loads go out before the wait for its slot
+      const bool ready = a.drop.thr && a.keep_ready;
+      uint4 kb = make_uint4(0u, 0u, 0u, 0u);
+      if (ready) kb = __ldg(reinterpret_cast<const uint4*>(a.keep + ((size_t)it * 128 + r) * 16));
+      const int b = it / a.nh;
+      const float mv = r < S && a.mask ? a.mask[(size_t)b * S + r] : 0.0f;
       if (!mbar_wait(&aux_free[j], ((n >> 1) & 1) ^ 1, a.err, 58)) break;
-      if (a.drop.thr && a.keep_ready) {
+      if (ready) {
         // drawn ahead of this kernel (by the LayerNorm forward before it)
-        *reinterpret_cast<uint4*>(sbits + j * kPFwdBits + r * 16) =
-            __ldg(reinterpret_cast<const uint4*>(a.keep + ((size_t)it * 128 + r) * 16));
+        *reinterpret_cast<uint4*>(sbits + j * kPFwdBits + r * 16) = kb;
       } else if (a.drop.thr) {
         const uint64_t e8 = (((uint64_t)it * S + (uint64_t)r) * (uint64_t)S) >> 3;
         uint32_t w[4];
@@ -1138,8 +1143,7 @@ __global__ void __launch_bounds__(kPFwdThreads, 1)
         *reinterpret_cast<uint4*>(sbits + j * kPFwdBits + r * 16) = kv;
         if (a.keep) *reinterpret_cast<uint4*>(a.keep + ((size_t)it * 128 + r) * 16) = kv;
       }
-      const int b = it / a.nh;
-      smask[j * 128 + r] = r < S ? (a.mask ? a.mask[(size_t)b * S + r] * kLog2e : 0.0f) : -INFINITY;
+      smask[j * 128 + r] = r < S ? mv * kLog2e : -INFINITY;
       mbar_arrive(&aux_full[j]);
     }
   } else {
