@@ -317,12 +317,11 @@ __global__ void __launch_bounds__(kLThreads, 1)
       bool ok = true;
       for (int j = 0; j < nt; ++j, ++g) {
         const int as = g & 1;
-        if (!(ok = mbar_wait(&aux_free[as], ((g >> 1) & 1) ^ 1, a.err, 87))) break;
-        uint8_t* ax = saux + as * kLAux;
         const int k0 = j * TILE;
+        // the tile's bits and mask value before the wait for the slot
+        const uint64_t e8 = (((uint64_t)bh * S + (uint64_t)(q0 + r)) * (uint64_t)S + (uint64_t)k0) >> 3;
+        uint32_t w[4] = {0u, 0u, 0u, 0u};
         if (a.drop.thr) {
-          const uint64_t e8 = (((uint64_t)bh * S + (uint64_t)(q0 + r)) * (uint64_t)S + (uint64_t)k0) >> 3;
-          uint32_t w[4];
 #pragma unroll
           for (int q = 0; q < 4; ++q) {
             uint32_t v = 0;
@@ -330,6 +329,12 @@ __global__ void __launch_bounds__(kLThreads, 1)
             for (int gg = 0; gg < 4; ++gg) v |= dropout_bits8(a.drop, 0, e8 + (uint64_t)(q * 4 + gg)) << (8 * gg);
             w[q] = v;
           }
+        }
+        const int key = k0 + r;
+        const float mv = key < S ? (a.mask ? __ldg(a.mask + (size_t)b * S + key) * kLog2e : 0.0f) : -INFINITY;
+        if (!(ok = mbar_wait(&aux_free[as], ((g >> 1) & 1) ^ 1, a.err, 87))) break;
+        uint8_t* ax = saux + as * kLAux;
+        if (a.drop.thr) {
           *reinterpret_cast<uint4*>(ax + r * 16) = make_uint4(w[0], w[1], w[2], w[3]);
           if (a.keep && row_ok) {
             // 16 bytes when they are 16-byte aligned (S % 128 == 0), else words or bytes
@@ -344,9 +349,7 @@ __global__ void __launch_bounds__(kLThreads, 1)
             }
           }
         }
-        const int key = k0 + r;
-        reinterpret_cast<float*>(ax + 2048)[r] =
-            key < S ? (a.mask ? a.mask[(size_t)b * S + key] * kLog2e : 0.0f) : -INFINITY;
+        reinterpret_cast<float*>(ax + 2048)[r] = mv;
         mbar_arrive(&aux_full[as]);
       }
       if (!ok) break;
@@ -497,26 +500,33 @@ constexpr int kBLKvSmem = 4 * TB + 4 * TB + 4 * TB + 2 * kBLAux + 1024 + 256;   
 constexpr int kBLQSmem = 4 * TB + 4 * TB + 2 * TB + 2 * kBLAux + 1024 + 256;    // Q/dO x2, K/V x2, dS pair
 
 // Helper-warp staging of one (query tile q0, key tile k0) pair of item bh:
-// lse2, D and the 16 keep-bit bytes of query row q0 + r, and the mask of key k0 + r.
-__device__ __forceinline__ void bl_stage_aux(const AttnTc& a, uint8_t* ax, int bh, int b, int q0, int k0, int r) {
+// lse2, D and the 16 keep-bit bytes of query row q0 + r, and the mask of key
+// k0 + r.  bl_load_aux issues every global load (before the wait for the
+// shared-memory slot, so the latencies overlap one another and the wait),
+// bl_store_aux writes the slot.
+struct BlAux {
+  uint4 kb;
+  float mv, lv, dv;
+};
+__device__ __forceinline__ BlAux bl_load_aux(const AttnTc& a, int bh, int b, int q0, int k0, int r) {
   const int S = a.S;
-  float* smask = reinterpret_cast<float*>(ax + 2048);
   const int q = q0 + r;
   const bool qv = q < S;
-  uint4 kb = make_uint4(~0u, ~0u, ~0u, ~0u);
+  BlAux x;
+  x.kb = make_uint4(~0u, ~0u, ~0u, ~0u);
   if (a.drop.thr) {
     if (!qv) {
-      kb = make_uint4(0u, 0u, 0u, 0u);
+      x.kb = make_uint4(0u, 0u, 0u, 0u);
     } else {
       const uint64_t e8 = (((uint64_t)bh * S + (uint64_t)q) * (uint64_t)S + (uint64_t)k0) >> 3;
       if (a.keep) {
         if ((e8 & 15) == 0) {
-          kb = __ldg(reinterpret_cast<const uint4*>(a.keep + e8));
+          x.kb = __ldg(reinterpret_cast<const uint4*>(a.keep + e8));
         } else {
           uint32_t w[4] = {0u, 0u, 0u, 0u};
 #pragma unroll
           for (int t = 0; t < 16; ++t) w[t >> 2] |= (uint32_t)__ldg(a.keep + e8 + t) << (8 * (t & 3));
-          kb = make_uint4(w[0], w[1], w[2], w[3]);
+          x.kb = make_uint4(w[0], w[1], w[2], w[3]);
         }
       } else {
         uint32_t w[4];
@@ -527,15 +537,22 @@ __device__ __forceinline__ void bl_stage_aux(const AttnTc& a, uint8_t* ax, int b
           for (int gg = 0; gg < 4; ++gg) v |= dropout_bits8(a.drop, 0, e8 + (uint64_t)(qq * 4 + gg)) << (8 * gg);
           w[qq] = v;
         }
-        kb = make_uint4(w[0], w[1], w[2], w[3]);
+        x.kb = make_uint4(w[0], w[1], w[2], w[3]);
       }
     }
   }
-  *reinterpret_cast<uint4*>(ax + r * 16) = kb;
   const int key = k0 + r;
-  smask[r] = key < S ? (a.mask ? a.mask[(size_t)b * S + key] * kLog2e : 0.0f) : -INFINITY;
-  smask[128 + r] = qv ? a.lse[(size_t)bh * S + q] * kLog2e : INFINITY;
-  smask[256 + r] = qv ? a.dvec[(size_t)bh * S + q] : 0.0f;
+  x.mv = key < S ? (a.mask ? __ldg(a.mask + (size_t)b * S + key) * kLog2e : 0.0f) : -INFINITY;
+  x.lv = qv ? __ldg(a.lse + (size_t)bh * S + q) * kLog2e : INFINITY;
+  x.dv = qv ? __ldg(a.dvec + (size_t)bh * S + q) : 0.0f;
+  return x;
+}
+__device__ __forceinline__ void bl_store_aux(uint8_t* ax, int r, const BlAux& x) {
+  float* smask = reinterpret_cast<float*>(ax + 2048);
+  *reinterpret_cast<uint4*>(ax + r * 16) = x.kb;
+  smask[r] = x.mv;
+  smask[128 + r] = x.lv;
+  smask[256 + r] = x.dv;
 }
 
 // Softmax-side work of one (query tile, key tile) pair for one thread: query
@@ -744,8 +761,9 @@ __global__ void __launch_bounds__(kBLThreads, 1)
       if (masked(b, j)) continue;
       for (int i = 0; i < nq; ++i, ++g) {
         const int as = g & 1;
+        const BlAux x = bl_load_aux(a, bh, b, i * TILE, j * TILE, r);
         if (!(ok = mbar_wait(&aux_free[as], ((g >> 1) & 1) ^ 1, a.err, 108))) break;
-        bl_stage_aux(a, saux + as * kBLAux, bh, b, i * TILE, j * TILE, r);
+        bl_store_aux(saux + as * kBLAux, r, x);
         mbar_arrive(&aux_full[as]);
       }
     }
@@ -939,8 +957,9 @@ __global__ void __launch_bounds__(kBLThreads, 1)
       const int nk = bl_key_tiles(a, b, nk_all);
       for (int j = 0; j < nk; ++j, ++g) {
         const int as = g & 1;
+        const BlAux x = bl_load_aux(a, bh, b, i * TILE, j * TILE, r);
         if (!(ok = mbar_wait(&aux_free[as], ((g >> 1) & 1) ^ 1, a.err, 128))) break;
-        bl_stage_aux(a, saux + as * kBLAux, bh, b, i * TILE, j * TILE, r);
+        bl_store_aux(saux + as * kBLAux, r, x);
         mbar_arrive(&aux_full[as]);
       }
     }
