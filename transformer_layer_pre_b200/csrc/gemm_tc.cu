@@ -266,15 +266,16 @@ __global__ void __launch_bounds__(kThreads, 1)
 // into shared memory (32 KB per 64-wide K block instead of 48 KB).  Commits multicast to both CTAs'
 // barriers; both CTAs' epilogues arrive on the leader's "accumulator empty"
 // barrier.  No TMA multicast is used.
-// Five stages (225 KB of shared memory with the epilogue's staging boxes):
-// measured against four on the layer's GEMMs in isolation, the K = 4096 and
-// 8192 launches gain 5-6 us and the others 1-3 us.
-constexpr int kPairStages = 5;
+// Six stages and one staging box per epilogue warp (225 KB of shared
+// memory): against five stages with two boxes per warp, measured on the
+// layer's GEMMs in isolation, 1-2 us faster per launch (the dW2|dU launch
+// 7.7 us); five stages had been 1-6 us faster than four.
+constexpr int kPairStages = 6;
 constexpr int kPairStageBytes = 2 * 128 * BK * 2;                  // A half + B half, 32 KB
 constexpr int kPairEpiWarps = 16;
 constexpr int kPairThreads = 64 + 32 * kPairEpiWarps;
 constexpr int kStageOut = 2048;                                    // one 32-row x 64-byte store box
-constexpr int kPairOutBytes = kPairEpiWarps * 2 * kStageOut;       // two staging buffers per epilogue warp
+constexpr int kPairOutBytes = kPairEpiWarps * kStageOut;           // one staging box per epilogue warp
 constexpr int kPairSmem = kPairStages * kPairStageBytes + kPairOutBytes + 1024 + 256;
 static_assert(kPairSmem <= 227 * 1024, "the pair kernel's shared memory exceeds a CTA's maximum");
 
@@ -332,12 +333,14 @@ struct SchedIter {
 };
 
 // Epilogue of one tile for epilogue warp (quarter, part) of this CTA:
-// TMEM accumulator `acc` -> fused epilogue -> staging box -> TMA store.
+// TMEM accumulator `acc` -> fused epilogue -> staging box -> TMA store.  The
+// warp has one staging box (32 rows x 64 bytes), reused chunk by chunk: each
+// write to it first waits until the box's previous store has read it.
 template <typename T, int KIND>
 __device__ __forceinline__ bool pair_epilogue_tile(const OutMaps& om, const TcArgs& g, const EpiParams& e, int t,
                                                    int rank, int quarter, int part, int lane, uint32_t tmem, int acc,
                                                    uint32_t aph, uint64_t* tfull,
-                                                   const uint32_t (&tempty_leader)[2], uint8_t* stage0, int& nbuf) {
+                                                   const uint32_t (&tempty_leader)[2], uint8_t* box) {
   constexpr int BN = 256;
   constexpr int HALF = 128;
   constexpr int CW = BN / (kPairEpiWarps / 4);              // 64 columns per warp
@@ -352,32 +355,32 @@ __device__ __forceinline__ bool pair_epilogue_tile(const OutMaps& om, const TcAr
   const int nbase = nb * BN + part * CW;
   const bool mrow = m < g.M;
   // The epilogue's (M, N) input (residual, U or GELU'(U)) of this warp's 32
-  // rows x 64 columns is loaded row-contiguously (8 lanes per 128-byte row
-  // segment, 4 rows per load) into the warp's two staging boxes, in the
-  // swizzled layout the outputs use; each lane then reads its own row from
-  // there and the outputs overwrite it in place.  (Row-per-lane 16-byte
-  // loads touched 32 lines per instruction.)
+  // rows x 64 columns is loaded row-contiguously (4 lanes per 64-byte row
+  // segment, 8 rows per load) while the main loop runs: its first 32 columns
+  // into the box, in the swizzled layout the outputs use, its second 32 into
+  // registers, copied into the box once the first chunk's store has read it.
+  // Each lane reads its own row from the box and the outputs overwrite it in
+  // place.  (Row-per-lane 16-byte loads touched 32 lines per instruction.)
   static_assert(!EpiAux<KIND>::kNeeds || (NOUT == 1 && OUT_ES == 2 && CW == 2 * SW), "aux staging layout");
   bool aux_on = false;
+  uint4 aux_hi[4];
+  const int ach = lane & 3, arow = lane >> 2;              // 16-byte chunk of the row segment, first row
   if constexpr (EpiAux<KIND>::kNeeds) {
     const T* ap = static_cast<const T*>(epi_aux_ptr(e, epi_base(KIND)));
     aux_on = ap != nullptr;
     if (aux_on) {
-      if (lane == 0) bulk_wait_read<0>();   // both boxes free: earlier stores from them have read them
+      if (lane == 0) bulk_wait_read<0>();   // the box's last store has read it
       __syncwarp();
-      const int ch = lane & 7;              // 16-byte chunk of the row's 128 bytes
-      const int n = nbase + ch * 8;
-      uint4 v[8];
 #pragma unroll
-      for (int k = 0; k < 8; ++k) {
-        const int mm = mrow0 + k * 4 + (lane >> 3);
-        v[k] = (mm < g.M && n < g.N) ? *reinterpret_cast<const uint4*>(ap + (size_t)mm * e.ldo + n)
-                                      : make_uint4(0u, 0u, 0u, 0u);
-      }
-#pragma unroll
-      for (int k = 0; k < 8; ++k) {
-        const int rl = k * 4 + (lane >> 3);   // row within the warp's 32
-        *reinterpret_cast<uint4*>(stage0 + (ch >> 2) * kStageOut + rl * 64 + (((ch & 3) ^ ((rl >> 1) & 3)) << 4)) = v[k];
+      for (int k = 0; k < 4; ++k) {
+        const int rl = arow + 8 * k;        // row within the warp's 32
+        const int mm = mrow0 + rl;
+        const int n0 = nbase + ach * 8, n1 = n0 + SW;
+        const uint4 lo = (mm < g.M && n0 < g.N) ? *reinterpret_cast<const uint4*>(ap + (size_t)mm * e.ldo + n0)
+                                                : make_uint4(0u, 0u, 0u, 0u);
+        aux_hi[k] = (mm < g.M && n1 < g.N) ? *reinterpret_cast<const uint4*>(ap + (size_t)mm * e.ldo + n1)
+                                           : make_uint4(0u, 0u, 0u, 0u);
+        *reinterpret_cast<uint4*>(box + rl * 64 + ((ach ^ ((rl >> 1) & 3)) << 4)) = lo;
       }
       __syncwarp();
     }
@@ -405,30 +408,36 @@ __device__ __forceinline__ bool pair_epilogue_tile(const OutMaps& om, const TcAr
       tc_fence_before();
       mbar_arrive_cluster(tempty_leader[acc]);
     }
-    uint8_t* sb0 = stage0 + (NOUT == 2 ? 0 : nbuf) * kStageOut;
-    uint8_t* sb1 = stage0 + kStageOut;
-    if (!aux_on) {
-      if (lane == 0) {
-        if constexpr (NOUT == 2) bulk_wait_read<0>();
-        else bulk_wait_read<1>();
-      }
+    if (!(aux_on && c0 == 0)) {
+      // the box's previous store has read it (the first chunk's aux load waited already)
+      if (lane == 0) bulk_wait_read<0>();
       __syncwarp();
+    }
+    if constexpr (EpiAux<KIND>::kNeeds) {
+      if (aux_on && c0 == SW) {
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const int rl = arow + 8 * k;
+          *reinterpret_cast<uint4*>(box + rl * 64 + ((ach ^ ((rl >> 1) & 3)) << 4)) = aux_hi[k];
+        }
+        __syncwarp();
+      }
     }
     if constexpr (OUT_ES == 4) {
       // 16 floats = four 16-byte chunks of the 64-byte row
 #pragma unroll
       for (int q = 0; q < 4; ++q)
-        *reinterpret_cast<float4*>(sb0 + lane * 64 + ((q ^ swz) << 4)) =
+        *reinterpret_cast<float4*>(box + lane * 64 + ((q ^ swz) << 4)) =
             make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
     } else {
+      float v2[NOUT == 2 ? SW : 1];
 #pragma unroll
       for (int q = 0; q < SW / 8; ++q) {
         const int n = nbase + c0 + q * 8;
         float* vq = v + q * 8;
-        float v2[8];
         float aux[8];
         if constexpr (EpiAux<KIND>::kNeeds) {
-          if (aux_on) unpack8<T>(*reinterpret_cast<const uint4*>(sb0 + lane * 64 + ((q ^ swz) << 4)), aux);
+          if (aux_on) unpack8<T>(*reinterpret_cast<const uint4*>(box + lane * 64 + ((q ^ swz) << 4)), aux);
           else {
 #pragma unroll
             for (int i = 0; i < 8; ++i) aux[i] = 0.0f;
@@ -442,9 +451,13 @@ __device__ __forceinline__ bool pair_epilogue_tile(const OutMaps& om, const TcAr
           const int j = (c0 >> 3) + q;
           if (kvalid) kb = ((j < 4 ? kpre.x : kpre.y) >> (8 * (j & 3))) & 0xFFu;
         }
-        if (mrow && n < g.N) epi_compute8<T, KIND>(e, m, n, *reinterpret_cast<float(*)[8]>(vq), v2, aux, kb);
-        store8<T>(reinterpret_cast<T*>(sb0 + lane * 64 + ((q ^ swz) << 4)), *reinterpret_cast<float(*)[8]>(vq));
-        if constexpr (NOUT == 2) store8<T>(reinterpret_cast<T*>(sb1 + lane * 64 + ((q ^ swz) << 4)), v2);
+        float w2[8];
+        if (mrow && n < g.N) epi_compute8<T, KIND>(e, m, n, *reinterpret_cast<float(*)[8]>(vq), w2, aux, kb);
+        store8<T>(reinterpret_cast<T*>(box + lane * 64 + ((q ^ swz) << 4)), *reinterpret_cast<float(*)[8]>(vq));
+        if constexpr (NOUT == 2) {
+#pragma unroll
+          for (int i = 0; i < 8; ++i) v2[q * 8 + i] = w2[i];
+        }
       }
       if constexpr (epi_sums_columns(KIND) && SW == 32) {
         // bias gradient of the FFN1 Linear fused in: column sums of the
@@ -461,6 +474,21 @@ __device__ __forceinline__ bool pair_epilogue_tile(const OutMaps& om, const TcAr
           if (col < g.N) e.colsum[(size_t)((mb * 2 + rank) * 4 + quarter) * g.N + col] = tot;
         }
       }
+      if constexpr (NOUT == 2) {
+        // the first output leaves, then the second takes the box
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          const int x = nbase + c0;
+          if (mrow0 < g.M && x < g.N) tma_store_2d(&om.out, box, x, mrow0);
+          bulk_commit();
+          bulk_wait_read<0>();
+        }
+        __syncwarp();
+#pragma unroll
+        for (int q = 0; q < SW / 8; ++q)
+          store8<T>(reinterpret_cast<T*>(box + lane * 64 + ((q ^ swz) << 4)), *reinterpret_cast<float(*)[8]>(v2 + q * 8));
+      }
     }
     fence_proxy_async_smem();
     __syncwarp();
@@ -472,19 +500,17 @@ __device__ __forceinline__ bool pair_epilogue_tile(const OutMaps& om, const TcAr
           const int c = x - which * e.hidden;
           const int bb = mrow0 / e.seq, s0 = mrow0 - bb * e.seq;
           const int y = which * om.qkv_heads_rows + (bb * e.heads + (c >> 6)) * e.seq + s0;
-          tma_store_2d(&om.out, sb0, c & 63, y);
+          tma_store_2d(&om.out, box, c & 63, y);
         }
       } else if constexpr (epi_base(KIND) == EPI_F32) {
-        if (mrow0 < g.M && x < g.N) tma_store_2d(&om.out, sb0, x, sp * om.split_rows + mrow0);
+        if (mrow0 < g.M && x < g.N) tma_store_2d(&om.out, box, x, sp * om.split_rows + mrow0);
+      } else if constexpr (NOUT == 2) {
+        if (e.out2 && mrow0 < g.M && x < g.N) tma_store_2d(&om.out2, box, x, mrow0);
       } else if (mrow0 < g.M && x < g.N) {
-        tma_store_2d(&om.out, sb0, x, mrow0);
-        if constexpr (NOUT == 2) {
-          if (e.out2) tma_store_2d(&om.out2, sb1, x, mrow0);
-        }
+        tma_store_2d(&om.out, box, x, mrow0);
       }
       bulk_commit();
     }
-    if constexpr (NOUT == 1) nbuf ^= 1;
   }
   return true;
 }
@@ -663,23 +689,22 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
     // TMA store, so global writes are whole lines.
     const int quarter = warp & 3;
     const int part = (warp - 2) >> 2;
-    uint8_t* stage0 = sout + (warp - 2) * 2 * kStageOut;
+    uint8_t* box = sout + (warp - 2) * kStageOut;
     const uint32_t tempty_leader[2] = {mapa_shared(smem_u32(&tempty[0]), 0), mapa_shared(smem_u32(&tempty[1]), 0)};
     int acc = 0;
     uint32_t aph = 0;
-    int nbuf = 0;
     SchedIter<KA != KB> it(sch, g0, cid, ncl);
     int gi, t;
     while (it.next(gi, t)) {
       bool ok;
       if constexpr (KA == KB)
         ok = pair_epilogue_tile<T, KA>(om0, g0, e0, t, (int)rank, quarter, part, lane, tmem, acc, aph, tfull,
-                                       tempty_leader, stage0, nbuf);
+                                       tempty_leader, box);
       else
         ok = gi ? pair_epilogue_tile<T, KB>(om1, g1, e1, t, (int)rank, quarter, part, lane, tmem, acc, aph, tfull,
-                                            tempty_leader, stage0, nbuf)
+                                            tempty_leader, box)
                 : pair_epilogue_tile<T, KA>(om0, g0, e0, t, (int)rank, quarter, part, lane, tmem, acc, aph, tfull,
-                                            tempty_leader, stage0, nbuf);
+                                            tempty_leader, box);
       if (!ok) break;
       acc ^= 1;
       if (acc == 0) aph ^= 1u;
