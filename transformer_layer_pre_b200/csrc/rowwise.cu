@@ -738,6 +738,7 @@ __global__ void __launch_bounds__(kFinThreads) colsum_finalize_kernel(const __gr
     const size_t step = (size_t)(fg.first[j + 1] - fg.first[j]) * kFinThreads;
     for (size_t i = (size_t)b * kFinThreads + threadIdx.x; i < n4; i += step) {
       float4 sum = p[i];
+#pragma unroll 4
       for (int k = 1; k < nparts; ++k) {
         const float4 v = p[k * st4 + i];
         sum.x += v.x; sum.y += v.y; sum.z += v.z; sum.w += v.w;
@@ -1021,7 +1022,9 @@ void colsum_finalize_list_run(const FinalizeList& fl, cudaStream_t s) {
   fg.first[0] = 0;
   for (int i = 0; i < fl.n; ++i) {
     const FinalizeJob& j = fl.job[i];
-    const int nb = j.stride ? (int)std::min<size_t>(((size_t)j.cols / 4 + kFinThreads - 1) / kFinThreads, 296)
+    // split-K sums: up to four blocks per SM, so a thread's partial loads
+    // come in about one round (the column-sum jobs fill the rest of the wave)
+    const int nb = j.stride ? (int)std::min<size_t>(((size_t)j.cols / 4 + kFinThreads - 1) / kFinThreads, 592)
                             : (j.cols + kFinCols - 1) / kFinCols;
     fg.first[i + 1] = fg.first[i] + std::max(nb, 1);
   }
