@@ -45,6 +45,10 @@ struct GemmDesc {
   // partials to this list (summed by a later colsum_finalize_list_run; the
   // scratch must stay untouched until then) instead of launching the sum
   FinalizeList* defer = nullptr;
+  // B was not written by the kernel launched just before this GEMM on its
+  // stream (a weight, or an activation of an earlier kernel): the tensor-core
+  // kernel then loads its first stages of B before it waits for that kernel
+  bool b_early = false;
 };
 
 enum EpiKind {

@@ -249,16 +249,24 @@ tl_status ensure_buffers(tl_layer* L) {
   return TL_OK;
 }
 
+// A GEMM whose B is a weight: never the output of the kernel before it, so
+// the tensor-core kernel may load B before it waits for that kernel.
 GemmDesc gdesc(tl_layer* L, int M, int N, int K, const void* A, int lda, bool ak, const void* B, int ldb, bool bk) {
-  return GemmDesc{M, N, K, A, lda, ak, B, ldb, bk, nullptr, 0};
+  GemmDesc g{M, N, K, A, lda, ak, B, ldb, bk, nullptr, 0};
+  g.b_early = true;
+  return g;
 }
 
 // A weight-gradient GEMM (float32 out) with split-K scratch `which` (0 W2,
-// 1 W1, 2 Wo, 3 Wqkv) whose split sum joins the closing finalize list.
+// 1 W1, 2 Wo, 3 Wqkv) whose split sum joins the closing finalize list.  Its
+// B is an activation the forward saved (G, the FFN input, ctx, the
+// attention input), not the output of the kernel before it, unless the
+// caller says otherwise (b_early = false).
 GemmDesc wdesc(tl_layer* L, int which, FinalizeList* fin, int M, int N, int K, const void* A, int lda, const void* B,
                int ldb) {
   GemmDesc g{M, N, K, A, lda, false, B, ldb, false, L->splitk[which], L->splitk_floats[which]};
   g.defer = fin;
+  g.b_early = true;
   return g;
 }
 
@@ -608,7 +616,9 @@ tl_status layer_backward(tl_layer* L, const void* x, const void* dy, const tl_we
     // the tensor-core GEMM sums dU's columns in its epilogue (db1)
     const bool fused_db1 = gemm_uses_tensor_cores(dt) != 0;
     if (fused_db1) edu.colsum = slot(db1_slot);
-    const GemmDesc gw2 = wdesc(L, 0, &fin, H, F, T, L->dz2, H, L->g, F);          // dW2 = dZ2^T G
+    GemmDesc gw2 = wdesc(L, 0, &fin, H, F, T, L->dz2, H, L->g, F);                // dW2 = dZ2^T G
+    // recompute mode: G was just rewritten by the GELU launch before this one
+    if (L->opt.gelu_checkpoint) gw2.b_early = false;
     const GemmDesc gdu = gdesc(L, T, F, H, L->dz2, H, true, w->w2, F, false);   // dU = (dZ2 W2) GELU'(U)
     if (L->g != L->big) {
       gemm2(L, gw2, ew2, gdu, edu, s);
