@@ -63,7 +63,6 @@ struct AttnTc {
   const float* dvec;    // precomputed D, or null to compute it in-kernel
   void* dqkv;
   float* colsum;        // fused QKV bias-gradient partials (persistent backward), or null
-  int fuse_dq;
   int ctx_tma;          // persistent kernels: ctx (forward) or dQKV (backward) rows leave by TMA store (S % 32 == 0)
   const int* kv_ext;    // per sequence, one past its last unmasked key (long forward), or null
   int keep_ready;       // persistent forward: the keep bits are already in `keep` (read, not drawn)
@@ -1722,7 +1721,6 @@ AttnTc make_args(int dt, const AttnArgs& a) {
   t.dvec = nullptr;
   t.dqkv = a.dqkv;
   t.colsum = a.colsum;
-  t.fuse_dq = 0;
   t.ctx_tma = 0;
   t.keep = a.keep;
   t.kv_ext = a.mask ? a.kv_ext : nullptr;
@@ -1806,7 +1804,6 @@ void bwd_t(const AttnArgs& a, cudaStream_t s) {
   }
   dvec_launch(t.bf16 ? DT_BF16 : DT_F16, a, s);
   t.dvec = a.dvec;
-  t.fuse_dq = 0;
   static bool lattr = false;
   if (!lattr) {
     cudaFuncSetAttribute(attn_bwd_kv_long<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, kBLKvSmem);
