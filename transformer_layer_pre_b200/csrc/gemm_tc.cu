@@ -614,9 +614,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
       bool have = it.next(gi, t);
       // B of the pair's first tile, when it is not the previous kernel's
       // output (a weight, or an earlier kernel's activation): its first
-      // stages (fresh, so their empty barriers need no wait) go out now.
-      // Measured in the layer step: 0.690 -> 0.653 ms (the eight GEMM
-      // launches 595 -> 553 us), so most of a launch's start was these loads.
+      // stages (fresh, so their empty barriers need no wait) go out now,
+      // riding on the previous kernel's tail.  Measured in the layer step:
+      // 0.690 -> 0.653 ms (the eight GEMM launches 595 -> 553 us); timed
+      // alone, with no kernel before, the launches do not change.
       int pre = 0;
       if (have) {
         const ItemArgs g = item_args(g0, g1, gi);
