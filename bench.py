@@ -346,7 +346,7 @@ def run_ours(args) -> None:
     inp = make_inputs(w)
     T = w.tokens
     layer = Layer(w.batch, w.seq, w.hidden, w.heads, w.ffn, w.attn_dropout, w.hidden_dropout, w.pre_layer_norm,
-                  w.seed, dtype=dt, gelu_checkpoint=w.gelu_checkpoint)
+                  w.seed, dtype=dt, gelu_checkpoint=w.gelu_checkpoint, stochastic_mode=args.stochastic_mode)
     wt = {n: inp.weights[0][n].to(dev) for n in WEIGHT_NAMES}
     mask = None if inp.mask is None else inp.mask.to(dev)
     # gradients are views of one flat buffer: data-parallel ranks average it with one all-reduce
@@ -510,7 +510,7 @@ def run_ours(args) -> None:
             "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": w.dtype, "data": "synthetic (seeded N(0,0.02) weights, N(0,1) x and dY)",
-            "config": dict(workload_config(w), graph=not args.no_graph), "tensor_peak_frac": tensor_frac,
+            "config": dict(workload_config(w), graph=not args.no_graph, stochastic_mode=args.stochastic_mode), "tensor_peak_frac": tensor_frac,
             "tensor_peak_frac_of_burst": tensor_frac_burst,
             "tensor_peak_frac_of_sustained": tensor_frac_sustained,
             "roofline": roofline, "kernel_classes": classes, "cpu_baseline": cpu,
@@ -547,6 +547,8 @@ def main() -> None:
     ap.add_argument("--workload", default=WORKLOAD, choices=sorted(WORKLOADS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-graph", action="store_true", help="launch every kernel eagerly instead of replaying a CUDA graph")
+    ap.add_argument("--stochastic-mode", action="store_true",
+                    help="relaxed determinism: bias, LayerNorm and split-K weight gradients summed with atomics")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

@@ -90,6 +90,18 @@ typedef struct {
                                     1: the tanh approximation 0.5 u (1 + tanh(sqrt(2/pi)
                                     (u + 0.044715 u^3))) ("AI-infra engineers and the
                                     Transformer", section 2.3), forward and backward */
+  int stochastic_mode;           /* 0 (default): every result is bitwise reproducible
+                                    (column sums and split-K weight gradients are summed
+                                    in a fixed order by a closing launch).  1: the
+                                    backward adds them straight into the gradient
+                                    outputs with float32 atomic adds, in arrival order,
+                                    and skips that launch ("DeepSpeed Transformer Kernel
+                                    usage guide", Step 2, stochastic_mode: a little
+                                    faster, not reproducible).  Only the bias and
+                                    LayerNorm gradients, and weight gradients whose K
+                                    (= tokens) is split, may then differ from run to
+                                    run, by float32 summation order; y, dx and every
+                                    other gradient stay bitwise the same as with 0. */
 } tl_options;
 
 /* The twelve parameter tensors, all passed on every call (Step 2: the layer

@@ -60,7 +60,7 @@ def oracle_config(w: Workload, batch: int, philox_offset: int = 0) -> oracle.Lay
 
 
 def run_gpu(inp: Inputs, layer: int = 0, gelu_checkpoint: bool | None = None, normalize_invertible=False,
-            philox_offset: int = 0, keep_x: bool = True) -> dict:
+            philox_offset: int = 0, keep_x: bool = True, stochastic_mode: bool = False) -> dict:
     """Forward + backward of one layer on cuda:0; returns float64 numpy arrays."""
     w = inp.workload
     b = inp.x.shape[0]
@@ -68,7 +68,8 @@ def run_gpu(inp: Inputs, layer: int = 0, gelu_checkpoint: bool | None = None, no
     ck = w.gelu_checkpoint if gelu_checkpoint is None else gelu_checkpoint
     L = Layer(b, w.seq, w.hidden, w.heads, w.ffn, w.attn_dropout, w.hidden_dropout, w.pre_layer_norm, w.seed,
               dtype=TORCH_DT[w.dtype], philox_offset=philox_offset, gelu_checkpoint=ck,
-              normalize_invertible=normalize_invertible, gelu_tanh=w.gelu == "tanh")
+              normalize_invertible=normalize_invertible, gelu_tanh=w.gelu == "tanh",
+              stochastic_mode=stochastic_mode)
     try:
         wt = {n: inp.weights[layer][n].to(dev) for n in WEIGHT_NAMES}
         x = inp.x.to(dev)

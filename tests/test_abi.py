@@ -74,6 +74,7 @@ def test_create_defaults_and_state_errors(lib):
         opt = tlp.Options()
         assert lib.layer_get_options(h, ctypes.byref(opt)) == TL_OK
         assert opt.dtype == 0 and opt.training == 1 and abs(opt.ln_eps - 1e-12) < 1e-18
+        assert opt.stochastic_mode == 0   # bitwise-reproducible by default
         assert lib.layer_workspace_bytes(h) == 0  # nothing allocated before options / forward
         w = tlp._Weights(*([1] * 12))
         st = lib.layer_backward(h, 1, 1, ctypes.byref(w), ctypes.byref(w), 1, None)

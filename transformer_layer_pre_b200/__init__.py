@@ -57,6 +57,7 @@ class Options(ctypes.Structure):
         ("normalize_invertible", ctypes.c_int),
         ("training", ctypes.c_int),
         ("gelu_tanh", ctypes.c_int),
+        ("stochastic_mode", ctypes.c_int),
     ]
 
 
@@ -151,7 +152,7 @@ class Layer:
     def __init__(self, batch, seq, hidden, heads, ffn=0, attn_dropout=0.0, hidden_dropout=0.0,
                  pre_layer_norm=True, seed=1234, dtype=torch.float16, ln_eps=1e-12, philox_offset=0,
                  gelu_checkpoint=False, attn_dropout_checkpoint=False, normalize_invertible=False,
-                 training=True, gelu_tanh=False):
+                 training=True, gelu_tanh=False, stochastic_mode=False):
         self.lib = load_library()
         self.handle = None
         h = ctypes.c_void_p()
@@ -173,6 +174,7 @@ class Layer:
         opt.normalize_invertible = int(normalize_invertible)
         opt.training = int(training)
         opt.gelu_tanh = int(gelu_tanh)
+        opt.stochastic_mode = int(stochastic_mode)
         self._check(self.lib.layer_set_options(self.handle, ctypes.byref(opt)))
 
     def _check(self, st: int) -> None:

@@ -63,6 +63,7 @@ struct AttnTc {
   const float* dvec;    // precomputed D, or null to compute it in-kernel
   void* dqkv;
   float* colsum;        // fused QKV bias-gradient partials (persistent backward), or null
+  int colsum_acc;       // 1: added into row 0 of colsum with atomics (arrival order)
   int ctx_tma;          // persistent kernels: ctx (forward) or dQKV (backward) rows leave by TMA store (S % 32 == 0)
   const int* kv_ext;    // per sequence, one past its last unmasked key (long forward), or null
   int keep_ready;       // persistent forward: the keep bits are already in `keep` (read, not drawn)
@@ -1619,7 +1620,10 @@ __global__ void __launch_bounds__(kPBwdThreads, 1)
           const bool rv = quarter * 32 + lane < S;
 #pragma unroll
           for (int c = 0; c < 32; ++c) x[c] = rv ? round_f<T>(x[c]) : 0.0f;
-          a.colsum[(size_t)(b * 4 + quarter) * 3 * a.H + w3 * a.H + h * HD + hf * 32 + lane] = warp_colsum32(x);
+          const float cs = warp_colsum32(x);
+          const int col = w3 * a.H + h * HD + hf * 32 + lane;
+          if (a.colsum_acc) atomicAdd(a.colsum + col, cs);
+          else a.colsum[(size_t)(b * 4 + quarter) * 3 * a.H + col] = cs;
         }
         if (!tma) {
           // rows r of the box: query r for dQ, key r for dK and dV; 4 lanes
@@ -1721,6 +1725,7 @@ AttnTc make_args(int dt, const AttnArgs& a) {
   t.dvec = nullptr;
   t.dqkv = a.dqkv;
   t.colsum = a.colsum;
+  t.colsum_acc = a.colsum_acc;
   t.ctx_tma = 0;
   t.keep = a.keep;
   t.kv_ext = a.mask ? a.kv_ext : nullptr;

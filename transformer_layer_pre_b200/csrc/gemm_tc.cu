@@ -286,6 +286,7 @@ struct OutMaps {
   CUtensorMap out2;   // EPI_BIAS_GELU's G
   int qkv_heads_rows; // EPI_QKV: rows of one of Q/K/V viewed as (B*heads*S, 64)
   int split_rows;     // EPI_F32: rows between split partials (M rounded up to 256)
+  int reduce_add;     // EPI_F32: 1 = every split adds its tile into the M-row output (TMA reduce-add)
 };
 
 // One GEMM of a pair launch: operand maps, output maps, sizes, epilogue.
@@ -472,7 +473,10 @@ __device__ __forceinline__ bool pair_epilogue_tile(const OutMaps& om, const TcAr
           for (int i = 0; i < 32; ++i) cs[i] = (mrow && nbase + c0 + i < g.N) ? round_f<T>(v[i]) : 0.0f;
           const float tot = warp_colsum32(cs);
           const int col = nbase + c0 + lane;
-          if (col < g.N) e.colsum[(size_t)((mb * 2 + rank) * 4 + quarter) * g.N + col] = tot;
+          if (col < g.N) {
+            if (e.accumulate) atomicAdd(e.colsum + col, tot);
+            else e.colsum[(size_t)((mb * 2 + rank) * 4 + quarter) * g.N + col] = tot;
+          }
         }
       }
       if constexpr (NOUT == 2) {
@@ -504,7 +508,10 @@ __device__ __forceinline__ bool pair_epilogue_tile(const OutMaps& om, const TcAr
           tma_store_2d(&om.out, box, c & 63, y);
         }
       } else if constexpr (epi_base(KIND) == EPI_F32) {
-        if (mrow0 < g.M && x < g.N) tma_store_2d(&om.out, box, x, sp * om.split_rows + mrow0);
+        if (mrow0 < g.M && x < g.N) {
+          if (om.reduce_add) tma_reduce_add_2d(&om.out, box, x, mrow0);
+          else tma_store_2d(&om.out, box, x, sp * om.split_rows + mrow0);
+        }
       } else if constexpr (NOUT == 2) {
         if (e.out2 && mrow0 < g.M && x < g.N) tma_store_2d(&om.out2, box, x, mrow0);
       } else if (mrow0 < g.M && x < g.N) {
@@ -920,8 +927,10 @@ bool build_pair_gemm(PairGemm& P, const GemmDesc& gd, const EpiParams& e, int sp
   const CUtensorMapDataType t16 = bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
   if constexpr (epi_base(KIND) == EPI_F32) {
     // split partials live in a workspace padded to whole 256-row tiles; the
-    // unsplit output is exactly M rows, so clipping keeps stores inside it
-    const uint64_t rows = g.splits > 1 ? (uint64_t)g.splits * om.split_rows : (uint64_t)gd.M;
+    // unsplit output (or the one the splits add into) is exactly M rows, so
+    // clipping keeps stores inside it
+    om.reduce_add = g.splits > 1 && e.accumulate ? 1 : 0;
+    const uint64_t rows = g.splits > 1 && !om.reduce_add ? (uint64_t)g.splits * om.split_rows : (uint64_t)gd.M;
     ok = make_map_t(&om.out, e.out, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, gd.N, rows, e.ldo, 32, 64);
   } else if constexpr (epi_base(KIND) == EPI_QKV) {
     om.qkv_heads_rows = e.tokens * (e.hidden / 64);
@@ -1014,7 +1023,7 @@ struct LaunchKey {
   std::string str() const { return std::string(reinterpret_cast<const char*>(w), n * sizeof(uint64_t)); }
 };
 
-static_assert(sizeof(EpiParams) == 184 && sizeof(GemmDesc) == 80 && sizeof(DropoutParams) == 24,
+static_assert(sizeof(EpiParams) == 192 && sizeof(GemmDesc) == 80 && sizeof(DropoutParams) == 24,
               "a field was added: the launch-cache key must list it");
 
 void key_drop(LaunchKey& k, const DropoutParams& d) {
@@ -1035,7 +1044,7 @@ void key_gemm(LaunchKey& k, const GemmDesc& g, const EpiParams& e, int kind, int
   k.add(e.seq); k.add(e.hidden); k.add(e.head_dim); k.add(e.heads); k.add(e.tokens); k.add(e.gelu_tanh);
   k.addp(e.gen_keep); k.addp(e.gen_keep2); k.add(e.gen_site); k.add(e.gen_n8);
   key_drop(k, e.gen_drop);
-  k.addp(e.colsum);
+  k.addp(e.colsum); k.add(e.accumulate);
 }
 
 std::mutex g_launch_mu;
@@ -1153,7 +1162,7 @@ int run_t(const GemmDesc& g, const EpiParams& e, cudaStream_t s) {
   if (!aligned16(g.A, g.lda) || !aligned16(g.B, g.ldb)) return 2;
   if (e.kind == EPI_F32) {
     const int splits = f32_splits(g);
-    if (splits > 1) {
+    if (splits > 1 && !e.accumulate) {
       EpiParams ep = e;
       ep.out = g.splitk_ws;
       int rc = launch_tc_pair<T, EPI_F32>(g, ep, splits, s);
@@ -1161,7 +1170,7 @@ int run_t(const GemmDesc& g, const EpiParams& e, cudaStream_t s) {
       f32_split_reduce(g, e, splits, s);
       return 0;
     }
-    return launch_tc_pair<T, EPI_F32>(g, e, 1, s);
+    return launch_tc_pair<T, EPI_F32>(g, e, splits, s);   // one split, or splits adding into e.out
   }
   switch (e.kind) {
     case EPI_QKV:
@@ -1196,14 +1205,15 @@ int run2_t(const GemmDesc& ga, const EpiParams& ea, const GemmDesc& gb, const Ep
   }
   const int splits = f32_splits(ga);
   EpiParams ep = ea;
-  if (splits > 1) ep.out = ga.splitk_ws;
+  const bool ws = splits > 1 && !ea.accumulate;   // partials to the workspace, summed after
+  if (ws) ep.out = ga.splitk_ws;
   const int rc =
       eb.kind == EPI_STORE   ? launch_tc_pair_group<T, EPI_F32, EPI_STORE>(ga, ep, splits, gb, eb, s)
       : eb.kind == EPI_MUL   ? launch_tc_pair_group<T, EPI_F32, EPI_MUL>(ga, ep, splits, gb, eb, s)
       : eb.gelu_tanh         ? launch_tc_pair_group<T, EPI_F32, EPI_DGELU | EPI_TANH>(ga, ep, splits, gb, eb, s)
                              : launch_tc_pair_group<T, EPI_F32, EPI_DGELU>(ga, ep, splits, gb, eb, s);
   if (rc) return rc;
-  if (splits > 1) f32_split_reduce(ga, ea, splits, s);
+  if (ws) f32_split_reduce(ga, ea, splits, s);
   return 0;
 }
 

@@ -92,6 +92,12 @@ struct EpiParams {
   // partial row per (256-row tile, CTA of the pair, TMEM lane quarter), i.e.
   // row (m / 256) * 8 + ((m % 256) / 128) * 4 + (m % 128) / 32; or null
   float* colsum;
+  // 1: add instead of store (arrival order, not a fixed one).  EPI_F32 on the
+  // tensor-core GEMM: the split-K partial tiles are added into `out` (by TMA
+  // reduce-add; no workspace, no closing sum), so `out` must hold zeros when
+  // K is split; `colsum`: every partial row is added into its single row
+  // (cols floats, which must hold zeros)
+  int accumulate;
 };
 
 // CTA pairs of the tensor-core pair kernel that have no tile in its last
@@ -162,6 +168,9 @@ struct LnBwdArgs {
   float* part_dbeta;
   float* part_dsum;     // column sums of drop_out, or null
   int rows, H;
+  // 1: every block adds its column sums into row 0 of part_* (the gradients
+  // themselves, holding zeros) with atomics instead of storing its own row
+  int part_acc;
 };
 // Upper bound of the partial rows ln_bwd_run writes (size of the part_* buffers).
 int ln_bwd_parts(int rows);
@@ -171,11 +180,22 @@ int ln_bwd_run(int dtype, const LnBwdArgs& a, cudaStream_t s);
 // ------------------------------------------------------------------ elementwise / reductions
 // out = dropout(in) (site, element t*H + c) with column partial sums of out.
 int rowdrop_parts(int rows);
+// With acc, every block adds its column sums into part_sum[0..H) (holding
+// zeros) with atomics instead of storing a row of its own.
 void dropout_rows_run(int dtype, const void* in, void* out, const DropoutParams& dp, int site, int rows, int H,
-                      float* part_sum, cudaStream_t s, const uint8_t* keep8 = nullptr);
-// Column partial sums of a (rows, cols) storage-typed matrix: (colsum_parts(rows), cols) floats.
+                      float* part_sum, cudaStream_t s, const uint8_t* keep8 = nullptr, int acc = 0);
+// Column partial sums of a (rows, cols) storage-typed matrix: (colsum_parts(rows), cols) floats
+// (with acc: added into part[0..cols), holding zeros, with atomics).
 int colsum_parts(int rows);
-void colsum_run(int dtype, const void* X, int rows, int cols, float* part, cudaStream_t s);
+void colsum_run(int dtype, const void* X, int rows, int cols, float* part, cudaStream_t s, int acc = 0);
+// Sets every listed float32 buffer to zero, in one launch.
+constexpr int kMaxZero = 16;
+struct ZeroList {
+  float* p[kMaxZero];
+  size_t n[kMaxZero];
+  int count;
+};
+void zero_list_run(const ZeroList& z, cudaStream_t s);
 // out[c] = sum_p part[p*cols + c] (fixed order).
 void colsum_finalize_run(const float* part, int nparts, int cols, float* out, cudaStream_t s);
 // Several finalizes in one launch, each job either
@@ -241,6 +261,9 @@ struct AttnArgs {
   // float32 matrix; written only by kernels that fuse it (see
   // attn_tc_fuses_colsum), else untouched
   float* colsum;
+  // 1: the partial rows are added into row 0 of `colsum` (holding zeros)
+  // with atomics instead
+  int colsum_acc;
 };
 void attn_fwd_run(int dtype, const AttnArgs& a, cudaStream_t s);
 void attn_bwd_run(int dtype, const AttnArgs& a, cudaStream_t s);

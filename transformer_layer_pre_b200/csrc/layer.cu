@@ -298,9 +298,14 @@ EpiParams epi(int kind, void* out, int ldo) {
 }
 
 // Column partial sums of a (T, cols) stored matrix into partial slot `slot`,
-// summed into `out` by the backward's closing finalize.
+// summed into `out` by the backward's closing finalize (stochastic mode:
+// added into `out`, which holds zeros, with atomics).
 void bias_grad(tl_layer* L, const void* X, int cols, int slot, float* out, FinalizeList& fin, cudaStream_t s) {
   ProfScope p_(PC_ROWWISE, s);
+  if (L->opt.stochastic_mode) {
+    colsum_run(L->opt.dtype, X, L->T, cols, out, s, 1);
+    return;
+  }
   float* part = L->part + (size_t)slot * L->part_floats;
   colsum_run(L->opt.dtype, X, L->T, cols, part, s);
   fin.job[fin.n++] = {part, out, colsum_parts(L->T), cols};
@@ -402,6 +407,7 @@ tl_status layer_set_options(tl_layer* L, const tl_options* o) {
   L->opt = *o;
   L->opt.training = o->training ? 1 : 0;
   L->opt.gelu_tanh = o->gelu_tanh ? 1 : 0;
+  L->opt.stochastic_mode = o->stochastic_mode ? 1 : 0;
   if (shared && shared_bytes >= scratch_size(L)) {
     L->scratch = shared;
     L->scratch_bytes = shared_bytes;
@@ -579,10 +585,36 @@ tl_status layer_backward(tl_layer* L, const void* x, const void* dy, const tl_we
   const DropoutParams dh = make_drop(L, L->ph);
   const bool keepbits = dh.thr != 0;   // the forward left the hidden-dropout keep bits
   // every parameter column sum (bias, gamma, beta gradients) leaves its
-  // producer as partial rows in a slot of its own; one launch at the end sums them
+  // producer as partial rows in a slot of its own; one launch at the end sums
+  // them.  Stochastic mode: the producers add them into the gradients
+  // themselves (zeroed first) with atomics, and so do the splits of a
+  // split-K weight gradient; nothing is left for a closing launch.
+  const bool relaxed = L->opt.stochastic_mode != 0;
   FinalizeList fin;
   fin.n = 0;
   auto slot = [&](int i) { return L->part + (size_t)i * L->part_floats; };
+  // where column sum `i` of gradient `out` goes
+  auto sink = [&](int i, float* out) { return relaxed ? out : slot(i); };
+  auto finish = [&](const FinalizeJob& j) {
+    if (!relaxed) fin.job[fin.n++] = j;
+  };
+  if (relaxed) {
+    ZeroList z;
+    z.count = 0;
+    auto zero = [&](float* p, size_t n) {
+      z.p[z.count] = p;
+      z.n[z.count++] = n;
+    };
+    zero(g->bqkv, 3 * (size_t)H); zero(g->bo, H); zero(g->ln1_g, H); zero(g->ln1_b, H);
+    zero(g->b1, F); zero(g->b2, H); zero(g->ln2_g, H); zero(g->ln2_b, H);
+    // the weight gradients whose K is split (those with split-K scratch)
+    if (L->splitk[0]) zero(g->w2, (size_t)H * F);
+    if (L->splitk[1]) zero(g->w1, (size_t)F * H);
+    if (L->splitk[2]) zero(g->wo, (size_t)H * H);
+    if (L->splitk[3]) zero(g->wqkv, (size_t)3 * H * H);
+    ProfScope p_(PC_ROWWISE, s);
+    zero_list_run(z, s);
+  }
 
   auto ln_bwd = [&](const void* dyln, const void* xin, const void* yln, const float* mean, const float* rstd,
                     const void* gamma, const void* beta, const void* res, void* dxo, void* drop_out, int site,
@@ -592,19 +624,22 @@ tl_status layer_backward(tl_layer* L, const void* x, const void* dy, const tl_we
     a.dy = dyln; a.x = inv ? nullptr : xin; a.y = inv ? yln : nullptr;
     a.mean = mean; a.rstd = rstd; a.gamma = gamma; a.beta = beta;
     a.res = res; a.dx = dxo; a.drop_out = drop_out; a.drop = dh; a.site = site; a.keep8 = keep8;
-    a.part_dgamma = slot(slot0); a.part_dbeta = slot(slot0 + 1); a.part_dsum = drop_out ? slot(slot0 + 2) : nullptr;
+    a.part_dgamma = sink(slot0, dgamma); a.part_dbeta = sink(slot0 + 1, dbeta);
+    a.part_dsum = drop_out ? sink(slot0 + 2, dsum) : nullptr;
+    a.part_acc = relaxed ? 1 : 0;
     a.rows = T; a.H = H;
     ProfScope p_(PC_LN_BWD, s);
     const int parts = ln_bwd_run(dt, a, s);
-    fin.job[fin.n++] = {a.part_dgamma, dgamma, parts, H};
-    fin.job[fin.n++] = {a.part_dbeta, dbeta, parts, H};
-    if (drop_out) fin.job[fin.n++] = {a.part_dsum, dsum, parts, H};
+    finish({a.part_dgamma, dgamma, parts, H, 0});
+    finish({a.part_dbeta, dbeta, parts, H, 0});
+    if (drop_out) finish({a.part_dsum, dsum, parts, H, 0});
   };
 
   // FFN block: dZ2 -> dW2, dU (into big), db1, then dW1 with the FFN input
   // gradient dU W1 (epilogue `edin`, output (T, H))
   auto ffn_bwd = [&](const void* ffn_in, const EpiParams& edin, int db1_slot) {
     EpiParams ew2 = epi(EPI_F32, g->w2, F);
+    ew2.accumulate = relaxed;
     if (L->opt.gelu_checkpoint) {
       ProfScope p_(PC_ROWWISE, s);
       gelu_run(dt, L->u, L->big, (size_t)T * F, L->opt.gelu_tanh ? 1 : 0, s);
@@ -615,7 +650,8 @@ tl_status layer_backward(tl_layer* L, const void* x, const void* dy, const tl_we
     edu.gelu_tanh = L->opt.gelu_tanh ? 1 : 0;
     // the tensor-core GEMM sums dU's columns in its epilogue (db1)
     const bool fused_db1 = gemm_uses_tensor_cores(dt) != 0;
-    if (fused_db1) edu.colsum = slot(db1_slot);
+    if (fused_db1) edu.colsum = sink(db1_slot, g->b1);
+    edu.accumulate = relaxed;
     GemmDesc gw2 = wdesc(L, 0, &fin, H, F, T, L->dz2, H, L->g, F);                // dW2 = dZ2^T G
     // recompute mode: G was just rewritten by the GELU launch before this one
     if (L->opt.gelu_checkpoint) gw2.b_early = false;
@@ -627,9 +663,10 @@ tl_status layer_backward(tl_layer* L, const void* x, const void* dy, const tl_we
       ProfScope p_(PC_GEMM, s);
       if (gemm_run(dt, gw2, ew2, s) != 0 || gemm_run(dt, gdu, edu, s) != 0) L->gemm_err = 1;
     }
-    if (fused_db1) fin.job[fin.n++] = {slot(db1_slot), g->b1, (T + 255) / 256 * 8, F};   // db1 from the GEMM
+    if (fused_db1) finish({slot(db1_slot), g->b1, (T + 255) / 256 * 8, F, 0});   // db1 from the GEMM
     else bias_grad(L, L->big, F, db1_slot, g->b1, fin, s);                                  // db1
     EpiParams ew1 = epi(EPI_F32, g->w1, H);
+    ew1.accumulate = relaxed;
     gemm2(L, wdesc(L, 1, &fin, F, H, T, L->big, F, ffn_in, H), ew1,          // dW1 = dU^T in
           gdesc(L, T, H, F, L->big, F, true, w->w1, H, false), edin, s);   // dU W1
   };
@@ -637,16 +674,21 @@ tl_status layer_backward(tl_layer* L, const void* x, const void* dy, const tl_we
   // dWqkv with the attention input gradient dQKV Wqkv (epilogue `edin`)
   auto attn_bwd_block = [&](const void* attn_in, const EpiParams& edin, int dbqkv_slot) {
     EpiParams ewo = epi(EPI_F32, g->wo, H);
+    ewo.accumulate = relaxed;
     EpiParams edc = epi(EPI_STORE, L->dctx, H);
     gemm2(L, wdesc(L, 2, &fin, H, H, T, L->da, H, L->ctx, H), ewo,           // dWo = dA^T ctx
           gdesc(L, T, H, H, L->da, H, true, w->wo, H, false), edc, s);     // dctx = dA Wo
     AttnArgs aa = attn_args(L, L->mask);
     const bool fused_dbqkv = attn_tc_supports(dt, aa) && attn_tc_fuses_colsum(dt, aa);
-    if (fused_dbqkv) aa.colsum = slot(dbqkv_slot);
+    if (fused_dbqkv) {
+      aa.colsum = sink(dbqkv_slot, g->bqkv);
+      aa.colsum_acc = relaxed ? 1 : 0;
+    }
     attn_bwd(L, aa, s);
-    if (fused_dbqkv) fin.job[fin.n++] = {slot(dbqkv_slot), g->bqkv, L->B * 4, 3 * H};   // from the attention
+    if (fused_dbqkv) finish({slot(dbqkv_slot), g->bqkv, L->B * 4, 3 * H, 0});   // from the attention
     else bias_grad(L, L->dqkv, 3 * H, dbqkv_slot, g->bqkv, fin, s);
     EpiParams ewq = epi(EPI_F32, g->wqkv, H);
+    ewq.accumulate = relaxed;
     gemm2(L, wdesc(L, 3, &fin, 3 * H, H, T, L->dqkv, 3 * H, attn_in, H), ewq,           // dWqkv = dQKV^T in
           gdesc(L, T, H, 3 * H, L->dqkv, 3 * H, true, w->wqkv, H, false), edin, s);  // dQKV Wqkv
   };
@@ -654,8 +696,8 @@ tl_status layer_backward(tl_layer* L, const void* x, const void* dy, const tl_we
   if (L->pre_ln) {
     {
       ProfScope p_(PC_ROWWISE, s);
-      dropout_rows_run(dt, dy, L->dz2, dh, 2, T, H, slot(0), s, keepbits ? L->keep2 : nullptr);
-      fin.job[fin.n++] = {slot(0), g->b2, rowdrop_parts(T), H};
+      dropout_rows_run(dt, dy, L->dz2, dh, 2, T, H, sink(0, g->b2), s, keepbits ? L->keep2 : nullptr, relaxed);
+      finish({slot(0), g->b2, rowdrop_parts(T), H, 0});
     }
     ffn_bwd(L->h2, epi(EPI_STORE, L->dh, H), 1);                         // dH2 = dU W1
     ln_bwd(L->dh, L->x2, L->h2, L->mean2, L->rstd2, w->ln2_g, w->ln2_b, dy, L->dx2, L->da, 1,

@@ -73,7 +73,14 @@ __device__ __forceinline__ void row_range(int rows, int& r0, int& r1) {
   r1 = min(rows, r0 + per);
 }
 
-__device__ __forceinline__ void store_part(float* part, int H, int col, const float (&acc)[8]) {
+// A block's column sums of 8 columns: its own row of `part` (summed later in
+// a fixed order) or, with add, added into row 0 (arrival order).
+__device__ __forceinline__ void store_part(float* part, int H, int col, const float (&acc)[8], int add) {
+  if (add) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) atomicAdd(part + col + i, acc[i]);
+    return;
+  }
   float* p = part + (size_t)blockIdx.x * H + col;
   reinterpret_cast<float4*>(p)[0] = make_float4(acc[0], acc[1], acc[2], acc[3]);
   reinterpret_cast<float4*>(p)[1] = make_float4(acc[4], acc[5], acc[6], acc[7]);
@@ -384,9 +391,9 @@ __global__ void __launch_bounds__(512) ln_bwd_kernel(LnBwdArgs a) {
     pipe.release(gi);
   }
   if (act) {
-    store_part(a.part_dgamma, H, col, dg);
-    store_part(a.part_dbeta, H, col, db);
-    if (a.part_dsum) store_part(a.part_dsum, H, col, ds);
+    store_part(a.part_dgamma, H, col, dg, a.part_acc);
+    store_part(a.part_dbeta, H, col, db, a.part_acc);
+    if (a.part_dsum) store_part(a.part_dsum, H, col, ds, a.part_acc);
   }
 }
 
@@ -547,7 +554,8 @@ __global__ void __launch_bounds__(kLnbPairs * 64, (sizeof(T) == 4 || (INV && DRO
       float t = 0.0f;
 #pragma unroll
       for (int w = 0; w < kLnbPairs; ++w) t += red[w * H + col];
-      part[(size_t)blockIdx.x * H + col] = t;
+      if (a.part_acc) atomicAdd(part + col, t);
+      else part[(size_t)blockIdx.x * H + col] = t;
     }
   };
   reduce(dg, a.part_dgamma);
@@ -560,7 +568,7 @@ template <typename T, int KR>
 __global__ void __launch_bounds__(512) dropout_rows_kernel(const T* __restrict__ in, T* __restrict__ out,
                                                            DropoutParams dp, int site, int rows, int H,
                                                            float* __restrict__ part,
-                                                           const uint8_t* __restrict__ keep8) {
+                                                           const uint8_t* __restrict__ keep8, int padd) {
   pdl_wait();
   pdl_launch_dependents();
   extern __shared__ __align__(128) uint8_t smem[];
@@ -595,7 +603,7 @@ __global__ void __launch_bounds__(512) dropout_rows_kernel(const T* __restrict__
     __syncthreads();
     pipe.release(gi);
   }
-  if (act) store_part(part, H, col, acc);
+  if (act) store_part(part, H, col, acc, padd);
 }
 
 // Dropout backward for H <= 1024 with precomputed keep bits: one warp per
@@ -609,7 +617,8 @@ template <typename T, int NCH>
 __global__ void __launch_bounds__(kDropWarps * 32) dropout_rows_warp_kernel(const T* __restrict__ in,
                                                                             T* __restrict__ out, float scale,
                                                                             int rows, int H, float* __restrict__ part,
-                                                                            const uint8_t* __restrict__ keep8) {
+                                                                            const uint8_t* __restrict__ keep8,
+                                                                            int padd) {
   pdl_wait();
   pdl_launch_dependents();
   extern __shared__ __align__(16) float dred[];   // [kDropWarps][H]
@@ -670,7 +679,8 @@ __global__ void __launch_bounds__(kDropWarps * 32) dropout_rows_warp_kernel(cons
     float t = 0.0f;
 #pragma unroll
     for (int w = 0; w < kDropWarps; ++w) t += dred[w * H + col];
-    part[(size_t)blockIdx.x * H + col] = t;
+    if (padd) atomicAdd(part + col, t);
+    else part[(size_t)blockIdx.x * H + col] = t;
   }
 }
 
@@ -679,7 +689,7 @@ constexpr int kColParts = 64;
 
 template <typename T>
 __global__ void __launch_bounds__(256) colsum_kernel(const T* __restrict__ X, int rows, int cols,
-                                                     float* __restrict__ part) {
+                                                     float* __restrict__ part, int padd) {
   pdl_wait();
   pdl_launch_dependents();
   __shared__ float red[8][256 + 8];
@@ -701,7 +711,8 @@ __global__ void __launch_bounds__(256) colsum_kernel(const T* __restrict__ X, in
   if (c < cols) {
     float s = 0.0f;
     for (int w = 0; w < 8; ++w) s += red[w][threadIdx.x];
-    part[(size_t)blockIdx.y * cols + c] = s;
+    if (padd) atomicAdd(part + c, s);
+    else part[(size_t)blockIdx.y * cols + c] = s;
   }
 }
 
@@ -894,12 +905,12 @@ int ln_bwd_t(const LnBwdArgs& a, cudaStream_t s) {
 
 template <typename T>
 void dropout_rows_t(const void* in, void* out, const DropoutParams& dp, int site, int rows, int H, float* part,
-                    cudaStream_t s, const uint8_t* keep8) {
+                    cudaStream_t s, const uint8_t* keep8, int padd) {
   TLP_KR_SWITCH(H, (int)sizeof(T), {
     const size_t sm = pipe_smem<T, KR, 1>(H);
     cudaFuncSetAttribute(dropout_rows_kernel<T, KR>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
     launch_pdl(dropout_rows_kernel<T, KR>, rowdrop_parts(rows), row_threads(H), sm, s,
-               static_cast<const T*>(in), static_cast<T*>(out), dp, site, rows, H, part, keep8);
+               static_cast<const T*>(in), static_cast<T*>(out), dp, site, rows, H, part, keep8, padd);
   });
   count_launch();
 }
@@ -951,37 +962,75 @@ int rowwise_take_error() {
 
 template <typename T>
 void dropout_rows_warp_t(const void* in, void* out, float scale, int rows, int H, float* part, cudaStream_t s,
-                         const uint8_t* keep8) {
+                         const uint8_t* keep8, int padd) {
   const size_t sm = (size_t)kDropWarps * H * sizeof(float);
   TLP_NCH_SWITCH(H, {
     if constexpr (NCH <= 4) {
       cudaFuncSetAttribute(dropout_rows_warp_kernel<T, NCH>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
       launch_pdl(dropout_rows_warp_kernel<T, NCH>, rowdrop_parts(rows), kDropWarps * 32, sm, s,
-                 static_cast<const T*>(in), static_cast<T*>(out), scale, rows, H, part, keep8);
+                 static_cast<const T*>(in), static_cast<T*>(out), scale, rows, H, part, keep8, padd);
     }
   });
   count_launch();
 }
 
 void dropout_rows_run(int dt, const void* in, void* out, const DropoutParams& dp, int site, int rows, int H,
-                      float* part, cudaStream_t s, const uint8_t* keep8) {
+                      float* part, cudaStream_t s, const uint8_t* keep8, int acc) {
+  const int padd = acc ? 1 : 0;
   if (keep8 && dp.thr && H <= 1024) {
     // keep bits at hand: the warp-per-row form (no Philox, no shared-memory pipeline)
-    if (dt == DT_F32) dropout_rows_warp_t<float>(in, out, dp.scale, rows, H, part, s, keep8);
-    else if (dt == DT_F16) dropout_rows_warp_t<half_t>(in, out, dp.scale, rows, H, part, s, keep8);
-    else dropout_rows_warp_t<bf16_t>(in, out, dp.scale, rows, H, part, s, keep8);
+    if (dt == DT_F32) dropout_rows_warp_t<float>(in, out, dp.scale, rows, H, part, s, keep8, padd);
+    else if (dt == DT_F16) dropout_rows_warp_t<half_t>(in, out, dp.scale, rows, H, part, s, keep8, padd);
+    else dropout_rows_warp_t<bf16_t>(in, out, dp.scale, rows, H, part, s, keep8, padd);
     return;
   }
-  if (dt == DT_F32) dropout_rows_t<float>(in, out, dp, site, rows, H, part, s, keep8);
-  else if (dt == DT_F16) dropout_rows_t<half_t>(in, out, dp, site, rows, H, part, s, keep8);
-  else dropout_rows_t<bf16_t>(in, out, dp, site, rows, H, part, s, keep8);
+  if (dt == DT_F32) dropout_rows_t<float>(in, out, dp, site, rows, H, part, s, keep8, padd);
+  else if (dt == DT_F16) dropout_rows_t<half_t>(in, out, dp, site, rows, H, part, s, keep8, padd);
+  else dropout_rows_t<bf16_t>(in, out, dp, site, rows, H, part, s, keep8, padd);
 }
 
-void colsum_run(int dt, const void* X, int rows, int cols, float* part, cudaStream_t s) {
+void colsum_run(int dt, const void* X, int rows, int cols, float* part, cudaStream_t s, int acc) {
   dim3 grid((cols + 255) / 256, colsum_parts(rows));
-  if (dt == DT_F32) launch_pdl(colsum_kernel<float>, grid, 256, 0, s, static_cast<const float*>(X), rows, cols, part);
-  else if (dt == DT_F16) launch_pdl(colsum_kernel<half_t>, grid, 256, 0, s, static_cast<const half_t*>(X), rows, cols, part);
-  else launch_pdl(colsum_kernel<bf16_t>, grid, 256, 0, s, static_cast<const bf16_t*>(X), rows, cols, part);
+  const int padd = acc ? 1 : 0;
+  if (dt == DT_F32)
+    launch_pdl(colsum_kernel<float>, grid, 256, 0, s, static_cast<const float*>(X), rows, cols, part, padd);
+  else if (dt == DT_F16)
+    launch_pdl(colsum_kernel<half_t>, grid, 256, 0, s, static_cast<const half_t*>(X), rows, cols, part, padd);
+  else launch_pdl(colsum_kernel<bf16_t>, grid, 256, 0, s, static_cast<const bf16_t*>(X), rows, cols, part, padd);
+  count_launch();
+}
+
+namespace {
+
+// Zeroes each listed buffer: 16-byte stores where the buffer is 16-byte
+// aligned, one float at a time for the rest.
+__global__ void __launch_bounds__(256) zero_list_kernel(ZeroList z) {
+  pdl_wait();
+  pdl_launch_dependents();
+  const size_t stride = (size_t)gridDim.x * blockDim.x;
+  const size_t tid = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
+  for (int j = 0; j < z.count; ++j) {
+    float* p = z.p[j];
+    const size_t n = z.n[j];
+    size_t head = 0;
+    if ((reinterpret_cast<uintptr_t>(p) & 15) == 0) {
+      const size_t n4 = n / 4;
+      float4* p4 = reinterpret_cast<float4*>(p);
+      for (size_t i = tid; i < n4; i += stride) p4[i] = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+      head = n4 * 4;
+    }
+    for (size_t i = head + tid; i < n; i += stride) p[i] = 0.0f;
+  }
+}
+
+}  // namespace
+
+void zero_list_run(const ZeroList& z, cudaStream_t s) {
+  if (z.count <= 0) return;
+  size_t total4 = 0;
+  for (int j = 0; j < z.count; ++j) total4 += (z.n[j] + 3) / 4;
+  const int blocks = (int)std::max<size_t>(1, std::min<size_t>((total4 + 255) / 256, 148 * 4));
+  launch_pdl(zero_list_kernel, blocks, 256, 0, s, z);
   count_launch();
 }
 
