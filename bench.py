@@ -148,10 +148,11 @@ def barrier() -> None:
 
 # ---------------------------------------------------------------- clocks
 class ClockSampler:
-    """Samples the GPU's SM clock, power and clock-event (throttle) reasons
-    through NVML every few milliseconds on a background thread (read-only
-    queries; no setting is touched).  Samples taken while `timed` is set
-    form the timed-region summary."""
+    """Samples the GPU's SM clock and clock-event (throttle) reasons through
+    NVML (read-only queries; no setting is touched): on a background thread
+    every 0.2 ms, and from the main thread through `sample()` while it waits
+    for the timed steps to finish.  Samples taken while `timed` is set form
+    the timed-region summary."""
 
     REASONS = (("nvmlClocksEventReasonHwSlowdown", "hw_slowdown"),
                ("nvmlClocksEventReasonHwThermalSlowdown", "hw_thermal_slowdown"),
@@ -165,6 +166,7 @@ class ClockSampler:
         self.smax = None
         self._stop = None
         self._thread = None
+        self._query = None
 
     def _handle(self, pynvml):
         """The NVML handle of CUDA device `index`, matched by PCI address
@@ -188,20 +190,28 @@ class ClockSampler:
         masks = [(getattr(pynvml, n), name) for n, name in self.REASONS]
         self._stop = threading.Event()
 
+        def query():
+            try:
+                sm = pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM)
+                r = pynvml.nvmlDeviceGetCurrentClocksEventReasons(h)
+                self.rows.append((float(sm), [name for m, name in masks if r & m]))
+            except Exception:
+                pass
+        self._query = query
+
         def loop():
-            while not self._stop.is_set():
+            while not self._stop.wait(self.period):
                 if self.timed:
-                    try:
-                        sm = pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM)
-                        r = pynvml.nvmlDeviceGetCurrentClocksEventReasons(h)
-                        self.rows.append((float(sm), [name for m, name in masks if r & m]))
-                    except Exception:
-                        pass
-                self._stop.wait(self.period)
+                    query()
 
         self._thread = threading.Thread(target=loop, daemon=True)
         self._thread.start()
         return self
+
+    def sample(self) -> None:
+        """One sample now (from the calling thread), if inside the timed region."""
+        if self.timed and self._query is not None:
+            self._query()
 
     def __exit__(self, *exc):
         if self._thread is not None:
@@ -214,7 +224,8 @@ class ClockSampler:
         reasons = sorted({n for _, rs in self.rows for n in rs})
         return {"sm_mhz": statistics.median(sm for sm, _ in self.rows), "sm_max_mhz": self.smax,
                 "reasons": reasons, "samples": len(self.rows),
-                "source": "NVML queries back to back (0.2 ms apart) over the timed regions"}
+                "source": "NVML queries 0.2 ms apart over the timed regions (a sampling thread, and the "
+                          "main thread while it waits for the last timed step)"}
 
 
 # ---------------------------------------------------------------- oracle (reference arm / CPU baseline)
@@ -393,6 +404,10 @@ def run_ours(args) -> None:
             runners[0]()
             exchange()
             b.record(stream)
+        # the steps run on the device meanwhile: sample the clocks until the last one ends
+        while not evs[-1][1].query():
+            clk.sample()
+            time.sleep(2e-4)
         torch.cuda.synchronize()
         clk.timed = False
         sys.setswitchinterval(switch)

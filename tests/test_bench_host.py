@@ -26,3 +26,38 @@ def test_recorded_traffic_tracks_kernel_sources(monkeypatch, tmp_path):
     # a changed kernel source invalidates the recorded counters
     monkeypatch.setattr(bench, "gemm_sources_digest", lambda: "0" * 64)
     assert bench.recorded_gemm_traffic(bench.WORKLOAD) is None
+
+
+def test_clock_sampler_reads_a_fake_nvml_and_only_reads(monkeypatch):
+    """The clock record: samples only inside the timed region, from the
+    main thread's sample() as well as the thread, throttle reasons decoded
+    from the reason mask; every NVML call it makes is a query."""
+    import types
+    calls = []
+    fake = types.SimpleNamespace(
+        NVML_CLOCK_SM=0,
+        nvmlClocksEventReasonHwSlowdown=0x8, nvmlClocksEventReasonHwThermalSlowdown=0x40,
+        nvmlClocksEventReasonSwThermalSlowdown=0x20, nvmlClocksEventReasonSwPowerCap=0x4)
+
+    def rec(name, value):
+        def f(*a):
+            calls.append(name)
+            return value
+        return f
+    fake.nvmlInit = rec("nvmlInit", None)
+    fake.nvmlDeviceGetHandleByPciBusId = rec("nvmlDeviceGetHandleByPciBusId", "h")
+    fake.nvmlDeviceGetHandleByIndex = rec("nvmlDeviceGetHandleByIndex", "h")
+    fake.nvmlDeviceGetMaxClockInfo = rec("nvmlDeviceGetMaxClockInfo", 1965)
+    fake.nvmlDeviceGetClockInfo = rec("nvmlDeviceGetClockInfo", 1800)
+    fake.nvmlDeviceGetCurrentClocksEventReasons = rec("nvmlDeviceGetCurrentClocksEventReasons", 0x4)
+    monkeypatch.setitem(sys.modules, "pynvml", fake)
+    with bench.ClockSampler(0, period_s=10.0) as clk:   # the thread wakes too rarely to sample
+        clk.sample()                                      # outside the timed region: ignored
+        clk.timed = True
+        clk.sample()
+        clk.sample()
+        clk.timed = False
+    s = clk.summary()
+    assert s["samples"] == 2 and s["sm_mhz"] == 1800 and s["sm_max_mhz"] == 1965
+    assert s["reasons"] == ["sw_power_cap"]
+    assert all(c == "nvmlInit" or c.startswith("nvmlDeviceGet") for c in calls)
