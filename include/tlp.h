@@ -135,6 +135,14 @@ void layer_default_options(tl_options* opt);
 tl_status layer_set_options(tl_layer* layer, const tl_options* opt);
 tl_status layer_get_options(const tl_layer* layer, tl_options* opt);
 
+/* Sets the dropout generator's key (seed, as given to layer_create) and 4th
+ * counter word (tl_options.philox_offset) for the next forward, without
+ * touching any buffer: a training loop gives each step masks of its own this
+ * way (a stack, for instance, philox_offset = step * layers + layer).  A
+ * backward always draws (or reads) the masks of the forward before it, so
+ * calling this between the two is allowed.  TL_EINVAL for a NULL layer. */
+tl_status layer_set_rng(tl_layer* layer, uint64_t seed, uint64_t philox_offset);
+
 /* Forward.  x, y: (batch, seq, hidden) storage dtype; y must not alias x.
  * mask: NULL or (batch, seq) float32 additive key mask (0 for a valid key,
  * -inf for padding), broadcast over heads and queries.  A query row whose

@@ -75,6 +75,11 @@ def test_create_defaults_and_state_errors(lib):
         assert lib.layer_get_options(h, ctypes.byref(opt)) == TL_OK
         assert opt.dtype == 0 and opt.training == 1 and abs(opt.ln_eps - 1e-12) < 1e-18
         assert opt.stochastic_mode == 0   # bitwise-reproducible by default
+        # the dropout generator's key and counter word change without a reallocation
+        assert lib.layer_set_rng(None, 1, 2) == TL_EINVAL
+        assert lib.layer_set_rng(h, 99, 7) == TL_OK
+        assert lib.layer_get_options(h, ctypes.byref(opt)) == TL_OK and opt.philox_offset == 7
+        assert lib.layer_workspace_bytes(h) == 0
         assert lib.layer_workspace_bytes(h) == 0  # nothing allocated before options / forward
         w = tlp._Weights(*([1] * 12))
         st = lib.layer_backward(h, 1, 1, ctypes.byref(w), ctypes.byref(w), 1, None)

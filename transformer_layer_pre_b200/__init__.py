@@ -27,7 +27,7 @@ WEIGHT_NAMES = (
 )
 DTYPE_CODES = {torch.float32: 0, torch.float16: 1, torch.bfloat16: 2}
 EXPORTED_SYMBOLS = (
-    "layer_create", "layer_default_options", "layer_set_options", "layer_get_options",
+    "layer_create", "layer_default_options", "layer_set_options", "layer_get_options", "layer_set_rng",
     "layer_forward", "layer_backward", "layer_workspace_bytes", "layer_last_error",
     "layer_destroy", "tl_dropout_keep_mask", "tl_device_check", "tl_profile_enable",
     "tl_profile_read", "tl_launch_count", "tl_bias_grad_noalloc", "tl_gelu_eval", "tl_status_string",
@@ -84,6 +84,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.layer_set_options.argtypes = [vp, ctypes.POINTER(Options)]
     lib.layer_set_options.restype = i
     lib.layer_get_options.argtypes = [vp, ctypes.POINTER(Options)]
+    lib.layer_set_rng.argtypes = [vp, u64, u64]
+    lib.layer_set_rng.restype = i
     lib.layer_get_options.restype = i
     lib.layer_forward.argtypes = [vp, vp, vp, ctypes.POINTER(_Weights), vp, vp]
     lib.layer_forward.restype = i
@@ -185,6 +187,11 @@ class Layer:
     @staticmethod
     def _weights(w: dict) -> _Weights:
         return _Weights(*[_ptr(w[n]) for n in WEIGHT_NAMES])
+
+    def set_rng(self, seed: int, philox_offset: int) -> None:
+        """Dropout key and 4th Philox counter word of the next forward (its
+        backward keeps the forward's); nothing is reallocated."""
+        self._check(self.lib.layer_set_rng(self.handle, seed, philox_offset))
 
     def forward(self, x, mask, weights, y=None, stream=None):
         """x (B, S, H) storage dtype on the device; mask (B, S) float32 or None."""

@@ -43,6 +43,10 @@ struct tl_layer {
   int pre_ln;
   uint64_t seed;
   tl_options opt;
+  // Philox key and 4th counter word of the current (or last training)
+  // forward: its backward uses them even if layer_set_rng changed seed and
+  // opt.philox_offset since
+  uint64_t drop_seed = 0, drop_offset = 0;
   int device = -1;
   char* arena = nullptr;          // saved activations (forward -> backward)
   size_t arena_bytes = 0;
@@ -95,8 +99,8 @@ tl_status check_cuda(tl_layer* L, const char* where) {
 
 DropoutParams make_drop(const tl_layer* L, float p) {
   DropoutParams d;
-  d.seed = L->seed;
-  d.offset = L->opt.philox_offset;
+  d.seed = L->drop_seed;
+  d.offset = L->drop_offset;
   const bool on = L->opt.training && p > 0.0f;
   d.thr = on ? (uint32_t)std::floor((double)p * 65536.0) : 0u;
   d.scale = on ? 1.0f / (1.0f - p) : 1.0f;
@@ -417,6 +421,13 @@ tl_status layer_set_options(tl_layer* L, const tl_options* o) {
   return ensure_buffers(L);
 }
 
+tl_status layer_set_rng(tl_layer* L, uint64_t seed, uint64_t philox_offset) {
+  if (!L) return TL_EINVAL;
+  L->seed = seed;
+  L->opt.philox_offset = philox_offset;
+  return TL_OK;
+}
+
 tl_status layer_get_options(const tl_layer* L, tl_options* o) {
   if (!L || !o) return TL_EINVAL;
   *o = L->opt;
@@ -472,6 +483,8 @@ tl_status layer_forward(tl_layer* L, const void* x, const float* mask, const tl_
   const int dt = L->opt.dtype, T = L->T, H = L->H, F = L->F;
   const bool train = L->opt.training != 0;
   L->have_fwd = false;
+  L->drop_seed = L->seed;
+  L->drop_offset = L->opt.philox_offset;
 
   EpiParams eq = epi(EPI_QKV, L->qkv, 3 * H);
   eq.bias = w->bqkv; eq.seq = L->S; eq.hidden = H; eq.head_dim = L->d; eq.heads = L->nh; eq.tokens = T;

@@ -64,6 +64,13 @@ class EncoderStack:
         self.dys: list = [None] * num_layers
         self.keep: list = [True] * num_layers
 
+    def set_step(self, step: int) -> None:
+        """Dropout masks of global step `step`: layer l draws with
+        philox_offset = step * num_layers + l (step 0 is the construction's
+        offset l), so no two (step, layer) pairs share masks."""
+        for l, layer in enumerate(self.layers):
+            layer.set_rng(self.seed, step * self.num_layers + l)
+
     def keep_decisions(self, step: int, theta_bar: float, gamma: float) -> list:
         """Progressive Layer Dropping: which layers run at global step `step`."""
         theta = pld_theta(theta_bar, gamma, step)
