@@ -8,7 +8,9 @@
 // copies, and each thread 8 consecutive columns of them, so column sums (bias
 // and LayerNorm-parameter gradients) accumulate in the owning thread's
 // registers in row order and leave as one partial row per block, summed by
-// tlp::colsum_finalize_run in block order: deterministic.
+// tlp::colsum_finalize_run in block order: deterministic.  (With the
+// stochastic-mode flag of a launch, each block instead adds its row into the
+// gradient itself with atomics.)
 #include <algorithm>
 
 #include "common.cuh"
