@@ -114,7 +114,8 @@ def full_clock(clocks: dict | None) -> bool:
     among the sampled reasons and a median within 3 % of the maximum."""
     if not clocks or not clocks.get("sm_mhz") or not clocks.get("sm_max_mhz"):
         return True
-    capped = any(r in ("sw_power_cap", "hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown")
+    capped = any(r in ("sw_power_cap", "hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown",
+                       "hw_power_brake_slowdown")
                  for r in clocks.get("reasons", []))
     return not capped and clocks["sm_mhz"] >= 0.97 * clocks["sm_max_mhz"]
 
@@ -154,10 +155,16 @@ class ClockSampler:
     for the timed steps to finish.  Samples taken while `timed` is set form
     the timed-region summary."""
 
-    REASONS = (("nvmlClocksEventReasonHwSlowdown", "hw_slowdown"),
-               ("nvmlClocksEventReasonHwThermalSlowdown", "hw_thermal_slowdown"),
+    # every clock-event reason NVML reports (read-only), under nvidia-smi's names
+    REASONS = (("nvmlClocksEventReasonGpuIdle", "gpu_idle"),
+               ("nvmlClocksEventReasonApplicationsClocksSetting", "applications_clocks_setting"),
+               ("nvmlClocksEventReasonSwPowerCap", "sw_power_cap"),
+               ("nvmlClocksEventReasonHwSlowdown", "hw_slowdown"),
+               ("nvmlClocksEventReasonSyncBoost", "sync_boost"),
                ("nvmlClocksEventReasonSwThermalSlowdown", "sw_thermal_slowdown"),
-               ("nvmlClocksEventReasonSwPowerCap", "sw_power_cap"))
+               ("nvmlClocksEventReasonHwThermalSlowdown", "hw_thermal_slowdown"),
+               ("nvmlClocksEventReasonHwPowerBrakeSlowdown", "hw_power_brake_slowdown"),
+               ("nvmlClocksEventReasonDisplayClockSetting", "display_clock_setting"))
 
     def __init__(self, index: int, period_s: float = 0.0002):
         self.index, self.period = index, period_s
@@ -187,7 +194,7 @@ class ClockSampler:
             self.smax = float(pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM))
         except Exception:   # no NVML: no clock record
             return self
-        masks = [(getattr(pynvml, n), name) for n, name in self.REASONS]
+        masks = [(getattr(pynvml, n), name) for n, name in self.REASONS if hasattr(pynvml, n)]
         self._stop = threading.Event()
 
         def query():

@@ -49,7 +49,8 @@ def test_clock_sampler_reads_a_fake_nvml_and_only_reads(monkeypatch):
     fake.nvmlDeviceGetHandleByIndex = rec("nvmlDeviceGetHandleByIndex", "h")
     fake.nvmlDeviceGetMaxClockInfo = rec("nvmlDeviceGetMaxClockInfo", 1965)
     fake.nvmlDeviceGetClockInfo = rec("nvmlDeviceGetClockInfo", 1800)
-    fake.nvmlDeviceGetCurrentClocksEventReasons = rec("nvmlDeviceGetCurrentClocksEventReasons", 0x4)
+    fake.nvmlDeviceGetCurrentClocksEventReasons = rec("nvmlDeviceGetCurrentClocksEventReasons", 0x6)
+    fake.nvmlClocksEventReasonApplicationsClocksSetting = 0x2
     monkeypatch.setitem(sys.modules, "pynvml", fake)
     with bench.ClockSampler(0, period_s=10.0) as clk:   # the thread wakes too rarely to sample
         clk.sample()                                      # outside the timed region: ignored
@@ -59,5 +60,5 @@ def test_clock_sampler_reads_a_fake_nvml_and_only_reads(monkeypatch):
         clk.timed = False
     s = clk.summary()
     assert s["samples"] == 2 and s["sm_mhz"] == 1800 and s["sm_max_mhz"] == 1965
-    assert s["reasons"] == ["sw_power_cap"]
+    assert s["reasons"] == ["applications_clocks_setting", "sw_power_cap"]
     assert all(c == "nvmlInit" or c.startswith("nvmlDeviceGet") for c in calls)
