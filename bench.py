@@ -532,7 +532,8 @@ def run_ours(args) -> None:
             "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": w.dtype, "data": "synthetic (seeded N(0,0.02) weights, N(0,1) x and dY)",
-            "config": dict(workload_config(w), graph=not args.no_graph, stochastic_mode=args.stochastic_mode), "tensor_peak_frac": tensor_frac,
+            "config": workload_config(w), "graph": not args.no_graph, "stochastic_mode": args.stochastic_mode,
+            "tensor_peak_frac": tensor_frac,
             "tensor_peak_frac_of_burst": tensor_frac_burst,
             "tensor_peak_frac_of_sustained": tensor_frac_sustained,
             "roofline": roofline, "kernel_classes": classes, "cpu_baseline": cpu,
